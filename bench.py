@@ -1,0 +1,345 @@
+"""Throughput of LSH self-attention forward + backward on B200.
+
+One step = lsh_attn_fwd (hash, sort, attention, round merge) followed by
+lsh_attn_bwd (backward prologue, attention backward, epilogue) on the
+64K-token workload (B=1, H=8, L=65536, d=64, n_buckets=1024, n_hashes=4,
+chunk 64, causal, bf16), inputs resident in HBM.  Prints one JSON line.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+Multi-GPU: launch one process per GPU with torch.distributed.run; each rank
+runs an independent replica of the workload (the (batch, head) slices are
+independent, so there is no data-path collective) and the time is the max
+over ranks.  --impl reference times the CPU oracle on the host cores instead.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from lsh_attention_02_b200 import synth  # noqa: E402
+
+METRIC = "LSH-attn fwd+bwd tokens/s at L=64K, 4 hashes; % of HBM/tensor roofline"
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def describe(w: synth.Workload) -> str:
+    mode = "fwd+bwd" if w.backward else "fwd"
+    extra = f" clustered{w.clustered}(sigma={w.sigma})" if w.clustered else ""
+    return (f"{w.name}: B{w.B} H{w.H} L{w.L} d{w.d} n_buckets{w.n_buckets} n_hashes{w.n_hashes} "
+            f"chunk{w.chunk} {'causal' if w.causal else 'non-causal'} {w.dtype} {mode}{extra}")
+
+
+# ------------------------------------------------------------------ algorithmic bytes / flops
+def algorithmic(w: synth.Workload) -> dict:
+    """Per-step algorithmic HBM bytes and FLOPs (e = element bytes, R = n_hashes, d = 64).
+
+    Whole step, staged formulation:      forward  L [d e (2 + 4R) + 24 R]
+                                         backward L [4 d e + 8 + R (4 d e + 16 + 4 d 4)]
+    per (batch, head).  Attention FLOPs: 4 (2m) d forward and 5 * 2 (2m) d backward per
+    token, head and round; the hash GEMM d * n_buckets per token, head and round."""
+    e = 2 if w.dtype == "bf16" else 4
+    d, R, L, m = w.d, w.n_hashes, w.L, w.chunk
+    bh = w.B * w.H
+    fwd = L * (d * e * (2 + 4 * R) + 24 * R)
+    bwd = L * (4 * d * e + 8 + R * (4 * d * e + 16 + 4 * d * 4)) if w.backward else 0
+    attn_flops = bh * L * R * (4 * 2 * m * d + (10 * 2 * m * d if w.backward else 0))
+    hash_flops = bh * L * R * d * w.n_buckets          # 2 flops x d x n_buckets/2 columns
+    # per-kernel compulsory bytes (each input read once, each output written once)
+    tok = bh * L
+    kern = {
+        "hash": tok * (d * e + 2 * R),                                  # x read, bucket ids written
+        "attn_fwd": tok * R * (2 * d * e + 4 + d * 2 + 4) + tok * 4,    # x, v rows + perm; o_r (bf16) + lse; norms
+        "combine": tok * (R * (d * 2 + 4) + d * e),                     # o_r, lse read; out written
+        "attn_bwd": tok * (3 * d * e + 12 + R * 4) + tok * 2 * d * 4 * 2,  # x, v, dY, LSE, delta, norms, perm;
+                                                                          # fp32 dx, dv accumulators in and out
+    }
+    return {"bytes": bh * (fwd + bwd), "attn_flops": attn_flops, "hash_flops": hash_flops, "kernel_bytes": kern}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            return json.load(f), "measured"
+    return dict(PEAKS_FALLBACK), "fallback"
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.QUERY}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *a):
+        self.lines = []
+        if self.proc is not None:
+            time.sleep(0.15)
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self) -> dict:
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in getattr(self, "lines", []):
+            f = [s.strip() for s in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1])); mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ our arm
+def run_ours(args, w: synth.Workload, rank: int, world: int) -> dict | None:
+    import torch
+    import torch.distributed as dist
+    import lsh_attention_02_b200 as lsh
+
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", device_id=dev, timeout=__import__("datetime").timedelta(seconds=120))
+
+    inp = synth.make_inputs(w.replace(seed=w.seed + 1000 * rank))
+    tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    host = {k: torch.from_numpy(v).to(tdt).pin_memory() for k, v in inp.items()}
+    x, v, R = host["x"].to(dev), host["v"].to(dev), host["R"].to(dev)
+    dy = host["dy"].to(dev) if w.backward else None
+    desc = lsh.desc_for(x, w.n_buckets, w.n_hashes, w.chunk, w.causal)
+    out, lse, perm = lsh.outputs_like(desc, x)
+    ws_f = lsh.workspace(desc, False, dev)
+    ws_b = lsh.workspace(desc, True, dev) if w.backward else None
+    dx = torch.empty_like(x); dv = torch.empty_like(v)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)   # > 126 MB L2
+
+    def step():
+        lsh.lsh_attn_fwd(desc, x, v, R, out, lse, perm, ws_f)
+        if w.backward:
+            lsh.lsh_attn_bwd(desc, x, v, R, out, lse, perm, dy, dx, dv, ws_b)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if lsh.lsh_attn_poll(ws_f) != 0 or (ws_b is not None and lsh.lsh_attn_poll(ws_b) != 0):
+        raise RuntimeError("device-side timeout during warm-up")
+
+    stream = torch.cuda.current_stream(dev)
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        lsh.trace_begin(64 * args.steps + 64)
+        for k in range(args.steps):
+            flush.zero_()
+            starts[k].record(stream)
+            step()
+            ends[k].record(stream)
+        torch.cuda.synchronize()
+        stages = lsh.trace_end()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    step_ms = float(sum(s.elapsed_time(e) for s, e in zip(starts, ends))) / args.steps
+    if lsh.lsh_attn_poll(ws_f) != 0 or (ws_b is not None and lsh.lsh_attn_poll(ws_b) != 0):
+        raise RuntimeError("device-side timeout during the timed steps")
+
+    # e2e: same step through the C ABI with host buffers, copies inside the timed region
+    e2e = None
+    if not args.no_e2e:
+        hout = torch.empty_like(out, device="cpu").pin_memory()
+        hdx = torch.empty_like(dx, device="cpu").pin_memory(); hdv = torch.empty_like(dv, device="cpu").pin_memory()
+        n_e2e = max(3, min(args.steps, 20))
+        e_s = torch.cuda.Event(enable_timing=True); e_e = torch.cuda.Event(enable_timing=True)
+        h2d = sum(t.numel() * t.element_size() for t in host.values())
+        d2h = hout.numel() * hout.element_size() + (2 * hdx.numel() * hdx.element_size() if w.backward else 0)
+        tot = 0.0
+        for k in range(n_e2e + 1):
+            flush.zero_()
+            e_s.record(stream)
+            x.copy_(host["x"], non_blocking=True); v.copy_(host["v"], non_blocking=True)
+            R.copy_(host["R"], non_blocking=True)
+            if w.backward:
+                dy.copy_(host["dy"], non_blocking=True)
+            step()
+            hout.copy_(out, non_blocking=True)
+            if w.backward:
+                hdx.copy_(dx, non_blocking=True); hdv.copy_(dv, non_blocking=True)
+            e_e.record(stream)
+            torch.cuda.synchronize()
+            if k > 0:
+                tot += e_s.elapsed_time(e_e)
+        e2e_ms = tot / n_e2e
+        e2e = {"value": w.tokens * world / (e2e_ms / 1e3), "unit": "tokens/s", "ms_per_step": e2e_ms,
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+
+    # max over ranks
+    t = torch.tensor([step_ms, e2e["ms_per_step"] if e2e else 0.0], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        dist.destroy_process_group()
+    step_ms = float(t[0])
+    if e2e:
+        e2e["ms_per_step"] = float(t[1])
+        e2e["value"] = w.tokens * world / (e2e["ms_per_step"] / 1e3)
+    if rank != 0:
+        return None
+
+    peaks, peak_src = load_peaks()
+    alg = algorithmic(w)
+    per_stage = {k: {"ms_per_step": ms / args.steps, "calls": c // args.steps, "kernels": kk // args.steps}
+                 for k, (ms, c, kk) in stages.items() if c}
+    launches = sum(kk for (_, _, kk) in stages.values())
+    # dominant kernel: the stage with the most time that is a single kernel we wrote
+    dom_name, dom = max(((k, s) for k, s in per_stage.items() if k in alg["kernel_bytes"]),
+                        key=lambda kv: kv[1]["ms_per_step"])
+    dom_launch_ms = dom["ms_per_step"] / max(dom["calls"], 1)
+    dom_bytes = alg["kernel_bytes"][dom_name] / max(dom["calls"], 1)
+    achieved = dom_bytes / (dom_launch_ms / 1e3) / 1e9
+    hbm = float(peaks["hbm_gbs"])
+    step_bytes_gbs = alg["bytes"] / (step_ms / 1e3) / 1e9
+    t_bytes = alg["bytes"] / (hbm * 1e9)
+    t_flops = alg["attn_flops"] / (float(peaks["bf16_tflops_sustained"]) * 1e12)
+    roof_ms = max(t_bytes, t_flops) * 1e3
+    res = {
+        "metric": METRIC, "value": w.tokens * world / (step_ms / 1e3), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
+        "data": "synthetic: seeded Philox4x32-10 + Box-Muller normals, rounded to bf16",
+        "config": {"workload": describe(w), "global_batch": w.B * world, "seq_len": w.L,
+                   "parallelism": f"{world} independent replica(s), no collective",
+                   "l2": "flushed between timed steps (256 MiB memset outside the step events)"},
+        "roofline": {"bound": "hbm", "kernel": dom_name, "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                     "frac": achieved / hbm, "peak_source": f"{peak_src} hbm_gbs", "traffic": None,
+                     "bytes_per_launch": dom_bytes, "launch_ms": dom_launch_ms},
+        "roofline_step": {"algorithmic_bytes": alg["bytes"], "achieved_gbs": step_bytes_gbs,
+                          "attn_flops": alg["attn_flops"], "hash_flops": alg["hash_flops"],
+                          "roofline_ms": roof_ms, "frac": roof_ms / step_ms,
+                          "peak_source": peak_src},
+        "stages": per_stage,
+        "gpu_launches": int(launches),
+        "e2e": e2e,
+    }
+    res["clocks"] = clk.summary()
+    return res
+
+
+# ------------------------------------------------------------------ oracle on the host cores
+def oracle_slices(w: synth.Workload, n_slices: int, threads: int, L: int | None = None) -> float:
+    """Runs the oracle forward (+ backward) on `n_slices` (batch, head) slices in
+    parallel with `threads` OpenMP threads; returns wall seconds."""
+    from oracle import oracle
+    ws = w.replace(B=1, H=n_slices, L=L or w.L)
+    inp = synth.make_inputs(ws)
+    os.environ["OMP_NUM_THREADS"] = str(threads)
+    t0 = time.perf_counter()
+    res = oracle.fwd(inp["x"], inp["v"], inp["R"], ws.n_buckets, ws.chunk, ws.causal)
+    if ws.backward:
+        oracle.bwd(inp["x"], inp["v"], inp["dy"], res["perm"], ws.chunk, ws.causal)
+    return time.perf_counter() - t0
+
+
+def cpu_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def cpu_baseline(w: synth.Workload) -> dict:
+    cores = cpu_cores()
+    n = max(1, min(cores, w.B * w.H))
+    secs = oracle_slices(w, n, n)
+    step_s = secs * (w.B * w.H) / n
+    return {"value": w.tokens / step_s, "unit": "tokens/s", "cores": n, "kind": "oracle",
+            "sample": f"{n} of {w.B * w.H} (batch, head) slices of {w.name}, full length, fwd"
+                      f"{'+bwd' if w.backward else ''}, one slice per OpenMP thread; {secs:.1f} s wall, "
+                      f"scaled by slice count"}
+
+
+def run_reference(args, w: synth.Workload) -> dict:
+    cores = cpu_cores()
+    n = max(1, min(cores, w.B * w.H))
+    for _ in range(args.warmup):                      # warm-up on a short slice
+        oracle_slices(w, 1, 1, L=max(w.chunk * 2, w.L // 64))
+    times = [oracle_slices(w, n, n) for _ in range(args.steps)]
+    step_s = float(np.mean(times)) * (w.B * w.H) / n
+    value = w.tokens / step_s
+    return {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": 1, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": step_s * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic: seeded Philox4x32-10 + Box-Muller normals",
+            "config": {"workload": describe(w), "global_batch": w.B, "seq_len": w.L,
+                       "parallelism": "host cores (OpenMP over (batch, head) slices)"},
+            "impl": "reference",
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": n, "kind": "oracle",
+                             "sample": f"{n} of {w.B * w.H} (batch, head) slices per step, full length; "
+                                       f"step time scaled by slice count"},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="long_64k", choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    w = synth.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args, w)), flush=True)
+        return
+    res = run_ours(args, w, rank, world)
+    if res is None:
+        return
+    if not args.no_cpu_baseline:
+        res["cpu_baseline"] = cpu_baseline(w)
+    print(json.dumps(res), flush=True)
+
+
+if __name__ == "__main__":
+    main()

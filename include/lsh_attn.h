@@ -1,0 +1,182 @@
+/*
+ * lsh_attn.h -- C ABI of the LSH self-attention library (shared query-key,
+ * forward and backward) for NVIDIA B200 (sm_100a).
+ *
+ * The operation is Reformer's LSH attention as described in the paper note
+ * "Reformer" (eightmm.github.io, on Kitaev, Kaiser, Levskaya, "Reformer: The
+ * Efficient Transformer", ICLR 2020):
+ *   - section "LSH Attention": hash h(x) into buckets, candidate set
+ *     N_LSH(i) = {j : h(q_i) = h(k_j)}, output
+ *     y_i = sum_{j in N(i)} softmax_j(q_i . k_j / sqrt(d_k)) v_j;
+ *   - section "Shared Query-Key Space": Q = K;
+ *   - section "Sorting and Chunking": hash -> sort by bucket -> attention in
+ *     chunks of nearby sorted positions;
+ *   - section "Multiple Hash Rounds": N(i) is the union over R rounds;
+ *   - section "Implementation Reading": the causal mask must survive the
+ *     sort; whether a token may attend to its own position.
+ *
+ * Where the note leaves a step open this library fixes it as follows:
+ *   hash      bucket = argmax over the n_buckets-vector [x R_r ; -x R_r]
+ *             (0-based; the lowest index wins an exact tie), x as stored;
+ *   sort      stable: inside a bucket, original positions increase;
+ *   chunks    sorted slots are cut into chunks of `chunk`; a query in chunk
+ *             c attends to the slots of chunks c-1 and c (chunk 0: itself
+ *             only); there is no bucket-equality mask inside that window;
+ *   keys      k_j = x_j / |x_j| (k_j = 0 when |x_j| = 0); queries are x_i as
+ *             stored; scores are q_i . k_j / sqrt(d);
+ *   self      a query never attends to its own position unless no other
+ *             candidate is left, in which case it attends to itself alone;
+ *   causal    key position <= query position, on ORIGINAL positions;
+ *   rounds    y_i = sum_r softmax_r(lse_r,i) o_r,i, where o_r and lse_r are
+ *             round r's output and natural-log logsumexp;
+ *   backward  gradients w.r.t. x (query and key role) and v with the
+ *             bucket assignment held fixed (it is piecewise constant);
+ *             no gradient w.r.t. R.
+ *
+ * Conventions shared by every entry point
+ *   - Every tensor argument is a DEVICE pointer owned by the caller,
+ *     16-byte aligned, contiguous, row-major:
+ *       qk, v, out, dout, dqk, dv   [B, H, L, d]      element type = dtype
+ *       R                           [n_hashes, d, n_buckets/2], dtype,
+ *                                   shared by every batch row and head
+ *       lse                         [B, H, n_hashes, L]   float32
+ *       perm                        [B, H, n_hashes, L]   int32: perm[s] is
+ *                                   the original position at sorted slot s
+ *       buckets                     [B, H, n_hashes, L]   uint16
+ *   - workspace: a caller-owned device buffer of at least
+ *     lsh_attn_workspace_size() bytes, 256-byte aligned.  The library never
+ *     allocates or frees memory.  One workspace must not be used by two
+ *     calls that may run at the same time.
+ *   - stream: a cudaStream_t (NULL = legacy default stream).  Every call is
+ *     asynchronous on that stream; arguments are checked on the host before
+ *     anything is launched, so an error status means nothing was launched,
+ *     except LSH_ERR_CUDA, which reports a launch failure.
+ *   - d must be 64.  fp32 inputs run on CUDA cores in fp32 (no TF32);
+ *     bf16 inputs run on the tensor cores with fp32 accumulation.
+ */
+#ifndef LSH_ATTN_H
+#define LSH_ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define LSH_ATTN_ABI_VERSION 1
+
+#if defined(__GNUC__)
+#define LSH_API __attribute__((visibility("default")))
+#else
+#define LSH_API
+#endif
+
+typedef enum {
+    LSH_OK = 0,
+    LSH_ERR_ARG = -1,          /* null pointer or unknown enum value            */
+    LSH_ERR_SHAPE = -2,        /* sizes inconsistent (e.g. L % chunk != 0)      */
+    LSH_ERR_ALIGN = -3,        /* a pointer is not 16-byte aligned              */
+    LSH_ERR_UNSUPPORTED = -4,  /* valid request this build does not run (d!=64, */
+                               /* or a forced implementation that cannot run it) */
+    LSH_ERR_CUDA = -5,         /* a CUDA launch or runtime call failed          */
+    LSH_ERR_TIMEOUT = -6,      /* a bounded device-side wait gave up            */
+    LSH_ERR_WORKSPACE = -7     /* workspace smaller than required               */
+} lsh_status;
+
+typedef enum { LSH_F32 = 0, LSH_BF16 = 1 } lsh_dtype;
+
+/* Which kernels run the attention and hash stages.  AUTO picks the tensor-core
+ * kernels for bf16 with chunk == 64 and L % 128 == 0, else the CUDA-core ones. */
+typedef enum { LSH_IMPL_AUTO = 0, LSH_IMPL_SIMT = 1, LSH_IMPL_TC = 2 } lsh_impl;
+
+typedef struct {
+    int32_t B, H, L, d;      /* batch, heads, sequence length, head dim (64)   */
+    int32_t n_buckets;       /* even, 2 .. 65536                               */
+    int32_t n_hashes;        /* rounds R >= 1                                  */
+    int32_t chunk;           /* chunk length m >= 1, L % m == 0                */
+    int32_t causal;          /* 0 or 1                                         */
+    int32_t dtype;           /* lsh_dtype                                      */
+    int32_t impl;            /* lsh_impl                                       */
+} lsh_attn_desc;
+
+/* Bytes of workspace needed by lsh_attn_fwd (for_backward = 0) or by
+ * lsh_attn_bwd (for_backward = 1; includes what a recomputed hash and sort
+ * need when perm is NULL).  Returns 0 for an invalid descriptor. */
+LSH_API size_t lsh_attn_workspace_size(const lsh_attn_desc *desc, int for_backward);
+
+/* Hash stage ("LSH Attention", hash equation): buckets[b,h,r,i] =
+ * argmax([x_i R_r ; -x_i R_r]) for every round r. */
+LSH_API lsh_status lsh_attn_hash(const lsh_attn_desc *desc, const void *qk, const void *R,
+                         uint16_t *buckets, void *workspace, size_t ws_bytes, void *stream);
+
+/* Sort stage ("Sorting and Chunking"): for every (b, h, r) segment, a stable
+ * segmented radix sort of positions by bucket id; writes perm. */
+LSH_API lsh_status lsh_attn_sort(const lsh_attn_desc *desc, const uint16_t *buckets, int32_t *perm,
+                         void *workspace, size_t ws_bytes, void *stream);
+
+/* Attention + round merge for a GIVEN permutation ("LSH Attention" output
+ * equation, "Multiple Hash Rounds"): gathers rows in sorted order, runs the
+ * chunked attention of every round, merges the rounds into out, and writes
+ * the per-round logsumexp lse in original order.  perm must hold, for every
+ * segment, a permutation of 0..L-1 (not checked on the device). */
+LSH_API lsh_status lsh_attn_fwd_sorted(const lsh_attn_desc *desc, const void *qk, const void *v,
+                               const int32_t *perm, void *out, float *lse,
+                               void *workspace, size_t ws_bytes, void *stream);
+
+/* Full forward: hash, sort, attention, merge.  perm_out (nullable) receives
+ * the permutation so that lsh_attn_bwd need not recompute it. */
+LSH_API lsh_status lsh_attn_fwd(const lsh_attn_desc *desc, const void *qk, const void *v, const void *R,
+                        void *out, float *lse, int32_t *perm_out,
+                        void *workspace, size_t ws_bytes, void *stream);
+
+/* Backward of lsh_attn_fwd: given out, lse (from the forward) and dout,
+ * writes dqk and dv.  perm may be NULL, in which case hash and sort are
+ * recomputed from qk and R (R is ignored when perm is given). */
+LSH_API lsh_status lsh_attn_bwd(const lsh_attn_desc *desc, const void *qk, const void *v, const void *R,
+                        const void *out, const float *lse, const int32_t *perm, const void *dout,
+                        void *dqk, void *dv, void *workspace, size_t ws_bytes, void *stream);
+
+/* Device-side status of the calls made with this workspace since the last
+ * poll: synchronises `stream`, returns LSH_ERR_TIMEOUT if a bounded wait in a
+ * kernel gave up, and clears the word.  Call it after a call, not during. */
+LSH_API lsh_status lsh_attn_poll(void *workspace, void *stream);
+
+/* Stage timing.  lsh_attn_trace_begin(capacity) creates `capacity` pairs of
+ * CUDA events and, until lsh_attn_trace_end, every entry point records one
+ * pair around each stage it enqueues (process-wide; not for concurrent use
+ * from several host threads).  lsh_attn_trace_end synchronises on the last
+ * event, adds each recorded stage's elapsed milliseconds into ms[stage],
+ * its invocation count into calls[stage] and the number of kernels it
+ * launched into kernels[stage] (arrays of n >= LSH_STAGE_COUNT entries,
+ * accumulated, not cleared), then destroys the events.  Stages beyond the
+ * capacity are not recorded; the return value is then LSH_ERR_WORKSPACE. */
+typedef enum {
+    LSH_STAGE_HASH = 0,      /* lsh_hash: rotations + argmax                    */
+    LSH_STAGE_SORT,          /* bucket_sort: radix passes                       */
+    LSH_STAGE_NORMS,         /* 1/|x| per row                                   */
+    LSH_STAGE_ATTN_FWD,      /* gather + chunk attention, per-round outputs     */
+    LSH_STAGE_COMBINE,       /* unsort_combine: merge rounds                    */
+    LSH_STAGE_BWD_PREP,      /* logsumexp over rounds, dY.Y, zero accumulators  */
+    LSH_STAGE_ATTN_BWD,      /* chunk attention backward                        */
+    LSH_STAGE_BWD_FINAL,     /* fp32 accumulators -> dqk, dv                    */
+    LSH_STAGE_COUNT
+} lsh_stage;
+
+LSH_API lsh_status lsh_attn_trace_begin(int32_t capacity);
+LSH_API lsh_status lsh_attn_trace_end(float *ms, int32_t *calls, int32_t *kernels, int32_t n);
+
+/* Human-readable name of a status code; never NULL. */
+LSH_API const char *lsh_attn_status_str(lsh_status status);
+
+/* Text of the last CUDA error seen by this thread ("" if none). */
+LSH_API const char *lsh_attn_last_error(void);
+
+/* LSH_ATTN_ABI_VERSION of the loaded library. */
+LSH_API int32_t lsh_attn_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LSH_ATTN_H */

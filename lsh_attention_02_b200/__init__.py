@@ -1,0 +1,211 @@
+"""Python binding of the LSH attention C ABI (liblsh_attn.so).
+
+Argument marshalling only: every step of the computation runs in the CUDA
+library.  Tensors are torch CUDA tensors (torch provides device memory and
+streams); each function passes their device pointers and the current CUDA
+stream to the C entry point of the same name.  The library is loaded on first
+use; if it is missing that call raises ImportError -- there is no CPU fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "liblsh_attn.so")
+
+LSH_F32, LSH_BF16 = 0, 1
+IMPL_AUTO, IMPL_SIMT, IMPL_TC = 0, 1, 2
+
+STATUS = {0: "LSH_OK", -1: "LSH_ERR_ARG", -2: "LSH_ERR_SHAPE", -3: "LSH_ERR_ALIGN",
+          -4: "LSH_ERR_UNSUPPORTED", -5: "LSH_ERR_CUDA", -6: "LSH_ERR_TIMEOUT", -7: "LSH_ERR_WORKSPACE"}
+
+EXPORTED = ("lsh_attn_workspace_size", "lsh_attn_hash", "lsh_attn_sort", "lsh_attn_fwd_sorted", "lsh_attn_fwd",
+            "lsh_attn_bwd", "lsh_attn_poll", "lsh_attn_trace_begin", "lsh_attn_trace_end",
+            "lsh_attn_status_str", "lsh_attn_last_error", "lsh_attn_abi_version")
+
+STAGES = ("hash", "sort", "norms", "attn_fwd", "combine", "bwd_prep", "attn_bwd", "bwd_final")
+
+
+class LshAttnError(RuntimeError):
+    def __init__(self, status: int, where: str, detail: str = ""):
+        self.status = status
+        super().__init__(f"{where}: {STATUS.get(status, status)}" + (f" ({detail})" if detail else ""))
+
+
+class Desc(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in
+                ("B", "H", "L", "d", "n_buckets", "n_hashes", "chunk", "causal", "dtype", "impl")]
+
+
+_lib = None
+
+
+def load_library(path: str = LIB_PATH):
+    """Loads liblsh_attn.so and declares its signatures (raises if absent)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise ImportError(f"{path} is missing: build it with `python -m lsh_attention_02_b200.build`")
+    L = ctypes.CDLL(path)
+    P = ctypes.c_void_p
+    DP = ctypes.POINTER(Desc)
+    S = ctypes.c_size_t
+    L.lsh_attn_workspace_size.argtypes = [DP, ctypes.c_int]
+    L.lsh_attn_workspace_size.restype = S
+    L.lsh_attn_hash.argtypes = [DP, P, P, P, P, S, P]
+    L.lsh_attn_sort.argtypes = [DP, P, P, P, S, P]
+    L.lsh_attn_fwd_sorted.argtypes = [DP, P, P, P, P, P, P, S, P]
+    L.lsh_attn_fwd.argtypes = [DP, P, P, P, P, P, P, P, S, P]
+    L.lsh_attn_bwd.argtypes = [DP, P, P, P, P, P, P, P, P, P, P, S, P]
+    L.lsh_attn_poll.argtypes = [P, P]
+    L.lsh_attn_trace_begin.argtypes = [ctypes.c_int32]
+    L.lsh_attn_trace_end.argtypes = [ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_int32),
+                                     ctypes.POINTER(ctypes.c_int32), ctypes.c_int32]
+    L.lsh_attn_status_str.argtypes = [ctypes.c_int]
+    L.lsh_attn_status_str.restype = ctypes.c_char_p
+    L.lsh_attn_last_error.argtypes = []
+    L.lsh_attn_last_error.restype = ctypes.c_char_p
+    L.lsh_attn_abi_version.argtypes = []
+    L.lsh_attn_abi_version.restype = ctypes.c_int32
+    for name in EXPORTED:
+        getattr(L, name).restype = getattr(L, name).restype or ctypes.c_int
+    _lib = L
+    return L
+
+
+def make_desc(B, H, L, d, n_buckets, n_hashes, chunk, causal, dtype, impl=IMPL_AUTO) -> Desc:
+    if isinstance(dtype, torch.dtype):
+        dtype = {torch.float32: LSH_F32, torch.bfloat16: LSH_BF16}[dtype]
+    return Desc(B, H, L, d, n_buckets, n_hashes, chunk, int(bool(causal)), dtype, impl)
+
+
+def desc_for(x: torch.Tensor, n_buckets: int, n_hashes: int, chunk: int, causal: bool, impl: int = IMPL_AUTO):
+    B, H, L, d = x.shape
+    return make_desc(B, H, L, d, n_buckets, n_hashes, chunk, causal, x.dtype, impl)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(t: torch.Tensor):
+    return ctypes.c_void_p(torch.cuda.current_stream(t.device).cuda_stream)
+
+
+def _check(rc: int, where: str):
+    if rc != 0:
+        detail = load_library().lsh_attn_last_error().decode() if rc == -5 else ""
+        raise LshAttnError(rc, where, detail)
+
+
+def workspace_size(desc: Desc, for_backward: bool) -> int:
+    return int(load_library().lsh_attn_workspace_size(ctypes.byref(desc), int(for_backward)))
+
+
+def workspace(desc: Desc, for_backward: bool, device) -> torch.Tensor:
+    n = workspace_size(desc, for_backward)
+    if n == 0:
+        raise LshAttnError(-1, "workspace_size", "invalid descriptor")
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def _ws(desc, for_backward, ref, ws):
+    return ws if ws is not None else workspace(desc, for_backward, ref.device)
+
+
+def lsh_attn_hash(desc: Desc, qk, R, buckets, ws=None):
+    ws = _ws(desc, False, qk, ws)
+    _check(load_library().lsh_attn_hash(ctypes.byref(desc), _ptr(qk), _ptr(R), _ptr(buckets), _ptr(ws),
+                                         ws.numel(), _stream(qk)), "lsh_attn_hash")
+    return buckets
+
+
+def lsh_attn_sort(desc: Desc, buckets, perm, ws=None):
+    ws = _ws(desc, False, buckets, ws)
+    _check(load_library().lsh_attn_sort(ctypes.byref(desc), _ptr(buckets), _ptr(perm), _ptr(ws), ws.numel(),
+                                         _stream(buckets)), "lsh_attn_sort")
+    return perm
+
+
+def lsh_attn_fwd_sorted(desc: Desc, qk, v, perm, out, lse, ws=None):
+    ws = _ws(desc, False, qk, ws)
+    _check(load_library().lsh_attn_fwd_sorted(ctypes.byref(desc), _ptr(qk), _ptr(v), _ptr(perm), _ptr(out),
+                                               _ptr(lse), _ptr(ws), ws.numel(), _stream(qk)),
+           "lsh_attn_fwd_sorted")
+    return out, lse
+
+
+def lsh_attn_fwd(desc: Desc, qk, v, R, out, lse, perm_out=None, ws=None):
+    ws = _ws(desc, False, qk, ws)
+    _check(load_library().lsh_attn_fwd(ctypes.byref(desc), _ptr(qk), _ptr(v), _ptr(R), _ptr(out), _ptr(lse),
+                                        _ptr(perm_out), _ptr(ws), ws.numel(), _stream(qk)), "lsh_attn_fwd")
+    return out, lse
+
+
+def lsh_attn_bwd(desc: Desc, qk, v, R, out, lse, perm, dout, dqk, dv, ws=None):
+    ws = _ws(desc, True, qk, ws)
+    _check(load_library().lsh_attn_bwd(ctypes.byref(desc), _ptr(qk), _ptr(v), _ptr(R), _ptr(out), _ptr(lse),
+                                        _ptr(perm), _ptr(dout), _ptr(dqk), _ptr(dv), _ptr(ws), ws.numel(),
+                                        _stream(qk)), "lsh_attn_bwd")
+    return dqk, dv
+
+
+def lsh_attn_poll(ws: torch.Tensor) -> int:
+    """Synchronises the current stream and returns the device status (0 or LSH_ERR_TIMEOUT)."""
+    return int(load_library().lsh_attn_poll(_ptr(ws), _stream(ws)))
+
+
+def trace_begin(capacity: int = 4096):
+    """Starts recording a CUDA event pair around every stage the library enqueues."""
+    _check(load_library().lsh_attn_trace_begin(int(capacity)), "lsh_attn_trace_begin")
+
+
+def trace_end() -> dict:
+    """Stops recording; returns {stage: (total_ms, calls, kernels)}."""
+    n = len(STAGES)
+    ms = (ctypes.c_float * n)(); calls = (ctypes.c_int32 * n)(); ker = (ctypes.c_int32 * n)()
+    _check(load_library().lsh_attn_trace_end(ms, calls, ker, n), "lsh_attn_trace_end")
+    return {name: (float(ms[i]), int(calls[i]), int(ker[i])) for i, name in enumerate(STAGES)}
+
+
+def outputs_like(desc: Desc, qk: torch.Tensor):
+    """Fresh (out, lse, perm) buffers for a forward call."""
+    B, H, L = desc.B, desc.H, desc.L
+    out = torch.empty_like(qk)
+    lse = torch.empty((B, H, desc.n_hashes, L), dtype=torch.float32, device=qk.device)
+    perm = torch.empty((B, H, desc.n_hashes, L), dtype=torch.int32, device=qk.device)
+    return out, lse, perm
+
+
+class LSHAttention(torch.autograd.Function):
+    """y = LSHAttention.apply(qk, v, R, n_buckets, chunk, causal[, impl]); gradients for qk and v."""
+
+    @staticmethod
+    def forward(ctx, qk, v, R, n_buckets, chunk, causal, impl=IMPL_AUTO):
+        qk = qk.contiguous(); v = v.contiguous(); R = R.contiguous()
+        desc = desc_for(qk, n_buckets, R.shape[0], chunk, causal, impl)
+        out, lse, perm = outputs_like(desc, qk)
+        lsh_attn_fwd(desc, qk, v, R, out, lse, perm)
+        ctx.desc = desc
+        ctx.save_for_backward(qk, v, R, out, lse, perm)
+        ctx.mark_non_differentiable(lse)
+        return out, lse
+
+    @staticmethod
+    def backward(ctx, dout, _dlse):
+        qk, v, R, out, lse, perm = ctx.saved_tensors
+        dqk = torch.empty_like(qk); dv = torch.empty_like(v)
+        lsh_attn_bwd(ctx.desc, qk, v, R, out, lse, perm, dout.contiguous(), dqk, dv)
+        return dqk, dv, None, None, None, None, None
+
+
+def lsh_attention(qk, v, R, n_buckets, chunk=64, causal=False, impl=IMPL_AUTO):
+    """Reformer LSH self-attention with shared query-key: returns (out, lse).
+
+    qk, v: [B, H, L, 64] CUDA tensors (float32 or bfloat16); R: [n_hashes, 64, n_buckets/2]."""
+    return LSHAttention.apply(qk, v, R, n_buckets, chunk, causal, impl)
+

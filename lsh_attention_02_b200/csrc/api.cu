@@ -1,0 +1,373 @@
+// C ABI of the LSH attention library: argument checks, workspace layout and
+// the launch sequence of each entry point.  Every entry point checks its
+// arguments on the host before launching anything and never allocates.
+#include <stdio.h>
+#include <string.h>
+
+#include "common.cuh"
+
+namespace lsh {
+
+static thread_local char g_last_error[256] = "";
+
+static lsh_status cuda_fail(cudaError_t e, const char *where)
+{
+    snprintf(g_last_error, sizeof(g_last_error), "%s: %s", where, cudaGetErrorString(e));
+    return LSH_ERR_CUDA;
+}
+
+#define LSH_TRY(expr, where)                                        \
+    do {                                                            \
+        cudaError_t e_ = (expr);                                    \
+        if (e_ != cudaSuccess) return cuda_fail(e_, where);         \
+    } while (0)
+
+static size_t align_up(size_t a, size_t b) { return (a + b - 1) / b * b; }
+
+// ------------------------------------------------------------------ stage trace
+struct Trace {
+    bool on = false;
+    int cap = 0, used = 0;
+    bool overflow = false;
+    cudaEvent_t *ev = nullptr;      // 2 per record
+    int *stage = nullptr, *kernels = nullptr;
+};
+static Trace g_trace;
+
+// Records one event pair around a stage; `fn` enqueues the stage's kernels.
+template <typename F>
+static cudaError_t staged(int stage, int n_kernels, cudaStream_t st, F fn)
+{
+    const bool rec = g_trace.on && g_trace.used < g_trace.cap;
+    if (g_trace.on && !rec) g_trace.overflow = true;
+    if (rec) {
+        cudaError_t e = cudaEventRecord(g_trace.ev[2 * g_trace.used], st);
+        if (e != cudaSuccess) return e;
+    }
+    cudaError_t e = fn();
+    if (e != cudaSuccess) return e;
+    if (rec) {
+        e = cudaEventRecord(g_trace.ev[2 * g_trace.used + 1], st);
+        if (e != cudaSuccess) return e;
+        g_trace.stage[g_trace.used] = stage;
+        g_trace.kernels[g_trace.used] = n_kernels;
+        ++g_trace.used;
+    }
+    return cudaSuccess;
+}
+
+Workspace plan_workspace(const Problem &p, bool backward, bool tc_attn, char *base)
+{
+    Workspace w{};
+    size_t off = 0;
+    auto take = [&](size_t bytes) -> char * {
+        char *ptr = base ? base + off : nullptr;
+        off = align_up(off + bytes, 256);
+        return ptr;
+    };
+    const size_t S = (size_t)p.S(), L = (size_t)p.L, T = (size_t)p.tokens();
+    const SortPlan sp = make_sort_plan(p.nb, p.L);
+    w.status = (uint32_t *)take(256);
+    w.invnorm = (float *)take(T * sizeof(float));
+    w.buckets = (uint16_t *)take(S * L * sizeof(uint16_t));
+    w.sort_keys = (uint16_t *)take(sp.passes > 1 ? S * L * sizeof(uint16_t) : 0);
+    w.sort_vals = (int32_t *)take(sp.passes > 1 ? S * L * sizeof(int32_t) : 0);
+    w.sort_counts = (uint32_t *)take(S * (size_t)sp.max_radix * sp.n_tiles * sizeof(uint32_t));
+    w.perm = (int32_t *)take(S * L * sizeof(int32_t));
+    if (!backward) {
+        w.o_r = take(S * L * kDim * (tc_attn ? 2 : 4));
+    } else {
+        w.lse_all = (float *)take(T * sizeof(float));
+        w.delta = (float *)take(T * sizeof(float));
+        w.self_only = (uint8_t *)take(tc_attn ? 0 : S * L);
+        w.dx_acc = (float *)take(T * kDim * sizeof(float));
+        w.dv_acc = (float *)take(T * kDim * sizeof(float));
+    }
+    w.bytes = off;
+    return w;
+}
+
+static lsh_status check_desc(const lsh_attn_desc *d, Problem *p)
+{
+    if (!d) return LSH_ERR_ARG;
+    if (d->dtype != LSH_F32 && d->dtype != LSH_BF16) return LSH_ERR_ARG;
+    if (d->impl != LSH_IMPL_AUTO && d->impl != LSH_IMPL_SIMT && d->impl != LSH_IMPL_TC) return LSH_ERR_ARG;
+    if (d->causal != 0 && d->causal != 1) return LSH_ERR_ARG;
+    if (d->B < 1 || d->H < 1 || d->L < 1 || d->n_hashes < 1 || d->chunk < 1) return LSH_ERR_SHAPE;
+    if (d->n_buckets < 2 || d->n_buckets % 2 != 0 || d->n_buckets > 65536) return LSH_ERR_SHAPE;
+    if (d->L % d->chunk != 0) return LSH_ERR_SHAPE;
+    if (d->d != kDim) return LSH_ERR_UNSUPPORTED;
+    long long segs = (long long)d->B * d->H * d->n_hashes;
+    if (segs > 65535) return LSH_ERR_UNSUPPORTED;     // grid.y of the per-segment kernels
+    p->B = d->B; p->H = d->H; p->L = d->L; p->d = d->d; p->nb = d->n_buckets;
+    p->R = d->n_hashes; p->m = d->chunk; p->causal = d->causal; p->dtype = d->dtype;
+    return LSH_OK;
+}
+
+// Which kernels run the attention (and the hash) for this request.
+struct Choice {
+    bool tc_attn;
+    bool tc_hash;
+};
+static lsh_status choose(const lsh_attn_desc *d, const Problem &p, Choice *c)
+{
+    bool attn_ok = attn_tc_supported(p), hash_ok = hash_tc_supported(p);
+    if (d->impl == LSH_IMPL_SIMT) { c->tc_attn = false; c->tc_hash = false; return LSH_OK; }
+    if (d->impl == LSH_IMPL_TC) {
+        if (!attn_ok) return LSH_ERR_UNSUPPORTED;
+        c->tc_attn = true;
+        c->tc_hash = hash_ok;
+        return LSH_OK;
+    }
+    c->tc_attn = attn_ok;
+    c->tc_hash = hash_ok;
+    return LSH_OK;
+}
+
+static bool aligned16(const void *ptr) { return ((uintptr_t)ptr & 15u) == 0; }
+
+static lsh_status check_ptrs(std::initializer_list<const void *> ptrs)
+{
+    for (const void *q : ptrs) if (!q) return LSH_ERR_ARG;
+    for (const void *q : ptrs) if (!aligned16(q)) return LSH_ERR_ALIGN;
+    return LSH_OK;
+}
+
+static lsh_status check_ws(void *ws, size_t ws_bytes, size_t need)
+{
+    if (!ws) return LSH_ERR_ARG;
+    if (((uintptr_t)ws & 255u) != 0) return LSH_ERR_ALIGN;
+    if (ws_bytes < need) return LSH_ERR_WORKSPACE;
+    return LSH_OK;
+}
+
+// hash + sort into perm (internal helper shared by fwd and bwd)
+static lsh_status run_hash_sort(const Problem &p, const Choice &c, const void *qk, const void *R, int32_t *perm,
+                                const Workspace &w, cudaStream_t st)
+{
+    LSH_TRY(staged(LSH_STAGE_HASH, 1, st, [&] {
+                return c.tc_hash ? launch_hash_tc(p, qk, R, w.buckets, w.status, st)
+                                 : launch_hash_simt(p, qk, R, w.buckets, st);
+            }), "hash");
+    LSH_TRY(staged(LSH_STAGE_SORT, 3 * make_sort_plan(p.nb, p.L).passes, st,
+                   [&] { return launch_sort(p, w.buckets, perm, w, st); }), "sort");
+    return LSH_OK;
+}
+
+static lsh_status run_attn_fwd(const Problem &p, const Choice &c, const void *qk, const void *v,
+                               const int32_t *perm, void *out, float *lse, const Workspace &w, cudaStream_t st)
+{
+    LSH_TRY(staged(LSH_STAGE_NORMS, 1, st, [&] { return launch_invnorm(p, qk, w.invnorm, st); }), "key norms");
+    LSH_TRY(staged(LSH_STAGE_ATTN_FWD, 1, st, [&] {
+                return c.tc_attn
+                           ? launch_attn_fwd_tc(p, qk, v, perm, w.invnorm, (__nv_bfloat16 *)w.o_r, lse, w.status, st)
+                           : launch_attn_fwd_simt(p, qk, v, perm, w.invnorm, (float *)w.o_r, lse, st);
+            }), "attention forward");
+    LSH_TRY(staged(LSH_STAGE_COMBINE, 1, st, [&] { return launch_combine(p, w.o_r, c.tc_attn, lse, out, st); }),
+            "round merge");
+    return LSH_OK;
+}
+
+}  // namespace lsh
+
+using namespace lsh;
+
+extern "C" {
+
+size_t lsh_attn_workspace_size(const lsh_attn_desc *desc, int for_backward)
+{
+    Problem p;
+    Choice c;
+    if (check_desc(desc, &p) != LSH_OK || choose(desc, p, &c) != LSH_OK) return 0;
+    return plan_workspace(p, for_backward != 0, c.tc_attn, nullptr).bytes;
+}
+
+lsh_status lsh_attn_hash(const lsh_attn_desc *desc, const void *qk, const void *R, uint16_t *buckets,
+                         void *workspace, size_t ws_bytes, void *stream)
+{
+    Problem p;
+    Choice c;
+    lsh_status s;
+    if ((s = check_desc(desc, &p)) != LSH_OK) return s;
+    if ((s = choose(desc, p, &c)) != LSH_OK) return s;
+    if ((s = check_ptrs({qk, R})) != LSH_OK) return s;
+    if (!buckets) return LSH_ERR_ARG;
+    Workspace w = plan_workspace(p, false, c.tc_attn, nullptr);
+    if ((s = check_ws(workspace, ws_bytes, w.bytes)) != LSH_OK) return s;
+    w = plan_workspace(p, false, c.tc_attn, (char *)workspace);
+    cudaStream_t st = (cudaStream_t)stream;
+    LSH_TRY(staged(LSH_STAGE_HASH, 1, st, [&] {
+                return c.tc_hash ? launch_hash_tc(p, qk, R, buckets, w.status, st)
+                                 : launch_hash_simt(p, qk, R, buckets, st);
+            }), "hash");
+    return LSH_OK;
+}
+
+lsh_status lsh_attn_sort(const lsh_attn_desc *desc, const uint16_t *buckets, int32_t *perm, void *workspace,
+                         size_t ws_bytes, void *stream)
+{
+    Problem p;
+    Choice c;
+    lsh_status s;
+    if ((s = check_desc(desc, &p)) != LSH_OK) return s;
+    if ((s = choose(desc, p, &c)) != LSH_OK) return s;
+    if (!buckets || !perm) return LSH_ERR_ARG;
+    Workspace w = plan_workspace(p, false, c.tc_attn, nullptr);
+    if ((s = check_ws(workspace, ws_bytes, w.bytes)) != LSH_OK) return s;
+    w = plan_workspace(p, false, c.tc_attn, (char *)workspace);
+    cudaStream_t st = (cudaStream_t)stream;
+    LSH_TRY(staged(LSH_STAGE_SORT, 3 * make_sort_plan(p.nb, p.L).passes, st,
+                   [&] { return launch_sort(p, buckets, perm, w, st); }), "sort");
+    return LSH_OK;
+}
+
+lsh_status lsh_attn_fwd_sorted(const lsh_attn_desc *desc, const void *qk, const void *v, const int32_t *perm,
+                               void *out, float *lse, void *workspace, size_t ws_bytes, void *stream)
+{
+    Problem p;
+    Choice c;
+    lsh_status s;
+    if ((s = check_desc(desc, &p)) != LSH_OK) return s;
+    if ((s = choose(desc, p, &c)) != LSH_OK) return s;
+    if ((s = check_ptrs({qk, v, out, lse})) != LSH_OK) return s;
+    if (!perm) return LSH_ERR_ARG;
+    Workspace w = plan_workspace(p, false, c.tc_attn, nullptr);
+    if ((s = check_ws(workspace, ws_bytes, w.bytes)) != LSH_OK) return s;
+    w = plan_workspace(p, false, c.tc_attn, (char *)workspace);
+    cudaStream_t st = (cudaStream_t)stream;
+    LSH_TRY(cudaMemsetAsync(w.status, 0, sizeof(uint32_t), st), "status reset");
+    return run_attn_fwd(p, c, qk, v, perm, out, lse, w, st);
+}
+
+lsh_status lsh_attn_fwd(const lsh_attn_desc *desc, const void *qk, const void *v, const void *R, void *out,
+                        float *lse, int32_t *perm_out, void *workspace, size_t ws_bytes, void *stream)
+{
+    Problem p;
+    Choice c;
+    lsh_status s;
+    if ((s = check_desc(desc, &p)) != LSH_OK) return s;
+    if ((s = choose(desc, p, &c)) != LSH_OK) return s;
+    if ((s = check_ptrs({qk, v, R, out, lse})) != LSH_OK) return s;
+    Workspace w = plan_workspace(p, false, c.tc_attn, nullptr);
+    if ((s = check_ws(workspace, ws_bytes, w.bytes)) != LSH_OK) return s;
+    w = plan_workspace(p, false, c.tc_attn, (char *)workspace);
+    cudaStream_t st = (cudaStream_t)stream;
+    int32_t *perm = perm_out ? perm_out : w.perm;
+    LSH_TRY(cudaMemsetAsync(w.status, 0, sizeof(uint32_t), st), "status reset");
+    if ((s = run_hash_sort(p, c, qk, R, perm, w, st)) != LSH_OK) return s;
+    return run_attn_fwd(p, c, qk, v, perm, out, lse, w, st);
+}
+
+lsh_status lsh_attn_bwd(const lsh_attn_desc *desc, const void *qk, const void *v, const void *R, const void *out,
+                        const float *lse, const int32_t *perm, const void *dout, void *dqk, void *dv,
+                        void *workspace, size_t ws_bytes, void *stream)
+{
+    Problem p;
+    Choice c;
+    lsh_status s;
+    if ((s = check_desc(desc, &p)) != LSH_OK) return s;
+    if ((s = choose(desc, p, &c)) != LSH_OK) return s;
+    if ((s = check_ptrs({qk, v, out, lse, dout, dqk, dv})) != LSH_OK) return s;
+    if (!perm && !R) return LSH_ERR_ARG;
+    Workspace w = plan_workspace(p, true, c.tc_attn, nullptr);
+    if ((s = check_ws(workspace, ws_bytes, w.bytes)) != LSH_OK) return s;
+    w = plan_workspace(p, true, c.tc_attn, (char *)workspace);
+    cudaStream_t st = (cudaStream_t)stream;
+    LSH_TRY(cudaMemsetAsync(w.status, 0, sizeof(uint32_t), st), "status reset");
+    if (!perm) {
+        if ((s = run_hash_sort(p, c, qk, R, w.perm, w, st)) != LSH_OK) return s;
+        perm = w.perm;
+    }
+    LSH_TRY(staged(LSH_STAGE_NORMS, 1, st, [&] { return launch_invnorm(p, qk, w.invnorm, st); }), "key norms");
+    LSH_TRY(staged(LSH_STAGE_BWD_PREP, 1, st, [&] {
+                return launch_bwd_prep(p, lse, out, dout, w.lse_all, w.delta, w.dx_acc, w.dv_acc, st);
+            }), "backward prologue");
+    LSH_TRY(staged(LSH_STAGE_ATTN_BWD, c.tc_attn ? 1 : 2, st, [&] {
+                return c.tc_attn ? launch_attn_bwd_tc(p, qk, v, dout, perm, w.invnorm, w.lse_all, w.delta, w.dx_acc,
+                                                      w.dv_acc, w.status, st)
+                                 : launch_attn_bwd_simt(p, qk, v, dout, perm, w.invnorm, w.lse_all, w.delta,
+                                                        w.self_only, w.dx_acc, w.dv_acc, st);
+            }), "attention backward");
+    LSH_TRY(staged(LSH_STAGE_BWD_FINAL, 1, st,
+                   [&] { return launch_bwd_finalize(p, w.dx_acc, w.dv_acc, dqk, dv, st); }),
+            "backward epilogue");
+    return LSH_OK;
+}
+
+lsh_status lsh_attn_poll(void *workspace, void *stream)
+{
+    if (!workspace) return LSH_ERR_ARG;
+    cudaStream_t st = (cudaStream_t)stream;
+    uint32_t word = 0;
+    LSH_TRY(cudaMemcpyAsync(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost, st), "status read");
+    LSH_TRY(cudaStreamSynchronize(st), "status read");
+    LSH_TRY(cudaMemsetAsync(workspace, 0, sizeof(word), st), "status clear");
+    return (word & kStatusTimeout) ? LSH_ERR_TIMEOUT : LSH_OK;
+}
+
+lsh_status lsh_attn_trace_begin(int32_t capacity)
+{
+    if (capacity < 1 || g_trace.on) return LSH_ERR_ARG;
+    Trace t;
+    t.cap = capacity;
+    t.ev = new cudaEvent_t[2 * (size_t)capacity];
+    t.stage = new int[capacity];
+    t.kernels = new int[capacity];
+    for (int i = 0; i < 2 * capacity; ++i) {
+        cudaError_t e = cudaEventCreate(&t.ev[i]);
+        if (e != cudaSuccess) {
+            for (int k = 0; k < i; ++k) cudaEventDestroy(t.ev[k]);
+            delete[] t.ev; delete[] t.stage; delete[] t.kernels;
+            return cuda_fail(e, "trace events");
+        }
+    }
+    t.on = true;
+    g_trace = t;
+    return LSH_OK;
+}
+
+lsh_status lsh_attn_trace_end(float *ms, int32_t *calls, int32_t *kernels, int32_t n)
+{
+    if (!g_trace.on) return LSH_ERR_ARG;
+    if (!ms || !calls || !kernels || n < LSH_STAGE_COUNT) return LSH_ERR_ARG;
+    Trace t = g_trace;
+    g_trace = Trace();
+    lsh_status rc = LSH_OK;
+    if (t.used > 0) {
+        cudaError_t e = cudaEventSynchronize(t.ev[2 * t.used - 1]);
+        if (e != cudaSuccess) rc = cuda_fail(e, "trace sync");
+    }
+    for (int i = 0; rc == LSH_OK && i < t.used; ++i) {
+        float x = 0.f;
+        cudaError_t e = cudaEventElapsedTime(&x, t.ev[2 * i], t.ev[2 * i + 1]);
+        if (e != cudaSuccess) { rc = cuda_fail(e, "trace elapsed"); break; }
+        ms[t.stage[i]] += x;
+        calls[t.stage[i]] += 1;
+        kernels[t.stage[i]] += t.kernels[i];
+    }
+    for (int i = 0; i < 2 * t.cap; ++i) cudaEventDestroy(t.ev[i]);
+    delete[] t.ev; delete[] t.stage; delete[] t.kernels;
+    if (rc == LSH_OK && t.overflow) rc = LSH_ERR_WORKSPACE;
+    return rc;
+}
+
+const char *lsh_attn_status_str(lsh_status status)
+{
+    switch (status) {
+    case LSH_OK: return "ok";
+    case LSH_ERR_ARG: return "invalid argument (null pointer or unknown enum value)";
+    case LSH_ERR_SHAPE: return "inconsistent sizes";
+    case LSH_ERR_ALIGN: return "pointer not aligned";
+    case LSH_ERR_UNSUPPORTED: return "unsupported configuration";
+    case LSH_ERR_CUDA: return "CUDA error";
+    case LSH_ERR_TIMEOUT: return "device-side wait timed out";
+    case LSH_ERR_WORKSPACE: return "workspace too small";
+    }
+    return "unknown status";
+}
+
+const char *lsh_attn_last_error(void) { return g_last_error; }
+
+int32_t lsh_attn_abi_version(void) { return LSH_ATTN_ABI_VERSION; }
+
+}  // extern "C"

@@ -1,0 +1,150 @@
+// Shared device helpers and the internal launch interface of the LSH
+// attention library.  Nothing here is part of the C ABI.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/lsh_attn.h"
+
+namespace lsh {
+
+constexpr int kDim = 64;              // head dimension supported by every kernel
+
+// ---------------------------------------------------------------- problem
+struct Problem {
+    int B, H, L, d, nb, R, m, causal, dtype;
+    long long BH() const { return (long long)B * H; }
+    long long S() const { return BH() * R; }         // (b, h, round) segments
+    long long tokens() const { return BH() * L; }
+};
+
+// ---------------------------------------------------------------- sort plan
+constexpr int kSortTile = 2048;       // positions per sort CTA
+constexpr int kSortThreads = 256;     // 8 warps x 32 lanes x 8 iterations
+
+struct SortPlan {
+    int passes;                       // 1 or 2
+    int shift[2];
+    int bits[2];
+    int n_tiles;
+    int max_radix;
+};
+SortPlan make_sort_plan(int n_buckets, int L);
+
+// ---------------------------------------------------------------- workspace
+struct Workspace {
+    uint32_t *status;                 // device status word (timeouts)
+    float *invnorm;                   // [BH, L]  1/|x| (0 for a zero row)
+    uint16_t *buckets;                // [S, L]
+    uint16_t *sort_keys;              // [S, L]   first-pass keys
+    int32_t *sort_vals;               // [S, L]   first-pass positions
+    uint32_t *sort_counts;            // [S, radix, tiles]
+    int32_t *perm;                    // [S, L]   internal permutation
+    void *o_r;                        // [S, L, 64] per-round outputs
+    float *lse_all;                   // [BH, L]  logsumexp over rounds
+    float *delta;                     // [BH, L]  dY . Y
+    uint8_t *self_only;               // [S, L]   per sorted slot
+    float *dx_acc;                    // [BH, L, 64]
+    float *dv_acc;                    // [BH, L, 64]
+    size_t bytes;
+};
+// Lays the workspace out from `base` (or from 0 when base is null, to size it).
+Workspace plan_workspace(const Problem &p, bool backward, bool tc_attn, char *base);
+
+// ---------------------------------------------------------------- helpers
+__device__ __forceinline__ float to_f(float a) { return a; }
+__device__ __forceinline__ float to_f(__nv_bfloat16 a) { return __bfloat162float(a); }
+template <typename T> __device__ __forceinline__ T from_f(float a);
+template <> __device__ __forceinline__ float from_f<float>(float a) { return a; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float a) { return __float2bfloat16_rn(a); }
+
+// Loads a 64-element row into registers as float.
+__device__ __forceinline__ void load_row(const float *p, float *r)
+{
+    const float4 *q = reinterpret_cast<const float4 *>(p);
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+        float4 a = q[k];
+        r[4 * k] = a.x; r[4 * k + 1] = a.y; r[4 * k + 2] = a.z; r[4 * k + 3] = a.w;
+    }
+}
+__device__ __forceinline__ void load_row(const __nv_bfloat16 *p, float *r)
+{
+    const uint4 *q = reinterpret_cast<const uint4 *>(p);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+        uint4 a = q[k];
+        const uint32_t w[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            r[8 * k + 2 * e] = __uint_as_float(w[e] << 16);
+            r[8 * k + 2 * e + 1] = __uint_as_float(w[e] & 0xFFFF0000u);
+        }
+    }
+}
+
+// Sequential fp32 dot product of two 64-vectors (fixed order, fused multiply-add).
+__device__ __forceinline__ float dot64(const float *a, const float *b)
+{
+    float s = 0.f;
+#pragma unroll
+    for (int k = 0; k < 64; ++k) s = fmaf(a[k], b[k], s);
+    return s;
+}
+
+__device__ __forceinline__ void store_row(float *p, const float *r)
+{
+    float4 *q = reinterpret_cast<float4 *>(p);
+#pragma unroll
+    for (int k = 0; k < 16; ++k) q[k] = make_float4(r[4 * k], r[4 * k + 1], r[4 * k + 2], r[4 * k + 3]);
+}
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
+{
+    __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t *>(&h);
+}
+__device__ __forceinline__ void store_row(__nv_bfloat16 *p, const float *r)
+{
+    uint4 *q = reinterpret_cast<uint4 *>(p);
+#pragma unroll
+    for (int k = 0; k < 8; ++k)
+        q[k] = make_uint4(pack_bf16x2(r[8 * k], r[8 * k + 1]), pack_bf16x2(r[8 * k + 2], r[8 * k + 3]),
+                          pack_bf16x2(r[8 * k + 4], r[8 * k + 5]), pack_bf16x2(r[8 * k + 6], r[8 * k + 7]));
+}
+
+// ---------------------------------------------------------------- launchers
+// Every launcher enqueues on `st` and returns cudaGetLastError().
+cudaError_t launch_invnorm(const Problem &p, const void *x, float *invnorm, cudaStream_t st);
+cudaError_t launch_hash_simt(const Problem &p, const void *x, const void *R, uint16_t *buckets, cudaStream_t st);
+cudaError_t launch_hash_tc(const Problem &p, const void *x, const void *R, uint16_t *buckets,
+                           uint32_t *status, cudaStream_t st);
+bool hash_tc_supported(const Problem &p);
+cudaError_t launch_sort(const Problem &p, const uint16_t *buckets, int32_t *perm, const Workspace &ws,
+                        cudaStream_t st);
+cudaError_t launch_attn_fwd_simt(const Problem &p, const void *x, const void *v, const int32_t *perm,
+                                 const float *invnorm, float *o_r, float *lse, cudaStream_t st);
+cudaError_t launch_attn_fwd_tc(const Problem &p, const void *x, const void *v, const int32_t *perm,
+                               const float *invnorm, __nv_bfloat16 *o_r, float *lse, uint32_t *status,
+                               cudaStream_t st);
+bool attn_tc_supported(const Problem &p);
+cudaError_t launch_combine(const Problem &p, const void *o_r, bool o_r_bf16, const float *lse, void *out,
+                           cudaStream_t st);
+cudaError_t launch_bwd_prep(const Problem &p, const float *lse, const void *out, const void *dout,
+                            float *lse_all, float *delta, float *dx_acc, float *dv_acc, cudaStream_t st);
+cudaError_t launch_attn_bwd_simt(const Problem &p, const void *x, const void *v, const void *dout,
+                                 const int32_t *perm, const float *invnorm, const float *lse_all,
+                                 const float *delta, uint8_t *self_only, float *dx_acc, float *dv_acc,
+                                 cudaStream_t st);
+cudaError_t launch_attn_bwd_tc(const Problem &p, const void *x, const void *v, const void *dout,
+                               const int32_t *perm, const float *invnorm, const float *lse_all,
+                               const float *delta, float *dx_acc, float *dv_acc, uint32_t *status,
+                               cudaStream_t st);
+cudaError_t launch_bwd_finalize(const Problem &p, const float *dx_acc, const float *dv_acc, void *dqk, void *dv,
+                                cudaStream_t st);
+
+// Status bits written by kernels into Workspace::status.
+constexpr uint32_t kStatusTimeout = 1u;
+
+}  // namespace lsh

@@ -1,0 +1,445 @@
+// CUDA-core kernels: key norms, the fp32 hash, chunked attention forward and
+// backward on CUDA cores, the round merge and the backward prologue/epilogue.
+//
+// These run every stage for fp32 inputs (no TF32 anywhere) and for shapes the
+// tensor-core kernels do not cover; the merge, backward prologue and epilogue
+// are memory-bound and serve both paths.
+//
+// Notation (paper note "Reformer"): x is the shared query-key ("Shared
+// Query-Key Space", Q = K); tau = 1/sqrt(d) ("LSH Attention", output
+// equation); a (b, h, r) segment holds one round's permutation.
+#include <math.h>
+
+#include "common.cuh"
+
+namespace lsh {
+
+// ------------------------------------------------------------------ norms
+// invnorm[row] = 1/|x_row| (fp32, IEEE sqrt and division), 0 for a zero row.
+template <typename T>
+__global__ void invnorm_kernel(const T *__restrict__ x, float *__restrict__ invnorm, long long rows)
+{
+    long long r = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (r >= rows) return;
+    float a[kDim];
+    load_row(x + r * kDim, a);
+    float s = dot64(a, a);
+    invnorm[r] = s > 0.f ? 1.0f / sqrtf(s) : 0.f;
+}
+
+cudaError_t launch_invnorm(const Problem &p, const void *x, float *invnorm, cudaStream_t st)
+{
+    long long rows = p.tokens();
+    unsigned grid = (unsigned)((rows + 127) / 128);
+    if (p.dtype == LSH_F32)
+        invnorm_kernel<float><<<grid, 128, 0, st>>>((const float *)x, invnorm, rows);
+    else
+        invnorm_kernel<__nv_bfloat16><<<grid, 128, 0, st>>>((const __nv_bfloat16 *)x, invnorm, rows);
+    return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------ hash
+// "LSH Attention", hash equation: bucket = argmax over [x R_r ; -x R_r].
+// One thread per (row, round); projections in fp32, sequential fma over d.
+// Exact ties keep the lowest index: +x R_r entries come before -x R_r ones.
+template <typename T>
+__global__ void hash_simt_kernel(const T *__restrict__ x, const T *__restrict__ R, uint16_t *__restrict__ buckets,
+                                 long long BH, int L, int n_hashes, int half)
+{
+    long long row = (long long)blockIdx.x * blockDim.x + threadIdx.x;   // (bh, i)
+    int r = blockIdx.y;
+    if (row >= BH * L) return;
+    float a[kDim];
+    load_row(x + row * kDim, a);
+    const T *Rr = R + (long long)r * kDim * half;
+    float best_p = -INFINITY, best_n = -INFINITY;
+    int idx_p = 0, idx_n = 0;
+    for (int k = 0; k < half; ++k) {
+        float s = 0.f;
+#pragma unroll 16
+        for (int t = 0; t < kDim; ++t) s = fmaf(a[t], to_f(Rr[(long long)t * half + k]), s);
+        if (s > best_p) { best_p = s; idx_p = k; }
+        if (-s > best_n) { best_n = -s; idx_n = k; }
+    }
+    int bucket = best_p >= best_n ? idx_p : half + idx_n;
+    long long bh = row / L;
+    int i = (int)(row % L);
+    buckets[(bh * n_hashes + r) * L + i] = (uint16_t)bucket;
+}
+
+cudaError_t launch_hash_simt(const Problem &p, const void *x, const void *R, uint16_t *buckets, cudaStream_t st)
+{
+    long long rows = p.tokens();
+    dim3 grid((unsigned)((rows + 127) / 128), p.R);
+    if (p.dtype == LSH_F32)
+        hash_simt_kernel<float><<<grid, 128, 0, st>>>((const float *)x, (const float *)R, buckets, p.BH(), p.L,
+                                                      p.R, p.nb / 2);
+    else
+        hash_simt_kernel<__nv_bfloat16><<<grid, 128, 0, st>>>((const __nv_bfloat16 *)x, (const __nv_bfloat16 *)R,
+                                                              buckets, p.BH(), p.L, p.R, p.nb / 2);
+    return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------ candidates
+// Window of sorted slot s: chunks c-1 and c ("Sorting and Chunking").  A slot
+// t != s is a candidate unless causal and its position exceeds the query's
+// ("Implementation Reading": the mask uses original positions).
+struct Window {
+    int w0, w1;
+};
+__device__ __forceinline__ Window window_of(int s, int m, int L)
+{
+    int c = s / m;
+    Window w;
+    w.w0 = c > 0 ? (c - 1) * m : 0;
+    w.w1 = min((c + 1) * m, L);
+    return w;
+}
+
+// ------------------------------------------------------------------ forward
+// One thread per (segment, sorted slot): full softmax over the window, output
+// and logsumexp written at the query's original position.
+template <typename T>
+__global__ void attn_fwd_simt_kernel(const T *__restrict__ x, const T *__restrict__ v,
+                                     const int32_t *__restrict__ perm, const float *__restrict__ invnorm,
+                                     float *__restrict__ o_r, float *__restrict__ lse, int L, int R, int m,
+                                     int causal, float tau)
+{
+    const long long seg = blockIdx.y;
+    const int s = blockIdx.x * blockDim.x + threadIdx.x;
+    if (s >= L) return;
+    const long long bh = seg / R;
+    const int32_t *P = perm + seg * L;
+    const T *X = x + bh * L * kDim;
+    const T *V = v + bh * L * kDim;
+    const float *IN = invnorm + bh * L;
+    const int i = P[s];
+    float q[kDim], kv[kDim];
+    load_row(X + (long long)i * kDim, q);
+    const Window w = window_of(s, m, L);
+    float mx = -INFINITY;
+    int cnt = 0;
+    for (int t = w.w0; t < w.w1; ++t) {
+        if (t == s) continue;
+        int j = P[t];
+        if (causal && j > i) continue;
+        load_row(X + (long long)j * kDim, kv);
+        float z = tau * (dot64(q, kv) * IN[j]);
+        mx = fmaxf(mx, z);
+        ++cnt;
+    }
+    float acc[kDim];
+    float lse_i;
+    if (cnt == 0) {                       // self is the only candidate
+        lse_i = tau * (dot64(q, q) * IN[i]);
+        load_row(V + (long long)i * kDim, acc);
+    } else {
+#pragma unroll
+        for (int k = 0; k < kDim; ++k) acc[k] = 0.f;
+        float l = 0.f;
+        for (int t = w.w0; t < w.w1; ++t) {
+            if (t == s) continue;
+            int j = P[t];
+            if (causal && j > i) continue;
+            load_row(X + (long long)j * kDim, kv);
+            float e = expf(tau * (dot64(q, kv) * IN[j]) - mx);
+            l += e;
+            load_row(V + (long long)j * kDim, kv);
+#pragma unroll
+            for (int k = 0; k < kDim; ++k) acc[k] = fmaf(e, kv[k], acc[k]);
+        }
+        float inv = 1.0f / l;
+#pragma unroll
+        for (int k = 0; k < kDim; ++k) acc[k] *= inv;
+        lse_i = mx + logf(l);
+    }
+    store_row(o_r + (seg * L + i) * kDim, acc);
+    lse[seg * L + i] = lse_i;
+}
+
+cudaError_t launch_attn_fwd_simt(const Problem &p, const void *x, const void *v, const int32_t *perm,
+                                 const float *invnorm, float *o_r, float *lse, cudaStream_t st)
+{
+    dim3 grid((p.L + 127) / 128, (unsigned)p.S());
+    float tau = 1.0f / sqrtf((float)p.d);
+    if (p.dtype == LSH_F32)
+        attn_fwd_simt_kernel<float><<<grid, 128, 0, st>>>((const float *)x, (const float *)v, perm, invnorm, o_r, lse,
+                                                          p.L, p.R, p.m, p.causal, tau);
+    else
+        attn_fwd_simt_kernel<__nv_bfloat16><<<grid, 128, 0, st>>>((const __nv_bfloat16 *)x,
+                                                                  (const __nv_bfloat16 *)v, perm, invnorm, o_r,
+                                                                  lse, p.L, p.R, p.m, p.causal, tau);
+    return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------ merge
+// "Multiple Hash Rounds": y_i = sum_r softmax_r(lse_r,i) o_r,i.
+// 16 threads per token, four features each.
+template <typename T, typename OT>
+__global__ void combine_kernel(const OT *__restrict__ o_r, const float *__restrict__ lse, T *__restrict__ out,
+                               long long tokens, int L, int R)
+{
+    long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    long long tok = gid >> 4;
+    int quad = (int)(gid & 15);
+    if (tok >= tokens) return;
+    long long bh = tok / L;
+    int i = (int)(tok % L);
+    float mx = -INFINITY;
+    for (int r = 0; r < R; ++r) mx = fmaxf(mx, lse[(bh * R + r) * L + i]);
+    float ssum = 0.f;
+    for (int r = 0; r < R; ++r) ssum += expf(lse[(bh * R + r) * L + i] - mx);
+    float big = mx + logf(ssum);
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int r = 0; r < R; ++r) {
+        float wr = expf(lse[(bh * R + r) * L + i] - big);
+        const OT *o = o_r + ((bh * R + r) * L + i) * kDim + quad * 4;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) acc[k] = fmaf(wr, to_f(o[k]), acc[k]);
+    }
+    T *y = out + tok * kDim + quad * 4;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) y[k] = from_f<T>(acc[k]);
+}
+
+cudaError_t launch_combine(const Problem &p, const void *o_r, bool o_r_bf16, const float *lse, void *out,
+                           cudaStream_t st)
+{
+    long long threads = p.tokens() * 16;
+    unsigned grid = (unsigned)((threads + 255) / 256);
+    if (p.dtype == LSH_F32) {
+        if (o_r_bf16) return cudaErrorInvalidValue;
+        combine_kernel<float, float><<<grid, 256, 0, st>>>((const float *)o_r, lse, (float *)out, p.tokens(), p.L,
+                                                           p.R);
+    } else if (o_r_bf16) {
+        combine_kernel<__nv_bfloat16, __nv_bfloat16><<<grid, 256, 0, st>>>(
+            (const __nv_bfloat16 *)o_r, lse, (__nv_bfloat16 *)out, p.tokens(), p.L, p.R);
+    } else {
+        combine_kernel<__nv_bfloat16, float><<<grid, 256, 0, st>>>((const float *)o_r, lse, (__nv_bfloat16 *)out,
+                                                                   p.tokens(), p.L, p.R);
+    }
+    return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------ backward prologue
+// LSE_i = logsumexp over rounds of lse_r,i and delta_i = dY_i . Y_i; also
+// zeroes the fp32 gradient accumulators.  16 threads per token.
+//
+// With P_rij = exp(z_rij - LSE_i) the merged output is y_i = sum_r,j P_rij v_j,
+// so the backward of every round uses P_rij and dz_rij = P_rij (dY_i.v_j - delta_i).
+template <typename T>
+__global__ void bwd_prep_kernel(const float *__restrict__ lse, const T *__restrict__ out, const T *__restrict__ dout,
+                                float *__restrict__ lse_all, float *__restrict__ delta, float *__restrict__ dx_acc,
+                                float *__restrict__ dv_acc, long long tokens, int L, int R)
+{
+    long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    long long tok = gid >> 4;
+    int quad = (int)(gid & 15);
+    bool valid = tok < tokens;
+    float part = 0.f;
+    if (valid) {
+        const T *y = out + tok * kDim + quad * 4;
+        const T *g = dout + tok * kDim + quad * 4;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) part = fmaf(to_f(g[k]), to_f(y[k]), part);
+        float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+        reinterpret_cast<float4 *>(dx_acc + tok * kDim)[quad] = z;
+        reinterpret_cast<float4 *>(dv_acc + tok * kDim)[quad] = z;
+    }
+#pragma unroll
+    for (int o = 8; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+    if (valid && quad == 0) {
+        long long bh = tok / L;
+        int i = (int)(tok % L);
+        float mx = -INFINITY;
+        for (int r = 0; r < R; ++r) mx = fmaxf(mx, lse[(bh * R + r) * L + i]);
+        float ssum = 0.f;
+        for (int r = 0; r < R; ++r) ssum += expf(lse[(bh * R + r) * L + i] - mx);
+        lse_all[tok] = mx + logf(ssum);
+        delta[tok] = part;
+    }
+}
+
+cudaError_t launch_bwd_prep(const Problem &p, const float *lse, const void *out, const void *dout,
+                            float *lse_all, float *delta, float *dx_acc, float *dv_acc, cudaStream_t st)
+{
+    long long threads = p.tokens() * 16;
+    unsigned grid = (unsigned)((threads + 255) / 256);
+    if (p.dtype == LSH_F32)
+        bwd_prep_kernel<float><<<grid, 256, 0, st>>>(lse, (const float *)out, (const float *)dout, lse_all, delta,
+                                                     dx_acc, dv_acc, p.tokens(), p.L, p.R);
+    else
+        bwd_prep_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(lse, (const __nv_bfloat16 *)out,
+                                                             (const __nv_bfloat16 *)dout, lse_all, delta, dx_acc,
+                                                             dv_acc, p.tokens(), p.L, p.R);
+    return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------ backward, query role
+// One thread per (segment, sorted slot s) with query position i:
+//   dx_i += sum_j dz_ij tau k_j,   k_j = x_j invnorm_j.
+// Also records whether the slot attends to itself alone (needed by the key pass).
+template <typename T>
+__global__ void attn_bwd_q_simt_kernel(const T *__restrict__ x, const T *__restrict__ v, const T *__restrict__ dout,
+                                       const int32_t *__restrict__ perm, const float *__restrict__ invnorm,
+                                       const float *__restrict__ lse_all, const float *__restrict__ delta,
+                                       uint8_t *__restrict__ self_only, float *__restrict__ dx_acc, int L, int R,
+                                       int m, int causal, float tau)
+{
+    const long long seg = blockIdx.y;
+    const int s = blockIdx.x * blockDim.x + threadIdx.x;
+    if (s >= L) return;
+    const long long bh = seg / R;
+    const int32_t *P = perm + seg * L;
+    const T *X = x + bh * L * kDim;
+    const T *V = v + bh * L * kDim;
+    const float *IN = invnorm + bh * L;
+    const int i = P[s];
+    float q[kDim], g[kDim], kv[kDim], dq[kDim];
+    load_row(X + (long long)i * kDim, q);
+    load_row(dout + (bh * L + i) * kDim, g);
+#pragma unroll
+    for (int k = 0; k < kDim; ++k) dq[k] = 0.f;
+    const float big = lse_all[bh * L + i], dl = delta[bh * L + i];
+    const Window w = window_of(s, m, L);
+    int cnt = 0;
+    for (int t = w.w0; t < w.w1; ++t) {
+        if (t == s) continue;
+        int j = P[t];
+        if (causal && j > i) continue;
+        ++cnt;
+        load_row(X + (long long)j * kDim, kv);
+        float pij = expf(tau * (dot64(q, kv) * IN[j]) - big);
+        float c = tau * IN[j];
+        float kvv[kDim];
+        load_row(V + (long long)j * kDim, kvv);
+        float dz = pij * (dot64(g, kvv) - dl);
+#pragma unroll
+        for (int k = 0; k < kDim; ++k) dq[k] = fmaf(dz * c, kv[k], dq[k]);
+    }
+    if (cnt == 0) {
+        float pij = expf(tau * (dot64(q, q) * IN[i]) - big);
+        load_row(V + (long long)i * kDim, kv);
+        float dz = pij * (dot64(g, kv) - dl);
+        float c = tau * IN[i];
+#pragma unroll
+        for (int k = 0; k < kDim; ++k) dq[k] = dz * c * q[k];
+    }
+    self_only[seg * L + s] = cnt == 0;
+    float *dst = dx_acc + (bh * L + i) * kDim;
+#pragma unroll
+    for (int k = 0; k < kDim; ++k) atomicAdd(dst + k, dq[k]);
+}
+
+// ------------------------------------------------------------------ backward, key role
+// One thread per (segment, sorted slot t) with key position j.  The queries
+// whose window holds t sit in chunks c(t) and c(t)+1:
+//   g_j  = sum_s dz_sj tau x_s          (gradient w.r.t. the unit key k_j)
+//   dx_j += invnorm_j (g_j - k_j (k_j . g_j)),   dv_j += sum_s P_sj dY_s.
+template <typename T>
+__global__ void attn_bwd_k_simt_kernel(const T *__restrict__ x, const T *__restrict__ v, const T *__restrict__ dout,
+                                       const int32_t *__restrict__ perm, const float *__restrict__ invnorm,
+                                       const float *__restrict__ lse_all, const float *__restrict__ delta,
+                                       const uint8_t *__restrict__ self_only, float *__restrict__ dx_acc,
+                                       float *__restrict__ dv_acc, int L, int R, int m, int causal, float tau)
+{
+    const long long seg = blockIdx.y;
+    const int t = blockIdx.x * blockDim.x + threadIdx.x;
+    if (t >= L) return;
+    const long long bh = seg / R;
+    const int32_t *P = perm + seg * L;
+    const T *X = x + bh * L * kDim;
+    const float *IN = invnorm + bh * L;
+    const int j = P[t];
+    float kx[kDim], vj[kDim], gk[kDim], dvj[kDim], q[kDim], g[kDim];
+    load_row(X + (long long)j * kDim, kx);
+    load_row(v + (bh * L + j) * kDim, vj);
+#pragma unroll
+    for (int k = 0; k < kDim; ++k) { gk[k] = 0.f; dvj[k] = 0.f; }
+    const float inj = IN[j];
+    const int c = t / m;
+    const int s0 = c * m, s1 = min((c + 2) * m, L);
+    for (int s = s0; s < s1; ++s) {
+        int i = P[s];
+        bool cand;
+        if (s == t) cand = self_only[seg * L + s] != 0;
+        else cand = !(causal && j > i);
+        if (!cand) continue;
+        load_row(X + (long long)i * kDim, q);
+        load_row(dout + (bh * L + i) * kDim, g);
+        float pij = expf(tau * (dot64(q, kx) * inj) - lse_all[bh * L + i]);
+        float dz = pij * (dot64(g, vj) - delta[bh * L + i]);
+#pragma unroll
+        for (int k = 0; k < kDim; ++k) {
+            gk[k] = fmaf(dz * tau, q[k], gk[k]);
+            dvj[k] = fmaf(pij, g[k], dvj[k]);
+        }
+    }
+    // through k_j = x_j / |x_j|: dx_j = invnorm_j (g - k (k . g)), k = x_j invnorm_j
+    float kg = 0.f;
+#pragma unroll
+    for (int k = 0; k < kDim; ++k) kg = fmaf(kx[k] * inj, gk[k], kg);
+    float *dxd = dx_acc + (bh * L + j) * kDim;
+    float *dvd = dv_acc + (bh * L + j) * kDim;
+#pragma unroll
+    for (int k = 0; k < kDim; ++k) {
+        atomicAdd(dxd + k, inj * (gk[k] - kx[k] * inj * kg));
+        atomicAdd(dvd + k, dvj[k]);
+    }
+}
+
+cudaError_t launch_attn_bwd_simt(const Problem &p, const void *x, const void *v, const void *dout,
+                                 const int32_t *perm, const float *invnorm, const float *lse_all,
+                                 const float *delta, uint8_t *self_only, float *dx_acc, float *dv_acc,
+                                 cudaStream_t st)
+{
+    dim3 grid((p.L + 127) / 128, (unsigned)p.S());
+    float tau = 1.0f / sqrtf((float)p.d);
+    if (p.dtype == LSH_F32) {
+        attn_bwd_q_simt_kernel<float><<<grid, 128, 0, st>>>((const float *)x, (const float *)v, (const float *)dout,
+                                                            perm, invnorm, lse_all, delta, self_only, dx_acc, p.L,
+                                                            p.R, p.m, p.causal, tau);
+        attn_bwd_k_simt_kernel<float><<<grid, 128, 0, st>>>((const float *)x, (const float *)v, (const float *)dout,
+                                                            perm, invnorm, lse_all, delta, self_only, dx_acc,
+                                                            dv_acc, p.L, p.R, p.m, p.causal, tau);
+    } else {
+        using B = __nv_bfloat16;
+        attn_bwd_q_simt_kernel<B><<<grid, 128, 0, st>>>((const B *)x, (const B *)v, (const B *)dout, perm, invnorm,
+                                                        lse_all, delta, self_only, dx_acc, p.L, p.R, p.m, p.causal,
+                                                        tau);
+        attn_bwd_k_simt_kernel<B><<<grid, 128, 0, st>>>((const B *)x, (const B *)v, (const B *)dout, perm, invnorm,
+                                                        lse_all, delta, self_only, dx_acc, dv_acc, p.L, p.R, p.m,
+                                                        p.causal, tau);
+    }
+    return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------ backward epilogue
+template <typename T>
+__global__ void bwd_finalize_kernel(const float *__restrict__ dx_acc, const float *__restrict__ dv_acc,
+                                    T *__restrict__ dqk, T *__restrict__ dv, long long n4)
+{
+    long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= n4) return;
+    float4 a = reinterpret_cast<const float4 *>(dx_acc)[i];
+    float4 b = reinterpret_cast<const float4 *>(dv_acc)[i];
+    T *o1 = dqk + 4 * i;
+    T *o2 = dv + 4 * i;
+    o1[0] = from_f<T>(a.x); o1[1] = from_f<T>(a.y); o1[2] = from_f<T>(a.z); o1[3] = from_f<T>(a.w);
+    o2[0] = from_f<T>(b.x); o2[1] = from_f<T>(b.y); o2[2] = from_f<T>(b.z); o2[3] = from_f<T>(b.w);
+}
+
+cudaError_t launch_bwd_finalize(const Problem &p, const float *dx_acc, const float *dv_acc, void *dqk, void *dv,
+                                cudaStream_t st)
+{
+    long long n4 = p.tokens() * kDim / 4;
+    unsigned grid = (unsigned)((n4 + 255) / 256);
+    if (p.dtype == LSH_F32)
+        bwd_finalize_kernel<float><<<grid, 256, 0, st>>>(dx_acc, dv_acc, (float *)dqk, (float *)dv, n4);
+    else
+        bwd_finalize_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(dx_acc, dv_acc, (__nv_bfloat16 *)dqk,
+                                                                 (__nv_bfloat16 *)dv, n4);
+    return cudaGetLastError();
+}
+
+}  // namespace lsh

@@ -1,0 +1,107 @@
+"""Host-side checks of the C ABI: the library loads, exports every entry point
+the header declares, and rejects bad arguments before touching the GPU."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from lsh_attention_02_b200 import build as lib_build
+import lsh_attention_02_b200 as lsh
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "lsh_attn.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    lib_build.build()
+    return lsh.load_library()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"LSH_API\s+[\w\s\*]+?\b(lsh_attn_\w+)\s*\(", text)))
+
+
+def test_header_declares_entry_points():
+    names = declared_functions()
+    for n in ["lsh_attn_fwd", "lsh_attn_bwd", "lsh_attn_workspace_size", "lsh_attn_hash", "lsh_attn_sort",
+              "lsh_attn_fwd_sorted", "lsh_attn_status_str"]:
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+    assert set(declared_functions()) <= set(lsh.EXPORTED)
+
+
+def test_abi_version(lib):
+    text = open(HEADER).read()
+    v = int(re.search(r"#define LSH_ATTN_ABI_VERSION (\d+)", text).group(1))
+    assert lib.lsh_attn_abi_version() == v
+
+
+def test_status_strings(lib):
+    for code in lsh.STATUS:
+        s = lib.lsh_attn_status_str(code)
+        assert s and isinstance(s, bytes)
+    assert lib.lsh_attn_status_str(42) == b"unknown status"
+
+
+def _desc(**kw):
+    base = dict(B=1, H=2, L=1024, d=64, n_buckets=16, n_hashes=2, chunk=64, causal=0, dtype=lsh.LSH_BF16,
+                impl=lsh.IMPL_AUTO)
+    base.update(kw)
+    return lsh.Desc(*[base[k] for k in ("B", "H", "L", "d", "n_buckets", "n_hashes", "chunk", "causal", "dtype",
+                                        "impl")])
+
+
+@pytest.mark.parametrize("kw,want", [
+    (dict(d=32), -4), (dict(L=1000), -2), (dict(n_buckets=15), -2), (dict(n_buckets=0), -2),
+    (dict(n_hashes=0), -2), (dict(chunk=0), -2), (dict(dtype=7), -1), (dict(impl=9), -1), (dict(causal=2), -1),
+    (dict(B=0), -2), (dict(n_buckets=131072), -2),
+])
+def test_invalid_descriptors_rejected(lib, kw, want):
+    d = _desc(**kw)
+    assert lib.lsh_attn_workspace_size(ctypes.byref(d), 0) == 0
+    fake = ctypes.c_void_p(1 << 20)
+    rc = lib.lsh_attn_fwd(ctypes.byref(d), fake, fake, fake, fake, fake, None, fake, 1 << 40, None)
+    assert rc == want
+
+
+def test_null_and_misaligned_pointers(lib):
+    d = _desc()
+    ws_n = lib.lsh_attn_workspace_size(ctypes.byref(d), 0)
+    assert ws_n > 0
+    ok = ctypes.c_void_p(1 << 20)
+    bad = ctypes.c_void_p((1 << 20) + 8)
+    assert lib.lsh_attn_fwd(ctypes.byref(d), None, ok, ok, ok, ok, None, ok, ws_n, None) == -1
+    assert lib.lsh_attn_fwd(ctypes.byref(d), bad, ok, ok, ok, ok, None, ok, ws_n, None) == -3
+    # workspace: null, misaligned (needs 256 B) and too small
+    assert lib.lsh_attn_fwd(ctypes.byref(d), ok, ok, ok, ok, ok, None, None, ws_n, None) == -1
+    assert lib.lsh_attn_fwd(ctypes.byref(d), ok, ok, ok, ok, ok, None, ctypes.c_void_p((1 << 20) + 16), ws_n,
+                            None) == -3
+    assert lib.lsh_attn_fwd(ctypes.byref(d), ok, ok, ok, ok, ok, None, ok, ws_n - 1, None) == -7
+    # backward needs either perm or rotations
+    wb = lib.lsh_attn_workspace_size(ctypes.byref(d), 1)
+    assert lib.lsh_attn_bwd(ctypes.byref(d), ok, ok, None, ok, ok, None, ok, ok, ok, ok, wb, None) == -1
+    assert lib.lsh_attn_bwd(ctypes.byref(d), ok, ok, ok, ok, ok, None, ok, ok, ok, ok, wb - 1, None) == -7
+
+
+def test_workspace_grows_with_problem(lib):
+    small = lib.lsh_attn_workspace_size(ctypes.byref(_desc()), 1)
+    big = lib.lsh_attn_workspace_size(ctypes.byref(_desc(L=4096)), 1)
+    assert 0 < small < big
+    # forcing the CUDA-core path is always possible; fwd and bwd sizes are both positive
+    for impl in (lsh.IMPL_AUTO, lsh.IMPL_SIMT):
+        for bwd in (0, 1):
+            assert lib.lsh_attn_workspace_size(ctypes.byref(_desc(impl=impl)), bwd) > 0
+
+
+def test_trace_end_without_begin_is_an_error(lib):
+    n = len(lsh.STAGES)
+    ms = (ctypes.c_float * n)(); c = (ctypes.c_int32 * n)(); k = (ctypes.c_int32 * n)()
+    assert lib.lsh_attn_trace_end(ms, c, k, n) == -1
+    assert lib.lsh_attn_trace_begin(0) == -1

@@ -1,0 +1,223 @@
+"""GPU parity: the CUDA library through its C ABI against the CPU oracle on the
+same seeded inputs.
+
+Bucket ids and permutations are compared bit for bit (an argmax flip is
+allowed only where the oracle's top-two gap is below 1e-6 relative, and is
+counted and printed).  To keep a flip from spreading, attention outputs and
+gradients are compared with the GPU's own permutation injected into the
+oracle.  Floating-point bounds: fp32 1e-4 max-abs; bf16 2e-2 max-abs and
+1e-2 relative L2.
+"""
+import numpy as np
+import pytest
+import torch
+
+import lsh_attention_02_b200 as lsh
+from lsh_attention_02_b200 import synth
+from oracle import oracle
+from tests.gpu_util import (NEAR_TIE, Run, assert_close, check_buckets, check_perm_is_stable_sort, errors,
+                            to_dev, to_host)
+
+pytestmark = pytest.mark.gpu
+
+IMPLS = [lsh.IMPL_SIMT, lsh.IMPL_AUTO]
+
+
+def small(name, **kw):
+    return synth.WORKLOADS[name].replace(**kw)
+
+
+def _flip_report(tag, flips, total):
+    print(f"[near-tie] {tag}: {flips} argmax flips out of {total} row-rounds")
+
+
+def full_check(w: synth.Workload, impl=lsh.IMPL_AUTO, heads=None):
+    """Runs fwd (+bwd) on the GPU for workload w and checks (b, h) slices `heads`
+    (all when None) against the oracle."""
+    inp = synth.make_inputs(w)
+    run = Run(inp, w.n_buckets, w.chunk, w.causal, w.dtype, impl)
+    B, H, L = w.B, w.H, w.L
+    sel = [(b, h) for b in range(B) for h in range(H)] if heads is None else heads
+    gb = run.host_buckets()
+    gperm = run.perm.cpu().numpy()
+    out, lse = to_host(run.out), run.lse.cpu().numpy().astype(np.float64)
+    check_perm_is_stable_sort(gperm, gb, f"{w.name} perm")
+    flips = 0
+    for b, h in sel:
+        xs, vs = inp["x"][b:b + 1, h:h + 1], inp["v"][b:b + 1, h:h + 1]
+        ref = oracle.fwd(xs, vs, inp["R"], w.n_buckets, w.chunk, w.causal)
+        flips += check_buckets(gb[b, h], ref["bucket"][0, 0], ref["margin"][0, 0], f"{w.name} ({b},{h})")
+        if flips == 0:
+            np.testing.assert_array_equal(gperm[b, h], ref["perm"][0, 0])
+        y, lr = oracle.fwd_perm(xs, vs, gperm[b:b + 1, h:h + 1], w.chunk, w.causal)
+        assert_close(out[b, h], y[0, 0], w.dtype, f"{w.name} ({b},{h}) out")
+        assert_close(lse[b, h], lr[0, 0], "f32" if w.dtype == "f32" else "bf16", f"{w.name} ({b},{h}) lse")
+        if w.backward:
+            dx, dv = oracle.bwd(xs, vs, inp["dy"][b:b + 1, h:h + 1], gperm[b:b + 1, h:h + 1], w.chunk, w.causal)
+            assert_close(to_host(run.dx[b, h]), dx[0, 0], w.dtype, f"{w.name} ({b},{h}) dqk")
+            assert_close(to_host(run.dv[b, h]), dv[0, 0], w.dtype, f"{w.name} ({b},{h}) dv")
+    _flip_report(w.name, flips, len(sel) * w.n_hashes * L)
+    return run
+
+
+# ------------------------------------------------------------------ stage: hash
+@pytest.mark.parametrize("impl", IMPLS)
+@pytest.mark.parametrize("dtype,nb,nh", [("f32", 16, 1), ("bf16", 64, 2), ("bf16", 1024, 3), ("bf16", 192, 2),
+                                         ("bf16", 2, 2), ("f32", 8192, 1)])
+def test_hash_bit_exact_up_to_near_ties(impl, dtype, nb, nh):
+    w = small("bf16_causal_4k", B=2, H=2, L=1024 if nb < 8192 else 256, n_buckets=nb, n_hashes=nh, dtype=dtype)
+    inp = synth.make_inputs(w)
+    x = to_dev(inp["x"], dtype); R = to_dev(inp["R"], dtype)
+    desc = lsh.desc_for(x, nb, nh, 64, True, impl)
+    bk = torch.empty((2, 2, nh, w.L), dtype=torch.int16, device="cuda")
+    lsh.lsh_attn_hash(desc, x, R, bk)
+    gb = bk.cpu().numpy().view(np.uint16).astype(np.int64)
+    flips = 0
+    for b in range(2):
+        for h in range(2):
+            for r in range(nh):
+                ob, mg = oracle.hash_round(inp["x"][b, h], inp["R"][r], nb)
+                flips += check_buckets(gb[b, h, r], ob, mg, f"hash nb={nb} ({b},{h},{r})")
+    _flip_report(f"hash {dtype} nb={nb}", flips, 4 * nh * w.L)
+
+
+# ------------------------------------------------------------------ stage: sort
+@pytest.mark.parametrize("L,nb,dist", [(1, 2, "uniform"), (64, 2, "uniform"), (2048, 16, "uniform"),
+                                       (2112, 1024, "uniform"), (12288, 192, "skewed"), (4096, 65536, "uniform"),
+                                       (65536, 1024, "one_bucket"), (10240, 8192, "skewed"),
+                                       (4160, 256, "descending")])
+def test_sort_bit_exact(L, nb, dist):
+    rng = np.random.default_rng(L + nb)
+    S = 3
+    if dist == "uniform":
+        b = rng.integers(0, nb, size=(S, L))
+    elif dist == "skewed":
+        b = np.minimum((rng.pareto(1.2, size=(S, L)) * 3).astype(np.int64), nb - 1)
+    elif dist == "one_bucket":
+        b = np.full((S, L), nb // 3)
+    else:
+        b = np.tile(np.arange(L)[::-1] % nb, (S, 1))
+    bk = torch.from_numpy(b.astype(np.uint16).view(np.int16).reshape(1, S, 1, L)).cuda()
+    perm = torch.empty((1, S, 1, L), dtype=torch.int32, device="cuda")
+    desc = lsh.make_desc(1, S, L, 64, nb, 1, 1, False, lsh.LSH_BF16)
+    lsh.lsh_attn_sort(desc, bk, perm)
+    got = perm.cpu().numpy().reshape(S, L)
+    for s in range(S):
+        np.testing.assert_array_equal(got[s], oracle.sort_segment(b[s]))
+
+
+# ------------------------------------------------------------------ stage: attention with a given permutation
+@pytest.mark.parametrize("impl", IMPLS)
+@pytest.mark.parametrize("dtype,causal,L,m,nh", [("f32", False, 1024, 64, 1), ("f32", True, 512, 32, 3),
+                                                 ("bf16", True, 1024, 64, 2), ("bf16", False, 2048, 64, 4),
+                                                 ("bf16", True, 960, 64, 2), ("f32", True, 48, 1, 2),
+                                                 ("bf16", True, 64, 64, 1), ("bf16", False, 128, 128, 2)])
+def test_attention_given_perm(impl, dtype, causal, L, m, nh):
+    w = small("bf16_causal_4k", B=1, H=3, L=L, n_buckets=16, n_hashes=nh, chunk=m, causal=causal, dtype=dtype)
+    inp = synth.make_inputs(w)
+    rng = np.random.default_rng(L + nh)
+    perm = np.stack([[rng.permutation(L) for _ in range(nh)] for _ in range(3)])[None].astype(np.int32)
+    x, v = to_dev(inp["x"], dtype), to_dev(inp["v"], dtype)
+    desc = lsh.desc_for(x, 16, nh, m, causal, impl)
+    out, lse, _ = lsh.outputs_like(desc, x)
+    lsh.lsh_attn_fwd_sorted(desc, x, v, torch.from_numpy(perm).cuda(), out, lse)
+    y, lr = oracle.fwd_perm(inp["x"], inp["v"], perm, m, causal)
+    assert_close(to_host(out), y, dtype, "out")
+    assert_close(lse.cpu().numpy(), lr, "f32" if dtype == "f32" else "bf16", "lse")
+
+
+# ------------------------------------------------------------------ whole path, small cases
+@pytest.mark.parametrize("impl", IMPLS)
+@pytest.mark.parametrize("dtype,causal,nb,nh,L", [("f32", False, 16, 1, 1024), ("f32", True, 16, 2, 512),
+                                                  ("bf16", True, 64, 2, 1024), ("bf16", False, 128, 3, 1152),
+                                                  ("bf16", True, 1024, 4, 2048), ("bf16", True, 2, 2, 256)])
+def test_forward_backward_small(impl, dtype, causal, nb, nh, L):
+    w = small("long_64k", B=2, H=2, L=L, n_buckets=nb, n_hashes=nh, causal=causal, dtype=dtype, backward=True)
+    full_check(w, impl)
+
+
+@pytest.mark.parametrize("impl", IMPLS)
+def test_clustered_inputs_small(impl):
+    w = small("image_12k", B=1, H=2, L=1536)
+    full_check(w, impl)
+
+
+@pytest.mark.parametrize("impl", IMPLS)
+def test_edge_cases(impl):
+    """Zero rows (key 0), duplicated rows, causal first token = its own value."""
+    w = small("long_64k", B=1, H=2, L=256, n_buckets=8, n_hashes=2, backward=True)
+    inp = synth.make_inputs(w)
+    inp["x"][0, 0, 5] = 0.0
+    inp["x"][0, 1, 10] = inp["x"][0, 1, 11]
+    run = Run(inp, w.n_buckets, w.chunk, True, "bf16", impl)
+    out = to_host(run.out)
+    np.testing.assert_array_equal(out[0, :, 0], inp["v"][0, :, 0])   # causal position 0 sees only itself
+    y, _ = oracle.fwd_perm(inp["x"], inp["v"], run.perm.cpu().numpy(), w.chunk, True)
+    assert_close(out, y, "bf16", "out")
+    dx, dv = oracle.bwd(inp["x"], inp["v"], inp["dy"], run.perm.cpu().numpy(), w.chunk, True)
+    assert_close(to_host(run.dx), dx, "bf16", "dqk")
+    assert_close(to_host(run.dv), dv, "bf16", "dv")
+
+
+def test_paths_agree():
+    """The tensor-core and CUDA-core paths give the same buckets and permutation
+    (when no near tie separates them) and outputs within the bf16 bound."""
+    w = small("long_64k", B=1, H=2, L=2048, backward=True)
+    inp = synth.make_inputs(w)
+    a = Run(inp, w.n_buckets, w.chunk, True, "bf16", lsh.IMPL_SIMT)
+    b = Run(inp, w.n_buckets, w.chunk, True, "bf16", lsh.IMPL_AUTO)
+    diff = (a.host_buckets() != b.host_buckets()).sum()
+    assert diff <= 4
+    if diff == 0:
+        assert torch.equal(a.perm, b.perm)
+        assert_close(to_host(b.out), to_host(a.out), "bf16", "out")
+
+
+# ------------------------------------------------------------------ the five workloads
+def test_workload_tiny_f32():
+    full_check(synth.WORKLOADS["tiny_f32"])
+
+
+def test_workload_bf16_causal_4k():
+    full_check(synth.WORKLOADS["bf16_causal_4k"], heads=[(0, 0), (3, 5), (7, 7)])
+
+
+def test_workload_long_64k_one_head():
+    full_check(synth.WORKLOADS["long_64k"], heads=[(0, 3)])
+
+
+def test_workload_image_12k_two_heads():
+    full_check(synth.WORKLOADS["image_12k"], heads=[(0, 0), (5, 6)])
+
+
+def test_workload_half_million_sampled():
+    """L = 524288: every permutation is checked against numpy's stable argsort
+    of the GPU buckets; bucket ids and outputs on sampled rows and slots."""
+    w = synth.WORKLOADS["half_million"]
+    inp = synth.make_inputs(w)
+    run = Run(inp, w.n_buckets, w.chunk, w.causal, w.dtype)
+    gb = run.host_buckets()
+    gperm = run.perm.cpu().numpy()
+    check_perm_is_stable_sort(gperm, gb, "half_million perm")
+    rng = np.random.default_rng(5)
+    out = to_host(run.out)
+    lse = run.lse.cpu().numpy().astype(np.float64)
+    flips = 0
+    for h in range(w.H):
+        rows = np.sort(rng.choice(w.L, size=1024, replace=False))
+        for r in range(w.n_hashes):
+            ob, mg = oracle.hash_round(inp["x"][0, h, rows], inp["R"][r], w.n_buckets)
+            flips += check_buckets(gb[0, h, r, rows], ob, mg, f"half_million h={h} r={r}")
+        # merged output at sampled positions: every round's slot of that position
+        pos = rows[:256]
+        o_r, l_r = [], []
+        for r in range(w.n_hashes):
+            inv = np.empty(w.L, np.int64); inv[gperm[0, h, r]] = np.arange(w.L)
+            o, l = oracle.attn_slots(inp["x"][0, h], inp["v"][0, h], gperm[0, h, r], w.chunk, w.causal, inv[pos])
+            o_r.append(o); l_r.append(l)
+            assert_close(lse[0, h, r, pos], l, "bf16", f"half_million lse h={h} r={r}")
+        o_r, l_r = np.stack(o_r), np.stack(l_r)
+        wts = np.exp(l_r - l_r.max(0)); wts /= wts.sum(0)
+        y = (wts[:, :, None] * o_r).sum(0)
+        assert_close(out[0, h, pos], y, "bf16", f"half_million out h={h}")
+    _flip_report("half_million sampled", flips, w.H * w.n_hashes * 1024)
