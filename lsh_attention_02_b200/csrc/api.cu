@@ -56,7 +56,7 @@ static cudaError_t staged(int stage, int n_kernels, cudaStream_t st, F fn)
     return cudaSuccess;
 }
 
-Workspace plan_workspace(const Problem &p, bool backward, bool tc_attn, char *base)
+Workspace plan_workspace(const Problem &p, bool backward, bool tc_attn, bool tc_hash, char *base)
 {
     Workspace w{};
     size_t off = 0;
@@ -68,6 +68,7 @@ Workspace plan_workspace(const Problem &p, bool backward, bool tc_attn, char *ba
     const size_t S = (size_t)p.S(), L = (size_t)p.L, T = (size_t)p.tokens();
     const SortPlan sp = make_sort_plan(p.nb, p.L);
     w.status = (uint32_t *)take(256);
+    w.rot = take(tc_hash ? hash_tc_scratch_bytes(p) : 0);
     w.invnorm = (float *)take(T * sizeof(float));
     w.buckets = (uint16_t *)take(S * L * sizeof(uint16_t));
     w.sort_keys = (uint16_t *)take(sp.passes > 1 ? S * L * sizeof(uint16_t) : 0);
@@ -145,8 +146,8 @@ static lsh_status check_ws(void *ws, size_t ws_bytes, size_t need)
 static lsh_status run_hash_sort(const Problem &p, const Choice &c, const void *qk, const void *R, int32_t *perm,
                                 const Workspace &w, cudaStream_t st)
 {
-    LSH_TRY(staged(LSH_STAGE_HASH, 1, st, [&] {
-                return c.tc_hash ? launch_hash_tc(p, qk, R, w.buckets, w.status, st)
+    LSH_TRY(staged(LSH_STAGE_HASH, c.tc_hash ? 2 : 1, st, [&] {
+                return c.tc_hash ? launch_hash_tc(p, qk, R, w.buckets, w.rot, w.status, st)
                                  : launch_hash_simt(p, qk, R, w.buckets, st);
             }), "hash");
     LSH_TRY(staged(LSH_STAGE_SORT, 3 * make_sort_plan(p.nb, p.L).passes, st,
@@ -179,7 +180,7 @@ size_t lsh_attn_workspace_size(const lsh_attn_desc *desc, int for_backward)
     Problem p;
     Choice c;
     if (check_desc(desc, &p) != LSH_OK || choose(desc, p, &c) != LSH_OK) return 0;
-    return plan_workspace(p, for_backward != 0, c.tc_attn, nullptr).bytes;
+    return plan_workspace(p, for_backward != 0, c.tc_attn, c.tc_hash, nullptr).bytes;
 }
 
 lsh_status lsh_attn_hash(const lsh_attn_desc *desc, const void *qk, const void *R, uint16_t *buckets,
@@ -192,12 +193,12 @@ lsh_status lsh_attn_hash(const lsh_attn_desc *desc, const void *qk, const void *
     if ((s = choose(desc, p, &c)) != LSH_OK) return s;
     if ((s = check_ptrs({qk, R})) != LSH_OK) return s;
     if (!buckets) return LSH_ERR_ARG;
-    Workspace w = plan_workspace(p, false, c.tc_attn, nullptr);
+    Workspace w = plan_workspace(p, false, c.tc_attn, c.tc_hash, nullptr);
     if ((s = check_ws(workspace, ws_bytes, w.bytes)) != LSH_OK) return s;
-    w = plan_workspace(p, false, c.tc_attn, (char *)workspace);
+    w = plan_workspace(p, false, c.tc_attn, c.tc_hash, (char *)workspace);
     cudaStream_t st = (cudaStream_t)stream;
-    LSH_TRY(staged(LSH_STAGE_HASH, 1, st, [&] {
-                return c.tc_hash ? launch_hash_tc(p, qk, R, buckets, w.status, st)
+    LSH_TRY(staged(LSH_STAGE_HASH, c.tc_hash ? 2 : 1, st, [&] {
+                return c.tc_hash ? launch_hash_tc(p, qk, R, buckets, w.rot, w.status, st)
                                  : launch_hash_simt(p, qk, R, buckets, st);
             }), "hash");
     return LSH_OK;
@@ -212,9 +213,9 @@ lsh_status lsh_attn_sort(const lsh_attn_desc *desc, const uint16_t *buckets, int
     if ((s = check_desc(desc, &p)) != LSH_OK) return s;
     if ((s = choose(desc, p, &c)) != LSH_OK) return s;
     if (!buckets || !perm) return LSH_ERR_ARG;
-    Workspace w = plan_workspace(p, false, c.tc_attn, nullptr);
+    Workspace w = plan_workspace(p, false, c.tc_attn, c.tc_hash, nullptr);
     if ((s = check_ws(workspace, ws_bytes, w.bytes)) != LSH_OK) return s;
-    w = plan_workspace(p, false, c.tc_attn, (char *)workspace);
+    w = plan_workspace(p, false, c.tc_attn, c.tc_hash, (char *)workspace);
     cudaStream_t st = (cudaStream_t)stream;
     LSH_TRY(staged(LSH_STAGE_SORT, 3 * make_sort_plan(p.nb, p.L).passes, st,
                    [&] { return launch_sort(p, buckets, perm, w, st); }), "sort");
@@ -231,9 +232,9 @@ lsh_status lsh_attn_fwd_sorted(const lsh_attn_desc *desc, const void *qk, const 
     if ((s = choose(desc, p, &c)) != LSH_OK) return s;
     if ((s = check_ptrs({qk, v, out, lse})) != LSH_OK) return s;
     if (!perm) return LSH_ERR_ARG;
-    Workspace w = plan_workspace(p, false, c.tc_attn, nullptr);
+    Workspace w = plan_workspace(p, false, c.tc_attn, c.tc_hash, nullptr);
     if ((s = check_ws(workspace, ws_bytes, w.bytes)) != LSH_OK) return s;
-    w = plan_workspace(p, false, c.tc_attn, (char *)workspace);
+    w = plan_workspace(p, false, c.tc_attn, c.tc_hash, (char *)workspace);
     cudaStream_t st = (cudaStream_t)stream;
     LSH_TRY(cudaMemsetAsync(w.status, 0, sizeof(uint32_t), st), "status reset");
     return run_attn_fwd(p, c, qk, v, perm, out, lse, w, st);
@@ -248,9 +249,9 @@ lsh_status lsh_attn_fwd(const lsh_attn_desc *desc, const void *qk, const void *v
     if ((s = check_desc(desc, &p)) != LSH_OK) return s;
     if ((s = choose(desc, p, &c)) != LSH_OK) return s;
     if ((s = check_ptrs({qk, v, R, out, lse})) != LSH_OK) return s;
-    Workspace w = plan_workspace(p, false, c.tc_attn, nullptr);
+    Workspace w = plan_workspace(p, false, c.tc_attn, c.tc_hash, nullptr);
     if ((s = check_ws(workspace, ws_bytes, w.bytes)) != LSH_OK) return s;
-    w = plan_workspace(p, false, c.tc_attn, (char *)workspace);
+    w = plan_workspace(p, false, c.tc_attn, c.tc_hash, (char *)workspace);
     cudaStream_t st = (cudaStream_t)stream;
     int32_t *perm = perm_out ? perm_out : w.perm;
     LSH_TRY(cudaMemsetAsync(w.status, 0, sizeof(uint32_t), st), "status reset");
@@ -269,9 +270,9 @@ lsh_status lsh_attn_bwd(const lsh_attn_desc *desc, const void *qk, const void *v
     if ((s = choose(desc, p, &c)) != LSH_OK) return s;
     if ((s = check_ptrs({qk, v, out, lse, dout, dqk, dv})) != LSH_OK) return s;
     if (!perm && !R) return LSH_ERR_ARG;
-    Workspace w = plan_workspace(p, true, c.tc_attn, nullptr);
+    Workspace w = plan_workspace(p, true, c.tc_attn, c.tc_hash, nullptr);
     if ((s = check_ws(workspace, ws_bytes, w.bytes)) != LSH_OK) return s;
-    w = plan_workspace(p, true, c.tc_attn, (char *)workspace);
+    w = plan_workspace(p, true, c.tc_attn, c.tc_hash, (char *)workspace);
     cudaStream_t st = (cudaStream_t)stream;
     LSH_TRY(cudaMemsetAsync(w.status, 0, sizeof(uint32_t), st), "status reset");
     if (!perm) {

@@ -36,6 +36,7 @@ SortPlan make_sort_plan(int n_buckets, int L);
 // ---------------------------------------------------------------- workspace
 struct Workspace {
     uint32_t *status;                 // device status word (timeouts)
+    void *rot;                        // rotations re-laid out for the tensor-core hash
     float *invnorm;                   // [BH, L]  1/|x| (0 for a zero row)
     uint16_t *buckets;                // [S, L]
     uint16_t *sort_keys;              // [S, L]   first-pass keys
@@ -51,7 +52,7 @@ struct Workspace {
     size_t bytes;
 };
 // Lays the workspace out from `base` (or from 0 when base is null, to size it).
-Workspace plan_workspace(const Problem &p, bool backward, bool tc_attn, char *base);
+Workspace plan_workspace(const Problem &p, bool backward, bool tc_attn, bool tc_hash, char *base);
 
 // ---------------------------------------------------------------- helpers
 __device__ __forceinline__ float to_f(float a) { return a; }
@@ -118,9 +119,10 @@ __device__ __forceinline__ void store_row(__nv_bfloat16 *p, const float *r)
 // Every launcher enqueues on `st` and returns cudaGetLastError().
 cudaError_t launch_invnorm(const Problem &p, const void *x, float *invnorm, cudaStream_t st);
 cudaError_t launch_hash_simt(const Problem &p, const void *x, const void *R, uint16_t *buckets, cudaStream_t st);
-cudaError_t launch_hash_tc(const Problem &p, const void *x, const void *R, uint16_t *buckets,
+cudaError_t launch_hash_tc(const Problem &p, const void *x, const void *R, uint16_t *buckets, void *scratch,
                            uint32_t *status, cudaStream_t st);
 bool hash_tc_supported(const Problem &p);
+size_t hash_tc_scratch_bytes(const Problem &p);
 cudaError_t launch_sort(const Problem &p, const uint16_t *buckets, int32_t *perm, const Workspace &ws,
                         cudaStream_t st);
 cudaError_t launch_attn_fwd_simt(const Problem &p, const void *x, const void *v, const int32_t *perm,

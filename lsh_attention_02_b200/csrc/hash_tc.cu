@@ -1,0 +1,243 @@
+// lsh_hash on the tensor cores: bucket = argmax over [x R_r ; -x R_r]
+// ("LSH Attention", hash equation; angular LSH with Gaussian rotations).
+//
+// For every round the rotation product x R_r is a dense [rows x 64] x
+// [64 x n_buckets/2] GEMM; it runs as tcgen05.mma (bf16 in, fp32 accumulate
+// in tensor memory) and the argmax is the epilogue, so the projections are
+// never written to memory.
+//
+// CTA = 256 rows (two M=128 tiles) x every round.  Warp roles:
+//   warps 0-7  epilogue: warp w reads TMEM lanes 32*(w%4).. of M-tile w/4,
+//              one row per thread, and keeps the running argmax;
+//   warp 8     producer: one bulk copy per (round, N-tile) of the rotation
+//              tile, pre-transposed and pre-swizzled in global memory, into a
+//              4-stage shared-memory ring;
+//   warp 9     MMA issuer: 4 K-steps x 2 M-tiles per N-tile into one of two
+//              TMEM accumulator buffers (double buffering lets the epilogue
+//              of tile t overlap the MMAs of tile t+1).
+//
+// Epilogue per N-tile of NT columns held in registers: pass 1 takes the
+// max and min with 3-input min/max; the larger of max and -min decides the
+// side ([+xR] wins an exact tie, as its indices come first); pass 2 finds the
+// lowest column equal to that extreme.  Tiles merge in index order, so the
+// result is the first maximum of [xR ; -xR], the oracle's tie rule.
+#include "tc_common.cuh"
+
+namespace lsh {
+
+namespace {
+
+constexpr int kRows = 256;          // rows per CTA
+constexpr int kMaxNT = 128;         // widest N-tile
+constexpr int kStages = 4;          // rotation-tile ring
+constexpr int kEpiWarps = 8;
+constexpr int kThreads = (kEpiWarps + 2) * 32;
+constexpr int kTmemCols = 512;      // 2 buffers x 2 M-tiles x kMaxNT
+
+struct HashSmem {
+    uint8_t A[kRows * 128];                 // x rows, K-major SW128   (32 KB)
+    uint8_t B[kStages][kMaxNT * 128];       // rotation tiles           (64 KB)
+    uint64_t full[kStages], empty[kStages];
+    uint64_t acc_full[2], acc_empty[2];
+    uint32_t tmem_base;
+    int abort;
+};
+
+// R [R, 64, half] (k-major per column) -> Rs [R, half, 64] rows of 64 k, with the
+// 16-byte chunks of row n stored at position (chunk ^ (n & 7)): the shared-memory
+// image of a K-major 128-byte-swizzled B operand, so one bulk copy lands a tile.
+__global__ void rot_swizzle_kernel(const __nv_bfloat16 *__restrict__ R, __nv_bfloat16 *__restrict__ Rs, int half,
+                                   int rounds)
+{
+    long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;   // over rounds * half * 64
+    long long total = (long long)rounds * half * kDim;
+    if (idx >= total) return;
+    int k = (int)(idx % kDim);
+    long long rn = idx / kDim;
+    int n = (int)(rn % half);
+    int r = (int)(rn / half);
+    __nv_bfloat16 val = R[((long long)r * kDim + k) * half + n];
+    const uint32_t off = tc::sw128_offset((uint32_t)n, (uint32_t)k);
+    *reinterpret_cast<__nv_bfloat16 *>(reinterpret_cast<uint8_t *>(Rs) + (long long)r * half * 128 + off) = val;
+}
+
+template <int NT>
+__global__ void __launch_bounds__(kThreads, 1)
+hash_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__restrict__ Rs,
+               uint16_t *__restrict__ buckets, long long rows_total, int L, int rounds, int half,
+               uint32_t *__restrict__ status)
+{
+    extern __shared__ uint8_t smem_raw[];
+    HashSmem &sm = *reinterpret_cast<HashSmem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const long long row0 = (long long)blockIdx.x * kRows;
+    const int n_nt = half / NT;
+    const int items = rounds * n_nt;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) { tc::mbar_init(&sm.full[s], 1); tc::mbar_init(&sm.empty[s], 1); }
+        for (int b = 0; b < 2; ++b) { tc::mbar_init(&sm.acc_full[b], 1); tc::mbar_init(&sm.acc_empty[b], kEpiWarps); }
+        sm.abort = 0;
+        tc::fence_mbar_init();
+    }
+    if (warp == 0) tc::tmem_alloc(&sm.tmem_base, kTmemCols);
+
+    // x rows -> A (K-major, 128-byte swizzle); rows past the end are zero.
+    for (int c = threadIdx.x; c < kRows * 8; c += kThreads) {
+        int r = c >> 3, ch = c & 7;
+        long long g = row0 + r;
+        uint4 val = make_uint4(0, 0, 0, 0);
+        if (g < rows_total) val = reinterpret_cast<const uint4 *>(x + g * kDim)[ch];
+        *reinterpret_cast<uint4 *>(sm.A + r * 128 + ((ch ^ (r & 7)) << 4)) = val;
+    }
+    tc::fence_async_smem();
+    tc::tc_fence_before();
+    __syncthreads();
+    tc::tc_fence_after();
+    const uint32_t tmem = sm.tmem_base;
+
+    if (warp == kEpiWarps) {
+        // ---------------- producer
+        if (lane == 0) {
+            for (int it = 0; it < items; ++it) {
+                const int s = it % kStages;
+                const uint32_t ph = (uint32_t)(it / kStages) & 1u;
+                if (it >= kStages && !tc::mbar_wait(&sm.empty[s], ph ^ 1u, &sm.abort, status)) break;
+                const int r = it / n_nt, nt = it % n_nt;
+                const __nv_bfloat16 *src = Rs + ((long long)r * half + (long long)nt * NT) * kDim;
+                tc::mbar_arrive_expect_tx(&sm.full[s], NT * 128);
+                tc::bulk_g2s(sm.B[s], src, NT * 128, &sm.full[s]);
+            }
+        }
+    } else if (warp == kEpiWarps + 1) {
+        // ---------------- MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idesc = tc::idesc_bf16(128, NT, 0, 0);
+            const uint32_t a0 = tc::smem_u32(sm.A);
+            for (int it = 0; it < items; ++it) {
+                const int s = it % kStages;
+                const uint32_t ph = (uint32_t)(it / kStages) & 1u;
+                const int ab = it & 1;
+                const uint32_t aph = (uint32_t)(it >> 1) & 1u;
+                if (!tc::mbar_wait(&sm.full[s], ph, &sm.abort, status)) break;
+                if (it >= 2 && !tc::mbar_wait(&sm.acc_empty[ab], aph ^ 1u, &sm.abort, status)) break;
+                tc::tc_fence_after();
+                const uint32_t b0 = tc::smem_u32(sm.B[s]);
+#pragma unroll
+                for (int mt = 0; mt < 2; ++mt) {
+                    const uint32_t d = tmem + (uint32_t)(ab * 2 * kMaxNT + mt * kMaxNT);
+#pragma unroll
+                    for (int k = 0; k < 4; ++k)
+                        tc::mma_bf16(d, tc::sw128_desc(a0 + mt * 128 * 128 + k * 32), tc::sw128_desc(b0 + k * 32),
+                                     idesc, k > 0);
+                }
+                tc::mma_commit(&sm.empty[s]);
+                tc::mma_commit(&sm.acc_full[ab]);
+            }
+        }
+    } else {
+        // ---------------- epilogue: one row per thread
+        const int q = warp & 3, mt = warp >> 2;
+        const int row = mt * 128 + q * 32 + lane;
+        const long long g = row0 + row;
+        const uint32_t lane_base = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(mt * kMaxNT);
+        float best = -INFINITY;
+        int bucket = 0;
+        for (int it = 0; it < items; ++it) {
+            const int ab = it & 1;
+            const uint32_t aph = (uint32_t)(it >> 1) & 1u;
+            if (!tc::mbar_wait(&sm.acc_full[ab], aph, &sm.abort, status)) break;
+            tc::tc_fence_after();
+            float v[NT];
+#pragma unroll
+            for (int c = 0; c < NT / 16; ++c) tc::tmem_ld16(lane_base + (uint32_t)(ab * 2 * kMaxNT + c * 16), v + c * 16);
+            tc::tmem_ld_wait();
+            tc::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(&sm.acc_empty[ab]);
+
+            // pass 1: extremes of the tile
+            float mx = v[0], mn = v[0];
+#pragma unroll
+            for (int j = 1; j + 1 < NT; j += 2) { mx = tc::max3f(mx, v[j], v[j + 1]); mn = tc::min3f(mn, v[j], v[j + 1]); }
+            mx = fmaxf(mx, v[NT - 1]);
+            mn = fminf(mn, v[NT - 1]);
+            const bool pos = mx >= -mn;
+            const float target = pos ? mx : mn;
+            // pass 2: lowest column holding the extreme
+            int js = NT - 1;
+#pragma unroll
+            for (int j = NT - 2; j >= 0; --j) js = (v[j] == target) ? j : js;
+            const int r = it / n_nt, nt = it % n_nt;
+            const float tbest = pos ? mx : -mn;
+            const int tb = (pos ? 0 : half) + nt * NT + js;
+            if (tbest > best || (tbest == best && tb < bucket)) { best = tbest; bucket = tb; }
+            if (nt == n_nt - 1) {
+                if (g < rows_total) {
+                    const long long bh = g / L;
+                    const int i = (int)(g % L);
+                    buckets[(bh * rounds + r) * L + i] = (uint16_t)bucket;
+                }
+                best = -INFINITY;
+                bucket = 0;
+            }
+        }
+    }
+
+    tc::tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc::tc_fence_after();
+        tc::tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+template <int NT>
+cudaError_t launch_nt(const Problem &p, const void *x, const __nv_bfloat16 *Rs, uint16_t *buckets, uint32_t *status,
+                      cudaStream_t st)
+{
+    // one CTA per SM: each holds all 512 TMEM columns
+    const size_t smem = std::max<size_t>(sizeof(HashSmem) + 1024, 120 * 1024);
+    cudaError_t e = cudaFuncSetAttribute(hash_tc_kernel<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    const long long rows = p.tokens();
+    const unsigned grid = (unsigned)((rows + kRows - 1) / kRows);
+    hash_tc_kernel<NT><<<grid, kThreads, smem, st>>>((const __nv_bfloat16 *)x, Rs, buckets, rows, p.L, p.R, p.nb / 2,
+                                                     status);
+    return cudaGetLastError();
+}
+
+int pick_nt(int half)
+{
+    if (half % 128 == 0) return 128;
+    if (half % 96 == 0) return 96;
+    if (half % 64 == 0) return 64;
+    if (half % 32 == 0) return 32;
+    return 0;
+}
+
+}  // namespace
+
+bool hash_tc_supported(const Problem &p) { return p.dtype == LSH_BF16 && p.d == kDim && pick_nt(p.nb / 2) != 0; }
+
+size_t hash_tc_scratch_bytes(const Problem &p) { return (size_t)p.R * (p.nb / 2) * kDim * sizeof(__nv_bfloat16); }
+
+cudaError_t launch_hash_tc(const Problem &p, const void *x, const void *R, uint16_t *buckets, void *scratch,
+                           uint32_t *status, cudaStream_t st)
+{
+    const int half = p.nb / 2;
+    __nv_bfloat16 *Rs = (__nv_bfloat16 *)scratch;
+    const long long total = (long long)p.R * half * kDim;
+    rot_swizzle_kernel<<<(unsigned)((total + 255) / 256), 256, 0, st>>>((const __nv_bfloat16 *)R, Rs, half, p.R);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    switch (pick_nt(half)) {
+    case 128: return launch_nt<128>(p, x, Rs, buckets, status, st);
+    case 96: return launch_nt<96>(p, x, Rs, buckets, status, st);
+    case 64: return launch_nt<64>(p, x, Rs, buckets, status, st);
+    case 32: return launch_nt<32>(p, x, Rs, buckets, status, st);
+    default: return cudaErrorInvalidValue;
+    }
+}
+
+}  // namespace lsh
