@@ -127,8 +127,12 @@ __device__ __forceinline__ void key_row_block(const Stage &st, uint8_t (*ET)[kK 
                 const int q = C0 + h * 32 + j + u;
                 const float4 qi = st.qinfo[q];
                 const int qp = __float_as_int(qi.w);
-                const bool valid = (causal ? (kpos < qp) : (kpos != qp)) || (kpos == qp && qi.z != 0.f);
-                const float p = valid ? exp2f(fmaf(s[j + u], sc, -qi.x)) : 0.f;
+                // branch-free mask: candidate if causal-earlier (or any other position when
+                // not causal), or the query itself when it has no other candidate
+                const int ordered = causal ? (kpos < qp) : (kpos != qp);
+                const int self = (kpos == qp) & (qi.z != 0.f);
+                const float e2 = tc::fast_exp2(fmaf(s[j + u], sc, -qi.x));
+                const float p = (ordered | self) ? e2 : 0.f;
                 pv[u] = p;
                 ev[u] = ec * p * (dp[j + u] - qi.y);
             }
@@ -209,6 +213,11 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_consta
 
     if (warp == kComputeWarps) {
         // ================= producer
+        if (lane == 0) {
+            tc::prefetch_tmap(&tm_x);
+            tc::prefetch_tmap(&tm_v);
+            tc::prefetch_tmap(&tm_g);
+        }
         int it = 0;
         for (long long tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++it) {
             const int s = it % kStages;
@@ -224,21 +233,20 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_consta
                 const int sl = slot0 + e;
                 st.pos[e] = (sl >= 0 && sl < L) ? P[sl] : -1;
             }
+            if (lane == 0) tc::mbar_expect_tx(&sm.full[s], kStageBytes);
             __syncwarp();
-            // TMA gathers: rows by global row index (-1 -> zero fill)
-            if (lane == 0) {
-                tc::mbar_expect_tx(&sm.full[s], kStageBytes);
-                for (int w = 0; w < kQ; w += 4) {
-                    int rr[4];
+            // TMA gathers, four rows per instruction, spread over the lanes
+            // (row index -1 = missing slot -> zero fill)
+            for (int gi = lane; gi < kQ / 4; gi += 32) {
+                int rr[4];
 #pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        const int p = st.pos[64 + w + u];
-                        rr[u] = p >= 0 ? (int)(rowbase + p) : -1;
-                    }
-                    tc::tma_gather4(st.X + w * 128, &tm_x, rr[0], rr[1], rr[2], rr[3], &sm.full[s]);
-                    tc::tma_gather4(st.G + w * 128, &tm_g, rr[0], rr[1], rr[2], rr[3], &sm.full[s]);
-                    if (w < kK) tc::tma_gather4(st.V + w * 128, &tm_v, rr[0], rr[1], rr[2], rr[3], &sm.full[s]);
+                for (int u = 0; u < 4; ++u) {
+                    const int p = st.pos[64 + 4 * gi + u];
+                    rr[u] = p >= 0 ? (int)(rowbase + p) : -1;
                 }
+                tc::tma_gather4(st.X + gi * 512, &tm_x, rr[0], rr[1], rr[2], rr[3], &sm.full[s]);
+                tc::tma_gather4(st.G + gi * 512, &tm_g, rr[0], rr[1], rr[2], rr[3], &sm.full[s]);
+                if (gi < kK / 4) tc::tma_gather4(st.V + gi * 512, &tm_v, rr[0], rr[1], rr[2], rr[3], &sm.full[s]);
             }
             // window minima of positions for the self flags (chunks 2k-1 .. 2k+2)
             int cmin[4];
@@ -253,17 +261,33 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_consta
                 for (int o = 16; o > 0; o >>= 1) mn = min(mn, __shfl_xor_sync(0xffffffffu, mn, o));
                 cmin[c] = mn;
             }
-            for (int q = lane; q < kQ; q += 32) {
-                const int p = st.pos[64 + q];
-                const int qa = q >> 6;
-                const int wmin = min(cmin[qa], cmin[qa + 1]);
-                float4 qi;
-                qi.x = p >= 0 ? lse_all[rowbase + p] * kLog2e : INFINITY;
-                qi.y = p >= 0 ? delta[rowbase + p] : 0.f;
-                qi.z = (p >= 0 && causal && p == wmin) ? 1.f : 0.f;
-                qi.w = __int_as_float(p);
-                st.qinfo[q] = qi;
-                if (q < kK) st.kinv[q] = p >= 0 ? invnorm[rowbase + p] : 0.f;
+            // per-query LSE / delta and per-key norms: all loads issued before any is used
+            {
+                int qp[kQ / 32];
+                float ql[kQ / 32], qd[kQ / 32], kn[kK / 32];
+#pragma unroll
+                for (int j = 0; j < kQ / 32; ++j) qp[j] = st.pos[64 + lane + 32 * j];
+#pragma unroll
+                for (int j = 0; j < kQ / 32; ++j) {
+                    const bool ok = qp[j] >= 0;
+                    ql[j] = ok ? lse_all[rowbase + qp[j]] : 0.f;
+                    qd[j] = ok ? delta[rowbase + qp[j]] : 0.f;
+                    if (j < kK / 32) kn[j] = ok ? invnorm[rowbase + qp[j]] : 0.f;
+                }
+#pragma unroll
+                for (int j = 0; j < kQ / 32; ++j) {
+                    const int q = lane + 32 * j;
+                    const int p = qp[j];
+                    const int qa = q >> 6;
+                    const int wmin = min(cmin[qa], cmin[qa + 1]);
+                    float4 qi;
+                    qi.x = p >= 0 ? ql[j] * kLog2e : INFINITY;
+                    qi.y = qd[j];
+                    qi.z = (p >= 0 && causal && p == wmin) ? 1.f : 0.f;
+                    qi.w = __int_as_float(p);
+                    st.qinfo[q] = qi;
+                    if (j < kK / 32) st.kinv[q] = kn[j];
+                }
             }
             if (lane == 0) st.tile = tile;
             __threadfence_block();

@@ -9,21 +9,34 @@
 // so one gathered tile serves as both MMA operands.
 //
 // Per tile:
-//   gather   rows x[perm[s]] and v[perm[s]] for the 192 window slots, 16-byte
-//            cp.async copies written straight into the 128-byte-swizzled
-//            K-major layout the tensor core reads;
+//   gather   rows x[perm[s]] and v[perm[s]] of the 192 window slots by TMA
+//            (tile::gather4, four rows per instruction) straight into the
+//            128-byte-swizzled layout the tensor core reads;
 //   S = Q K^T  tcgen05.mma M=128, N=192, K=64 into tensor memory (raw
 //            dot products x_i . x_j, bf16 in, fp32 accumulate);
 //   softmax  one query row per thread: s_ij = (x_i . x_j) / |x_j| / sqrt(d)
 //            (unit keys), masked to the window of the row's chunk, to
 //            earlier original positions when causal, and never the query's
 //            own position unless nothing else is left ("Implementation
-//            Reading"); full softmax (the window fits), P written as bf16;
-//   O = P V  tcgen05.mma M=128, N=64, K=192 (V read MN-major);
+//            Reading"); P is written as bf16 back into the S columns;
+//   O = P V  tcgen05.mma M=128, N=64, K=192 with A = P read from tensor
+//            memory and V read MN-major from shared memory;
 //   store    o_r and lse_r at the query's original position (the unsort).
 //
-// Two CTAs per SM (96 KB shared memory, 256 TMEM columns each) overlap one
-// CTA's gather and MMAs with the other's softmax.
+// Scores satisfy s_ij <= tau |x_i| (Cauchy-Schwarz with unit keys), so the
+// softmax uses M = tau |x_i| in place of the row maximum: one sweep, no max
+// pass.  A warp whose rows have tau |x_i| so large that exp(s - M) could leave
+// the normal fp32 range first finds the exact maximum.  A query with no
+// other candidate (causal: its position is the smallest of its window) keeps
+// its own key, whose score is tau |x_i|, so p = 1 there and lse = tau |x_i|.
+//
+// Warp roles (persistent CTA, one per SM):
+//   warps 0-3, 4-7  two softmax groups working on alternate tiles, each with
+//                   its own 256 TMEM columns (S/P 192, O 64), so one group's
+//                   softmax overlaps the other's MMAs and stores;
+//   warp 8          producer: positions, key norms and window minima, then TMA
+//                   row gathers, into a 3-stage shared-memory ring;
+//   warp 9          MMA issuer.
 #include "tc_common.cuh"
 
 namespace lsh {
@@ -32,139 +45,120 @@ namespace {
 
 constexpr int kQ = 128;             // query slots per tile
 constexpr int kW = 192;             // window rows (keys)
-constexpr int kThreads = 128;
-constexpr int kTmemCols = 256;      // S: 192 columns, O: 64 columns
+constexpr int kStages = 3;
+constexpr int kThreads = 320;
+constexpr int kTmemCols = 512;
+constexpr uint32_t kGroupCols = 256;
+constexpr uint32_t kOCol = 192;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
+constexpr uint32_t kStageBytes = 2 * kW * 128;
 
-struct FwdSmem {
+struct alignas(1024) Stage {
     uint8_t X[kW * 128];            // gathered x rows, K-major SW128 (24 KB)
     uint8_t V[kW * 128];            // gathered v rows (24 KB)
-    uint8_t P[3][kQ * 128];         // probabilities, 3 K-blocks of 64 keys (48 KB)
-    alignas(16) int32_t pos[kW];
-    alignas(16) float inv[kW];
-    uint64_t bar_s, bar_o;
+    alignas(16) int32_t pos[kW];    // original positions of the window slots (-1: none)
+    alignas(16) float sinv[kW];     // tau * log2(e) / |x_j| (0 for a zero row or no row)
+    alignas(16) float inv[kW];      // 1 / |x_j|
+    int32_t cmin[3];                // smallest position in each window chunk (INT_MAX if none)
+};
+
+struct FwdSmem {
+    Stage st[kStages];
+    uint64_t full[kStages], empty[kStages];
+    uint64_t s_full[2], p_full[2], o_full[2], o_free[2];
     uint32_t tmem_base;
     int abort;
 };
 
-// Softmax of one query row (thread) over the 128 window columns its chunk may
-// see: window columns [BASE, BASE + 128) (chunk 2k: BASE = 0, chunk 2k+1:
-// BASE = 64); `jlo` skips the missing chunk -1 of the first tile.  Writes the
-// row of P (bf16, zeros elsewhere) into shared memory.
-//
-// Scores are s_j = tau (x_i . x_j) / |x_j| <= tau |x_i| (Cauchy-Schwarz), so
-// M = tau |x_i| bounds the row maximum and p_j = exp(s_j - M) needs no max
-// pass: one sweep over tensor memory gives P and l = sum p_j, and
-// lse = M + log(l).  When the bound is so loose that every p_j would
-// underflow (|x_i| in the hundreds) the warp redoes the row with the exact
-// maximum.  A row with no candidate at all attends to itself (p = 1 there,
-// lse = tau |x_i|).
+struct TileCoord {
+    int r, k;
+    long long bh, seg;
+};
+__device__ __forceinline__ TileCoord tile_coord(long long tile, int R, int n_k)
+{
+    // order (bh, k, r): tiles in flight at the same time share a head's rows in L2
+    TileCoord c;
+    c.r = (int)(tile % R);
+    const long long bk = tile / R;
+    c.k = (int)(bk % n_k);
+    c.bh = bk / n_k;
+    c.seg = c.bh * R + c.r;
+    return c;
+}
+
+// Softmax of one query row (thread) over window columns [BASE, BASE + 128)
+// (chunk 2k: BASE = 0, chunk 2k+1: BASE = 64); `jlo` skips the missing chunk
+// -1 of a segment's first tile.  P is written as packed bf16 pairs into the
+// row's own S columns (key j -> column j/2), in place: chunk c of 16 scores is
+// read before packed columns BASE/2 + [8c, 8c+8) are written, and those never
+// reach an unread chunk.  Columns outside the row's window get zeros.
 template <int BASE>
-__device__ __forceinline__ void softmax_row(FwdSmem &sm, uint32_t taddr, bool ok, int jlo, int i, int qpos, float qinv,
+__device__ __forceinline__ void softmax_row(const Stage &st, uint32_t tl, int jlo, int qpos, float qinv, int self_only,
                                             int causal, float tau, float &l, float &row_lse)
 {
-    const float sl2 = tau * kLog2e;
-    const float bound = qinv > 0.f ? tau / qinv : 0.f;      // tau |x_i|
-    // pass over the 8 TMEM chunks of 16 columns; `shift` is the log2-domain offset
-    auto sweep = [&](float shift, float &lsum, bool &any) {
-        lsum = 0.f;
-        any = false;
-#pragma unroll 1
-        for (int c = 0; c < 8; ++c) {
-            float v[16];
-            if (ok) {
-                tc::tmem_ld16(taddr + (uint32_t)(BASE + c * 16), v);
-                tc::tmem_ld_wait();
-            }
-            uint32_t w[8];
-#pragma unroll
-            for (int e4 = 0; e4 < 16; e4 += 4) {
-                const int4 kp = *reinterpret_cast<const int4 *>(&sm.pos[BASE + c * 16 + e4]);
-                const float4 kv = *reinterpret_cast<const float4 *>(&sm.inv[BASE + c * 16 + e4]);
-                const int kpa[4] = {kp.x, kp.y, kp.z, kp.w};
-                const float kva[4] = {kv.x, kv.y, kv.z, kv.w};
-                float pe[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int j = c * 16 + e4 + e;
-                    const bool valid = (j >= jlo) && (causal ? (kpa[e] < qpos) : (kpa[e] != qpos));
-                    const float p = exp2f(fmaf(v[e4 + e], kva[e] * sl2, -shift));
-                    pe[e] = valid ? p : 0.f;
-                    any |= valid;
-                    lsum += pe[e];
-                }
-                w[e4 / 2] = pack_bf16x2(pe[0], pe[1]);
-                w[e4 / 2 + 1] = pack_bf16x2(pe[2], pe[3]);
-            }
-            // window column BASE + 16c .. +15 -> P block (BASE + 16c) / 64, chunks 2 at a time
-            const int col = BASE + c * 16;
-            uint8_t *blk = sm.P[col >> 6];
-            const int ch0 = (col & 63) >> 3;
-            *reinterpret_cast<uint4 *>(blk + i * 128 + ((ch0 ^ (i & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
-            *reinterpret_cast<uint4 *>(blk + i * 128 + (((ch0 + 1) ^ (i & 7)) << 4)) = make_uint4(w[4], w[5], w[6], w[7]);
-        }
-    };
-    float lsum;
-    bool any;
-    sweep(bound * kLog2e, lsum, any);
-    l = lsum;
-    row_lse = bound + kLn2 * log2f(lsum);
-    // exact-maximum redo for rows whose bound underflowed every term
-    const bool redo = any && !(lsum > 1e-30f);
-    if (__any_sync(0xffffffffu, redo)) {
+    const float bound = qinv > 0.f ? tau / qinv : 0.f;        // tau |x_i| >= every score of the row
+    float shift2 = bound * kLog2e;                              // log2-domain offset
+    // exp(s - bound) stays normal unless bound - s, <= 2 bound, exceeds ~100 in log2 units
+    const bool wide = 2.f * bound * kLog2e > 100.f;
+    if (__any_sync(0xffffffffu, wide)) {
         float mx = -INFINITY;
 #pragma unroll 1
         for (int c = 0; c < 8; ++c) {
             float v[16];
-            if (ok) {
-                tc::tmem_ld16(taddr + (uint32_t)(BASE + c * 16), v);
-                tc::tmem_ld_wait();
-            }
+            tc::tmem_ld16(tl + (uint32_t)(BASE + c * 16), v);
+            tc::tmem_ld_wait();
 #pragma unroll
             for (int e = 0; e < 16; ++e) {
                 const int j = c * 16 + e;
-                const int kp = sm.pos[BASE + j];
-                const bool valid = (j >= jlo) && (causal ? (kp < qpos) : (kp != qpos));
-                if (valid) mx = fmaxf(mx, v[e] * sm.inv[BASE + j] * tau);
+                const int kp = st.pos[BASE + j];
+                const int ok = ((j >= jlo) & (causal ? (kp < qpos) : (kp != qpos))) | (self_only & (kp == qpos));
+                mx = ok ? fmaxf(mx, v[e] * st.sinv[BASE + j]) : mx;
             }
         }
-        // every thread of the warp takes part (tcgen05.ld is warp-wide); rows that
-        // did not need the redo recompute exactly what they already wrote
-        const float shift = redo ? mx * kLog2e : bound * kLog2e;
-        float l2;
-        bool any2;
-        sweep(shift, l2, any2);
-        if (redo) {
-            l = l2;
-            row_lse = mx + kLn2 * log2f(l2);
-        }
+        if (wide && mx > -INFINITY) shift2 = mx;
     }
-    // zero the columns outside [BASE, BASE + 128)
-    {
-        constexpr int zcol = BASE == 0 ? 128 : 0;
-        uint8_t *blk = sm.P[zcol >> 6];
+    float lsum = 0.f;
+#pragma unroll 1
+    for (int c = 0; c < 8; ++c) {
+        float v[16];
+        tc::tmem_ld16(tl + (uint32_t)(BASE + c * 16), v);
+        tc::tmem_ld_wait();
+        uint32_t w[8];
 #pragma unroll
-        for (int ch = 0; ch < 8; ++ch)
-            *reinterpret_cast<uint4 *>(blk + i * 128 + ((ch ^ (i & 7)) << 4)) = make_uint4(0, 0, 0, 0);
+        for (int e4 = 0; e4 < 16; e4 += 4) {
+            const int4 kp = *reinterpret_cast<const int4 *>(&st.pos[BASE + c * 16 + e4]);
+            const float4 ks = *reinterpret_cast<const float4 *>(&st.sinv[BASE + c * 16 + e4]);
+            const int kpa[4] = {kp.x, kp.y, kp.z, kp.w};
+            const float ksa[4] = {ks.x, ks.y, ks.z, ks.w};
+            float pe[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int j = c * 16 + e4 + e;
+                const int ok =
+                    ((j >= jlo) & (causal ? (kpa[e] < qpos) : (kpa[e] != qpos))) | (self_only & (kpa[e] == qpos));
+                const float p = tc::fast_exp2(fmaf(v[e4 + e], ksa[e], -shift2));
+                pe[e] = ok ? p : 0.f;
+                lsum += pe[e];
+            }
+            w[e4 / 2] = pack_bf16x2(pe[0], pe[1]);
+            w[e4 / 2 + 1] = pack_bf16x2(pe[2], pe[3]);
+        }
+        tc::tmem_st8(tl + (uint32_t)(BASE / 2 + c * 8), w);
     }
-    if (!any) {
-        // nothing but the query itself: p = 1 on its own column (window row 64 + i)
-        const int col = 64 + i;
-        uint8_t *blk = sm.P[col >> 6];
-        const int cc = col & 63;
-        const int ch = cc >> 3;
-        uint32_t w[4] = {0, 0, 0, 0};
-        const int e = cc & 7;
-        w[e >> 1] = (e & 1) ? 0x3F800000u : 0x00003F80u;       // bf16 1.0 in the low or high half
-        *reinterpret_cast<uint4 *>(blk + i * 128 + ((ch ^ (i & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
-        l = 1.f;
-        row_lse = bound;                                         // tau * x_i . (x_i / |x_i|)
+    // zeros for the keys outside this row's window (packed columns of keys 128..191 or 0..63)
+    {
+        const uint32_t z[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+        constexpr uint32_t zc = BASE == 0 ? 64 : 0;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tc::tmem_st8(tl + zc + c * 8, z);
     }
+    l = lsum;
+    row_lse = kLn2 * (shift2 + log2f(lsum));
 }
 
-__global__ void __launch_bounds__(kThreads, 2)
-attn_fwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__restrict__ v,
+__global__ void __launch_bounds__(kThreads, 1)
+attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_v,
                    const int32_t *__restrict__ perm, const float *__restrict__ invnorm,
                    __nv_bfloat16 *__restrict__ o_r, float *__restrict__ lse, int L, int R, long long n_tiles,
                    int causal, float tau, uint32_t *__restrict__ status)
@@ -175,8 +169,16 @@ attn_fwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
     const int n_k = L / kQ;
 
     if (tid == 0) {
-        tc::mbar_init(&sm.bar_s, 1);
-        tc::mbar_init(&sm.bar_o, 1);
+        for (int s = 0; s < kStages; ++s) {
+            tc::mbar_init(&sm.full[s], 1);
+            tc::mbar_init(&sm.empty[s], 4);
+        }
+        for (int g = 0; g < 2; ++g) {
+            tc::mbar_init(&sm.s_full[g], 1);
+            tc::mbar_init(&sm.p_full[g], 4);
+            tc::mbar_init(&sm.o_full[g], 1);
+            tc::mbar_init(&sm.o_free[g], 4);
+        }
         sm.abort = 0;
         tc::fence_mbar_init();
     }
@@ -185,101 +187,150 @@ attn_fwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
     __syncthreads();
     tc::tc_fence_after();
     const uint32_t tmem = sm.tmem_base;
-    const uint32_t tS = tmem, tO = tmem + kW;
-    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
-    uint32_t phase = 0;
+    const float sl2 = tau * kLog2e;
 
-    for (long long tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, phase ^= 1u) {
-        // tile order (bh, k, r): concurrent tiles share a head's rows in L2
-        const int r = (int)(tile % R);
-        const long long bk = tile / R;
-        const int k = (int)(bk % n_k);
-        const long long bh = bk / n_k;
-        const long long seg = bh * R + r;
-        const int32_t *P = perm + seg * L;
-        const __nv_bfloat16 *X = x + bh * L * kDim;
-        const __nv_bfloat16 *V = v + bh * L * kDim;
-        const int slot0 = k * kQ - 64;          // window slot of row 0
-
-        // ---- positions and key norms of the window
-        for (int w = tid; w < kW; w += kThreads) {
-            int s = slot0 + w;
-            int p = s >= 0 ? P[s] : -1;
-            sm.pos[w] = p;
-            sm.inv[w] = p >= 0 ? invnorm[bh * L + p] : 0.f;
+    if (warp == 8) {
+        // ================= producer
+        if (lane == 0) {
+            tc::prefetch_tmap(&tm_x);
+            tc::prefetch_tmap(&tm_v);
         }
-        __syncthreads();
-        // ---- gather rows into the swizzled operand tiles
-        for (int c = tid; c < kW * 8; c += kThreads) {
-            int w = c >> 3, ch = c & 7;
-            uint32_t off = (uint32_t)w * 128u + (uint32_t)((ch ^ (w & 7)) << 4);
-            int p = sm.pos[w];
-            if (p >= 0) {
-                tc::cp_async16(sm.X + off, X + (long long)p * kDim + ch * 8);
-                tc::cp_async16(sm.V + off, V + (long long)p * kDim + ch * 8);
-            } else {
-                *reinterpret_cast<uint4 *>(sm.X + off) = make_uint4(0, 0, 0, 0);
-                *reinterpret_cast<uint4 *>(sm.V + off) = make_uint4(0, 0, 0, 0);
+        int it = 0;
+        for (long long tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++it) {
+            const int s = it % kStages;
+            if (it >= kStages &&
+                !tc::mbar_wait(&sm.empty[s], (uint32_t)((it / kStages) - 1) & 1u, &sm.abort, status))
+                break;
+            Stage &st = sm.st[s];
+            const TileCoord tcd = tile_coord(tile, R, n_k);
+            const int32_t *P = perm + tcd.seg * L;
+            const long long rowbase = tcd.bh * L;
+            const int slot0 = tcd.k * kQ - 64;
+            int pj[kW / 32];
+#pragma unroll
+            for (int j = 0; j < kW / 32; ++j) {
+                const int sl = slot0 + lane + 32 * j;
+                pj[j] = sl >= 0 ? P[sl] : -1;
+                st.pos[lane + 32 * j] = pj[j];
+            }
+            if (lane == 0) tc::mbar_expect_tx(&sm.full[s], kStageBytes);
+            __syncwarp();
+            for (int gi = lane; gi < kW / 4; gi += 32) {
+                int rr[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int p = st.pos[4 * gi + u];
+                    rr[u] = p >= 0 ? (int)(rowbase + p) : -1;
+                }
+                tc::tma_gather4(st.X + gi * 512, &tm_x, rr[0], rr[1], rr[2], rr[3], &sm.full[s]);
+                tc::tma_gather4(st.V + gi * 512, &tm_v, rr[0], rr[1], rr[2], rr[3], &sm.full[s]);
+            }
+            float nv[kW / 32];
+#pragma unroll
+            for (int j = 0; j < kW / 32; ++j) nv[j] = pj[j] >= 0 ? invnorm[rowbase + pj[j]] : 0.f;
+#pragma unroll
+            for (int j = 0; j < kW / 32; ++j) {
+                st.inv[lane + 32 * j] = nv[j];
+                st.sinv[lane + 32 * j] = nv[j] * sl2;
+            }
+            // smallest position of each window chunk: window chunk c holds lanes' j = 2c, 2c + 1
+#pragma unroll
+            for (int c = 0; c < 3; ++c) {
+                int mn = min(pj[2 * c] >= 0 ? pj[2 * c] : INT_MAX, pj[2 * c + 1] >= 0 ? pj[2 * c + 1] : INT_MAX);
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) mn = min(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+                if (lane == 0) st.cmin[c] = mn;
+            }
+            __threadfence_block();
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(&sm.full[s]);
+        }
+    } else if (warp == 9) {
+        // ================= MMA issuer: S of tile t+1 is issued before O of tile t
+        if (lane == 0) {
+            constexpr uint32_t id_s = tc::idesc_bf16(128, kW, 0, 0);
+            constexpr uint32_t id_o = tc::idesc_bf16(128, kDim, 0, 1);
+            int prev_it = -1;
+            int it = 0;
+            for (long long tile = blockIdx.x;; tile += gridDim.x, ++it) {
+                const bool have = tile < n_tiles;
+                if (have) {
+                    const int s = it % kStages, g = it & 1;
+                    bool ok = tc::mbar_wait(&sm.full[s], (uint32_t)(it / kStages) & 1u, &sm.abort, status);
+                    if (ok && it >= 2)
+                        ok = tc::mbar_wait(&sm.o_free[g], (uint32_t)((it >> 1) - 1) & 1u, &sm.abort, status);
+                    if (!ok) break;
+                    tc::tc_fence_after();
+                    const uint32_t xs = tc::smem_u32(sm.st[s].X);
+                    const uint32_t d = tmem + (uint32_t)g * kGroupCols;
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        tc::mma_bf16(d, tc::sw128_desc(xs + 64 * 128 + kk * 32), tc::sw128_desc(xs + kk * 32), id_s,
+                                     kk > 0);
+                    tc::mma_commit(&sm.s_full[g]);
+                }
+                if (prev_it >= 0) {
+                    const int ps = prev_it % kStages, pg = prev_it & 1;
+                    if (!tc::mbar_wait(&sm.p_full[pg], (uint32_t)(prev_it >> 1) & 1u, &sm.abort, status)) break;
+                    tc::tc_fence_after();
+                    const uint32_t vs = tc::smem_u32(sm.st[ps].V);
+                    const uint32_t base = tmem + (uint32_t)pg * kGroupCols;
+#pragma unroll
+                    for (int kk = 0; kk < 12; ++kk)
+                        tc::mma_bf16_ts(base + kOCol, base + kk * 8, tc::sw128_desc(vs + kk * 16 * 128), id_o, kk > 0);
+                    tc::mma_commit(&sm.o_full[pg]);
+                }
+                if (!have) break;
+                prev_it = it;
             }
         }
-        tc::cp_async_commit();
-        tc::cp_async_wait<0>();
-        tc::fence_async_smem();
-        __syncthreads();
-
-        // ---- S = Q K^T
-        if (tid == 0) {
+    } else {
+        // ================= softmax groups: group g takes the CTA's tiles it = g, g + 2, ...
+        const int g = warp >> 2, q = warp & 3;
+        const int i = q * 32 + lane;                             // query row = TMEM lane
+        const uint32_t tl = tmem + (uint32_t)g * kGroupCols + ((uint32_t)(q * 32) << 16);
+        int it = g;
+        for (long long tile = blockIdx.x + (long long)g * gridDim.x; tile < n_tiles;
+             tile += 2LL * gridDim.x, it += 2) {
+            const int s = it % kStages;
+            const uint32_t gph = (uint32_t)(it >> 1) & 1u;
+            if (!tc::mbar_wait(&sm.full[s], (uint32_t)(it / kStages) & 1u, &sm.abort, status)) break;
+            if (!tc::mbar_wait(&sm.s_full[g], gph, &sm.abort, status)) break;
             tc::tc_fence_after();
-            constexpr uint32_t idesc = tc::idesc_bf16(128, kW, 0, 0);
-            const uint32_t xs = tc::smem_u32(sm.X);
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-                tc::mma_bf16(tS, tc::sw128_desc(xs + 64 * 128 + kk * 32), tc::sw128_desc(xs + kk * 32), idesc, kk > 0);
-            tc::mma_commit(&sm.bar_s);
-        }
-        bool ok = tc::mbar_wait(&sm.bar_s, phase, &sm.abort, status);
-        tc::tc_fence_after();
-
-        // ---- softmax, one query row per thread
-        const int i = warp * 32 + lane;                 // query row in tile = window row 64 + i
-        const int qpos = sm.pos[64 + i];
-        const float qinv = sm.inv[64 + i];
-        float l = 1.f, row_lse = 0.f;
-        if (warp < 2)
-            softmax_row<0>(sm, tS + lane_off, ok, k == 0 ? 64 : 0, i, qpos, qinv, causal, tau, l, row_lse);
-        else
-            softmax_row<64>(sm, tS + lane_off, ok, 0, i, qpos, qinv, causal, tau, l, row_lse);
-        tc::fence_async_smem();
-        tc::tc_fence_before();
-        __syncthreads();
-
-        // ---- O = P V
-        if (tid == 0 && ok) {
+            const Stage &st = sm.st[s];
+            const TileCoord tcd = tile_coord(tile, R, n_k);
+            const int qpos = st.pos[64 + i];
+            const float qinv = st.inv[64 + i];
+            // query chunk a (0: 2k, 1: 2k+1) sees window chunks a and a+1
+            const int a = i >> 6;
+            const int self_only = causal && qpos == min(st.cmin[a], st.cmin[a + 1]);
+            float l, row_lse;
+            if (q < 2)
+                softmax_row<0>(st, tl, tcd.k == 0 ? 64 : 0, qpos, qinv, self_only, causal, tau, l, row_lse);
+            else
+                softmax_row<64>(st, tl, 0, qpos, qinv, self_only, causal, tau, l, row_lse);
+            tc::tmem_st_wait();
+            tc::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(&sm.p_full[g]);
+            if (!tc::mbar_wait(&sm.o_full[g], gph, &sm.abort, status)) break;
             tc::tc_fence_after();
-            constexpr uint32_t idesc = tc::idesc_bf16(128, kDim, 0, 1);
-            const uint32_t vs = tc::smem_u32(sm.V);
-#pragma unroll
-            for (int kk = 0; kk < 12; ++kk) {
-                const uint32_t pa = tc::smem_u32(sm.P[kk >> 2]) + (kk & 3) * 32;
-                tc::mma_bf16(tO, tc::sw128_desc(pa), tc::sw128_desc(vs + kk * 16 * 128), idesc, kk > 0);
-            }
-            tc::mma_commit(&sm.bar_o);
-        }
-        ok = ok && tc::mbar_wait(&sm.bar_o, phase, &sm.abort, status);
-        tc::tc_fence_after();
-        if (ok) {
             float o[kDim];
 #pragma unroll
-            for (int c = 0; c < 4; ++c) tc::tmem_ld16(tO + lane_off + (uint32_t)(c * 16), o + c * 16);
+            for (int c = 0; c < 4; ++c) tc::tmem_ld16(tl + kOCol + (uint32_t)(c * 16), o + c * 16);
             tc::tmem_ld_wait();
+            tc::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+                tc::mbar_arrive(&sm.o_free[g]);
+                tc::mbar_arrive(&sm.empty[s]);
+            }
             const float rl = 1.0f / l;
 #pragma unroll
             for (int d = 0; d < kDim; ++d) o[d] *= rl;
-            store_row(o_r + (seg * L + qpos) * kDim, o);
-            lse[seg * L + qpos] = row_lse;
+            store_row(o_r + (tcd.seg * L + qpos) * kDim, o);
+            lse[tcd.seg * L + qpos] = row_lse;
         }
-        tc::tc_fence_before();
-        if (__syncthreads_or(sm.abort != 0)) break;     // uniform exit after a timed-out wait
     }
 
     tc::tc_fence_before();
@@ -294,13 +345,15 @@ attn_fwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
 
 bool attn_tc_supported(const Problem &p)
 {
-    return p.dtype == LSH_BF16 && p.d == kDim && p.m == 64 && p.L % kQ == 0;
+    return p.dtype == LSH_BF16 && p.d == kDim && p.m == 64 && p.L % kQ == 0 && p.tokens() < (1LL << 31);
 }
 
 cudaError_t launch_attn_fwd_tc(const Problem &p, const void *x, const void *v, const int32_t *perm,
                                const float *invnorm, __nv_bfloat16 *o_r, float *lse, uint32_t *status,
                                cudaStream_t st)
 {
+    CUtensorMap tx, tv;
+    if (!tc::make_row_tmap(&tx, x, p.tokens()) || !tc::make_row_tmap(&tv, v, p.tokens())) return cudaErrorInvalidValue;
     const size_t smem = sizeof(FwdSmem) + 1024;
     cudaError_t e = cudaFuncSetAttribute(attn_fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
@@ -308,9 +361,8 @@ cudaError_t launch_attn_fwd_tc(const Problem &p, const void *x, const void *v, c
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const long long n_tiles = p.S() * (p.L / kQ);
-    const unsigned grid = (unsigned)std::min<long long>(n_tiles, 2LL * sms);
-    attn_fwd_tc_kernel<<<grid, kThreads, smem, st>>>((const __nv_bfloat16 *)x, (const __nv_bfloat16 *)v, perm,
-                                                     invnorm, o_r, lse, p.L, p.R, n_tiles, p.causal,
+    const unsigned grid = (unsigned)std::min<long long>(n_tiles, (long long)sms);
+    attn_fwd_tc_kernel<<<grid, kThreads, smem, st>>>(tx, tv, perm, invnorm, o_r, lse, p.L, p.R, n_tiles, p.causal,
                                                      1.0f / sqrtf((float)p.d), status);
     return cudaGetLastError();
 }
