@@ -31,11 +31,12 @@
 // Warp roles (persistent CTA, one per SM):
 //   warps 0-7  compute: warp w owns TMEM lanes 32*(w%4).. (key rows) and query
 //              columns half (w/4); elementwise step, then the epilogue;
-//   warp 8     producer: positions, per-query LSE / delta / self flags and
-//              per-key norms into a 2-stage ring, then TMA row gathers
-//              (tile::gather4, 128-byte swizzle) of x, v and dY rows;
-//   warp 9     MMA issuer.
-// The producer runs up to two tiles ahead, so gathers overlap compute.
+//   warps 8-11 producer: positions, per-query LSE / delta / self flags and
+//              per-key norms into a 2-stage ring, then 16-byte cp.async
+//              gathers of the x, v and dY rows straight into the swizzled
+//              operand layout; a stage is published once the next stage's
+//              copies are in flight;
+//   warp 12    MMA issuer.
 #include "tc_common.cuh"
 
 namespace lsh {
@@ -46,10 +47,12 @@ constexpr int kK = 128;             // key slots per tile
 constexpr int kQ = 192;             // query slots per tile
 constexpr int kStages = 2;
 constexpr int kComputeWarps = 8;
-constexpr int kThreads = (kComputeWarps + 2) * 32;
+constexpr int kProducerWarps = 4;
+constexpr int kProducerThreads = kProducerWarps * 32;
+constexpr int kMmaWarp = kComputeWarps + kProducerWarps;
+constexpr int kThreads = (kMmaWarp + 1) * 32;
 constexpr int kTmemCols = 512;
 constexpr float kLog2e = 1.4426950408889634f;
-constexpr uint32_t kStageBytes = (kQ + kK + kQ) * 128;   // x, v, dY rows landed by TMA per tile
 
 // TMEM columns.  Elementwise phase: S^T [0,192), P^T packed [192,288), dP^T [288,480).
 // After it: dV [0,64), G [64,128), dQ rows 0-127 [128,192), dQ rows 64-191 [288,352).
@@ -63,7 +66,7 @@ struct alignas(1024) Stage {
     alignas(16) int32_t pos[256];   // positions of slots [128k - 64, 128k + 192); -1 if none
     alignas(16) float4 qinfo[kQ];   // {LSE * log2 e (+inf if none), delta, self flag, position bits}
     alignas(16) float kinv[kK];
-    long long tile;
+    int32_t cmin[4];                // smallest position of chunks 2k-1 .. 2k+2 (INT_MAX if none)
 };
 
 struct BwdSmem {
@@ -87,18 +90,15 @@ __device__ __forceinline__ void red_row(float *dst, const float *r)
     for (int c = 0; c < 16; ++c) red_add_v4(dst + 4 * c, r[4 * c], r[4 * c + 1], r[4 * c + 2], r[4 * c + 3]);
 }
 
-// bf16 row `row` of a K-major SW128 tile -> 64 floats.
-__device__ __forceinline__ void smem_row(const uint8_t *tile, int row, float *out)
+// Chunk `ch` (elements 8ch .. 8ch+7) of bf16 row `row` of a K-major SW128 tile.
+__device__ __forceinline__ void smem_chunk(const uint8_t *tile, int row, int ch, float *out)
 {
+    const uint4 u = *reinterpret_cast<const uint4 *>(tile + row * 128 + ((ch ^ (row & 7)) << 4));
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
-    for (int ch = 0; ch < 8; ++ch) {
-        const uint4 u = *reinterpret_cast<const uint4 *>(tile + row * 128 + ((ch ^ (row & 7)) << 4));
-        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            out[ch * 8 + 2 * e] = __uint_as_float(w[e] << 16);
-            out[ch * 8 + 2 * e + 1] = __uint_as_float(w[e] & 0xFFFF0000u);
-        }
+    for (int e = 0; e < 4; ++e) {
+        out[2 * e] = __uint_as_float(w[e] << 16);
+        out[2 * e + 1] = __uint_as_float(w[e] & 0xFFFF0000u);
     }
 }
 
@@ -181,9 +181,8 @@ __device__ __forceinline__ TileCoord tile_coord(long long tile, int R, int n_k)
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
-attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_v,
-                   const __grid_constant__ CUtensorMap tm_g, const __nv_bfloat16 *__restrict__ x,
-                   const int32_t *__restrict__ perm, const float *__restrict__ invnorm,
+attn_bwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__restrict__ v,
+                   const __nv_bfloat16 *__restrict__ dout, const int32_t *__restrict__ perm, const float *__restrict__ invnorm,
                    const float *__restrict__ lse_all, const float *__restrict__ delta, float *__restrict__ dx_acc,
                    float *__restrict__ dv_acc, int L, int R, long long n_tiles, int causal, float tau,
                    uint32_t *__restrict__ status)
@@ -195,7 +194,7 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_consta
 
     if (tid == 0) {
         for (int s = 0; s < kStages; ++s) {
-            tc::mbar_init(&sm.full[s], 1);
+            tc::mbar_init(&sm.full[s], kProducerThreads);
             tc::mbar_init(&sm.empty[s], kComputeWarps);
         }
         tc::mbar_init(&sm.bar_s, 1);
@@ -211,90 +210,78 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_consta
     tc::tc_fence_after();
     const uint32_t tmem = sm.tmem_base;
 
-    if (warp == kComputeWarps) {
-        // ================= producer
-        if (lane == 0) {
-            tc::prefetch_tmap(&tm_x);
-            tc::prefetch_tmap(&tm_v);
-            tc::prefetch_tmap(&tm_g);
-        }
+    if (warp >= kComputeWarps && warp < kMmaWarp) {
+        // ================= producer group
+        const int ptid = tid - kComputeWarps * 32, pw = ptid >> 5;
+        int prev_s = -1;
         int it = 0;
         for (long long tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++it) {
             const int s = it % kStages;
-            if (it >= kStages &&
-                !tc::mbar_wait(&sm.empty[s], (uint32_t)((it / kStages) - 1) & 1u, &sm.abort, status))
-                break;
+            bool ok = it < kStages ||
+                      tc::mbar_wait(&sm.empty[s], (uint32_t)((it / kStages) - 1) & 1u, &sm.abort, status);
+            if (tc::named_bar_or(1, kProducerThreads, !ok)) { prev_s = -1; break; }
             Stage &st = sm.st[s];
             const TileCoord tcd = tile_coord(tile, R, n_k);
             const int32_t *P = perm + tcd.seg * L;
             const long long rowbase = tcd.bh * L;
             const int slot0 = tcd.k * kK - 64;
-            for (int e = lane; e < 256; e += 32) {
+            // positions of slots [128k - 64, 128k + 192): two per thread, loads clamped in range
+            for (int e = ptid; e < 256; e += kProducerThreads) {
                 const int sl = slot0 + e;
-                st.pos[e] = (sl >= 0 && sl < L) ? P[sl] : -1;
+                const int pl = P[min(max(sl, 0), L - 1)];
+                st.pos[e] = (sl >= 0 && sl < L) ? pl : -1;
             }
-            if (lane == 0) tc::mbar_expect_tx(&sm.full[s], kStageBytes);
-            __syncwarp();
-            // TMA gathers, four rows per instruction, spread over the lanes
-            // (row index -1 = missing slot -> zero fill)
-            for (int gi = lane; gi < kQ / 4; gi += 32) {
-                int rr[4];
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const int p = st.pos[64 + 4 * gi + u];
-                    rr[u] = p >= 0 ? (int)(rowbase + p) : -1;
-                }
-                tc::tma_gather4(st.X + gi * 512, &tm_x, rr[0], rr[1], rr[2], rr[3], &sm.full[s]);
-                tc::tma_gather4(st.G + gi * 512, &tm_g, rr[0], rr[1], rr[2], rr[3], &sm.full[s]);
-                if (gi < kK / 4) tc::tma_gather4(st.V + gi * 512, &tm_v, rr[0], rr[1], rr[2], rr[3], &sm.full[s]);
+            tc::named_bar_sync(1, kProducerThreads);
+            // x, dY rows of the 192 query slots and v rows of the 128 key slots
+            for (int c = ptid; c < (2 * kQ + kK) * 8; c += kProducerThreads) {
+                const int t = c < kQ * 8 ? 0 : (c < 2 * kQ * 8 ? 1 : 2);
+                const int idx = c - (t == 0 ? 0 : t == 1 ? kQ * 8 : 2 * kQ * 8);
+                const int row = idx >> 3, ch = idx & 7;
+                const uint32_t off = (uint32_t)row * 128u + (uint32_t)((ch ^ (row & 7)) << 4);
+                uint8_t *dst = (t == 0 ? st.X : t == 1 ? st.G : st.V) + off;
+                const __nv_bfloat16 *srcb = t == 0 ? x : t == 1 ? dout : v;
+                const int p = st.pos[64 + row];
+                if (p >= 0) tc::cp_async16(dst, srcb + (rowbase + p) * kDim + ch * 8);
+                else *reinterpret_cast<uint4 *>(dst) = make_uint4(0, 0, 0, 0);
             }
-            // window minima of positions for the self flags (chunks 2k-1 .. 2k+2)
-            int cmin[4];
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                int mn = INT_MAX;
-                for (int e = lane; e < 64; e += 32) {
-                    const int p = st.pos[c * 64 + e];
-                    if (p >= 0) mn = min(mn, p);
-                }
+            tc::cp_async_commit();
+            // smallest position of chunks 2k-1 .. 2k+2 (one warp each)
+            {
+                const int a0 = st.pos[pw * 64 + lane], a1 = st.pos[pw * 64 + 32 + lane];
+                int mn = min(a0 >= 0 ? a0 : INT_MAX, a1 >= 0 ? a1 : INT_MAX);
 #pragma unroll
                 for (int o = 16; o > 0; o >>= 1) mn = min(mn, __shfl_xor_sync(0xffffffffu, mn, o));
-                cmin[c] = mn;
+                if (lane == 0) st.cmin[pw] = mn;
             }
-            // per-query LSE / delta and per-key norms: all loads issued before any is used
-            {
-                int qp[kQ / 32];
-                float ql[kQ / 32], qd[kQ / 32], kn[kK / 32];
-#pragma unroll
-                for (int j = 0; j < kQ / 32; ++j) qp[j] = st.pos[64 + lane + 32 * j];
-#pragma unroll
-                for (int j = 0; j < kQ / 32; ++j) {
-                    const bool ok = qp[j] >= 0;
-                    ql[j] = ok ? lse_all[rowbase + qp[j]] : 0.f;
-                    qd[j] = ok ? delta[rowbase + qp[j]] : 0.f;
-                    if (j < kK / 32) kn[j] = ok ? invnorm[rowbase + qp[j]] : 0.f;
-                }
-#pragma unroll
-                for (int j = 0; j < kQ / 32; ++j) {
-                    const int q = lane + 32 * j;
-                    const int p = qp[j];
-                    const int qa = q >> 6;
-                    const int wmin = min(cmin[qa], cmin[qa + 1]);
-                    float4 qi;
-                    qi.x = p >= 0 ? ql[j] * kLog2e : INFINITY;
-                    qi.y = qd[j];
-                    qi.z = (p >= 0 && causal && p == wmin) ? 1.f : 0.f;
-                    qi.w = __int_as_float(p);
-                    st.qinfo[q] = qi;
-                    if (j < kK / 32) st.kinv[q] = kn[j];
-                }
+            tc::named_bar_sync(1, kProducerThreads);
+            // per-query LSE, delta, self flag; per-key norm (loads clamped in range, then selected)
+            for (int q = ptid; q < kQ; q += kProducerThreads) {
+                const int p = st.pos[64 + q];
+                const long long rp = rowbase + max(p, 0);
+                const float lv = lse_all[rp], dv = delta[rp], nv = invnorm[rp];
+                const int qa = q >> 6;
+                const int wmin = min(st.cmin[qa], st.cmin[qa + 1]);
+                float4 qi;
+                qi.x = p >= 0 ? lv * kLog2e : INFINITY;
+                qi.y = p >= 0 ? dv : 0.f;
+                qi.z = (p >= 0 && causal && p == wmin) ? 1.f : 0.f;
+                qi.w = __int_as_float(p);
+                st.qinfo[q] = qi;
+                if (q < kK) st.kinv[q] = p >= 0 ? nv : 0.f;
             }
-            if (lane == 0) st.tile = tile;
-            __threadfence_block();
-            __syncwarp();
-            if (lane == 0) tc::mbar_arrive(&sm.full[s]);
+            if (prev_s >= 0) {
+                tc::cp_async_wait<1>();
+                tc::fence_async_smem();
+                tc::mbar_arrive(&sm.full[prev_s]);
+            }
+            prev_s = s;
         }
-    } else if (warp == kComputeWarps + 1) {
+        if (prev_s >= 0) {
+            tc::cp_async_wait<0>();
+            tc::fence_async_smem();
+            tc::mbar_arrive(&sm.full[prev_s]);
+        }
+    } else if (warp == kMmaWarp) {
         // ================= MMA issuer
         if (lane == 0) {
             constexpr uint32_t id_s = tc::idesc_bf16(128, kQ, 0, 0);
@@ -390,14 +377,23 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_consta
 #pragma unroll
                 for (int c = 0; c < 4; ++c) tc::tmem_ld16(tl + cG + c * 16, a + c * 16);
                 tc::tmem_ld_wait();
-                float xr[kDim];
-                smem_row(st.X, kr, xr);
+                // key-role correction g - inv^2 (g . x) x, reading x_k from shared memory twice
                 float gx = 0.f;
 #pragma unroll
-                for (int d = 0; d < kDim; ++d) gx = fmaf(a[d], xr[d], gx);
+                for (int ch = 0; ch < 8; ++ch) {
+                    float xr[8];
+                    smem_chunk(st.X, kr, ch, xr);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) gx = fmaf(a[ch * 8 + e], xr[e], gx);
+                }
                 const float cf = kinv * kinv * gx;
 #pragma unroll
-                for (int d = 0; d < kDim; ++d) a[d] = fmaf(-cf, xr[d], a[d]);
+                for (int ch = 0; ch < 8; ++ch) {
+                    float xr[8];
+                    smem_chunk(st.X, kr, ch, xr);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) a[ch * 8 + e] = fmaf(-cf, xr[e], a[ch * 8 + e]);
+                }
                 red_row(dx_acc + (rowbase + kpos) * kDim, a);           // key role of key kr
                 if (quad >= 2) {                                         // query row 64 + kr (chunk 2k+2)
 #pragma unroll
@@ -430,11 +426,6 @@ cudaError_t launch_attn_bwd_tc(const Problem &p, const void *x, const void *v, c
                                const float *invnorm, const float *lse_all, const float *delta, float *dx_acc,
                                float *dv_acc, uint32_t *status, cudaStream_t st)
 {
-    CUtensorMap tx, tv, tg;
-    const long long rows = p.tokens();
-    if (rows >= (1LL << 31)) return cudaErrorInvalidValue;
-    if (!tc::make_row_tmap(&tx, x, rows) || !tc::make_row_tmap(&tv, v, rows) || !tc::make_row_tmap(&tg, dout, rows))
-        return cudaErrorInvalidValue;
     const size_t smem = sizeof(BwdSmem) + 1024;
     cudaError_t e = cudaFuncSetAttribute(attn_bwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
@@ -443,7 +434,8 @@ cudaError_t launch_attn_bwd_tc(const Problem &p, const void *x, const void *v, c
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const long long n_tiles = p.S() * (p.L / kK);
     const unsigned grid = (unsigned)std::min<long long>(n_tiles, (long long)sms);
-    attn_bwd_tc_kernel<<<grid, kThreads, smem, st>>>(tx, tv, tg, (const __nv_bfloat16 *)x, perm, invnorm, lse_all,
+    attn_bwd_tc_kernel<<<grid, kThreads, smem, st>>>((const __nv_bfloat16 *)x, (const __nv_bfloat16 *)v,
+                                                     (const __nv_bfloat16 *)dout, perm, invnorm, lse_all,
                                                      delta, dx_acc, dv_acc, p.L, p.R, n_tiles, p.causal,
                                                      1.0f / sqrtf((float)p.d), status);
     return cudaGetLastError();

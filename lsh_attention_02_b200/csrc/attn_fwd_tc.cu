@@ -9,9 +9,9 @@
 // so one gathered tile serves as both MMA operands.
 //
 // Per tile:
-//   gather   rows x[perm[s]] and v[perm[s]] of the 192 window slots by TMA
-//            (tile::gather4, four rows per instruction) straight into the
-//            128-byte-swizzled layout the tensor core reads;
+//   gather   rows x[perm[s]] and v[perm[s]] of the 192 window slots, copied
+//            with cp.async straight into the 128-byte-swizzled layout the
+//            tensor core reads;
 //   S = Q K^T  tcgen05.mma M=128, N=192, K=64 into tensor memory (raw
 //            dot products x_i . x_j, bf16 in, fp32 accumulate);
 //   softmax  one query row per thread: s_ij = (x_i . x_j) / |x_j| / sqrt(d)
@@ -34,9 +34,11 @@
 //   warps 0-3, 4-7  two softmax groups working on alternate tiles, each with
 //                   its own 256 TMEM columns (S/P 192, O 64), so one group's
 //                   softmax overlaps the other's MMAs and stores;
-//   warp 8          producer: positions, key norms and window minima, then TMA
-//                   row gathers, into a 3-stage shared-memory ring;
-//   warp 9          MMA issuer.
+//   warps 8-11      producer: positions, key norms and window minima, then
+//                   16-byte cp.async gathers (a warp instruction moves four
+//                   whole rows) into a 3-stage shared-memory ring; a stage is
+//                   released once the next stage's copies are in flight;
+//   warp 12         MMA issuer.
 #include "tc_common.cuh"
 
 namespace lsh {
@@ -46,13 +48,16 @@ namespace {
 constexpr int kQ = 128;             // query slots per tile
 constexpr int kW = 192;             // window rows (keys)
 constexpr int kStages = 3;
-constexpr int kThreads = 320;
+constexpr int kSoftmaxWarps = 8;   // two groups of four
+constexpr int kProducerWarps = 4;
+constexpr int kProducerThreads = kProducerWarps * 32;
+constexpr int kMmaWarp = kSoftmaxWarps + kProducerWarps;
+constexpr int kThreads = (kMmaWarp + 1) * 32;
 constexpr int kTmemCols = 512;
 constexpr uint32_t kGroupCols = 256;
 constexpr uint32_t kOCol = 192;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
-constexpr uint32_t kStageBytes = 2 * kW * 128;
 
 struct alignas(1024) Stage {
     uint8_t X[kW * 128];            // gathered x rows, K-major SW128 (24 KB)
@@ -90,9 +95,9 @@ __device__ __forceinline__ TileCoord tile_coord(long long tile, int R, int n_k)
 // Softmax of one query row (thread) over window columns [BASE, BASE + 128)
 // (chunk 2k: BASE = 0, chunk 2k+1: BASE = 64); `jlo` skips the missing chunk
 // -1 of a segment's first tile.  P is written as packed bf16 pairs into the
-// row's own S columns (key j -> column j/2), in place: chunk c of 16 scores is
-// read before packed columns BASE/2 + [8c, 8c+8) are written, and those never
-// reach an unread chunk.  Columns outside the row's window get zeros.
+// row's own S columns (key j -> column j/2), in place: each half of 64 scores
+// is read before packed columns BASE/2 + [32h, 32h + 32) are written, and
+// those never reach an unread half.  Columns outside the row's window get zeros.
 template <int BASE>
 __device__ __forceinline__ void softmax_row(const Stage &st, uint32_t tl, int jlo, int qpos, float qinv, int self_only,
                                             int causal, float tau, float &l, float &row_lse)
@@ -120,31 +125,36 @@ __device__ __forceinline__ void softmax_row(const Stage &st, uint32_t tl, int jl
     }
     float lsum = 0.f;
 #pragma unroll 1
-    for (int c = 0; c < 8; ++c) {
-        float v[16];
-        tc::tmem_ld16(tl + (uint32_t)(BASE + c * 16), v);
+    for (int h = 0; h < 2; ++h) {
+        float v[64];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tc::tmem_ld16(tl + (uint32_t)(BASE + h * 64 + c * 16), v + c * 16);
         tc::tmem_ld_wait();
-        uint32_t w[8];
 #pragma unroll
-        for (int e4 = 0; e4 < 16; e4 += 4) {
-            const int4 kp = *reinterpret_cast<const int4 *>(&st.pos[BASE + c * 16 + e4]);
-            const float4 ks = *reinterpret_cast<const float4 *>(&st.sinv[BASE + c * 16 + e4]);
-            const int kpa[4] = {kp.x, kp.y, kp.z, kp.w};
-            const float ksa[4] = {ks.x, ks.y, ks.z, ks.w};
-            float pe[4];
+        for (int c = 0; c < 4; ++c) {
+            uint32_t w[8];
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int j = c * 16 + e4 + e;
-                const int ok =
-                    ((j >= jlo) & (causal ? (kpa[e] < qpos) : (kpa[e] != qpos))) | (self_only & (kpa[e] == qpos));
-                const float p = tc::fast_exp2(fmaf(v[e4 + e], ksa[e], -shift2));
-                pe[e] = ok ? p : 0.f;
-                lsum += pe[e];
+            for (int e4 = 0; e4 < 16; e4 += 4) {
+                const int j0 = h * 64 + c * 16 + e4;
+                const int4 kp = *reinterpret_cast<const int4 *>(&st.pos[BASE + j0]);
+                const float4 ks = *reinterpret_cast<const float4 *>(&st.sinv[BASE + j0]);
+                const int kpa[4] = {kp.x, kp.y, kp.z, kp.w};
+                const float ksa[4] = {ks.x, ks.y, ks.z, ks.w};
+                float pe[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int j = j0 + e;
+                    const int ok = ((j >= jlo) & (causal ? (kpa[e] < qpos) : (kpa[e] != qpos))) |
+                                   (self_only & (kpa[e] == qpos));
+                    const float p = tc::fast_exp2(fmaf(v[c * 16 + e4 + e], ksa[e], -shift2));
+                    pe[e] = ok ? p : 0.f;
+                    lsum += pe[e];
+                }
+                w[e4 / 2] = pack_bf16x2(pe[0], pe[1]);
+                w[e4 / 2 + 1] = pack_bf16x2(pe[2], pe[3]);
             }
-            w[e4 / 2] = pack_bf16x2(pe[0], pe[1]);
-            w[e4 / 2 + 1] = pack_bf16x2(pe[2], pe[3]);
+            tc::tmem_st8(tl + (uint32_t)(BASE / 2 + h * 32 + c * 8), w);
         }
-        tc::tmem_st8(tl + (uint32_t)(BASE / 2 + c * 8), w);
     }
     // zeros for the keys outside this row's window (packed columns of keys 128..191 or 0..63)
     {
@@ -158,7 +168,7 @@ __device__ __forceinline__ void softmax_row(const Stage &st, uint32_t tl, int jl
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
-attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_v,
+attn_fwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__restrict__ v,
                    const int32_t *__restrict__ perm, const float *__restrict__ invnorm,
                    __nv_bfloat16 *__restrict__ o_r, float *__restrict__ lse, int L, int R, long long n_tiles,
                    int causal, float tau, uint32_t *__restrict__ status)
@@ -170,7 +180,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_consta
 
     if (tid == 0) {
         for (int s = 0; s < kStages; ++s) {
-            tc::mbar_init(&sm.full[s], 1);
+            tc::mbar_init(&sm.full[s], kProducerThreads);
             tc::mbar_init(&sm.empty[s], 4);
         }
         for (int g = 0; g < 2; ++g) {
@@ -189,63 +199,65 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_consta
     const uint32_t tmem = sm.tmem_base;
     const float sl2 = tau * kLog2e;
 
-    if (warp == 8) {
-        // ================= producer
-        if (lane == 0) {
-            tc::prefetch_tmap(&tm_x);
-            tc::prefetch_tmap(&tm_v);
-        }
+    if (warp >= kSoftmaxWarps && warp < kMmaWarp) {
+        // ================= producer group
+        const int ptid = tid - kSoftmaxWarps * 32, pw = ptid >> 5;
+        int prev_s = -1;
         int it = 0;
         for (long long tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++it) {
             const int s = it % kStages;
-            if (it >= kStages &&
-                !tc::mbar_wait(&sm.empty[s], (uint32_t)((it / kStages) - 1) & 1u, &sm.abort, status))
-                break;
+            bool ok = it < kStages ||
+                      tc::mbar_wait(&sm.empty[s], (uint32_t)((it / kStages) - 1) & 1u, &sm.abort, status);
+            if (tc::named_bar_or(1, kProducerThreads, !ok)) { prev_s = -1; break; }
             Stage &st = sm.st[s];
             const TileCoord tcd = tile_coord(tile, R, n_k);
             const int32_t *P = perm + tcd.seg * L;
             const long long rowbase = tcd.bh * L;
             const int slot0 = tcd.k * kQ - 64;
-            int pj[kW / 32];
-#pragma unroll
-            for (int j = 0; j < kW / 32; ++j) {
-                const int sl = slot0 + lane + 32 * j;
-                pj[j] = sl >= 0 ? P[sl] : -1;
-                st.pos[lane + 32 * j] = pj[j];
+            for (int e = ptid; e < kW; e += kProducerThreads) {
+                const int sl = slot0 + e;                      // <= L - 1 always
+                const int pl = P[max(sl, 0)];
+                const int p = sl >= 0 ? pl : -1;
+                const float nv = invnorm[rowbase + max(p, 0)];
+                st.pos[e] = p;
+                st.inv[e] = p >= 0 ? nv : 0.f;
+                st.sinv[e] = p >= 0 ? nv * sl2 : 0.f;
             }
-            if (lane == 0) tc::mbar_expect_tx(&sm.full[s], kStageBytes);
-            __syncwarp();
-            for (int gi = lane; gi < kW / 4; gi += 32) {
-                int rr[4];
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const int p = st.pos[4 * gi + u];
-                    rr[u] = p >= 0 ? (int)(rowbase + p) : -1;
-                }
-                tc::tma_gather4(st.X + gi * 512, &tm_x, rr[0], rr[1], rr[2], rr[3], &sm.full[s]);
-                tc::tma_gather4(st.V + gi * 512, &tm_v, rr[0], rr[1], rr[2], rr[3], &sm.full[s]);
-            }
-            float nv[kW / 32];
-#pragma unroll
-            for (int j = 0; j < kW / 32; ++j) nv[j] = pj[j] >= 0 ? invnorm[rowbase + pj[j]] : 0.f;
-#pragma unroll
-            for (int j = 0; j < kW / 32; ++j) {
-                st.inv[lane + 32 * j] = nv[j];
-                st.sinv[lane + 32 * j] = nv[j] * sl2;
-            }
-            // smallest position of each window chunk: window chunk c holds lanes' j = 2c, 2c + 1
-#pragma unroll
-            for (int c = 0; c < 3; ++c) {
-                int mn = min(pj[2 * c] >= 0 ? pj[2 * c] : INT_MAX, pj[2 * c + 1] >= 0 ? pj[2 * c + 1] : INT_MAX);
+            tc::named_bar_sync(1, kProducerThreads);
+            if (pw < 3) {
+                // smallest position of window chunk pw (INT_MAX when the chunk is missing)
+                const int a0 = st.pos[pw * 64 + lane], a1 = st.pos[pw * 64 + 32 + lane];
+                int mn = min(a0 >= 0 ? a0 : INT_MAX, a1 >= 0 ? a1 : INT_MAX);
 #pragma unroll
                 for (int o = 16; o > 0; o >>= 1) mn = min(mn, __shfl_xor_sync(0xffffffffu, mn, o));
-                if (lane == 0) st.cmin[c] = mn;
+                if (lane == 0) st.cmin[pw] = mn;
             }
-            __threadfence_block();
-            __syncwarp();
-            if (lane == 0) tc::mbar_arrive(&sm.full[s]);
+            // x and v rows: thread -> one 16-byte chunk, eight consecutive threads -> one row
+            for (int c = ptid; c < 2 * kW * 8; c += kProducerThreads) {
+                const int t = c >= kW * 8;
+                const int idx = c - t * kW * 8;
+                const int row = idx >> 3, ch = idx & 7;
+                const uint32_t off = (uint32_t)row * 128u + (uint32_t)((ch ^ (row & 7)) << 4);
+                uint8_t *dst = (t ? st.V : st.X) + off;
+                const int p = st.pos[row];
+                if (p >= 0) tc::cp_async16(dst, (t ? v : x) + (rowbase + p) * kDim + ch * 8);
+                else *reinterpret_cast<uint4 *>(dst) = make_uint4(0, 0, 0, 0);
+            }
+            tc::cp_async_commit();
+            if (prev_s >= 0) {
+                // the previous stage's copies have landed: publish it
+                tc::cp_async_wait<1>();
+                tc::fence_async_smem();
+                tc::mbar_arrive(&sm.full[prev_s]);
+            }
+            prev_s = s;
         }
-    } else if (warp == 9) {
+        if (prev_s >= 0) {
+            tc::cp_async_wait<0>();
+            tc::fence_async_smem();
+            tc::mbar_arrive(&sm.full[prev_s]);
+        }
+    } else if (warp == kMmaWarp) {
         // ================= MMA issuer: S of tile t+1 is issued before O of tile t
         if (lane == 0) {
             constexpr uint32_t id_s = tc::idesc_bf16(128, kW, 0, 0);
@@ -352,8 +364,6 @@ cudaError_t launch_attn_fwd_tc(const Problem &p, const void *x, const void *v, c
                                const float *invnorm, __nv_bfloat16 *o_r, float *lse, uint32_t *status,
                                cudaStream_t st)
 {
-    CUtensorMap tx, tv;
-    if (!tc::make_row_tmap(&tx, x, p.tokens()) || !tc::make_row_tmap(&tv, v, p.tokens())) return cudaErrorInvalidValue;
     const size_t smem = sizeof(FwdSmem) + 1024;
     cudaError_t e = cudaFuncSetAttribute(attn_fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
@@ -362,7 +372,7 @@ cudaError_t launch_attn_fwd_tc(const Problem &p, const void *x, const void *v, c
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const long long n_tiles = p.S() * (p.L / kQ);
     const unsigned grid = (unsigned)std::min<long long>(n_tiles, (long long)sms);
-    attn_fwd_tc_kernel<<<grid, kThreads, smem, st>>>(tx, tv, perm, invnorm, o_r, lse, p.L, p.R, n_tiles, p.causal,
+    attn_fwd_tc_kernel<<<grid, kThreads, smem, st>>>((const __nv_bfloat16 *)x, (const __nv_bfloat16 *)v, perm, invnorm, o_r, lse, p.L, p.R, n_tiles, p.causal,
                                                      1.0f / sqrtf((float)p.d), status);
     return cudaGetLastError();
 }
