@@ -32,18 +32,20 @@ def _stale() -> bool:
     return any(os.path.getmtime(p) > t for p in deps)
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    if not force and not _stale():
+def build(force: bool = False, verbose: bool = False, phase_trace: bool = False) -> str:
+    """Compiles the library; phase_trace=True builds liblsh_attn_trace.so with the
+    per-phase timestamp points compiled in (a tuning build, never the default)."""
+    lib = LIB.replace(".so", "_trace.so") if phase_trace else LIB
+    if not force and not phase_trace and not _stale():
         return LIB
-    tmp = LIB + f".tmp{os.getpid()}"
-    cmd = [nvcc(), *ARCH, *FLAGS, "-o", tmp, *sources()]
+    tmp = lib + f".tmp{os.getpid()}"
+    cmd = [nvcc(), *ARCH, *FLAGS, *(["-DLSH_PHASE_TRACE"] if phase_trace else []), "-o", tmp, *sources()]
     if verbose:
         print(" ".join(cmd), file=sys.stderr)
     subprocess.check_call(cmd)
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":
-    build(force="--force" in sys.argv, verbose=True)
-    print(LIB)
+    print(build(force="--force" in sys.argv, verbose=True, phase_trace="--phase-trace" in sys.argv))

@@ -158,7 +158,9 @@ static lsh_status run_hash_sort(const Problem &p, const Choice &c, const void *q
 static lsh_status run_attn_fwd(const Problem &p, const Choice &c, const void *qk, const void *v,
                                const int32_t *perm, void *out, float *lse, const Workspace &w, cudaStream_t st)
 {
-    LSH_TRY(staged(LSH_STAGE_NORMS, 1, st, [&] { return launch_invnorm(p, qk, w.invnorm, st); }), "key norms");
+    // the tensor-core forward computes the key norms from its gathered rows
+    if (!c.tc_attn)
+        LSH_TRY(staged(LSH_STAGE_NORMS, 1, st, [&] { return launch_invnorm(p, qk, w.invnorm, st); }), "key norms");
     LSH_TRY(staged(LSH_STAGE_ATTN_FWD, 1, st, [&] {
                 return c.tc_attn
                            ? launch_attn_fwd_tc(p, qk, v, perm, w.invnorm, (__nv_bfloat16 *)w.o_r, lse, w.status, st)
@@ -403,3 +405,4 @@ bool make_row_tmap(CUtensorMap *map, const void *base, long long rows)
 
 }  // namespace tc
 }  // namespace lsh
+

@@ -34,8 +34,7 @@
 //   warps 8-11 producer: positions, per-query LSE / delta / self flags and
 //              per-key norms into a 2-stage ring, then 16-byte cp.async
 //              gathers of the x, v and dY rows straight into the swizzled
-//              operand layout; a stage is published once the next stage's
-//              copies are in flight;
+//              operand layout;
 //   warp 12    MMA issuer.
 #include "tc_common.cuh"
 
@@ -213,13 +212,14 @@ attn_bwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
     if (warp >= kComputeWarps && warp < kMmaWarp) {
         // ================= producer group
         const int ptid = tid - kComputeWarps * 32, pw = ptid >> 5;
-        int prev_s = -1;
         int it = 0;
         for (long long tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++it) {
             const int s = it % kStages;
+            if (ptid == 0) LSH_PHASE(1, 0, it, 0);
             bool ok = it < kStages ||
                       tc::mbar_wait(&sm.empty[s], (uint32_t)((it / kStages) - 1) & 1u, &sm.abort, status);
-            if (tc::named_bar_or(1, kProducerThreads, !ok)) { prev_s = -1; break; }
+            if (tc::named_bar_or(1, kProducerThreads, !ok)) break;
+            if (ptid == 0) LSH_PHASE(1, 0, it, 1);
             Stage &st = sm.st[s];
             const TileCoord tcd = tile_coord(tile, R, n_k);
             const int32_t *P = perm + tcd.seg * L;
@@ -245,6 +245,7 @@ attn_bwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
                 else *reinterpret_cast<uint4 *>(dst) = make_uint4(0, 0, 0, 0);
             }
             tc::cp_async_commit();
+            if (ptid == 0) LSH_PHASE(1, 0, it, 2);
             // smallest position of chunks 2k-1 .. 2k+2 (one warp each)
             {
                 const int a0 = st.pos[pw * 64 + lane], a1 = st.pos[pw * 64 + 32 + lane];
@@ -269,17 +270,12 @@ attn_bwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
                 st.qinfo[q] = qi;
                 if (q < kK) st.kinv[q] = p >= 0 ? nv : 0.f;
             }
-            if (prev_s >= 0) {
-                tc::cp_async_wait<1>();
-                tc::fence_async_smem();
-                tc::mbar_arrive(&sm.full[prev_s]);
-            }
-            prev_s = s;
-        }
-        if (prev_s >= 0) {
+            if (ptid == 0) LSH_PHASE(1, 0, it, 3);
+            // with two stages the producer cannot run further ahead: publish this stage now
             tc::cp_async_wait<0>();
             tc::fence_async_smem();
-            tc::mbar_arrive(&sm.full[prev_s]);
+            tc::mbar_arrive(&sm.full[s]);
+            if (ptid == 0) LSH_PHASE(1, 0, it, 4);
         }
     } else if (warp == kMmaWarp) {
         // ================= MMA issuer
@@ -292,8 +288,11 @@ attn_bwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
             for (long long tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++it) {
                 const int s = it % kStages;
                 const uint32_t ph = (uint32_t)it & 1u;
+                LSH_PHASE(1, 1, it, 0);
                 if (!tc::mbar_wait(&sm.full[s], (uint32_t)(it / kStages) & 1u, &sm.abort, status)) break;
+                LSH_PHASE(1, 1, it, 1);
                 if (it > 0 && !tc::mbar_wait(&sm.bar_free, ph ^ 1u, &sm.abort, status)) break;
+                LSH_PHASE(1, 1, it, 2);
                 tc::tc_fence_after();
                 const Stage &st = sm.st[s];
                 const uint32_t xs = tc::smem_u32(st.X), vs = tc::smem_u32(st.V), gs = tc::smem_u32(st.G);
@@ -304,6 +303,7 @@ attn_bwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
                 }
                 tc::mma_commit(&sm.bar_s);
                 if (!tc::mbar_wait(&sm.bar_p, ph, &sm.abort, status)) break;
+                LSH_PHASE(1, 1, it, 3);
                 tc::tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < 12; ++kk) {
@@ -320,6 +320,7 @@ attn_bwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
                                  id_q, kk > 0);
                 }
                 tc::mma_commit(&sm.bar_o);
+                LSH_PHASE(1, 1, it, 4);
             }
         }
     } else {
@@ -331,13 +332,16 @@ attn_bwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
         for (long long tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++it) {
             const int s = it % kStages;
             const uint32_t ph = (uint32_t)it & 1u;
+            if (tid == 0) LSH_PHASE(1, 2, it, 0);
             if (!tc::mbar_wait(&sm.full[s], (uint32_t)(it / kStages) & 1u, &sm.abort, status)) break;
+            if (tid == 0) LSH_PHASE(1, 2, it, 1);
             const Stage &st = sm.st[s];
             const TileCoord tcd = tile_coord(tile, R, n_k);
             const long long rowbase = tcd.bh * L;
             const int kpos = st.pos[64 + kr];
             const float kinv = st.kinv[kr];
             if (!tc::mbar_wait(&sm.bar_s, ph, &sm.abort, status)) break;
+            if (tid == 0) LSH_PHASE(1, 2, it, 2);
             tc::tc_fence_after();
             // ---- elementwise
             if (quad < 2) {                          // keys of chunk 2k: queries of chunks 2k, 2k+1
@@ -360,7 +364,9 @@ attn_bwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
             tc::tc_fence_before();
             __syncwarp();
             if (lane == 0) tc::mbar_arrive(&sm.bar_p);
+            if (tid == 0) LSH_PHASE(1, 2, it, 3);
             if (!tc::mbar_wait(&sm.bar_o, ph, &sm.abort, status)) break;
+            if (tid == 0) LSH_PHASE(1, 2, it, 4);
             tc::tc_fence_after();
             // ---- epilogue: reductions into the fp32 accumulators
             float a[kDim];
@@ -403,6 +409,7 @@ attn_bwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
                     if (qp >= 0) red_row(dx_acc + (rowbase + qp) * kDim, a);
                 }
             }
+            if (tid == 0) LSH_PHASE(1, 2, it, 5);
             tc::tc_fence_before();
             __syncwarp();
             if (lane == 0) {
@@ -442,3 +449,5 @@ cudaError_t launch_attn_bwd_tc(const Problem &p, const void *x, const void *v, c
 }
 
 }  // namespace lsh
+
+LSH_PHASE_EXPORT(bwd)

@@ -10,8 +10,8 @@
 //
 // Per tile:
 //   gather   rows x[perm[s]] and v[perm[s]] of the 192 window slots, copied
-//            with cp.async straight into the 128-byte-swizzled layout the
-//            tensor core reads;
+//            straight into the 128-byte-swizzled layout the tensor core reads;
+//   norms    1/|x_j| of the window rows, from the gathered tile;
 //   S = Q K^T  tcgen05.mma M=128, N=192, K=64 into tensor memory (raw
 //            dot products x_i . x_j, bf16 in, fp32 accumulate);
 //   softmax  one query row per thread: s_ij = (x_i . x_j) / |x_j| / sqrt(d)
@@ -34,10 +34,12 @@
 //   warps 0-3, 4-7  two softmax groups working on alternate tiles, each with
 //                   its own 256 TMEM columns (S/P 192, O 64), so one group's
 //                   softmax overlaps the other's MMAs and stores;
-//   warps 8-11      producer: positions, key norms and window minima, then
-//                   16-byte cp.async gathers (a warp instruction moves four
-//                   whole rows) into a 3-stage shared-memory ring; a stage is
-//                   released once the next stage's copies are in flight;
+//   warps 8-11      producer: positions (loaded a tile ahead) and window
+//                   minima; x rows by TMA (tile::gather4, four rows per
+//                   instruction) and v rows by 16-byte cp.async, so both copy
+//                   engines work at once, into a 3-stage shared-memory ring; a
+//                   stage is published once the next stage's copies are in
+//                   flight;
 //   warp 12         MMA issuer.
 #include "tc_common.cuh"
 
@@ -93,39 +95,28 @@ __device__ __forceinline__ TileCoord tile_coord(long long tile, int R, int n_k)
 }
 
 // Softmax of one query row (thread) over window columns [BASE, BASE + 128)
-// (chunk 2k: BASE = 0, chunk 2k+1: BASE = 64); `jlo` skips the missing chunk
-// -1 of a segment's first tile.  P is written as packed bf16 pairs into the
-// row's own S columns (key j -> column j/2), in place: each half of 64 scores
-// is read before packed columns BASE/2 + [32h, 32h + 32) are written, and
-// those never reach an unread half.  Columns outside the row's window get zeros.
-template <int BASE>
-__device__ __forceinline__ void softmax_row(const Stage &st, uint32_t tl, int jlo, int qpos, float qinv, int self_only,
-                                            int causal, float tau, float &l, float &row_lse)
+// (chunk 2k: BASE = 0, chunk 2k+1: BASE = 64).  FIRST: the segment's first
+// tile, whose chunk -1 (window columns 0..63) does not exist.  P is written as
+// packed bf16 pairs into the row's own S columns (key j -> column j/2), in
+// place: each half of 64 scores is read before packed columns
+// BASE/2 + [32h, 32h + 32) are written, and those never reach an unread half.
+// Columns outside the row's window get zeros.  Returns l = sum of p.
+//
+// Candidates: keys at an earlier original position (causal) or at any other
+// position (non-causal).  A causal row with none (its position is the
+// smallest of its window) gets l = 0 here and is patched by the caller.
+template <int BASE, bool CAUSAL, bool FIRST>
+__device__ __forceinline__ float softmax_sweep(const Stage &st, uint32_t tl, int qpos, float shift2)
 {
-    const float bound = qinv > 0.f ? tau / qinv : 0.f;        // tau |x_i| >= every score of the row
-    float shift2 = bound * kLog2e;                              // log2-domain offset
-    // exp(s - bound) stays normal unless bound - s, <= 2 bound, exceeds ~100 in log2 units
-    const bool wide = 2.f * bound * kLog2e > 100.f;
-    if (__any_sync(0xffffffffu, wide)) {
-        float mx = -INFINITY;
-#pragma unroll 1
-        for (int c = 0; c < 8; ++c) {
-            float v[16];
-            tc::tmem_ld16(tl + (uint32_t)(BASE + c * 16), v);
-            tc::tmem_ld_wait();
-#pragma unroll
-            for (int e = 0; e < 16; ++e) {
-                const int j = c * 16 + e;
-                const int kp = st.pos[BASE + j];
-                const int ok = ((j >= jlo) & (causal ? (kp < qpos) : (kp != qpos))) | (self_only & (kp == qpos));
-                mx = ok ? fmaxf(mx, v[e] * st.sinv[BASE + j]) : mx;
-            }
-        }
-        if (wide && mx > -INFINITY) shift2 = mx;
-    }
     float lsum = 0.f;
 #pragma unroll 1
     for (int h = 0; h < 2; ++h) {
+        if (FIRST && BASE == 0 && h == 0) {                     // missing chunk -1
+            const uint32_t z[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+#pragma unroll
+            for (int c = 0; c < 4; ++c) tc::tmem_st8(tl + (uint32_t)(c * 8), z);
+            continue;
+        }
         float v[64];
 #pragma unroll
         for (int c = 0; c < 4; ++c) tc::tmem_ld16(tl + (uint32_t)(BASE + h * 64 + c * 16), v + c * 16);
@@ -143,9 +134,7 @@ __device__ __forceinline__ void softmax_row(const Stage &st, uint32_t tl, int jl
                 float pe[4];
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                    const int j = j0 + e;
-                    const int ok = ((j >= jlo) & (causal ? (kpa[e] < qpos) : (kpa[e] != qpos))) |
-                                   (self_only & (kpa[e] == qpos));
+                    const bool ok = CAUSAL ? (kpa[e] < qpos) : (kpa[e] != qpos);
                     const float p = tc::fast_exp2(fmaf(v[c * 16 + e4 + e], ksa[e], -shift2));
                     pe[e] = ok ? p : 0.f;
                     lsum += pe[e];
@@ -156,22 +145,102 @@ __device__ __forceinline__ void softmax_row(const Stage &st, uint32_t tl, int jl
             tc::tmem_st8(tl + (uint32_t)(BASE / 2 + h * 32 + c * 8), w);
         }
     }
-    // zeros for the keys outside this row's window (packed columns of keys 128..191 or 0..63)
     {
         const uint32_t z[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-        constexpr uint32_t zc = BASE == 0 ? 64 : 0;
+        constexpr uint32_t zc = BASE == 0 ? 64 : 0;             // packed columns of keys 128..191 or 0..63
 #pragma unroll
         for (int c = 0; c < 4; ++c) tc::tmem_st8(tl + zc + c * 8, z);
     }
-    l = lsum;
-    row_lse = kLn2 * (shift2 + log2f(lsum));
+    return lsum;
+}
+
+// Exact row maximum of the log2-domain scores (only for rows whose bound
+// tau |x_i| is so loose that exp(s - bound) could leave the normal range).
+template <int BASE, bool CAUSAL>
+__device__ __forceinline__ float exact_max(const Stage &st, uint32_t tl, int jlo, int qpos)
+{
+    float mx = -INFINITY;
+#pragma unroll 1
+    for (int c = 0; c < 8; ++c) {
+        float v[16];
+        tc::tmem_ld16(tl + (uint32_t)(BASE + c * 16), v);
+        tc::tmem_ld_wait();
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+            const int j = c * 16 + e;
+            const int kp = st.pos[BASE + j];
+            const bool ok = (j >= jlo) && (CAUSAL ? (kp < qpos) : (kp != qpos));
+            mx = ok ? fmaxf(mx, v[e] * st.sinv[BASE + j]) : mx;
+        }
+    }
+    return mx;
+}
+
+template <int BASE, bool CAUSAL, bool FIRST>
+__device__ __forceinline__ void softmax_row(const Stage &st, uint32_t tl, int i, int qpos, float qinv, bool self_only,
+                                            float tau, float &l, float &row_lse)
+{
+    const float bound = qinv > 0.f ? tau / qinv : 0.f;        // tau |x_i| >= every score of the row
+    float shift2 = bound * kLog2e;                              // log2-domain offset
+    const bool wide = 2.f * bound * kLog2e > 100.f;             // bound - s <= 2 bound
+    if (__any_sync(0xffffffffu, wide)) {
+        const float mx = exact_max<BASE, CAUSAL>(st, tl, FIRST && BASE == 0 ? 64 : 0, qpos);
+        if (wide && mx > -INFINITY) shift2 = mx;
+    }
+    l = softmax_sweep<BASE, CAUSAL, FIRST>(st, tl, qpos, shift2);
+    row_lse = kLn2 * (shift2 + log2f(l));
+    if (CAUSAL && __any_sync(0xffffffffu, self_only)) {
+        // A row with no candidate attends to itself: p = 1 on its own key (window
+        // row 64 + i), lse = tau x_i . (x_i / |x_i|) = tau |x_i|.  The warp's 32 own
+        // keys occupy packed columns 32 + i/2 - (lane/2); each lane edits its own row.
+        const int lane = i & 31;
+        const uint32_t col0 = (uint32_t)((64 + (i - lane)) >> 1);
+        float w[16];
+        tc::tmem_st_wait();
+        tc::tmem_ld16(tl + col0, w);
+        tc::tmem_ld_wait();
+        uint32_t u[16];
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+            const uint32_t one = (lane & 1) ? 0x3F800000u : 0x00003F80u;
+            u[c] = (self_only && c == (lane >> 1)) ? one : __float_as_uint(w[c]);
+        }
+        tc::tmem_st16(tl + col0, u);
+        if (self_only) {
+            l = 1.f;
+            row_lse = bound;
+        }
+    }
+}
+
+// Key norms of the window rows from the gathered x tile: sinv = tau log2(e) / |x_j|
+// and inv = 1 / |x_j| (0 for a zero or missing row), sum of squares in element
+// order with fused multiply-adds, as the norms kernel does.
+__device__ __forceinline__ void window_norms(Stage &st, int t, float sl2)
+{
+    for (int row = t; row < kW; row += 128) {
+        float ssq = 0.f;
+#pragma unroll
+        for (int ch = 0; ch < 8; ++ch) {
+            const uint4 u = *reinterpret_cast<const uint4 *>(st.X + row * 128 + ((ch ^ (row & 7)) << 4));
+            const uint32_t wd[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float a = __uint_as_float(wd[e] << 16), b = __uint_as_float(wd[e] & 0xFFFF0000u);
+                ssq = fmaf(a, a, ssq);
+                ssq = fmaf(b, b, ssq);
+            }
+        }
+        const float nv = ssq > 0.f ? 1.0f / sqrtf(ssq) : 0.f;
+        st.inv[row] = nv;
+        st.sinv[row] = nv * sl2;
+    }
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
-attn_fwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__restrict__ v,
-                   const int32_t *__restrict__ perm, const float *__restrict__ invnorm,
-                   __nv_bfloat16 *__restrict__ o_r, float *__restrict__ lse, int L, int R, long long n_tiles,
-                   int causal, float tau, uint32_t *__restrict__ status)
+attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __nv_bfloat16 *__restrict__ v,
+                   const int32_t *__restrict__ perm, __nv_bfloat16 *__restrict__ o_r, float *__restrict__ lse, int L,
+                   int R, long long n_tiles, int causal, float tau, uint32_t *__restrict__ status)
 {
     extern __shared__ uint8_t smem_raw[];
     FwdSmem &sm = *reinterpret_cast<FwdSmem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -202,28 +271,62 @@ attn_fwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
     if (warp >= kSoftmaxWarps && warp < kMmaWarp) {
         // ================= producer group
         const int ptid = tid - kSoftmaxWarps * 32, pw = ptid >> 5;
+        if (ptid == 0) tc::prefetch_tmap(&tm_x);
+        // positions of the next tile, loaded a tile ahead (two slots per thread)
+        int pn[2] = {-1, -1};
+        auto load_pos = [&](long long tile) {
+            const TileCoord c = tile_coord(tile, R, n_k);
+            const int32_t *P = perm + c.seg * L;
+            const int slot0 = c.k * kQ - 64;
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                const int e = ptid + j * kProducerThreads;
+                const int sl = slot0 + min(e, kW - 1);         // <= L - 1
+                const int pl = P[max(sl, 0)];
+                pn[j] = (e < kW && sl >= 0) ? pl : -1;
+            }
+        };
+        if (blockIdx.x < n_tiles) load_pos(blockIdx.x);
         int prev_s = -1;
         int it = 0;
         for (long long tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++it) {
             const int s = it % kStages;
+            if (ptid == 0) LSH_PHASE(0, 0, it, 0);
             bool ok = it < kStages ||
                       tc::mbar_wait(&sm.empty[s], (uint32_t)((it / kStages) - 1) & 1u, &sm.abort, status);
             if (tc::named_bar_or(1, kProducerThreads, !ok)) { prev_s = -1; break; }
+            if (ptid == 0) LSH_PHASE(0, 0, it, 1);
             Stage &st = sm.st[s];
-            const TileCoord tcd = tile_coord(tile, R, n_k);
-            const int32_t *P = perm + tcd.seg * L;
-            const long long rowbase = tcd.bh * L;
-            const int slot0 = tcd.k * kQ - 64;
-            for (int e = ptid; e < kW; e += kProducerThreads) {
-                const int sl = slot0 + e;                      // <= L - 1 always
-                const int pl = P[max(sl, 0)];
-                const int p = sl >= 0 ? pl : -1;
-                const float nv = invnorm[rowbase + max(p, 0)];
-                st.pos[e] = p;
-                st.inv[e] = p >= 0 ? nv : 0.f;
-                st.sinv[e] = p >= 0 ? nv * sl2 : 0.f;
+            const long long rowbase = tile_coord(tile, R, n_k).bh * L;
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                const int e = ptid + j * kProducerThreads;
+                if (e < kW) st.pos[e] = pn[j];
             }
+            if (ptid == 0) tc::mbar_expect_tx(&sm.full[s], kW * 128);
             tc::named_bar_sync(1, kProducerThreads);
+            if (tile + gridDim.x < n_tiles) load_pos(tile + gridDim.x);   // overlaps the copies below
+            if (ptid == 0) LSH_PHASE(0, 0, it, 2);
+            // x rows by TMA (four rows per gather, zero fill for a missing slot), v rows by cp.async
+            if (pw == 0) {
+                for (int gi = lane; gi < kW / 4; gi += 32) {
+                    int rr[4];
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const int p = st.pos[4 * gi + u];
+                        rr[u] = p >= 0 ? (int)(rowbase + p) : -1;
+                    }
+                    tc::tma_gather4(st.X + gi * 512, &tm_x, rr[0], rr[1], rr[2], rr[3], &sm.full[s]);
+                }
+            }
+            for (int c = ptid; c < kW * 8; c += kProducerThreads) {
+                const int row = c >> 3, ch = c & 7;
+                const uint32_t off = (uint32_t)row * 128u + (uint32_t)((ch ^ (row & 7)) << 4);
+                const int p = st.pos[row];
+                if (p >= 0) tc::cp_async16(st.V + off, v + (rowbase + p) * kDim + ch * 8);
+                else *reinterpret_cast<uint4 *>(st.V + off) = make_uint4(0, 0, 0, 0);
+            }
+            tc::cp_async_commit();
             if (pw < 3) {
                 // smallest position of window chunk pw (INT_MAX when the chunk is missing)
                 const int a0 = st.pos[pw * 64 + lane], a1 = st.pos[pw * 64 + 32 + lane];
@@ -232,24 +335,14 @@ attn_fwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
                 for (int o = 16; o > 0; o >>= 1) mn = min(mn, __shfl_xor_sync(0xffffffffu, mn, o));
                 if (lane == 0) st.cmin[pw] = mn;
             }
-            // x and v rows: thread -> one 16-byte chunk, eight consecutive threads -> one row
-            for (int c = ptid; c < 2 * kW * 8; c += kProducerThreads) {
-                const int t = c >= kW * 8;
-                const int idx = c - t * kW * 8;
-                const int row = idx >> 3, ch = idx & 7;
-                const uint32_t off = (uint32_t)row * 128u + (uint32_t)((ch ^ (row & 7)) << 4);
-                uint8_t *dst = (t ? st.V : st.X) + off;
-                const int p = st.pos[row];
-                if (p >= 0) tc::cp_async16(dst, (t ? v : x) + (rowbase + p) * kDim + ch * 8);
-                else *reinterpret_cast<uint4 *>(dst) = make_uint4(0, 0, 0, 0);
-            }
-            tc::cp_async_commit();
+            if (ptid == 0) LSH_PHASE(0, 0, it, 3);
             if (prev_s >= 0) {
                 // the previous stage's copies have landed: publish it
                 tc::cp_async_wait<1>();
                 tc::fence_async_smem();
                 tc::mbar_arrive(&sm.full[prev_s]);
             }
+            if (ptid == 0) LSH_PHASE(0, 0, it, 4);
             prev_s = s;
         }
         if (prev_s >= 0) {
@@ -268,10 +361,12 @@ attn_fwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
                 const bool have = tile < n_tiles;
                 if (have) {
                     const int s = it % kStages, g = it & 1;
+                    LSH_PHASE(0, 1, it, 0);
                     bool ok = tc::mbar_wait(&sm.full[s], (uint32_t)(it / kStages) & 1u, &sm.abort, status);
                     if (ok && it >= 2)
                         ok = tc::mbar_wait(&sm.o_free[g], (uint32_t)((it >> 1) - 1) & 1u, &sm.abort, status);
                     if (!ok) break;
+                    LSH_PHASE(0, 1, it, 1);
                     tc::tc_fence_after();
                     const uint32_t xs = tc::smem_u32(sm.st[s].X);
                     const uint32_t d = tmem + (uint32_t)g * kGroupCols;
@@ -280,10 +375,12 @@ attn_fwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
                         tc::mma_bf16(d, tc::sw128_desc(xs + 64 * 128 + kk * 32), tc::sw128_desc(xs + kk * 32), id_s,
                                      kk > 0);
                     tc::mma_commit(&sm.s_full[g]);
+                    LSH_PHASE(0, 1, it, 2);
                 }
                 if (prev_it >= 0) {
                     const int ps = prev_it % kStages, pg = prev_it & 1;
                     if (!tc::mbar_wait(&sm.p_full[pg], (uint32_t)(prev_it >> 1) & 1u, &sm.abort, status)) break;
+                    LSH_PHASE(0, 1, prev_it, 3);
                     tc::tc_fence_after();
                     const uint32_t vs = tc::smem_u32(sm.st[ps].V);
                     const uint32_t base = tmem + (uint32_t)pg * kGroupCols;
@@ -291,6 +388,7 @@ attn_fwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
                     for (int kk = 0; kk < 12; ++kk)
                         tc::mma_bf16_ts(base + kOCol, base + kk * 8, tc::sw128_desc(vs + kk * 16 * 128), id_o, kk > 0);
                     tc::mma_commit(&sm.o_full[pg]);
+                    LSH_PHASE(0, 1, prev_it, 4);
                 }
                 if (!have) break;
                 prev_it = it;
@@ -300,32 +398,47 @@ attn_fwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
         // ================= softmax groups: group g takes the CTA's tiles it = g, g + 2, ...
         const int g = warp >> 2, q = warp & 3;
         const int i = q * 32 + lane;                             // query row = TMEM lane
+        const int gt = i;                                        // thread index inside the group
         const uint32_t tl = tmem + (uint32_t)g * kGroupCols + ((uint32_t)(q * 32) << 16);
         int it = g;
         for (long long tile = blockIdx.x + (long long)g * gridDim.x; tile < n_tiles;
              tile += 2LL * gridDim.x, it += 2) {
             const int s = it % kStages;
             const uint32_t gph = (uint32_t)(it >> 1) & 1u;
+            const bool mark = gt == 0;
+            if (mark) LSH_PHASE(0, 2 + g, it, 0);
             if (!tc::mbar_wait(&sm.full[s], (uint32_t)(it / kStages) & 1u, &sm.abort, status)) break;
+            if (mark) LSH_PHASE(0, 2 + g, it, 1);
+            Stage &st = sm.st[s];
+            window_norms(st, gt, sl2);
+            tc::named_bar_sync(2 + g, 128);
             if (!tc::mbar_wait(&sm.s_full[g], gph, &sm.abort, status)) break;
+            if (mark) LSH_PHASE(0, 2 + g, it, 2);
             tc::tc_fence_after();
-            const Stage &st = sm.st[s];
             const TileCoord tcd = tile_coord(tile, R, n_k);
             const int qpos = st.pos[64 + i];
             const float qinv = st.inv[64 + i];
             // query chunk a (0: 2k, 1: 2k+1) sees window chunks a and a+1
             const int a = i >> 6;
-            const int self_only = causal && qpos == min(st.cmin[a], st.cmin[a + 1]);
+            const bool self_only = causal && qpos == min(st.cmin[a], st.cmin[a + 1]);
+            const bool first = tcd.k == 0;
             float l, row_lse;
-            if (q < 2)
-                softmax_row<0>(st, tl, tcd.k == 0 ? 64 : 0, qpos, qinv, self_only, causal, tau, l, row_lse);
-            else
-                softmax_row<64>(st, tl, 0, qpos, qinv, self_only, causal, tau, l, row_lse);
+            if (causal) {
+                if (q >= 2) softmax_row<64, true, false>(st, tl, i, qpos, qinv, self_only, tau, l, row_lse);
+                else if (first) softmax_row<0, true, true>(st, tl, i, qpos, qinv, self_only, tau, l, row_lse);
+                else softmax_row<0, true, false>(st, tl, i, qpos, qinv, self_only, tau, l, row_lse);
+            } else {
+                if (q >= 2) softmax_row<64, false, false>(st, tl, i, qpos, qinv, false, tau, l, row_lse);
+                else if (first) softmax_row<0, false, true>(st, tl, i, qpos, qinv, false, tau, l, row_lse);
+                else softmax_row<0, false, false>(st, tl, i, qpos, qinv, false, tau, l, row_lse);
+            }
             tc::tmem_st_wait();
             tc::tc_fence_before();
             __syncwarp();
             if (lane == 0) tc::mbar_arrive(&sm.p_full[g]);
+            if (mark) LSH_PHASE(0, 2 + g, it, 3);
             if (!tc::mbar_wait(&sm.o_full[g], gph, &sm.abort, status)) break;
+            if (mark) LSH_PHASE(0, 2 + g, it, 4);
             tc::tc_fence_after();
             float o[kDim];
 #pragma unroll
@@ -342,6 +455,7 @@ attn_fwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
             for (int d = 0; d < kDim; ++d) o[d] *= rl;
             store_row(o_r + (tcd.seg * L + qpos) * kDim, o);
             lse[tcd.seg * L + qpos] = row_lse;
+            if (mark) LSH_PHASE(0, 2 + g, it, 5);
         }
     }
 
@@ -364,6 +478,9 @@ cudaError_t launch_attn_fwd_tc(const Problem &p, const void *x, const void *v, c
                                const float *invnorm, __nv_bfloat16 *o_r, float *lse, uint32_t *status,
                                cudaStream_t st)
 {
+    (void)invnorm;      // key norms are computed in the kernel from the gathered rows
+    CUtensorMap tx;
+    if (!tc::make_row_tmap(&tx, x, p.tokens())) return cudaErrorInvalidValue;
     const size_t smem = sizeof(FwdSmem) + 1024;
     cudaError_t e = cudaFuncSetAttribute(attn_fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
@@ -372,9 +489,11 @@ cudaError_t launch_attn_fwd_tc(const Problem &p, const void *x, const void *v, c
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const long long n_tiles = p.S() * (p.L / kQ);
     const unsigned grid = (unsigned)std::min<long long>(n_tiles, (long long)sms);
-    attn_fwd_tc_kernel<<<grid, kThreads, smem, st>>>((const __nv_bfloat16 *)x, (const __nv_bfloat16 *)v, perm, invnorm, o_r, lse, p.L, p.R, n_tiles, p.causal,
-                                                     1.0f / sqrtf((float)p.d), status);
+    attn_fwd_tc_kernel<<<grid, kThreads, smem, st>>>(tx, (const __nv_bfloat16 *)v, perm, o_r, lse, p.L, p.R, n_tiles,
+                                                     p.causal, 1.0f / sqrtf((float)p.d), status);
     return cudaGetLastError();
 }
 
 }  // namespace lsh
+
+LSH_PHASE_EXPORT(fwd)

@@ -19,6 +19,29 @@
 
 #include "common.cuh"
 
+// Optional phase timestamps for tuning (build with -DLSH_PHASE_TRACE): CTA 0
+// records clock64() at named points of its first 32 tiles into the
+// translation unit's lsh_phase_trace[role][tile][event];
+// LSH_PHASE_EXPORT(name) defines lsh_attn_phase_trace_<name>(out) to copy it
+// to the host.  Compiled out otherwise.
+#ifdef LSH_PHASE_TRACE
+static __device__ long long lsh_phase_trace[4][32][8];
+#define LSH_PHASE(kern, role, it, ev)                                                             \
+    do {                                                                                          \
+        if (blockIdx.x == 0 && (it) >= 0 && (it) < 32) lsh_phase_trace[role][it][ev] = clock64(); \
+    } while (0)
+#define LSH_PHASE_EXPORT(name)                                                                    \
+    extern "C" LSH_API int lsh_attn_phase_trace_##name(long long *out)                            \
+    {                                                                                             \
+        return (int)cudaMemcpyFromSymbol(out, lsh_phase_trace, sizeof(lsh_phase_trace));          \
+    }
+#else
+#define LSH_PHASE(kern, role, it, ev) \
+    do {                              \
+    } while (0)
+#define LSH_PHASE_EXPORT(name)
+#endif
+
 namespace lsh {
 namespace tc {
 
@@ -80,6 +103,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
     const long long t0 = clock64();
     while (true) {
         if (mbar_try_wait(bar, parity)) return true;
+        __nanosleep(32);                  // leave issue slots to the warps doing work
         if (*abort) return false;
         if (clock64() - t0 > budget) {
             *abort = 1;
