@@ -35,11 +35,10 @@
 //                   its own 256 TMEM columns (S/P 192, O 64), so one group's
 //                   softmax overlaps the other's MMAs and stores;
 //   warps 8-11      producer: positions (loaded a tile ahead) and window
-//                   minima; x rows by TMA (tile::gather4, four rows per
-//                   instruction) and v rows by 16-byte cp.async, so both copy
-//                   engines work at once, into a 3-stage shared-memory ring; a
-//                   stage is published once the next stage's copies are in
-//                   flight;
+//                   minima; x and v rows by 16-byte cp.async (eight threads
+//                   per row, zero fill for a missing slot) into a 3-stage
+//                   shared-memory ring; a stage is published once the next
+//                   stage's copies are in flight;
 //   warp 12         MMA issuer.
 #include "tc_common.cuh"
 
@@ -238,7 +237,7 @@ __device__ __forceinline__ void window_norms(Stage &st, int t, float sl2)
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
-attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __nv_bfloat16 *__restrict__ v,
+attn_fwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__restrict__ v,
                    const int32_t *__restrict__ perm, __nv_bfloat16 *__restrict__ o_r, float *__restrict__ lse, int L,
                    int R, long long n_tiles, int causal, float tau, uint32_t *__restrict__ status)
 {
@@ -271,7 +270,6 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __nv_bfloat16
     if (warp >= kSoftmaxWarps && warp < kMmaWarp) {
         // ================= producer group
         const int ptid = tid - kSoftmaxWarps * 32, pw = ptid >> 5;
-        if (ptid == 0) tc::prefetch_tmap(&tm_x);
         // positions of the next tile, loaded a tile ahead (two slots per thread)
         int pn[2] = {-1, -1};
         auto load_pos = [&](long long tile) {
@@ -303,28 +301,25 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __nv_bfloat16
                 const int e = ptid + j * kProducerThreads;
                 if (e < kW) st.pos[e] = pn[j];
             }
-            if (ptid == 0) tc::mbar_expect_tx(&sm.full[s], kW * 128);
             tc::named_bar_sync(1, kProducerThreads);
             if (tile + gridDim.x < n_tiles) load_pos(tile + gridDim.x);   // overlaps the copies below
             if (ptid == 0) LSH_PHASE(0, 0, it, 2);
-            // x rows by TMA (four rows per gather, zero fill for a missing slot), v rows by cp.async
-            if (pw == 0) {
-                for (int gi = lane; gi < kW / 4; gi += 32) {
-                    int rr[4];
+            // x and v rows: thread t copies 16-byte chunk t % 8 of rows t / 8 + 16 j
+            // (zero fill for a missing slot); every position is read first for ILP
+            {
+                const int ch = ptid & 7, r0 = ptid >> 3;
+                int pr[kW / 16];
 #pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        const int p = st.pos[4 * gi + u];
-                        rr[u] = p >= 0 ? (int)(rowbase + p) : -1;
-                    }
-                    tc::tma_gather4(st.X + gi * 512, &tm_x, rr[0], rr[1], rr[2], rr[3], &sm.full[s]);
+                for (int j = 0; j < kW / 16; ++j) pr[j] = st.pos[r0 + 16 * j];
+#pragma unroll
+                for (int j = 0; j < kW / 16; ++j) {
+                    const int row = r0 + 16 * j;
+                    const uint32_t off = (uint32_t)row * 128u + (uint32_t)((ch ^ (row & 7)) << 4);
+                    const long long src = (rowbase + max(pr[j], 0)) * kDim + ch * 8;
+                    const uint32_t nb = pr[j] >= 0 ? 16u : 0u;
+                    tc::cp_async16_zfill(st.X + off, x + src, nb);
+                    tc::cp_async16_zfill(st.V + off, v + src, nb);
                 }
-            }
-            for (int c = ptid; c < kW * 8; c += kProducerThreads) {
-                const int row = c >> 3, ch = c & 7;
-                const uint32_t off = (uint32_t)row * 128u + (uint32_t)((ch ^ (row & 7)) << 4);
-                const int p = st.pos[row];
-                if (p >= 0) tc::cp_async16(st.V + off, v + (rowbase + p) * kDim + ch * 8);
-                else *reinterpret_cast<uint4 *>(st.V + off) = make_uint4(0, 0, 0, 0);
             }
             tc::cp_async_commit();
             if (pw < 3) {
@@ -351,47 +346,65 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __nv_bfloat16
             tc::mbar_arrive(&sm.full[prev_s]);
         }
     } else if (warp == kMmaWarp) {
-        // ================= MMA issuer: S of tile t+1 is issued before O of tile t
+        // ================= MMA issuer
+        // S = Q K^T of a tile needs its stage loaded and its group's TMEM free;
+        // O = P V needs the tile's P.  Whichever is ready is issued first, so a
+        // late stage never holds back the O of the tile before it.
         if (lane == 0) {
             constexpr uint32_t id_s = tc::idesc_bf16(128, kW, 0, 0);
             constexpr uint32_t id_o = tc::idesc_bf16(128, kDim, 0, 1);
-            int prev_it = -1;
-            int it = 0;
-            for (long long tile = blockIdx.x;; tile += gridDim.x, ++it) {
-                const bool have = tile < n_tiles;
-                if (have) {
-                    const int s = it % kStages, g = it & 1;
-                    LSH_PHASE(0, 1, it, 0);
-                    bool ok = tc::mbar_wait(&sm.full[s], (uint32_t)(it / kStages) & 1u, &sm.abort, status);
-                    if (ok && it >= 2)
-                        ok = tc::mbar_wait(&sm.o_free[g], (uint32_t)((it >> 1) - 1) & 1u, &sm.abort, status);
-                    if (!ok) break;
-                    LSH_PHASE(0, 1, it, 1);
-                    tc::tc_fence_after();
-                    const uint32_t xs = tc::smem_u32(sm.st[s].X);
-                    const uint32_t d = tmem + (uint32_t)g * kGroupCols;
+            long long n_mine = 0;
+            if (blockIdx.x < n_tiles) n_mine = (n_tiles - 1 - blockIdx.x) / gridDim.x + 1;
+            int next_s = 0, next_o = 0;                     // next tile (local index) for S and for O
+            long long t0 = clock64();
+            while (next_o < n_mine) {
+                bool progressed = false;
+                if (next_s < n_mine && next_s <= next_o + 1) {
+                    const int it = next_s, s = it % kStages, g = it & 1;
+                    if (tc::mbar_test_wait(&sm.full[s], (uint32_t)(it / kStages) & 1u) &&
+                        (it < 2 || tc::mbar_test_wait(&sm.o_free[g], (uint32_t)((it >> 1) - 1) & 1u))) {
+                        LSH_PHASE(0, 1, it, 1);
+                        tc::tc_fence_after();
+                        const uint32_t xs = tc::smem_u32(sm.st[s].X);
+                        const uint32_t d = tmem + (uint32_t)g * kGroupCols;
 #pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)
-                        tc::mma_bf16(d, tc::sw128_desc(xs + 64 * 128 + kk * 32), tc::sw128_desc(xs + kk * 32), id_s,
-                                     kk > 0);
-                    tc::mma_commit(&sm.s_full[g]);
-                    LSH_PHASE(0, 1, it, 2);
+                        for (int kk = 0; kk < 4; ++kk)
+                            tc::mma_bf16(d, tc::sw128_desc(xs + 64 * 128 + kk * 32), tc::sw128_desc(xs + kk * 32),
+                                         id_s, kk > 0);
+                        tc::mma_commit(&sm.s_full[g]);
+                        LSH_PHASE(0, 1, it, 2);
+                        ++next_s;
+                        progressed = true;
+                    }
                 }
-                if (prev_it >= 0) {
-                    const int ps = prev_it % kStages, pg = prev_it & 1;
-                    if (!tc::mbar_wait(&sm.p_full[pg], (uint32_t)(prev_it >> 1) & 1u, &sm.abort, status)) break;
-                    LSH_PHASE(0, 1, prev_it, 3);
-                    tc::tc_fence_after();
-                    const uint32_t vs = tc::smem_u32(sm.st[ps].V);
-                    const uint32_t base = tmem + (uint32_t)pg * kGroupCols;
+                if (next_o < next_s) {
+                    const int it = next_o, s = it % kStages, g = it & 1;
+                    if (tc::mbar_test_wait(&sm.p_full[g], (uint32_t)(it >> 1) & 1u)) {
+                        LSH_PHASE(0, 1, it, 3);
+                        tc::tc_fence_after();
+                        const uint32_t vs = tc::smem_u32(sm.st[s].V);
+                        const uint32_t base = tmem + (uint32_t)g * kGroupCols;
 #pragma unroll
-                    for (int kk = 0; kk < 12; ++kk)
-                        tc::mma_bf16_ts(base + kOCol, base + kk * 8, tc::sw128_desc(vs + kk * 16 * 128), id_o, kk > 0);
-                    tc::mma_commit(&sm.o_full[pg]);
-                    LSH_PHASE(0, 1, prev_it, 4);
+                        for (int kk = 0; kk < 12; ++kk)
+                            tc::mma_bf16_ts(base + kOCol, base + kk * 8, tc::sw128_desc(vs + kk * 16 * 128), id_o,
+                                            kk > 0);
+                        tc::mma_commit(&sm.o_full[g]);
+                        LSH_PHASE(0, 1, it, 4);
+                        ++next_o;
+                        progressed = true;
+                    }
                 }
-                if (!have) break;
-                prev_it = it;
+                if (progressed) {
+                    t0 = clock64();
+                } else {
+                    if (*reinterpret_cast<volatile int *>(&sm.abort)) break;
+                    if (clock64() - t0 > tc::kWaitCycles) {
+                        sm.abort = 1;
+                        atomicOr(status, kStatusTimeout);
+                        break;
+                    }
+                    __nanosleep(20);
+                }
             }
         }
     } else {
@@ -479,8 +492,6 @@ cudaError_t launch_attn_fwd_tc(const Problem &p, const void *x, const void *v, c
                                cudaStream_t st)
 {
     (void)invnorm;      // key norms are computed in the kernel from the gathered rows
-    CUtensorMap tx;
-    if (!tc::make_row_tmap(&tx, x, p.tokens())) return cudaErrorInvalidValue;
     const size_t smem = sizeof(FwdSmem) + 1024;
     cudaError_t e = cudaFuncSetAttribute(attn_fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
@@ -489,7 +500,7 @@ cudaError_t launch_attn_fwd_tc(const Problem &p, const void *x, const void *v, c
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const long long n_tiles = p.S() * (p.L / kQ);
     const unsigned grid = (unsigned)std::min<long long>(n_tiles, (long long)sms);
-    attn_fwd_tc_kernel<<<grid, kThreads, smem, st>>>(tx, (const __nv_bfloat16 *)v, perm, o_r, lse, p.L, p.R, n_tiles,
+    attn_fwd_tc_kernel<<<grid, kThreads, smem, st>>>((const __nv_bfloat16 *)x, (const __nv_bfloat16 *)v, perm, o_r, lse, p.L, p.R, n_tiles,
                                                      p.causal, 1.0f / sqrtf((float)p.d), status);
     return cudaGetLastError();
 }
