@@ -281,7 +281,9 @@ lsh_status lsh_attn_bwd(const lsh_attn_desc *desc, const void *qk, const void *v
         if ((s = run_hash_sort(p, c, qk, R, w.perm, w, st)) != LSH_OK) return s;
         perm = w.perm;
     }
-    LSH_TRY(staged(LSH_STAGE_NORMS, 1, st, [&] { return launch_invnorm(p, qk, w.invnorm, st); }), "key norms");
+    // the tensor-core backward computes the key norms from its gathered rows
+    if (!c.tc_attn)
+        LSH_TRY(staged(LSH_STAGE_NORMS, 1, st, [&] { return launch_invnorm(p, qk, w.invnorm, st); }), "key norms");
     LSH_TRY(staged(LSH_STAGE_BWD_PREP, 1, st, [&] {
                 return launch_bwd_prep(p, lse, out, dout, w.lse_all, w.delta, w.dx_acc, w.dv_acc, st);
             }), "backward prologue");

@@ -64,7 +64,6 @@ struct alignas(1024) Stage {
     uint8_t G[kQ * 128];            // dY rows of the query slots                           24 KB
     alignas(16) int32_t pos[256];   // positions of slots [128k - 64, 128k + 192); -1 if none
     alignas(16) float4 qinfo[kQ];   // {LSE * log2 e (+inf if none), delta, self flag, position bits}
-    alignas(16) float kinv[kK];
     int32_t cmin[4];                // smallest position of chunks 2k-1 .. 2k+2 (INT_MAX if none)
 };
 
@@ -102,10 +101,12 @@ __device__ __forceinline__ void smem_chunk(const uint8_t *tile, int row, int ch,
 }
 
 // Elementwise step for key row kr over query columns [C0, C0 + 64): P^T (bf16)
-// into TMEM columns cPT + C0/2, E^T into shared-memory block C0/64.
-template <int C0>
+// into TMEM columns cPT + C0/2, E^T into shared-memory block C0/64.  A
+// candidate is a query at a later original position (causal) or at any other
+// position; a query with no other candidate is patched in by self_fixup.
+template <int C0, bool CAUSAL>
 __device__ __forceinline__ void key_row_block(const Stage &st, uint8_t (*ET)[kK * 128], uint32_t tl, int kr, int kpos,
-                                              float kinv, int causal, float tau)
+                                              float kinv, float tau)
 {
     const float sc = tau * kinv * kLog2e;
     const float ec = tau * kinv;
@@ -123,17 +124,12 @@ __device__ __forceinline__ void key_row_block(const Stage &st, uint8_t (*ET)[kK 
             float pv[2], ev[2];
 #pragma unroll
             for (int u = 0; u < 2; ++u) {
-                const int q = C0 + h * 32 + j + u;
-                const float4 qi = st.qinfo[q];
+                const float4 qi = st.qinfo[C0 + h * 32 + j + u];
                 const int qp = __float_as_int(qi.w);
-                // branch-free mask: candidate if causal-earlier (or any other position when
-                // not causal), or the query itself when it has no other candidate
-                const int ordered = causal ? (kpos < qp) : (kpos != qp);
-                const int self = (kpos == qp) & (qi.z != 0.f);
+                const bool ok = CAUSAL ? (kpos < qp) : (kpos != qp);
                 const float e2 = tc::fast_exp2(fmaf(s[j + u], sc, -qi.x));
-                const float p = (ordered | self) ? e2 : 0.f;
-                pv[u] = p;
-                ev[u] = ec * p * (dp[j + u] - qi.y);
+                pv[u] = ok ? e2 : 0.f;
+                ev[u] = ec * pv[u] * (dp[j + u] - qi.y);
             }
             pw[j / 2] = pack_bf16x2(pv[0], pv[1]);
             ew[j / 2] = pack_bf16x2(ev[0], ev[1]);
@@ -147,6 +143,55 @@ __device__ __forceinline__ void key_row_block(const Stage &st, uint8_t (*ET)[kK 
             *reinterpret_cast<uint4 *>(ET[blk] + off) =
                 make_uint4(ew[4 * c4], ew[4 * c4 + 1], ew[4 * c4 + 2], ew[4 * c4 + 3]);
         }
+    }
+}
+
+// Causal queries with no other candidate attend to themselves: for key row kr
+// (< 128) the query of the same slot is column kr.  Where that query is flagged,
+// P^T[kr][kr] = exp(s - LSE) and E^T[kr][kr] = tau inv (P (dY.v - delta)) are
+// written over the zeros key_row_block left.  Run by the warps that own columns
+// [32 quad, 32 quad + 32); tcgen05 loads and stores stay warp-wide.
+__device__ __forceinline__ void self_fixup(const Stage &st, uint8_t (*ET)[kK * 128], uint32_t tl, int quad, int lane,
+                                           float kinv, float tau)
+{
+    const int kr = quad * 32 + lane;
+    const float4 qi = st.qinfo[kr];
+    const bool me = qi.z != 0.f;
+    if (!__any_sync(0xffffffffu, me)) return;
+    const uint32_t cb = (uint32_t)(quad * 32);
+    float sv[32], dv[32];
+    tc::tmem_ld16(tl + cS + cb, sv);
+    tc::tmem_ld16(tl + cS + cb + 16, sv + 16);
+    tc::tmem_ld16(tl + cD + cb, dv);
+    tc::tmem_ld16(tl + cD + cb + 16, dv + 16);
+    tc::tmem_st_wait();
+    float pk[16];
+    tc::tmem_ld16(tl + cPT + cb / 2, pk);
+    tc::tmem_ld_wait();
+    float s_self = 0.f, d_self = 0.f;
+#pragma unroll
+    for (int c = 0; c < 32; ++c) {
+        s_self = (c == lane) ? sv[c] : s_self;
+        d_self = (c == lane) ? dv[c] : d_self;
+    }
+    const float p = tc::fast_exp2(fmaf(s_self, tau * kinv * kLog2e, -qi.x));
+    const float e = tau * kinv * p * (d_self - qi.y);
+    uint32_t u[16];
+#pragma unroll
+    for (int c = 0; c < 16; ++c) {
+        uint32_t w = __float_as_uint(pk[c]);
+        if (me && c == (lane >> 1)) {
+            const __nv_bfloat16 hb = __float2bfloat16_rn(p);
+            const uint32_t hv = (uint32_t)(*reinterpret_cast<const uint16_t *>(&hb));
+            w = (lane & 1) ? ((w & 0x0000FFFFu) | (hv << 16)) : ((w & 0xFFFF0000u) | hv);
+        }
+        u[c] = w;
+    }
+    tc::tmem_st16(tl + cPT + cb / 2, u);
+    if (me) {
+        const int q = kr;                                   // query column of this row's own slot
+        uint8_t *chunk = ET[q >> 6] + kr * 128 + (((((q & 63) >> 3)) ^ (kr & 7)) << 4);
+        reinterpret_cast<__nv_bfloat16 *>(chunk)[q & 7] = __float2bfloat16_rn(e);
     }
 }
 
@@ -212,6 +257,20 @@ attn_bwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
     if (warp >= kComputeWarps && warp < kMmaWarp) {
         // ================= producer group
         const int ptid = tid - kComputeWarps * 32, pw = ptid >> 5;
+        // positions of slots [128k - 64, 128k + 192) of the next tile, loaded a tile ahead
+        int pn[2];
+        auto load_pos = [&](long long tile) {
+            const TileCoord c = tile_coord(tile, R, n_k);
+            const int32_t *P = perm + c.seg * L;
+            const int slot0 = c.k * kK - 64;
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                const int sl = slot0 + ptid + j * kProducerThreads;
+                const int pl = P[min(max(sl, 0), L - 1)];
+                pn[j] = (sl >= 0 && sl < L) ? pl : -1;
+            }
+        };
+        if (blockIdx.x < n_tiles) load_pos(blockIdx.x);
         int it = 0;
         for (long long tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++it) {
             const int s = it % kStages;
@@ -221,28 +280,38 @@ attn_bwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
             if (tc::named_bar_or(1, kProducerThreads, !ok)) break;
             if (ptid == 0) LSH_PHASE(1, 0, it, 1);
             Stage &st = sm.st[s];
-            const TileCoord tcd = tile_coord(tile, R, n_k);
-            const int32_t *P = perm + tcd.seg * L;
-            const long long rowbase = tcd.bh * L;
-            const int slot0 = tcd.k * kK - 64;
-            // positions of slots [128k - 64, 128k + 192): two per thread, loads clamped in range
-            for (int e = ptid; e < 256; e += kProducerThreads) {
-                const int sl = slot0 + e;
-                const int pl = P[min(max(sl, 0), L - 1)];
-                st.pos[e] = (sl >= 0 && sl < L) ? pl : -1;
-            }
+            const long long rowbase = tile_coord(tile, R, n_k).bh * L;
+            st.pos[ptid] = pn[0];
+            st.pos[ptid + kProducerThreads] = pn[1];
             tc::named_bar_sync(1, kProducerThreads);
-            // x, dY rows of the 192 query slots and v rows of the 128 key slots
-            for (int c = ptid; c < (2 * kQ + kK) * 8; c += kProducerThreads) {
-                const int t = c < kQ * 8 ? 0 : (c < 2 * kQ * 8 ? 1 : 2);
-                const int idx = c - (t == 0 ? 0 : t == 1 ? kQ * 8 : 2 * kQ * 8);
-                const int row = idx >> 3, ch = idx & 7;
-                const uint32_t off = (uint32_t)row * 128u + (uint32_t)((ch ^ (row & 7)) << 4);
-                uint8_t *dst = (t == 0 ? st.X : t == 1 ? st.G : st.V) + off;
-                const __nv_bfloat16 *srcb = t == 0 ? x : t == 1 ? dout : v;
-                const int p = st.pos[64 + row];
-                if (p >= 0) tc::cp_async16(dst, srcb + (rowbase + p) * kDim + ch * 8);
-                else *reinterpret_cast<uint4 *>(dst) = make_uint4(0, 0, 0, 0);
+            // per-query LSE and delta: loads issued now, used after the copies are issued
+            int qp[2];
+            float ql[2], qd[2];
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                const int q = min(ptid + j * kProducerThreads, kQ - 1);
+                qp[j] = st.pos[64 + q];
+                const long long rp = rowbase + max(qp[j], 0);
+                ql[j] = lse_all[rp];
+                qd[j] = delta[rp];
+            }
+            // x, dY rows of the 192 query slots and v rows of the 128 key slots: thread t
+            // copies chunk t % 8 of rows t / 8 + 16 j (zero fill for a missing slot)
+            {
+                const int ch = ptid & 7, r0 = ptid >> 3;
+                int pr[kQ / 16];
+#pragma unroll
+                for (int j = 0; j < kQ / 16; ++j) pr[j] = st.pos[64 + r0 + 16 * j];
+#pragma unroll
+                for (int j = 0; j < kQ / 16; ++j) {
+                    const int row = r0 + 16 * j;
+                    const uint32_t off = (uint32_t)row * 128u + (uint32_t)((ch ^ (row & 7)) << 4);
+                    const long long src = (rowbase + max(pr[j], 0)) * kDim + ch * 8;
+                    const uint32_t nb = pr[j] >= 0 ? 16u : 0u;
+                    tc::cp_async16_zfill(st.X + off, x + src, nb);
+                    tc::cp_async16_zfill(st.G + off, dout + src, nb);
+                    if (row < kK) tc::cp_async16_zfill(st.V + off, v + src, nb);
+                }
             }
             tc::cp_async_commit();
             if (ptid == 0) LSH_PHASE(1, 0, it, 2);
@@ -255,21 +324,22 @@ attn_bwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
                 if (lane == 0) st.cmin[pw] = mn;
             }
             tc::named_bar_sync(1, kProducerThreads);
-            // per-query LSE, delta, self flag; per-key norm (loads clamped in range, then selected)
-            for (int q = ptid; q < kQ; q += kProducerThreads) {
-                const int p = st.pos[64 + q];
-                const long long rp = rowbase + max(p, 0);
-                const float lv = lse_all[rp], dv = delta[rp], nv = invnorm[rp];
-                const int qa = q >> 6;
-                const int wmin = min(st.cmin[qa], st.cmin[qa + 1]);
-                float4 qi;
-                qi.x = p >= 0 ? lv * kLog2e : INFINITY;
-                qi.y = p >= 0 ? dv : 0.f;
-                qi.z = (p >= 0 && causal && p == wmin) ? 1.f : 0.f;
-                qi.w = __int_as_float(p);
-                st.qinfo[q] = qi;
-                if (q < kK) st.kinv[q] = p >= 0 ? nv : 0.f;
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                const int q = ptid + j * kProducerThreads;
+                if (q < kQ) {
+                    const int p = qp[j];
+                    const int qa = q >> 6;
+                    const int wmin = min(st.cmin[qa], st.cmin[qa + 1]);
+                    float4 qi;
+                    qi.x = p >= 0 ? ql[j] * kLog2e : INFINITY;
+                    qi.y = p >= 0 ? qd[j] : 0.f;
+                    qi.z = (p >= 0 && causal && p == wmin) ? 1.f : 0.f;
+                    qi.w = __int_as_float(p);
+                    st.qinfo[q] = qi;
+                }
             }
+            if (tile + gridDim.x < n_tiles) load_pos(tile + gridDim.x);
             if (ptid == 0) LSH_PHASE(1, 0, it, 3);
             // with two stages the producer cannot run further ahead: publish this stage now
             tc::cp_async_wait<0>();
@@ -339,24 +409,55 @@ attn_bwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
             const TileCoord tcd = tile_coord(tile, R, n_k);
             const long long rowbase = tcd.bh * L;
             const int kpos = st.pos[64 + kr];
-            const float kinv = st.kinv[kr];
+            // 1/|x_k| of this key row from the gathered tile (sum of squares in element order)
+            float kinv;
+            {
+                float ssq = 0.f;
+#pragma unroll
+                for (int ch = 0; ch < 8; ++ch) {
+                    float xr[8];
+                    smem_chunk(st.X, kr, ch, xr);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) ssq = fmaf(xr[e], xr[e], ssq);
+                }
+                kinv = ssq > 0.f ? 1.0f / sqrtf(ssq) : 0.f;
+            }
             if (!tc::mbar_wait(&sm.bar_s, ph, &sm.abort, status)) break;
             if (tid == 0) LSH_PHASE(1, 2, it, 2);
             tc::tc_fence_after();
             // ---- elementwise
-            if (quad < 2) {                          // keys of chunk 2k: queries of chunks 2k, 2k+1
-                if (half == 0) {
-                    key_row_block<0>(st, sm.ET, tl, kr, kpos, kinv, causal, tau);
-                    zero_block<128>(sm.ET, tl, kr);
-                } else {
-                    key_row_block<64>(st, sm.ET, tl, kr, kpos, kinv, causal, tau);
+            if (causal) {
+                if (quad < 2) {                      // keys of chunk 2k: queries of chunks 2k, 2k+1
+                    if (half == 0) {
+                        key_row_block<0, true>(st, sm.ET, tl, kr, kpos, kinv, tau);
+                        zero_block<128>(sm.ET, tl, kr);
+                    } else {
+                        key_row_block<64, true>(st, sm.ET, tl, kr, kpos, kinv, tau);
+                    }
+                } else {                             // keys of chunk 2k+1: queries of chunks 2k+1, 2k+2
+                    if (half == 0) {
+                        key_row_block<64, true>(st, sm.ET, tl, kr, kpos, kinv, tau);
+                        zero_block<0>(sm.ET, tl, kr);
+                    } else {
+                        key_row_block<128, true>(st, sm.ET, tl, kr, kpos, kinv, tau);
+                    }
                 }
-            } else {                                 // keys of chunk 2k+1: queries of chunks 2k+1, 2k+2
-                if (half == 0) {
-                    key_row_block<64>(st, sm.ET, tl, kr, kpos, kinv, causal, tau);
-                    zero_block<0>(sm.ET, tl, kr);
+                if (half == 0) self_fixup(st, sm.ET, tl, quad, lane, kinv, tau);
+            } else {
+                if (quad < 2) {
+                    if (half == 0) {
+                        key_row_block<0, false>(st, sm.ET, tl, kr, kpos, kinv, tau);
+                        zero_block<128>(sm.ET, tl, kr);
+                    } else {
+                        key_row_block<64, false>(st, sm.ET, tl, kr, kpos, kinv, tau);
+                    }
                 } else {
-                    key_row_block<128>(st, sm.ET, tl, kr, kpos, kinv, causal, tau);
+                    if (half == 0) {
+                        key_row_block<64, false>(st, sm.ET, tl, kr, kpos, kinv, tau);
+                        zero_block<0>(sm.ET, tl, kr);
+                    } else {
+                        key_row_block<128, false>(st, sm.ET, tl, kr, kpos, kinv, tau);
+                    }
                 }
             }
             tc::tmem_st_wait();
