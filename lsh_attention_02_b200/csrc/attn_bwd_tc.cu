@@ -31,11 +31,11 @@
 // Warp roles (persistent CTA, one per SM):
 //   warps 0-7  compute: warp w owns TMEM lanes 32*(w%4).. (key rows) and query
 //              columns half (w/4); elementwise step, then the epilogue;
-//   warps 8-11 producer: positions, per-query LSE / delta / self flags and
+//   warps 8-10 producer: positions, per-query LSE / delta / self flags and
 //              per-key norms into a 2-stage ring, then 16-byte cp.async
 //              gathers of the x, v and dY rows straight into the swizzled
 //              operand layout;
-//   warp 12    MMA issuer.
+//   warp 11    MMA issuer.
 #include "tc_common.cuh"
 
 namespace lsh {
@@ -46,7 +46,7 @@ constexpr int kK = 128;             // key slots per tile
 constexpr int kQ = 192;             // query slots per tile
 constexpr int kStages = 2;
 constexpr int kComputeWarps = 8;
-constexpr int kProducerWarps = 4;
+constexpr int kProducerWarps = 3;
 constexpr int kProducerThreads = kProducerWarps * 32;
 constexpr int kMmaWarp = kComputeWarps + kProducerWarps;
 constexpr int kThreads = (kMmaWarp + 1) * 32;
@@ -82,10 +82,26 @@ __device__ __forceinline__ void red_add_v4(float *addr, float a, float b, float 
                  : "memory");
 }
 
-__device__ __forceinline__ void red_row(float *dst, const float *r)
+// Adds each lane's 64-float row `a` to row `rowg` of `acc` (skipped when
+// rowg < 0) with coalesced vector reductions: the warp's 32 rows go through
+// its 8 KB staging buffer (16-byte chunks swizzled by lane against bank
+// conflicts), then each reduction instruction covers two whole rows.
+__device__ __forceinline__ void flush_rows(uint8_t *stg, int lane, const float *a, float *acc, long long rowg)
 {
 #pragma unroll
-    for (int c = 0; c < 16; ++c) red_add_v4(dst + 4 * c, r[4 * c], r[4 * c + 1], r[4 * c + 2], r[4 * c + 3]);
+    for (int c = 0; c < 16; ++c)
+        *reinterpret_cast<float4 *>(stg + lane * 256 + ((c ^ (lane & 15)) << 4)) =
+            make_float4(a[4 * c], a[4 * c + 1], a[4 * c + 2], a[4 * c + 3]);
+    __syncwarp();
+    const int c = lane & 15;
+#pragma unroll 4
+    for (int it = 0; it < 16; ++it) {
+        const int rr = 2 * it + (lane >> 4);
+        const long long rg = __shfl_sync(0xffffffffu, rowg, rr);
+        const float4 val = *reinterpret_cast<const float4 *>(stg + rr * 256 + ((c ^ (rr & 15)) << 4));
+        if (rg >= 0) red_add_v4(acc + rg * kDim + 4 * c, val.x, val.y, val.z, val.w);
+    }
+    __syncwarp();
 }
 
 // Chunk `ch` (elements 8ch .. 8ch+7) of bf16 row `row` of a K-major SW128 tile.
@@ -258,16 +274,18 @@ attn_bwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
         // ================= producer group
         const int ptid = tid - kComputeWarps * 32, pw = ptid >> 5;
         // positions of slots [128k - 64, 128k + 192) of the next tile, loaded a tile ahead
-        int pn[2];
+        constexpr int kPosPer = (256 + kProducerThreads - 1) / kProducerThreads;
+        int pn[kPosPer];
         auto load_pos = [&](long long tile) {
             const TileCoord c = tile_coord(tile, R, n_k);
             const int32_t *P = perm + c.seg * L;
             const int slot0 = c.k * kK - 64;
 #pragma unroll
-            for (int j = 0; j < 2; ++j) {
-                const int sl = slot0 + ptid + j * kProducerThreads;
+            for (int j = 0; j < kPosPer; ++j) {
+                const int e = ptid + j * kProducerThreads;
+                const int sl = slot0 + e;
                 const int pl = P[min(max(sl, 0), L - 1)];
-                pn[j] = (sl >= 0 && sl < L) ? pl : -1;
+                pn[j] = (e < 256 && sl >= 0 && sl < L) ? pl : -1;
             }
         };
         if (blockIdx.x < n_tiles) load_pos(blockIdx.x);
@@ -281,10 +299,14 @@ attn_bwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
             if (ptid == 0) LSH_PHASE(1, 0, it, 1);
             Stage &st = sm.st[s];
             const long long rowbase = tile_coord(tile, R, n_k).bh * L;
-            st.pos[ptid] = pn[0];
-            st.pos[ptid + kProducerThreads] = pn[1];
+#pragma unroll
+            for (int j = 0; j < kPosPer; ++j) {
+                const int e = ptid + j * kProducerThreads;
+                if (e < 256) st.pos[e] = pn[j];
+            }
             tc::named_bar_sync(1, kProducerThreads);
             // per-query LSE and delta: loads issued now, used after the copies are issued
+            static_assert(kQ == 2 * kProducerThreads, "two queries per producer thread");
             int qp[2];
             float ql[2], qd[2];
 #pragma unroll
@@ -296,15 +318,16 @@ attn_bwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
                 qd[j] = delta[rp];
             }
             // x, dY rows of the 192 query slots and v rows of the 128 key slots: thread t
-            // copies chunk t % 8 of rows t / 8 + 16 j (zero fill for a missing slot)
+            // copies chunk t % 8 of rows t / 8 + 12 j (zero fill for a missing slot)
             {
+                constexpr int kRowStep = kProducerThreads / 8;
                 const int ch = ptid & 7, r0 = ptid >> 3;
-                int pr[kQ / 16];
+                int pr[kQ / kRowStep];
 #pragma unroll
-                for (int j = 0; j < kQ / 16; ++j) pr[j] = st.pos[64 + r0 + 16 * j];
+                for (int j = 0; j < kQ / kRowStep; ++j) pr[j] = st.pos[64 + r0 + kRowStep * j];
 #pragma unroll
-                for (int j = 0; j < kQ / 16; ++j) {
-                    const int row = r0 + 16 * j;
+                for (int j = 0; j < kQ / kRowStep; ++j) {
+                    const int row = r0 + kRowStep * j;
                     const uint32_t off = (uint32_t)row * 128u + (uint32_t)((ch ^ (row & 7)) << 4);
                     const long long src = (rowbase + max(pr[j], 0)) * kDim + ch * 8;
                     const uint32_t nb = pr[j] >= 0 ? 16u : 0u;
@@ -315,13 +338,13 @@ attn_bwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
             }
             tc::cp_async_commit();
             if (ptid == 0) LSH_PHASE(1, 0, it, 2);
-            // smallest position of chunks 2k-1 .. 2k+2 (one warp each)
-            {
-                const int a0 = st.pos[pw * 64 + lane], a1 = st.pos[pw * 64 + 32 + lane];
+            // smallest position of chunks 2k-1 .. 2k+2 (warp w takes chunks w, w + 3)
+            for (int c = pw; c < 4; c += kProducerWarps) {
+                const int a0 = st.pos[c * 64 + lane], a1 = st.pos[c * 64 + 32 + lane];
                 int mn = min(a0 >= 0 ? a0 : INT_MAX, a1 >= 0 ? a1 : INT_MAX);
 #pragma unroll
                 for (int o = 16; o > 0; o >>= 1) mn = min(mn, __shfl_xor_sync(0xffffffffu, mn, o));
-                if (lane == 0) st.cmin[pw] = mn;
+                if (lane == 0) st.cmin[c] = mn;
             }
             tc::named_bar_sync(1, kProducerThreads);
 #pragma unroll
@@ -469,17 +492,20 @@ attn_bwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
             if (!tc::mbar_wait(&sm.bar_o, ph, &sm.abort, status)) break;
             if (tid == 0) LSH_PHASE(1, 2, it, 4);
             tc::tc_fence_after();
-            // ---- epilogue: reductions into the fp32 accumulators
+            // ---- epilogue: reductions into the fp32 accumulators.  The staging
+            // buffers reuse memory the MMAs no longer read: E^T and this stage's v rows.
+            uint8_t *stg = warp < 6 ? reinterpret_cast<uint8_t *>(sm.ET) + warp * 8192
+                                    : const_cast<uint8_t *>(st.V) + (warp - 6) * 8192;
             float a[kDim];
             if (half == 0) {
 #pragma unroll
                 for (int c = 0; c < 4; ++c) tc::tmem_ld16(tl + cDV + c * 16, a + c * 16);
                 tc::tmem_ld_wait();
-                red_row(dv_acc + (rowbase + kpos) * kDim, a);
+                flush_rows(stg, lane, a, dv_acc, rowbase + kpos);
 #pragma unroll
                 for (int c = 0; c < 4; ++c) tc::tmem_ld16(tl + cQa + c * 16, a + c * 16);
                 tc::tmem_ld_wait();
-                red_row(dx_acc + (rowbase + kpos) * kDim, a);        // query row kr = key slot kr
+                flush_rows(stg, lane, a, dx_acc, rowbase + kpos);         // query row kr = key slot kr
             } else {
 #pragma unroll
                 for (int c = 0; c < 4; ++c) tc::tmem_ld16(tl + cG + c * 16, a + c * 16);
@@ -501,13 +527,13 @@ attn_bwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
 #pragma unroll
                     for (int e = 0; e < 8; ++e) a[ch * 8 + e] = fmaf(-cf, xr[e], a[ch * 8 + e]);
                 }
-                red_row(dx_acc + (rowbase + kpos) * kDim, a);           // key role of key kr
-                if (quad >= 2) {                                         // query row 64 + kr (chunk 2k+2)
+                flush_rows(stg, lane, a, dx_acc, rowbase + kpos);         // key role of key kr
+                if (quad >= 2) {                                          // query row 64 + kr (chunk 2k+2)
 #pragma unroll
                     for (int c = 0; c < 4; ++c) tc::tmem_ld16(tl + cQb + c * 16, a + c * 16);
                     tc::tmem_ld_wait();
                     const int qp = __float_as_int(st.qinfo[64 + kr].w);
-                    if (qp >= 0) red_row(dx_acc + (rowbase + qp) * kDim, a);
+                    flush_rows(stg, lane, a, dx_acc, qp >= 0 ? rowbase + qp : -1LL);
                 }
             }
             if (tid == 0) LSH_PHASE(1, 2, it, 5);

@@ -34,12 +34,12 @@
 //   warps 0-3, 4-7  two softmax groups working on alternate tiles, each with
 //                   its own 256 TMEM columns (S/P 192, O 64), so one group's
 //                   softmax overlaps the other's MMAs and stores;
-//   warps 8-11      producer: positions (loaded a tile ahead) and window
+//   warps 8-10      producer: positions (loaded a tile ahead) and window
 //                   minima; x and v rows by 16-byte cp.async (eight threads
 //                   per row, zero fill for a missing slot) into a 3-stage
 //                   shared-memory ring; a stage is published once the next
 //                   stage's copies are in flight;
-//   warp 12         MMA issuer.
+//   warp 11         MMA issuer.
 #include "tc_common.cuh"
 
 namespace lsh {
@@ -50,10 +50,12 @@ constexpr int kQ = 128;             // query slots per tile
 constexpr int kW = 192;             // window rows (keys)
 constexpr int kStages = 3;
 constexpr int kSoftmaxWarps = 8;   // two groups of four
-constexpr int kProducerWarps = 4;
+constexpr int kProducerWarps = 3;
 constexpr int kProducerThreads = kProducerWarps * 32;
 constexpr int kMmaWarp = kSoftmaxWarps + kProducerWarps;
 constexpr int kThreads = (kMmaWarp + 1) * 32;
+static_assert(kW == 2 * kProducerThreads, "two window positions per producer thread");
+static_assert(kW % (kProducerThreads / 8) == 0, "rows split evenly over the producer");
 constexpr int kTmemCols = 512;
 constexpr uint32_t kGroupCols = 256;
 constexpr uint32_t kOCol = 192;
@@ -278,10 +280,10 @@ attn_fwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
             const int slot0 = c.k * kQ - 64;
 #pragma unroll
             for (int j = 0; j < 2; ++j) {
-                const int e = ptid + j * kProducerThreads;
-                const int sl = slot0 + min(e, kW - 1);         // <= L - 1
+                const int e = ptid + j * kProducerThreads;     // kW = 2 * kProducerThreads
+                const int sl = slot0 + e;                      // <= L - 1
                 const int pl = P[max(sl, 0)];
-                pn[j] = (e < kW && sl >= 0) ? pl : -1;
+                pn[j] = sl >= 0 ? pl : -1;
             }
         };
         if (blockIdx.x < n_tiles) load_pos(blockIdx.x);
@@ -296,24 +298,22 @@ attn_fwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
             if (ptid == 0) LSH_PHASE(0, 0, it, 1);
             Stage &st = sm.st[s];
             const long long rowbase = tile_coord(tile, R, n_k).bh * L;
-#pragma unroll
-            for (int j = 0; j < 2; ++j) {
-                const int e = ptid + j * kProducerThreads;
-                if (e < kW) st.pos[e] = pn[j];
-            }
+            st.pos[ptid] = pn[0];
+            st.pos[ptid + kProducerThreads] = pn[1];
             tc::named_bar_sync(1, kProducerThreads);
             if (tile + gridDim.x < n_tiles) load_pos(tile + gridDim.x);   // overlaps the copies below
             if (ptid == 0) LSH_PHASE(0, 0, it, 2);
-            // x and v rows: thread t copies 16-byte chunk t % 8 of rows t / 8 + 16 j
+            // x and v rows: thread t copies 16-byte chunk t % 8 of rows t / 8 + 12 j
             // (zero fill for a missing slot); every position is read first for ILP
             {
+                constexpr int kRowStep = kProducerThreads / 8;
                 const int ch = ptid & 7, r0 = ptid >> 3;
-                int pr[kW / 16];
+                int pr[kW / kRowStep];
 #pragma unroll
-                for (int j = 0; j < kW / 16; ++j) pr[j] = st.pos[r0 + 16 * j];
+                for (int j = 0; j < kW / kRowStep; ++j) pr[j] = st.pos[r0 + kRowStep * j];
 #pragma unroll
-                for (int j = 0; j < kW / 16; ++j) {
-                    const int row = r0 + 16 * j;
+                for (int j = 0; j < kW / kRowStep; ++j) {
+                    const int row = r0 + kRowStep * j;
                     const uint32_t off = (uint32_t)row * 128u + (uint32_t)((ch ^ (row & 7)) << 4);
                     const long long src = (rowbase + max(pr[j], 0)) * kDim + ch * 8;
                     const uint32_t nb = pr[j] >= 0 ? 16u : 0u;
