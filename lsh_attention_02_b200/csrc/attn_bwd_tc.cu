@@ -72,6 +72,7 @@ struct BwdSmem {
     uint8_t ET[3][kK * 128];        // tau inv_j dS^T, 3 blocks of 64 queries (48 KB)
     uint64_t full[kStages], empty[kStages];
     uint64_t bar_s, bar_p, bar_o, bar_free;
+    uint64_t xchg[4];               // key-role rows staged for the partner warp, per lane quadrant
     uint32_t tmem_base;
     int abort;
 };
@@ -261,6 +262,7 @@ attn_bwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
         tc::mbar_init(&sm.bar_p, kComputeWarps);
         tc::mbar_init(&sm.bar_o, 1);
         tc::mbar_init(&sm.bar_free, kComputeWarps);
+        for (int q = 0; q < 4; ++q) tc::mbar_init(&sm.xchg[q], 1);
         sm.abort = 0;
         tc::fence_mbar_init();
     }
@@ -496,6 +498,8 @@ attn_bwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
             // buffers reuse memory the MMAs no longer read: E^T and this stage's v rows.
             uint8_t *stg = warp < 6 ? reinterpret_cast<uint8_t *>(sm.ET) + warp * 8192
                                     : const_cast<uint8_t *>(st.V) + (warp - 6) * 8192;
+            // Slot kr is both key kr and query kr: its key-role row (from the warp of
+            // half 1) is added to its query-role row (half 0) before one reduction.
             float a[kDim];
             if (half == 0) {
 #pragma unroll
@@ -505,8 +509,24 @@ attn_bwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
 #pragma unroll
                 for (int c = 0; c < 4; ++c) tc::tmem_ld16(tl + cQa + c * 16, a + c * 16);
                 tc::tmem_ld_wait();
-                flush_rows(stg, lane, a, dx_acc, rowbase + kpos);         // query row kr = key slot kr
+                // partner's key-role row staged (bounded wait, as every wait here)
+                if (!tc::mbar_wait(&sm.xchg[quad], ph, &sm.abort, status)) break;
+                const uint8_t *pst = warp + 4 < 6 ? reinterpret_cast<const uint8_t *>(sm.ET) + (warp + 4) * 8192
+                                                  : st.V + (warp + 4 - 6) * 8192;
+#pragma unroll
+                for (int c = 0; c < 16; ++c) {
+                    const float4 g = *reinterpret_cast<const float4 *>(pst + lane * 256 + ((c ^ (lane & 15)) << 4));
+                    a[4 * c] += g.x; a[4 * c + 1] += g.y; a[4 * c + 2] += g.z; a[4 * c + 3] += g.w;
+                }
+                flush_rows(stg, lane, a, dx_acc, rowbase + kpos);
             } else {
+                if (quad >= 2) {                                          // query row 64 + kr (chunk 2k+2)
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) tc::tmem_ld16(tl + cQb + c * 16, a + c * 16);
+                    tc::tmem_ld_wait();
+                    const int qp = __float_as_int(st.qinfo[64 + kr].w);
+                    flush_rows(stg, lane, a, dx_acc, qp >= 0 ? rowbase + qp : -1LL);
+                }
 #pragma unroll
                 for (int c = 0; c < 4; ++c) tc::tmem_ld16(tl + cG + c * 16, a + c * 16);
                 tc::tmem_ld_wait();
@@ -527,14 +547,13 @@ attn_bwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
 #pragma unroll
                     for (int e = 0; e < 8; ++e) a[ch * 8 + e] = fmaf(-cf, xr[e], a[ch * 8 + e]);
                 }
-                flush_rows(stg, lane, a, dx_acc, rowbase + kpos);         // key role of key kr
-                if (quad >= 2) {                                          // query row 64 + kr (chunk 2k+2)
+                // stage the row for the partner warp of half 0 (same layout as flush_rows)
 #pragma unroll
-                    for (int c = 0; c < 4; ++c) tc::tmem_ld16(tl + cQb + c * 16, a + c * 16);
-                    tc::tmem_ld_wait();
-                    const int qp = __float_as_int(st.qinfo[64 + kr].w);
-                    flush_rows(stg, lane, a, dx_acc, qp >= 0 ? rowbase + qp : -1LL);
-                }
+                for (int c = 0; c < 16; ++c)
+                    *reinterpret_cast<float4 *>(stg + lane * 256 + ((c ^ (lane & 15)) << 4)) =
+                        make_float4(a[4 * c], a[4 * c + 1], a[4 * c + 2], a[4 * c + 3]);
+                __syncwarp();
+                if (lane == 0) tc::mbar_arrive(&sm.xchg[quad]);
             }
             if (tid == 0) LSH_PHASE(1, 2, it, 5);
             tc::tc_fence_before();

@@ -156,18 +156,35 @@ hash_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__restr
             __syncwarp();
             if (lane == 0) tc::mbar_arrive(&sm.acc_empty[ab]);
 
-            // pass 1: extremes of the tile
-            float mx = v[0], mn = v[0];
+            // pass 1: extremes of the tile, four independent chains per extreme
+            constexpr int Q = NT / 4;
+            float mxq[4], mnq[4];
 #pragma unroll
-            for (int j = 1; j + 1 < NT; j += 2) { mx = tc::max3f(mx, v[j], v[j + 1]); mn = tc::min3f(mn, v[j], v[j + 1]); }
-            mx = fmaxf(mx, v[NT - 1]);
-            mn = fminf(mn, v[NT - 1]);
+            for (int qq = 0; qq < 4; ++qq) {
+                const int j0 = qq * Q;
+                float a = fmaxf(v[j0], v[j0 + 1]), b = fminf(v[j0], v[j0 + 1]);
+#pragma unroll
+                for (int j = j0 + 2; j < j0 + Q; j += 2) {
+                    a = tc::max3f(a, v[j], v[j + 1]);
+                    b = tc::min3f(b, v[j], v[j + 1]);
+                }
+                mxq[qq] = a;
+                mnq[qq] = b;
+            }
+            const float mx = fmaxf(fmaxf(mxq[0], mxq[1]), fmaxf(mxq[2], mxq[3]));
+            const float mn = fminf(fminf(mnq[0], mnq[1]), fminf(mnq[2], mnq[3]));
             const bool pos = mx >= -mn;
             const float target = pos ? mx : mn;
-            // pass 2: lowest column holding the extreme
-            int js = NT - 1;
+            // pass 2: lowest column holding the extreme (four chains, then the smallest)
+            int jq[4];
 #pragma unroll
-            for (int j = NT - 2; j >= 0; --j) js = (v[j] == target) ? j : js;
+            for (int qq = 0; qq < 4; ++qq) {
+                int jj = NT;
+#pragma unroll
+                for (int j = qq * Q + Q - 1; j >= qq * Q; --j) jj = (v[j] == target) ? j : jj;
+                jq[qq] = jj;
+            }
+            const int js = min(min(jq[0], jq[1]), min(jq[2], jq[3]));
             const int r = it / n_nt, nt = it % n_nt;
             const float tbest = pos ? mx : -mn;
             const int tb = (pos ? 0 : half) + nt * NT + js;

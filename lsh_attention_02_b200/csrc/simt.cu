@@ -202,18 +202,54 @@ __global__ void combine_kernel(const OT *__restrict__ o_r, const float *__restri
     for (int k = 0; k < 4; ++k) y[k] = from_f<T>(acc[k]);
 }
 
+// bf16 round outputs: 8 threads per token, eight features each (16-byte loads
+// and stores); the token's logsumexps are read by every thread of its group.
+__global__ void combine_bf16_kernel(const __nv_bfloat16 *__restrict__ o_r, const float *__restrict__ lse,
+                                    __nv_bfloat16 *__restrict__ out, long long tokens, int L, int R)
+{
+    long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    long long tok = gid >> 3;
+    int oct = (int)(gid & 7);
+    if (tok >= tokens) return;
+    long long bh = tok / L;
+    int i = (int)(tok % L);
+    const float *lp = lse + bh * R * (long long)L + i;
+    float mx = -INFINITY;
+    for (int r = 0; r < R; ++r) mx = fmaxf(mx, lp[(long long)r * L]);
+    float ssum = 0.f;
+    for (int r = 0; r < R; ++r) ssum += expf(lp[(long long)r * L] - mx);
+    const float big = mx + logf(ssum);
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    for (int r = 0; r < R; ++r) {
+        const float wr = expf(lp[(long long)r * L] - big);
+        const uint4 u = reinterpret_cast<const uint4 *>(o_r + ((bh * R + r) * L + i) * kDim)[oct];
+        const uint32_t wd[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            acc[2 * e] = fmaf(wr, __uint_as_float(wd[e] << 16), acc[2 * e]);
+            acc[2 * e + 1] = fmaf(wr, __uint_as_float(wd[e] & 0xFFFF0000u), acc[2 * e + 1]);
+        }
+    }
+    reinterpret_cast<uint4 *>(out + tok * kDim)[oct] =
+        make_uint4(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]), pack_bf16x2(acc[4], acc[5]),
+                   pack_bf16x2(acc[6], acc[7]));
+}
+
 cudaError_t launch_combine(const Problem &p, const void *o_r, bool o_r_bf16, const float *lse, void *out,
                            cudaStream_t st)
 {
+    if (p.dtype == LSH_BF16 && o_r_bf16) {
+        long long threads = p.tokens() * 8;
+        combine_bf16_kernel<<<(unsigned)((threads + 255) / 256), 256, 0, st>>>(
+            (const __nv_bfloat16 *)o_r, lse, (__nv_bfloat16 *)out, p.tokens(), p.L, p.R);
+        return cudaGetLastError();
+    }
     long long threads = p.tokens() * 16;
     unsigned grid = (unsigned)((threads + 255) / 256);
     if (p.dtype == LSH_F32) {
         if (o_r_bf16) return cudaErrorInvalidValue;
         combine_kernel<float, float><<<grid, 256, 0, st>>>((const float *)o_r, lse, (float *)out, p.tokens(), p.L,
                                                            p.R);
-    } else if (o_r_bf16) {
-        combine_kernel<__nv_bfloat16, __nv_bfloat16><<<grid, 256, 0, st>>>(
-            (const __nv_bfloat16 *)o_r, lse, (__nv_bfloat16 *)out, p.tokens(), p.L, p.R);
     } else {
         combine_kernel<__nv_bfloat16, float><<<grid, 256, 0, st>>>((const float *)o_r, lse, (__nv_bfloat16 *)out,
                                                                    p.tokens(), p.L, p.R);
@@ -260,9 +296,55 @@ __global__ void bwd_prep_kernel(const float *__restrict__ lse, const T *__restri
     }
 }
 
+__global__ void bwd_prep_bf16_kernel(const float *__restrict__ lse, const __nv_bfloat16 *__restrict__ out,
+                                     const __nv_bfloat16 *__restrict__ dout, float *__restrict__ lse_all,
+                                     float *__restrict__ delta, float *__restrict__ dx_acc,
+                                     float *__restrict__ dv_acc, long long tokens, int L, int R)
+{
+    long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    long long tok = gid >> 3;
+    int oct = (int)(gid & 7);
+    bool valid = tok < tokens;
+    float part = 0.f;
+    if (valid) {
+        const uint4 yu = reinterpret_cast<const uint4 *>(out + tok * kDim)[oct];
+        const uint4 gu = reinterpret_cast<const uint4 *>(dout + tok * kDim)[oct];
+        const uint32_t yw[4] = {yu.x, yu.y, yu.z, yu.w}, gw[4] = {gu.x, gu.y, gu.z, gu.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            part = fmaf(__uint_as_float(gw[e] << 16), __uint_as_float(yw[e] << 16), part);
+            part = fmaf(__uint_as_float(gw[e] & 0xFFFF0000u), __uint_as_float(yw[e] & 0xFFFF0000u), part);
+        }
+        const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+        float4 *dxp = reinterpret_cast<float4 *>(dx_acc + tok * kDim) + 2 * oct;
+        float4 *dvp = reinterpret_cast<float4 *>(dv_acc + tok * kDim) + 2 * oct;
+        dxp[0] = z; dxp[1] = z; dvp[0] = z; dvp[1] = z;
+    }
+#pragma unroll
+    for (int o = 4; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+    if (valid && oct == 0) {
+        long long bh = tok / L;
+        int i = (int)(tok % L);
+        const float *lp = lse + bh * R * (long long)L + i;
+        float mx = -INFINITY;
+        for (int r = 0; r < R; ++r) mx = fmaxf(mx, lp[(long long)r * L]);
+        float ssum = 0.f;
+        for (int r = 0; r < R; ++r) ssum += expf(lp[(long long)r * L] - mx);
+        lse_all[tok] = mx + logf(ssum);
+        delta[tok] = part;
+    }
+}
+
 cudaError_t launch_bwd_prep(const Problem &p, const float *lse, const void *out, const void *dout,
                             float *lse_all, float *delta, float *dx_acc, float *dv_acc, cudaStream_t st)
 {
+    if (p.dtype == LSH_BF16) {
+        long long threads = p.tokens() * 8;
+        bwd_prep_bf16_kernel<<<(unsigned)((threads + 255) / 256), 256, 0, st>>>(
+            lse, (const __nv_bfloat16 *)out, (const __nv_bfloat16 *)dout, lse_all, delta, dx_acc, dv_acc,
+            p.tokens(), p.L, p.R);
+        return cudaGetLastError();
+    }
     long long threads = p.tokens() * 16;
     unsigned grid = (unsigned)((threads + 255) / 256);
     if (p.dtype == LSH_F32)

@@ -179,6 +179,12 @@ __device__ __forceinline__ void named_bar_sync(int id, int nthreads)
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
+// Arrive (without waiting) on hardware barrier `id` counting `nthreads` threads.
+__device__ __forceinline__ void named_bar_arrive(int id, int nthreads)
+{
+    asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
 // Barrier among `nthreads` threads on hardware barrier `id`; returns the OR of
 // `pred` over the participants (a uniform decision, e.g. to leave a loop).
 __device__ __forceinline__ bool named_bar_or(int id, int nthreads, bool pred)
