@@ -241,6 +241,7 @@ __device__ __forceinline__ TileCoord tile_coord(long long tile, int R, int n_k)
     return c;
 }
 
+template <bool CAUSAL>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_bwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__restrict__ v,
                    const __nv_bfloat16 *__restrict__ dout, const int32_t *__restrict__ perm, const float *__restrict__ invnorm,
@@ -451,40 +452,22 @@ attn_bwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
             if (tid == 0) LSH_PHASE(1, 2, it, 2);
             tc::tc_fence_after();
             // ---- elementwise
-            if (causal) {
-                if (quad < 2) {                      // keys of chunk 2k: queries of chunks 2k, 2k+1
-                    if (half == 0) {
-                        key_row_block<0, true>(st, sm.ET, tl, kr, kpos, kinv, tau);
-                        zero_block<128>(sm.ET, tl, kr);
-                    } else {
-                        key_row_block<64, true>(st, sm.ET, tl, kr, kpos, kinv, tau);
-                    }
-                } else {                             // keys of chunk 2k+1: queries of chunks 2k+1, 2k+2
-                    if (half == 0) {
-                        key_row_block<64, true>(st, sm.ET, tl, kr, kpos, kinv, tau);
-                        zero_block<0>(sm.ET, tl, kr);
-                    } else {
-                        key_row_block<128, true>(st, sm.ET, tl, kr, kpos, kinv, tau);
-                    }
-                }
-                if (half == 0) self_fixup(st, sm.ET, tl, quad, lane, kinv, tau);
-            } else {
-                if (quad < 2) {
-                    if (half == 0) {
-                        key_row_block<0, false>(st, sm.ET, tl, kr, kpos, kinv, tau);
-                        zero_block<128>(sm.ET, tl, kr);
-                    } else {
-                        key_row_block<64, false>(st, sm.ET, tl, kr, kpos, kinv, tau);
-                    }
+            if (quad < 2) {                          // keys of chunk 2k: queries of chunks 2k, 2k+1
+                if (half == 0) {
+                    key_row_block<0, CAUSAL>(st, sm.ET, tl, kr, kpos, kinv, tau);
+                    zero_block<128>(sm.ET, tl, kr);
                 } else {
-                    if (half == 0) {
-                        key_row_block<64, false>(st, sm.ET, tl, kr, kpos, kinv, tau);
-                        zero_block<0>(sm.ET, tl, kr);
-                    } else {
-                        key_row_block<128, false>(st, sm.ET, tl, kr, kpos, kinv, tau);
-                    }
+                    key_row_block<64, CAUSAL>(st, sm.ET, tl, kr, kpos, kinv, tau);
+                }
+            } else {                                 // keys of chunk 2k+1: queries of chunks 2k+1, 2k+2
+                if (half == 0) {
+                    key_row_block<64, CAUSAL>(st, sm.ET, tl, kr, kpos, kinv, tau);
+                    zero_block<0>(sm.ET, tl, kr);
+                } else {
+                    key_row_block<128, CAUSAL>(st, sm.ET, tl, kr, kpos, kinv, tau);
                 }
             }
+            if (CAUSAL && half == 0) self_fixup(st, sm.ET, tl, quad, lane, kinv, tau);
             tc::tmem_st_wait();
             tc::fence_async_smem();
             tc::tc_fence_before();
@@ -520,13 +503,6 @@ attn_bwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
                 }
                 flush_rows(stg, lane, a, dx_acc, rowbase + kpos);
             } else {
-                if (quad >= 2) {                                          // query row 64 + kr (chunk 2k+2)
-#pragma unroll
-                    for (int c = 0; c < 4; ++c) tc::tmem_ld16(tl + cQb + c * 16, a + c * 16);
-                    tc::tmem_ld_wait();
-                    const int qp = __float_as_int(st.qinfo[64 + kr].w);
-                    flush_rows(stg, lane, a, dx_acc, qp >= 0 ? rowbase + qp : -1LL);
-                }
 #pragma unroll
                 for (int c = 0; c < 4; ++c) tc::tmem_ld16(tl + cG + c * 16, a + c * 16);
                 tc::tmem_ld_wait();
@@ -554,6 +530,15 @@ attn_bwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
                         make_float4(a[4 * c], a[4 * c + 1], a[4 * c + 2], a[4 * c + 3]);
                 __syncwarp();
                 if (lane == 0) tc::mbar_arrive(&sm.xchg[quad]);
+                if (quad >= 2) {                                          // query row 64 + kr (chunk 2k+2)
+                    // own buffer in this stage's dY rows, which the MMAs no longer read
+                    uint8_t *stg2 = const_cast<uint8_t *>(st.G) + (quad - 2) * 8192;
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) tc::tmem_ld16(tl + cQb + c * 16, a + c * 16);
+                    tc::tmem_ld_wait();
+                    const int qp = __float_as_int(st.qinfo[64 + kr].w);
+                    flush_rows(stg2, lane, a, dx_acc, qp >= 0 ? rowbase + qp : -1LL);
+                }
             }
             if (tid == 0) LSH_PHASE(1, 2, it, 5);
             tc::tc_fence_before();
@@ -580,14 +565,15 @@ cudaError_t launch_attn_bwd_tc(const Problem &p, const void *x, const void *v, c
                                float *dv_acc, uint32_t *status, cudaStream_t st)
 {
     const size_t smem = sizeof(BwdSmem) + 1024;
-    cudaError_t e = cudaFuncSetAttribute(attn_bwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    auto kern = p.causal ? attn_bwd_tc_kernel<true> : attn_bwd_tc_kernel<false>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const long long n_tiles = p.S() * (p.L / kK);
     const unsigned grid = (unsigned)std::min<long long>(n_tiles, (long long)sms);
-    attn_bwd_tc_kernel<<<grid, kThreads, smem, st>>>((const __nv_bfloat16 *)x, (const __nv_bfloat16 *)v,
+    kern<<<grid, kThreads, smem, st>>>((const __nv_bfloat16 *)x, (const __nv_bfloat16 *)v,
                                                      (const __nv_bfloat16 *)dout, perm, invnorm, lse_all,
                                                      delta, dx_acc, dv_acc, p.L, p.R, n_tiles, p.causal,
                                                      1.0f / sqrtf((float)p.d), status);

@@ -238,6 +238,7 @@ __device__ __forceinline__ void window_norms(Stage &st, int t, float sl2)
     }
 }
 
+template <bool CAUSAL>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_fwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__restrict__ v,
                    const int32_t *__restrict__ perm, __nv_bfloat16 *__restrict__ o_r, float *__restrict__ lse, int L,
@@ -433,18 +434,12 @@ attn_fwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
             const float qinv = st.inv[64 + i];
             // query chunk a (0: 2k, 1: 2k+1) sees window chunks a and a+1
             const int a = i >> 6;
-            const bool self_only = causal && qpos == min(st.cmin[a], st.cmin[a + 1]);
+            const bool self_only = CAUSAL && qpos == min(st.cmin[a], st.cmin[a + 1]);
             const bool first = tcd.k == 0;
             float l, row_lse;
-            if (causal) {
-                if (q >= 2) softmax_row<64, true, false>(st, tl, i, qpos, qinv, self_only, tau, l, row_lse);
-                else if (first) softmax_row<0, true, true>(st, tl, i, qpos, qinv, self_only, tau, l, row_lse);
-                else softmax_row<0, true, false>(st, tl, i, qpos, qinv, self_only, tau, l, row_lse);
-            } else {
-                if (q >= 2) softmax_row<64, false, false>(st, tl, i, qpos, qinv, false, tau, l, row_lse);
-                else if (first) softmax_row<0, false, true>(st, tl, i, qpos, qinv, false, tau, l, row_lse);
-                else softmax_row<0, false, false>(st, tl, i, qpos, qinv, false, tau, l, row_lse);
-            }
+            if (q >= 2) softmax_row<64, CAUSAL, false>(st, tl, i, qpos, qinv, self_only, tau, l, row_lse);
+            else if (first) softmax_row<0, CAUSAL, true>(st, tl, i, qpos, qinv, self_only, tau, l, row_lse);
+            else softmax_row<0, CAUSAL, false>(st, tl, i, qpos, qinv, self_only, tau, l, row_lse);
             tc::tmem_st_wait();
             tc::tc_fence_before();
             __syncwarp();
@@ -493,14 +488,15 @@ cudaError_t launch_attn_fwd_tc(const Problem &p, const void *x, const void *v, c
 {
     (void)invnorm;      // key norms are computed in the kernel from the gathered rows
     const size_t smem = sizeof(FwdSmem) + 1024;
-    cudaError_t e = cudaFuncSetAttribute(attn_fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    auto kern = p.causal ? attn_fwd_tc_kernel<true> : attn_fwd_tc_kernel<false>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const long long n_tiles = p.S() * (p.L / kQ);
     const unsigned grid = (unsigned)std::min<long long>(n_tiles, (long long)sms);
-    attn_fwd_tc_kernel<<<grid, kThreads, smem, st>>>((const __nv_bfloat16 *)x, (const __nv_bfloat16 *)v, perm, o_r, lse, p.L, p.R, n_tiles,
+    kern<<<grid, kThreads, smem, st>>>((const __nv_bfloat16 *)x, (const __nv_bfloat16 *)v, perm, o_r, lse, p.L, p.R, n_tiles,
                                                      p.causal, 1.0f / sqrtf((float)p.d), status);
     return cudaGetLastError();
 }
