@@ -166,6 +166,13 @@ typedef enum {
 LSH_API lsh_status lsh_attn_trace_begin(int32_t capacity);
 LSH_API lsh_status lsh_attn_trace_end(float *ms, int32_t *calls, int32_t *kernels, int32_t n);
 
+/* Self-test of the bounded device-side waits: launches one CTA that waits on a
+ * barrier nothing completes, for `budget_cycles` SM cycles (>= 0).  The wait
+ * gives up, sets the timeout bit in the status word at the start of
+ * `workspace` (any buffer of >= 256 bytes, 256-byte aligned) and the kernel
+ * returns; lsh_attn_poll then reports LSH_ERR_TIMEOUT.  Nothing faults. */
+LSH_API lsh_status lsh_attn_selftest_timeout(void *workspace, int64_t budget_cycles, void *stream);
+
 /* Human-readable name of a status code; never NULL. */
 LSH_API const char *lsh_attn_status_str(lsh_status status);
 

@@ -23,7 +23,8 @@ STATUS = {0: "LSH_OK", -1: "LSH_ERR_ARG", -2: "LSH_ERR_SHAPE", -3: "LSH_ERR_ALIG
           -4: "LSH_ERR_UNSUPPORTED", -5: "LSH_ERR_CUDA", -6: "LSH_ERR_TIMEOUT", -7: "LSH_ERR_WORKSPACE"}
 
 EXPORTED = ("lsh_attn_workspace_size", "lsh_attn_hash", "lsh_attn_sort", "lsh_attn_fwd_sorted", "lsh_attn_fwd",
-            "lsh_attn_bwd", "lsh_attn_poll", "lsh_attn_trace_begin", "lsh_attn_trace_end",
+            "lsh_attn_bwd", "lsh_attn_poll", "lsh_attn_selftest_timeout", "lsh_attn_trace_begin",
+            "lsh_attn_trace_end",
             "lsh_attn_status_str", "lsh_attn_last_error", "lsh_attn_abi_version")
 
 STAGES = ("hash", "sort", "norms", "attn_fwd", "combine", "bwd_prep", "attn_bwd", "bwd_final")
@@ -62,6 +63,7 @@ def load_library(path: str = LIB_PATH):
     L.lsh_attn_fwd.argtypes = [DP, P, P, P, P, P, P, P, S, P]
     L.lsh_attn_bwd.argtypes = [DP, P, P, P, P, P, P, P, P, P, P, S, P]
     L.lsh_attn_poll.argtypes = [P, P]
+    L.lsh_attn_selftest_timeout.argtypes = [P, ctypes.c_int64, P]
     L.lsh_attn_trace_begin.argtypes = [ctypes.c_int32]
     L.lsh_attn_trace_end.argtypes = [ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_int32),
                                      ctypes.POINTER(ctypes.c_int32), ctypes.c_int32]
@@ -157,6 +159,12 @@ def lsh_attn_bwd(desc: Desc, qk, v, R, out, lse, perm, dout, dqk, dv, ws=None):
 def lsh_attn_poll(ws: torch.Tensor) -> int:
     """Synchronises the current stream and returns the device status (0 or LSH_ERR_TIMEOUT)."""
     return int(load_library().lsh_attn_poll(_ptr(ws), _stream(ws)))
+
+
+def lsh_attn_selftest_timeout(ws: torch.Tensor, budget_cycles: int):
+    """Runs the bounded-wait self-test kernel on the current stream (see the header)."""
+    _check(load_library().lsh_attn_selftest_timeout(_ptr(ws), int(budget_cycles), _stream(ws)),
+           "lsh_attn_selftest_timeout")
 
 
 def trace_begin(capacity: int = 4096):

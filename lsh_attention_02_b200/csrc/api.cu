@@ -310,6 +310,16 @@ lsh_status lsh_attn_poll(void *workspace, void *stream)
     return (word & kStatusTimeout) ? LSH_ERR_TIMEOUT : LSH_OK;
 }
 
+lsh_status lsh_attn_selftest_timeout(void *workspace, int64_t budget_cycles, void *stream)
+{
+    if (!workspace) return LSH_ERR_ARG;
+    if (((uintptr_t)workspace & 255u) != 0) return LSH_ERR_ALIGN;
+    if (budget_cycles < 0) return LSH_ERR_ARG;
+    LSH_TRY(launch_wait_selftest((uint32_t *)workspace, (long long)budget_cycles, (cudaStream_t)stream),
+            "wait self-test");
+    return LSH_OK;
+}
+
 lsh_status lsh_attn_trace_begin(int32_t capacity)
 {
     if (capacity < 1 || g_trace.on) return LSH_ERR_ARG;

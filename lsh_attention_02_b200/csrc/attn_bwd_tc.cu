@@ -63,7 +63,10 @@ struct alignas(1024) Stage {
     uint8_t V[kK * 128];            // v rows of the key slots                              16 KB
     uint8_t G[kQ * 128];            // dY rows of the query slots                           24 KB
     alignas(16) int32_t pos[256];   // positions of slots [128k - 64, 128k + 192); -1 if none
-    alignas(16) float4 qinfo[kQ];   // {LSE * log2 e (+inf if none), delta, self flag, position bits}
+    alignas(16) int32_t qpos[kQ];   // original position of each query slot (-1 if none)
+    alignas(16) float qlse2[kQ];    // LSE * log2(e) (+inf if none)
+    alignas(16) float qdelta[kQ];   // dY . y
+    alignas(16) int32_t qlim[kQ];   // causal key bound: position + 1 when the query attends to itself alone
     int32_t cmin[4];                // smallest position of chunks 2k-1 .. 2k+2 (INT_MAX if none)
 };
 
@@ -120,7 +123,8 @@ __device__ __forceinline__ void smem_chunk(const uint8_t *tile, int row, int ch,
 // Elementwise step for key row kr over query columns [C0, C0 + 64): P^T (bf16)
 // into TMEM columns cPT + C0/2, E^T into shared-memory block C0/64.  A
 // candidate is a query at a later original position (causal) or at any other
-// position; a query with no other candidate is patched in by self_fixup.
+// position; a causal query with no other candidate takes its own key.  Query
+// metadata is read four queries per vector load.
 template <int C0, bool CAUSAL>
 __device__ __forceinline__ void key_row_block(const Stage &st, uint8_t (*ET)[kK * 128], uint32_t tl, int kr, int kpos,
                                               float kinv, float tau)
@@ -137,19 +141,27 @@ __device__ __forceinline__ void key_row_block(const Stage &st, uint8_t (*ET)[kK 
         tc::tmem_ld_wait();
         uint32_t pw[16], ew[16];
 #pragma unroll
-        for (int j = 0; j < 32; j += 2) {
-            float pv[2], ev[2];
+        for (int j4 = 0; j4 < 32; j4 += 4) {
+            const int q0 = C0 + h * 32 + j4;
+            // causal: key admitted iff its position < qlim; otherwise iff it differs from the query
+            const int4 qp4 = *reinterpret_cast<const int4 *>(CAUSAL ? &st.qlim[q0] : &st.qpos[q0]);
+            const float4 ql4 = *reinterpret_cast<const float4 *>(&st.qlse2[q0]);
+            const float4 qd4 = *reinterpret_cast<const float4 *>(&st.qdelta[q0]);
+            const int qp[4] = {qp4.x, qp4.y, qp4.z, qp4.w};
+            const float ql[4] = {ql4.x, ql4.y, ql4.z, ql4.w};
+            const float qd[4] = {qd4.x, qd4.y, qd4.z, qd4.w};
+            float pv[4], ev[4];
 #pragma unroll
-            for (int u = 0; u < 2; ++u) {
-                const float4 qi = st.qinfo[C0 + h * 32 + j + u];
-                const int qp = __float_as_int(qi.w);
-                const bool ok = CAUSAL ? (kpos < qp) : (kpos != qp);
-                const float e2 = tc::fast_exp2(fmaf(s[j + u], sc, -qi.x));
+            for (int u = 0; u < 4; ++u) {
+                const bool ok = CAUSAL ? (kpos < qp[u]) : (kpos != qp[u]);
+                const float e2 = tc::fast_exp2(fmaf(s[j4 + u], sc, -ql[u]));
                 pv[u] = ok ? e2 : 0.f;
-                ev[u] = ec * pv[u] * (dp[j + u] - qi.y);
+                ev[u] = ec * pv[u] * (dp[j4 + u] - qd[u]);
             }
-            pw[j / 2] = pack_bf16x2(pv[0], pv[1]);
-            ew[j / 2] = pack_bf16x2(ev[0], ev[1]);
+            pw[j4 / 2] = pack_bf16x2(pv[0], pv[1]);
+            pw[j4 / 2 + 1] = pack_bf16x2(pv[2], pv[3]);
+            ew[j4 / 2] = pack_bf16x2(ev[0], ev[1]);
+            ew[j4 / 2 + 1] = pack_bf16x2(ev[2], ev[3]);
         }
         tc::tmem_st16(tl + cPT + C0 / 2 + h * 16, pw);
         constexpr int blk = C0 / 64;
@@ -160,55 +172,6 @@ __device__ __forceinline__ void key_row_block(const Stage &st, uint8_t (*ET)[kK 
             *reinterpret_cast<uint4 *>(ET[blk] + off) =
                 make_uint4(ew[4 * c4], ew[4 * c4 + 1], ew[4 * c4 + 2], ew[4 * c4 + 3]);
         }
-    }
-}
-
-// Causal queries with no other candidate attend to themselves: for key row kr
-// (< 128) the query of the same slot is column kr.  Where that query is flagged,
-// P^T[kr][kr] = exp(s - LSE) and E^T[kr][kr] = tau inv (P (dY.v - delta)) are
-// written over the zeros key_row_block left.  Run by the warps that own columns
-// [32 quad, 32 quad + 32); tcgen05 loads and stores stay warp-wide.
-__device__ __forceinline__ void self_fixup(const Stage &st, uint8_t (*ET)[kK * 128], uint32_t tl, int quad, int lane,
-                                           float kinv, float tau)
-{
-    const int kr = quad * 32 + lane;
-    const float4 qi = st.qinfo[kr];
-    const bool me = qi.z != 0.f;
-    if (!__any_sync(0xffffffffu, me)) return;
-    const uint32_t cb = (uint32_t)(quad * 32);
-    float sv[32], dv[32];
-    tc::tmem_ld16(tl + cS + cb, sv);
-    tc::tmem_ld16(tl + cS + cb + 16, sv + 16);
-    tc::tmem_ld16(tl + cD + cb, dv);
-    tc::tmem_ld16(tl + cD + cb + 16, dv + 16);
-    tc::tmem_st_wait();
-    float pk[16];
-    tc::tmem_ld16(tl + cPT + cb / 2, pk);
-    tc::tmem_ld_wait();
-    float s_self = 0.f, d_self = 0.f;
-#pragma unroll
-    for (int c = 0; c < 32; ++c) {
-        s_self = (c == lane) ? sv[c] : s_self;
-        d_self = (c == lane) ? dv[c] : d_self;
-    }
-    const float p = tc::fast_exp2(fmaf(s_self, tau * kinv * kLog2e, -qi.x));
-    const float e = tau * kinv * p * (d_self - qi.y);
-    uint32_t u[16];
-#pragma unroll
-    for (int c = 0; c < 16; ++c) {
-        uint32_t w = __float_as_uint(pk[c]);
-        if (me && c == (lane >> 1)) {
-            const __nv_bfloat16 hb = __float2bfloat16_rn(p);
-            const uint32_t hv = (uint32_t)(*reinterpret_cast<const uint16_t *>(&hb));
-            w = (lane & 1) ? ((w & 0x0000FFFFu) | (hv << 16)) : ((w & 0xFFFF0000u) | hv);
-        }
-        u[c] = w;
-    }
-    tc::tmem_st16(tl + cPT + cb / 2, u);
-    if (me) {
-        const int q = kr;                                   // query column of this row's own slot
-        uint8_t *chunk = ET[q >> 6] + kr * 128 + (((((q & 63) >> 3)) ^ (kr & 7)) << 4);
-        reinterpret_cast<__nv_bfloat16 *>(chunk)[q & 7] = __float2bfloat16_rn(e);
     }
 }
 
@@ -357,12 +320,10 @@ attn_bwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
                     const int p = qp[j];
                     const int qa = q >> 6;
                     const int wmin = min(st.cmin[qa], st.cmin[qa + 1]);
-                    float4 qi;
-                    qi.x = p >= 0 ? ql[j] * kLog2e : INFINITY;
-                    qi.y = p >= 0 ? qd[j] : 0.f;
-                    qi.z = (p >= 0 && causal && p == wmin) ? 1.f : 0.f;
-                    qi.w = __int_as_float(p);
-                    st.qinfo[q] = qi;
+                    st.qpos[q] = p;
+                    st.qlse2[q] = p >= 0 ? ql[j] * kLog2e : INFINITY;
+                    st.qdelta[q] = p >= 0 ? qd[j] : 0.f;
+                    st.qlim[q] = (p >= 0 && p == wmin) ? p + 1 : p;
                 }
             }
             if (tile + gridDim.x < n_tiles) load_pos(tile + gridDim.x);
@@ -467,7 +428,6 @@ attn_bwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
                     key_row_block<128, CAUSAL>(st, sm.ET, tl, kr, kpos, kinv, tau);
                 }
             }
-            if (CAUSAL && half == 0) self_fixup(st, sm.ET, tl, quad, lane, kinv, tau);
             tc::tmem_st_wait();
             tc::fence_async_smem();
             tc::tc_fence_before();
@@ -489,11 +449,13 @@ attn_bwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
                 for (int c = 0; c < 4; ++c) tc::tmem_ld16(tl + cDV + c * 16, a + c * 16);
                 tc::tmem_ld_wait();
                 flush_rows(stg, lane, a, dv_acc, rowbase + kpos);
+                if (tid == 0) LSH_PHASE(1, 2, it, 6);
 #pragma unroll
                 for (int c = 0; c < 4; ++c) tc::tmem_ld16(tl + cQa + c * 16, a + c * 16);
                 tc::tmem_ld_wait();
                 // partner's key-role row staged (bounded wait, as every wait here)
                 if (!tc::mbar_wait(&sm.xchg[quad], ph, &sm.abort, status)) break;
+                if (tid == 0) LSH_PHASE(1, 2, it, 7);
                 const uint8_t *pst = warp + 4 < 6 ? reinterpret_cast<const uint8_t *>(sm.ET) + (warp + 4) * 8192
                                                   : st.V + (warp + 4 - 6) * 8192;
 #pragma unroll
@@ -503,9 +465,11 @@ attn_bwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
                 }
                 flush_rows(stg, lane, a, dx_acc, rowbase + kpos);
             } else {
+                if (tid == 128) LSH_PHASE(1, 3, it, 0);
 #pragma unroll
                 for (int c = 0; c < 4; ++c) tc::tmem_ld16(tl + cG + c * 16, a + c * 16);
                 tc::tmem_ld_wait();
+                if (tid == 128) LSH_PHASE(1, 3, it, 1);
                 // key-role correction g - inv^2 (g . x) x, reading x_k from shared memory twice
                 float gx = 0.f;
 #pragma unroll
@@ -530,13 +494,14 @@ attn_bwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
                         make_float4(a[4 * c], a[4 * c + 1], a[4 * c + 2], a[4 * c + 3]);
                 __syncwarp();
                 if (lane == 0) tc::mbar_arrive(&sm.xchg[quad]);
+                if (tid == 128) LSH_PHASE(1, 3, it, 2);
                 if (quad >= 2) {                                          // query row 64 + kr (chunk 2k+2)
                     // own buffer in this stage's dY rows, which the MMAs no longer read
                     uint8_t *stg2 = const_cast<uint8_t *>(st.G) + (quad - 2) * 8192;
 #pragma unroll
                     for (int c = 0; c < 4; ++c) tc::tmem_ld16(tl + cQb + c * 16, a + c * 16);
                     tc::tmem_ld_wait();
-                    const int qp = __float_as_int(st.qinfo[64 + kr].w);
+                    const int qp = st.qpos[64 + kr];
                     flush_rows(stg2, lane, a, dx_acc, qp >= 0 ? rowbase + qp : -1LL);
                 }
             }

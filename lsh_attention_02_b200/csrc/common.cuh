@@ -146,6 +146,8 @@ cudaError_t launch_attn_bwd_tc(const Problem &p, const void *x, const void *v, c
 cudaError_t launch_bwd_finalize(const Problem &p, const float *dx_acc, const float *dv_acc, void *dqk, void *dv,
                                 cudaStream_t st);
 
+cudaError_t launch_wait_selftest(uint32_t *status, long long budget, cudaStream_t st);
+
 // Status bits written by kernels into Workspace::status.
 constexpr uint32_t kStatusTimeout = 1u;
 

@@ -221,3 +221,17 @@ def test_workload_half_million_sampled():
         y = (wts[:, :, None] * o_r).sum(0)
         assert_close(out[0, h, pos], y, "bf16", f"half_million out h={h}")
     _flip_report("half_million sampled", flips, w.H * w.n_hashes * 1024)
+
+
+# ------------------------------------------------------------------ failure detection
+def test_bounded_wait_reports_timeout():
+    """A device wait that nothing completes gives up after its budget and the
+    status word reports it; the context stays usable."""
+    ws = torch.zeros(1024, dtype=torch.uint8, device="cuda")
+    assert lsh.lsh_attn_poll(ws) == 0
+    lsh.lsh_attn_selftest_timeout(ws, 2_000_000)          # about a millisecond
+    assert lsh.lsh_attn_poll(ws) == -6                     # LSH_ERR_TIMEOUT
+    assert lsh.lsh_attn_poll(ws) == 0                      # cleared by the poll
+    w = small("long_64k", B=1, H=1, L=256, backward=False)
+    run = Run(synth.make_inputs(w), w.n_buckets, w.chunk, w.causal, w.dtype)
+    assert torch.isfinite(run.out.float()).all()
