@@ -115,6 +115,49 @@ LSH_API lsh_status lsh_attn_hash(const lsh_attn_desc *desc, const void *qk, cons
 LSH_API lsh_status lsh_attn_sort(const lsh_attn_desc *desc, const uint16_t *buckets, int32_t *perm,
                          void *workspace, size_t ws_bytes, void *stream);
 
+/* Upper bound on the scratch that lsh_attn_sort_static can use (bytes, per
+ * device). */
+#define LSH_ATTN_SORT_STATIC_MAX_BYTES ((size_t)16 << 20)
+
+/* Allocation-free sort.  The paper has no counterpart: it is a library
+ * convenience, not a step of the method.  It computes exactly what
+ * lsh_attn_sort computes (same kernels, same perm), but takes no workspace:
+ * its scratch (first-pass keys and positions, per-tile digit counters) lives
+ * in one fixed device array of LSH_ATTN_SORT_STATIC_MAX_BYTES per device,
+ * which is part of the library's static device memory.
+ *
+ * Who needs it: a caller that must not allocate device memory when it sorts,
+ * or has no allocator at hand.  Examples: code that runs inside a memory
+ * pool's own callbacks (allocating there would re-enter the pool), a service
+ * that fixes its memory footprint at start-up and forbids allocation
+ * afterwards, or a plain C caller that holds device pointers handed to it by
+ * another component but no way to obtain a workspace.  The call makes no
+ * cudaMalloc/cudaFree and calls no library that allocates.
+ *
+ * Set-up: the first call on each device looks up the array's device address
+ * (cudaGetSymbolAddress), which may make the CUDA runtime load the library's
+ * device code; later calls on that device reuse the cached address.  Make the
+ * first call on each device before any stream capture begins.
+ *
+ * Sizes: the scratch needed grows with B*H*n_hashes*L (6 bytes per position
+ * when n_buckets > 256, plus a few counters per 2048 positions).  A
+ * descriptor that needs more than LSH_ATTN_SORT_STATIC_MAX_BYTES is rejected
+ * with LSH_ERR_WORKSPACE before anything is launched, and
+ * lsh_attn_last_error() names the bytes needed and the limit; use
+ * lsh_attn_sort with a workspace for such sizes.  Other argument errors are
+ * those of lsh_attn_sort.
+ *
+ * Nothing in the scratch needs to start at zero: every pass writes each
+ * counter and each slot before reading it.
+ *
+ * Concurrency: all calls on one device share the same array.  Two calls
+ * whose kernels can overlap in time (different streams without ordering
+ * between them, or different host threads on unordered streams) race on it
+ * and produce wrong permutations.  Issue calls on one device in stream order.
+ */
+LSH_API lsh_status lsh_attn_sort_static(const lsh_attn_desc *desc, const uint16_t *buckets, int32_t *perm,
+                                        void *stream);
+
 /* Attention + round merge for a GIVEN permutation ("LSH Attention" output
  * equation, "Multiple Hash Rounds"): gathers rows in sorted order, runs the
  * chunked attention of every round, merges the rounds into out, and writes

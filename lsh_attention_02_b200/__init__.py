@@ -22,7 +22,7 @@ IMPL_AUTO, IMPL_SIMT, IMPL_TC = 0, 1, 2
 STATUS = {0: "LSH_OK", -1: "LSH_ERR_ARG", -2: "LSH_ERR_SHAPE", -3: "LSH_ERR_ALIGN",
           -4: "LSH_ERR_UNSUPPORTED", -5: "LSH_ERR_CUDA", -6: "LSH_ERR_TIMEOUT", -7: "LSH_ERR_WORKSPACE"}
 
-EXPORTED = ("lsh_attn_workspace_size", "lsh_attn_hash", "lsh_attn_sort", "lsh_attn_fwd_sorted", "lsh_attn_fwd",
+EXPORTED = ("lsh_attn_workspace_size", "lsh_attn_hash", "lsh_attn_sort", "lsh_attn_sort_static", "lsh_attn_fwd_sorted", "lsh_attn_fwd",
             "lsh_attn_bwd", "lsh_attn_poll", "lsh_attn_selftest_timeout", "lsh_attn_trace_begin",
             "lsh_attn_trace_end",
             "lsh_attn_status_str", "lsh_attn_last_error", "lsh_attn_abi_version")
@@ -59,6 +59,7 @@ def load_library(path: str = LIB_PATH):
     L.lsh_attn_workspace_size.restype = S
     L.lsh_attn_hash.argtypes = [DP, P, P, P, P, S, P]
     L.lsh_attn_sort.argtypes = [DP, P, P, P, S, P]
+    L.lsh_attn_sort_static.argtypes = [DP, P, P, P]
     L.lsh_attn_fwd_sorted.argtypes = [DP, P, P, P, P, P, P, S, P]
     L.lsh_attn_fwd.argtypes = [DP, P, P, P, P, P, P, P, S, P]
     L.lsh_attn_bwd.argtypes = [DP, P, P, P, P, P, P, P, P, P, P, S, P]
@@ -130,6 +131,17 @@ def lsh_attn_sort(desc: Desc, buckets, perm, ws=None):
     ws = _ws(desc, False, buckets, ws)
     _check(load_library().lsh_attn_sort(ctypes.byref(desc), _ptr(buckets), _ptr(perm), _ptr(ws), ws.numel(),
                                          _stream(buckets)), "lsh_attn_sort")
+    return perm
+
+
+def lsh_attn_sort_static(desc: Desc, buckets, perm):
+    """Same result as lsh_attn_sort, with the library's fixed per-device
+    scratch instead of a workspace (no allocation; calls on one device must
+    not overlap in time)."""
+    rc = load_library().lsh_attn_sort_static(ctypes.byref(desc), _ptr(buckets), _ptr(perm), _stream(buckets))
+    if rc == -7:
+        raise LshAttnError(rc, "lsh_attn_sort_static", load_library().lsh_attn_last_error().decode())
+    _check(rc, "lsh_attn_sort_static")
     return perm
 
 

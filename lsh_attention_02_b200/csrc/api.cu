@@ -224,6 +224,31 @@ lsh_status lsh_attn_sort(const lsh_attn_desc *desc, const uint16_t *buckets, int
     return LSH_OK;
 }
 
+lsh_status lsh_attn_sort_static(const lsh_attn_desc *desc, const uint16_t *buckets, int32_t *perm, void *stream)
+{
+    Problem p;
+    Choice c;
+    lsh_status s;
+    if ((s = check_desc(desc, &p)) != LSH_OK) return s;
+    if ((s = choose(desc, p, &c)) != LSH_OK) return s;
+    if (!buckets || !perm) return LSH_ERR_ARG;
+    size_t need = 0;
+    plan_sort_scratch(p, nullptr, &need);
+    if (need > kStaticSortScratchBytes) {
+        snprintf(g_last_error, sizeof(g_last_error),
+                 "lsh_attn_sort_static: needs %zu bytes of scratch, limit is %zu; use lsh_attn_sort", need,
+                 kStaticSortScratchBytes);
+        return LSH_ERR_WORKSPACE;
+    }
+    void *base = nullptr;
+    LSH_TRY(static_sort_scratch(&base), "lsh_attn_sort_static: scratch address");
+    const Workspace w = plan_sort_scratch(p, (char *)base, nullptr);
+    cudaStream_t st = (cudaStream_t)stream;
+    LSH_TRY(staged(LSH_STAGE_SORT, 3 * make_sort_plan(p.nb, p.L).passes, st,
+                   [&] { return launch_sort(p, buckets, perm, w, st); }), "sort_static");
+    return LSH_OK;
+}
+
 lsh_status lsh_attn_fwd_sorted(const lsh_attn_desc *desc, const void *qk, const void *v, const int32_t *perm,
                                void *out, float *lse, void *workspace, size_t ws_bytes, void *stream)
 {

@@ -54,6 +54,13 @@ struct Workspace {
 // Lays the workspace out from `base` (or from 0 when base is null, to size it).
 Workspace plan_workspace(const Problem &p, bool backward, bool tc_attn, bool tc_hash, char *base);
 
+// Fixed-size sort scratch of lsh_attn_sort_static (bytes per device).
+constexpr size_t kStaticSortScratchBytes = LSH_ATTN_SORT_STATIC_MAX_BYTES;
+// Lays out only the sort fields (keys, values, counters) from `base`; *bytes = total.
+Workspace plan_sort_scratch(const Problem &p, char *base, size_t *bytes);
+// Device address of this device's fixed sort scratch (looked up on first use).
+cudaError_t static_sort_scratch(void **ptr);
+
 // ---------------------------------------------------------------- helpers
 __device__ __forceinline__ float to_f(float a) { return a; }
 __device__ __forceinline__ float to_f(__nv_bfloat16 a) { return __bfloat162float(a); }

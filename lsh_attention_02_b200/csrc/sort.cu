@@ -16,6 +16,8 @@
 //           element is written at offset + rank.
 // Pass 0 reads the bucket ids in position order with the position as the
 // value; the last pass writes only the values, i.e. the permutation.
+#include <mutex>
+
 #include "common.cuh"
 
 namespace lsh {
@@ -169,6 +171,52 @@ cudaError_t launch_sort(const Problem &p, const uint16_t *buckets, int32_t *perm
         vin = ws.sort_vals;
     }
     return cudaGetLastError();
+}
+
+// ------------------------------------------------------------ fixed scratch
+// Scratch of lsh_attn_sort_static: one array per device, part of this
+// module's static device memory, so the entry point itself never allocates.
+// The driver creates it when the module is loaded; its address is looked up
+// once per device and cached.
+static __device__ __align__(256) unsigned char g_sort_scratch[kStaticSortScratchBytes];
+
+Workspace plan_sort_scratch(const Problem &p, char *base, size_t *bytes)
+{
+    Workspace w{};
+    size_t off = 0;
+    auto take = [&](size_t n) -> char * {
+        char *ptr = base ? base + off : nullptr;
+        off = (off + n + 255) / 256 * 256;
+        return ptr;
+    };
+    const size_t S = (size_t)p.S(), L = (size_t)p.L;
+    const SortPlan sp = make_sort_plan(p.nb, p.L);
+    w.sort_keys = (uint16_t *)take(sp.passes > 1 ? S * L * sizeof(uint16_t) : 0);
+    w.sort_vals = (int32_t *)take(sp.passes > 1 ? S * L * sizeof(int32_t) : 0);
+    w.sort_counts = (uint32_t *)take(S * (size_t)sp.max_radix * sp.n_tiles * sizeof(uint32_t));
+    w.bytes = off;
+    if (bytes) *bytes = off;
+    return w;
+}
+
+cudaError_t static_sort_scratch(void **ptr)
+{
+    constexpr int kMaxDevices = 64;
+    static std::mutex mu;
+    static void *addr[kMaxDevices] = {};
+    int dev = -1;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!addr[dev]) {
+        void *a = nullptr;
+        e = cudaGetSymbolAddress(&a, g_sort_scratch);
+        if (e != cudaSuccess) return e;
+        addr[dev] = a;
+    }
+    *ptr = addr[dev];
+    return cudaSuccess;
 }
 
 }  // namespace lsh
