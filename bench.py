@@ -66,6 +66,35 @@ def algorithmic(w: synth.Workload) -> dict:
     return {"bytes": bh * (fwd + bwd), "attn_flops": attn_flops, "hash_flops": hash_flops, "kernel_bytes": kern}
 
 
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one launch, from
+# one ncu capture of the kernel on the named workload (summarised under
+# profiles/).  A record counts only while the kernel's sources hash to the
+# value taken with it; after any change the traffic is reported as null.
+NCU_TRAFFIC = {
+    ("long_64k", "attn_bwd"): {"bytes": 750_689_536, "files": ("attn_bwd_tc.cu", "tc_common.cuh", "common.cuh"),
+                               "sha256": "ea743f565d90f0177c5f88393831a155fe8645a356e082cb002720884f486faa"},
+    ("long_64k", "attn_fwd"): {"bytes": 368_524_032, "files": ("attn_fwd_tc.cu", "tc_common.cuh", "common.cuh"),
+                               "sha256": "b8d8ee19bf7f8d9c4e776564e7005764dec97c42c7cee0391ca2af6bf8505d33"},
+    ("long_64k", "hash"): {"bytes": 68_290_560, "files": ("hash_tc.cu", "tc_common.cuh", "common.cuh"),
+                           "sha256": "8bb118e6381c44c159c320ff3dcadba86676c55af3af2c336ff7574987e94010"},
+}
+
+
+def ncu_traffic(workload: str, kernel: str):
+    rec = NCU_TRAFFIC.get((workload, kernel))
+    if rec is None:
+        return None
+    import hashlib
+    h = hashlib.sha256()
+    for f in rec["files"]:
+        path = os.path.join(ROOT, "lsh_attention_02_b200", "csrc", f)
+        if not os.path.exists(path):
+            return None
+        with open(path, "rb") as fh:
+            h.update(fh.read())
+    return float(rec["bytes"]) if h.hexdigest() == rec["sha256"] else None
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -247,7 +276,8 @@ def run_ours(args, w: synth.Workload, rank: int, world: int) -> dict | None:
                    "parallelism": f"{world} independent replica(s), no collective",
                    "l2": "flushed between timed steps (256 MiB memset outside the step events)"},
         "roofline": {"bound": "hbm", "kernel": dom_name, "achieved": achieved, "peak": hbm, "unit": "GB/s",
-                     "frac": achieved / hbm, "peak_source": f"{peak_src} hbm_gbs", "traffic": None,
+                     "frac": achieved / hbm, "peak_source": f"{peak_src} hbm_gbs",
+                     "traffic": ncu_traffic(w.name, dom_name),
                      "bytes_per_launch": dom_bytes, "launch_ms": dom_launch_ms},
         "roofline_step": {"algorithmic_bytes": alg["bytes"], "achieved_gbs": step_bytes_gbs,
                           "attn_flops": alg["attn_flops"], "hash_flops": alg["hash_flops"],
