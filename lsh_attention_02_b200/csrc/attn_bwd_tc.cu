@@ -90,13 +90,15 @@ __device__ __forceinline__ void red_add_v4(float *addr, float a, float b, float 
 // rowg < 0) with coalesced vector reductions: the warp's 32 rows go through
 // its 8 KB staging buffer (16-byte chunks swizzled by lane against bank
 // conflicts), then each reduction instruction covers two whole rows.
-__device__ __forceinline__ void flush_rows(uint8_t *stg, int lane, const float *a, float *acc, long long rowg)
+__device__ __forceinline__ void flush_rows(uint8_t *stg, int lane, const float *a, float *acc, long long rowg,
+                                           int ph_role = -1, int ph_it = 0, int ph_ev = 0)
 {
 #pragma unroll
     for (int c = 0; c < 16; ++c)
         *reinterpret_cast<float4 *>(stg + lane * 256 + ((c ^ (lane & 15)) << 4)) =
             make_float4(a[4 * c], a[4 * c + 1], a[4 * c + 2], a[4 * c + 3]);
     __syncwarp();
+    if (ph_role >= 0 && lane == 0) LSH_PHASE(1, ph_role, ph_it, ph_ev);
     const int c = lane & 15;
 #pragma unroll 4
     for (int it = 0; it < 16; ++it) {
@@ -106,6 +108,7 @@ __device__ __forceinline__ void flush_rows(uint8_t *stg, int lane, const float *
         if (rg >= 0) red_add_v4(acc + rg * kDim + 4 * c, val.x, val.y, val.z, val.w);
     }
     __syncwarp();
+    if (ph_role >= 0 && lane == 0) LSH_PHASE(1, ph_role, ph_it, ph_ev + 1);
 }
 
 // Chunk `ch` (elements 8ch .. 8ch+7) of bf16 row `row` of a K-major SW128 tile.
@@ -445,14 +448,18 @@ attn_bwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
             // half 1) is added to its query-role row (half 0) before one reduction.
             float a[kDim];
             if (half == 0) {
+                const int prole = warp == 0 ? 4 : warp == 2 ? 5 : -1;
+                if (prole >= 0 && lane == 0) LSH_PHASE(1, prole, it, 0);
 #pragma unroll
                 for (int c = 0; c < 4; ++c) tc::tmem_ld16(tl + cDV + c * 16, a + c * 16);
                 tc::tmem_ld_wait();
-                flush_rows(stg, lane, a, dv_acc, rowbase + kpos);
+                if (prole >= 0 && lane == 0) LSH_PHASE(1, prole, it, 1);
+                flush_rows(stg, lane, a, dv_acc, rowbase + kpos, prole, it, 2);
                 if (tid == 0) LSH_PHASE(1, 2, it, 6);
 #pragma unroll
                 for (int c = 0; c < 4; ++c) tc::tmem_ld16(tl + cQa + c * 16, a + c * 16);
                 tc::tmem_ld_wait();
+                if (prole >= 0 && lane == 0) LSH_PHASE(1, prole, it, 4);
                 // partner's key-role row staged (bounded wait, as every wait here)
                 if (!tc::mbar_wait(&sm.xchg[quad], ph, &sm.abort, status)) break;
                 if (tid == 0) LSH_PHASE(1, 2, it, 7);
@@ -463,7 +470,8 @@ attn_bwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
                     const float4 g = *reinterpret_cast<const float4 *>(pst + lane * 256 + ((c ^ (lane & 15)) << 4));
                     a[4 * c] += g.x; a[4 * c + 1] += g.y; a[4 * c + 2] += g.z; a[4 * c + 3] += g.w;
                 }
-                flush_rows(stg, lane, a, dx_acc, rowbase + kpos);
+                if (prole >= 0 && lane == 0) LSH_PHASE(1, prole, it, 5);
+                flush_rows(stg, lane, a, dx_acc, rowbase + kpos, prole, it, 6);
             } else {
                 if (tid == 128) LSH_PHASE(1, 3, it, 0);
 #pragma unroll
@@ -501,8 +509,9 @@ attn_bwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
 #pragma unroll
                     for (int c = 0; c < 4; ++c) tc::tmem_ld16(tl + cQb + c * 16, a + c * 16);
                     tc::tmem_ld_wait();
+                    if (warp == 6 && lane == 0) LSH_PHASE(1, 6, it, 0);
                     const int qp = st.qpos[64 + kr];
-                    flush_rows(stg2, lane, a, dx_acc, qp >= 0 ? rowbase + qp : -1LL);
+                    flush_rows(stg2, lane, a, dx_acc, qp >= 0 ? rowbase + qp : -1LL, warp == 6 ? 6 : -1, it, 1);
                 }
             }
             if (tid == 0) LSH_PHASE(1, 2, it, 5);

@@ -36,7 +36,7 @@
 //                   softmax overlaps the other's MMAs and stores;
 //   warps 8-10      producer: positions (loaded a tile ahead) and window
 //                   minima; x and v rows by 16-byte cp.async (eight threads
-//                   per row, zero fill for a missing slot) into a 3-stage
+//                   per row, zero fill for a missing slot) into a 4-stage
 //                   shared-memory ring; a stage is published once the next
 //                   stage's copies are in flight;
 //   warp 11         MMA issuer.
@@ -48,7 +48,7 @@ namespace {
 
 constexpr int kQ = 128;             // query slots per tile
 constexpr int kW = 192;             // window rows (keys)
-constexpr int kStages = 3;
+constexpr int kStages = 4;
 constexpr int kSoftmaxWarps = 8;   // two groups of four
 constexpr int kProducerWarps = 3;
 constexpr int kProducerThreads = kProducerWarps * 32;

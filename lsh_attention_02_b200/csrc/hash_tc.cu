@@ -19,7 +19,8 @@
 // Epilogue per N-tile of NT columns held in registers: pass 1 takes the
 // max and min with 3-input min/max; the larger of max and -min decides the
 // side ([+xR] wins an exact tie, as its indices come first); pass 2 finds the
-// lowest column equal to that extreme.  Tiles merge in index order, so the
+// lowest column equal to that extreme with exact 0/1 flags from saturating
+// FMAs (see the epilogue).  Tiles merge in index order, so the
 // result is the first maximum of [xR ; -xR], the oracle's tie rule.
 #include "tc_common.cuh"
 
@@ -73,6 +74,7 @@ hash_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__restr
     const long long row0 = (long long)blockIdx.x * kRows;
     const int n_nt = half / NT;
     const int items = rounds * n_nt;
+    if (threadIdx.x == 0) LSH_PHASE(0, 3, 0, 0);
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) { tc::mbar_init(&sm.full[s], 1); tc::mbar_init(&sm.empty[s], 1); }
@@ -95,6 +97,7 @@ hash_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__restr
     __syncthreads();
     tc::tc_fence_after();
     const uint32_t tmem = sm.tmem_base;
+    if (threadIdx.x == 0) LSH_PHASE(0, 3, 0, 1);
 
     if (warp == kEpiWarps) {
         // ---------------- producer
@@ -102,7 +105,9 @@ hash_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__restr
             for (int it = 0; it < items; ++it) {
                 const int s = it % kStages;
                 const uint32_t ph = (uint32_t)(it / kStages) & 1u;
+                LSH_PHASE(0, 1, it, 0);
                 if (it >= kStages && !tc::mbar_wait(&sm.empty[s], ph ^ 1u, &sm.abort, status)) break;
+                LSH_PHASE(0, 1, it, 1);
                 const int r = it / n_nt, nt = it % n_nt;
                 const __nv_bfloat16 *src = Rs + ((long long)r * half + (long long)nt * NT) * kDim;
                 tc::mbar_arrive_expect_tx(&sm.full[s], NT * 128);
@@ -119,8 +124,11 @@ hash_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__restr
                 const uint32_t ph = (uint32_t)(it / kStages) & 1u;
                 const int ab = it & 1;
                 const uint32_t aph = (uint32_t)(it >> 1) & 1u;
+                LSH_PHASE(0, 2, it, 0);
                 if (!tc::mbar_wait(&sm.full[s], ph, &sm.abort, status)) break;
+                LSH_PHASE(0, 2, it, 1);
                 if (it >= 2 && !tc::mbar_wait(&sm.acc_empty[ab], aph ^ 1u, &sm.abort, status)) break;
+                LSH_PHASE(0, 2, it, 2);
                 tc::tc_fence_after();
                 const uint32_t b0 = tc::smem_u32(sm.B[s]);
 #pragma unroll
@@ -133,6 +141,7 @@ hash_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__restr
                 }
                 tc::mma_commit(&sm.empty[s]);
                 tc::mma_commit(&sm.acc_full[ab]);
+                LSH_PHASE(0, 2, it, 3);
             }
         }
     } else {
@@ -146,7 +155,9 @@ hash_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__restr
         for (int it = 0; it < items; ++it) {
             const int ab = it & 1;
             const uint32_t aph = (uint32_t)(it >> 1) & 1u;
+            if (threadIdx.x == 0) LSH_PHASE(0, 0, it, 0);
             if (!tc::mbar_wait(&sm.acc_full[ab], aph, &sm.abort, status)) break;
+            if (threadIdx.x == 0) LSH_PHASE(0, 0, it, 1);
             tc::tc_fence_after();
             float v[NT];
 #pragma unroll
@@ -155,6 +166,7 @@ hash_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__restr
             tc::tc_fence_before();
             __syncwarp();
             if (lane == 0) tc::mbar_arrive(&sm.acc_empty[ab]);
+            if (threadIdx.x == 0) LSH_PHASE(0, 0, it, 2);
 
             // pass 1: extremes of the tile, four independent chains per extreme
             constexpr int Q = NT / 4;
@@ -175,20 +187,54 @@ hash_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__restr
             const float mn = fminf(fminf(mnq[0], mnq[1]), fminf(mnq[2], mnq[3]));
             const bool pos = mx >= -mn;
             const float target = pos ? mx : mn;
-            // pass 2: lowest column holding the extreme (four chains, then the smallest)
-            int jq[4];
+            // pass 2: lowest column holding the extreme.  U = |extreme| bounds every
+            // |v| of the tile; with B = 2^(24 - e(U)), (U - side * v_j) * B is exactly
+            // 0 where v_j is the extreme and at least 1 elsewhere (the closest float
+            // below U is 2^(e(U) - 24) away), so a saturating FMA gives a 0/1 flag
+            // without a compare.  Sixteen flags per chain are summed as the bits of
+            // an integer kept in the mantissa of 2^23 + sum (exact), and the first
+            // clear bit is the column.  This runs on the FMA pipe while pass 1 uses
+            // the ALU pipe.  Extremes below 2^-103 (B would not be finite) take the
+            // compare-and-select form.
+            if (threadIdx.x == 0) LSH_PHASE(0, 0, it, 3);
+            const float U = pos ? mx : -mn;
+            const int be = (__float_as_int(U) >> 23) & 0xFF;
+            int js;
+            if (__any_sync(0xffffffffu, U != 0.f && be < 24)) {
+                int jq[4];
 #pragma unroll
-            for (int qq = 0; qq < 4; ++qq) {
-                int jj = NT;
+                for (int qq = 0; qq < 4; ++qq) {
+                    int jj = NT;
 #pragma unroll
-                for (int j = qq * Q + Q - 1; j >= qq * Q; --j) jj = (v[j] == target) ? j : jj;
-                jq[qq] = jj;
+                    for (int j = qq * Q + Q - 1; j >= qq * Q; --j) jj = (v[j] == target) ? j : jj;
+                    jq[qq] = jj;
+                }
+                js = min(min(jq[0], jq[1]), min(jq[2], jq[3]));
+            } else {
+                const float B = __int_as_float(min(278 - be, 253) << 23);
+                const float nsB = pos ? -B : B;
+                const float UB = U * B;
+                constexpr int NC = NT / 16;
+                float acc[NC];
+#pragma unroll
+                for (int c = 0; c < NC; ++c) acc[c] = 8388608.f;
+#pragma unroll
+                for (int k = 0; k < 16; ++k)
+#pragma unroll
+                    for (int c = 0; c < NC; ++c)
+                        acc[c] = fmaf(tc::fma_sat(v[c * 16 + k], nsB, UB), (float)(1 << k), acc[c]);
+                js = NT;
+#pragma unroll
+                for (int c = NC - 1; c >= 0; --c) {
+                    const uint32_t eq = ~__float_as_uint(acc[c]) & 0xFFFFu;
+                    js = eq ? c * 16 + __ffs((int)eq) - 1 : js;
+                }
             }
-            const int js = min(min(jq[0], jq[1]), min(jq[2], jq[3]));
             const int r = it / n_nt, nt = it % n_nt;
             const float tbest = pos ? mx : -mn;
             const int tb = (pos ? 0 : half) + nt * NT + js;
             if (tbest > best || (tbest == best && tb < bucket)) { best = tbest; bucket = tb; }
+            if (threadIdx.x == 0) LSH_PHASE(0, 0, it, 4);
             if (nt == n_nt - 1) {
                 if (g < rows_total) {
                     const long long bh = g / L;
@@ -203,6 +249,7 @@ hash_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__restr
 
     tc::tc_fence_before();
     __syncthreads();
+    if (threadIdx.x == 0) LSH_PHASE(0, 3, 0, 2);
     if (warp == 0) {
         tc::tc_fence_after();
         tc::tmem_dealloc(tmem, kTmemCols);
@@ -258,3 +305,5 @@ cudaError_t launch_hash_tc(const Problem &p, const void *x, const void *R, uint1
 }
 
 }  // namespace lsh
+
+LSH_PHASE_EXPORT(hash)

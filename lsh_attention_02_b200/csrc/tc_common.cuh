@@ -25,7 +25,7 @@
 // LSH_PHASE_EXPORT(name) defines lsh_attn_phase_trace_<name>(out) to copy it
 // to the host.  Compiled out otherwise.
 #ifdef LSH_PHASE_TRACE
-static __device__ long long lsh_phase_trace[4][32][8];
+static __device__ long long lsh_phase_trace[8][32][8];
 #define LSH_PHASE(kern, role, it, ev)                                                             \
     do {                                                                                          \
         if (blockIdx.x == 0 && (it) >= 0 && (it) < 32) lsh_phase_trace[role][it][ev] = clock64(); \
@@ -346,6 +346,13 @@ __device__ __forceinline__ float min3f(float a, float b, float c)
 {
     float r;
     asm("min.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+// a * b + c rounded once, clamped to [0, 1]
+__device__ __forceinline__ float fma_sat(float a, float b, float c)
+{
+    float r;
+    asm("fma.rn.sat.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
     return r;
 }
 

@@ -81,6 +81,55 @@ def test_hash_bit_exact_up_to_near_ties(impl, dtype, nb, nh):
     _flip_report(f"hash {dtype} nb={nb}", flips, 4 * nh * w.L)
 
 
+@pytest.mark.parametrize("impl", IMPLS)
+def test_hash_extreme_magnitudes_and_exact_ties(impl):
+    """Rows by blocks of 128 (whole warps alike): zero rows, signed one-hot rows
+    (the projection is a row of R exactly, so equal bf16 entries make exact ties
+    that must go to the lowest index), and Gaussian rows scaled by 2^-110, 2^-60
+    and 2^40; one block mixes 2^-110 rows with plain ones.  Zero and one-hot rows
+    must match bit for bit; the others up to near ties."""
+    nb, nh, L = 1024, 2, 1024
+    w = small("bf16_causal_4k", B=1, H=2, L=L, n_buckets=nb, n_hashes=nh)
+    inp = synth.make_inputs(w)
+    x = inp["x"].astype(np.float64).copy()
+    exact = np.zeros((2, L), dtype=bool)
+    for h in range(2):
+        for i in range(L):
+            blk = i // 128
+            onehot = np.zeros(64)
+            onehot[(i * 7 + h) % 64] = 1.0
+            if blk == 0:
+                x[0, h, i] = 0.0
+            elif blk == 1:
+                x[0, h, i] = onehot * 2.0 ** (i % 3 - 1)
+            elif blk == 2:
+                x[0, h, i] *= 2.0 ** -110
+            elif blk == 3:
+                x[0, h, i] *= 2.0 ** -60
+            elif blk == 4:
+                x[0, h, i] *= 2.0 ** 40
+            elif blk == 5:
+                x[0, h, i] = onehot * 2.0 ** -110
+            elif blk == 6:
+                x[0, h, i] *= 2.0 ** -110 if i % 2 == 0 else 1.0
+            else:
+                x[0, h, i] = -onehot
+            exact[h, i] = blk in (0, 1, 5, 7)
+    xd = to_dev(x.astype(np.float32), "bf16"); R = to_dev(inp["R"], "bf16")
+    desc = lsh.desc_for(xd, nb, nh, 64, True, impl)
+    bk = torch.empty((1, 2, nh, L), dtype=torch.int16, device="cuda")
+    lsh.lsh_attn_hash(desc, xd, R, bk)
+    gb = bk.cpu().numpy().view(np.uint16).astype(np.int64)
+    flips = 0
+    for h in range(2):
+        for r in range(nh):
+            ob, mg = oracle.hash_round(x[0, h].astype(np.float32), inp["R"][r], nb)
+            e = exact[h]
+            np.testing.assert_array_equal(gb[0, h, r][e], ob[e], err_msg=f"exact rows h={h} r={r}")
+            flips += check_buckets(gb[0, h, r][~e], ob[~e], mg[~e], f"scaled rows h={h} r={r}")
+    _flip_report("hash extreme magnitudes", flips, 2 * nh * L)
+
+
 # ------------------------------------------------------------------ stage: sort
 @pytest.mark.parametrize("L,nb,dist", [(1, 2, "uniform"), (64, 2, "uniform"), (2048, 16, "uniform"),
                                        (2112, 1024, "uniform"), (12288, 192, "skewed"), (4096, 65536, "uniform"),
