@@ -21,6 +21,9 @@
 //   dV   = P^T dYq   (A from TMEM, M=128, N=64, K=192)
 //   G    = E^T Xq    (M=128, N=64, K=192)
 //   dQ   = E Xk      (E^T read MN-major; two M=128 halves over the 192 queries, K=128)
+// Query slot r < 128 is also key slot r, so G and the first dQ half accumulate
+// into one TMEM block; the key-role correction needs g_j . x_j, which equals
+// sum_i e_ij (x_i . x_j) and is summed from S^T during the elementwise step.
 // Gradients of every round are added into fp32 accumulators with vector
 // reductions (red.global.add.v4.f32); their summation order is not fixed.
 //
@@ -54,9 +57,9 @@ constexpr int kTmemCols = 512;
 constexpr float kLog2e = 1.4426950408889634f;
 
 // TMEM columns.  Elementwise phase: S^T [0,192), P^T packed [192,288), dP^T [288,480).
-// After it: dV [0,64), G [64,128), dQ rows 0-127 [128,192), dQ rows 64-191 [288,352).
 constexpr uint32_t cS = 0, cPT = 192, cD = 288;
-constexpr uint32_t cDV = 0, cG = 64, cQa = 128, cQb = 288;
+// After it: dV [0,64), G + dQ rows 0-127 [64,128), dQ rows 64-191 [288,352).
+constexpr uint32_t cDV = 0, cDX = 64, cQb = 288;
 
 struct alignas(1024) Stage {
     uint8_t X[kQ * 128];            // x rows of the query slots (first 128 = key slots)   24 KB
@@ -75,7 +78,8 @@ struct BwdSmem {
     uint8_t ET[3][kK * 128];        // tau inv_j dS^T, 3 blocks of 64 queries (48 KB)
     uint64_t full[kStages], empty[kStages];
     uint64_t bar_s, bar_p, bar_o, bar_free;
-    uint64_t xchg[4];               // key-role rows staged for the partner warp, per lane quadrant
+    uint64_t gx_ready;              // the second half's partial sums of g . x are in gxh
+    float gxh[kK];
     uint32_t tmem_base;
     int abort;
 };
@@ -90,7 +94,7 @@ __device__ __forceinline__ void red_add_v4(float *addr, float a, float b, float 
 // rowg < 0) with coalesced vector reductions: the warp's 32 rows go through
 // its 8 KB staging buffer (16-byte chunks swizzled by lane against bank
 // conflicts), then each reduction instruction covers two whole rows.
-__device__ __forceinline__ void flush_rows(uint8_t *stg, int lane, const float *a, float *acc, long long rowg,
+__device__ __forceinline__ void flush_rows(uint8_t *stg, int lane, const float *a, float *acc, int rowg,
                                            int ph_role = -1, int ph_it = 0, int ph_ev = 0)
 {
 #pragma unroll
@@ -103,12 +107,32 @@ __device__ __forceinline__ void flush_rows(uint8_t *stg, int lane, const float *
 #pragma unroll 4
     for (int it = 0; it < 16; ++it) {
         const int rr = 2 * it + (lane >> 4);
-        const long long rg = __shfl_sync(0xffffffffu, rowg, rr);
+        const int rg = __shfl_sync(0xffffffffu, rowg, rr);
         const float4 val = *reinterpret_cast<const float4 *>(stg + rr * 256 + ((c ^ (rr & 15)) << 4));
-        if (rg >= 0) red_add_v4(acc + rg * kDim + 4 * c, val.x, val.y, val.z, val.w);
+        if (rg >= 0) red_add_v4(acc + (long long)rg * kDim + 4 * c, val.x, val.y, val.z, val.w);
     }
     __syncwarp();
     if (ph_role >= 0 && lane == 0) LSH_PHASE(1, ph_role, ph_it, ph_ev + 1);
+}
+
+// As flush_rows for 32 columns: adds a[0..32) to columns [col0, col0 + 32) of
+// row `rowg`; each reduction instruction covers four rows.
+__device__ __forceinline__ void flush_rows32(uint8_t *stg, int lane, const float *a, float *acc, int rowg, int col0)
+{
+#pragma unroll
+    for (int c = 0; c < 8; ++c)
+        *reinterpret_cast<float4 *>(stg + lane * 128 + ((c ^ (lane & 7)) << 4)) =
+            make_float4(a[4 * c], a[4 * c + 1], a[4 * c + 2], a[4 * c + 3]);
+    __syncwarp();
+    const int c = lane & 7;
+#pragma unroll 4
+    for (int it = 0; it < 8; ++it) {
+        const int rr = 4 * it + (lane >> 3);
+        const int rg = __shfl_sync(0xffffffffu, rowg, rr);
+        const float4 val = *reinterpret_cast<const float4 *>(stg + rr * 128 + ((c ^ (rr & 7)) << 4));
+        if (rg >= 0) red_add_v4(acc + (long long)rg * kDim + col0 + 4 * c, val.x, val.y, val.z, val.w);
+    }
+    __syncwarp();
 }
 
 // Chunk `ch` (elements 8ch .. 8ch+7) of bf16 row `row` of a K-major SW128 tile.
@@ -127,13 +151,15 @@ __device__ __forceinline__ void smem_chunk(const uint8_t *tile, int row, int ch,
 // into TMEM columns cPT + C0/2, E^T into shared-memory block C0/64.  A
 // candidate is a query at a later original position (causal) or at any other
 // position; a causal query with no other candidate takes its own key.  Query
-// metadata is read four queries per vector load.
+// metadata is read four queries per vector load.  Returns this block's part of
+// g . x = sum_i e_i (x_i . x_k).
 template <int C0, bool CAUSAL>
-__device__ __forceinline__ void key_row_block(const Stage &st, uint8_t (*ET)[kK * 128], uint32_t tl, int kr, int kpos,
+__device__ __forceinline__ float key_row_block(const Stage &st, uint8_t (*ET)[kK * 128], uint32_t tl, int kr, int kpos,
                                               float kinv, float tau)
 {
     const float sc = tau * kinv * kLog2e;
     const float ec = tau * kinv;
+    float gx = 0.f;
 #pragma unroll
     for (int h = 0; h < 2; ++h) {                       // two halves of 32 query columns
         float s[32], dp[32];
@@ -160,6 +186,7 @@ __device__ __forceinline__ void key_row_block(const Stage &st, uint8_t (*ET)[kK 
                 const float e2 = tc::fast_exp2(fmaf(s[j4 + u], sc, -ql[u]));
                 pv[u] = ok ? e2 : 0.f;
                 ev[u] = ec * pv[u] * (dp[j4 + u] - qd[u]);
+                gx = fmaf(ev[u], s[j4 + u], gx);
             }
             pw[j4 / 2] = pack_bf16x2(pv[0], pv[1]);
             pw[j4 / 2 + 1] = pack_bf16x2(pv[2], pv[3]);
@@ -176,6 +203,7 @@ __device__ __forceinline__ void key_row_block(const Stage &st, uint8_t (*ET)[kK 
                 make_uint4(ew[4 * c4], ew[4 * c4 + 1], ew[4 * c4 + 2], ew[4 * c4 + 3]);
         }
     }
+    return gx;
 }
 
 // Zero P^T and E^T for query columns [C0, C0 + 64) of key row kr.
@@ -229,7 +257,7 @@ attn_bwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
         tc::mbar_init(&sm.bar_p, kComputeWarps);
         tc::mbar_init(&sm.bar_o, 1);
         tc::mbar_init(&sm.bar_free, kComputeWarps);
-        for (int q = 0; q < 4; ++q) tc::mbar_init(&sm.xchg[q], 1);
+        tc::mbar_init(&sm.gx_ready, kComputeWarps / 2);
         sm.abort = 0;
         tc::fence_mbar_init();
     }
@@ -369,13 +397,13 @@ attn_bwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
                 for (int kk = 0; kk < 12; ++kk) {
                     const uint32_t ea = (kk < 4 ? e0 : kk < 8 ? e1 : e2) + (kk & 3) * 32;
                     tc::mma_bf16_ts(tmem + cDV, tmem + cPT + kk * 8, tc::sw128_desc(gs + kk * 2048), id_kv, kk > 0);
-                    tc::mma_bf16(tmem + cG, tc::sw128_desc(ea), tc::sw128_desc(xs + kk * 2048), id_kv, kk > 0);
+                    tc::mma_bf16(tmem + cDX, tc::sw128_desc(ea), tc::sw128_desc(xs + kk * 2048), id_kv, kk > 0);
                 }
                 // E = (E^T)^T read MN-major: 64-query blocks 16 KB apart (leading byte offset)
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
-                    tc::mma_bf16(tmem + cQa, tc::sw128_desc(e0 + kk * 2048, kK * 128), tc::sw128_desc(xs + kk * 2048),
-                                 id_q, kk > 0);
+                    tc::mma_bf16(tmem + cDX, tc::sw128_desc(e0 + kk * 2048, kK * 128), tc::sw128_desc(xs + kk * 2048),
+                                 id_q, true);
                     tc::mma_bf16(tmem + cQb, tc::sw128_desc(e1 + kk * 2048, kK * 128), tc::sw128_desc(xs + kk * 2048),
                                  id_q, kk > 0);
                 }
@@ -416,26 +444,31 @@ attn_bwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
             if (tid == 0) LSH_PHASE(1, 2, it, 2);
             tc::tc_fence_after();
             // ---- elementwise
+            float gx;                                // partial g . x of key row kr
             if (quad < 2) {                          // keys of chunk 2k: queries of chunks 2k, 2k+1
                 if (half == 0) {
-                    key_row_block<0, CAUSAL>(st, sm.ET, tl, kr, kpos, kinv, tau);
+                    gx = key_row_block<0, CAUSAL>(st, sm.ET, tl, kr, kpos, kinv, tau);
                     zero_block<128>(sm.ET, tl, kr);
                 } else {
-                    key_row_block<64, CAUSAL>(st, sm.ET, tl, kr, kpos, kinv, tau);
+                    gx = key_row_block<64, CAUSAL>(st, sm.ET, tl, kr, kpos, kinv, tau);
                 }
             } else {                                 // keys of chunk 2k+1: queries of chunks 2k+1, 2k+2
                 if (half == 0) {
-                    key_row_block<64, CAUSAL>(st, sm.ET, tl, kr, kpos, kinv, tau);
+                    gx = key_row_block<64, CAUSAL>(st, sm.ET, tl, kr, kpos, kinv, tau);
                     zero_block<0>(sm.ET, tl, kr);
                 } else {
-                    key_row_block<128, CAUSAL>(st, sm.ET, tl, kr, kpos, kinv, tau);
+                    gx = key_row_block<128, CAUSAL>(st, sm.ET, tl, kr, kpos, kinv, tau);
                 }
             }
+            if (half == 1) sm.gxh[kr] = gx;
             tc::tmem_st_wait();
             tc::fence_async_smem();
             tc::tc_fence_before();
             __syncwarp();
-            if (lane == 0) tc::mbar_arrive(&sm.bar_p);
+            if (lane == 0) {
+                tc::mbar_arrive(&sm.bar_p);
+                if (half == 1) tc::mbar_arrive(&sm.gx_ready);
+            }
             if (tid == 0) LSH_PHASE(1, 2, it, 3);
             if (!tc::mbar_wait(&sm.bar_o, ph, &sm.abort, status)) break;
             if (tid == 0) LSH_PHASE(1, 2, it, 4);
@@ -444,50 +477,18 @@ attn_bwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
             // buffers reuse memory the MMAs no longer read: E^T and this stage's v rows.
             uint8_t *stg = warp < 6 ? reinterpret_cast<uint8_t *>(sm.ET) + warp * 8192
                                     : const_cast<uint8_t *>(st.V) + (warp - 6) * 8192;
-            // Slot kr is both key kr and query kr: its key-role row (from the warp of
-            // half 1) is added to its query-role row (half 0) before one reduction.
+            const int krow = kpos >= 0 ? (int)rowbase + kpos : -1;
             float a[kDim];
             if (half == 0) {
+                // slot kr: query-role dQ plus key-role g, less inv^2 (g . x) x
                 const int prole = warp == 0 ? 4 : warp == 2 ? 5 : -1;
                 if (prole >= 0 && lane == 0) LSH_PHASE(1, prole, it, 0);
+                if (!tc::mbar_wait(&sm.gx_ready, ph, &sm.abort, status)) break;
+                const float cf = kinv * kinv * (gx + sm.gxh[kr]);
 #pragma unroll
-                for (int c = 0; c < 4; ++c) tc::tmem_ld16(tl + cDV + c * 16, a + c * 16);
+                for (int c = 0; c < 4; ++c) tc::tmem_ld16(tl + cDX + c * 16, a + c * 16);
                 tc::tmem_ld_wait();
                 if (prole >= 0 && lane == 0) LSH_PHASE(1, prole, it, 1);
-                flush_rows(stg, lane, a, dv_acc, rowbase + kpos, prole, it, 2);
-                if (tid == 0) LSH_PHASE(1, 2, it, 6);
-#pragma unroll
-                for (int c = 0; c < 4; ++c) tc::tmem_ld16(tl + cQa + c * 16, a + c * 16);
-                tc::tmem_ld_wait();
-                if (prole >= 0 && lane == 0) LSH_PHASE(1, prole, it, 4);
-                // partner's key-role row staged (bounded wait, as every wait here)
-                if (!tc::mbar_wait(&sm.xchg[quad], ph, &sm.abort, status)) break;
-                if (tid == 0) LSH_PHASE(1, 2, it, 7);
-                const uint8_t *pst = warp + 4 < 6 ? reinterpret_cast<const uint8_t *>(sm.ET) + (warp + 4) * 8192
-                                                  : st.V + (warp + 4 - 6) * 8192;
-#pragma unroll
-                for (int c = 0; c < 16; ++c) {
-                    const float4 g = *reinterpret_cast<const float4 *>(pst + lane * 256 + ((c ^ (lane & 15)) << 4));
-                    a[4 * c] += g.x; a[4 * c + 1] += g.y; a[4 * c + 2] += g.z; a[4 * c + 3] += g.w;
-                }
-                if (prole >= 0 && lane == 0) LSH_PHASE(1, prole, it, 5);
-                flush_rows(stg, lane, a, dx_acc, rowbase + kpos, prole, it, 6);
-            } else {
-                if (tid == 128) LSH_PHASE(1, 3, it, 0);
-#pragma unroll
-                for (int c = 0; c < 4; ++c) tc::tmem_ld16(tl + cG + c * 16, a + c * 16);
-                tc::tmem_ld_wait();
-                if (tid == 128) LSH_PHASE(1, 3, it, 1);
-                // key-role correction g - inv^2 (g . x) x, reading x_k from shared memory twice
-                float gx = 0.f;
-#pragma unroll
-                for (int ch = 0; ch < 8; ++ch) {
-                    float xr[8];
-                    smem_chunk(st.X, kr, ch, xr);
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) gx = fmaf(a[ch * 8 + e], xr[e], gx);
-                }
-                const float cf = kinv * kinv * gx;
 #pragma unroll
                 for (int ch = 0; ch < 8; ++ch) {
                     float xr[8];
@@ -495,24 +496,36 @@ attn_bwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
 #pragma unroll
                     for (int e = 0; e < 8; ++e) a[ch * 8 + e] = fmaf(-cf, xr[e], a[ch * 8 + e]);
                 }
-                // stage the row for the partner warp of half 0 (same layout as flush_rows)
+                flush_rows(stg, lane, a, dx_acc, krow, prole, it, 2);
+                if (quad >= 2) {                     // first half of the dV columns of these rows
 #pragma unroll
-                for (int c = 0; c < 16; ++c)
-                    *reinterpret_cast<float4 *>(stg + lane * 256 + ((c ^ (lane & 15)) << 4)) =
-                        make_float4(a[4 * c], a[4 * c + 1], a[4 * c + 2], a[4 * c + 3]);
-                __syncwarp();
-                if (lane == 0) tc::mbar_arrive(&sm.xchg[quad]);
-                if (tid == 128) LSH_PHASE(1, 3, it, 2);
-                if (quad >= 2) {                                          // query row 64 + kr (chunk 2k+2)
-                    // own buffer in this stage's dY rows, which the MMAs no longer read
+                    for (int c = 0; c < 2; ++c) tc::tmem_ld16(tl + cDV + c * 16, a + c * 16);
+                    tc::tmem_ld_wait();
+                    flush_rows32(stg, lane, a, dv_acc, krow, 0);
+                }
+                if (prole >= 0 && lane == 0) LSH_PHASE(1, prole, it, 4);
+            } else {
+                if (tid == 128) LSH_PHASE(1, 3, it, 0);
+                if (quad < 2) {
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) tc::tmem_ld16(tl + cDV + c * 16, a + c * 16);
+                    tc::tmem_ld_wait();
+                    flush_rows(stg, lane, a, dv_acc, krow);
+                } else {
+#pragma unroll
+                    for (int c = 0; c < 2; ++c) tc::tmem_ld16(tl + cDV + 32 + c * 16, a + c * 16);
+                    tc::tmem_ld_wait();
+                    flush_rows32(stg, lane, a, dv_acc, krow, 32);
+                    // query row 64 + kr (chunk 2k+2), staged in this stage's dY rows
                     uint8_t *stg2 = const_cast<uint8_t *>(st.G) + (quad - 2) * 8192;
 #pragma unroll
                     for (int c = 0; c < 4; ++c) tc::tmem_ld16(tl + cQb + c * 16, a + c * 16);
                     tc::tmem_ld_wait();
                     if (warp == 6 && lane == 0) LSH_PHASE(1, 6, it, 0);
                     const int qp = st.qpos[64 + kr];
-                    flush_rows(stg2, lane, a, dx_acc, qp >= 0 ? rowbase + qp : -1LL, warp == 6 ? 6 : -1, it, 1);
+                    flush_rows(stg2, lane, a, dx_acc, qp >= 0 ? (int)rowbase + qp : -1, warp == 6 ? 6 : -1, it, 1);
                 }
+                if (tid == 128) LSH_PHASE(1, 3, it, 1);
             }
             if (tid == 0) LSH_PHASE(1, 2, it, 5);
             tc::tc_fence_before();
