@@ -419,7 +419,7 @@ int32_t lsh_attn_abi_version(void) { return LSH_ATTN_ABI_VERSION; }
 namespace lsh {
 namespace tc {
 
-bool make_row_tmap(CUtensorMap *map, const void *base, long long rows)
+bool make_row_tmap(CUtensorMap *map, const void *base, long long rows, int box_rows)
 {
     static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
     if (!encode) {
@@ -432,7 +432,7 @@ bool make_row_tmap(CUtensorMap *map, const void *base, long long rows)
     }
     const cuuint64_t dims[2] = {(cuuint64_t)kDim, (cuuint64_t)rows};
     const cuuint64_t strides[1] = {(cuuint64_t)kDim * 2};
-    const cuuint32_t box[2] = {(cuuint32_t)kDim, 1};
+    const cuuint32_t box[2] = {(cuuint32_t)kDim, (cuuint32_t)box_rows};
     const cuuint32_t estr[2] = {1, 1};
     CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,

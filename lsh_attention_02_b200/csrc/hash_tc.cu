@@ -6,15 +6,19 @@
 // in tensor memory) and the argmax is the epilogue, so the projections are
 // never written to memory.
 //
-// CTA = 256 rows (two M=128 tiles) x every round.  Warp roles:
+// Persistent CTAs (one per SM) walk blocks of 256 rows (two M=128 tiles);
+// each block runs every round.  Warp roles:
 //   warps 0-7  epilogue: warp w reads TMEM lanes 32*(w%4).. of M-tile w/4,
 //              one row per thread, and keeps the running argmax;
-//   warp 8     producer: one bulk copy per (round, N-tile) of the rotation
-//              tile, pre-transposed and pre-swizzled in global memory, into a
-//              4-stage shared-memory ring;
-//   warp 9     MMA issuer: 4 K-steps x 2 M-tiles per N-tile into one of two
+//   warp 8     producer: the next block's x rows by two TMA tile loads into
+//              the idle one of two A buffers, and one bulk copy per (round,
+//              N-tile) of the rotation tile, pre-transposed and pre-swizzled
+//              in global memory, into a 4-stage shared-memory ring;
+//   warp 9     MMA issuer: 4 K-steps per M-tile and N-tile into one of two
 //              TMEM accumulator buffers (double buffering lets the epilogue
-//              of tile t overlap the MMAs of tile t+1).
+//              of tile t overlap the MMAs of tile t+1), with a completion
+//              barrier per M-tile so the two epilogue halves start apart and
+//              their ALU- and FMA-heavy passes overlap.
 //
 // Epilogue per N-tile of NT columns held in registers: pass 1 takes the
 // max and min with 3-input min/max; the larger of max and -min decides the
@@ -28,7 +32,7 @@ namespace lsh {
 
 namespace {
 
-constexpr int kRows = 256;          // rows per CTA
+constexpr int kRows = 256;          // rows per block
 constexpr int kMaxNT = 128;         // widest N-tile
 constexpr int kStages = 4;          // rotation-tile ring
 constexpr int kEpiWarps = 8;
@@ -36,10 +40,11 @@ constexpr int kThreads = (kEpiWarps + 2) * 32;
 constexpr int kTmemCols = 512;      // 2 buffers x 2 M-tiles x kMaxNT
 
 struct HashSmem {
-    uint8_t A[kRows * 128];                 // x rows, K-major SW128   (32 KB)
-    uint8_t B[kStages][kMaxNT * 128];       // rotation tiles           (64 KB)
+    uint8_t A[2][kRows * 128];              // x rows of two row blocks, K-major SW128 (64 KB)
+    uint8_t B[kStages][kMaxNT * 128];       // rotation tiles (64 KB)
     uint64_t full[kStages], empty[kStages];
-    uint64_t acc_full[2], acc_empty[2];
+    uint64_t a_full[2], a_empty[2];
+    uint64_t acc_full[2][2], acc_empty[2];  // [buffer][M-tile]
     uint32_t tmem_base;
     int abort;
 };
@@ -64,35 +69,31 @@ __global__ void rot_swizzle_kernel(const __nv_bfloat16 *__restrict__ R, __nv_bfl
 
 template <int NT>
 __global__ void __launch_bounds__(kThreads, 1)
-hash_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__restrict__ Rs,
+hash_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __nv_bfloat16 *__restrict__ Rs,
                uint16_t *__restrict__ buckets, long long rows_total, int L, int rounds, int half,
                uint32_t *__restrict__ status)
 {
     extern __shared__ uint8_t smem_raw[];
     HashSmem &sm = *reinterpret_cast<HashSmem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const long long row0 = (long long)blockIdx.x * kRows;
     const int n_nt = half / NT;
     const int items = rounds * n_nt;
+    const long long n_blocks = (rows_total + kRows - 1) / kRows;
     if (threadIdx.x == 0) LSH_PHASE(0, 3, 0, 0);
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) { tc::mbar_init(&sm.full[s], 1); tc::mbar_init(&sm.empty[s], 1); }
-        for (int b = 0; b < 2; ++b) { tc::mbar_init(&sm.acc_full[b], 1); tc::mbar_init(&sm.acc_empty[b], kEpiWarps); }
+        for (int b = 0; b < 2; ++b) {
+            tc::mbar_init(&sm.a_full[b], 1);
+            tc::mbar_init(&sm.a_empty[b], 1);
+            tc::mbar_init(&sm.acc_full[b][0], 1);
+            tc::mbar_init(&sm.acc_full[b][1], 1);
+            tc::mbar_init(&sm.acc_empty[b], kEpiWarps);
+        }
         sm.abort = 0;
         tc::fence_mbar_init();
     }
     if (warp == 0) tc::tmem_alloc(&sm.tmem_base, kTmemCols);
-
-    // x rows -> A (K-major, 128-byte swizzle); rows past the end are zero.
-    for (int c = threadIdx.x; c < kRows * 8; c += kThreads) {
-        int r = c >> 3, ch = c & 7;
-        long long g = row0 + r;
-        uint4 val = make_uint4(0, 0, 0, 0);
-        if (g < rows_total) val = reinterpret_cast<const uint4 *>(x + g * kDim)[ch];
-        *reinterpret_cast<uint4 *>(sm.A + r * 128 + ((ch ^ (r & 7)) << 4)) = val;
-    }
-    tc::fence_async_smem();
     tc::tc_fence_before();
     __syncthreads();
     tc::tc_fence_after();
@@ -102,147 +103,178 @@ hash_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__restr
     if (warp == kEpiWarps) {
         // ---------------- producer
         if (lane == 0) {
-            for (int it = 0; it < items; ++it) {
-                const int s = it % kStages;
-                const uint32_t ph = (uint32_t)(it / kStages) & 1u;
-                LSH_PHASE(0, 1, it, 0);
-                if (it >= kStages && !tc::mbar_wait(&sm.empty[s], ph ^ 1u, &sm.abort, status)) break;
-                LSH_PHASE(0, 1, it, 1);
-                const int r = it / n_nt, nt = it % n_nt;
-                const __nv_bfloat16 *src = Rs + ((long long)r * half + (long long)nt * NT) * kDim;
-                tc::mbar_arrive_expect_tx(&sm.full[s], NT * 128);
-                tc::bulk_g2s(sm.B[s], src, NT * 128, &sm.full[s]);
+            tc::prefetch_tmap(&xmap);
+            auto load_a = [&](long long blk, int bi) -> bool {
+                const int ab = bi & 1;
+                if (bi >= 2 && !tc::mbar_wait(&sm.a_empty[ab], (uint32_t)((bi >> 1) - 1) & 1u, &sm.abort, status))
+                    return false;
+                tc::mbar_arrive_expect_tx(&sm.a_full[ab], kRows * 128);
+                tc::tma_load_2d(sm.A[ab], &xmap, 0, (int)(blk * kRows), &sm.a_full[ab]);
+                tc::tma_load_2d(sm.A[ab] + 128 * 128, &xmap, 0, (int)(blk * kRows + 128), &sm.a_full[ab]);
+                return true;
+            };
+            bool ok = blockIdx.x >= n_blocks || load_a(blockIdx.x, 0);
+            int it = 0, bi = 0;
+            for (long long blk = blockIdx.x; ok && blk < n_blocks; blk += gridDim.x, ++bi) {
+                const int prefetch_at = min(kStages, items) - 1;
+                for (int i = 0; i < items; ++i, ++it) {
+                    const int s = it % kStages;
+                    const uint32_t ph = (uint32_t)(it / kStages) & 1u;
+                    LSH_PHASE(0, 1, it, 0);
+                    if (it >= kStages && !tc::mbar_wait(&sm.empty[s], ph ^ 1u, &sm.abort, status)) { ok = false; break; }
+                    LSH_PHASE(0, 1, it, 1);
+                    const int r = i / n_nt, nt = i % n_nt;
+                    const __nv_bfloat16 *src = Rs + ((long long)r * half + (long long)nt * NT) * kDim;
+                    tc::mbar_arrive_expect_tx(&sm.full[s], NT * 128);
+                    tc::bulk_g2s(sm.B[s], src, NT * 128, &sm.full[s]);
+                    // the next block's rows, once this block's MMAs have started
+                    if (i == prefetch_at && blk + gridDim.x < n_blocks && !load_a(blk + gridDim.x, bi + 1)) {
+                        ok = false;
+                        break;
+                    }
+                }
             }
         }
     } else if (warp == kEpiWarps + 1) {
         // ---------------- MMA issuer
         if (lane == 0) {
             constexpr uint32_t idesc = tc::idesc_bf16(128, NT, 0, 0);
-            const uint32_t a0 = tc::smem_u32(sm.A);
-            for (int it = 0; it < items; ++it) {
-                const int s = it % kStages;
-                const uint32_t ph = (uint32_t)(it / kStages) & 1u;
-                const int ab = it & 1;
-                const uint32_t aph = (uint32_t)(it >> 1) & 1u;
-                LSH_PHASE(0, 2, it, 0);
-                if (!tc::mbar_wait(&sm.full[s], ph, &sm.abort, status)) break;
-                LSH_PHASE(0, 2, it, 1);
-                if (it >= 2 && !tc::mbar_wait(&sm.acc_empty[ab], aph ^ 1u, &sm.abort, status)) break;
-                LSH_PHASE(0, 2, it, 2);
-                tc::tc_fence_after();
-                const uint32_t b0 = tc::smem_u32(sm.B[s]);
+            int it = 0, bi = 0;
+            bool ok = true;
+            for (long long blk = blockIdx.x; ok && blk < n_blocks; blk += gridDim.x, ++bi) {
+                const int xa = bi & 1;
+                if (!tc::mbar_wait(&sm.a_full[xa], (uint32_t)(bi >> 1) & 1u, &sm.abort, status)) break;
+                const uint32_t a0 = tc::smem_u32(sm.A[xa]);
+                for (int i = 0; i < items; ++i, ++it) {
+                    const int s = it % kStages;
+                    const uint32_t ph = (uint32_t)(it / kStages) & 1u;
+                    const int ab = it & 1;
+                    const uint32_t aph = (uint32_t)(it >> 1) & 1u;
+                    LSH_PHASE(0, 2, it, 0);
+                    if (!tc::mbar_wait(&sm.full[s], ph, &sm.abort, status)) { ok = false; break; }
+                    LSH_PHASE(0, 2, it, 1);
+                    if (it >= 2 && !tc::mbar_wait(&sm.acc_empty[ab], aph ^ 1u, &sm.abort, status)) { ok = false; break; }
+                    LSH_PHASE(0, 2, it, 2);
+                    tc::tc_fence_after();
+                    const uint32_t b0 = tc::smem_u32(sm.B[s]);
 #pragma unroll
-                for (int mt = 0; mt < 2; ++mt) {
-                    const uint32_t d = tmem + (uint32_t)(ab * 2 * kMaxNT + mt * kMaxNT);
+                    for (int mt = 0; mt < 2; ++mt) {
+                        const uint32_t d = tmem + (uint32_t)(ab * 2 * kMaxNT + mt * kMaxNT);
 #pragma unroll
-                    for (int k = 0; k < 4; ++k)
-                        tc::mma_bf16(d, tc::sw128_desc(a0 + mt * 128 * 128 + k * 32), tc::sw128_desc(b0 + k * 32),
-                                     idesc, k > 0);
+                        for (int k = 0; k < 4; ++k)
+                            tc::mma_bf16(d, tc::sw128_desc(a0 + mt * 128 * 128 + k * 32), tc::sw128_desc(b0 + k * 32),
+                                         idesc, k > 0);
+                        tc::mma_commit(&sm.acc_full[ab][mt]);
+                    }
+                    tc::mma_commit(&sm.empty[s]);
+                    LSH_PHASE(0, 2, it, 3);
                 }
-                tc::mma_commit(&sm.empty[s]);
-                tc::mma_commit(&sm.acc_full[ab]);
-                LSH_PHASE(0, 2, it, 3);
+                if (ok) tc::mma_commit(&sm.a_empty[xa]);
             }
         }
     } else {
         // ---------------- epilogue: one row per thread
         const int q = warp & 3, mt = warp >> 2;
-        const int row = mt * 128 + q * 32 + lane;
-        const long long g = row0 + row;
         const uint32_t lane_base = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(mt * kMaxNT);
-        float best = -INFINITY;
-        int bucket = 0;
-        for (int it = 0; it < items; ++it) {
-            const int ab = it & 1;
-            const uint32_t aph = (uint32_t)(it >> 1) & 1u;
-            if (threadIdx.x == 0) LSH_PHASE(0, 0, it, 0);
-            if (!tc::mbar_wait(&sm.acc_full[ab], aph, &sm.abort, status)) break;
-            if (threadIdx.x == 0) LSH_PHASE(0, 0, it, 1);
-            tc::tc_fence_after();
-            float v[NT];
+        int it = 0;
+        bool ok = true;
+        for (long long blk = blockIdx.x; ok && blk < n_blocks; blk += gridDim.x) {
+            const long long g = blk * kRows + mt * 128 + q * 32 + lane;
+            float best = -INFINITY;
+            int bucket = 0;
+            for (int i = 0; i < items; ++i, ++it) {
+                const int ab = it & 1;
+                const uint32_t aph = (uint32_t)(it >> 1) & 1u;
+                if (threadIdx.x == 0) LSH_PHASE(0, 0, it, 0);
+                if (!tc::mbar_wait(&sm.acc_full[ab][mt], aph, &sm.abort, status)) { ok = false; break; }
+                if (threadIdx.x == 0) LSH_PHASE(0, 0, it, 1);
+                tc::tc_fence_after();
+                float v[NT];
 #pragma unroll
-            for (int c = 0; c < NT / 16; ++c) tc::tmem_ld16(lane_base + (uint32_t)(ab * 2 * kMaxNT + c * 16), v + c * 16);
-            tc::tmem_ld_wait();
-            tc::tc_fence_before();
-            __syncwarp();
-            if (lane == 0) tc::mbar_arrive(&sm.acc_empty[ab]);
-            if (threadIdx.x == 0) LSH_PHASE(0, 0, it, 2);
+                for (int c = 0; c < NT / 16; ++c)
+                    tc::tmem_ld16(lane_base + (uint32_t)(ab * 2 * kMaxNT + c * 16), v + c * 16);
+                tc::tmem_ld_wait();
+                tc::tc_fence_before();
+                __syncwarp();
+                if (lane == 0) tc::mbar_arrive(&sm.acc_empty[ab]);
+                if (threadIdx.x == 0) LSH_PHASE(0, 0, it, 2);
 
-            // pass 1: extremes of the tile, four independent chains per extreme
-            constexpr int Q = NT / 4;
-            float mxq[4], mnq[4];
-#pragma unroll
-            for (int qq = 0; qq < 4; ++qq) {
-                const int j0 = qq * Q;
-                float a = fmaxf(v[j0], v[j0 + 1]), b = fminf(v[j0], v[j0 + 1]);
-#pragma unroll
-                for (int j = j0 + 2; j < j0 + Q; j += 2) {
-                    a = tc::max3f(a, v[j], v[j + 1]);
-                    b = tc::min3f(b, v[j], v[j + 1]);
-                }
-                mxq[qq] = a;
-                mnq[qq] = b;
-            }
-            const float mx = fmaxf(fmaxf(mxq[0], mxq[1]), fmaxf(mxq[2], mxq[3]));
-            const float mn = fminf(fminf(mnq[0], mnq[1]), fminf(mnq[2], mnq[3]));
-            const bool pos = mx >= -mn;
-            const float target = pos ? mx : mn;
-            // pass 2: lowest column holding the extreme.  U = |extreme| bounds every
-            // |v| of the tile; with B = 2^(24 - e(U)), (U - side * v_j) * B is exactly
-            // 0 where v_j is the extreme and at least 1 elsewhere (the closest float
-            // below U is 2^(e(U) - 24) away), so a saturating FMA gives a 0/1 flag
-            // without a compare.  Sixteen flags per chain are summed as the bits of
-            // an integer kept in the mantissa of 2^23 + sum (exact), and the first
-            // clear bit is the column.  This runs on the FMA pipe while pass 1 uses
-            // the ALU pipe.  Extremes below 2^-103 (B would not be finite) take the
-            // compare-and-select form.
-            if (threadIdx.x == 0) LSH_PHASE(0, 0, it, 3);
-            const float U = pos ? mx : -mn;
-            const int be = (__float_as_int(U) >> 23) & 0xFF;
-            int js;
-            if (__any_sync(0xffffffffu, U != 0.f && be < 24)) {
-                int jq[4];
+                // pass 1: extremes of the tile, four independent chains per extreme
+                constexpr int Q = NT / 4;
+                float mxq[4], mnq[4];
 #pragma unroll
                 for (int qq = 0; qq < 4; ++qq) {
-                    int jj = NT;
+                    const int j0 = qq * Q;
+                    float a = fmaxf(v[j0], v[j0 + 1]), b = fminf(v[j0], v[j0 + 1]);
 #pragma unroll
-                    for (int j = qq * Q + Q - 1; j >= qq * Q; --j) jj = (v[j] == target) ? j : jj;
-                    jq[qq] = jj;
+                    for (int j = j0 + 2; j < j0 + Q; j += 2) {
+                        a = tc::max3f(a, v[j], v[j + 1]);
+                        b = tc::min3f(b, v[j], v[j + 1]);
+                    }
+                    mxq[qq] = a;
+                    mnq[qq] = b;
                 }
-                js = min(min(jq[0], jq[1]), min(jq[2], jq[3]));
-            } else {
-                const float B = __int_as_float(min(278 - be, 253) << 23);
-                const float nsB = pos ? -B : B;
-                const float UB = U * B;
-                constexpr int NC = NT / 16;
-                float acc[NC];
+                const float mx = fmaxf(fmaxf(mxq[0], mxq[1]), fmaxf(mxq[2], mxq[3]));
+                const float mn = fminf(fminf(mnq[0], mnq[1]), fminf(mnq[2], mnq[3]));
+                const bool pos = mx >= -mn;
+                const float target = pos ? mx : mn;
+                if (threadIdx.x == 0) LSH_PHASE(0, 0, it, 3);
+                // pass 2: lowest column holding the extreme.  U = |extreme| bounds every
+                // |v| of the tile; with B = 2^(24 - e(U)), (U - side * v_j) * B is exactly
+                // 0 where v_j is the extreme and at least 1 elsewhere (the closest float
+                // below U is 2^(e(U) - 24) away), so a saturating FMA gives a 0/1 flag
+                // without a compare.  Sixteen flags per chain are summed as the bits of
+                // an integer kept in the mantissa of 2^23 + sum (exact), and the first
+                // clear bit is the column.  This runs on the FMA pipe while pass 1 uses
+                // the ALU pipe.  Extremes below 2^-103 (B would not be finite) take the
+                // compare-and-select form.
+                const float U = pos ? mx : -mn;
+                const int be = (__float_as_int(U) >> 23) & 0xFF;
+                int js;
+                if (__any_sync(0xffffffffu, U != 0.f && be < 24)) {
+                    int jq[4];
 #pragma unroll
-                for (int c = 0; c < NC; ++c) acc[c] = 8388608.f;
+                    for (int qq = 0; qq < 4; ++qq) {
+                        int jj = NT;
 #pragma unroll
-                for (int k = 0; k < 16; ++k)
+                        for (int j = qq * Q + Q - 1; j >= qq * Q; --j) jj = (v[j] == target) ? j : jj;
+                        jq[qq] = jj;
+                    }
+                    js = min(min(jq[0], jq[1]), min(jq[2], jq[3]));
+                } else {
+                    const float B = __int_as_float(min(278 - be, 253) << 23);
+                    const float nsB = pos ? -B : B;
+                    const float UB = U * B;
+                    constexpr int NC = NT / 16;
+                    float acc[NC];
 #pragma unroll
-                    for (int c = 0; c < NC; ++c)
-                        acc[c] = fmaf(tc::fma_sat(v[c * 16 + k], nsB, UB), (float)(1 << k), acc[c]);
-                js = NT;
+                    for (int c = 0; c < NC; ++c) acc[c] = 8388608.f;
 #pragma unroll
-                for (int c = NC - 1; c >= 0; --c) {
-                    const uint32_t eq = ~__float_as_uint(acc[c]) & 0xFFFFu;
-                    js = eq ? c * 16 + __ffs((int)eq) - 1 : js;
+                    for (int k = 0; k < 16; ++k)
+#pragma unroll
+                        for (int c = 0; c < NC; ++c)
+                            acc[c] = fmaf(tc::fma_sat(v[c * 16 + k], nsB, UB), (float)(1 << k), acc[c]);
+                    js = NT;
+#pragma unroll
+                    for (int c = NC - 1; c >= 0; --c) {
+                        const uint32_t eq = ~__float_as_uint(acc[c]) & 0xFFFFu;
+                        js = eq ? c * 16 + __ffs((int)eq) - 1 : js;
+                    }
                 }
-            }
-            const int r = it / n_nt, nt = it % n_nt;
-            const float tbest = pos ? mx : -mn;
-            const int tb = (pos ? 0 : half) + nt * NT + js;
-            if (tbest > best || (tbest == best && tb < bucket)) { best = tbest; bucket = tb; }
-            if (threadIdx.x == 0) LSH_PHASE(0, 0, it, 4);
-            if (nt == n_nt - 1) {
-                if (g < rows_total) {
-                    const long long bh = g / L;
-                    const int i = (int)(g % L);
-                    buckets[(bh * rounds + r) * L + i] = (uint16_t)bucket;
+                const int r = i / n_nt, nt = i % n_nt;
+                const float tbest = pos ? mx : -mn;
+                const int tb = (pos ? 0 : half) + nt * NT + js;
+                if (tbest > best || (tbest == best && tb < bucket)) { best = tbest; bucket = tb; }
+                if (threadIdx.x == 0) LSH_PHASE(0, 0, it, 4);
+                if (nt == n_nt - 1) {
+                    if (g < rows_total) {
+                        const long long bh = g / L;
+                        const int pos_i = (int)(g % L);
+                        buckets[(bh * rounds + r) * L + pos_i] = (uint16_t)bucket;
+                    }
+                    best = -INFINITY;
+                    bucket = 0;
                 }
-                best = -INFINITY;
-                bucket = 0;
             }
         }
     }
@@ -261,13 +293,18 @@ cudaError_t launch_nt(const Problem &p, const void *x, const __nv_bfloat16 *Rs, 
                       cudaStream_t st)
 {
     // one CTA per SM: each holds all 512 TMEM columns
-    const size_t smem = std::max<size_t>(sizeof(HashSmem) + 1024, 120 * 1024);
+    const size_t smem = sizeof(HashSmem) + 1024;
     cudaError_t e = cudaFuncSetAttribute(hash_tc_kernel<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const long long rows = p.tokens();
-    const unsigned grid = (unsigned)((rows + kRows - 1) / kRows);
-    hash_tc_kernel<NT><<<grid, kThreads, smem, st>>>((const __nv_bfloat16 *)x, Rs, buckets, rows, p.L, p.R, p.nb / 2,
-                                                     status);
+    CUtensorMap xmap;
+    if (!tc::make_row_tmap(&xmap, x, rows, 128)) return cudaErrorInvalidValue;
+    int dev = 0, sms = 148;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+    const long long blocks = (rows + kRows - 1) / kRows;
+    const unsigned grid = (unsigned)std::min<long long>(blocks, sms);
+    hash_tc_kernel<NT><<<grid, kThreads, smem, st>>>(xmap, Rs, buckets, rows, p.L, p.R, p.nb / 2, status);
     return cudaGetLastError();
 }
 
@@ -282,7 +319,13 @@ int pick_nt(int half)
 
 }  // namespace
 
-bool hash_tc_supported(const Problem &p) { return p.dtype == LSH_BF16 && p.d == kDim && pick_nt(p.nb / 2) != 0; }
+// Rows are addressed by 32-bit TMA coordinates; a problem smaller than one
+// 128-row TMA box takes the SIMT hash.
+bool hash_tc_supported(const Problem &p)
+{
+    return p.dtype == LSH_BF16 && p.d == kDim && pick_nt(p.nb / 2) != 0 && p.tokens() >= 128 &&
+           p.tokens() < (1LL << 31) - kRows;
+}
 
 size_t hash_tc_scratch_bytes(const Problem &p) { return (size_t)p.R * (p.nb / 2) * kDim * sizeof(__nv_bfloat16); }
 

@@ -159,17 +159,16 @@ __device__ __forceinline__ void cp_async_arrive(uint64_t *bar)
     asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
-// TMA row gather: rows r0..r3 (64 bf16 each) of a 2-D [rows, 64] tensor map
-// with a one-row box and 128-byte swizzle land as four consecutive swizzled
-// rows at `dst` (512 bytes, dst 512-byte aligned inside a 1024-byte-aligned
-// tile).  A row index outside the tensor (e.g. -1) is filled with zeros.
-__device__ __forceinline__ void tma_gather4(void *dst, const CUtensorMap *map, int r0, int r1, int r2, int r3,
-                                            uint64_t *bar)
+// TMA tile load (no multicast): the box of a 2-D tensor map at coordinates
+// (c0 = element within a row, c1 = row) lands at `dst` in the map's swizzled
+// layout; rows outside the tensor are filled with zeros.  Completion is
+// counted on `bar` in bytes.
+__device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, int c0, int c1, uint64_t *bar)
 {
     asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(smem_u32(dst)),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(0), "r"(r0), "r"(r1), "r"(r2), "r"(r3)
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1)
         : "memory");
 }
 
@@ -357,9 +356,10 @@ __device__ __forceinline__ float fma_sat(float a, float b, float c)
 }
 
 // Host: 2-D tensor map over `rows` rows of 64 bf16 (128 bytes) starting at
-// `base`, one-row box, 128-byte swizzle, zero fill outside.  Returns false if
-// the driver entry point is unavailable or rejects the arguments.
-bool make_row_tmap(CUtensorMap *map, const void *base, long long rows);
+// `base`, a box of `box_rows` whole rows, 128-byte swizzle, zero fill outside.
+// Returns false if the driver entry point is unavailable or rejects the
+// arguments.
+bool make_row_tmap(CUtensorMap *map, const void *base, long long rows, int box_rows);
 
 }  // namespace tc
 }  // namespace lsh
