@@ -79,6 +79,7 @@ struct BwdSmem {
     uint64_t full[kStages], empty[kStages];
     uint64_t bar_s, bar_p, bar_o, bar_free;
     uint64_t gx_ready;              // the second half's partial sums of g . x are in gxh
+    uint64_t epi_done;              // every compute warp finished the previous tile's epilogue
     float gxh[kK];
     uint32_t tmem_base;
     int abort;
@@ -258,6 +259,7 @@ attn_bwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
         tc::mbar_init(&sm.bar_o, 1);
         tc::mbar_init(&sm.bar_free, kComputeWarps);
         tc::mbar_init(&sm.gx_ready, kComputeWarps / 2);
+        tc::mbar_init(&sm.epi_done, kComputeWarps);
         sm.abort = 0;
         tc::fence_mbar_init();
     }
@@ -443,7 +445,9 @@ attn_bwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
             if (!tc::mbar_wait(&sm.bar_s, ph, &sm.abort, status)) break;
             if (tid == 0) LSH_PHASE(1, 2, it, 2);
             tc::tc_fence_after();
-            // ---- elementwise
+            // ---- elementwise.  E^T and gxh are rewritten here: wait until no warp still
+            // stages the previous tile's rows in them.
+            if (it > 0 && !tc::mbar_wait(&sm.epi_done, (uint32_t)(it - 1) & 1u, &sm.abort, status)) break;
             float gx;                                // partial g . x of key row kr
             if (quad < 2) {                          // keys of chunk 2k: queries of chunks 2k, 2k+1
                 if (half == 0) {
@@ -478,17 +482,30 @@ attn_bwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
             uint8_t *stg = warp < 6 ? reinterpret_cast<uint8_t *>(sm.ET) + warp * 8192
                                     : const_cast<uint8_t *>(st.V) + (warp - 6) * 8192;
             const int krow = kpos >= 0 ? (int)rowbase + kpos : -1;
-            float a[kDim];
+            // Every warp first moves its outputs from tensor memory to registers and
+            // releases the columns, so the next tile's S^T and dP^T products run while
+            // this tile's rows are reduced.
+            float a[kDim], b[kDim / 2];
+            auto release_tmem = [&] {
+                tc::tmem_ld_wait();
+                tc::tc_fence_before();
+                __syncwarp();
+                if (lane == 0) tc::mbar_arrive(&sm.bar_free);
+            };
             if (half == 0) {
                 // slot kr: query-role dQ plus key-role g, less inv^2 (g . x) x
                 const int prole = warp == 0 ? 4 : warp == 2 ? 5 : -1;
                 if (prole >= 0 && lane == 0) LSH_PHASE(1, prole, it, 0);
-                if (!tc::mbar_wait(&sm.gx_ready, ph, &sm.abort, status)) break;
-                const float cf = kinv * kinv * (gx + sm.gxh[kr]);
 #pragma unroll
                 for (int c = 0; c < 4; ++c) tc::tmem_ld16(tl + cDX + c * 16, a + c * 16);
-                tc::tmem_ld_wait();
+                if (quad >= 2) {                     // first half of the dV columns of these rows
+#pragma unroll
+                    for (int c = 0; c < 2; ++c) tc::tmem_ld16(tl + cDV + c * 16, b + c * 16);
+                }
+                release_tmem();
                 if (prole >= 0 && lane == 0) LSH_PHASE(1, prole, it, 1);
+                if (!tc::mbar_wait(&sm.gx_ready, ph, &sm.abort, status)) break;
+                const float cf = kinv * kinv * (gx + sm.gxh[kr]);
 #pragma unroll
                 for (int ch = 0; ch < 8; ++ch) {
                     float xr[8];
@@ -497,31 +514,26 @@ attn_bwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
                     for (int e = 0; e < 8; ++e) a[ch * 8 + e] = fmaf(-cf, xr[e], a[ch * 8 + e]);
                 }
                 flush_rows(stg, lane, a, dx_acc, krow, prole, it, 2);
-                if (quad >= 2) {                     // first half of the dV columns of these rows
-#pragma unroll
-                    for (int c = 0; c < 2; ++c) tc::tmem_ld16(tl + cDV + c * 16, a + c * 16);
-                    tc::tmem_ld_wait();
-                    flush_rows32(stg, lane, a, dv_acc, krow, 0);
-                }
+                if (quad >= 2) flush_rows32(stg, lane, b, dv_acc, krow, 0);
                 if (prole >= 0 && lane == 0) LSH_PHASE(1, prole, it, 4);
             } else {
                 if (tid == 128) LSH_PHASE(1, 3, it, 0);
                 if (quad < 2) {
 #pragma unroll
                     for (int c = 0; c < 4; ++c) tc::tmem_ld16(tl + cDV + c * 16, a + c * 16);
-                    tc::tmem_ld_wait();
+                    release_tmem();
                     flush_rows(stg, lane, a, dv_acc, krow);
                 } else {
+                    // second half of the dV columns, and query row 64 + kr (chunk 2k+2)
 #pragma unroll
-                    for (int c = 0; c < 2; ++c) tc::tmem_ld16(tl + cDV + 32 + c * 16, a + c * 16);
-                    tc::tmem_ld_wait();
-                    flush_rows32(stg, lane, a, dv_acc, krow, 32);
-                    // query row 64 + kr (chunk 2k+2), staged in this stage's dY rows
-                    uint8_t *stg2 = const_cast<uint8_t *>(st.G) + (quad - 2) * 8192;
+                    for (int c = 0; c < 2; ++c) tc::tmem_ld16(tl + cDV + 32 + c * 16, b + c * 16);
 #pragma unroll
                     for (int c = 0; c < 4; ++c) tc::tmem_ld16(tl + cQb + c * 16, a + c * 16);
-                    tc::tmem_ld_wait();
+                    release_tmem();
+                    flush_rows32(stg, lane, b, dv_acc, krow, 32);
                     if (warp == 6 && lane == 0) LSH_PHASE(1, 6, it, 0);
+                    // staged in this stage's dY rows, which the MMAs no longer read
+                    uint8_t *stg2 = const_cast<uint8_t *>(st.G) + (quad - 2) * 8192;
                     const int qp = st.qpos[64 + kr];
                     flush_rows(stg2, lane, a, dx_acc, qp >= 0 ? (int)rowbase + qp : -1, warp == 6 ? 6 : -1, it, 1);
                 }
@@ -531,8 +543,8 @@ attn_bwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
             tc::tc_fence_before();
             __syncwarp();
             if (lane == 0) {
-                tc::mbar_arrive(&sm.bar_free);
                 tc::mbar_arrive(&sm.empty[s]);
+                tc::mbar_arrive(&sm.epi_done);
             }
         }
     }
