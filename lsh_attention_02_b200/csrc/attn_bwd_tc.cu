@@ -48,6 +48,7 @@ namespace {
 constexpr int kK = 128;             // key slots per tile
 constexpr int kQ = 192;             // query slots per tile
 constexpr int kStages = 2;
+constexpr int kRun = 8;             // consecutive key tiles of one segment per work unit
 constexpr int kComputeWarps = 8;
 constexpr int kProducerWarps = 3;
 constexpr int kProducerThreads = kProducerWarps * 32;
@@ -76,6 +77,7 @@ struct alignas(1024) Stage {
 struct BwdSmem {
     Stage st[kStages];
     uint8_t ET[3][kK * 128];        // tau inv_j dS^T, 3 blocks of 64 queries (48 KB)
+    uint8_t carry[2][64 * 256];     // fp32 dQ rows of chunk 2k+2 handed to the next tile (2 x 16 KB)
     uint64_t full[kStages], empty[kStages];
     uint64_t bar_s, bar_p, bar_o, bar_free;
     uint64_t gx_ready;              // the second half's partial sums of g . x are in gxh
@@ -95,45 +97,41 @@ __device__ __forceinline__ void red_add_v4(float *addr, float a, float b, float 
 // rowg < 0) with coalesced vector reductions: the warp's 32 rows go through
 // its 8 KB staging buffer (16-byte chunks swizzled by lane against bank
 // conflicts), then each reduction instruction covers two whole rows.
-__device__ __forceinline__ void flush_rows(uint8_t *stg, int lane, const float *a, float *acc, int rowg,
-                                           int ph_role = -1, int ph_it = 0, int ph_ev = 0)
+__device__ __forceinline__ void stage_rows(uint8_t *stg, int lane, const float *a)
 {
 #pragma unroll
     for (int c = 0; c < 16; ++c)
         *reinterpret_cast<float4 *>(stg + lane * 256 + ((c ^ (lane & 15)) << 4)) =
             make_float4(a[4 * c], a[4 * c + 1], a[4 * c + 2], a[4 * c + 3]);
     __syncwarp();
-    if (ph_role >= 0 && lane == 0) LSH_PHASE(1, ph_role, ph_it, ph_ev);
+}
+// `add` (nullable): 32 more rows in the same staged layout, added on the way.
+__device__ __forceinline__ void reduce_rows(const uint8_t *stg, int lane, float *acc, int rowg,
+                                            const uint8_t *add = nullptr)
+{
     const int c = lane & 15;
 #pragma unroll 4
     for (int it = 0; it < 16; ++it) {
         const int rr = 2 * it + (lane >> 4);
         const int rg = __shfl_sync(0xffffffffu, rowg, rr);
-        const float4 val = *reinterpret_cast<const float4 *>(stg + rr * 256 + ((c ^ (rr & 15)) << 4));
+        const uint32_t off = rr * 256 + ((c ^ (rr & 15)) << 4);
+        float4 val = *reinterpret_cast<const float4 *>(stg + off);
+        if (add) {
+            const float4 g = *reinterpret_cast<const float4 *>(add + off);
+            val.x += g.x; val.y += g.y; val.z += g.z; val.w += g.w;
+        }
         if (rg >= 0) red_add_v4(acc + (long long)rg * kDim + 4 * c, val.x, val.y, val.z, val.w);
     }
     __syncwarp();
-    if (ph_role >= 0 && lane == 0) LSH_PHASE(1, ph_role, ph_it, ph_ev + 1);
 }
-
-// As flush_rows for 32 columns: adds a[0..32) to columns [col0, col0 + 32) of
-// row `rowg`; each reduction instruction covers four rows.
-__device__ __forceinline__ void flush_rows32(uint8_t *stg, int lane, const float *a, float *acc, int rowg, int col0)
+__device__ __forceinline__ void flush_rows(uint8_t *stg, int lane, const float *a, float *acc, int rowg,
+                                           int ph_role = -1, int ph_it = 0, int ph_ev = 0,
+                                           const uint8_t *add = nullptr)
 {
-#pragma unroll
-    for (int c = 0; c < 8; ++c)
-        *reinterpret_cast<float4 *>(stg + lane * 128 + ((c ^ (lane & 7)) << 4)) =
-            make_float4(a[4 * c], a[4 * c + 1], a[4 * c + 2], a[4 * c + 3]);
-    __syncwarp();
-    const int c = lane & 7;
-#pragma unroll 4
-    for (int it = 0; it < 8; ++it) {
-        const int rr = 4 * it + (lane >> 3);
-        const int rg = __shfl_sync(0xffffffffu, rowg, rr);
-        const float4 val = *reinterpret_cast<const float4 *>(stg + rr * 128 + ((c ^ (rr & 7)) << 4));
-        if (rg >= 0) red_add_v4(acc + (long long)rg * kDim + col0 + 4 * c, val.x, val.y, val.z, val.w);
-    }
-    __syncwarp();
+    stage_rows(stg, lane, a);
+    if (ph_role >= 0 && lane == 0) LSH_PHASE(1, ph_role, ph_it, ph_ev);
+    reduce_rows(stg, lane, acc, rowg, add);
+    if (ph_role >= 0 && lane == 0) LSH_PHASE(1, ph_role, ph_it, ph_ev + 1);
 }
 
 // Chunk `ch` (elements 8ch .. 8ch+7) of bf16 row `row` of a K-major SW128 tile.
@@ -221,19 +219,38 @@ __device__ __forceinline__ void zero_block(uint8_t (*ET)[kK * 128], uint32_t tl,
     }
 }
 
+// Work unit u = (bh, run, r) with r fastest: key tiles k = kRun * run .. of
+// segment (bh, r), taken in order by one CTA, so the dQ rows of chunk 2k+2
+// that tile k computes can be handed to tile k+1 instead of being reduced
+// twice.  Units in flight at the same time share one head's rows in L2.
+struct TileIter {
+    long long unit;                 // >= n_units: done
+    int j;                          // tile within the unit
+};
 struct TileCoord {
     int r, k;
     long long bh, seg;
+    bool next_adjacent;             // the CTA's next tile is (seg, k + 1)
 };
-__device__ __forceinline__ TileCoord tile_coord(long long tile, int R, int n_k)
+__device__ __forceinline__ TileCoord tile_coord(const TileIter &t, int R, int n_k, int n_runs)
 {
     TileCoord c;
-    c.r = (int)(tile % R);
-    const long long bk = tile / R;
-    c.k = (int)(bk % n_k);
-    c.bh = bk / n_k;
+    c.r = (int)(t.unit % R);
+    const long long br = t.unit / R;
+    c.k = (int)(br % n_runs) * kRun + t.j;
+    c.bh = br / n_runs;
     c.seg = c.bh * R + c.r;
+    c.next_adjacent = t.j + 1 < kRun && c.k + 1 < n_k;
     return c;
+}
+__device__ __forceinline__ void tile_advance(TileIter &t, int R, int n_k, int n_runs)
+{
+    if (tile_coord(t, R, n_k, n_runs).next_adjacent) {
+        ++t.j;
+    } else {
+        t.unit += gridDim.x;
+        t.j = 0;
+    }
 }
 
 template <bool CAUSAL>
@@ -241,13 +258,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 attn_bwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__restrict__ v,
                    const __nv_bfloat16 *__restrict__ dout, const int32_t *__restrict__ perm, const float *__restrict__ invnorm,
                    const float *__restrict__ lse_all, const float *__restrict__ delta, float *__restrict__ dx_acc,
-                   float *__restrict__ dv_acc, int L, int R, long long n_tiles, int causal, float tau,
+                   float *__restrict__ dv_acc, int L, int R, long long n_units, int causal, float tau,
                    uint32_t *__restrict__ status)
 {
     extern __shared__ uint8_t smem_raw[];
     BwdSmem &sm = *reinterpret_cast<BwdSmem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int n_k = L / kK;
+    const int n_runs = (n_k + kRun - 1) / kRun;
 
     if (tid == 0) {
         for (int s = 0; s < kStages; ++s) {
@@ -275,8 +293,8 @@ attn_bwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
         // positions of slots [128k - 64, 128k + 192) of the next tile, loaded a tile ahead
         constexpr int kPosPer = (256 + kProducerThreads - 1) / kProducerThreads;
         int pn[kPosPer];
-        auto load_pos = [&](long long tile) {
-            const TileCoord c = tile_coord(tile, R, n_k);
+        auto load_pos = [&](const TileIter &t) {
+            const TileCoord c = tile_coord(t, R, n_k, n_runs);
             const int32_t *P = perm + c.seg * L;
             const int slot0 = c.k * kK - 64;
 #pragma unroll
@@ -287,9 +305,9 @@ attn_bwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
                 pn[j] = (e < 256 && sl >= 0 && sl < L) ? pl : -1;
             }
         };
-        if (blockIdx.x < n_tiles) load_pos(blockIdx.x);
-        int it = 0;
-        for (long long tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++it) {
+        TileIter ti{blockIdx.x, 0};
+        if (ti.unit < n_units) load_pos(ti);
+        for (int it = 0; ti.unit < n_units; ++it) {
             const int s = it % kStages;
             if (ptid == 0) LSH_PHASE(1, 0, it, 0);
             bool ok = it < kStages ||
@@ -297,7 +315,7 @@ attn_bwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
             if (tc::named_bar_or(1, kProducerThreads, !ok)) break;
             if (ptid == 0) LSH_PHASE(1, 0, it, 1);
             Stage &st = sm.st[s];
-            const long long rowbase = tile_coord(tile, R, n_k).bh * L;
+            const long long rowbase = tile_coord(ti, R, n_k, n_runs).bh * L;
 #pragma unroll
             for (int j = 0; j < kPosPer; ++j) {
                 const int e = ptid + j * kProducerThreads;
@@ -359,7 +377,8 @@ attn_bwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
                     st.qlim[q] = (p >= 0 && p == wmin) ? p + 1 : p;
                 }
             }
-            if (tile + gridDim.x < n_tiles) load_pos(tile + gridDim.x);
+            tile_advance(ti, R, n_k, n_runs);
+            if (ti.unit < n_units) load_pos(ti);
             if (ptid == 0) LSH_PHASE(1, 0, it, 3);
             // with two stages the producer cannot run further ahead: publish this stage now
             tc::cp_async_wait<0>();
@@ -374,8 +393,8 @@ attn_bwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
             constexpr uint32_t id_kv = tc::idesc_bf16(128, kDim, 0, 1);   // A K-major, B MN-major
             constexpr uint32_t id_q = tc::idesc_bf16(128, kDim, 1, 1);    // A MN-major, B MN-major
             const uint32_t e0 = tc::smem_u32(sm.ET[0]), e1 = tc::smem_u32(sm.ET[1]), e2 = tc::smem_u32(sm.ET[2]);
-            int it = 0;
-            for (long long tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++it) {
+            TileIter ti{blockIdx.x, 0};
+            for (int it = 0; ti.unit < n_units; ++it, tile_advance(ti, R, n_k, n_runs)) {
                 const int s = it % kStages;
                 const uint32_t ph = (uint32_t)it & 1u;
                 LSH_PHASE(1, 1, it, 0);
@@ -418,15 +437,16 @@ attn_bwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
         const int quad = warp & 3, half = warp >> 2;
         const int kr = quad * 32 + lane;
         const uint32_t tl = tmem + ((uint32_t)(quad * 32) << 16);
-        int it = 0;
-        for (long long tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++it) {
+        TileIter ti{blockIdx.x, 0};
+        bool carry_in = false;                       // this tile's chunk-2k rows hold a handed-over dQ part
+        for (int it = 0; ti.unit < n_units; ++it, tile_advance(ti, R, n_k, n_runs)) {
             const int s = it % kStages;
             const uint32_t ph = (uint32_t)it & 1u;
             if (tid == 0) LSH_PHASE(1, 2, it, 0);
             if (!tc::mbar_wait(&sm.full[s], (uint32_t)(it / kStages) & 1u, &sm.abort, status)) break;
             if (tid == 0) LSH_PHASE(1, 2, it, 1);
             const Stage &st = sm.st[s];
-            const TileCoord tcd = tile_coord(tile, R, n_k);
+            const TileCoord tcd = tile_coord(ti, R, n_k, n_runs);
             const long long rowbase = tcd.bh * L;
             const int kpos = st.pos[64 + kr];
             // 1/|x_k| of this key row from the gathered tile (sum of squares in element order)
@@ -485,7 +505,7 @@ attn_bwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
             // Every warp first moves its outputs from tensor memory to registers and
             // releases the columns, so the next tile's S^T and dP^T products run while
             // this tile's rows are reduced.
-            float a[kDim], b[kDim / 2];
+            float a[kDim];
             auto release_tmem = [&] {
                 tc::tmem_ld_wait();
                 tc::tc_fence_before();
@@ -498,10 +518,6 @@ attn_bwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
                 if (prole >= 0 && lane == 0) LSH_PHASE(1, prole, it, 0);
 #pragma unroll
                 for (int c = 0; c < 4; ++c) tc::tmem_ld16(tl + cDX + c * 16, a + c * 16);
-                if (quad >= 2) {                     // first half of the dV columns of these rows
-#pragma unroll
-                    for (int c = 0; c < 2; ++c) tc::tmem_ld16(tl + cDV + c * 16, b + c * 16);
-                }
                 release_tmem();
                 if (prole >= 0 && lane == 0) LSH_PHASE(1, prole, it, 1);
                 if (!tc::mbar_wait(&sm.gx_ready, ph, &sm.abort, status)) break;
@@ -513,8 +529,9 @@ attn_bwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
 #pragma unroll
                     for (int e = 0; e < 8; ++e) a[ch * 8 + e] = fmaf(-cf, xr[e], a[ch * 8 + e]);
                 }
-                flush_rows(stg, lane, a, dx_acc, krow, prole, it, 2);
-                if (quad >= 2) flush_rows32(stg, lane, b, dv_acc, krow, 0);
+                // chunk 2k rows: plus the previous tile's part of their dQ, when handed over
+                const uint8_t *add = quad < 2 && carry_in ? sm.carry[(it - 1) & 1] + quad * 32 * 256 : nullptr;
+                flush_rows(stg, lane, a, dx_acc, krow, prole, it, 2, add);
                 if (prole >= 0 && lane == 0) LSH_PHASE(1, prole, it, 4);
             } else {
                 if (tid == 128) LSH_PHASE(1, 3, it, 0);
@@ -524,18 +541,35 @@ attn_bwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
                     release_tmem();
                     flush_rows(stg, lane, a, dv_acc, krow);
                 } else {
-                    // second half of the dV columns, and query row 64 + kr (chunk 2k+2)
+                    // the dV row (staged first), then query row 64 + kr (chunk 2k+2): handed
+                    // to the next tile when that is k+1 of this segment, else reduced here,
+                    // staged in this stage's dY rows, which the MMAs no longer read
 #pragma unroll
-                    for (int c = 0; c < 2; ++c) tc::tmem_ld16(tl + cDV + 32 + c * 16, b + c * 16);
+                    for (int c = 0; c < 4; ++c) tc::tmem_ld16(tl + cDV + c * 16, a + c * 16);
+                    tc::tmem_ld_wait();
+                    stage_rows(stg, lane, a);
 #pragma unroll
                     for (int c = 0; c < 4; ++c) tc::tmem_ld16(tl + cQb + c * 16, a + c * 16);
                     release_tmem();
-                    flush_rows32(stg, lane, b, dv_acc, krow, 32);
                     if (warp == 6 && lane == 0) LSH_PHASE(1, 6, it, 0);
-                    // staged in this stage's dY rows, which the MMAs no longer read
                     uint8_t *stg2 = const_cast<uint8_t *>(st.G) + (quad - 2) * 8192;
-                    const int qp = st.qpos[64 + kr];
-                    flush_rows(stg2, lane, a, dx_acc, qp >= 0 ? (int)rowbase + qp : -1, warp == 6 ? 6 : -1, it, 1);
+                    if (tcd.next_adjacent) {
+                        const int cr = kr - 64;
+                        uint8_t *cb = sm.carry[it & 1] + cr * 256;
+#pragma unroll
+                        for (int c = 0; c < 16; ++c)
+                            *reinterpret_cast<float4 *>(cb + ((c ^ (cr & 15)) << 4)) =
+                                make_float4(a[4 * c], a[4 * c + 1], a[4 * c + 2], a[4 * c + 3]);
+                    } else {
+                        stage_rows(stg2, lane, a);
+                    }
+                    reduce_rows(stg, lane, dv_acc, krow);
+                    if (warp == 6 && lane == 0) LSH_PHASE(1, 6, it, 1);
+                    if (!tcd.next_adjacent) {
+                        const int qp = st.qpos[64 + kr];
+                        reduce_rows(stg2, lane, dx_acc, qp >= 0 ? (int)rowbase + qp : -1);
+                    }
+                    if (warp == 6 && lane == 0) LSH_PHASE(1, 6, it, 2);
                 }
                 if (tid == 128) LSH_PHASE(1, 3, it, 1);
             }
@@ -546,6 +580,7 @@ attn_bwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
                 tc::mbar_arrive(&sm.empty[s]);
                 tc::mbar_arrive(&sm.epi_done);
             }
+            carry_in = tcd.next_adjacent;
         }
     }
 
@@ -563,6 +598,7 @@ cudaError_t launch_attn_bwd_tc(const Problem &p, const void *x, const void *v, c
                                const float *invnorm, const float *lse_all, const float *delta, float *dx_acc,
                                float *dv_acc, uint32_t *status, cudaStream_t st)
 {
+    static_assert(sizeof(BwdSmem) + 1024 <= 232448, "shared memory per CTA");
     const size_t smem = sizeof(BwdSmem) + 1024;
     auto kern = p.causal ? attn_bwd_tc_kernel<true> : attn_bwd_tc_kernel<false>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -570,11 +606,11 @@ cudaError_t launch_attn_bwd_tc(const Problem &p, const void *x, const void *v, c
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    const long long n_tiles = p.S() * (p.L / kK);
-    const unsigned grid = (unsigned)std::min<long long>(n_tiles, (long long)sms);
+    const long long n_units = p.S() * ((p.L / kK + kRun - 1) / kRun);
+    const unsigned grid = (unsigned)std::min<long long>(n_units, (long long)sms);
     kern<<<grid, kThreads, smem, st>>>((const __nv_bfloat16 *)x, (const __nv_bfloat16 *)v,
                                                      (const __nv_bfloat16 *)dout, perm, invnorm, lse_all,
-                                                     delta, dx_acc, dv_acc, p.L, p.R, n_tiles, p.causal,
+                                                     delta, dx_acc, dv_acc, p.L, p.R, n_units, p.causal,
                                                      1.0f / sqrtf((float)p.d), status);
     return cudaGetLastError();
 }
