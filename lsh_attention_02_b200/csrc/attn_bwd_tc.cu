@@ -87,10 +87,11 @@ struct BwdSmem {
     int abort;
 };
 
+// Nothing in the kernel reads the accumulators, so the reduction carries no
+// memory clobber: shared-memory loads around it may be scheduled freely.
 __device__ __forceinline__ void red_add_v4(float *addr, float a, float b, float c, float d)
 {
-    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
-                 : "memory");
+    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b), "f"(c), "f"(d));
 }
 
 // Adds each lane's 64-float row `a` to row `rowg` of `acc` (skipped when
@@ -146,62 +147,79 @@ __device__ __forceinline__ void smem_chunk(const uint8_t *tile, int row, int ch,
     }
 }
 
+// One step of 16 query columns [C0 + 16 STEP, +16) of key row kr from the
+// S^T and dP^T values s, dp: P^T into TMEM, E^T into shared memory.
+template <bool CAUSAL, int STEP>
+__device__ __forceinline__ void key_row_step(const Stage &st, uint8_t (*ET)[kK * 128], uint32_t tl, int kr, int kpos,
+                                             int C0, float sc, float ec, const float *s, const float *dp, float &gx)
+{
+    uint32_t pw[8], ew[8];
+#pragma unroll
+    for (int j4 = 0; j4 < 16; j4 += 4) {
+        const int q0 = C0 + STEP * 16 + j4;
+        // causal: key admitted iff its position < qlim; otherwise iff it differs from the query
+        const int4 qp4 = *reinterpret_cast<const int4 *>(CAUSAL ? &st.qlim[q0] : &st.qpos[q0]);
+        const float4 ql4 = *reinterpret_cast<const float4 *>(&st.qlse2[q0]);
+        const float4 qd4 = *reinterpret_cast<const float4 *>(&st.qdelta[q0]);
+        const int qp[4] = {qp4.x, qp4.y, qp4.z, qp4.w};
+        const float ql[4] = {ql4.x, ql4.y, ql4.z, ql4.w};
+        const float qd[4] = {qd4.x, qd4.y, qd4.z, qd4.w};
+        float pv[4], ev[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const bool ok = CAUSAL ? (kpos < qp[u]) : (kpos != qp[u]);
+            const float e2 = tc::fast_exp2(fmaf(s[j4 + u], sc, -ql[u]));
+            pv[u] = ok ? e2 : 0.f;
+            ev[u] = ec * pv[u] * (dp[j4 + u] - qd[u]);
+            gx = fmaf(ev[u], s[j4 + u], gx);
+        }
+        pw[j4 / 2] = pack_bf16x2(pv[0], pv[1]);
+        pw[j4 / 2 + 1] = pack_bf16x2(pv[2], pv[3]);
+        ew[j4 / 2] = pack_bf16x2(ev[0], ev[1]);
+        ew[j4 / 2 + 1] = pack_bf16x2(ev[2], ev[3]);
+    }
+    tc::tmem_st8(tl + cPT + C0 / 2 + STEP * 8, pw);
+    const int blk = C0 >> 6;
+#pragma unroll
+    for (int c2 = 0; c2 < 2; ++c2) {
+        const int ch = STEP * 2 + c2;
+        const uint32_t off = (uint32_t)kr * 128u + (uint32_t)((ch ^ (kr & 7)) << 4);
+        *reinterpret_cast<uint4 *>(ET[blk] + off) = make_uint4(ew[4 * c2], ew[4 * c2 + 1], ew[4 * c2 + 2], ew[4 * c2 + 3]);
+    }
+}
+
 // Elementwise step for key row kr over query columns [C0, C0 + 64): P^T (bf16)
-// into TMEM columns cPT + C0/2, E^T into shared-memory block C0/64.  A
+// into TMEM columns cPT + C0/2, E^T into shared-memory block C0/64, in four
+// steps of 16 columns whose tensor-memory loads run one step ahead.  A
 // candidate is a query at a later original position (causal) or at any other
 // position; a causal query with no other candidate takes its own key.  Query
 // metadata is read four queries per vector load.  Returns this block's part of
-// g . x = sum_i e_i (x_i . x_k).
-template <int C0, bool CAUSAL>
+// g . x = sum_i e_i (x_i . x_k).  C0 is a run-time value so that the warps of
+// all three column blocks share one copy of the code.
+template <bool CAUSAL>
 __device__ __forceinline__ float key_row_block(const Stage &st, uint8_t (*ET)[kK * 128], uint32_t tl, int kr, int kpos,
-                                              float kinv, float tau)
+                                           int C0, float kinv, float tau)
 {
     const float sc = tau * kinv * kLog2e;
     const float ec = tau * kinv;
     float gx = 0.f;
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {                       // two halves of 32 query columns
-        float s[32], dp[32];
-        tc::tmem_ld16(tl + cS + C0 + h * 32, s);
-        tc::tmem_ld16(tl + cS + C0 + h * 32 + 16, s + 16);
-        tc::tmem_ld16(tl + cD + C0 + h * 32, dp);
-        tc::tmem_ld16(tl + cD + C0 + h * 32 + 16, dp + 16);
-        tc::tmem_ld_wait();
-        uint32_t pw[16], ew[16];
-#pragma unroll
-        for (int j4 = 0; j4 < 32; j4 += 4) {
-            const int q0 = C0 + h * 32 + j4;
-            // causal: key admitted iff its position < qlim; otherwise iff it differs from the query
-            const int4 qp4 = *reinterpret_cast<const int4 *>(CAUSAL ? &st.qlim[q0] : &st.qpos[q0]);
-            const float4 ql4 = *reinterpret_cast<const float4 *>(&st.qlse2[q0]);
-            const float4 qd4 = *reinterpret_cast<const float4 *>(&st.qdelta[q0]);
-            const int qp[4] = {qp4.x, qp4.y, qp4.z, qp4.w};
-            const float ql[4] = {ql4.x, ql4.y, ql4.z, ql4.w};
-            const float qd[4] = {qd4.x, qd4.y, qd4.z, qd4.w};
-            float pv[4], ev[4];
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const bool ok = CAUSAL ? (kpos < qp[u]) : (kpos != qp[u]);
-                const float e2 = tc::fast_exp2(fmaf(s[j4 + u], sc, -ql[u]));
-                pv[u] = ok ? e2 : 0.f;
-                ev[u] = ec * pv[u] * (dp[j4 + u] - qd[u]);
-                gx = fmaf(ev[u], s[j4 + u], gx);
-            }
-            pw[j4 / 2] = pack_bf16x2(pv[0], pv[1]);
-            pw[j4 / 2 + 1] = pack_bf16x2(pv[2], pv[3]);
-            ew[j4 / 2] = pack_bf16x2(ev[0], ev[1]);
-            ew[j4 / 2 + 1] = pack_bf16x2(ev[2], ev[3]);
-        }
-        tc::tmem_st16(tl + cPT + C0 / 2 + h * 16, pw);
-        constexpr int blk = C0 / 64;
-#pragma unroll
-        for (int c4 = 0; c4 < 4; ++c4) {
-            const int ch = h * 4 + c4;
-            const uint32_t off = (uint32_t)kr * 128u + (uint32_t)((ch ^ (kr & 7)) << 4);
-            *reinterpret_cast<uint4 *>(ET[blk] + off) =
-                make_uint4(ew[4 * c4], ew[4 * c4 + 1], ew[4 * c4 + 2], ew[4 * c4 + 3]);
-        }
-    }
+    float sa[16], da[16], sb[16], db[16];
+    tc::tmem_ld16(tl + cS + C0, sa);
+    tc::tmem_ld16(tl + cD + C0, da);
+    tc::tmem_ld_wait();
+    tc::tmem_ld16(tl + cS + C0 + 16, sb);
+    tc::tmem_ld16(tl + cD + C0 + 16, db);
+    key_row_step<CAUSAL, 0>(st, ET, tl, kr, kpos, C0, sc, ec, sa, da, gx);
+    tc::tmem_ld_wait();
+    tc::tmem_ld16(tl + cS + C0 + 32, sa);
+    tc::tmem_ld16(tl + cD + C0 + 32, da);
+    key_row_step<CAUSAL, 1>(st, ET, tl, kr, kpos, C0, sc, ec, sb, db, gx);
+    tc::tmem_ld_wait();
+    tc::tmem_ld16(tl + cS + C0 + 48, sb);
+    tc::tmem_ld16(tl + cD + C0 + 48, db);
+    key_row_step<CAUSAL, 2>(st, ET, tl, kr, kpos, C0, sc, ec, sa, da, gx);
+    tc::tmem_ld_wait();
+    key_row_step<CAUSAL, 3>(st, ET, tl, kr, kpos, C0, sc, ec, sb, db, gx);
     return gx;
 }
 
@@ -468,24 +486,21 @@ attn_bwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
             // ---- elementwise.  E^T and gxh are rewritten here: wait until no warp still
             // stages the previous tile's rows in them.
             if (it > 0 && !tc::mbar_wait(&sm.epi_done, (uint32_t)(it - 1) & 1u, &sm.abort, status)) break;
+            const int erole_ev = warp == 0 ? 0 : warp == 4 ? 4 : -1;
+            if (erole_ev >= 0 && lane == 0) LSH_PHASE(1, 7, it, erole_ev);
             float gx;                                // partial g . x of key row kr
-            if (quad < 2) {                          // keys of chunk 2k: queries of chunks 2k, 2k+1
-                if (half == 0) {
-                    gx = key_row_block<0, CAUSAL>(st, sm.ET, tl, kr, kpos, kinv, tau);
-                    zero_block<128>(sm.ET, tl, kr);
-                } else {
-                    gx = key_row_block<64, CAUSAL>(st, sm.ET, tl, kr, kpos, kinv, tau);
-                }
-            } else {                                 // keys of chunk 2k+1: queries of chunks 2k+1, 2k+2
-                if (half == 0) {
-                    gx = key_row_block<64, CAUSAL>(st, sm.ET, tl, kr, kpos, kinv, tau);
-                    zero_block<0>(sm.ET, tl, kr);
-                } else {
-                    gx = key_row_block<128, CAUSAL>(st, sm.ET, tl, kr, kpos, kinv, tau);
-                }
+            // keys of chunk 2k (quads 0, 1) see queries of chunks 2k, 2k+1 (columns 0..127),
+            // keys of chunk 2k+1 those of chunks 2k+1, 2k+2 (64..191); each half takes 64
+            const int c0 = quad < 2 ? half * 64 : 64 + half * 64;
+            gx = key_row_block<CAUSAL>(st, sm.ET, tl, kr, kpos, c0, kinv, tau);
+            if (half == 0) {
+                if (quad < 2) zero_block<128>(sm.ET, tl, kr);
+                else zero_block<0>(sm.ET, tl, kr);
             }
+            if (erole_ev >= 0 && lane == 0) LSH_PHASE(1, 7, it, erole_ev + 1);
             if (half == 1) sm.gxh[kr] = gx;
             tc::tmem_st_wait();
+            if (erole_ev >= 0 && lane == 0) LSH_PHASE(1, 7, it, erole_ev + 2);
             tc::fence_async_smem();
             tc::tc_fence_before();
             __syncwarp();
