@@ -106,8 +106,9 @@ __device__ __forceinline__ TileCoord tile_coord(long long tile, int R, int n_k)
 // Candidates: keys at an earlier original position (causal) or at any other
 // position (non-causal).  A causal row with none (its position is the
 // smallest of its window) gets l = 0 here and is patched by the caller.
-template <int BASE, bool CAUSAL, bool FIRST>
-__device__ __forceinline__ float softmax_sweep(const Stage &st, uint32_t tl, int qpos, float shift2)
+template <bool CAUSAL>
+__device__ __forceinline__ float softmax_sweep(const Stage &st, uint32_t tl, int qpos, float shift2, int BASE,
+                                               bool FIRST)
 {
     float lsum = 0.f;
 #pragma unroll 1
@@ -148,7 +149,7 @@ __device__ __forceinline__ float softmax_sweep(const Stage &st, uint32_t tl, int
     }
     {
         const uint32_t z[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-        constexpr uint32_t zc = BASE == 0 ? 64 : 0;             // packed columns of keys 128..191 or 0..63
+        const uint32_t zc = BASE == 0 ? 64 : 0;                 // packed columns of keys 128..191 or 0..63
 #pragma unroll
         for (int c = 0; c < 4; ++c) tc::tmem_st8(tl + zc + c * 8, z);
     }
@@ -157,8 +158,8 @@ __device__ __forceinline__ float softmax_sweep(const Stage &st, uint32_t tl, int
 
 // Exact row maximum of the log2-domain scores (only for rows whose bound
 // tau |x_i| is so loose that exp(s - bound) could leave the normal range).
-template <int BASE, bool CAUSAL>
-__device__ __forceinline__ float exact_max(const Stage &st, uint32_t tl, int jlo, int qpos)
+template <bool CAUSAL>
+__device__ __forceinline__ float exact_max(const Stage &st, uint32_t tl, int jlo, int qpos, int BASE)
 {
     float mx = -INFINITY;
 #pragma unroll 1
@@ -177,18 +178,18 @@ __device__ __forceinline__ float exact_max(const Stage &st, uint32_t tl, int jlo
     return mx;
 }
 
-template <int BASE, bool CAUSAL, bool FIRST>
+template <bool CAUSAL>
 __device__ __forceinline__ void softmax_row(const Stage &st, uint32_t tl, int i, int qpos, float qinv, bool self_only,
-                                            float tau, float &l, float &row_lse)
+                                            float tau, int BASE, bool FIRST, float &l, float &row_lse)
 {
     const float bound = qinv > 0.f ? tau / qinv : 0.f;        // tau |x_i| >= every score of the row
     float shift2 = bound * kLog2e;                              // log2-domain offset
     const bool wide = 2.f * bound * kLog2e > 100.f;             // bound - s <= 2 bound
     if (__any_sync(0xffffffffu, wide)) {
-        const float mx = exact_max<BASE, CAUSAL>(st, tl, FIRST && BASE == 0 ? 64 : 0, qpos);
+        const float mx = exact_max<CAUSAL>(st, tl, FIRST && BASE == 0 ? 64 : 0, qpos, BASE);
         if (wide && mx > -INFINITY) shift2 = mx;
     }
-    l = softmax_sweep<BASE, CAUSAL, FIRST>(st, tl, qpos, shift2);
+    l = softmax_sweep<CAUSAL>(st, tl, qpos, shift2, BASE, FIRST);
     row_lse = kLn2 * (shift2 + log2f(l));
     if (CAUSAL && __any_sync(0xffffffffu, self_only)) {
         // A row with no candidate attends to itself: p = 1 on its own key (window
@@ -437,9 +438,8 @@ attn_fwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
             const bool self_only = CAUSAL && qpos == min(st.cmin[a], st.cmin[a + 1]);
             const bool first = tcd.k == 0;
             float l, row_lse;
-            if (q >= 2) softmax_row<64, CAUSAL, false>(st, tl, i, qpos, qinv, self_only, tau, l, row_lse);
-            else if (first) softmax_row<0, CAUSAL, true>(st, tl, i, qpos, qinv, self_only, tau, l, row_lse);
-            else softmax_row<0, CAUSAL, false>(st, tl, i, qpos, qinv, self_only, tau, l, row_lse);
+            // one run-time-parameterised copy of the row code for every warp (instruction cache)
+            softmax_row<CAUSAL>(st, tl, i, qpos, qinv, self_only, tau, q >= 2 ? 64 : 0, first && q < 2, l, row_lse);
             tc::tmem_st_wait();
             tc::tc_fence_before();
             __syncwarp();
