@@ -136,6 +136,24 @@ __device__ __forceinline__ void flush_rows(uint8_t *stg, int lane, const float *
 }
 
 // Chunk `ch` (elements 8ch .. 8ch+7) of bf16 row `row` of a K-major SW128 tile.
+__device__ __forceinline__ void smem_chunk(const uint8_t *tile, int row, int ch, float *out);
+
+// 1/|x| of row `row` of a gathered K-major SW128 tile (sum of squares in element
+// order; 0 for a zero row).
+__device__ __forceinline__ float key_inv_norm(const uint8_t *X, int row)
+{
+    float ssq = 0.f;
+#pragma unroll
+    for (int ch = 0; ch < 8; ++ch) {
+        float xr[8];
+        smem_chunk(X, row, ch, xr);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) ssq = fmaf(xr[e], xr[e], ssq);
+    }
+    return ssq > 0.f ? 1.0f / sqrtf(ssq) : 0.f;
+}
+
+// Chunk `ch` (elements 8ch .. 8ch+7) of bf16 row `row` of a K-major SW128 tile.
 __device__ __forceinline__ void smem_chunk(const uint8_t *tile, int row, int ch, float *out)
 {
     const uint4 u = *reinterpret_cast<const uint4 *>(tile + row * 128 + ((ch ^ (row & 7)) << 4));
@@ -457,6 +475,8 @@ attn_bwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
         const uint32_t tl = tmem + ((uint32_t)(quad * 32) << 16);
         TileIter ti{blockIdx.x, 0};
         bool carry_in = false;                       // this tile's chunk-2k rows hold a handed-over dQ part
+        bool have_next_kinv = false;
+        float next_kinv = 0.f;
         for (int it = 0; ti.unit < n_units; ++it, tile_advance(ti, R, n_k, n_runs)) {
             const int s = it % kStages;
             const uint32_t ph = (uint32_t)it & 1u;
@@ -467,19 +487,8 @@ attn_bwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
             const TileCoord tcd = tile_coord(ti, R, n_k, n_runs);
             const long long rowbase = tcd.bh * L;
             const int kpos = st.pos[64 + kr];
-            // 1/|x_k| of this key row from the gathered tile (sum of squares in element order)
-            float kinv;
-            {
-                float ssq = 0.f;
-#pragma unroll
-                for (int ch = 0; ch < 8; ++ch) {
-                    float xr[8];
-                    smem_chunk(st.X, kr, ch, xr);
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) ssq = fmaf(xr[e], xr[e], ssq);
-                }
-                kinv = ssq > 0.f ? 1.0f / sqrtf(ssq) : 0.f;
-            }
+            // 1/|x_k| of this key row, unless computed while the previous tile's products ran
+            const float kinv = have_next_kinv ? next_kinv : key_inv_norm(st.X, kr);
             if (!tc::mbar_wait(&sm.bar_s, ph, &sm.abort, status)) break;
             if (tid == 0) LSH_PHASE(1, 2, it, 2);
             tc::tc_fence_after();
@@ -509,6 +518,18 @@ attn_bwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
                 if (half == 1) tc::mbar_arrive(&sm.gx_ready);
             }
             if (tid == 0) LSH_PHASE(1, 2, it, 3);
+            // the next tile's key norm while this tile's products run
+            have_next_kinv = false;
+            {
+                TileIter nx = ti;
+                tile_advance(nx, R, n_k, n_runs);
+                if (nx.unit < n_units) {
+                    const int s2 = (it + 1) % kStages;
+                    if (!tc::mbar_wait(&sm.full[s2], (uint32_t)((it + 1) / kStages) & 1u, &sm.abort, status)) break;
+                    next_kinv = key_inv_norm(sm.st[s2].X, kr);
+                    have_next_kinv = true;
+                }
+            }
             if (!tc::mbar_wait(&sm.bar_o, ph, &sm.abort, status)) break;
             if (tid == 0) LSH_PHASE(1, 2, it, 4);
             tc::tc_fence_after();
