@@ -204,6 +204,9 @@ __global__ void combine_kernel(const OT *__restrict__ o_r, const float *__restri
 
 // bf16 round outputs: 8 threads per token, eight features each (16-byte loads
 // and stores); the token's logsumexps are read by every thread of its group.
+// RMAX > 0: the R <= RMAX round rows are all loaded before any arithmetic, so
+// their memory latencies overlap; RMAX = 0 handles any R one round at a time.
+template <int RMAX>
 __global__ void combine_bf16_kernel(const __nv_bfloat16 *__restrict__ o_r, const float *__restrict__ lse,
                                     __nv_bfloat16 *__restrict__ out, long long tokens, int L, int R)
 {
@@ -214,21 +217,44 @@ __global__ void combine_bf16_kernel(const __nv_bfloat16 *__restrict__ o_r, const
     long long bh = tok / L;
     int i = (int)(tok % L);
     const float *lp = lse + bh * R * (long long)L + i;
-    float mx = -INFINITY;
-    for (int r = 0; r < R; ++r) mx = fmaxf(mx, lp[(long long)r * L]);
-    float ssum = 0.f;
-    for (int r = 0; r < R; ++r) ssum += expf(lp[(long long)r * L] - mx);
-    const float big = mx + logf(ssum);
+    const uint4 *orow = reinterpret_cast<const uint4 *>(o_r + (bh * R * (long long)L + i) * kDim) + oct;
+    const long long rstride = (long long)L * kDim / 8;          // one round, in 16-byte units
     float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    for (int r = 0; r < R; ++r) {
-        const float wr = expf(lp[(long long)r * L] - big);
-        const uint4 u = reinterpret_cast<const uint4 *>(o_r + ((bh * R + r) * L + i) * kDim)[oct];
+    auto accumulate = [&](float wr, const uint4 &u) {
         const uint32_t wd[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
             acc[2 * e] = fmaf(wr, __uint_as_float(wd[e] << 16), acc[2 * e]);
             acc[2 * e + 1] = fmaf(wr, __uint_as_float(wd[e] & 0xFFFF0000u), acc[2 * e + 1]);
         }
+    };
+    if (RMAX > 0) {
+        uint4 u[RMAX > 0 ? RMAX : 1];
+        float lr[RMAX > 0 ? RMAX : 1];
+#pragma unroll
+        for (int r = 0; r < RMAX; ++r) {
+            u[r] = r < R ? __ldg(orow + r * rstride) : make_uint4(0, 0, 0, 0);
+            lr[r] = r < R ? __ldg(lp + (long long)r * L) : -INFINITY;
+        }
+        float mx = -INFINITY;
+#pragma unroll
+        for (int r = 0; r < RMAX; ++r) mx = fmaxf(mx, lr[r]);
+        float w[RMAX > 0 ? RMAX : 1], ssum = 0.f;
+#pragma unroll
+        for (int r = 0; r < RMAX; ++r) {
+            w[r] = r < R ? expf(lr[r] - mx) : 0.f;
+            ssum += w[r];
+        }
+        const float inv = 1.f / ssum;
+#pragma unroll
+        for (int r = 0; r < RMAX; ++r) accumulate(w[r] * inv, u[r]);
+    } else {
+        float mx = -INFINITY;
+        for (int r = 0; r < R; ++r) mx = fmaxf(mx, lp[(long long)r * L]);
+        float ssum = 0.f;
+        for (int r = 0; r < R; ++r) ssum += expf(lp[(long long)r * L] - mx);
+        const float big = mx + logf(ssum);
+        for (int r = 0; r < R; ++r) accumulate(expf(lp[(long long)r * L] - big), orow[r * rstride]);
     }
     reinterpret_cast<uint4 *>(out + tok * kDim)[oct] =
         make_uint4(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]), pack_bf16x2(acc[4], acc[5]),
@@ -240,8 +266,9 @@ cudaError_t launch_combine(const Problem &p, const void *o_r, bool o_r_bf16, con
 {
     if (p.dtype == LSH_BF16 && o_r_bf16) {
         long long threads = p.tokens() * 8;
-        combine_bf16_kernel<<<(unsigned)((threads + 255) / 256), 256, 0, st>>>(
-            (const __nv_bfloat16 *)o_r, lse, (__nv_bfloat16 *)out, p.tokens(), p.L, p.R);
+        const unsigned grid = (unsigned)((threads + 255) / 256);
+        auto kern = p.R <= 4 ? combine_bf16_kernel<4> : p.R <= 8 ? combine_bf16_kernel<8> : combine_bf16_kernel<0>;
+        kern<<<grid, 256, 0, st>>>((const __nv_bfloat16 *)o_r, lse, (__nv_bfloat16 *)out, p.tokens(), p.L, p.R);
         return cudaGetLastError();
     }
     long long threads = p.tokens() * 16;

@@ -63,7 +63,7 @@ def full_check(w: synth.Workload, impl=lsh.IMPL_AUTO, heads=None):
 # ------------------------------------------------------------------ stage: hash
 @pytest.mark.parametrize("impl", IMPLS)
 @pytest.mark.parametrize("dtype,nb,nh", [("f32", 16, 1), ("bf16", 64, 2), ("bf16", 1024, 3), ("bf16", 192, 2),
-                                         ("bf16", 2, 2), ("f32", 8192, 1)])
+                                         ("bf16", 128, 2), ("bf16", 2, 2), ("f32", 8192, 1)])
 def test_hash_bit_exact_up_to_near_ties(impl, dtype, nb, nh):
     w = small("bf16_causal_4k", B=2, H=2, L=1024 if nb < 8192 else 256, n_buckets=nb, n_hashes=nh, dtype=dtype)
     inp = synth.make_inputs(w)
