@@ -74,7 +74,7 @@ struct alignas(1024) Stage {
 struct FwdSmem {
     Stage st[kStages];
     uint64_t full[kStages], empty[kStages];
-    uint64_t s_full[2], p_full[2], o_full[2], o_free[2];
+    uint64_t s_full[2], p_half[2], p_full[2], o_full[2], o_free[2];  // p_half: P of keys 0..63 written
     uint32_t tmem_base;
     int abort;
 };
@@ -108,50 +108,62 @@ __device__ __forceinline__ TileCoord tile_coord(long long tile, int R, int n_k)
 // smallest of its window) gets l = 0 here and is patched by the caller.
 template <bool CAUSAL>
 __device__ __forceinline__ float softmax_sweep(const Stage &st, uint32_t tl, int qpos, float shift2, int BASE,
-                                               bool FIRST)
+                                               bool FIRST, uint64_t *half_done)
 {
     float lsum = 0.f;
+    const uint32_t z[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    // Keys 0..63 must be complete for every row after the first half-sweep: rows
+    // of chunk 2k+1 (BASE 64) cannot see them and clear their packed columns
+    // first (their S columns there are unused); rows of chunk 2k clear keys
+    // 128..191 last, since those packed columns still hold S values they read.
+    if (BASE != 0) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tc::tmem_st8(tl + (uint32_t)(c * 8), z);
+    }
 #pragma unroll 1
     for (int h = 0; h < 2; ++h) {
         if (FIRST && BASE == 0 && h == 0) {                     // missing chunk -1
-            const uint32_t z[8] = {0, 0, 0, 0, 0, 0, 0, 0};
 #pragma unroll
             for (int c = 0; c < 4; ++c) tc::tmem_st8(tl + (uint32_t)(c * 8), z);
-            continue;
-        }
-        float v[64];
-#pragma unroll
-        for (int c = 0; c < 4; ++c) tc::tmem_ld16(tl + (uint32_t)(BASE + h * 64 + c * 16), v + c * 16);
-        tc::tmem_ld_wait();
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-            uint32_t w[8];
-#pragma unroll
-            for (int e4 = 0; e4 < 16; e4 += 4) {
-                const int j0 = h * 64 + c * 16 + e4;
-                const int4 kp = *reinterpret_cast<const int4 *>(&st.pos[BASE + j0]);
-                const float4 ks = *reinterpret_cast<const float4 *>(&st.sinv[BASE + j0]);
-                const int kpa[4] = {kp.x, kp.y, kp.z, kp.w};
-                const float ksa[4] = {ks.x, ks.y, ks.z, ks.w};
-                float pe[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const bool ok = CAUSAL ? (kpa[e] < qpos) : (kpa[e] != qpos);
-                    const float p = tc::fast_exp2(fmaf(v[c * 16 + e4 + e], ksa[e], -shift2));
-                    pe[e] = ok ? p : 0.f;
-                    lsum += pe[e];
+        } else {
+            float v[64];
+    #pragma unroll
+            for (int c = 0; c < 4; ++c) tc::tmem_ld16(tl + (uint32_t)(BASE + h * 64 + c * 16), v + c * 16);
+            tc::tmem_ld_wait();
+    #pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                uint32_t w[8];
+    #pragma unroll
+                for (int e4 = 0; e4 < 16; e4 += 4) {
+                    const int j0 = h * 64 + c * 16 + e4;
+                    const int4 kp = *reinterpret_cast<const int4 *>(&st.pos[BASE + j0]);
+                    const float4 ks = *reinterpret_cast<const float4 *>(&st.sinv[BASE + j0]);
+                    const int kpa[4] = {kp.x, kp.y, kp.z, kp.w};
+                    const float ksa[4] = {ks.x, ks.y, ks.z, ks.w};
+                    float pe[4];
+    #pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const bool ok = CAUSAL ? (kpa[e] < qpos) : (kpa[e] != qpos);
+                        const float p = tc::fast_exp2(fmaf(v[c * 16 + e4 + e], ksa[e], -shift2));
+                        pe[e] = ok ? p : 0.f;
+                        lsum += pe[e];
+                    }
+                    w[e4 / 2] = pack_bf16x2(pe[0], pe[1]);
+                    w[e4 / 2 + 1] = pack_bf16x2(pe[2], pe[3]);
                 }
-                w[e4 / 2] = pack_bf16x2(pe[0], pe[1]);
-                w[e4 / 2 + 1] = pack_bf16x2(pe[2], pe[3]);
+                tc::tmem_st8(tl + (uint32_t)(BASE / 2 + h * 32 + c * 8), w);
             }
-            tc::tmem_st8(tl + (uint32_t)(BASE / 2 + h * 32 + c * 8), w);
+        }
+        if (h == 0) {
+            tc::tmem_st_wait();
+            tc::tc_fence_before();
+            __syncwarp();
+            if ((threadIdx.x & 31) == 0) tc::mbar_arrive(half_done);
         }
     }
-    {
-        const uint32_t z[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-        const uint32_t zc = BASE == 0 ? 64 : 0;                 // packed columns of keys 128..191 or 0..63
+    if (BASE == 0) {
 #pragma unroll
-        for (int c = 0; c < 4; ++c) tc::tmem_st8(tl + zc + c * 8, z);
+        for (int c = 0; c < 4; ++c) tc::tmem_st8(tl + 64 + (uint32_t)(c * 8), z);
     }
     return lsum;
 }
@@ -180,7 +192,8 @@ __device__ __forceinline__ float exact_max(const Stage &st, uint32_t tl, int jlo
 
 template <bool CAUSAL>
 __device__ __forceinline__ void softmax_row(const Stage &st, uint32_t tl, int i, int qpos, float qinv, bool self_only,
-                                            float tau, int BASE, bool FIRST, float &l, float &row_lse)
+                                            float tau, int BASE, bool FIRST, uint64_t *half_done, float &l,
+                                            float &row_lse)
 {
     const float bound = qinv > 0.f ? tau / qinv : 0.f;        // tau |x_i| >= every score of the row
     float shift2 = bound * kLog2e;                              // log2-domain offset
@@ -189,7 +202,7 @@ __device__ __forceinline__ void softmax_row(const Stage &st, uint32_t tl, int i,
         const float mx = exact_max<CAUSAL>(st, tl, FIRST && BASE == 0 ? 64 : 0, qpos, BASE);
         if (wide && mx > -INFINITY) shift2 = mx;
     }
-    l = softmax_sweep<CAUSAL>(st, tl, qpos, shift2, BASE, FIRST);
+    l = softmax_sweep<CAUSAL>(st, tl, qpos, shift2, BASE, FIRST, half_done);
     row_lse = kLn2 * (shift2 + log2f(l));
     if (CAUSAL && __any_sync(0xffffffffu, self_only)) {
         // A row with no candidate attends to itself: p = 1 on its own key (window
@@ -257,6 +270,7 @@ attn_fwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
         }
         for (int g = 0; g < 2; ++g) {
             tc::mbar_init(&sm.s_full[g], 1);
+            tc::mbar_init(&sm.p_half[g], 4);
             tc::mbar_init(&sm.p_full[g], 4);
             tc::mbar_init(&sm.o_full[g], 1);
             tc::mbar_init(&sm.o_free[g], 4);
@@ -357,7 +371,7 @@ attn_fwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
             constexpr uint32_t id_o = tc::idesc_bf16(128, kDim, 0, 1);
             long long n_mine = 0;
             if (blockIdx.x < n_tiles) n_mine = (n_tiles - 1 - blockIdx.x) / gridDim.x + 1;
-            int next_s = 0, next_o = 0;                     // next tile (local index) for S and for O
+            int next_s = 0, next_oh = 0, next_o = 0;        // next tile (local index) for S, O's first keys, O
             long long t0 = clock64();
             while (next_o < n_mine) {
                 bool progressed = false;
@@ -379,7 +393,22 @@ attn_fwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
                         progressed = true;
                     }
                 }
-                if (next_o < next_s) {
+                if (next_oh < next_s) {
+                    // keys 0..63 as soon as every row's P there is written
+                    const int it = next_oh, s = it % kStages, g = it & 1;
+                    if (tc::mbar_test_wait(&sm.p_half[g], (uint32_t)(it >> 1) & 1u)) {
+                        tc::tc_fence_after();
+                        const uint32_t vs = tc::smem_u32(sm.st[s].V);
+                        const uint32_t base = tmem + (uint32_t)g * kGroupCols;
+#pragma unroll
+                        for (int kk = 0; kk < 4; ++kk)
+                            tc::mma_bf16_ts(base + kOCol, base + kk * 8, tc::sw128_desc(vs + kk * 16 * 128), id_o,
+                                            kk > 0);
+                        ++next_oh;
+                        progressed = true;
+                    }
+                }
+                if (next_o < next_oh) {
                     const int it = next_o, s = it % kStages, g = it & 1;
                     if (tc::mbar_test_wait(&sm.p_full[g], (uint32_t)(it >> 1) & 1u)) {
                         LSH_PHASE(0, 1, it, 3);
@@ -387,9 +416,9 @@ attn_fwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
                         const uint32_t vs = tc::smem_u32(sm.st[s].V);
                         const uint32_t base = tmem + (uint32_t)g * kGroupCols;
 #pragma unroll
-                        for (int kk = 0; kk < 12; ++kk)
+                        for (int kk = 4; kk < 12; ++kk)
                             tc::mma_bf16_ts(base + kOCol, base + kk * 8, tc::sw128_desc(vs + kk * 16 * 128), id_o,
-                                            kk > 0);
+                                            true);
                         tc::mma_commit(&sm.o_full[g]);
                         LSH_PHASE(0, 1, it, 4);
                         ++next_o;
@@ -439,7 +468,8 @@ attn_fwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
             const bool first = tcd.k == 0;
             float l, row_lse;
             // one run-time-parameterised copy of the row code for every warp (instruction cache)
-            softmax_row<CAUSAL>(st, tl, i, qpos, qinv, self_only, tau, q >= 2 ? 64 : 0, first && q < 2, l, row_lse);
+            softmax_row<CAUSAL>(st, tl, i, qpos, qinv, self_only, tau, q >= 2 ? 64 : 0, first && q < 2, &sm.p_half[g], l,
+                                row_lse);
             tc::tmem_st_wait();
             tc::tc_fence_before();
             __syncwarp();

@@ -179,7 +179,8 @@ def test_attention_given_perm(impl, dtype, causal, L, m, nh):
 @pytest.mark.parametrize("impl", IMPLS)
 @pytest.mark.parametrize("dtype,causal,nb,nh,L", [("f32", False, 16, 1, 1024), ("f32", True, 16, 2, 512),
                                                   ("bf16", True, 64, 2, 1024), ("bf16", False, 128, 3, 1152),
-                                                  ("bf16", True, 1024, 4, 2048), ("bf16", True, 2, 2, 256)])
+                                                  ("bf16", True, 1024, 4, 2048), ("bf16", True, 2, 2, 256),
+                                                  ("bf16", True, 256, 3, 1408)])
 def test_forward_backward_small(impl, dtype, causal, nb, nh, L):
     w = small("long_64k", B=2, H=2, L=L, n_buckets=nb, n_hashes=nh, causal=causal, dtype=dtype, backward=True)
     full_check(w, impl)
