@@ -83,6 +83,7 @@ struct BwdSmem {
     uint64_t gx_ready;              // the second half's partial sums of g . x are in gxh
     uint64_t epi_done;              // every compute warp finished the previous tile's epilogue
     float gxh[kK];
+    alignas(16) int ridx[kComputeWarps][2][32];   // row indices of the staged rows, per warp
     uint32_t tmem_base;
     int abort;
 };
@@ -96,42 +97,48 @@ __device__ __forceinline__ void red_add_v4(float *addr, float a, float b, float 
 
 // Adds each lane's 64-float row `a` to row `rowg` of `acc` (skipped when
 // rowg < 0) with coalesced vector reductions: the warp's 32 rows go through
-// its 8 KB staging buffer (16-byte chunks swizzled by lane against bank
-// conflicts), then each reduction instruction covers two whole rows.
-__device__ __forceinline__ void stage_rows(uint8_t *stg, int lane, const float *a)
+// its 8 KB staging buffer (16-byte chunks swizzled by row against bank
+// conflicts) and their row indices through `ridx` (32 ints), then each
+// reduction instruction covers two whole rows, r and r + 16.
+__device__ __forceinline__ void stage_rows(uint8_t *stg, int *ridx, int lane, const float *a, int rowg)
 {
 #pragma unroll
     for (int c = 0; c < 16; ++c)
         *reinterpret_cast<float4 *>(stg + lane * 256 + ((c ^ (lane & 15)) << 4)) =
             make_float4(a[4 * c], a[4 * c + 1], a[4 * c + 2], a[4 * c + 3]);
+    ridx[lane] = rowg;
     __syncwarp();
 }
 // `add` (nullable): 32 more rows in the same staged layout, added on the way.
-__device__ __forceinline__ void reduce_rows(const uint8_t *stg, int lane, float *acc, int rowg,
+__device__ __forceinline__ void reduce_rows(const uint8_t *stg, const int *ridx, int lane, float *acc,
                                             const uint8_t *add = nullptr)
 {
-    const int c = lane & 15;
-#pragma unroll 4
-    for (int it = 0; it < 16; ++it) {
-        const int rr = 2 * it + (lane >> 4);
-        const int rg = __shfl_sync(0xffffffffu, rowg, rr);
-        const uint32_t off = rr * 256 + ((c ^ (rr & 15)) << 4);
-        float4 val = *reinterpret_cast<const float4 *>(stg + off);
-        if (add) {
-            const float4 g = *reinterpret_cast<const float4 *>(add + off);
-            val.x += g.x; val.y += g.y; val.z += g.z; val.w += g.w;
+    const int c = lane & 15, r0 = (lane >> 4) * 16;
+#pragma unroll 1
+    for (int k = 0; k < 4; ++k) {
+        const int4 r4 = *reinterpret_cast<const int4 *>(ridx + r0 + 4 * k);
+        const int rows[4] = {r4.x, r4.y, r4.z, r4.w};
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int it = 4 * k + u;
+            const uint32_t off = (r0 + it) * 256 + ((c ^ it) << 4);
+            float4 val = *reinterpret_cast<const float4 *>(stg + off);
+            if (add) {
+                const float4 g = *reinterpret_cast<const float4 *>(add + off);
+                val.x += g.x; val.y += g.y; val.z += g.z; val.w += g.w;
+            }
+            if (rows[u] >= 0) red_add_v4(acc + (long long)rows[u] * kDim + 4 * c, val.x, val.y, val.z, val.w);
         }
-        if (rg >= 0) red_add_v4(acc + (long long)rg * kDim + 4 * c, val.x, val.y, val.z, val.w);
     }
     __syncwarp();
 }
-__device__ __forceinline__ void flush_rows(uint8_t *stg, int lane, const float *a, float *acc, int rowg,
+__device__ __forceinline__ void flush_rows(uint8_t *stg, int *ridx, int lane, const float *a, float *acc, int rowg,
                                            int ph_role = -1, int ph_it = 0, int ph_ev = 0,
                                            const uint8_t *add = nullptr)
 {
-    stage_rows(stg, lane, a);
+    stage_rows(stg, ridx, lane, a, rowg);
     if (ph_role >= 0 && lane == 0) LSH_PHASE(1, ph_role, ph_it, ph_ev);
-    reduce_rows(stg, lane, acc, rowg, add);
+    reduce_rows(stg, ridx, lane, acc, add);
     if (ph_role >= 0 && lane == 0) LSH_PHASE(1, ph_role, ph_it, ph_ev + 1);
 }
 
@@ -567,7 +574,7 @@ attn_bwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
                 }
                 // chunk 2k rows: plus the previous tile's part of their dQ, when handed over
                 const uint8_t *add = quad < 2 && carry_in ? sm.carry[(it - 1) & 1] + quad * 32 * 256 : nullptr;
-                flush_rows(stg, lane, a, dx_acc, krow, prole, it, 2, add);
+                flush_rows(stg, sm.ridx[warp][0], lane, a, dx_acc, krow, prole, it, 2, add);
                 if (prole >= 0 && lane == 0) LSH_PHASE(1, prole, it, 4);
             } else {
                 if (tid == 128) LSH_PHASE(1, 3, it, 0);
@@ -575,7 +582,7 @@ attn_bwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
 #pragma unroll
                     for (int c = 0; c < 4; ++c) tc::tmem_ld16(tl + cDV + c * 16, a + c * 16);
                     release_tmem();
-                    flush_rows(stg, lane, a, dv_acc, krow);
+                    flush_rows(stg, sm.ridx[warp][0], lane, a, dv_acc, krow);
                 } else {
                     // the dV row (staged first), then query row 64 + kr (chunk 2k+2): handed
                     // to the next tile when that is k+1 of this segment, else reduced here,
@@ -583,7 +590,7 @@ attn_bwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
 #pragma unroll
                     for (int c = 0; c < 4; ++c) tc::tmem_ld16(tl + cDV + c * 16, a + c * 16);
                     tc::tmem_ld_wait();
-                    stage_rows(stg, lane, a);
+                    stage_rows(stg, sm.ridx[warp][0], lane, a, krow);
 #pragma unroll
                     for (int c = 0; c < 4; ++c) tc::tmem_ld16(tl + cQb + c * 16, a + c * 16);
                     release_tmem();
@@ -597,14 +604,12 @@ attn_bwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
                             *reinterpret_cast<float4 *>(cb + ((c ^ (cr & 15)) << 4)) =
                                 make_float4(a[4 * c], a[4 * c + 1], a[4 * c + 2], a[4 * c + 3]);
                     } else {
-                        stage_rows(stg2, lane, a);
-                    }
-                    reduce_rows(stg, lane, dv_acc, krow);
-                    if (warp == 6 && lane == 0) LSH_PHASE(1, 6, it, 1);
-                    if (!tcd.next_adjacent) {
                         const int qp = st.qpos[64 + kr];
-                        reduce_rows(stg2, lane, dx_acc, qp >= 0 ? (int)rowbase + qp : -1);
+                        stage_rows(stg2, sm.ridx[warp][1], lane, a, qp >= 0 ? (int)rowbase + qp : -1);
                     }
+                    reduce_rows(stg, sm.ridx[warp][0], lane, dv_acc);
+                    if (warp == 6 && lane == 0) LSH_PHASE(1, 6, it, 1);
+                    if (!tcd.next_adjacent) reduce_rows(stg2, sm.ridx[warp][1], lane, dx_acc);
                     if (warp == 6 && lane == 0) LSH_PHASE(1, 6, it, 2);
                 }
                 if (tid == 128) LSH_PHASE(1, 3, it, 1);
