@@ -325,22 +325,43 @@ def cpu_baseline(w: synth.Workload) -> dict:
 
 
 def run_reference(args, w: synth.Workload) -> dict:
+    """The oracle as it stands, timed on the host cores.  Each step is a bounded
+    sample of the workload: min(cores, B*H) (batch, head) slices of
+    min(L, 4096) tokens with the workload's buckets, rounds, chunk and mask, one
+    slice per OpenMP thread (about a second of CPU work), so a --steps 200 run
+    ends in a few minutes (the oracle's cost is linear in L).  tokens/s counts
+    sequence tokens as the metric does (a (batch, head) slice of Ls tokens is
+    Ls / H of them); ms_per_step is the whole workload's step at that rate."""
+    from oracle import oracle
     cores = cpu_cores()
     n = max(1, min(cores, w.B * w.H))
-    for _ in range(args.warmup):                      # warm-up on a short slice
-        oracle_slices(w, 1, 1, L=max(w.chunk * 2, w.L // 64))
-    times = [oracle_slices(w, n, n) for _ in range(args.steps)]
-    step_s = float(np.mean(times)) * (w.B * w.H) / n
-    value = w.tokens / step_s
+    Ls = min(w.L, 4096)
+    ws = w.replace(B=1, H=n, L=Ls)
+    inp = synth.make_inputs(ws)
+    os.environ["OMP_NUM_THREADS"] = str(n)
+
+    def step() -> float:
+        t0 = time.perf_counter()
+        res = oracle.fwd(inp["x"], inp["v"], inp["R"], ws.n_buckets, ws.chunk, ws.causal)
+        if ws.backward:
+            oracle.bwd(inp["x"], inp["v"], inp["dy"], res["perm"], ws.chunk, ws.causal)
+        return time.perf_counter() - t0
+
+    for _ in range(args.warmup):
+        step()
+    times = [step() for _ in range(args.steps)]
+    # the metric counts sequence tokens (B * L per step, each with all H heads)
+    value = n * Ls / float(np.mean(times)) * w.tokens / (w.B * w.H * w.L)
+    sample = (f"{n} (batch, head) slices of {Ls} tokens per step (of {w.B * w.H} x {w.L} in {w.name}), "
+              f"fwd{'+bwd' if w.backward else ''}, one slice per OpenMP thread; {float(np.mean(times)):.2f} s per step")
     return {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": 1, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": step_s * 1e3, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "f64", "data": "synthetic: seeded Philox4x32-10 + Box-Muller normals",
+            "warmup": args.warmup, "ms_per_step": w.tokens / value * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic: seeded Philox4x32-10 + Box-Muller normals",
             "config": {"workload": describe(w), "global_batch": w.B, "seq_len": w.L,
                        "parallelism": "host cores (OpenMP over (batch, head) slices)"},
             "impl": "reference",
-            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": n, "kind": "oracle",
-                             "sample": f"{n} of {w.B * w.H} (batch, head) slices per step, full length; "
-                                       f"step time scaled by slice count"},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": n, "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
