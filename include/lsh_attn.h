@@ -100,6 +100,18 @@ typedef struct {
     int32_t impl;            /* lsh_impl                                       */
 } lsh_attn_desc;
 
+/* Random rotations on the HOST ("LSH Attention": one random rotation per
+ * round, entries N(0, 1)): fills R_host[n_hashes, d, n_buckets/2] (float32, or
+ * bfloat16 bits as uint16 when desc->dtype is LSH_BF16; caller-owned host
+ * memory of n_hashes * d * n_buckets/2 elements) from `seed` with
+ * Philox4x32-10 and the Box-Muller transform, rounded to float32 and then,
+ * for bf16, to bfloat16 (nearest, ties to even).  The same seed always gives
+ * the same rotations.  Only the descriptor's dtype, d, n_buckets and n_hashes
+ * are used.  Errors: LSH_ERR_ARG (null pointer, unknown dtype), LSH_ERR_SHAPE
+ * (n_buckets odd, < 2 or > 65536; d or n_hashes < 1).  Nothing runs on the
+ * device. */
+LSH_API lsh_status lsh_attn_make_rotations(uint64_t seed, const lsh_attn_desc *desc, void *R_host);
+
 /* Bytes of workspace needed by lsh_attn_fwd (for_backward = 0) or by
  * lsh_attn_bwd (for_backward = 1; includes what a recomputed hash and sort
  * need when perm is NULL).  Returns 0 for an invalid descriptor. */
@@ -179,6 +191,16 @@ LSH_API lsh_status lsh_attn_fwd(const lsh_attn_desc *desc, const void *qk, const
 LSH_API lsh_status lsh_attn_bwd(const lsh_attn_desc *desc, const void *qk, const void *v, const void *R,
                         const void *out, const float *lse, const int32_t *perm, const void *dout,
                         void *dqk, void *dv, void *workspace, size_t ws_bytes, void *stream);
+
+/* Parity bookkeeping: the number of (row, round) pairs of the last hash
+ * (lsh_attn_hash, or the hash inside lsh_attn_fwd / lsh_attn_bwd) whose two
+ * largest entries of [x R_r ; -x R_r] differ by less than 1e-6 of the
+ * largest magnitude, so that a rounding difference could change the bucket.
+ * Counted only in the tuning build (liblsh_attn_trace.so), where every hash
+ * also runs a CUDA-core pass that recomputes the projections in fp32;
+ * synchronises the device.  Returns -1 in the regular build, -2 on a CUDA
+ * error. */
+LSH_API int lsh_attn_last_near_ties(void);
 
 /* Device-side status of the calls made with this workspace since the last
  * poll: synchronises `stream`, returns LSH_ERR_TIMEOUT if a bounded wait in a

@@ -22,9 +22,9 @@ IMPL_AUTO, IMPL_SIMT, IMPL_TC = 0, 1, 2
 STATUS = {0: "LSH_OK", -1: "LSH_ERR_ARG", -2: "LSH_ERR_SHAPE", -3: "LSH_ERR_ALIGN",
           -4: "LSH_ERR_UNSUPPORTED", -5: "LSH_ERR_CUDA", -6: "LSH_ERR_TIMEOUT", -7: "LSH_ERR_WORKSPACE"}
 
-EXPORTED = ("lsh_attn_workspace_size", "lsh_attn_hash", "lsh_attn_sort", "lsh_attn_sort_static", "lsh_attn_fwd_sorted", "lsh_attn_fwd",
+EXPORTED = ("lsh_attn_make_rotations", "lsh_attn_workspace_size", "lsh_attn_hash", "lsh_attn_sort", "lsh_attn_sort_static", "lsh_attn_fwd_sorted", "lsh_attn_fwd",
             "lsh_attn_bwd", "lsh_attn_poll", "lsh_attn_selftest_timeout", "lsh_attn_trace_begin",
-            "lsh_attn_trace_end",
+            "lsh_attn_trace_end", "lsh_attn_last_near_ties",
             "lsh_attn_status_str", "lsh_attn_last_error", "lsh_attn_abi_version")
 
 STAGES = ("hash", "sort", "norms", "attn_fwd", "combine", "bwd_prep", "attn_bwd", "bwd_final")
@@ -55,6 +55,7 @@ def load_library(path: str = LIB_PATH):
     P = ctypes.c_void_p
     DP = ctypes.POINTER(Desc)
     S = ctypes.c_size_t
+    L.lsh_attn_make_rotations.argtypes = [ctypes.c_uint64, DP, P]
     L.lsh_attn_workspace_size.argtypes = [DP, ctypes.c_int]
     L.lsh_attn_workspace_size.restype = S
     L.lsh_attn_hash.argtypes = [DP, P, P, P, P, S, P]
@@ -68,6 +69,8 @@ def load_library(path: str = LIB_PATH):
     L.lsh_attn_trace_begin.argtypes = [ctypes.c_int32]
     L.lsh_attn_trace_end.argtypes = [ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_int32),
                                      ctypes.POINTER(ctypes.c_int32), ctypes.c_int32]
+    L.lsh_attn_last_near_ties.argtypes = []
+    L.lsh_attn_last_near_ties.restype = ctypes.c_int
     L.lsh_attn_status_str.argtypes = [ctypes.c_int]
     L.lsh_attn_status_str.restype = ctypes.c_char_p
     L.lsh_attn_last_error.argtypes = []
@@ -103,6 +106,17 @@ def _check(rc: int, where: str):
     if rc != 0:
         detail = load_library().lsh_attn_last_error().decode() if rc == -5 else ""
         raise LshAttnError(rc, where, detail)
+
+
+def make_rotations(desc: Desc, seed: int) -> torch.Tensor:
+    """Host tensor R [n_hashes, d, n_buckets/2] (float32 or bfloat16) drawn from
+    `seed` by the library's generator."""
+    shape = (desc.n_hashes, desc.d, desc.n_buckets // 2)
+    dt = torch.bfloat16 if desc.dtype == LSH_BF16 else torch.float32
+    R = torch.empty(shape, dtype=dt)
+    _check(load_library().lsh_attn_make_rotations(ctypes.c_uint64(seed), ctypes.byref(desc), _ptr(R)),
+           "lsh_attn_make_rotations")
+    return R
 
 
 def workspace_size(desc: Desc, for_backward: bool) -> int:

@@ -150,6 +150,7 @@ static lsh_status run_hash_sort(const Problem &p, const Choice &c, const void *q
                 return c.tc_hash ? launch_hash_tc(p, qk, R, w.buckets, w.rot, w.status, st)
                                  : launch_hash_simt(p, qk, R, w.buckets, st);
             }), "hash");
+    LSH_TRY(launch_near_ties(p, qk, R, st), "near-tie count");
     LSH_TRY(staged(LSH_STAGE_SORT, 3 * make_sort_plan(p.nb, p.L).passes, st,
                    [&] { return launch_sort(p, w.buckets, perm, w, st); }), "sort");
     return LSH_OK;
@@ -203,6 +204,7 @@ lsh_status lsh_attn_hash(const lsh_attn_desc *desc, const void *qk, const void *
                 return c.tc_hash ? launch_hash_tc(p, qk, R, buckets, w.rot, w.status, st)
                                  : launch_hash_simt(p, qk, R, buckets, st);
             }), "hash");
+    LSH_TRY(launch_near_ties(p, qk, R, st), "near-tie count");
     return LSH_OK;
 }
 
@@ -222,6 +224,12 @@ lsh_status lsh_attn_sort(const lsh_attn_desc *desc, const uint16_t *buckets, int
     LSH_TRY(staged(LSH_STAGE_SORT, 3 * make_sort_plan(p.nb, p.L).passes, st,
                    [&] { return launch_sort(p, buckets, perm, w, st); }), "sort");
     return LSH_OK;
+}
+
+int lsh_attn_last_near_ties(void)
+{
+    const long long v = read_near_ties();
+    return v > 0x7FFFFFFFLL ? 0x7FFFFFFF : (int)v;
 }
 
 lsh_status lsh_attn_sort_static(const lsh_attn_desc *desc, const uint16_t *buckets, int32_t *perm, void *stream)

@@ -126,6 +126,10 @@ __device__ __forceinline__ void store_row(__nv_bfloat16 *p, const float *r)
 // Every launcher enqueues on `st` and returns cudaGetLastError().
 cudaError_t launch_invnorm(const Problem &p, const void *x, float *invnorm, cudaStream_t st);
 cudaError_t launch_hash_simt(const Problem &p, const void *x, const void *R, uint16_t *buckets, cudaStream_t st);
+// Near-tie count of a hash (tuning build only; a no-op elsewhere) and its read-back
+// (-1 when not compiled in, -2 on a CUDA error).
+cudaError_t launch_near_ties(const Problem &p, const void *x, const void *R, cudaStream_t st);
+long long read_near_ties();
 cudaError_t launch_hash_tc(const Problem &p, const void *x, const void *R, uint16_t *buckets, void *scratch,
                            uint32_t *status, cudaStream_t st);
 bool hash_tc_supported(const Problem &p);

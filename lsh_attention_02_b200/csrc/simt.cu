@@ -80,6 +80,69 @@ cudaError_t launch_hash_simt(const Problem &p, const void *x, const void *R, uin
     return cudaGetLastError();
 }
 
+// ------------------------------------------------------------------ near ties
+// Parity bookkeeping (compiled into the tuning build only): the number of
+// (row, round) pairs whose two largest entries of [x R_r ; -x R_r] (fp32,
+// sequential fma over d) differ by less than 1e-6 of the largest magnitude,
+// i.e. whose bucket a rounding difference could flip.
+#ifdef LSH_PHASE_TRACE
+static __device__ unsigned long long g_near_ties;
+
+__global__ void near_tie_reset_kernel() { g_near_ties = 0ull; }
+
+template <typename T>
+__global__ void near_tie_kernel(const T *__restrict__ x, const T *__restrict__ R, long long BH, int L, int half)
+{
+    long long row = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    int r = blockIdx.y;
+    if (row >= BH * L) return;
+    float a[kDim];
+    load_row(x + row * kDim, a);
+    const T *Rr = R + (long long)r * kDim * half;
+    float t1 = -INFINITY, t2 = -INFINITY;                  // largest and second largest of [p ; -p]
+    for (int k = 0; k < half; ++k) {
+        float s = 0.f;
+#pragma unroll 16
+        for (int t = 0; t < kDim; ++t) s = fmaf(a[t], to_f(Rr[(long long)t * half + k]), s);
+        const float hi = fmaxf(s, -s), lo = fminf(s, -s);
+        if (hi > t1) { t2 = fmaxf(t1, lo); t1 = hi; }
+        else { t2 = fmaxf(t2, hi); }
+    }
+    const float margin = (t1 - t2) / fmaxf(fabsf(t1), 1e-30f);
+    if (margin < 1e-6f) atomicAdd(&g_near_ties, 1ull);
+}
+#endif
+
+cudaError_t launch_near_ties(const Problem &p, const void *x, const void *R, cudaStream_t st)
+{
+#ifdef LSH_PHASE_TRACE
+    near_tie_reset_kernel<<<1, 1, 0, st>>>();
+    long long rows = p.tokens();
+    dim3 grid((unsigned)((rows + 127) / 128), p.R);
+    if (p.dtype == LSH_F32)
+        near_tie_kernel<float><<<grid, 128, 0, st>>>((const float *)x, (const float *)R, p.BH(), p.L, p.nb / 2);
+    else
+        near_tie_kernel<__nv_bfloat16><<<grid, 128, 0, st>>>((const __nv_bfloat16 *)x, (const __nv_bfloat16 *)R,
+                                                              p.BH(), p.L, p.nb / 2);
+    return cudaGetLastError();
+#else
+    (void)p; (void)x; (void)R; (void)st;
+    return cudaSuccess;
+#endif
+}
+
+long long read_near_ties()
+{
+#ifdef LSH_PHASE_TRACE
+    unsigned long long v = 0;
+    if (cudaDeviceSynchronize() != cudaSuccess) return -2;
+    if (cudaMemcpyFromSymbol(&v, g_near_ties, sizeof(v)) != cudaSuccess) return -2;
+    return (long long)v;
+#else
+    return -1;
+#endif
+}
+
 // ------------------------------------------------------------------ candidates
 // Window of sorted slot s: chunks c-1 and c ("Sorting and Chunking").  A slot
 // t != s is a candidate unless causal and its position exceeds the query's

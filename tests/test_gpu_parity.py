@@ -285,3 +285,52 @@ def test_bounded_wait_reports_timeout():
     w = small("long_64k", B=1, H=1, L=256, backward=False)
     run = Run(synth.make_inputs(w), w.n_buckets, w.chunk, w.causal, w.dtype)
     assert torch.isfinite(run.out.float()).all()
+
+
+# ------------------------------------------------------------------ near-tie bookkeeping
+_NEAR_TIE_SCRIPT = r"""
+import json, sys
+import numpy as np, torch
+sys.path.insert(0, {root!r})
+import lsh_attention_02_b200 as lsh
+from lsh_attention_02_b200 import build, synth
+import os
+trace = build.LIB.replace(".so", "_trace.so")
+lsh.load_library(trace if os.path.exists(trace) else build.build(phase_trace=True))
+w = synth.WORKLOADS["bf16_causal_4k"].replace(B=1, H=2, L=1024, n_buckets=64, n_hashes=2)
+inp = synth.make_inputs(w)
+inp["x"][0, 0, :5] = 0.0
+inp["x"][0, 1, 100:105] = 0.0
+x = torch.from_numpy(inp["x"]).cuda().to(torch.bfloat16)
+R = torch.from_numpy(inp["R"]).cuda().to(torch.bfloat16)
+desc = lsh.desc_for(x, w.n_buckets, w.n_hashes, w.chunk, w.causal)
+bk = torch.empty((1, 2, 2, w.L), dtype=torch.int16, device="cuda")
+lsh.lsh_attn_hash(desc, x, R, bk)
+print(json.dumps({{"count": lsh.load_library().lsh_attn_last_near_ties()}}))
+"""
+
+
+def test_near_tie_count_in_tuning_build():
+    """The tuning build counts (row, round) pairs whose top-two gap is below
+    1e-6: every zero row is an exact tie in each round; the other rows count
+    only if the oracle also sees them within a small relative gap."""
+    import json
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    r = subprocess.run([sys.executable, "-c", _NEAR_TIE_SCRIPT.format(root=root)], capture_output=True, text=True,
+                       timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    count = json.loads(r.stdout.strip().splitlines()[-1])["count"]
+    w = synth.WORKLOADS["bf16_causal_4k"].replace(B=1, H=2, L=1024, n_buckets=64, n_hashes=2)
+    inp = synth.make_inputs(w)
+    inp["x"][0, 0, :5] = 0.0
+    inp["x"][0, 1, 100:105] = 0.0
+    close = 0
+    for h in range(2):
+        for rr in range(2):
+            _, mg = oracle.hash_round(inp["x"][0, h], inp["R"][rr], w.n_buckets)
+            close += int((mg < 1e-4).sum())
+    assert 20 <= count <= close, (count, close)
+    assert lsh.load_library().lsh_attn_last_near_ties() == -1     # the regular build does not count
