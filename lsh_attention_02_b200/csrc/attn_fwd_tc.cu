@@ -521,9 +521,9 @@ cudaError_t launch_attn_fwd_tc(const Problem &p, const void *x, const void *v, c
     auto kern = p.causal ? attn_fwd_tc_kernel<true> : attn_fwd_tc_kernel<false>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    int dev = 0, sms = 148;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    int dev = 0, sms = 0;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
     const long long n_tiles = p.S() * (p.L / kQ);
     const unsigned grid = (unsigned)std::min<long long>(n_tiles, (long long)sms);
     kern<<<grid, kThreads, smem, st>>>((const __nv_bfloat16 *)x, (const __nv_bfloat16 *)v, perm, o_r, lse, p.L, p.R, n_tiles,
