@@ -77,7 +77,7 @@ typedef enum {
     LSH_ERR_ARG = -1,          /* null pointer or unknown enum value            */
     LSH_ERR_SHAPE = -2,        /* sizes inconsistent (e.g. L % chunk != 0)      */
     LSH_ERR_ALIGN = -3,        /* a pointer is not 16-byte aligned              */
-    LSH_ERR_UNSUPPORTED = -4,  /* valid request this build does not run (d!=64, */
+    LSH_ERR_UNSUPPORTED = -4,  /* valid request the library does not run (d!=64,  */
                                /* or a forced implementation that cannot run it) */
     LSH_ERR_CUDA = -5,         /* a CUDA launch or runtime call failed          */
     LSH_ERR_TIMEOUT = -6,      /* a bounded device-side wait gave up            */
