@@ -5,6 +5,8 @@ d=64, bf16 e=2, R=4, m=64):
   backward per (b, h): L [4 d e + 8 + R (4 d e + 16 + 4 d 4)] = 65536 * 6728
   attention FLOPs per token, head, round: 4 (2m) d = 32768 forward,
   5 * 2 (2m) d = 81920 backward; hash: d * n_buckets = 65536."""
+import pytest
+
 import bench
 from lsh_attention_02_b200 import synth
 
@@ -29,3 +31,15 @@ def test_whole_job_rate_counts_every_rank():
     w = synth.WORKLOADS["long_64k"]
     assert bench.whole_job_tokens_per_s(w, 1, 1.0) == 65536 * 1000.0
     assert bench.whole_job_tokens_per_s(w, 4, 2.0) == 4 * 65536 * 500.0
+
+
+def test_step_roofline_bytes_bound_and_hash_inclusive():
+    a = bench.algorithmic(synth.WORKLOADS["long_64k"])
+    r = bench.step_roofline(a, 6443.2, 1410.0, 1.65)
+    assert r["roofline_ms"] == pytest.approx(4_785_700_864 / 6443.2e9 * 1e3)      # bytes bound: 0.743 ms
+    assert r["roofline_ms_with_hash"] == r["roofline_ms"]                        # 377 GFLOP take 0.27 ms
+    assert r["frac"] == pytest.approx(r["roofline_ms"] / 1.65)
+    h = bench.algorithmic(synth.WORKLOADS["half_million"])                      # nb = 8192: the hash GEMM decides
+    rh = bench.step_roofline(h, 6443.2, 1410.0, 2.68)
+    assert rh["roofline_ms_with_hash"] == pytest.approx((h["attn_flops"] + h["hash_flops"]) / 1410e12 * 1e3)
+    assert rh["roofline_ms_with_hash"] > 3 * rh["roofline_ms"]
