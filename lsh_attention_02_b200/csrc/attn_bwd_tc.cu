@@ -34,10 +34,10 @@
 // Warp roles (persistent CTA, one per SM):
 //   warps 0-7  compute: warp w owns TMEM lanes 32*(w%4).. (key rows) and query
 //              columns half (w/4); elementwise step, then the epilogue;
-//   warps 8-10 producer: positions, per-query LSE / delta / self flags and
-//              per-key norms into a 2-stage ring, then 16-byte cp.async
-//              gathers of the x, v and dY rows straight into the swizzled
-//              operand layout;
+//   warps 8-10 producer: positions, per-query LSE, delta and causal key
+//              bounds into a 2-stage ring, and 16-byte cp.async gathers of
+//              the x, v and dY rows straight into the swizzled operand
+//              layout (key norms are computed by the compute warps);
 //   warp 11    MMA issuer.
 #include "tc_common.cuh"
 
