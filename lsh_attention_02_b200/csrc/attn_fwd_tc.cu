@@ -360,6 +360,8 @@ attn_fwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
             tc::cp_async_wait<0>();
             tc::fence_async_smem();
             tc::mbar_arrive(&sm.full[prev_s]);
+        } else {
+            tc::cp_async_wait<0>();         // given up: let this thread's copies land before the CTA ends
         }
     } else if (warp == kMmaWarp) {
         // ================= MMA issuer

@@ -114,7 +114,7 @@ hash_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __nv_bfloat16 *__
                 return true;
             };
             bool ok = blockIdx.x >= n_blocks || load_a(blockIdx.x, 0);
-            int it = 0, bi = 0;
+            int it = 0, bi = 0, r_issued = 0, a_issued = blockIdx.x < n_blocks ? 1 : 0;
             for (long long blk = blockIdx.x; ok && blk < n_blocks; blk += gridDim.x, ++bi) {
                 const int prefetch_at = min(kStages, items) - 1;
                 for (int i = 0; i < items; ++i, ++it) {
@@ -127,12 +127,23 @@ hash_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __nv_bfloat16 *__
                     const __nv_bfloat16 *src = Rs + ((long long)r * half + (long long)nt * NT) * kDim;
                     tc::mbar_arrive_expect_tx(&sm.full[s], NT * 128);
                     tc::bulk_g2s(sm.B[s], src, NT * 128, &sm.full[s]);
+                    ++r_issued;
                     // the next block's rows, once this block's MMAs have started
-                    if (i == prefetch_at && blk + gridDim.x < n_blocks && !load_a(blk + gridDim.x, bi + 1)) {
-                        ok = false;
-                        break;
+                    if (i == prefetch_at && blk + gridDim.x < n_blocks) {
+                        if (!load_a(blk + gridDim.x, bi + 1)) { ok = false; break; }
+                        ++a_issued;
                     }
                 }
+            }
+            if (!ok) {
+                // given up: before the CTA ends, let the copies this thread started land
+                // (bounded waits on the barriers that count their bytes)
+                int stop = 0;
+                const long long budget = 1000000;
+                for (int j = r_issued > kStages ? r_issued - kStages : 0; j < r_issued; ++j)
+                    tc::mbar_wait(&sm.full[j % kStages], (uint32_t)(j / kStages) & 1u, &stop, status, budget);
+                for (int b = a_issued > 2 ? a_issued - 2 : 0; b < a_issued; ++b)
+                    tc::mbar_wait(&sm.a_full[b & 1], (uint32_t)(b >> 1) & 1u, &stop, status, budget);
             }
         }
     } else if (warp == kEpiWarps + 1) {
