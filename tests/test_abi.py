@@ -105,3 +105,22 @@ def test_trace_end_without_begin_is_an_error(lib):
     ms = (ctypes.c_float * n)(); c = (ctypes.c_int32 * n)(); k = (ctypes.c_int32 * n)()
     assert lib.lsh_attn_trace_end(ms, c, k, n) == -1
     assert lib.lsh_attn_trace_begin(0) == -1
+
+
+def test_near_tie_count_not_compiled_in_regular_build(lib):
+    lib.lsh_attn_last_near_ties.restype = ctypes.c_int
+    assert lib.lsh_attn_last_near_ties() == -1
+
+
+def test_static_sort_rejects_oversize_before_any_device_call(lib):
+    """Two-pass sort (65536 buckets) of 32 segments x 131072 positions needs
+    24 MiB of scratch, over the 16 MiB limit: refused on the host, with the
+    sizes in the error text; the (never dereferenced) pointers are fakes."""
+    import lsh_attention_02_b200 as lsh
+    desc = lsh.make_desc(1, 32, 131072, 64, 65536, 1, 64, False, lsh.LSH_BF16)
+    fake = ctypes.c_void_p(0x1000)
+    lib.lsh_attn_sort_static.argtypes = [ctypes.POINTER(lsh.Desc), ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]
+    assert lib.lsh_attn_sort_static(ctypes.byref(desc), fake, fake, None) == -7
+    lib.lsh_attn_last_error.restype = ctypes.c_char_p
+    msg = lib.lsh_attn_last_error().decode()
+    assert "lsh_attn_sort_static" in msg and str(16 << 20) in msg
