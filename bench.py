@@ -32,6 +32,13 @@ METRIC = "LSH-attn fwd+bwd tokens/s at L=64K, 4 hashes; % of HBM/tensor roofline
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
+def bench_config(w: synth.Workload, world: int) -> dict:
+    """The `config` object of both arms' JSON lines (identical for the same run shape)."""
+    return {"workload": describe(w), "global_batch": w.B * world, "seq_len": w.L,
+            "parallelism": f"{world} independent replica(s), no collective",
+            "l2": "flushed between timed steps (256 MiB memset outside the step events)"}
+
+
 def describe(w: synth.Workload) -> str:
     mode = "fwd+bwd" if w.backward else "fwd"
     extra = f" clustered{w.clustered}(sigma={w.sigma})" if w.clustered else ""
@@ -63,7 +70,10 @@ def algorithmic(w: synth.Workload) -> dict:
         "attn_bwd": tok * (3 * d * e + 12 + R * 4) + tok * 2 * d * 4 * 2,  # x, v, dY, LSE, delta, norms, perm;
                                                                           # fp32 dx, dv accumulators in and out
     }
-    return {"bytes": bh * (fwd + bwd), "attn_flops": attn_flops, "hash_flops": hash_flops, "kernel_bytes": kern}
+    flops = {"hash": hash_flops, "attn_fwd": bh * L * R * 4 * 2 * m * d,
+             "attn_bwd": bh * L * R * 10 * 2 * m * d if w.backward else 0, "combine": 0}
+    return {"bytes": bh * (fwd + bwd), "attn_flops": attn_flops, "hash_flops": hash_flops, "kernel_bytes": kern,
+            "kernel_flops": flops}
 
 
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one launch, from
@@ -217,6 +227,7 @@ def run_ours(args, w: synth.Workload, rank: int, world: int) -> dict | None:
     ws_b = lsh.workspace(desc, True, dev) if w.backward else None
     dx = torch.empty_like(x); dv = torch.empty_like(v)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)   # > 126 MB L2
+    torch.cuda.reset_peak_memory_stats(dev)
 
     def step():
         lsh.lsh_attn_fwd(desc, x, v, R, out, lse, perm, ws_f)
@@ -248,6 +259,10 @@ def run_ours(args, w: synth.Workload, rank: int, world: int) -> dict | None:
         dist.barrier()
     torch.cuda.synchronize()
     step_ms = float(sum(s.elapsed_time(e) for s, e in zip(starts, ends))) / args.steps
+    # device memory of the step: inputs, outputs, permutation, workspaces (the L2
+    # flush buffer is not part of it)
+    peak_bytes = int(torch.cuda.max_memory_allocated(dev)) - flush.numel()
+    ws_bytes = {"fwd": int(ws_f.numel()), "bwd": int(ws_b.numel()) if ws_b is not None else 0}
     if lsh.lsh_attn_poll(ws_f) != 0 or (ws_b is not None and lsh.lsh_attn_poll(ws_b) != 0):
         raise RuntimeError("device-side timeout during the timed steps")
 
@@ -299,8 +314,16 @@ def run_ours(args, w: synth.Workload, rank: int, world: int) -> dict | None:
                         key=lambda kv: kv[1]["ms_per_step"])
     dom_launch_ms = dom["ms_per_step"] / max(dom["calls"], 1)
     dom_bytes = alg["kernel_bytes"][dom_name] / max(dom["calls"], 1)
-    achieved = dom_bytes / (dom_launch_ms / 1e3) / 1e9
+    dom_flops = alg["kernel_flops"].get(dom_name, 0.0) / max(dom["calls"], 1)
     hbm = float(peaks["hbm_gbs"])
+    tensor = float(peaks["bf16_tflops_sustained"])
+    # the bound is whichever of bytes at the HBM peak and FLOPs at the bf16 peak
+    # takes longer for this kernel
+    t_hbm, t_tc = dom_bytes / (hbm * 1e9), dom_flops / (tensor * 1e12)
+    if t_tc > t_hbm:
+        bound, achieved, peak, unit = "tensor", dom_flops / (dom_launch_ms / 1e3) / 1e12, tensor, "TFLOP/s"
+    else:
+        bound, achieved, peak, unit = "hbm", dom_bytes / (dom_launch_ms / 1e3) / 1e9, hbm, "GB/s"
     step_bytes_gbs = alg["bytes"] / (step_ms / 1e3) / 1e9
     roof = step_roofline(alg, hbm, float(peaks["bf16_tflops_sustained"]), step_ms)
     res = {
@@ -308,18 +331,22 @@ def run_ours(args, w: synth.Workload, rank: int, world: int) -> dict | None:
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
         "data": f"synthetic: seeded Philox4x32-10 + Box-Muller normals, rounded to {w.dtype}",
-        "config": {"workload": describe(w), "global_batch": w.B * world, "seq_len": w.L,
-                   "parallelism": f"{world} independent replica(s), no collective",
-                   "l2": "flushed between timed steps (256 MiB memset outside the step events)"},
-        "roofline": {"bound": "hbm", "kernel": dom_name, "achieved": achieved, "peak": hbm, "unit": "GB/s",
-                     "frac": achieved / hbm, "peak_source": f"{peak_src} hbm_gbs",
+        "config": bench_config(w, world),
+        "roofline": {"bound": bound, "kernel": dom_name, "achieved": achieved, "peak": peak, "unit": unit,
+                     "frac": achieved / peak,
+                     "peak_source": f"{peak_src} {'hbm_gbs' if bound == 'hbm' else 'bf16_tflops_sustained'}",
                      "traffic": ncu_traffic(w.name, dom_name),
-                     "bytes_per_launch": dom_bytes, "launch_ms": dom_launch_ms},
+                     "bytes_per_launch": dom_bytes, "flops_per_launch": dom_flops, "launch_ms": dom_launch_ms,
+                     "hbm_frac": dom_bytes / (dom_launch_ms / 1e3) / 1e9 / hbm,
+                     "tensor_frac": dom_flops / (dom_launch_ms / 1e3) / 1e12 / tensor},
         "roofline_step": {"algorithmic_bytes": alg["bytes"], "achieved_gbs": step_bytes_gbs,
                           "attn_flops": alg["attn_flops"], "hash_flops": alg["hash_flops"], **roof,
                           "peak_source": peak_src},
         "stages": per_stage,
         "gpu_launches": int(launches),
+        "memory": {"peak_device_bytes": peak_bytes, "workspace_bytes": ws_bytes,
+                   "counts": "inputs, outputs, permutation and workspaces (torch allocator peak, "
+                             "L2 flush buffer excluded)"},
         "e2e": e2e,
     }
     res["clocks"] = clk.summary()
@@ -359,14 +386,14 @@ def cpu_baseline(w: synth.Workload) -> dict:
                       f"scaled by slice count"}
 
 
-def run_reference(args, w: synth.Workload) -> dict:
+def run_reference(args, w: synth.Workload, world: int = 1) -> dict:
     """The oracle as it stands, timed on the host cores.  Each step is a bounded
     sample of the workload: min(cores, B*H) (batch, head) slices of
     min(L, 4096) tokens with the workload's buckets, rounds, chunk and mask, one
     slice per OpenMP thread (about a second of CPU work), so a --steps 200 run
-    ends in a few minutes (the oracle's cost is linear in L).  tokens/s counts
-    sequence tokens as the metric does (a (batch, head) slice of Ls tokens is
-    Ls / H of them); ms_per_step is the whole workload's step at that rate."""
+    ends in a few minutes (the oracle's cost is linear in L).  ms_per_step is
+    the measured time of one such sampled step; tokens/s counts sequence tokens
+    as the metric does (a (batch, head) slice of Ls tokens is Ls / H of them)."""
     from oracle import oracle
     cores = cpu_cores()
     n = max(1, min(cores, w.B * w.H))
@@ -385,17 +412,18 @@ def run_reference(args, w: synth.Workload) -> dict:
     for _ in range(args.warmup):
         step()
     times = [step() for _ in range(args.steps)]
-    # the metric counts sequence tokens (B * L per step, each with all H heads)
-    value = n * Ls / float(np.mean(times)) * w.tokens / (w.B * w.H * w.L)
-    sample = (f"{n} (batch, head) slices of {Ls} tokens per step (of {w.B * w.H} x {w.L} in {w.name}), "
-              f"fwd{'+bwd' if w.backward else ''}, one slice per OpenMP thread; {float(np.mean(times)):.2f} s per step")
-    return {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": 1, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": w.tokens / value * 1e3, "higher_is_better": True,
+    step_s = float(np.mean(times))
+    seq_tokens = n * Ls / w.H                  # sequence tokens covered by one sampled step
+    value = seq_tokens / step_s
+    sample = (f"each step: {n} (batch, head) slices of {Ls} tokens (of {w.B * w.H} x {w.L} in {w.name}), "
+              f"fwd{'+bwd' if w.backward else ''}, one slice per OpenMP thread = {seq_tokens:g} sequence tokens "
+              f"in {step_s:.3f} s; ms_per_step is that sampled step")
+    return {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": step_s * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic: seeded Philox4x32-10 + Box-Muller normals",
-            "config": {"workload": describe(w), "global_batch": w.B, "seq_len": w.L,
-                       "parallelism": "host cores (OpenMP over (batch, head) slices)"},
-            "impl": "reference",
+            "config": bench_config(w, world),
+            "impl": "reference", "sampled": True,
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": n, "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
@@ -417,7 +445,7 @@ def main():
     w = synth.WORKLOADS[args.workload]
     if args.impl == "reference":
         if rank == 0:
-            print(json.dumps(run_reference(args, w)), flush=True)
+            print(json.dumps(run_reference(args, w, world)), flush=True)
         return
     res = run_ours(args, w, rank, world)
     if res is None:

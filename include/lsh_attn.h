@@ -51,8 +51,13 @@
  *     asynchronous on that stream; arguments are checked on the host before
  *     anything is launched, so an error status means nothing was launched,
  *     except LSH_ERR_CUDA, which reports a launch failure.
- *   - d must be 64.  fp32 inputs run on CUDA cores in fp32 (no TF32);
- *     bf16 inputs run on the tensor cores with fp32 accumulation.
+ *   - Which kernels run is fixed by the dtype, never chosen at run time:
+ *     fp32 inputs run on CUDA cores in fp32 (no TF32), any chunk with
+ *     L % chunk == 0; bf16 inputs run on the tensor cores (bf16 operands,
+ *     fp32 accumulation) and require chunk == 64 and L % 64 == 0.  A bf16
+ *     descriptor outside that envelope is refused with LSH_ERR_UNSUPPORTED
+ *     before anything is launched; there is no slower substitute path.
+ *     d must be 64 for both.
  */
 #ifndef LSH_ATTN_H
 #define LSH_ATTN_H
@@ -64,7 +69,7 @@
 extern "C" {
 #endif
 
-#define LSH_ATTN_ABI_VERSION 1
+#define LSH_ATTN_ABI_VERSION 2
 
 #if defined(__GNUC__)
 #define LSH_API __attribute__((visibility("default")))
@@ -77,8 +82,8 @@ typedef enum {
     LSH_ERR_ARG = -1,          /* null pointer or unknown enum value            */
     LSH_ERR_SHAPE = -2,        /* sizes inconsistent (e.g. L % chunk != 0)      */
     LSH_ERR_ALIGN = -3,        /* a pointer is not 16-byte aligned              */
-    LSH_ERR_UNSUPPORTED = -4,  /* valid request the library does not run (d!=64,  */
-                               /* or a forced implementation that cannot run it) */
+    LSH_ERR_UNSUPPORTED = -4,  /* valid request outside what the kernels run     */
+                               /* (d != 64; bf16 with chunk != 64 or L % 64 != 0) */
     LSH_ERR_CUDA = -5,         /* a CUDA launch or runtime call failed          */
     LSH_ERR_TIMEOUT = -6,      /* a bounded device-side wait gave up            */
     LSH_ERR_WORKSPACE = -7     /* workspace smaller than required               */
@@ -86,9 +91,20 @@ typedef enum {
 
 typedef enum { LSH_F32 = 0, LSH_BF16 = 1 } lsh_dtype;
 
-/* Which kernels run the attention and hash stages.  AUTO picks the tensor-core
- * kernels for bf16 with chunk == 64 and L % 128 == 0, else the CUDA-core ones. */
-typedef enum { LSH_IMPL_AUTO = 0, LSH_IMPL_SIMT = 1, LSH_IMPL_TC = 2 } lsh_impl;
+/* Optional semantics (lsh_attn_desc.flags, bitwise OR; 0 = the defaults above).
+ *   LSH_FLAG_BUCKET_MASK   strict candidate set of section "LSH Attention",
+ *                          N_LSH(i) = {j : h(q_i) = h(k_j)}: inside the chunk
+ *                          window a key is a candidate only if it shares the
+ *                          query's bucket in that round.
+ *   LSH_FLAG_SELF_PENALTY  the other answer to the same-token question of
+ *                          "Implementation Reading": the query's own position is
+ *                          always a candidate, with the fixed score
+ *                          LSH_SELF_PENALTY_SCORE in place of q_i . k_i / sqrt(d),
+ *                          so it carries weight only when nothing else is left.
+ * Unknown bits are rejected with LSH_ERR_ARG. */
+#define LSH_FLAG_BUCKET_MASK 1
+#define LSH_FLAG_SELF_PENALTY 2
+#define LSH_SELF_PENALTY_SCORE (-1.0e5f)
 
 typedef struct {
     int32_t B, H, L, d;      /* batch, heads, sequence length, head dim (64)   */
@@ -97,7 +113,7 @@ typedef struct {
     int32_t chunk;           /* chunk length m >= 1, L % m == 0                */
     int32_t causal;          /* 0 or 1                                         */
     int32_t dtype;           /* lsh_dtype                                      */
-    int32_t impl;            /* lsh_impl                                       */
+    int32_t flags;           /* LSH_FLAG_* bits, 0 for the default semantics   */
 } lsh_attn_desc;
 
 /* Random rotations on the HOST ("LSH Attention": one random rotation per
@@ -146,10 +162,11 @@ LSH_API lsh_status lsh_attn_sort(const lsh_attn_desc *desc, const uint16_t *buck
  * another component but no way to obtain a workspace.  The call makes no
  * cudaMalloc/cudaFree and calls no library that allocates.
  *
- * Set-up: the first call on each device looks up the array's device address
- * (cudaGetSymbolAddress), which may make the CUDA runtime load the library's
- * device code; later calls on that device reuse the cached address.  Make the
- * first call on each device before any stream capture begins.
+ * Set-up: every call looks up the array's device address on the current
+ * device (cudaGetSymbolAddress); nothing is cached, so a device reset or a
+ * different current context leaves no stale address behind.  The first call
+ * on a device may make the CUDA runtime load the library's device code, so
+ * make it before any stream capture begins.
  *
  * Sizes: the scratch needed grows with B*H*n_hashes*L (6 bytes per position
  * when n_buckets > 256, plus a few counters per 2048 positions).  A
@@ -174,7 +191,9 @@ LSH_API lsh_status lsh_attn_sort_static(const lsh_attn_desc *desc, const uint16_
  * equation, "Multiple Hash Rounds"): gathers rows in sorted order, runs the
  * chunked attention of every round, merges the rounds into out, and writes
  * the per-round logsumexp lse in original order.  perm must hold, for every
- * segment, a permutation of 0..L-1 (not checked on the device). */
+ * segment, a permutation of 0..L-1.  Entries outside [0, L) are ignored
+ * and reported by lsh_attn_poll (LSH_ERR_ARG); a repeated entry is not
+ * detected and gives undefined values at the positions involved. */
 LSH_API lsh_status lsh_attn_fwd_sorted(const lsh_attn_desc *desc, const void *qk, const void *v,
                                const int32_t *perm, void *out, float *lse,
                                void *workspace, size_t ws_bytes, void *stream);
@@ -204,7 +223,10 @@ LSH_API int lsh_attn_last_near_ties(void);
 
 /* Device-side status of the calls made with this workspace since the last
  * poll: synchronises `stream`, returns LSH_ERR_TIMEOUT if a bounded wait in a
- * kernel gave up, and clears the word.  Call it after a call, not during. */
+ * kernel gave up, else LSH_ERR_ARG if a kernel read a permutation entry
+ * outside [0, L) (such an entry is treated as an empty slot: nothing is read
+ * or written at it, and positions it should have covered get no output), and
+ * clears the word.  Call it after a call, not during. */
 LSH_API lsh_status lsh_attn_poll(void *workspace, void *stream);
 
 /* Stage timing.  lsh_attn_trace_begin(capacity) creates `capacity` pairs of

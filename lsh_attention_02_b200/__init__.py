@@ -17,7 +17,8 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "liblsh_attn.so")
 
 LSH_F32, LSH_BF16 = 0, 1
-IMPL_AUTO, IMPL_SIMT, IMPL_TC = 0, 1, 2
+FLAG_BUCKET_MASK, FLAG_SELF_PENALTY = 1, 2      # lsh_attn_desc.flags bits
+SELF_PENALTY_SCORE = -1.0e5
 
 STATUS = {0: "LSH_OK", -1: "LSH_ERR_ARG", -2: "LSH_ERR_SHAPE", -3: "LSH_ERR_ALIGN",
           -4: "LSH_ERR_UNSUPPORTED", -5: "LSH_ERR_CUDA", -6: "LSH_ERR_TIMEOUT", -7: "LSH_ERR_WORKSPACE"}
@@ -38,7 +39,7 @@ class LshAttnError(RuntimeError):
 
 class Desc(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in
-                ("B", "H", "L", "d", "n_buckets", "n_hashes", "chunk", "causal", "dtype", "impl")]
+                ("B", "H", "L", "d", "n_buckets", "n_hashes", "chunk", "causal", "dtype", "flags")]
 
 
 _lib = None
@@ -83,15 +84,15 @@ def load_library(path: str = LIB_PATH):
     return L
 
 
-def make_desc(B, H, L, d, n_buckets, n_hashes, chunk, causal, dtype, impl=IMPL_AUTO) -> Desc:
+def make_desc(B, H, L, d, n_buckets, n_hashes, chunk, causal, dtype, flags=0) -> Desc:
     if isinstance(dtype, torch.dtype):
         dtype = {torch.float32: LSH_F32, torch.bfloat16: LSH_BF16}[dtype]
-    return Desc(B, H, L, d, n_buckets, n_hashes, chunk, int(bool(causal)), dtype, impl)
+    return Desc(B, H, L, d, n_buckets, n_hashes, chunk, int(bool(causal)), dtype, flags)
 
 
-def desc_for(x: torch.Tensor, n_buckets: int, n_hashes: int, chunk: int, causal: bool, impl: int = IMPL_AUTO):
+def desc_for(x: torch.Tensor, n_buckets: int, n_hashes: int, chunk: int, causal: bool, flags: int = 0):
     B, H, L, d = x.shape
-    return make_desc(B, H, L, d, n_buckets, n_hashes, chunk, causal, x.dtype, impl)
+    return make_desc(B, H, L, d, n_buckets, n_hashes, chunk, causal, x.dtype, flags)
 
 
 def _ptr(t):
@@ -216,12 +217,12 @@ def outputs_like(desc: Desc, qk: torch.Tensor):
 
 
 class LSHAttention(torch.autograd.Function):
-    """y = LSHAttention.apply(qk, v, R, n_buckets, chunk, causal[, impl]); gradients for qk and v."""
+    """y = LSHAttention.apply(qk, v, R, n_buckets, chunk, causal[, flags]); gradients for qk and v."""
 
     @staticmethod
-    def forward(ctx, qk, v, R, n_buckets, chunk, causal, impl=IMPL_AUTO):
+    def forward(ctx, qk, v, R, n_buckets, chunk, causal, flags=0):
         qk = qk.contiguous(); v = v.contiguous(); R = R.contiguous()
-        desc = desc_for(qk, n_buckets, R.shape[0], chunk, causal, impl)
+        desc = desc_for(qk, n_buckets, R.shape[0], chunk, causal, flags)
         out, lse, perm = outputs_like(desc, qk)
         lsh_attn_fwd(desc, qk, v, R, out, lse, perm)
         ctx.desc = desc
@@ -237,9 +238,10 @@ class LSHAttention(torch.autograd.Function):
         return dqk, dv, None, None, None, None, None
 
 
-def lsh_attention(qk, v, R, n_buckets, chunk=64, causal=False, impl=IMPL_AUTO):
+def lsh_attention(qk, v, R, n_buckets, chunk=64, causal=False, flags=0):
     """Reformer LSH self-attention with shared query-key: returns (out, lse).
 
-    qk, v: [B, H, L, 64] CUDA tensors (float32 or bfloat16); R: [n_hashes, 64, n_buckets/2]."""
-    return LSHAttention.apply(qk, v, R, n_buckets, chunk, causal, impl)
+    qk, v: [B, H, L, 64] CUDA tensors (float32 or bfloat16); R: [n_hashes, 64, n_buckets/2];
+    flags: FLAG_BUCKET_MASK | FLAG_SELF_PENALTY (0 = the default semantics)."""
+    return LSHAttention.apply(qk, v, R, n_buckets, chunk, causal, flags)
 

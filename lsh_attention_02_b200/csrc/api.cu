@@ -92,8 +92,8 @@ static lsh_status check_desc(const lsh_attn_desc *d, Problem *p)
 {
     if (!d) return LSH_ERR_ARG;
     if (d->dtype != LSH_F32 && d->dtype != LSH_BF16) return LSH_ERR_ARG;
-    if (d->impl != LSH_IMPL_AUTO && d->impl != LSH_IMPL_SIMT && d->impl != LSH_IMPL_TC) return LSH_ERR_ARG;
     if (d->causal != 0 && d->causal != 1) return LSH_ERR_ARG;
+    if (d->flags & ~(LSH_FLAG_BUCKET_MASK | LSH_FLAG_SELF_PENALTY)) return LSH_ERR_ARG;
     if (d->B < 1 || d->H < 1 || d->L < 1 || d->n_hashes < 1 || d->chunk < 1) return LSH_ERR_SHAPE;
     if (d->n_buckets < 2 || d->n_buckets % 2 != 0 || d->n_buckets > 65536) return LSH_ERR_SHAPE;
     if (d->L % d->chunk != 0) return LSH_ERR_SHAPE;
@@ -101,28 +101,28 @@ static lsh_status check_desc(const lsh_attn_desc *d, Problem *p)
     long long segs = (long long)d->B * d->H * d->n_hashes;
     if (segs > 65535) return LSH_ERR_UNSUPPORTED;     // grid.y of the per-segment kernels
     p->B = d->B; p->H = d->H; p->L = d->L; p->d = d->d; p->nb = d->n_buckets;
-    p->R = d->n_hashes; p->m = d->chunk; p->causal = d->causal; p->dtype = d->dtype;
+    p->R = d->n_hashes; p->m = d->chunk; p->causal = d->causal; p->dtype = d->dtype; p->flags = d->flags;
     return LSH_OK;
 }
 
-// Which kernels run the attention (and the hash) for this request.
+// bf16 hash and attention run on the tensor-core kernels only; a request they
+// do not cover is refused (the sort alone does not depend on the dtype).
+static lsh_status check_envelope(const Problem &p)
+{
+    if (p.flags != 0) return LSH_ERR_UNSUPPORTED;      // optional semantics: not built yet
+    if (p.dtype == LSH_BF16 && !(attn_tc_supported(p) && hash_tc_supported(p))) return LSH_ERR_UNSUPPORTED;
+    return LSH_OK;
+}
+
+// Which kernels run is fixed by the dtype: bf16 -> tensor cores, fp32 -> CUDA cores (no TF32).
 struct Choice {
     bool tc_attn;
     bool tc_hash;
 };
-static lsh_status choose(const lsh_attn_desc *d, const Problem &p, Choice *c)
+static Choice choose(const Problem &p)
 {
-    bool attn_ok = attn_tc_supported(p), hash_ok = hash_tc_supported(p);
-    if (d->impl == LSH_IMPL_SIMT) { c->tc_attn = false; c->tc_hash = false; return LSH_OK; }
-    if (d->impl == LSH_IMPL_TC) {
-        if (!attn_ok) return LSH_ERR_UNSUPPORTED;
-        c->tc_attn = true;
-        c->tc_hash = hash_ok;
-        return LSH_OK;
-    }
-    c->tc_attn = attn_ok;
-    c->tc_hash = hash_ok;
-    return LSH_OK;
+    const bool tc = p.dtype == LSH_BF16;
+    return Choice{tc, tc};
 }
 
 static bool aligned16(const void *ptr) { return ((uintptr_t)ptr & 15u) == 0; }
@@ -165,7 +165,7 @@ static lsh_status run_attn_fwd(const Problem &p, const Choice &c, const void *qk
     LSH_TRY(staged(LSH_STAGE_ATTN_FWD, 1, st, [&] {
                 return c.tc_attn
                            ? launch_attn_fwd_tc(p, qk, v, perm, w.invnorm, (__nv_bfloat16 *)w.o_r, lse, w.status, st)
-                           : launch_attn_fwd_simt(p, qk, v, perm, w.invnorm, (float *)w.o_r, lse, st);
+                           : launch_attn_fwd_simt(p, qk, v, perm, w.invnorm, (float *)w.o_r, lse, w.status, st);
             }), "attention forward");
     LSH_TRY(staged(LSH_STAGE_COMBINE, 1, st, [&] { return launch_combine(p, w.o_r, c.tc_attn, lse, out, st); }),
             "round merge");
@@ -182,7 +182,8 @@ size_t lsh_attn_workspace_size(const lsh_attn_desc *desc, int for_backward)
 {
     Problem p;
     Choice c;
-    if (check_desc(desc, &p) != LSH_OK || choose(desc, p, &c) != LSH_OK) return 0;
+    if (check_desc(desc, &p) != LSH_OK) return 0;
+    c = choose(p);
     return plan_workspace(p, for_backward != 0, c.tc_attn, c.tc_hash, nullptr).bytes;
 }
 
@@ -193,7 +194,8 @@ lsh_status lsh_attn_hash(const lsh_attn_desc *desc, const void *qk, const void *
     Choice c;
     lsh_status s;
     if ((s = check_desc(desc, &p)) != LSH_OK) return s;
-    if ((s = choose(desc, p, &c)) != LSH_OK) return s;
+    if ((s = check_envelope(p)) != LSH_OK) return s;
+    c = choose(p);
     if ((s = check_ptrs({qk, R})) != LSH_OK) return s;
     if (!buckets) return LSH_ERR_ARG;
     Workspace w = plan_workspace(p, false, c.tc_attn, c.tc_hash, nullptr);
@@ -215,7 +217,7 @@ lsh_status lsh_attn_sort(const lsh_attn_desc *desc, const uint16_t *buckets, int
     Choice c;
     lsh_status s;
     if ((s = check_desc(desc, &p)) != LSH_OK) return s;
-    if ((s = choose(desc, p, &c)) != LSH_OK) return s;
+    c = choose(p);
     if (!buckets || !perm) return LSH_ERR_ARG;
     Workspace w = plan_workspace(p, false, c.tc_attn, c.tc_hash, nullptr);
     if ((s = check_ws(workspace, ws_bytes, w.bytes)) != LSH_OK) return s;
@@ -235,10 +237,8 @@ int lsh_attn_last_near_ties(void)
 lsh_status lsh_attn_sort_static(const lsh_attn_desc *desc, const uint16_t *buckets, int32_t *perm, void *stream)
 {
     Problem p;
-    Choice c;
     lsh_status s;
     if ((s = check_desc(desc, &p)) != LSH_OK) return s;
-    if ((s = choose(desc, p, &c)) != LSH_OK) return s;
     if (!buckets || !perm) return LSH_ERR_ARG;
     size_t need = 0;
     plan_sort_scratch(p, nullptr, &need);
@@ -264,7 +264,8 @@ lsh_status lsh_attn_fwd_sorted(const lsh_attn_desc *desc, const void *qk, const 
     Choice c;
     lsh_status s;
     if ((s = check_desc(desc, &p)) != LSH_OK) return s;
-    if ((s = choose(desc, p, &c)) != LSH_OK) return s;
+    if ((s = check_envelope(p)) != LSH_OK) return s;
+    c = choose(p);
     if ((s = check_ptrs({qk, v, out, lse})) != LSH_OK) return s;
     if (!perm) return LSH_ERR_ARG;
     Workspace w = plan_workspace(p, false, c.tc_attn, c.tc_hash, nullptr);
@@ -282,7 +283,8 @@ lsh_status lsh_attn_fwd(const lsh_attn_desc *desc, const void *qk, const void *v
     Choice c;
     lsh_status s;
     if ((s = check_desc(desc, &p)) != LSH_OK) return s;
-    if ((s = choose(desc, p, &c)) != LSH_OK) return s;
+    if ((s = check_envelope(p)) != LSH_OK) return s;
+    c = choose(p);
     if ((s = check_ptrs({qk, v, R, out, lse})) != LSH_OK) return s;
     Workspace w = plan_workspace(p, false, c.tc_attn, c.tc_hash, nullptr);
     if ((s = check_ws(workspace, ws_bytes, w.bytes)) != LSH_OK) return s;
@@ -302,7 +304,8 @@ lsh_status lsh_attn_bwd(const lsh_attn_desc *desc, const void *qk, const void *v
     Choice c;
     lsh_status s;
     if ((s = check_desc(desc, &p)) != LSH_OK) return s;
-    if ((s = choose(desc, p, &c)) != LSH_OK) return s;
+    if ((s = check_envelope(p)) != LSH_OK) return s;
+    c = choose(p);
     if ((s = check_ptrs({qk, v, out, lse, dout, dqk, dv})) != LSH_OK) return s;
     if (!perm && !R) return LSH_ERR_ARG;
     Workspace w = plan_workspace(p, true, c.tc_attn, c.tc_hash, nullptr);
@@ -324,7 +327,7 @@ lsh_status lsh_attn_bwd(const lsh_attn_desc *desc, const void *qk, const void *v
                 return c.tc_attn ? launch_attn_bwd_tc(p, qk, v, dout, perm, w.invnorm, w.lse_all, w.delta, w.dx_acc,
                                                       w.dv_acc, w.status, st)
                                  : launch_attn_bwd_simt(p, qk, v, dout, perm, w.invnorm, w.lse_all, w.delta,
-                                                        w.self_only, w.dx_acc, w.dv_acc, st);
+                                                        w.self_only, w.dx_acc, w.dv_acc, w.status, st);
             }), "attention backward");
     LSH_TRY(staged(LSH_STAGE_BWD_FINAL, 1, st,
                    [&] { return launch_bwd_finalize(p, w.dx_acc, w.dv_acc, dqk, dv, st); }),
@@ -340,7 +343,8 @@ lsh_status lsh_attn_poll(void *workspace, void *stream)
     LSH_TRY(cudaMemcpyAsync(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost, st), "status read");
     LSH_TRY(cudaStreamSynchronize(st), "status read");
     LSH_TRY(cudaMemsetAsync(workspace, 0, sizeof(word), st), "status clear");
-    return (word & kStatusTimeout) ? LSH_ERR_TIMEOUT : LSH_OK;
+    if (word & kStatusTimeout) return LSH_ERR_TIMEOUT;
+    return (word & kStatusBadPerm) ? LSH_ERR_ARG : LSH_OK;
 }
 
 lsh_status lsh_attn_selftest_timeout(void *workspace, int64_t budget_cycles, void *stream)

@@ -84,6 +84,7 @@ struct BwdSmem {
     uint64_t epi_done;              // every compute warp finished the previous tile's epilogue
     float gxh[kK];
     alignas(16) int ridx[kComputeWarps][2][32];   // row indices of the staged rows, per warp
+    uint64_t drain;                 // timeout path: the MMA issuer's last products
     uint32_t tmem_base;
     int abort;
 };
@@ -307,7 +308,7 @@ attn_bwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
     extern __shared__ uint8_t smem_raw[];
     BwdSmem &sm = *reinterpret_cast<BwdSmem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int n_k = L / kK;
+    const int n_k = (L + kK - 1) / kK;          // the last tile may hold one chunk only
     const int n_runs = (n_k + kRun - 1) / kRun;
 
     if (tid == 0) {
@@ -321,6 +322,7 @@ attn_bwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
         tc::mbar_init(&sm.bar_free, kComputeWarps);
         tc::mbar_init(&sm.gx_ready, kComputeWarps / 2);
         tc::mbar_init(&sm.epi_done, kComputeWarps);
+        tc::mbar_init(&sm.drain, 1);
         sm.abort = 0;
         tc::fence_mbar_init();
     }
@@ -344,8 +346,12 @@ attn_bwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
             for (int j = 0; j < kPosPer; ++j) {
                 const int e = ptid + j * kProducerThreads;
                 const int sl = slot0 + e;
+                const bool in = e < 256 && sl >= 0 && sl < L;
                 const int pl = P[min(max(sl, 0), L - 1)];
-                pn[j] = (e < 256 && sl >= 0 && sl < L) ? pl : -1;
+                // a permutation entry outside [0, L) leaves its slot empty and is reported
+                const bool good = (unsigned)pl < (unsigned)L;
+                if (in && !good) atomicOr(status, kStatusBadPerm);
+                pn[j] = in && good ? pl : -1;
             }
         };
         TileIter ti{blockIdx.x, 0};
@@ -474,6 +480,7 @@ attn_bwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
                 tc::mma_commit(&sm.bar_o);
                 LSH_PHASE(1, 1, it, 4);
             }
+            if (*reinterpret_cast<volatile int *>(&sm.abort)) tc::mma_drain(&sm.drain, status);
         }
     } else {
         // ================= compute warps
@@ -647,7 +654,7 @@ cudaError_t launch_attn_bwd_tc(const Problem &p, const void *x, const void *v, c
     int dev = 0, sms = 0;
     if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
     if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
-    const long long n_units = p.S() * ((p.L / kK + kRun - 1) / kRun);
+    const long long n_units = p.S() * (((p.L + kK - 1) / kK + kRun - 1) / kRun);
     const unsigned grid = (unsigned)std::min<long long>(n_units, (long long)sms);
     kern<<<grid, kThreads, smem, st>>>((const __nv_bfloat16 *)x, (const __nv_bfloat16 *)v,
                                                      (const __nv_bfloat16 *)dout, perm, invnorm, lse_all,

@@ -75,6 +75,7 @@ struct FwdSmem {
     Stage st[kStages];
     uint64_t full[kStages], empty[kStages];
     uint64_t s_full[2], p_half[2], p_full[2], o_full[2], o_free[2];  // p_half: P of keys 0..63 written
+    uint64_t drain;                 // timeout path: the MMA issuer's last products
     uint32_t tmem_base;
     int abort;
 };
@@ -261,7 +262,7 @@ attn_fwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
     extern __shared__ uint8_t smem_raw[];
     FwdSmem &sm = *reinterpret_cast<FwdSmem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int n_k = L / kQ;
+    const int n_k = (L + kQ - 1) / kQ;          // the last tile may hold one chunk only
 
     if (tid == 0) {
         for (int s = 0; s < kStages; ++s) {
@@ -275,6 +276,7 @@ attn_fwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
             tc::mbar_init(&sm.o_full[g], 1);
             tc::mbar_init(&sm.o_free[g], 4);
         }
+        tc::mbar_init(&sm.drain, 1);
         sm.abort = 0;
         tc::fence_mbar_init();
     }
@@ -290,6 +292,9 @@ attn_fwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
         const int ptid = tid - kSoftmaxWarps * 32, pw = ptid >> 5;
         // positions of the next tile, loaded a tile ahead (two slots per thread)
         int pn[2] = {-1, -1};
+        // A slot outside [0, L) (chunk -1, or the missing chunk of a last tile
+        // when L % 128 == 64) is empty (-1); so is a permutation entry outside
+        // [0, L), which is also reported in the status word.
         auto load_pos = [&](long long tile) {
             const TileCoord c = tile_coord(tile, R, n_k);
             const int32_t *P = perm + c.seg * L;
@@ -297,9 +302,12 @@ attn_fwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
 #pragma unroll
             for (int j = 0; j < 2; ++j) {
                 const int e = ptid + j * kProducerThreads;     // kW = 2 * kProducerThreads
-                const int sl = slot0 + e;                      // <= L - 1
-                const int pl = P[max(sl, 0)];
-                pn[j] = sl >= 0 ? pl : -1;
+                const int sl = slot0 + e;
+                const bool in = sl >= 0 && sl < L;
+                const int pl = P[min(max(sl, 0), L - 1)];
+                const bool good = (unsigned)pl < (unsigned)L;
+                if (in && !good) atomicOr(status, kStatusBadPerm);
+                pn[j] = in && good ? pl : -1;
             }
         };
         if (blockIdx.x < n_tiles) load_pos(blockIdx.x);
@@ -439,6 +447,7 @@ attn_fwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
                     __nanosleep(20);
                 }
             }
+            if (*reinterpret_cast<volatile int *>(&sm.abort)) tc::mma_drain(&sm.drain, status);
         }
     } else {
         // ================= softmax groups: group g takes the CTA's tiles it = g, g + 2, ...
@@ -493,8 +502,10 @@ attn_fwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
             const float rl = 1.0f / l;
 #pragma unroll
             for (int d = 0; d < kDim; ++d) o[d] *= rl;
-            store_row(o_r + (tcd.seg * L + qpos) * kDim, o);
-            lse[tcd.seg * L + qpos] = row_lse;
+            if (qpos >= 0) {                     // an empty query slot has no output
+                store_row(o_r + (tcd.seg * L + qpos) * kDim, o);
+                lse[tcd.seg * L + qpos] = row_lse;
+            }
             if (mark) LSH_PHASE(0, 2 + g, it, 5);
         }
     }
@@ -511,7 +522,7 @@ attn_fwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
 
 bool attn_tc_supported(const Problem &p)
 {
-    return p.dtype == LSH_BF16 && p.d == kDim && p.m == 64 && p.L % kQ == 0 && p.tokens() < (1LL << 31);
+    return p.dtype == LSH_BF16 && p.d == kDim && p.m == 64 && p.L % 64 == 0 && p.tokens() < (1LL << 31);
 }
 
 cudaError_t launch_attn_fwd_tc(const Problem &p, const void *x, const void *v, const int32_t *perm,
@@ -526,7 +537,7 @@ cudaError_t launch_attn_fwd_tc(const Problem &p, const void *x, const void *v, c
     int dev = 0, sms = 0;
     if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
     if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
-    const long long n_tiles = p.S() * (p.L / kQ);
+    const long long n_tiles = p.S() * ((p.L + kQ - 1) / kQ);
     const unsigned grid = (unsigned)std::min<long long>(n_tiles, (long long)sms);
     kern<<<grid, kThreads, smem, st>>>((const __nv_bfloat16 *)x, (const __nv_bfloat16 *)v, perm, o_r, lse, p.L, p.R, n_tiles,
                                                      p.causal, 1.0f / sqrtf((float)p.d), status);

@@ -14,7 +14,7 @@ constexpr int kDim = 64;              // head dimension supported by every kerne
 
 // ---------------------------------------------------------------- problem
 struct Problem {
-    int B, H, L, d, nb, R, m, causal, dtype;
+    int B, H, L, d, nb, R, m, causal, dtype, flags;
     long long BH() const { return (long long)B * H; }
     long long S() const { return BH() * R; }         // (b, h, round) segments
     long long tokens() const { return BH() * L; }
@@ -137,7 +137,7 @@ size_t hash_tc_scratch_bytes(const Problem &p);
 cudaError_t launch_sort(const Problem &p, const uint16_t *buckets, int32_t *perm, const Workspace &ws,
                         cudaStream_t st);
 cudaError_t launch_attn_fwd_simt(const Problem &p, const void *x, const void *v, const int32_t *perm,
-                                 const float *invnorm, float *o_r, float *lse, cudaStream_t st);
+                                 const float *invnorm, float *o_r, float *lse, uint32_t *status, cudaStream_t st);
 cudaError_t launch_attn_fwd_tc(const Problem &p, const void *x, const void *v, const int32_t *perm,
                                const float *invnorm, __nv_bfloat16 *o_r, float *lse, uint32_t *status,
                                cudaStream_t st);
@@ -149,7 +149,7 @@ cudaError_t launch_bwd_prep(const Problem &p, const float *lse, const void *out,
 cudaError_t launch_attn_bwd_simt(const Problem &p, const void *x, const void *v, const void *dout,
                                  const int32_t *perm, const float *invnorm, const float *lse_all,
                                  const float *delta, uint8_t *self_only, float *dx_acc, float *dv_acc,
-                                 cudaStream_t st);
+                                 uint32_t *status, cudaStream_t st);
 cudaError_t launch_attn_bwd_tc(const Problem &p, const void *x, const void *v, const void *dout,
                                const int32_t *perm, const float *invnorm, const float *lse_all,
                                const float *delta, float *dx_acc, float *dv_acc, uint32_t *status,
@@ -160,6 +160,7 @@ cudaError_t launch_bwd_finalize(const Problem &p, const float *dx_acc, const flo
 cudaError_t launch_wait_selftest(uint32_t *status, long long budget, cudaStream_t st);
 
 // Status bits written by kernels into Workspace::status.
-constexpr uint32_t kStatusTimeout = 1u;
+constexpr uint32_t kStatusTimeout = 1u;     // a bounded wait gave up
+constexpr uint32_t kStatusBadPerm = 2u;     // a permutation entry outside [0, L) was read (and ignored)
 
 }  // namespace lsh

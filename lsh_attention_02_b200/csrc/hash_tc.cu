@@ -45,38 +45,43 @@ struct HashSmem {
     uint64_t full[kStages], empty[kStages];
     uint64_t a_full[2], a_empty[2];
     uint64_t acc_full[2][2], acc_empty[2];  // [buffer][M-tile]
+    uint64_t drain;                         // timeout path: the MMA issuer's last products
     uint32_t tmem_base;
     int abort;
 };
 
-// R [R, 64, half] (k-major per column) -> Rs [R, half, 64] rows of 64 k, with the
+// R [R, 64, half] (k-major per column) -> Rs [R, hp, 64] rows of 64 k, with the
 // 16-byte chunks of row n stored at position (chunk ^ (n & 7)): the shared-memory
 // image of a K-major 128-byte-swizzled B operand, so one bulk copy lands a tile.
+// Columns n >= half (padding up to hp, a multiple of the N-tile) are zero: their
+// projections are exactly 0, which never displaces the first maximum of a real
+// column (max(xR) >= 0 or -min(xR) > 0 decides the side with a real column, and
+// real columns come first in index order).
 __global__ void rot_swizzle_kernel(const __nv_bfloat16 *__restrict__ R, __nv_bfloat16 *__restrict__ Rs, int half,
-                                   int rounds)
+                                   int hp, int rounds)
 {
-    long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;   // over rounds * half * 64
-    long long total = (long long)rounds * half * kDim;
+    long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;   // over rounds * hp * 64
+    long long total = (long long)rounds * hp * kDim;
     if (idx >= total) return;
     int k = (int)(idx % kDim);
     long long rn = idx / kDim;
-    int n = (int)(rn % half);
-    int r = (int)(rn / half);
-    __nv_bfloat16 val = R[((long long)r * kDim + k) * half + n];
+    int n = (int)(rn % hp);
+    int r = (int)(rn / hp);
+    __nv_bfloat16 val = n < half ? R[((long long)r * kDim + k) * half + n] : __float2bfloat16_rn(0.f);
     const uint32_t off = tc::sw128_offset((uint32_t)n, (uint32_t)k);
-    *reinterpret_cast<__nv_bfloat16 *>(reinterpret_cast<uint8_t *>(Rs) + (long long)r * half * 128 + off) = val;
+    *reinterpret_cast<__nv_bfloat16 *>(reinterpret_cast<uint8_t *>(Rs) + (long long)r * hp * 128 + off) = val;
 }
 
 template <int NT>
 __global__ void __launch_bounds__(kThreads, 1)
 hash_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __nv_bfloat16 *__restrict__ Rs,
-               uint16_t *__restrict__ buckets, long long rows_total, int L, int rounds, int half,
+               uint16_t *__restrict__ buckets, long long rows_total, int L, int rounds, int half, int hp,
                uint32_t *__restrict__ status)
 {
     extern __shared__ uint8_t smem_raw[];
     HashSmem &sm = *reinterpret_cast<HashSmem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int n_nt = half / NT;
+    const int n_nt = hp / NT;                  // hp: half rounded up to a whole N-tile
     const int items = rounds * n_nt;
     const long long n_blocks = (rows_total + kRows - 1) / kRows;
     if (threadIdx.x == 0) LSH_PHASE(0, 3, 0, 0);
@@ -90,6 +95,7 @@ hash_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __nv_bfloat16 *__
             tc::mbar_init(&sm.acc_full[b][1], 1);
             tc::mbar_init(&sm.acc_empty[b], kEpiWarps);
         }
+        tc::mbar_init(&sm.drain, 1);
         sm.abort = 0;
         tc::fence_mbar_init();
     }
@@ -124,7 +130,7 @@ hash_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __nv_bfloat16 *__
                     if (it >= kStages && !tc::mbar_wait(&sm.empty[s], ph ^ 1u, &sm.abort, status)) { ok = false; break; }
                     LSH_PHASE(0, 1, it, 1);
                     const int r = i / n_nt, nt = i % n_nt;
-                    const __nv_bfloat16 *src = Rs + ((long long)r * half + (long long)nt * NT) * kDim;
+                    const __nv_bfloat16 *src = Rs + ((long long)r * hp + (long long)nt * NT) * kDim;
                     tc::mbar_arrive_expect_tx(&sm.full[s], NT * 128);
                     tc::bulk_g2s(sm.B[s], src, NT * 128, &sm.full[s]);
                     ++r_issued;
@@ -182,6 +188,7 @@ hash_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __nv_bfloat16 *__
                 }
                 if (ok) tc::mma_commit(&sm.a_empty[xa]);
             }
+            if (*reinterpret_cast<volatile int *>(&sm.abort)) tc::mma_drain(&sm.drain, status);
         }
     } else {
         // ---------------- epilogue: one row per thread
@@ -300,8 +307,8 @@ hash_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __nv_bfloat16 *__
 }
 
 template <int NT>
-cudaError_t launch_nt(const Problem &p, const void *x, const __nv_bfloat16 *Rs, uint16_t *buckets, uint32_t *status,
-                      cudaStream_t st)
+cudaError_t launch_nt(const Problem &p, const void *x, const __nv_bfloat16 *Rs, int hp, uint16_t *buckets,
+                      uint32_t *status, cudaStream_t st)
 {
     // one CTA per SM: each holds all 512 TMEM columns
     const size_t smem = sizeof(HashSmem) + 1024;
@@ -315,46 +322,53 @@ cudaError_t launch_nt(const Problem &p, const void *x, const __nv_bfloat16 *Rs, 
     if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
     const long long blocks = (rows + kRows - 1) / kRows;
     const unsigned grid = (unsigned)std::min<long long>(blocks, sms);
-    hash_tc_kernel<NT><<<grid, kThreads, smem, st>>>(xmap, Rs, buckets, rows, p.L, p.R, p.nb / 2, status);
+    hash_tc_kernel<NT><<<grid, kThreads, smem, st>>>(xmap, Rs, buckets, rows, p.L, p.R, p.nb / 2, hp, status);
     return cudaGetLastError();
 }
 
+// N-tile width: the widest of 128, 96, 64 that divides n_buckets/2, else 32
+// with the last tile padded by zero rotation columns.
 int pick_nt(int half)
 {
     if (half % 128 == 0) return 128;
     if (half % 96 == 0) return 96;
     if (half % 64 == 0) return 64;
-    if (half % 32 == 0) return 32;
-    return 0;
+    return 32;
+}
+int padded_half(int half)
+{
+    const int nt = pick_nt(half);
+    return (half + nt - 1) / nt * nt;
 }
 
 }  // namespace
 
-// Rows are addressed by 32-bit TMA coordinates; a problem smaller than one
-// 128-row TMA box takes the SIMT hash.
+// Rows are addressed by 32-bit TMA coordinates in boxes of 128 rows.
 bool hash_tc_supported(const Problem &p)
 {
-    return p.dtype == LSH_BF16 && p.d == kDim && pick_nt(p.nb / 2) != 0 && p.tokens() >= 128 &&
-           p.tokens() < (1LL << 31) - kRows;
+    return p.dtype == LSH_BF16 && p.d == kDim && p.tokens() >= 128 && p.tokens() < (1LL << 31) - kRows;
 }
 
-size_t hash_tc_scratch_bytes(const Problem &p) { return (size_t)p.R * (p.nb / 2) * kDim * sizeof(__nv_bfloat16); }
+size_t hash_tc_scratch_bytes(const Problem &p)
+{
+    return (size_t)p.R * padded_half(p.nb / 2) * kDim * sizeof(__nv_bfloat16);
+}
 
 cudaError_t launch_hash_tc(const Problem &p, const void *x, const void *R, uint16_t *buckets, void *scratch,
                            uint32_t *status, cudaStream_t st)
 {
-    const int half = p.nb / 2;
+    const int half = p.nb / 2, hp = padded_half(half);
     __nv_bfloat16 *Rs = (__nv_bfloat16 *)scratch;
-    const long long total = (long long)p.R * half * kDim;
-    rot_swizzle_kernel<<<(unsigned)((total + 255) / 256), 256, 0, st>>>((const __nv_bfloat16 *)R, Rs, half, p.R);
+    const long long total = (long long)p.R * hp * kDim;
+    rot_swizzle_kernel<<<(unsigned)((total + 255) / 256), 256, 0, st>>>((const __nv_bfloat16 *)R, Rs, half, hp,
+                                                                        p.R);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     switch (pick_nt(half)) {
-    case 128: return launch_nt<128>(p, x, Rs, buckets, status, st);
-    case 96: return launch_nt<96>(p, x, Rs, buckets, status, st);
-    case 64: return launch_nt<64>(p, x, Rs, buckets, status, st);
-    case 32: return launch_nt<32>(p, x, Rs, buckets, status, st);
-    default: return cudaErrorInvalidValue;
+    case 128: return launch_nt<128>(p, x, Rs, hp, buckets, status, st);
+    case 96: return launch_nt<96>(p, x, Rs, hp, buckets, status, st);
+    case 64: return launch_nt<64>(p, x, Rs, hp, buckets, status, st);
+    default: return launch_nt<32>(p, x, Rs, hp, buckets, status, st);
     }
 }
 

@@ -29,12 +29,10 @@ __global__ void invnorm_kernel(const T *__restrict__ x, float *__restrict__ invn
 
 cudaError_t launch_invnorm(const Problem &p, const void *x, float *invnorm, cudaStream_t st)
 {
+    if (p.dtype != LSH_F32) return cudaErrorInvalidValue;      // the tensor-core kernels compute their own norms
     long long rows = p.tokens();
     unsigned grid = (unsigned)((rows + 127) / 128);
-    if (p.dtype == LSH_F32)
-        invnorm_kernel<float><<<grid, 128, 0, st>>>((const float *)x, invnorm, rows);
-    else
-        invnorm_kernel<__nv_bfloat16><<<grid, 128, 0, st>>>((const __nv_bfloat16 *)x, invnorm, rows);
+    invnorm_kernel<float><<<grid, 128, 0, st>>>((const float *)x, invnorm, rows);
     return cudaGetLastError();
 }
 
@@ -69,14 +67,11 @@ __global__ void hash_simt_kernel(const T *__restrict__ x, const T *__restrict__ 
 
 cudaError_t launch_hash_simt(const Problem &p, const void *x, const void *R, uint16_t *buckets, cudaStream_t st)
 {
+    if (p.dtype != LSH_F32) return cudaErrorInvalidValue;      // bf16 runs on the tensor-core hash
     long long rows = p.tokens();
     dim3 grid((unsigned)((rows + 127) / 128), p.R);
-    if (p.dtype == LSH_F32)
-        hash_simt_kernel<float><<<grid, 128, 0, st>>>((const float *)x, (const float *)R, buckets, p.BH(), p.L,
-                                                      p.R, p.nb / 2);
-    else
-        hash_simt_kernel<__nv_bfloat16><<<grid, 128, 0, st>>>((const __nv_bfloat16 *)x, (const __nv_bfloat16 *)R,
-                                                              buckets, p.BH(), p.L, p.R, p.nb / 2);
+    hash_simt_kernel<float><<<grid, 128, 0, st>>>((const float *)x, (const float *)R, buckets, p.BH(), p.L, p.R,
+                                                  p.nb / 2);
     return cudaGetLastError();
 }
 
@@ -159,6 +154,15 @@ __device__ __forceinline__ Window window_of(int s, int m, int L)
     return w;
 }
 
+// A permutation entry outside [0, L) marks an empty slot: it is skipped and
+// reported in the status word.
+__device__ __forceinline__ bool valid_pos(int j, int L, uint32_t *status)
+{
+    if ((unsigned)j < (unsigned)L) return true;
+    atomicOr(status, kStatusBadPerm);
+    return false;
+}
+
 // ------------------------------------------------------------------ forward
 // One thread per (segment, sorted slot): full softmax over the window, output
 // and logsumexp written at the query's original position.
@@ -166,7 +170,7 @@ template <typename T>
 __global__ void attn_fwd_simt_kernel(const T *__restrict__ x, const T *__restrict__ v,
                                      const int32_t *__restrict__ perm, const float *__restrict__ invnorm,
                                      float *__restrict__ o_r, float *__restrict__ lse, int L, int R, int m,
-                                     int causal, float tau)
+                                     int causal, float tau, uint32_t *__restrict__ status)
 {
     const long long seg = blockIdx.y;
     const int s = blockIdx.x * blockDim.x + threadIdx.x;
@@ -177,6 +181,7 @@ __global__ void attn_fwd_simt_kernel(const T *__restrict__ x, const T *__restric
     const T *V = v + bh * L * kDim;
     const float *IN = invnorm + bh * L;
     const int i = P[s];
+    if (!valid_pos(i, L, status)) return;          // an empty slot has no output
     float q[kDim], kv[kDim];
     load_row(X + (long long)i * kDim, q);
     const Window w = window_of(s, m, L);
@@ -185,6 +190,7 @@ __global__ void attn_fwd_simt_kernel(const T *__restrict__ x, const T *__restric
     for (int t = w.w0; t < w.w1; ++t) {
         if (t == s) continue;
         int j = P[t];
+        if (!valid_pos(j, L, status)) continue;
         if (causal && j > i) continue;
         load_row(X + (long long)j * kDim, kv);
         float z = tau * (dot64(q, kv) * IN[j]);
@@ -203,6 +209,7 @@ __global__ void attn_fwd_simt_kernel(const T *__restrict__ x, const T *__restric
         for (int t = w.w0; t < w.w1; ++t) {
             if (t == s) continue;
             int j = P[t];
+            if (!valid_pos(j, L, status)) continue;
             if (causal && j > i) continue;
             load_row(X + (long long)j * kDim, kv);
             float e = expf(tau * (dot64(q, kv) * IN[j]) - mx);
@@ -221,17 +228,13 @@ __global__ void attn_fwd_simt_kernel(const T *__restrict__ x, const T *__restric
 }
 
 cudaError_t launch_attn_fwd_simt(const Problem &p, const void *x, const void *v, const int32_t *perm,
-                                 const float *invnorm, float *o_r, float *lse, cudaStream_t st)
+                                 const float *invnorm, float *o_r, float *lse, uint32_t *status, cudaStream_t st)
 {
+    if (p.dtype != LSH_F32) return cudaErrorInvalidValue;      // bf16 runs on the tensor-core kernels
     dim3 grid((p.L + 127) / 128, (unsigned)p.S());
     float tau = 1.0f / sqrtf((float)p.d);
-    if (p.dtype == LSH_F32)
-        attn_fwd_simt_kernel<float><<<grid, 128, 0, st>>>((const float *)x, (const float *)v, perm, invnorm, o_r, lse,
-                                                          p.L, p.R, p.m, p.causal, tau);
-    else
-        attn_fwd_simt_kernel<__nv_bfloat16><<<grid, 128, 0, st>>>((const __nv_bfloat16 *)x,
-                                                                  (const __nv_bfloat16 *)v, perm, invnorm, o_r,
-                                                                  lse, p.L, p.R, p.m, p.causal, tau);
+    attn_fwd_simt_kernel<float><<<grid, 128, 0, st>>>((const float *)x, (const float *)v, perm, invnorm, o_r, lse,
+                                                      p.L, p.R, p.m, p.causal, tau, status);
     return cudaGetLastError();
 }
 
@@ -456,7 +459,7 @@ __global__ void attn_bwd_q_simt_kernel(const T *__restrict__ x, const T *__restr
                                        const int32_t *__restrict__ perm, const float *__restrict__ invnorm,
                                        const float *__restrict__ lse_all, const float *__restrict__ delta,
                                        uint8_t *__restrict__ self_only, float *__restrict__ dx_acc, int L, int R,
-                                       int m, int causal, float tau)
+                                       int m, int causal, float tau, uint32_t *__restrict__ status)
 {
     const long long seg = blockIdx.y;
     const int s = blockIdx.x * blockDim.x + threadIdx.x;
@@ -467,6 +470,10 @@ __global__ void attn_bwd_q_simt_kernel(const T *__restrict__ x, const T *__restr
     const T *V = v + bh * L * kDim;
     const float *IN = invnorm + bh * L;
     const int i = P[s];
+    if (!valid_pos(i, L, status)) {
+        self_only[seg * L + s] = 0;
+        return;
+    }
     float q[kDim], g[kDim], kv[kDim], dq[kDim];
     load_row(X + (long long)i * kDim, q);
     load_row(dout + (bh * L + i) * kDim, g);
@@ -478,6 +485,7 @@ __global__ void attn_bwd_q_simt_kernel(const T *__restrict__ x, const T *__restr
     for (int t = w.w0; t < w.w1; ++t) {
         if (t == s) continue;
         int j = P[t];
+        if (!valid_pos(j, L, status)) continue;
         if (causal && j > i) continue;
         ++cnt;
         load_row(X + (long long)j * kDim, kv);
@@ -513,7 +521,8 @@ __global__ void attn_bwd_k_simt_kernel(const T *__restrict__ x, const T *__restr
                                        const int32_t *__restrict__ perm, const float *__restrict__ invnorm,
                                        const float *__restrict__ lse_all, const float *__restrict__ delta,
                                        const uint8_t *__restrict__ self_only, float *__restrict__ dx_acc,
-                                       float *__restrict__ dv_acc, int L, int R, int m, int causal, float tau)
+                                       float *__restrict__ dv_acc, int L, int R, int m, int causal, float tau,
+                                       uint32_t *__restrict__ status)
 {
     const long long seg = blockIdx.y;
     const int t = blockIdx.x * blockDim.x + threadIdx.x;
@@ -523,6 +532,7 @@ __global__ void attn_bwd_k_simt_kernel(const T *__restrict__ x, const T *__restr
     const T *X = x + bh * L * kDim;
     const float *IN = invnorm + bh * L;
     const int j = P[t];
+    if (!valid_pos(j, L, status)) return;
     float kx[kDim], vj[kDim], gk[kDim], dvj[kDim], q[kDim], g[kDim];
     load_row(X + (long long)j * kDim, kx);
     load_row(v + (bh * L + j) * kDim, vj);
@@ -533,6 +543,7 @@ __global__ void attn_bwd_k_simt_kernel(const T *__restrict__ x, const T *__restr
     const int s0 = c * m, s1 = min((c + 2) * m, L);
     for (int s = s0; s < s1; ++s) {
         int i = P[s];
+        if (!valid_pos(i, L, status)) continue;
         bool cand;
         if (s == t) cand = self_only[seg * L + s] != 0;
         else cand = !(causal && j > i);
@@ -563,26 +574,17 @@ __global__ void attn_bwd_k_simt_kernel(const T *__restrict__ x, const T *__restr
 cudaError_t launch_attn_bwd_simt(const Problem &p, const void *x, const void *v, const void *dout,
                                  const int32_t *perm, const float *invnorm, const float *lse_all,
                                  const float *delta, uint8_t *self_only, float *dx_acc, float *dv_acc,
-                                 cudaStream_t st)
+                                 uint32_t *status, cudaStream_t st)
 {
+    if (p.dtype != LSH_F32) return cudaErrorInvalidValue;      // bf16 runs on the tensor-core kernels
     dim3 grid((p.L + 127) / 128, (unsigned)p.S());
     float tau = 1.0f / sqrtf((float)p.d);
-    if (p.dtype == LSH_F32) {
-        attn_bwd_q_simt_kernel<float><<<grid, 128, 0, st>>>((const float *)x, (const float *)v, (const float *)dout,
-                                                            perm, invnorm, lse_all, delta, self_only, dx_acc, p.L,
-                                                            p.R, p.m, p.causal, tau);
-        attn_bwd_k_simt_kernel<float><<<grid, 128, 0, st>>>((const float *)x, (const float *)v, (const float *)dout,
-                                                            perm, invnorm, lse_all, delta, self_only, dx_acc,
-                                                            dv_acc, p.L, p.R, p.m, p.causal, tau);
-    } else {
-        using B = __nv_bfloat16;
-        attn_bwd_q_simt_kernel<B><<<grid, 128, 0, st>>>((const B *)x, (const B *)v, (const B *)dout, perm, invnorm,
-                                                        lse_all, delta, self_only, dx_acc, p.L, p.R, p.m, p.causal,
-                                                        tau);
-        attn_bwd_k_simt_kernel<B><<<grid, 128, 0, st>>>((const B *)x, (const B *)v, (const B *)dout, perm, invnorm,
-                                                        lse_all, delta, self_only, dx_acc, dv_acc, p.L, p.R, p.m,
-                                                        p.causal, tau);
-    }
+    attn_bwd_q_simt_kernel<float><<<grid, 128, 0, st>>>((const float *)x, (const float *)v, (const float *)dout,
+                                                        perm, invnorm, lse_all, delta, self_only, dx_acc, p.L,
+                                                        p.R, p.m, p.causal, tau, status);
+    attn_bwd_k_simt_kernel<float><<<grid, 128, 0, st>>>((const float *)x, (const float *)v, (const float *)dout,
+                                                        perm, invnorm, lse_all, delta, self_only, dx_acc,
+                                                        dv_acc, p.L, p.R, p.m, p.causal, tau, status);
     return cudaGetLastError();
 }
 

@@ -16,7 +16,6 @@
 //           element is written at offset + rank.
 // Pass 0 reads the bucket ids in position order with the position as the
 // value; the last pass writes only the values, i.e. the permutation.
-#include <mutex>
 
 #include "common.cuh"
 
@@ -177,7 +176,7 @@ cudaError_t launch_sort(const Problem &p, const uint16_t *buckets, int32_t *perm
 // Scratch of lsh_attn_sort_static: one array per device, part of this
 // module's static device memory, so the entry point itself never allocates.
 // The driver creates it when the module is loaded; its address is looked up
-// once per device and cached.
+// on each call.
 static __device__ __align__(256) unsigned char g_sort_scratch[kStaticSortScratchBytes];
 
 Workspace plan_sort_scratch(const Problem &p, char *base, size_t *bytes)
@@ -201,21 +200,13 @@ Workspace plan_sort_scratch(const Problem &p, char *base, size_t *bytes)
 
 cudaError_t static_sort_scratch(void **ptr)
 {
-    constexpr int kMaxDevices = 64;
-    static std::mutex mu;
-    static void *addr[kMaxDevices] = {};
-    int dev = -1;
-    cudaError_t e = cudaGetDevice(&dev);
+    // Looked up on every call, on the current device and context: the address
+    // is not cached, so a device reset (which reloads the module) or another
+    // current context never leaves a stale pointer.
+    void *a = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&a, g_sort_scratch);
     if (e != cudaSuccess) return e;
-    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-    std::lock_guard<std::mutex> lock(mu);
-    if (!addr[dev]) {
-        void *a = nullptr;
-        e = cudaGetSymbolAddress(&a, g_sort_scratch);
-        if (e != cudaSuccess) return e;
-        addr[dev] = a;
-    }
-    *ptr = addr[dev];
+    *ptr = a;
     return cudaSuccess;
 }
 

@@ -251,6 +251,17 @@ __device__ __forceinline__ void mma_commit(uint64_t *bar)
                  : "memory");
 }
 
+// Timeout path of an MMA-issuing thread: waits (bounded, ~1M cycles) until
+// every tcgen05.mma it issued has completed, so that no product still writes
+// tensor memory when the CTA releases it.  `drain_bar` is a barrier of count 1
+// used for nothing else.
+__device__ __forceinline__ void mma_drain(uint64_t *drain_bar, uint32_t *status)
+{
+    mma_commit(drain_bar);
+    int stop = 0;
+    mbar_wait(drain_bar, 0, &stop, status, 1000000);
+}
+
 // Each thread of the warp reads 16 consecutive 32-bit columns of its own lane.
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float *v)
 {

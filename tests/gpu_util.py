@@ -66,12 +66,12 @@ def check_perm_is_stable_sort(perm: np.ndarray, buckets: np.ndarray, what: str):
 class Run:
     """One forward (and optionally backward) through the C ABI, as the benchmark calls it."""
 
-    def __init__(self, inp: dict, n_buckets: int, chunk: int, causal: bool, dtype: str, impl=lsh.IMPL_AUTO):
+    def __init__(self, inp: dict, n_buckets: int, chunk: int, causal: bool, dtype: str, flags: int = 0):
         self.dtype = dtype
         self.x = to_dev(inp["x"], dtype)
         self.v = to_dev(inp["v"], dtype)
         self.R = to_dev(inp["R"], dtype)
-        self.desc = lsh.desc_for(self.x, n_buckets, inp["R"].shape[0], chunk, causal, impl)
+        self.desc = lsh.desc_for(self.x, n_buckets, inp["R"].shape[0], chunk, causal, flags)
         self.out, self.lse, self.perm = lsh.outputs_like(self.desc, self.x)
         self.ws = lsh.workspace(self.desc, False, self.x.device)
         lsh.lsh_attn_fwd(self.desc, self.x, self.v, self.R, self.out, self.lse, self.perm, self.ws)

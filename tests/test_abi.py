@@ -52,15 +52,15 @@ def test_status_strings(lib):
 
 def _desc(**kw):
     base = dict(B=1, H=2, L=1024, d=64, n_buckets=16, n_hashes=2, chunk=64, causal=0, dtype=lsh.LSH_BF16,
-                impl=lsh.IMPL_AUTO)
+                flags=0)
     base.update(kw)
     return lsh.Desc(*[base[k] for k in ("B", "H", "L", "d", "n_buckets", "n_hashes", "chunk", "causal", "dtype",
-                                        "impl")])
+                                        "flags")])
 
 
 @pytest.mark.parametrize("kw,want", [
     (dict(d=32), -4), (dict(L=1000), -2), (dict(n_buckets=15), -2), (dict(n_buckets=0), -2),
-    (dict(n_hashes=0), -2), (dict(chunk=0), -2), (dict(dtype=7), -1), (dict(impl=9), -1), (dict(causal=2), -1),
+    (dict(n_hashes=0), -2), (dict(chunk=0), -2), (dict(dtype=7), -1), (dict(flags=4), -1), (dict(causal=2), -1),
     (dict(B=0), -2), (dict(n_buckets=131072), -2),
 ])
 def test_invalid_descriptors_rejected(lib, kw, want):
@@ -94,10 +94,27 @@ def test_workspace_grows_with_problem(lib):
     small = lib.lsh_attn_workspace_size(ctypes.byref(_desc()), 1)
     big = lib.lsh_attn_workspace_size(ctypes.byref(_desc(L=4096)), 1)
     assert 0 < small < big
-    # forcing the CUDA-core path is always possible; fwd and bwd sizes are both positive
-    for impl in (lsh.IMPL_AUTO, lsh.IMPL_SIMT):
+    # fwd and bwd sizes are positive for both element types
+    for dtype in (lsh.LSH_F32, lsh.LSH_BF16):
         for bwd in (0, 1):
-            assert lib.lsh_attn_workspace_size(ctypes.byref(_desc(impl=impl)), bwd) > 0
+            assert lib.lsh_attn_workspace_size(ctypes.byref(_desc(dtype=dtype)), bwd) > 0
+
+
+@pytest.mark.parametrize("kw", [dict(chunk=32), dict(chunk=128), dict(chunk=1, L=96), dict(B=1, H=1, L=64)])
+def test_bf16_outside_tensor_core_envelope_refused(lib, kw):
+    """bf16 runs on the tensor-core kernels only (chunk 64, L % 64 == 0, at least
+    128 rows): any other bf16 request is refused with LSH_ERR_UNSUPPORTED by every
+    computing entry point before anything is launched (the fake pointers are never
+    dereferenced), while the same shape in fp32 is accepted by the checks."""
+    d = _desc(**kw)
+    fake = ctypes.c_void_p(1 << 20)
+    big = 1 << 40
+    assert lib.lsh_attn_fwd(ctypes.byref(d), fake, fake, fake, fake, fake, None, fake, big, None) == -4
+    assert lib.lsh_attn_fwd_sorted(ctypes.byref(d), fake, fake, fake, fake, fake, fake, big, None) == -4
+    assert lib.lsh_attn_hash(ctypes.byref(d), fake, fake, fake, fake, big, None) == -4
+    assert lib.lsh_attn_bwd(ctypes.byref(d), fake, fake, fake, fake, fake, fake, fake, fake, fake, fake, big,
+                            None) == -4
+    assert lib.lsh_attn_workspace_size(ctypes.byref(_desc(**kw, **{"dtype": lsh.LSH_F32})), 0) > 0
 
 
 def test_trace_end_without_begin_is_an_error(lib):

@@ -1,6 +1,7 @@
 """The C ABI used from plain C (no Python objects, no PyTorch): a program
 linked against the library and the CUDA runtime compiles here; on a GPU it
-runs one fp32 forward and checks it against the CPU oracle."""
+runs one fp32 forward (CUDA-core kernels) and one bf16 forward + backward
+(tensor-core kernels) and checks them against the CPU oracle."""
 import os
 import subprocess
 

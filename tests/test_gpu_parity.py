@@ -20,9 +20,6 @@ from tests.gpu_util import (NEAR_TIE, Run, assert_close, check_buckets, check_pe
 
 pytestmark = pytest.mark.gpu
 
-IMPLS = [lsh.IMPL_SIMT, lsh.IMPL_AUTO]
-
-
 def small(name, **kw):
     return synth.WORKLOADS[name].replace(**kw)
 
@@ -31,11 +28,11 @@ def _flip_report(tag, flips, total):
     print(f"[near-tie] {tag}: {flips} argmax flips out of {total} row-rounds")
 
 
-def full_check(w: synth.Workload, impl=lsh.IMPL_AUTO, heads=None):
+def full_check(w: synth.Workload, heads=None, inp=None):
     """Runs fwd (+bwd) on the GPU for workload w and checks (b, h) slices `heads`
     (all when None) against the oracle."""
-    inp = synth.make_inputs(w)
-    run = Run(inp, w.n_buckets, w.chunk, w.causal, w.dtype, impl)
+    inp = synth.make_inputs(w) if inp is None else inp
+    run = Run(inp, w.n_buckets, w.chunk, w.causal, w.dtype)
     B, H, L = w.B, w.H, w.L
     sel = [(b, h) for b in range(B) for h in range(H)] if heads is None else heads
     gb = run.host_buckets()
@@ -61,14 +58,16 @@ def full_check(w: synth.Workload, impl=lsh.IMPL_AUTO, heads=None):
 
 
 # ------------------------------------------------------------------ stage: hash
-@pytest.mark.parametrize("impl", IMPLS)
 @pytest.mark.parametrize("dtype,nb,nh", [("f32", 16, 1), ("bf16", 64, 2), ("bf16", 1024, 3), ("bf16", 192, 2),
-                                         ("bf16", 128, 2), ("bf16", 2, 2), ("f32", 8192, 1)])
-def test_hash_bit_exact_up_to_near_ties(impl, dtype, nb, nh):
+                                         ("bf16", 128, 2), ("bf16", 2, 2), ("f32", 8192, 1), ("bf16", 8192, 2),
+                                         ("bf16", 6, 2), ("bf16", 100, 1), ("bf16", 200, 2), ("f32", 6, 2)])
+def test_hash_bit_exact_up_to_near_ties(dtype, nb, nh):
+    """Bucket counts whose half is a multiple of 128, 96 or 64 use whole N-tiles;
+    the others (2, 6, 100, 200) pad the last tile with zero rotation columns."""
     w = small("bf16_causal_4k", B=2, H=2, L=1024 if nb < 8192 else 256, n_buckets=nb, n_hashes=nh, dtype=dtype)
     inp = synth.make_inputs(w)
     x = to_dev(inp["x"], dtype); R = to_dev(inp["R"], dtype)
-    desc = lsh.desc_for(x, nb, nh, 64, True, impl)
+    desc = lsh.desc_for(x, nb, nh, 64, True)
     bk = torch.empty((2, 2, nh, w.L), dtype=torch.int16, device="cuda")
     lsh.lsh_attn_hash(desc, x, R, bk)
     gb = bk.cpu().numpy().view(np.uint16).astype(np.int64)
@@ -81,8 +80,7 @@ def test_hash_bit_exact_up_to_near_ties(impl, dtype, nb, nh):
     _flip_report(f"hash {dtype} nb={nb}", flips, 4 * nh * w.L)
 
 
-@pytest.mark.parametrize("impl", IMPLS)
-def test_hash_extreme_magnitudes_and_exact_ties(impl):
+def test_hash_extreme_magnitudes_and_exact_ties():
     """Rows by blocks of 128 (whole warps alike): zero rows, signed one-hot rows
     (the projection is a row of R exactly, so equal bf16 entries make exact ties
     that must go to the lowest index), and Gaussian rows scaled by 2^-110, 2^-60
@@ -116,7 +114,7 @@ def test_hash_extreme_magnitudes_and_exact_ties(impl):
                 x[0, h, i] = -onehot
             exact[h, i] = blk in (0, 1, 5, 7)
     xd = to_dev(x.astype(np.float32), "bf16"); R = to_dev(inp["R"], "bf16")
-    desc = lsh.desc_for(xd, nb, nh, 64, True, impl)
+    desc = lsh.desc_for(xd, nb, nh, 64, True)
     bk = torch.empty((1, 2, nh, L), dtype=torch.int16, device="cuda")
     lsh.lsh_attn_hash(desc, xd, R, bk)
     gb = bk.cpu().numpy().view(np.uint16).astype(np.int64)
@@ -156,18 +154,20 @@ def test_sort_bit_exact(L, nb, dist):
 
 
 # ------------------------------------------------------------------ stage: attention with a given permutation
-@pytest.mark.parametrize("impl", IMPLS)
 @pytest.mark.parametrize("dtype,causal,L,m,nh", [("f32", False, 1024, 64, 1), ("f32", True, 512, 32, 3),
                                                  ("bf16", True, 1024, 64, 2), ("bf16", False, 2048, 64, 4),
                                                  ("bf16", True, 960, 64, 2), ("f32", True, 48, 1, 2),
-                                                 ("bf16", True, 64, 64, 1), ("bf16", False, 128, 128, 2)])
-def test_attention_given_perm(impl, dtype, causal, L, m, nh):
+                                                 ("bf16", True, 64, 64, 1), ("f32", False, 128, 128, 2),
+                                                 ("bf16", False, 576, 64, 3), ("bf16", True, 192, 64, 2)])
+def test_attention_given_perm(dtype, causal, L, m, nh):
+    """L = 960, 576, 192 and 64 leave the last 128-slot tile of the tensor-core
+    kernels with one chunk only."""
     w = small("bf16_causal_4k", B=1, H=3, L=L, n_buckets=16, n_hashes=nh, chunk=m, causal=causal, dtype=dtype)
     inp = synth.make_inputs(w)
     rng = np.random.default_rng(L + nh)
     perm = np.stack([[rng.permutation(L) for _ in range(nh)] for _ in range(3)])[None].astype(np.int32)
     x, v = to_dev(inp["x"], dtype), to_dev(inp["v"], dtype)
-    desc = lsh.desc_for(x, 16, nh, m, causal, impl)
+    desc = lsh.desc_for(x, 16, nh, m, causal)
     out, lse, _ = lsh.outputs_like(desc, x)
     lsh.lsh_attn_fwd_sorted(desc, x, v, torch.from_numpy(perm).cuda(), out, lse)
     y, lr = oracle.fwd_perm(inp["x"], inp["v"], perm, m, causal)
@@ -176,30 +176,47 @@ def test_attention_given_perm(impl, dtype, causal, L, m, nh):
 
 
 # ------------------------------------------------------------------ whole path, small cases
-@pytest.mark.parametrize("impl", IMPLS)
 @pytest.mark.parametrize("dtype,causal,nb,nh,L", [("f32", False, 16, 1, 1024), ("f32", True, 16, 2, 512),
                                                   ("bf16", True, 64, 2, 1024), ("bf16", False, 128, 3, 1152),
                                                   ("bf16", True, 1024, 4, 2048), ("bf16", True, 2, 2, 256),
-                                                  ("bf16", True, 256, 3, 1408)])
-def test_forward_backward_small(impl, dtype, causal, nb, nh, L):
+                                                  ("bf16", True, 256, 3, 1408), ("bf16", True, 64, 2, 960),
+                                                  ("bf16", False, 6, 2, 704), ("f32", True, 6, 2, 320)])
+def test_forward_backward_small(dtype, causal, nb, nh, L):
     w = small("long_64k", B=2, H=2, L=L, n_buckets=nb, n_hashes=nh, causal=causal, dtype=dtype, backward=True)
-    full_check(w, impl)
+    full_check(w)
 
 
-@pytest.mark.parametrize("impl", IMPLS)
-def test_clustered_inputs_small(impl):
+def test_clustered_inputs_small():
     w = small("image_12k", B=1, H=2, L=1536)
-    full_check(w, impl)
+    full_check(w)
 
 
-@pytest.mark.parametrize("impl", IMPLS)
-def test_edge_cases(impl):
+@pytest.mark.parametrize("causal", [True, False])
+def test_wide_rows_forward_backward(causal):
+    """Rows with |x| of 300 to 2000 next to ordinary rows (|x| about 8), so that
+    warps of the forward kernel hold both: for such rows the bound tau |x| on
+    the scores is loose enough that the softmax first finds the exact row
+    maximum.  Outputs and both gradients against the oracle."""
+    w = small("long_64k", B=1, H=2, L=2048, n_buckets=64, n_hashes=2, causal=causal, backward=True)
+    inp = synth.make_inputs(w)
+    rng = np.random.default_rng(11)
+    x = inp["x"].astype(np.float64)
+    wide = rng.random(x.shape[:3]) < 0.4
+    target = rng.uniform(300.0, 2000.0, size=x.shape[:3])
+    scale = np.where(wide, target / np.linalg.norm(x, axis=-1), 1.0)
+    inp["x"] = synth.round_to_bf16((x * scale[..., None]).astype(np.float32))
+    norms = np.linalg.norm(inp["x"].astype(np.float64), axis=-1)
+    assert (norms > 277).mean() > 0.3 and (norms < 20).mean() > 0.3
+    full_check(w, inp=inp)
+
+
+def test_edge_cases():
     """Zero rows (key 0), duplicated rows, causal first token = its own value."""
     w = small("long_64k", B=1, H=2, L=256, n_buckets=8, n_hashes=2, backward=True)
     inp = synth.make_inputs(w)
     inp["x"][0, 0, 5] = 0.0
     inp["x"][0, 1, 10] = inp["x"][0, 1, 11]
-    run = Run(inp, w.n_buckets, w.chunk, True, "bf16", impl)
+    run = Run(inp, w.n_buckets, w.chunk, True, "bf16")
     out = to_host(run.out)
     np.testing.assert_array_equal(out[0, :, 0], inp["v"][0, :, 0])   # causal position 0 sees only itself
     y, _ = oracle.fwd_perm(inp["x"], inp["v"], run.perm.cpu().numpy(), w.chunk, True)
@@ -209,18 +226,77 @@ def test_edge_cases(impl):
     assert_close(to_host(run.dv), dv, "bf16", "dv")
 
 
-def test_paths_agree():
-    """The tensor-core and CUDA-core paths give the same buckets and permutation
-    (when no near tie separates them) and outputs within the bf16 bound."""
-    w = small("long_64k", B=1, H=2, L=2048, backward=True)
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_backward_recomputes_permutation_when_not_given(dtype):
+    """lsh_attn_bwd with perm = NULL hashes and sorts again from qk and R in its
+    own workspace: the gradients match the oracle and the perm-given call."""
+    w = small("long_64k", B=1, H=2, L=1024, n_buckets=64, n_hashes=2, causal=True, dtype=dtype, backward=True)
     inp = synth.make_inputs(w)
-    a = Run(inp, w.n_buckets, w.chunk, True, "bf16", lsh.IMPL_SIMT)
-    b = Run(inp, w.n_buckets, w.chunk, True, "bf16", lsh.IMPL_AUTO)
-    diff = (a.host_buckets() != b.host_buckets()).sum()
-    assert diff <= 4
-    if diff == 0:
-        assert torch.equal(a.perm, b.perm)
-        assert_close(to_host(b.out), to_host(a.out), "bf16", "out")
+    run = Run(inp, w.n_buckets, w.chunk, w.causal, w.dtype)
+    dx = torch.empty_like(run.x); dv = torch.empty_like(run.v)
+    wsb = lsh.workspace(run.desc, True, run.x.device)
+    lsh.lsh_attn_bwd(run.desc, run.x, run.v, run.R, run.out, run.lse, None, run.dy, dx, dv, wsb)
+    assert lsh.lsh_attn_poll(wsb) == 0
+    assert_close(to_host(dx), to_host(run.dx), dtype, "dqk recomputed vs given perm")
+    assert_close(to_host(dv), to_host(run.dv), dtype, "dv recomputed vs given perm")
+    gperm = run.perm.cpu().numpy()
+    odx, odv = oracle.bwd(inp["x"], inp["v"], inp["dy"], gperm, w.chunk, w.causal)
+    assert_close(to_host(dx), odx, dtype, "dqk recomputed vs oracle")
+    assert_close(to_host(dv), odv, dtype, "dv recomputed vs oracle")
+
+
+@pytest.mark.parametrize("dtype,L", [("bf16", 1024), ("bf16", 960), ("f32", 512)])
+def test_permutation_entries_out_of_range_are_reported(dtype, L):
+    """A permutation entry outside [0, L) is treated as an empty slot by the
+    forward and backward kernels (nothing is read or written at it) and
+    lsh_attn_poll reports LSH_ERR_ARG; every other output stays finite and the
+    next call with a valid permutation is exact again."""
+    nh = 2
+    w = small("long_64k", B=1, H=2, L=L, n_buckets=64, n_hashes=nh, causal=True, dtype=dtype, backward=True)
+    inp = synth.make_inputs(w)
+    rng = np.random.default_rng(3)
+    perm = np.stack([[rng.permutation(L) for _ in range(nh)] for _ in range(2)])[None].astype(np.int32)
+    bad = perm.copy()
+    lost = {(0, 1, bad[0, 0, 1, 5]), (1, 0, bad[0, 1, 0, 70])}
+    bad[0, 0, 1, 5] = L + 3
+    bad[0, 1, 0, 70] = -7
+    x, v, dy = to_dev(inp["x"], dtype), to_dev(inp["v"], dtype), to_dev(inp["dy"], dtype)
+    desc = lsh.desc_for(x, w.n_buckets, nh, w.chunk, w.causal)
+    out, lse, _ = lsh.outputs_like(desc, x)
+    lse.fill_(0.0)
+    out.zero_()
+    ws = lsh.workspace(desc, False, x.device)
+    lsh.lsh_attn_fwd_sorted(desc, x, v, torch.from_numpy(bad).cuda(), out, lse, ws)
+    assert lsh.lsh_attn_poll(ws) == -1                   # LSH_ERR_ARG
+    lse_h = lse.cpu().numpy()
+    for h, r, pos in lost:
+        lse_h[0, h, r, pos] = 0.0                        # never written
+    assert np.isfinite(lse_h).all()
+    dx = torch.empty_like(x); dvv = torch.empty_like(v)
+    wsb = lsh.workspace(desc, True, x.device)
+    lsh.lsh_attn_bwd(desc, x, v, None, out, lse, torch.from_numpy(bad).cuda(), dy, dx, dvv, wsb)
+    assert lsh.lsh_attn_poll(wsb) == -1
+    lsh.lsh_attn_fwd_sorted(desc, x, v, torch.from_numpy(perm).cuda(), out, lse, ws)
+    assert lsh.lsh_attn_poll(ws) == 0
+    y, lr = oracle.fwd_perm(inp["x"], inp["v"], perm, w.chunk, w.causal)
+    assert_close(to_host(out), y, dtype, "out after a bad call")
+
+
+def test_backward_run_to_run_drift_is_one_rounding_step():
+    """The backward adds every round's gradient rows into fp32 accumulators with
+    atomic vector reductions, so their summation order is not fixed.  Two runs on
+    the same inputs may differ only by the final rounding: elementwise at most
+    one bf16 step (2^-7 of the larger magnitude)."""
+    w = small("long_64k", B=1, H=2, L=8192, backward=True)
+    inp = synth.make_inputs(w)
+    a = Run(inp, w.n_buckets, w.chunk, w.causal, w.dtype)
+    b = Run(inp, w.n_buckets, w.chunk, w.causal, w.dtype)
+    assert torch.equal(a.perm, b.perm) and torch.equal(a.out, b.out)
+    for name, u, t in [("dqk", a.dx, b.dx), ("dv", a.dv, b.dv)]:
+        u, t = to_host(u), to_host(t)
+        bound = 2.0 ** -7 * np.maximum(np.abs(u), np.abs(t))
+        assert (np.abs(u - t) <= bound).all(), name
+        print(f"[drift] {name}: {(u != t).mean():.2e} of elements differ between two runs")
 
 
 # ------------------------------------------------------------------ the five workloads
