@@ -38,6 +38,16 @@
  *   backward      gradients w.r.t. x (query role, key role through the
  *                 normalisation) and v; buckets and permutation held fixed.
  *
+ * Two optional readings, each switched on by an argument:
+ *   bucket mask   the strict candidate set N_LSH(i) = {j : h(q_i) = h(k_j)}
+ *                 of [CAND]: inside the window only keys in the query's
+ *                 bucket (of that round) are candidates;
+ *   self penalty  the other answer to the same-token question of [MASK]:
+ *                 the query's own position is always a candidate, with the
+ *                 fixed score ORACLE_SELF_PENALTY instead of q.k/sqrt(d), so
+ *                 it matters only when nothing else is left (its score does
+ *                 not depend on x, so it passes no gradient to x).
+ *
  * Parity pins: see the oracle tests (dense special case, softmax sums,
  * stable order, identical rounds, finite differences, brute-force
  * candidate enumeration, two-bucket sign hash).
@@ -51,6 +61,10 @@
 #endif
 
 #define ORACLE_EXPORT __attribute__((visibility("default")))
+
+/* Score of the query's own position in the self-penalty reading (natural-log
+ * units, the same scale as q.k/sqrt(d)). */
+#define ORACLE_SELF_PENALTY (-1.0e5)
 
 /* ------------------------------------------------------------------ */
 /* [HASH] one hash round for n rows: bucket = argmax [x.R ; -x.R].      */
@@ -124,8 +138,13 @@ static void normalise_keys(const double *x, long L, int d, double *khat, double 
 
 /* [CAND] + [SORT] + [MASK]: the candidate positions of sorted slot s.
  * Window: slots of chunk c = s / m and of chunk c - 1 (if c > 0).
- * Returns the number of candidates written to cand (self alone if none). */
-static long candidates(const int32_t *perm, long L, int m, int causal, long s, int32_t *cand)
+ * bucket (nullable): bucket id of every position in this round; when given,
+ * only keys in the query's bucket are candidates.  Returns the number of
+ * candidates written to cand; *self_in = 1 when the query's own position is
+ * among them (then it is the last entry): always in the self-penalty reading,
+ * else only when nothing else is left. */
+static long candidates(const int32_t *perm, long L, int m, int causal, const int32_t *bucket, int self_penalty,
+                       long s, int32_t *cand, int *self_in)
 {
     long c = s / m;
     long w0 = c > 0 ? (c - 1) * m : 0;
@@ -137,9 +156,14 @@ static long candidates(const int32_t *perm, long L, int m, int causal, long s, i
         if (t == s) continue;                    /* self removed ... */
         int32_t j = perm[t];
         if (causal && j > i) continue;           /* causal on original positions */
+        if (bucket && bucket[j] != bucket[i]) continue;   /* strict N_LSH */
         cand[nc++] = j;
     }
-    if (nc == 0) cand[nc++] = i;                 /* ... unless it is the only candidate */
+    *self_in = 0;
+    if (self_penalty || nc == 0) {               /* ... unless it is the only candidate */
+        cand[nc++] = i;
+        *self_in = 1;
+    }
     return nc;
 }
 
@@ -147,7 +171,7 @@ static long candidates(const int32_t *perm, long L, int m, int causal, long s, i
  * (all slots when slots == NULL).  Writes o and lse at the ORIGINAL
  * position of each query when scatter != 0, else at the list index. */
 static int attn_round_impl(const double *x, const double *v, long L, int d,
-                           const int32_t *perm, int m, int causal,
+                           const int32_t *perm, int m, int causal, const int32_t *bucket, int self_penalty,
                            const int64_t *slots, long nslots, int scatter,
                            double *o, double *lse)
 {
@@ -162,12 +186,13 @@ static int attn_round_impl(const double *x, const double *v, long L, int d,
     for (long q = 0; q < count; ++q) {
         long s = slots ? (long)slots[q] : q;
         int32_t i = perm[s];
-        long nc = candidates(perm, L, m, causal, s, cand);
+        int self_in;
+        long nc = candidates(perm, L, m, causal, bucket, self_penalty, s, cand, &self_in);
         double zmax = -INFINITY;
         for (long a = 0; a < nc; ++a) {
             double dot = 0.0;
             for (int t = 0; t < d; ++t) dot += x[(size_t)i * d + t] * khat[(size_t)cand[a] * d + t];
-            z[a] = tau * dot;
+            z[a] = (self_penalty && self_in && a == nc - 1) ? ORACLE_SELF_PENALTY : tau * dot;
             if (z[a] > zmax) zmax = z[a];
         }
         double l = 0.0;
@@ -187,19 +212,19 @@ static int attn_round_impl(const double *x, const double *v, long L, int d,
 }
 
 ORACLE_EXPORT int oracle_attn_round(const double *x, const double *v, long L, int d,
-                                    const int32_t *perm, int m, int causal,
-                                    double *o, double *lse)
+                                    const int32_t *perm, int m, int causal, const int32_t *bucket,
+                                    int self_penalty, double *o, double *lse)
 {
-    return attn_round_impl(x, v, L, d, perm, m, causal, NULL, L, 1, o, lse);
+    return attn_round_impl(x, v, L, d, perm, m, causal, bucket, self_penalty, NULL, L, 1, o, lse);
 }
 
 /* Same as oracle_attn_round for a list of sorted slots; outputs follow the list. */
 ORACLE_EXPORT int oracle_attn_slots(const double *x, const double *v, long L, int d,
-                                    const int32_t *perm, int m, int causal,
-                                    const int64_t *slots, long nslots,
+                                    const int32_t *perm, int m, int causal, const int32_t *bucket,
+                                    int self_penalty, const int64_t *slots, long nslots,
                                     double *o, double *lse)
 {
-    return attn_round_impl(x, v, L, d, perm, m, causal, slots, nslots, 0, o, lse);
+    return attn_round_impl(x, v, L, d, perm, m, causal, bucket, self_penalty, slots, nslots, 0, o, lse);
 }
 
 /* [ROUNDS] y_i = sum_r softmax_r(lse_r,i) o_r,i; also returns LSE_i = logsumexp_r lse_r,i. */
@@ -224,9 +249,11 @@ ORACLE_EXPORT int oracle_combine(const double *o, const double *lse, int R, long
 
 /* Whole forward for one (batch, head): hash every round, sort, attend, combine.
  * x, v [L, d]; R [n_hashes, d, n_buckets/2]; outputs y [L, d], lse [n_hashes, L],
- * perm [n_hashes, L], bucket [n_hashes, L], margin [n_hashes, L] (nullable). */
+ * perm [n_hashes, L], bucket [n_hashes, L], margin [n_hashes, L] (nullable).
+ * bucket_mask / self_penalty: the optional readings (see the top of the file). */
 ORACLE_EXPORT int oracle_fwd_head(const double *x, const double *v, long L, int d,
                                   const double *R, int n_buckets, int n_hashes, int m, int causal,
+                                  int bucket_mask, int self_penalty,
                                   double *y, double *lse, int32_t *perm, int32_t *bucket, double *margin)
 {
     const int half = n_buckets / 2;
@@ -238,6 +265,7 @@ ORACLE_EXPORT int oracle_fwd_head(const double *x, const double *v, long L, int 
                           margin ? margin + (size_t)r * L : NULL);
         rc |= oracle_sort(bucket + (size_t)r * L, L, perm + (size_t)r * L);
         rc |= oracle_attn_round(x, v, L, d, perm + (size_t)r * L, m, causal,
+                                bucket_mask ? bucket + (size_t)r * L : NULL, self_penalty,
                                 o + (size_t)r * L * d, lse + (size_t)r * L);
     }
     if (rc == 0) rc = oracle_combine(o, lse, n_hashes, L, d, y, NULL);
@@ -245,16 +273,18 @@ ORACLE_EXPORT int oracle_fwd_head(const double *x, const double *v, long L, int 
     return rc;
 }
 
-/* Forward with given permutations (one per round); same outputs minus hashing. */
+/* Forward with given permutations (one per round); same outputs minus hashing.
+ * bucket (nullable, [n_hashes, L] by position): given -> the bucket mask. */
 ORACLE_EXPORT int oracle_fwd_head_perm(const double *x, const double *v, long L, int d,
                                        const int32_t *perm, int n_hashes, int m, int causal,
-                                       double *y, double *lse)
+                                       const int32_t *bucket, int self_penalty, double *y, double *lse)
 {
     double *o = (double *)malloc(sizeof(double) * (size_t)n_hashes * L * d);
     if (!o) return -1;
     int rc = 0;
     for (int r = 0; r < n_hashes && rc == 0; ++r)
         rc |= oracle_attn_round(x, v, L, d, perm + (size_t)r * L, m, causal,
+                                bucket ? bucket + (size_t)r * L : NULL, self_penalty,
                                 o + (size_t)r * L * d, lse + (size_t)r * L);
     if (rc == 0) rc = oracle_combine(o, lse, n_hashes, L, d, y, NULL);
     free(o);
@@ -271,10 +301,12 @@ ORACLE_EXPORT int oracle_fwd_head_perm(const double *x, const double *v, long L,
  *   dx_i      += dz_rij / sqrt(d) * k_j                 (query role)
  *   dk_j      += dz_rij / sqrt(d) * x_i                 (key role)
  *   dx_j      += (dk_j - k_j (k_j . dk_j)) / |x_j|      (through k_j = x_j/|x_j|)
- * Accumulated in a fixed order (round, slot, candidate). */
+ * Accumulated in a fixed order (round, slot, candidate).  In the self-penalty
+ * reading the query's own entry has a constant score: it adds P G_i to dv_i
+ * and nothing to dx.  bucket (nullable, [n_hashes, L]): given -> bucket mask. */
 ORACLE_EXPORT int oracle_bwd_head(const double *x, const double *v, const double *dy, long L, int d,
                                   const int32_t *perm, int n_hashes, int m, int causal,
-                                  double *dx, double *dv)
+                                  const int32_t *bucket, int self_penalty, double *dx, double *dv)
 {
     double *y = (double *)malloc(sizeof(double) * (size_t)L * d);
     double *lse = (double *)malloc(sizeof(double) * (size_t)n_hashes * L);
@@ -289,6 +321,7 @@ ORACLE_EXPORT int oracle_bwd_head(const double *x, const double *v, const double
     rc = 0;
     for (int r = 0; r < n_hashes && rc == 0; ++r)
         rc |= oracle_attn_round(x, v, L, d, perm + (size_t)r * L, m, causal,
+                                bucket ? bucket + (size_t)r * L : NULL, self_penalty,
                                 o + (size_t)r * L * d, lse + (size_t)r * L);
     if (rc) goto done;
     oracle_combine(o, lse, n_hashes, L, d, y, big);
@@ -303,12 +336,20 @@ ORACLE_EXPORT int oracle_bwd_head(const double *x, const double *v, const double
             const double *xi = x + (size_t)i * d, *gi = dy + (size_t)i * d;
             double delta = 0.0;
             for (int t = 0; t < d; ++t) delta += gi[t] * y[(size_t)i * d + t];
-            long nc = candidates(pr, L, m, causal, s, cand);
+            int self_in;
+            long nc = candidates(pr, L, m, causal, bucket ? bucket + (size_t)r * L : NULL, self_penalty, s, cand,
+                                 &self_in);
             for (long a = 0; a < nc; ++a) {
                 int32_t j = cand[a];
                 const double *kj = khat + (size_t)j * d, *vj = v + (size_t)j * d;
                 double dot = 0.0, gv = 0.0;
                 for (int t = 0; t < d; ++t) { dot += xi[t] * kj[t]; gv += gi[t] * vj[t]; }
+                if (self_penalty && self_in && a == nc - 1) {
+                    /* constant score: value path only */
+                    double p = exp(ORACLE_SELF_PENALTY - big[i]);
+                    for (int t = 0; t < d; ++t) dv[(size_t)j * d + t] += p * gi[t];
+                    continue;
+                }
                 double p = exp(tau * dot - big[i]);
                 double dz = p * (gv - delta);
                 for (int t = 0; t < d; ++t) {
@@ -338,43 +379,46 @@ done:
 /* ------------------------------------------------------------------ */
 ORACLE_EXPORT int oracle_fwd_batch(const double *x, const double *v, long BH, long L, int d,
                                    const double *R, int n_buckets, int n_hashes, int m, int causal,
+                                   int bucket_mask, int self_penalty,
                                    double *y, double *lse, int32_t *perm, int32_t *bucket, double *margin)
 {
     int rc = 0;
 #pragma omp parallel for schedule(dynamic, 1) reduction(| : rc)
     for (long h = 0; h < BH; ++h) {
         size_t rows = (size_t)h * L, segs = (size_t)h * n_hashes * L;
-        rc |= oracle_fwd_head(x + rows * d, v + rows * d, L, d, R, n_buckets, n_hashes, m, causal,
-                              y + rows * d, lse + segs, perm + segs, bucket + segs,
+        rc |= oracle_fwd_head(x + rows * d, v + rows * d, L, d, R, n_buckets, n_hashes, m, causal, bucket_mask,
+                              self_penalty, y + rows * d, lse + segs, perm + segs, bucket + segs,
                               margin ? margin + segs : NULL);
     }
     return rc;
 }
 
+/* bucket (nullable) [BH, n_hashes, L] by position: given -> the bucket mask. */
 ORACLE_EXPORT int oracle_fwd_perm_batch(const double *x, const double *v, long BH, long L, int d,
                                         const int32_t *perm, int n_hashes, int m, int causal,
-                                        double *y, double *lse)
+                                        const int32_t *bucket, int self_penalty, double *y, double *lse)
 {
     int rc = 0;
 #pragma omp parallel for schedule(dynamic, 1) reduction(| : rc)
     for (long h = 0; h < BH; ++h) {
         size_t rows = (size_t)h * L, segs = (size_t)h * n_hashes * L;
         rc |= oracle_fwd_head_perm(x + rows * d, v + rows * d, L, d, perm + segs, n_hashes, m, causal,
-                                   y + rows * d, lse + segs);
+                                   bucket ? bucket + segs : NULL, self_penalty, y + rows * d, lse + segs);
     }
     return rc;
 }
 
 ORACLE_EXPORT int oracle_bwd_batch(const double *x, const double *v, const double *dy, long BH, long L,
                                    int d, const int32_t *perm, int n_hashes, int m, int causal,
-                                   double *dx, double *dv)
+                                   const int32_t *bucket, int self_penalty, double *dx, double *dv)
 {
     int rc = 0;
 #pragma omp parallel for schedule(dynamic, 1) reduction(| : rc)
     for (long h = 0; h < BH; ++h) {
         size_t rows = (size_t)h * L, segs = (size_t)h * n_hashes * L;
         rc |= oracle_bwd_head(x + rows * d, v + rows * d, dy + rows * d, L, d, perm + segs, n_hashes,
-                              m, causal, dx + rows * d, dv + rows * d);
+                              m, causal, bucket ? bucket + segs : NULL, self_penalty, dx + rows * d,
+                              dv + rows * d);
     }
     return rc;
 }

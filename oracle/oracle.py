@@ -41,14 +41,14 @@ def lib():
         L = ctypes.CDLL(_LIB)
         L.oracle_hash.argtypes = [_D, _L, _C, _D, _C, _I32, _D]
         L.oracle_sort.argtypes = [_I32, _L, _I32]
-        L.oracle_attn_round.argtypes = [_D, _D, _L, _C, _I32, _C, _C, _D, _D]
-        L.oracle_attn_slots.argtypes = [_D, _D, _L, _C, _I32, _C, _C, _I64, _L, _D, _D]
+        L.oracle_attn_round.argtypes = [_D, _D, _L, _C, _I32, _C, _C, _I32, _C, _D, _D]
+        L.oracle_attn_slots.argtypes = [_D, _D, _L, _C, _I32, _C, _C, _I32, _C, _I64, _L, _D, _D]
         L.oracle_combine.argtypes = [_D, _D, _C, _L, _C, _D, _D]
-        L.oracle_fwd_head.argtypes = [_D, _D, _L, _C, _D, _C, _C, _C, _C, _D, _D, _I32, _I32, _D]
-        L.oracle_bwd_head.argtypes = [_D, _D, _D, _L, _C, _I32, _C, _C, _C, _D, _D]
-        L.oracle_fwd_batch.argtypes = [_D, _D, _L, _L, _C, _D, _C, _C, _C, _C, _D, _D, _I32, _I32, _D]
-        L.oracle_fwd_perm_batch.argtypes = [_D, _D, _L, _L, _C, _I32, _C, _C, _C, _D, _D]
-        L.oracle_bwd_batch.argtypes = [_D, _D, _D, _L, _L, _C, _I32, _C, _C, _C, _D, _D]
+        L.oracle_fwd_head.argtypes = [_D, _D, _L, _C, _D, _C, _C, _C, _C, _C, _C, _D, _D, _I32, _I32, _D]
+        L.oracle_bwd_head.argtypes = [_D, _D, _D, _L, _C, _I32, _C, _C, _C, _I32, _C, _D, _D]
+        L.oracle_fwd_batch.argtypes = [_D, _D, _L, _L, _C, _D, _C, _C, _C, _C, _C, _C, _D, _D, _I32, _I32, _D]
+        L.oracle_fwd_perm_batch.argtypes = [_D, _D, _L, _L, _C, _I32, _C, _C, _C, _I32, _C, _D, _D]
+        L.oracle_bwd_batch.argtypes = [_D, _D, _D, _L, _L, _C, _I32, _C, _C, _C, _I32, _C, _D, _D]
         L.oracle_max_threads.argtypes = []
         _lib = L
     return _lib
@@ -60,6 +60,15 @@ def _d(a):
 
 def _p(a, t):
     return a.ctypes.data_as(t)
+
+
+def _bucket(bucket, shape):
+    """Optional bucket ids by position (the bucket-mask reading): int32 array or None."""
+    if bucket is None:
+        return None, None
+    b = np.ascontiguousarray(bucket, dtype=np.int32)
+    assert b.shape == tuple(shape), (b.shape, shape)
+    return b, _p(b, _I32)
 
 
 def _check(rc):
@@ -88,24 +97,28 @@ def sort_segment(bucket):
     return perm
 
 
-def attn_round(x, v, perm, chunk, causal):
-    """One round: o [L, d] and lse [L] in original order."""
+def attn_round(x, v, perm, chunk, causal, bucket=None, self_penalty=False):
+    """One round: o [L, d] and lse [L] in original order.  bucket [L] (by
+    position) switches on the bucket mask; self_penalty the penalty reading."""
     x = _d(x); v = _d(v); perm = np.ascontiguousarray(perm, dtype=np.int32)
     L, d = x.shape
+    b, bp = _bucket(bucket, (L,))
     o = np.empty((L, d)); lse = np.empty(L)
     _check(lib().oracle_attn_round(_p(x, _D), _p(v, _D), L, d, _p(perm, _I32), int(chunk), int(causal),
-                                   _p(o, _D), _p(lse, _D)))
+                                   bp, int(bool(self_penalty)), _p(o, _D), _p(lse, _D)))
     return o, lse
 
 
-def attn_slots(x, v, perm, chunk, causal, slots):
+def attn_slots(x, v, perm, chunk, causal, slots, bucket=None, self_penalty=False):
     """One round for selected sorted slots: o [n, d], lse [n] in list order."""
     x = _d(x); v = _d(v); perm = np.ascontiguousarray(perm, dtype=np.int32)
     slots = np.ascontiguousarray(slots, dtype=np.int64)
     L, d = x.shape
+    b, bp = _bucket(bucket, (L,))
     o = np.empty((slots.size, d)); lse = np.empty(slots.size)
     _check(lib().oracle_attn_slots(_p(x, _D), _p(v, _D), L, d, _p(perm, _I32), int(chunk), int(causal),
-                                   _p(slots, _I64), slots.size, _p(o, _D), _p(lse, _D)))
+                                   bp, int(bool(self_penalty)), _p(slots, _I64), slots.size, _p(o, _D),
+                                   _p(lse, _D)))
     return o, lse
 
 
@@ -118,7 +131,7 @@ def combine(o, lse):
     return y, big
 
 
-def fwd(x, v, R, n_buckets, chunk, causal):
+def fwd(x, v, R, n_buckets, chunk, causal, bucket_mask=False, self_penalty=False):
     """Full forward on [B, H, L, d] inputs with rotations R [n_hashes, d, n_buckets/2].
 
     Returns dict with y [B,H,L,d], lse/perm/bucket/margin [B,H,n_hashes,L]."""
@@ -129,28 +142,33 @@ def fwd(x, v, R, n_buckets, chunk, causal):
     lse = np.empty((B, H, nh, L)); mg = np.empty((B, H, nh, L))
     perm = np.empty((B, H, nh, L), np.int32); bk = np.empty((B, H, nh, L), np.int32)
     _check(lib().oracle_fwd_batch(_p(x, _D), _p(v, _D), B * H, L, d, _p(R, _D), int(n_buckets), nh,
-                                  int(chunk), int(causal), _p(y, _D), _p(lse, _D), _p(perm, _I32),
+                                  int(chunk), int(causal), int(bool(bucket_mask)), int(bool(self_penalty)),
+                                  _p(y, _D), _p(lse, _D), _p(perm, _I32),
                                   _p(bk, _I32), _p(mg, _D)))
     return {"y": y, "lse": lse, "perm": perm, "bucket": bk, "margin": mg}
 
 
-def fwd_perm(x, v, perm, chunk, causal):
-    """Forward with given permutations perm [B,H,n_hashes,L]: y [B,H,L,d], lse [B,H,n_hashes,L]."""
+def fwd_perm(x, v, perm, chunk, causal, bucket=None, self_penalty=False):
+    """Forward with given permutations perm [B,H,n_hashes,L]: y [B,H,L,d], lse [B,H,n_hashes,L].
+    bucket [B,H,n_hashes,L] (by position) switches on the bucket mask."""
     x = _d(x); v = _d(v); perm = np.ascontiguousarray(perm, dtype=np.int32)
     B, H, L, d = x.shape
     nh = perm.shape[2]
+    b, bp = _bucket(bucket, perm.shape)
     y = np.empty_like(x); lse = np.empty((B, H, nh, L))
     _check(lib().oracle_fwd_perm_batch(_p(x, _D), _p(v, _D), B * H, L, d, _p(perm, _I32), nh,
-                                       int(chunk), int(causal), _p(y, _D), _p(lse, _D)))
+                                       int(chunk), int(causal), bp, int(bool(self_penalty)), _p(y, _D),
+                                       _p(lse, _D)))
     return y, lse
 
 
-def bwd(x, v, dy, perm, chunk, causal):
+def bwd(x, v, dy, perm, chunk, causal, bucket=None, self_penalty=False):
     """Gradients (dx, dv) [B,H,L,d] of sum(y * dy) with permutations perm [B,H,n_hashes,L]."""
     x = _d(x); v = _d(v); dy = _d(dy); perm = np.ascontiguousarray(perm, dtype=np.int32)
     B, H, L, d = x.shape
     nh = perm.shape[2]
+    b, bp = _bucket(bucket, perm.shape)
     dx = np.empty_like(x); dv = np.empty_like(x)
     _check(lib().oracle_bwd_batch(_p(x, _D), _p(v, _D), _p(dy, _D), B * H, L, d, _p(perm, _I32), nh,
-                                  int(chunk), int(causal), _p(dx, _D), _p(dv, _D)))
+                                  int(chunk), int(causal), bp, int(bool(self_penalty)), _p(dx, _D), _p(dv, _D)))
     return dx, dv

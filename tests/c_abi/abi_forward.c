@@ -16,9 +16,10 @@
 
 /* test infrastructure: the oracle's forward for one (batch, head) */
 int oracle_fwd_head_perm(const double *x, const double *v, long L, int d, const int32_t *perm, int n_hashes, int m,
-                         int causal, double *y, double *lse);
+                         int causal, const int32_t *bucket, int self_penalty, double *y, double *lse);
 int oracle_bwd_head(const double *x, const double *v, const double *dy, long L, int d, const int32_t *perm,
-                    int n_hashes, int m, int causal, double *dx, double *dv);
+                    int n_hashes, int m, int causal, const int32_t *bucket, int self_penalty, double *dx,
+                    double *dv);
 
 /* float -> bfloat16 bits, round to nearest even (finite inputs), and back */
 static uint16_t to_bf16(float f)
@@ -103,7 +104,7 @@ static int run_f32(void)
             xd[i] = x[(size_t)bh * L * d + i];
             vd[i] = v[(size_t)bh * L * d + i];
         }
-        CHECK(oracle_fwd_head_perm(xd, vd, L, d, perm + (size_t)bh * nh * L, nh, m, causal, yd, ld));
+        CHECK(oracle_fwd_head_perm(xd, vd, L, d, perm + (size_t)bh * nh * L, nh, m, causal, NULL, 0, yd, ld));
         for (size_t i = 0; i < (size_t)L * d; ++i) err = fmax(err, fabs(yd[i] - out[(size_t)bh * L * d + i]));
         for (size_t i = 0; i < (size_t)nh * L; ++i) lerr = fmax(lerr, fabs(ld[i] - lse[(size_t)bh * nh * L + i]));
     }
@@ -178,8 +179,8 @@ static int run_bf16(void)
             gd[i] = from_bf16(g[bh * hd + i]);
         }
         const int32_t *pb = perm + (size_t)bh * nh * L;
-        CHECK(oracle_fwd_head_perm(xd, vd, L, d, pb, nh, m, causal, yd, ld));
-        CHECK(oracle_bwd_head(xd, vd, gd, L, d, pb, nh, m, causal, dxd, dvd));
+        CHECK(oracle_fwd_head_perm(xd, vd, L, d, pb, nh, m, causal, NULL, 0, yd, ld));
+        CHECK(oracle_bwd_head(xd, vd, gd, L, d, pb, nh, m, causal, NULL, 0, dxd, dvd));
         bf16_errors(out + bh * hd, yd, hd, &e_out, &n_out, &s_out);
         bf16_errors(dqk + bh * hd, dxd, hd, &e_dx, &n_dx, &s_dx);
         bf16_errors(dv + bh * hd, dvd, hd, &e_dv, &n_dv, &s_dv);
