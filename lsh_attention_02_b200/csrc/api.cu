@@ -109,7 +109,6 @@ static lsh_status check_desc(const lsh_attn_desc *d, Problem *p)
 // do not cover is refused (the sort alone does not depend on the dtype).
 static lsh_status check_envelope(const Problem &p)
 {
-    if (p.flags != 0) return LSH_ERR_UNSUPPORTED;      // optional semantics: not built yet
     if (p.dtype == LSH_BF16 && !(attn_tc_supported(p) && hash_tc_supported(p))) return LSH_ERR_UNSUPPORTED;
     return LSH_OK;
 }
@@ -164,8 +163,9 @@ static lsh_status run_attn_fwd(const Problem &p, const Choice &c, const void *qk
         LSH_TRY(staged(LSH_STAGE_NORMS, 1, st, [&] { return launch_invnorm(p, qk, w.invnorm, st); }), "key norms");
     LSH_TRY(staged(LSH_STAGE_ATTN_FWD, 1, st, [&] {
                 return c.tc_attn
-                           ? launch_attn_fwd_tc(p, qk, v, perm, w.invnorm, (__nv_bfloat16 *)w.o_r, lse, w.status, st)
-                           : launch_attn_fwd_simt(p, qk, v, perm, w.invnorm, (float *)w.o_r, lse, w.status, st);
+                           ? launch_attn_fwd_tc(p, qk, v, perm, w.buckets, (__nv_bfloat16 *)w.o_r, lse, w.status, st)
+                           : launch_attn_fwd_simt(p, qk, v, perm, w.invnorm, w.buckets, (float *)w.o_r, lse,
+                                                  w.status, st);
             }), "attention forward");
     LSH_TRY(staged(LSH_STAGE_COMBINE, 1, st, [&] { return launch_combine(p, w.o_r, c.tc_attn, lse, out, st); }),
             "round merge");
@@ -268,6 +268,7 @@ lsh_status lsh_attn_fwd_sorted(const lsh_attn_desc *desc, const void *qk, const 
     c = choose(p);
     if ((s = check_ptrs({qk, v, out, lse})) != LSH_OK) return s;
     if (!perm) return LSH_ERR_ARG;
+    if (p.flags & LSH_FLAG_BUCKET_MASK) return LSH_ERR_ARG;     // needs bucket ids: use lsh_attn_fwd
     Workspace w = plan_workspace(p, false, c.tc_attn, c.tc_hash, nullptr);
     if ((s = check_ws(workspace, ws_bytes, w.bytes)) != LSH_OK) return s;
     w = plan_workspace(p, false, c.tc_attn, c.tc_hash, (char *)workspace);
@@ -307,7 +308,8 @@ lsh_status lsh_attn_bwd(const lsh_attn_desc *desc, const void *qk, const void *v
     if ((s = check_envelope(p)) != LSH_OK) return s;
     c = choose(p);
     if ((s = check_ptrs({qk, v, out, lse, dout, dqk, dv})) != LSH_OK) return s;
-    if (!perm && !R) return LSH_ERR_ARG;
+    const bool mask = (p.flags & LSH_FLAG_BUCKET_MASK) != 0;
+    if ((!perm || mask) && !R) return LSH_ERR_ARG;             // the hash is recomputed from R
     Workspace w = plan_workspace(p, true, c.tc_attn, c.tc_hash, nullptr);
     if ((s = check_ws(workspace, ws_bytes, w.bytes)) != LSH_OK) return s;
     w = plan_workspace(p, true, c.tc_attn, c.tc_hash, (char *)workspace);
@@ -316,6 +318,12 @@ lsh_status lsh_attn_bwd(const lsh_attn_desc *desc, const void *qk, const void *v
     if (!perm) {
         if ((s = run_hash_sort(p, c, qk, R, w.perm, w, st)) != LSH_OK) return s;
         perm = w.perm;
+    } else if (mask) {
+        // the bucket mask needs the bucket ids of this call's rounds
+        LSH_TRY(staged(LSH_STAGE_HASH, c.tc_hash ? 2 : 1, st, [&] {
+                    return c.tc_hash ? launch_hash_tc(p, qk, R, w.buckets, w.rot, w.status, st)
+                                     : launch_hash_simt(p, qk, R, w.buckets, st);
+                }), "hash");
     }
     // the tensor-core backward computes the key norms from its gathered rows
     if (!c.tc_attn)
@@ -324,10 +332,10 @@ lsh_status lsh_attn_bwd(const lsh_attn_desc *desc, const void *qk, const void *v
                 return launch_bwd_prep(p, lse, out, dout, w.lse_all, w.delta, w.dx_acc, w.dv_acc, st);
             }), "backward prologue");
     LSH_TRY(staged(LSH_STAGE_ATTN_BWD, c.tc_attn ? 1 : 2, st, [&] {
-                return c.tc_attn ? launch_attn_bwd_tc(p, qk, v, dout, perm, w.invnorm, w.lse_all, w.delta, w.dx_acc,
+                return c.tc_attn ? launch_attn_bwd_tc(p, qk, v, dout, perm, w.buckets, w.lse_all, w.delta, w.dx_acc,
                                                       w.dv_acc, w.status, st)
-                                 : launch_attn_bwd_simt(p, qk, v, dout, perm, w.invnorm, w.lse_all, w.delta,
-                                                        w.self_only, w.dx_acc, w.dv_acc, w.status, st);
+                                 : launch_attn_bwd_simt(p, qk, v, dout, perm, w.invnorm, w.buckets, w.lse_all,
+                                                        w.delta, w.self_only, w.dx_acc, w.dv_acc, w.status, st);
             }), "attention backward");
     LSH_TRY(staged(LSH_STAGE_BWD_FINAL, 1, st,
                    [&] { return launch_bwd_finalize(p, w.dx_acc, w.dv_acc, dqk, dv, st); }),

@@ -70,9 +70,15 @@ struct alignas(1024) Stage {
     alignas(16) int32_t qpos[kQ];   // original position of each query slot (-1 if none)
     alignas(16) float qlse2[kQ];    // LSE * log2(e) (+inf if none)
     alignas(16) float qdelta[kQ];   // dY . y
-    alignas(16) int32_t qlim[kQ];   // causal key bound: position + 1 when the query attends to itself alone
+    alignas(16) int32_t qlim[kQ];   // causal: key bound, position + 1 when the query attends to itself alone;
+                                    // otherwise: the one key position it does not take (-2: none)
+    alignas(16) int32_t bk[256];    // bucket of slots [128k - 64, 128k + 192) (-1 if none); bucket mask only
     int32_t cmin[4];                // smallest position of chunks 2k-1 .. 2k+2 (INT_MAX if none)
 };
+
+// Optional readings (template parameter FL, bits of lsh_attn_desc.flags).
+constexpr int kMask = LSH_FLAG_BUCKET_MASK, kPen = LSH_FLAG_SELF_PENALTY;
+constexpr float kSelfPenalty = LSH_SELF_PENALTY_SCORE;
 
 struct BwdSmem {
     Stage st[kStages];
@@ -173,30 +179,40 @@ __device__ __forceinline__ void smem_chunk(const uint8_t *tile, int row, int ch,
     }
 }
 
-// One step of 16 query columns [C0 + 16 STEP, +16) of key row kr from the
-// S^T and dP^T values s, dp: P^T into TMEM, E^T into shared memory.
-template <bool CAUSAL, int STEP>
+// One step of 16 query columns [C0 + 16 STEP, +16) of key row kr (position
+// kpos, bucket kb) from the S^T and dP^T values s, dp: P^T into TMEM, E^T into
+// shared memory.  With the self penalty, a lone query's own entry has the
+// constant score kSelfPenalty: its P uses that score and its E is 0.
+template <bool CAUSAL, int FL, int STEP>
 __device__ __forceinline__ void key_row_step(const Stage &st, uint8_t (*ET)[kK * 128], uint32_t tl, int kr, int kpos,
-                                             int C0, float sc, float ec, const float *s, const float *dp, float &gx)
+                                             int kb, int C0, float sc, float ec, const float *s, const float *dp,
+                                             float &gx)
 {
     uint32_t pw[8], ew[8];
 #pragma unroll
     for (int j4 = 0; j4 < 16; j4 += 4) {
         const int q0 = C0 + STEP * 16 + j4;
-        // causal: key admitted iff its position < qlim; otherwise iff it differs from the query
-        const int4 qp4 = *reinterpret_cast<const int4 *>(CAUSAL ? &st.qlim[q0] : &st.qpos[q0]);
+        // causal: key admitted iff its position < qlim; otherwise iff it differs from qlim
+        const int4 qp4 = *reinterpret_cast<const int4 *>(&st.qlim[q0]);
         const float4 ql4 = *reinterpret_cast<const float4 *>(&st.qlse2[q0]);
         const float4 qd4 = *reinterpret_cast<const float4 *>(&st.qdelta[q0]);
+        const int4 qb4 = (FL & kMask) ? *reinterpret_cast<const int4 *>(&st.bk[64 + q0]) : make_int4(0, 0, 0, 0);
+        const int4 qo4 = (FL & kPen) ? *reinterpret_cast<const int4 *>(&st.qpos[q0]) : make_int4(0, 0, 0, 0);
         const int qp[4] = {qp4.x, qp4.y, qp4.z, qp4.w};
         const float ql[4] = {ql4.x, ql4.y, ql4.z, ql4.w};
         const float qd[4] = {qd4.x, qd4.y, qd4.z, qd4.w};
+        const int qb[4] = {qb4.x, qb4.y, qb4.z, qb4.w};
+        const int qo[4] = {qo4.x, qo4.y, qo4.z, qo4.w};
         float pv[4], ev[4];
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
-            const bool ok = CAUSAL ? (kpos < qp[u]) : (kpos != qp[u]);
-            const float e2 = tc::fast_exp2(fmaf(s[j4 + u], sc, -ql[u]));
+            bool ok = CAUSAL ? (kpos < qp[u]) : (kpos != qp[u]);
+            if (FL & kMask) ok = ok && kb == qb[u];
+            const bool own = (FL & kPen) && kpos == qo[u];
+            const float arg = own ? kSelfPenalty * kLog2e - ql[u] : fmaf(s[j4 + u], sc, -ql[u]);
+            const float e2 = tc::fast_exp2(arg);
             pv[u] = ok ? e2 : 0.f;
-            ev[u] = ec * pv[u] * (dp[j4 + u] - qd[u]);
+            ev[u] = own ? 0.f : ec * pv[u] * (dp[j4 + u] - qd[u]);
             gx = fmaf(ev[u], s[j4 + u], gx);
         }
         pw[j4 / 2] = pack_bf16x2(pv[0], pv[1]);
@@ -222,9 +238,9 @@ __device__ __forceinline__ void key_row_step(const Stage &st, uint8_t (*ET)[kK *
 // metadata is read four queries per vector load.  Returns this block's part of
 // g . x = sum_i e_i (x_i . x_k).  C0 is a run-time value so that the warps of
 // all three column blocks share one copy of the code.
-template <bool CAUSAL>
+template <bool CAUSAL, int FL>
 __device__ __forceinline__ float key_row_block(const Stage &st, uint8_t (*ET)[kK * 128], uint32_t tl, int kr, int kpos,
-                                           int C0, float kinv, float tau)
+                                               int kb, int C0, float kinv, float tau)
 {
     const float sc = tau * kinv * kLog2e;
     const float ec = tau * kinv;
@@ -235,17 +251,17 @@ __device__ __forceinline__ float key_row_block(const Stage &st, uint8_t (*ET)[kK
     tc::tmem_ld_wait();
     tc::tmem_ld16(tl + cS + C0 + 16, sb);
     tc::tmem_ld16(tl + cD + C0 + 16, db);
-    key_row_step<CAUSAL, 0>(st, ET, tl, kr, kpos, C0, sc, ec, sa, da, gx);
+    key_row_step<CAUSAL, FL, 0>(st, ET, tl, kr, kpos, kb, C0, sc, ec, sa, da, gx);
     tc::tmem_ld_wait();
     tc::tmem_ld16(tl + cS + C0 + 32, sa);
     tc::tmem_ld16(tl + cD + C0 + 32, da);
-    key_row_step<CAUSAL, 1>(st, ET, tl, kr, kpos, C0, sc, ec, sb, db, gx);
+    key_row_step<CAUSAL, FL, 1>(st, ET, tl, kr, kpos, kb, C0, sc, ec, sb, db, gx);
     tc::tmem_ld_wait();
     tc::tmem_ld16(tl + cS + C0 + 48, sb);
     tc::tmem_ld16(tl + cD + C0 + 48, db);
-    key_row_step<CAUSAL, 2>(st, ET, tl, kr, kpos, C0, sc, ec, sa, da, gx);
+    key_row_step<CAUSAL, FL, 2>(st, ET, tl, kr, kpos, kb, C0, sc, ec, sa, da, gx);
     tc::tmem_ld_wait();
-    key_row_step<CAUSAL, 3>(st, ET, tl, kr, kpos, C0, sc, ec, sb, db, gx);
+    key_row_step<CAUSAL, FL, 3>(st, ET, tl, kr, kpos, kb, C0, sc, ec, sb, db, gx);
     return gx;
 }
 
@@ -297,13 +313,13 @@ __device__ __forceinline__ void tile_advance(TileIter &t, int R, int n_k, int n_
     }
 }
 
-template <bool CAUSAL>
+template <bool CAUSAL, int FL>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_bwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__restrict__ v,
-                   const __nv_bfloat16 *__restrict__ dout, const int32_t *__restrict__ perm, const float *__restrict__ invnorm,
-                   const float *__restrict__ lse_all, const float *__restrict__ delta, float *__restrict__ dx_acc,
-                   float *__restrict__ dv_acc, int L, int R, long long n_units, int causal, float tau,
-                   uint32_t *__restrict__ status)
+                   const __nv_bfloat16 *__restrict__ dout, const int32_t *__restrict__ perm,
+                   const uint16_t *__restrict__ bkt, const float *__restrict__ lse_all,
+                   const float *__restrict__ delta, float *__restrict__ dx_acc, float *__restrict__ dv_acc, int L,
+                   int R, long long n_units, float tau, uint32_t *__restrict__ status)
 {
     extern __shared__ uint8_t smem_raw[];
     BwdSmem &sm = *reinterpret_cast<BwdSmem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -337,7 +353,7 @@ attn_bwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
         const int ptid = tid - kComputeWarps * 32, pw = ptid >> 5;
         // positions of slots [128k - 64, 128k + 192) of the next tile, loaded a tile ahead
         constexpr int kPosPer = (256 + kProducerThreads - 1) / kProducerThreads;
-        int pn[kPosPer];
+        int pn[kPosPer], bn[kPosPer];
         auto load_pos = [&](const TileIter &t) {
             const TileCoord c = tile_coord(t, R, n_k, n_runs);
             const int32_t *P = perm + c.seg * L;
@@ -352,6 +368,7 @@ attn_bwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
                 const bool good = (unsigned)pl < (unsigned)L;
                 if (in && !good) atomicOr(status, kStatusBadPerm);
                 pn[j] = in && good ? pl : -1;
+                if (FL & kMask) bn[j] = pn[j] >= 0 ? (int)bkt[c.seg * L + pn[j]] : -1;
             }
         };
         TileIter ti{blockIdx.x, 0};
@@ -368,9 +385,13 @@ attn_bwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
 #pragma unroll
             for (int j = 0; j < kPosPer; ++j) {
                 const int e = ptid + j * kProducerThreads;
-                if (e < 256) st.pos[e] = pn[j];
+                if (e < 256) {
+                    st.pos[e] = pn[j];
+                    if (FL & kMask) st.bk[e] = bn[j];
+                }
             }
             tc::named_bar_sync(1, kProducerThreads);
+            const int tile_k = tile_coord(ti, R, n_k, n_runs).k;
             // per-query LSE and delta: loads issued now, used after the copies are issued
             static_assert(kQ == 2 * kProducerThreads, "two queries per producer thread");
             int qp[2];
@@ -405,7 +426,7 @@ attn_bwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
             tc::cp_async_commit();
             if (ptid == 0) LSH_PHASE(1, 0, it, 2);
             // smallest position of chunks 2k-1 .. 2k+2 (warp w takes chunks w, w + 3)
-            for (int c = pw; c < 4; c += kProducerWarps) {
+            for (int c = pw; c < 4 && CAUSAL && !(FL & kMask); c += kProducerWarps) {
                 const int a0 = st.pos[c * 64 + lane], a1 = st.pos[c * 64 + 32 + lane];
                 int mn = min(a0 >= 0 ? a0 : INT_MAX, a1 >= 0 ? a1 : INT_MAX);
 #pragma unroll
@@ -418,12 +439,25 @@ attn_bwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
                 const int q = ptid + j * kProducerThreads;
                 if (q < kQ) {
                     const int p = qp[j];
-                    const int qa = q >> 6;
-                    const int wmin = min(st.cmin[qa], st.cmin[qa + 1]);
+                    // Does the query attend to itself alone?  Causal, no mask: its position is
+                    // the smallest of its window (chunks 2k-1+q/64 and 2k+q/64).  With the bucket
+                    // mask: the stable sort keeps a bucket's slots contiguous and in position
+                    // order, so it has a candidate iff the slot before it (or, non-causal, after
+                    // it) lies in its window and holds the same bucket.  Non-causal, no mask: never.
+                    bool lone = false;
+                    if (FL & kMask) {
+                        const int e = 64 + q, slot = tile_k * kK + q, b = st.bk[e];
+                        const bool prev = slot >= 1 && st.bk[e - 1] == b;
+                        const bool next = !CAUSAL && (slot & 63) != 63 && st.bk[e + 1] == b;
+                        lone = p >= 0 && !prev && !next;
+                    } else if (CAUSAL) {
+                        const int qa = q >> 6;
+                        lone = p >= 0 && p == min(st.cmin[qa], st.cmin[qa + 1]);
+                    }
                     st.qpos[q] = p;
                     st.qlse2[q] = p >= 0 ? ql[j] * kLog2e : INFINITY;
                     st.qdelta[q] = p >= 0 ? qd[j] : 0.f;
-                    st.qlim[q] = (p >= 0 && p == wmin) ? p + 1 : p;
+                    st.qlim[q] = CAUSAL ? (lone ? p + 1 : p) : (lone ? -2 : p);
                 }
             }
             tile_advance(ti, R, n_k, n_runs);
@@ -501,6 +535,7 @@ attn_bwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
             const TileCoord tcd = tile_coord(ti, R, n_k, n_runs);
             const long long rowbase = tcd.bh * L;
             const int kpos = st.pos[64 + kr];
+            const int kb = (FL & kMask) ? st.bk[64 + kr] : 0;
             // 1/|x_k| of this key row, unless computed while the previous tile's products ran
             const float kinv = have_next_kinv ? next_kinv : key_inv_norm(st.X, kr);
             if (!tc::mbar_wait(&sm.bar_s, ph, &sm.abort, status)) break;
@@ -515,7 +550,7 @@ attn_bwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
             // keys of chunk 2k (quads 0, 1) see queries of chunks 2k, 2k+1 (columns 0..127),
             // keys of chunk 2k+1 those of chunks 2k+1, 2k+2 (64..191); each half takes 64
             const int c0 = quad < 2 ? half * 64 : 64 + half * 64;
-            gx = key_row_block<CAUSAL>(st, sm.ET, tl, kr, kpos, c0, kinv, tau);
+            gx = key_row_block<CAUSAL, FL>(st, sm.ET, tl, kr, kpos, kb, c0, kinv, tau);
             if (half == 0) {
                 if (quad < 2) zero_block<128>(sm.ET, tl, kr);
                 else zero_block<0>(sm.ET, tl, kr);
@@ -642,13 +677,14 @@ attn_bwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
 
 }  // namespace
 
-cudaError_t launch_attn_bwd_tc(const Problem &p, const void *x, const void *v, const void *dout, const int32_t *perm,
-                               const float *invnorm, const float *lse_all, const float *delta, float *dx_acc,
-                               float *dv_acc, uint32_t *status, cudaStream_t st)
+template <bool CAUSAL, int FL>
+static cudaError_t launch_bwd(const Problem &p, const void *x, const void *v, const void *dout, const int32_t *perm,
+                              const uint16_t *bkt, const float *lse_all, const float *delta, float *dx_acc,
+                              float *dv_acc, uint32_t *status, cudaStream_t st)
 {
     static_assert(sizeof(BwdSmem) + 1024 <= 232448, "shared memory per CTA");
     const size_t smem = sizeof(BwdSmem) + 1024;
-    auto kern = p.causal ? attn_bwd_tc_kernel<true> : attn_bwd_tc_kernel<false>;
+    auto kern = attn_bwd_tc_kernel<CAUSAL, FL>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     int dev = 0, sms = 0;
@@ -657,10 +693,33 @@ cudaError_t launch_attn_bwd_tc(const Problem &p, const void *x, const void *v, c
     const long long n_units = p.S() * (((p.L + kK - 1) / kK + kRun - 1) / kRun);
     const unsigned grid = (unsigned)std::min<long long>(n_units, (long long)sms);
     kern<<<grid, kThreads, smem, st>>>((const __nv_bfloat16 *)x, (const __nv_bfloat16 *)v,
-                                                     (const __nv_bfloat16 *)dout, perm, invnorm, lse_all,
-                                                     delta, dx_acc, dv_acc, p.L, p.R, n_units, p.causal,
-                                                     1.0f / sqrtf((float)p.d), status);
+                                       (const __nv_bfloat16 *)dout, perm, bkt, lse_all, delta, dx_acc, dv_acc, p.L,
+                                       p.R, n_units, 1.0f / sqrtf((float)p.d), status);
     return cudaGetLastError();
+}
+
+cudaError_t launch_attn_bwd_tc(const Problem &p, const void *x, const void *v, const void *dout, const int32_t *perm,
+                               const uint16_t *bkt, const float *lse_all, const float *delta, float *dx_acc,
+                               float *dv_acc, uint32_t *status, cudaStream_t st)
+{
+    // key norms are computed in the kernel from the gathered rows
+    const int fl = p.flags & (kMask | kPen);
+#define LSH_BWD_CASE(C, F) return launch_bwd<C, F>(p, x, v, dout, perm, bkt, lse_all, delta, dx_acc, dv_acc, status, st)
+    if (p.causal) {
+        switch (fl) {
+        case 0: LSH_BWD_CASE(true, 0);
+        case kMask: LSH_BWD_CASE(true, kMask);
+        case kPen: LSH_BWD_CASE(true, kPen);
+        default: LSH_BWD_CASE(true, kMask | kPen);
+        }
+    }
+    switch (fl) {
+    case 0: LSH_BWD_CASE(false, 0);
+    case kMask: LSH_BWD_CASE(false, kMask);
+    case kPen: LSH_BWD_CASE(false, kPen);
+    default: LSH_BWD_CASE(false, kMask | kPen);
+    }
+#undef LSH_BWD_CASE
 }
 
 }  // namespace lsh

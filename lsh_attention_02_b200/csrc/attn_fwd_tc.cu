@@ -16,9 +16,11 @@
 //            dot products x_i . x_j, bf16 in, fp32 accumulate);
 //   softmax  one query row per thread: s_ij = (x_i . x_j) / |x_j| / sqrt(d)
 //            (unit keys), masked to the window of the row's chunk, to
-//            earlier original positions when causal, and never the query's
-//            own position unless nothing else is left ("Implementation
-//            Reading"); P is written as bf16 back into the S columns;
+//            earlier original positions when causal, optionally to the
+//            query's bucket ("LSH Attention", strict candidate set), and
+//            never the query's own position unless nothing else is left
+//            ("Implementation Reading"); P is written as bf16 back into the
+//            S columns;
 //   O = P V  tcgen05.mma M=128, N=64, K=192 with A = P read from tensor
 //            memory and V read MN-major from shared memory;
 //   store    o_r and lse_r at the query's original position (the unsort).
@@ -27,8 +29,11 @@
 // softmax uses M = tau |x_i| in place of the row maximum: one sweep, no max
 // pass.  A warp whose rows have tau |x_i| so large that exp(s - M) could leave
 // the normal fp32 range first finds the exact maximum.  A query with no
-// other candidate (causal: its position is the smallest of its window) keeps
-// its own key, whose score is tau |x_i|, so p = 1 there and lse = tau |x_i|.
+// other candidate (its softmax sum is 0) keeps its own key, whose score is
+// tau |x_i|, so p = 1 there and lse = tau |x_i|; with the self penalty its
+// lse is the penalty score.  Where other candidates exist the penalised self
+// entry's weight exp(penalty - lse) is 0 in fp32 (|x_i| < 8e5), so it is left
+// out.
 //
 // Warp roles (persistent CTA, one per SM):
 //   warps 0-3, 4-7  two softmax groups working on alternate tiles, each with
@@ -68,8 +73,22 @@ struct alignas(1024) Stage {
     alignas(16) int32_t pos[kW];    // original positions of the window slots (-1: none)
     alignas(16) float sinv[kW];     // tau * log2(e) / |x_j| (0 for a zero row or no row)
     alignas(16) float inv[kW];      // 1 / |x_j|
-    int32_t cmin[3];                // smallest position in each window chunk (INT_MAX if none)
+    alignas(16) int32_t kb[kW];     // bucket of each window slot (-1: none); bucket mask only
 };
+
+// Optional readings (template parameter FL, bits of lsh_attn_desc.flags).
+constexpr int kMask = LSH_FLAG_BUCKET_MASK, kPen = LSH_FLAG_SELF_PENALTY;
+constexpr float kSelfPenalty = LSH_SELF_PENALTY_SCORE;
+
+// Key j (position kp, bucket kb) is a candidate of query position qpos (bucket
+// qb): causal -- an earlier position (an empty slot, -1, never is); otherwise
+// any other position; with the bucket mask also the same bucket.
+template <bool CAUSAL, int FL>
+__device__ __forceinline__ bool admit(int kp, int qpos, int kb, int qb)
+{
+    const bool ok = CAUSAL ? (unsigned)kp < (unsigned)qpos : kp != qpos;
+    return (FL & kMask) ? ok && kb == qb : ok;
+}
 
 struct FwdSmem {
     Stage st[kStages];
@@ -104,11 +123,10 @@ __device__ __forceinline__ TileCoord tile_coord(long long tile, int R, int n_k)
 // BASE/2 + [32h, 32h + 32) are written, and those never reach an unread half.
 // Columns outside the row's window get zeros.  Returns l = sum of p.
 //
-// Candidates: keys at an earlier original position (causal) or at any other
-// position (non-causal).  A causal row with none (its position is the
-// smallest of its window) gets l = 0 here and is patched by the caller.
-template <bool CAUSAL>
-__device__ __forceinline__ float softmax_sweep(const Stage &st, uint32_t tl, int qpos, float shift2, int BASE,
+// Candidates: see admit().  A row with none gets l = 0 here and is patched by
+// the caller.
+template <bool CAUSAL, int FL>
+__device__ __forceinline__ float softmax_sweep(const Stage &st, uint32_t tl, int qpos, int qb, float shift2, int BASE,
                                                bool FIRST, uint64_t *half_done)
 {
     float lsum = 0.f;
@@ -139,12 +157,15 @@ __device__ __forceinline__ float softmax_sweep(const Stage &st, uint32_t tl, int
                     const int j0 = h * 64 + c * 16 + e4;
                     const int4 kp = *reinterpret_cast<const int4 *>(&st.pos[BASE + j0]);
                     const float4 ks = *reinterpret_cast<const float4 *>(&st.sinv[BASE + j0]);
+                    const int4 kb = (FL & kMask) ? *reinterpret_cast<const int4 *>(&st.kb[BASE + j0])
+                                                 : make_int4(0, 0, 0, 0);
                     const int kpa[4] = {kp.x, kp.y, kp.z, kp.w};
+                    const int kba[4] = {kb.x, kb.y, kb.z, kb.w};
                     const float ksa[4] = {ks.x, ks.y, ks.z, ks.w};
                     float pe[4];
     #pragma unroll
                     for (int e = 0; e < 4; ++e) {
-                        const bool ok = CAUSAL ? (kpa[e] < qpos) : (kpa[e] != qpos);
+                        const bool ok = admit<CAUSAL, FL>(kpa[e], qpos, kba[e], qb);
                         const float p = tc::fast_exp2(fmaf(v[c * 16 + e4 + e], ksa[e], -shift2));
                         pe[e] = ok ? p : 0.f;
                         lsum += pe[e];
@@ -171,8 +192,8 @@ __device__ __forceinline__ float softmax_sweep(const Stage &st, uint32_t tl, int
 
 // Exact row maximum of the log2-domain scores (only for rows whose bound
 // tau |x_i| is so loose that exp(s - bound) could leave the normal range).
-template <bool CAUSAL>
-__device__ __forceinline__ float exact_max(const Stage &st, uint32_t tl, int jlo, int qpos, int BASE)
+template <bool CAUSAL, int FL>
+__device__ __forceinline__ float exact_max(const Stage &st, uint32_t tl, int jlo, int qpos, int qb, int BASE)
 {
     float mx = -INFINITY;
 #pragma unroll 1
@@ -183,16 +204,18 @@ __device__ __forceinline__ float exact_max(const Stage &st, uint32_t tl, int jlo
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
             const int j = c * 16 + e;
-            const int kp = st.pos[BASE + j];
-            const bool ok = (j >= jlo) && (CAUSAL ? (kp < qpos) : (kp != qpos));
+            const bool ok = (j >= jlo) && admit<CAUSAL, FL>(st.pos[BASE + j], qpos, st.kb[BASE + j], qb);
             mx = ok ? fmaxf(mx, v[e] * st.sinv[BASE + j]) : mx;
         }
     }
     return mx;
 }
 
-template <bool CAUSAL>
-__device__ __forceinline__ void softmax_row(const Stage &st, uint32_t tl, int i, int qpos, float qinv, bool self_only,
+// A row has no candidate exactly when its sum l is 0: every admitted term is at
+// least 2^-100 (exp2 of an argument >= -2 bound log2(e) >= -100 when the row is
+// not wide, and the row maximum gives 1 when it is).
+template <bool CAUSAL, int FL>
+__device__ __forceinline__ void softmax_row(const Stage &st, uint32_t tl, int i, int qpos, int qb, float qinv,
                                             float tau, int BASE, bool FIRST, uint64_t *half_done, float &l,
                                             float &row_lse)
 {
@@ -200,15 +223,17 @@ __device__ __forceinline__ void softmax_row(const Stage &st, uint32_t tl, int i,
     float shift2 = bound * kLog2e;                              // log2-domain offset
     const bool wide = 2.f * bound * kLog2e > 100.f;             // bound - s <= 2 bound
     if (__any_sync(0xffffffffu, wide)) {
-        const float mx = exact_max<CAUSAL>(st, tl, FIRST && BASE == 0 ? 64 : 0, qpos, BASE);
+        const float mx = exact_max<CAUSAL, FL>(st, tl, FIRST && BASE == 0 ? 64 : 0, qpos, qb, BASE);
         if (wide && mx > -INFINITY) shift2 = mx;
     }
-    l = softmax_sweep<CAUSAL>(st, tl, qpos, shift2, BASE, FIRST, half_done);
+    l = softmax_sweep<CAUSAL, FL>(st, tl, qpos, qb, shift2, BASE, FIRST, half_done);
     row_lse = kLn2 * (shift2 + log2f(l));
-    if (CAUSAL && __any_sync(0xffffffffu, self_only)) {
+    const bool self_only = qpos >= 0 && l == 0.f;
+    if (__any_sync(0xffffffffu, self_only)) {
         // A row with no candidate attends to itself: p = 1 on its own key (window
-        // row 64 + i), lse = tau x_i . (x_i / |x_i|) = tau |x_i|.  The warp's 32 own
-        // keys occupy packed columns 32 + i/2 - (lane/2); each lane edits its own row.
+        // row 64 + i), lse = tau x_i . (x_i / |x_i|) = tau |x_i| (with the self
+        // penalty: lse = the penalty score).  The warp's 32 own keys occupy packed
+        // columns 32 + i/2 - (lane/2); each lane edits its own row.
         const int lane = i & 31;
         const uint32_t col0 = (uint32_t)((64 + (i - lane)) >> 1);
         float w[16];
@@ -224,7 +249,7 @@ __device__ __forceinline__ void softmax_row(const Stage &st, uint32_t tl, int i,
         tc::tmem_st16(tl + col0, u);
         if (self_only) {
             l = 1.f;
-            row_lse = bound;
+            row_lse = (FL & kPen) ? kSelfPenalty : bound;
         }
     }
 }
@@ -253,11 +278,11 @@ __device__ __forceinline__ void window_norms(Stage &st, int t, float sl2)
     }
 }
 
-template <bool CAUSAL>
+template <bool CAUSAL, int FL>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_fwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__restrict__ v,
-                   const int32_t *__restrict__ perm, __nv_bfloat16 *__restrict__ o_r, float *__restrict__ lse, int L,
-                   int R, long long n_tiles, int causal, float tau, uint32_t *__restrict__ status)
+                   const int32_t *__restrict__ perm, const uint16_t *__restrict__ bkt, __nv_bfloat16 *__restrict__ o_r,
+                   float *__restrict__ lse, int L, int R, long long n_tiles, float tau, uint32_t *__restrict__ status)
 {
     extern __shared__ uint8_t smem_raw[];
     FwdSmem &sm = *reinterpret_cast<FwdSmem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -289,9 +314,10 @@ attn_fwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
 
     if (warp >= kSoftmaxWarps && warp < kMmaWarp) {
         // ================= producer group
-        const int ptid = tid - kSoftmaxWarps * 32, pw = ptid >> 5;
-        // positions of the next tile, loaded a tile ahead (two slots per thread)
-        int pn[2] = {-1, -1};
+        const int ptid = tid - kSoftmaxWarps * 32;
+        // positions (and, with the bucket mask, buckets) of the next tile, loaded a
+        // tile ahead (two slots per thread)
+        int pn[2] = {-1, -1}, bn[2] = {-1, -1};
         // A slot outside [0, L) (chunk -1, or the missing chunk of a last tile
         // when L % 128 == 64) is empty (-1); so is a permutation entry outside
         // [0, L), which is also reported in the status word.
@@ -308,6 +334,7 @@ attn_fwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
                 const bool good = (unsigned)pl < (unsigned)L;
                 if (in && !good) atomicOr(status, kStatusBadPerm);
                 pn[j] = in && good ? pl : -1;
+                if (FL & kMask) bn[j] = pn[j] >= 0 ? (int)bkt[c.seg * L + pn[j]] : -1;
             }
         };
         if (blockIdx.x < n_tiles) load_pos(blockIdx.x);
@@ -324,6 +351,10 @@ attn_fwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
             const long long rowbase = tile_coord(tile, R, n_k).bh * L;
             st.pos[ptid] = pn[0];
             st.pos[ptid + kProducerThreads] = pn[1];
+            if (FL & kMask) {
+                st.kb[ptid] = bn[0];
+                st.kb[ptid + kProducerThreads] = bn[1];
+            }
             tc::named_bar_sync(1, kProducerThreads);
             if (tile + gridDim.x < n_tiles) load_pos(tile + gridDim.x);   // overlaps the copies below
             if (ptid == 0) LSH_PHASE(0, 0, it, 2);
@@ -346,14 +377,6 @@ attn_fwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
                 }
             }
             tc::cp_async_commit();
-            if (pw < 3) {
-                // smallest position of window chunk pw (INT_MAX when the chunk is missing)
-                const int a0 = st.pos[pw * 64 + lane], a1 = st.pos[pw * 64 + 32 + lane];
-                int mn = min(a0 >= 0 ? a0 : INT_MAX, a1 >= 0 ? a1 : INT_MAX);
-#pragma unroll
-                for (int o = 16; o > 0; o >>= 1) mn = min(mn, __shfl_xor_sync(0xffffffffu, mn, o));
-                if (lane == 0) st.cmin[pw] = mn;
-            }
             if (ptid == 0) LSH_PHASE(0, 0, it, 3);
             if (prev_s >= 0) {
                 // the previous stage's copies have landed: publish it
@@ -472,15 +495,13 @@ attn_fwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
             tc::tc_fence_after();
             const TileCoord tcd = tile_coord(tile, R, n_k);
             const int qpos = st.pos[64 + i];
+            const int qb = (FL & kMask) ? st.kb[64 + i] : 0;
             const float qinv = st.inv[64 + i];
-            // query chunk a (0: 2k, 1: 2k+1) sees window chunks a and a+1
-            const int a = i >> 6;
-            const bool self_only = CAUSAL && qpos == min(st.cmin[a], st.cmin[a + 1]);
             const bool first = tcd.k == 0;
             float l, row_lse;
             // one run-time-parameterised copy of the row code for every warp (instruction cache)
-            softmax_row<CAUSAL>(st, tl, i, qpos, qinv, self_only, tau, q >= 2 ? 64 : 0, first && q < 2, &sm.p_half[g], l,
-                                row_lse);
+            softmax_row<CAUSAL, FL>(st, tl, i, qpos, qb, qinv, tau, q >= 2 ? 64 : 0, first && q < 2, &sm.p_half[g],
+                                    l, row_lse);
             tc::tmem_st_wait();
             tc::tc_fence_before();
             __syncwarp();
@@ -525,13 +546,12 @@ bool attn_tc_supported(const Problem &p)
     return p.dtype == LSH_BF16 && p.d == kDim && p.m == 64 && p.L % 64 == 0 && p.tokens() < (1LL << 31);
 }
 
-cudaError_t launch_attn_fwd_tc(const Problem &p, const void *x, const void *v, const int32_t *perm,
-                               const float *invnorm, __nv_bfloat16 *o_r, float *lse, uint32_t *status,
-                               cudaStream_t st)
+template <bool CAUSAL, int FL>
+static cudaError_t launch_fwd(const Problem &p, const void *x, const void *v, const int32_t *perm,
+                              const uint16_t *bkt, __nv_bfloat16 *o_r, float *lse, uint32_t *status, cudaStream_t st)
 {
-    (void)invnorm;      // key norms are computed in the kernel from the gathered rows
     const size_t smem = sizeof(FwdSmem) + 1024;
-    auto kern = p.causal ? attn_fwd_tc_kernel<true> : attn_fwd_tc_kernel<false>;
+    auto kern = attn_fwd_tc_kernel<CAUSAL, FL>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     int dev = 0, sms = 0;
@@ -539,9 +559,31 @@ cudaError_t launch_attn_fwd_tc(const Problem &p, const void *x, const void *v, c
     if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
     const long long n_tiles = p.S() * ((p.L + kQ - 1) / kQ);
     const unsigned grid = (unsigned)std::min<long long>(n_tiles, (long long)sms);
-    kern<<<grid, kThreads, smem, st>>>((const __nv_bfloat16 *)x, (const __nv_bfloat16 *)v, perm, o_r, lse, p.L, p.R, n_tiles,
-                                                     p.causal, 1.0f / sqrtf((float)p.d), status);
+    kern<<<grid, kThreads, smem, st>>>((const __nv_bfloat16 *)x, (const __nv_bfloat16 *)v, perm, bkt, o_r, lse, p.L,
+                                       p.R, n_tiles, 1.0f / sqrtf((float)p.d), status);
     return cudaGetLastError();
+}
+
+cudaError_t launch_attn_fwd_tc(const Problem &p, const void *x, const void *v, const int32_t *perm,
+                               const uint16_t *bkt, __nv_bfloat16 *o_r, float *lse, uint32_t *status,
+                               cudaStream_t st)
+{
+    // key norms are computed in the kernel from the gathered rows
+    const int fl = p.flags & (kMask | kPen);
+    if (p.causal) {
+        switch (fl) {
+        case 0: return launch_fwd<true, 0>(p, x, v, perm, bkt, o_r, lse, status, st);
+        case kMask: return launch_fwd<true, kMask>(p, x, v, perm, bkt, o_r, lse, status, st);
+        case kPen: return launch_fwd<true, kPen>(p, x, v, perm, bkt, o_r, lse, status, st);
+        default: return launch_fwd<true, kMask | kPen>(p, x, v, perm, bkt, o_r, lse, status, st);
+        }
+    }
+    switch (fl) {
+    case 0: return launch_fwd<false, 0>(p, x, v, perm, bkt, o_r, lse, status, st);
+    case kMask: return launch_fwd<false, kMask>(p, x, v, perm, bkt, o_r, lse, status, st);
+    case kPen: return launch_fwd<false, kPen>(p, x, v, perm, bkt, o_r, lse, status, st);
+    default: return launch_fwd<false, kMask | kPen>(p, x, v, perm, bkt, o_r, lse, status, st);
+    }
 }
 
 }  // namespace lsh

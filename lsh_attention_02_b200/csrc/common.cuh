@@ -136,10 +136,12 @@ bool hash_tc_supported(const Problem &p);
 size_t hash_tc_scratch_bytes(const Problem &p);
 cudaError_t launch_sort(const Problem &p, const uint16_t *buckets, int32_t *perm, const Workspace &ws,
                         cudaStream_t st);
+// bkt: bucket ids by position [S, L], read only under LSH_FLAG_BUCKET_MASK (may be null otherwise)
 cudaError_t launch_attn_fwd_simt(const Problem &p, const void *x, const void *v, const int32_t *perm,
-                                 const float *invnorm, float *o_r, float *lse, uint32_t *status, cudaStream_t st);
+                                 const float *invnorm, const uint16_t *bkt, float *o_r, float *lse,
+                                 uint32_t *status, cudaStream_t st);
 cudaError_t launch_attn_fwd_tc(const Problem &p, const void *x, const void *v, const int32_t *perm,
-                               const float *invnorm, __nv_bfloat16 *o_r, float *lse, uint32_t *status,
+                               const uint16_t *bkt, __nv_bfloat16 *o_r, float *lse, uint32_t *status,
                                cudaStream_t st);
 bool attn_tc_supported(const Problem &p);
 cudaError_t launch_combine(const Problem &p, const void *o_r, bool o_r_bf16, const float *lse, void *out,
@@ -147,11 +149,11 @@ cudaError_t launch_combine(const Problem &p, const void *o_r, bool o_r_bf16, con
 cudaError_t launch_bwd_prep(const Problem &p, const float *lse, const void *out, const void *dout,
                             float *lse_all, float *delta, float *dx_acc, float *dv_acc, cudaStream_t st);
 cudaError_t launch_attn_bwd_simt(const Problem &p, const void *x, const void *v, const void *dout,
-                                 const int32_t *perm, const float *invnorm, const float *lse_all,
-                                 const float *delta, uint8_t *self_only, float *dx_acc, float *dv_acc,
-                                 uint32_t *status, cudaStream_t st);
+                                 const int32_t *perm, const float *invnorm, const uint16_t *bkt,
+                                 const float *lse_all, const float *delta, uint8_t *self_only, float *dx_acc,
+                                 float *dv_acc, uint32_t *status, cudaStream_t st);
 cudaError_t launch_attn_bwd_tc(const Problem &p, const void *x, const void *v, const void *dout,
-                               const int32_t *perm, const float *invnorm, const float *lse_all,
+                               const int32_t *perm, const uint16_t *bkt, const float *lse_all,
                                const float *delta, float *dx_acc, float *dv_acc, uint32_t *status,
                                cudaStream_t st);
 cudaError_t launch_bwd_finalize(const Problem &p, const float *dx_acc, const float *dv_acc, void *dqk, void *dv,

@@ -163,35 +163,60 @@ __device__ __forceinline__ bool valid_pos(int j, int L, uint32_t *status)
     return false;
 }
 
+// ------------------------------------------------------------------ candidates
+// Optional readings (lsh_attn_desc.flags): `bkt` (nullable) holds the bucket id
+// of every position of the segment, and only keys in the query's bucket are
+// candidates (strict N_LSH, "LSH Attention"); `self_penalty` gives the query's
+// own position the constant score kSelfPenalty instead of removing it.  When
+// other candidates exist that entry's weight exp(kSelfPenalty - lse) is below
+// 2^-149 for every |x_i| < 8e5, i.e. exactly 0 in fp32, so only a query with no
+// other candidate uses it.
+constexpr float kSelfPenalty = LSH_SELF_PENALTY_SCORE;
+
+struct SlotView {
+    const int32_t *P;
+    const uint16_t *Bk;
+    int L, causal;
+    uint32_t *status;
+    // key slot t (!= the query's slot) is a candidate of query position i in bucket bi
+    __device__ __forceinline__ bool candidate(int t, int i, int bi, int &j) const
+    {
+        j = P[t];
+        if (!valid_pos(j, L, status)) return false;
+        if (causal && j > i) return false;
+        return !Bk || Bk[j] == bi;
+    }
+};
+
 // ------------------------------------------------------------------ forward
 // One thread per (segment, sorted slot): full softmax over the window, output
 // and logsumexp written at the query's original position.
 template <typename T>
 __global__ void attn_fwd_simt_kernel(const T *__restrict__ x, const T *__restrict__ v,
                                      const int32_t *__restrict__ perm, const float *__restrict__ invnorm,
-                                     float *__restrict__ o_r, float *__restrict__ lse, int L, int R, int m,
-                                     int causal, float tau, uint32_t *__restrict__ status)
+                                     const uint16_t *__restrict__ bkt, float *__restrict__ o_r,
+                                     float *__restrict__ lse, int L, int R, int m, int causal, int self_penalty,
+                                     float tau, uint32_t *__restrict__ status)
 {
     const long long seg = blockIdx.y;
     const int s = blockIdx.x * blockDim.x + threadIdx.x;
     if (s >= L) return;
     const long long bh = seg / R;
-    const int32_t *P = perm + seg * L;
+    const SlotView sv{perm + seg * L, bkt ? bkt + seg * L : nullptr, L, causal, status};
     const T *X = x + bh * L * kDim;
     const T *V = v + bh * L * kDim;
     const float *IN = invnorm + bh * L;
-    const int i = P[s];
+    const int i = sv.P[s];
     if (!valid_pos(i, L, status)) return;          // an empty slot has no output
+    const int bi = sv.Bk ? sv.Bk[i] : 0;
     float q[kDim], kv[kDim];
     load_row(X + (long long)i * kDim, q);
     const Window w = window_of(s, m, L);
     float mx = -INFINITY;
     int cnt = 0;
     for (int t = w.w0; t < w.w1; ++t) {
-        if (t == s) continue;
-        int j = P[t];
-        if (!valid_pos(j, L, status)) continue;
-        if (causal && j > i) continue;
+        int j;
+        if (t == s || !sv.candidate(t, i, bi, j)) continue;
         load_row(X + (long long)j * kDim, kv);
         float z = tau * (dot64(q, kv) * IN[j]);
         mx = fmaxf(mx, z);
@@ -200,17 +225,15 @@ __global__ void attn_fwd_simt_kernel(const T *__restrict__ x, const T *__restric
     float acc[kDim];
     float lse_i;
     if (cnt == 0) {                       // self is the only candidate
-        lse_i = tau * (dot64(q, q) * IN[i]);
+        lse_i = self_penalty ? kSelfPenalty : tau * (dot64(q, q) * IN[i]);
         load_row(V + (long long)i * kDim, acc);
     } else {
 #pragma unroll
         for (int k = 0; k < kDim; ++k) acc[k] = 0.f;
         float l = 0.f;
         for (int t = w.w0; t < w.w1; ++t) {
-            if (t == s) continue;
-            int j = P[t];
-            if (!valid_pos(j, L, status)) continue;
-            if (causal && j > i) continue;
+            int j;
+            if (t == s || !sv.candidate(t, i, bi, j)) continue;
             load_row(X + (long long)j * kDim, kv);
             float e = expf(tau * (dot64(q, kv) * IN[j]) - mx);
             l += e;
@@ -228,13 +251,15 @@ __global__ void attn_fwd_simt_kernel(const T *__restrict__ x, const T *__restric
 }
 
 cudaError_t launch_attn_fwd_simt(const Problem &p, const void *x, const void *v, const int32_t *perm,
-                                 const float *invnorm, float *o_r, float *lse, uint32_t *status, cudaStream_t st)
+                                 const float *invnorm, const uint16_t *bkt, float *o_r, float *lse,
+                                 uint32_t *status, cudaStream_t st)
 {
     if (p.dtype != LSH_F32) return cudaErrorInvalidValue;      // bf16 runs on the tensor-core kernels
     dim3 grid((p.L + 127) / 128, (unsigned)p.S());
     float tau = 1.0f / sqrtf((float)p.d);
-    attn_fwd_simt_kernel<float><<<grid, 128, 0, st>>>((const float *)x, (const float *)v, perm, invnorm, o_r, lse,
-                                                      p.L, p.R, p.m, p.causal, tau, status);
+    attn_fwd_simt_kernel<float><<<grid, 128, 0, st>>>(
+        (const float *)x, (const float *)v, perm, invnorm, (p.flags & LSH_FLAG_BUCKET_MASK) ? bkt : nullptr, o_r,
+        lse, p.L, p.R, p.m, p.causal, (p.flags & LSH_FLAG_SELF_PENALTY) ? 1 : 0, tau, status);
     return cudaGetLastError();
 }
 
@@ -454,26 +479,29 @@ cudaError_t launch_bwd_prep(const Problem &p, const float *lse, const void *out,
 // One thread per (segment, sorted slot s) with query position i:
 //   dx_i += sum_j dz_ij tau k_j,   k_j = x_j invnorm_j.
 // Also records whether the slot attends to itself alone (needed by the key pass).
+// With the self penalty that lone entry has a constant score: no gradient to x.
 template <typename T>
 __global__ void attn_bwd_q_simt_kernel(const T *__restrict__ x, const T *__restrict__ v, const T *__restrict__ dout,
                                        const int32_t *__restrict__ perm, const float *__restrict__ invnorm,
-                                       const float *__restrict__ lse_all, const float *__restrict__ delta,
-                                       uint8_t *__restrict__ self_only, float *__restrict__ dx_acc, int L, int R,
-                                       int m, int causal, float tau, uint32_t *__restrict__ status)
+                                       const uint16_t *__restrict__ bkt, const float *__restrict__ lse_all,
+                                       const float *__restrict__ delta, uint8_t *__restrict__ self_only,
+                                       float *__restrict__ dx_acc, int L, int R, int m, int causal,
+                                       int self_penalty, float tau, uint32_t *__restrict__ status)
 {
     const long long seg = blockIdx.y;
     const int s = blockIdx.x * blockDim.x + threadIdx.x;
     if (s >= L) return;
     const long long bh = seg / R;
-    const int32_t *P = perm + seg * L;
+    const SlotView sv{perm + seg * L, bkt ? bkt + seg * L : nullptr, L, causal, status};
     const T *X = x + bh * L * kDim;
     const T *V = v + bh * L * kDim;
     const float *IN = invnorm + bh * L;
-    const int i = P[s];
+    const int i = sv.P[s];
     if (!valid_pos(i, L, status)) {
         self_only[seg * L + s] = 0;
         return;
     }
+    const int bi = sv.Bk ? sv.Bk[i] : 0;
     float q[kDim], g[kDim], kv[kDim], dq[kDim];
     load_row(X + (long long)i * kDim, q);
     load_row(dout + (bh * L + i) * kDim, g);
@@ -483,10 +511,8 @@ __global__ void attn_bwd_q_simt_kernel(const T *__restrict__ x, const T *__restr
     const Window w = window_of(s, m, L);
     int cnt = 0;
     for (int t = w.w0; t < w.w1; ++t) {
-        if (t == s) continue;
-        int j = P[t];
-        if (!valid_pos(j, L, status)) continue;
-        if (causal && j > i) continue;
+        int j;
+        if (t == s || !sv.candidate(t, i, bi, j)) continue;
         ++cnt;
         load_row(X + (long long)j * kDim, kv);
         float pij = expf(tau * (dot64(q, kv) * IN[j]) - big);
@@ -497,7 +523,7 @@ __global__ void attn_bwd_q_simt_kernel(const T *__restrict__ x, const T *__restr
 #pragma unroll
         for (int k = 0; k < kDim; ++k) dq[k] = fmaf(dz * c, kv[k], dq[k]);
     }
-    if (cnt == 0) {
+    if (cnt == 0 && !self_penalty) {
         float pij = expf(tau * (dot64(q, q) * IN[i]) - big);
         load_row(V + (long long)i * kDim, kv);
         float dz = pij * (dot64(g, kv) - dl);
@@ -516,23 +542,27 @@ __global__ void attn_bwd_q_simt_kernel(const T *__restrict__ x, const T *__restr
 // whose window holds t sit in chunks c(t) and c(t)+1:
 //   g_j  = sum_s dz_sj tau x_s          (gradient w.r.t. the unit key k_j)
 //   dx_j += invnorm_j (g_j - k_j (k_j . g_j)),   dv_j += sum_s P_sj dY_s.
+// A lone query's own entry with the self penalty has P = exp(kSelfPenalty - LSE)
+// and a constant score: it adds to dv only.
 template <typename T>
 __global__ void attn_bwd_k_simt_kernel(const T *__restrict__ x, const T *__restrict__ v, const T *__restrict__ dout,
                                        const int32_t *__restrict__ perm, const float *__restrict__ invnorm,
-                                       const float *__restrict__ lse_all, const float *__restrict__ delta,
-                                       const uint8_t *__restrict__ self_only, float *__restrict__ dx_acc,
-                                       float *__restrict__ dv_acc, int L, int R, int m, int causal, float tau,
-                                       uint32_t *__restrict__ status)
+                                       const uint16_t *__restrict__ bkt, const float *__restrict__ lse_all,
+                                       const float *__restrict__ delta, const uint8_t *__restrict__ self_only,
+                                       float *__restrict__ dx_acc, float *__restrict__ dv_acc, int L, int R, int m,
+                                       int causal, int self_penalty, float tau, uint32_t *__restrict__ status)
 {
     const long long seg = blockIdx.y;
     const int t = blockIdx.x * blockDim.x + threadIdx.x;
     if (t >= L) return;
     const long long bh = seg / R;
     const int32_t *P = perm + seg * L;
+    const uint16_t *Bk = bkt ? bkt + seg * L : nullptr;
     const T *X = x + bh * L * kDim;
     const float *IN = invnorm + bh * L;
     const int j = P[t];
     if (!valid_pos(j, L, status)) return;
+    const int bj = Bk ? Bk[j] : 0;
     float kx[kDim], vj[kDim], gk[kDim], dvj[kDim], q[kDim], g[kDim];
     load_row(X + (long long)j * kDim, kx);
     load_row(v + (bh * L + j) * kDim, vj);
@@ -544,10 +574,19 @@ __global__ void attn_bwd_k_simt_kernel(const T *__restrict__ x, const T *__restr
     for (int s = s0; s < s1; ++s) {
         int i = P[s];
         if (!valid_pos(i, L, status)) continue;
-        bool cand;
-        if (s == t) cand = self_only[seg * L + s] != 0;
-        else cand = !(causal && j > i);
-        if (!cand) continue;
+        if (s == t) {
+            if (self_only[seg * L + s] == 0) continue;
+            if (self_penalty) {
+                load_row(dout + (bh * L + i) * kDim, g);
+                const float pij = expf(kSelfPenalty - lse_all[bh * L + i]);
+#pragma unroll
+                for (int k = 0; k < kDim; ++k) dvj[k] = fmaf(pij, g[k], dvj[k]);
+                continue;
+            }
+        } else {
+            if (causal && j > i) continue;
+            if (Bk && Bk[i] != bj) continue;
+        }
         load_row(X + (long long)i * kDim, q);
         load_row(dout + (bh * L + i) * kDim, g);
         float pij = expf(tau * (dot64(q, kx) * inj) - lse_all[bh * L + i]);
@@ -572,19 +611,21 @@ __global__ void attn_bwd_k_simt_kernel(const T *__restrict__ x, const T *__restr
 }
 
 cudaError_t launch_attn_bwd_simt(const Problem &p, const void *x, const void *v, const void *dout,
-                                 const int32_t *perm, const float *invnorm, const float *lse_all,
-                                 const float *delta, uint8_t *self_only, float *dx_acc, float *dv_acc,
-                                 uint32_t *status, cudaStream_t st)
+                                 const int32_t *perm, const float *invnorm, const uint16_t *bkt,
+                                 const float *lse_all, const float *delta, uint8_t *self_only, float *dx_acc,
+                                 float *dv_acc, uint32_t *status, cudaStream_t st)
 {
     if (p.dtype != LSH_F32) return cudaErrorInvalidValue;      // bf16 runs on the tensor-core kernels
     dim3 grid((p.L + 127) / 128, (unsigned)p.S());
     float tau = 1.0f / sqrtf((float)p.d);
+    const uint16_t *bk = (p.flags & LSH_FLAG_BUCKET_MASK) ? bkt : nullptr;
+    const int pen = (p.flags & LSH_FLAG_SELF_PENALTY) ? 1 : 0;
     attn_bwd_q_simt_kernel<float><<<grid, 128, 0, st>>>((const float *)x, (const float *)v, (const float *)dout,
-                                                        perm, invnorm, lse_all, delta, self_only, dx_acc, p.L,
-                                                        p.R, p.m, p.causal, tau, status);
+                                                        perm, invnorm, bk, lse_all, delta, self_only, dx_acc, p.L,
+                                                        p.R, p.m, p.causal, pen, tau, status);
     attn_bwd_k_simt_kernel<float><<<grid, 128, 0, st>>>((const float *)x, (const float *)v, (const float *)dout,
-                                                        perm, invnorm, lse_all, delta, self_only, dx_acc,
-                                                        dv_acc, p.L, p.R, p.m, p.causal, tau, status);
+                                                        perm, invnorm, bk, lse_all, delta, self_only, dx_acc,
+                                                        dv_acc, p.L, p.R, p.m, p.causal, pen, tau, status);
     return cudaGetLastError();
 }
 

@@ -141,3 +141,18 @@ def test_static_sort_rejects_oversize_before_any_device_call(lib):
     lib.lsh_attn_last_error.restype = ctypes.c_char_p
     msg = lib.lsh_attn_last_error().decode()
     assert "lsh_attn_sort_static" in msg and str(16 << 20) in msg
+
+
+@pytest.mark.parametrize("flags", [1, 2, 3])
+def test_flags_accepted_and_their_argument_rules(lib, flags):
+    """The optional readings are accepted by the checks; the bucket mask needs
+    bucket ids, so lsh_attn_fwd_sorted refuses it and lsh_attn_bwd needs R to
+    recompute them (fake pointers, never dereferenced)."""
+    d = _desc(flags=flags)
+    assert lib.lsh_attn_workspace_size(ctypes.byref(d), 1) > 0
+    fake = ctypes.c_void_p(1 << 20)
+    big = 1 << 40
+    if flags & 1:
+        assert lib.lsh_attn_fwd_sorted(ctypes.byref(d), fake, fake, fake, fake, fake, fake, big, None) == -1
+        assert lib.lsh_attn_bwd(ctypes.byref(d), fake, fake, None, fake, fake, fake, fake, fake, fake, fake, big,
+                                None) == -1

@@ -299,6 +299,42 @@ def test_backward_run_to_run_drift_is_one_rounding_step():
         print(f"[drift] {name}: {(u != t).mean():.2e} of elements differ between two runs")
 
 
+# ------------------------------------------------------------------ optional readings (flags)
+@pytest.mark.parametrize("dtype,causal,flags,nb,L", [
+    ("bf16", True, lsh.FLAG_BUCKET_MASK, 64, 1024), ("bf16", False, lsh.FLAG_BUCKET_MASK, 64, 1024),
+    ("bf16", True, lsh.FLAG_SELF_PENALTY, 64, 1024), ("bf16", False, lsh.FLAG_SELF_PENALTY, 64, 1024),
+    ("bf16", False, 3, 256, 960), ("bf16", True, 3, 1024, 2048), ("bf16", True, lsh.FLAG_BUCKET_MASK, 2, 576),
+    ("f32", True, lsh.FLAG_BUCKET_MASK, 16, 512), ("f32", False, 3, 16, 512), ("f32", True, lsh.FLAG_SELF_PENALTY, 16, 256),
+])
+def test_flags_forward_backward(dtype, causal, flags, nb, L):
+    """Bucket mask ("LSH Attention", strict N_LSH) and self penalty
+    ("Implementation Reading", same-token question): outputs, lse and both
+    gradients against the oracle's readings, with the GPU's permutation and
+    bucket ids.  Many queries have no same-bucket key in their window, so the
+    lone-query paths run often."""
+    w = small("long_64k", B=1, H=2, L=L, n_buckets=nb, n_hashes=2, causal=causal, dtype=dtype, backward=True)
+    inp = synth.make_inputs(w)
+    run = Run(inp, w.n_buckets, w.chunk, w.causal, w.dtype, flags)
+    gb = run.host_buckets()
+    gperm = run.perm.cpu().numpy()
+    check_perm_is_stable_sort(gperm, gb, "flags perm")
+    flips = 0
+    for h in range(2):
+        ref = oracle.fwd(inp["x"][:, h:h + 1], inp["v"][:, h:h + 1], inp["R"], nb, w.chunk, causal)
+        flips += check_buckets(gb[0, h], ref["bucket"][0, 0], ref["margin"][0, 0], f"flags ({h})")
+    bk = gb if flags & lsh.FLAG_BUCKET_MASK else None
+    pen = bool(flags & lsh.FLAG_SELF_PENALTY)
+    y, lr = oracle.fwd_perm(inp["x"], inp["v"], gperm, w.chunk, causal, bucket=bk, self_penalty=pen)
+    lone = np.isclose(lr, lsh.SELF_PENALTY_SCORE) if pen else np.zeros_like(lr, dtype=bool)
+    print(f"[flags {flags}] {int(lone.sum())} penalised lone (row, round) pairs of {lr.size}")
+    assert_close(to_host(run.out), y, dtype, "out")
+    assert_close(run.lse.cpu().numpy(), lr, "f32" if dtype == "f32" else "bf16", "lse")
+    dx, dv = oracle.bwd(inp["x"], inp["v"], inp["dy"], gperm, w.chunk, causal, bucket=bk, self_penalty=pen)
+    assert_close(to_host(run.dx), dx, dtype, "dqk")
+    assert_close(to_host(run.dv), dv, dtype, "dv")
+    _flip_report(f"flags {flags}", flips, 2 * 2 * L)
+
+
 # ------------------------------------------------------------------ the five workloads
 def test_workload_tiny_f32():
     full_check(synth.WORKLOADS["tiny_f32"])
