@@ -42,6 +42,11 @@
  *   bucket mask   the strict candidate set N_LSH(i) = {j : h(q_i) = h(k_j)}
  *                 of [CAND]: inside the window only keys in the query's
  *                 bucket (of that round) are candidates;
+ *   local window  the local self-attention of the HF blog summary (page
+ *                 "The Reformer - Pushing the limits of language modeling",
+ *                 "Approach / What changed"): no hashing, positions in their
+ *                 own order, chunk c attends to chunks c - before .. c + after
+ *                 (the LSH window is before = 1, after = 0 on sorted slots);
  *   self penalty  the other answer to the same-token question of [MASK]:
  *                 the query's own position is always a candidate, with the
  *                 fixed score ORACLE_SELF_PENALTY instead of q.k/sqrt(d), so
@@ -137,18 +142,20 @@ static void normalise_keys(const double *x, long L, int d, double *khat, double 
 }
 
 /* [CAND] + [SORT] + [MASK]: the candidate positions of sorted slot s.
- * Window: slots of chunk c = s / m and of chunk c - 1 (if c > 0).
+ * Window: slots of chunks c - before .. c + after, c = s / m, clipped to
+ * [0, L) (before = 1, after = 0 for LSH attention).
  * bucket (nullable): bucket id of every position in this round; when given,
  * only keys in the query's bucket are candidates.  Returns the number of
  * candidates written to cand; *self_in = 1 when the query's own position is
  * among them (then it is the last entry): always in the self-penalty reading,
  * else only when nothing else is left. */
-static long candidates(const int32_t *perm, long L, int m, int causal, const int32_t *bucket, int self_penalty,
-                       long s, int32_t *cand, int *self_in)
+static long candidates(const int32_t *perm, long L, int m, int before, int after, int causal,
+                       const int32_t *bucket, int self_penalty, long s, int32_t *cand, int *self_in)
 {
     long c = s / m;
-    long w0 = c > 0 ? (c - 1) * m : 0;
-    long w1 = (c + 1) * m;
+    long w0 = (c - before) * m;
+    if (w0 < 0) w0 = 0;
+    long w1 = (c + after + 1) * m;
     if (w1 > L) w1 = L;
     int32_t i = perm[s];
     long nc = 0;
@@ -171,14 +178,15 @@ static long candidates(const int32_t *perm, long L, int m, int causal, const int
  * (all slots when slots == NULL).  Writes o and lse at the ORIGINAL
  * position of each query when scatter != 0, else at the list index. */
 static int attn_round_impl(const double *x, const double *v, long L, int d,
-                           const int32_t *perm, int m, int causal, const int32_t *bucket, int self_penalty,
-                           const int64_t *slots, long nslots, int scatter,
+                           const int32_t *perm, int m, int before, int after, int causal, const int32_t *bucket,
+                           int self_penalty, const int64_t *slots, long nslots, int scatter,
                            double *o, double *lse)
 {
+    const size_t wmax = (size_t)(before + after + 1) * m + 1;
     double *khat = (double *)malloc(sizeof(double) * (size_t)L * d);
     double *norm = (double *)malloc(sizeof(double) * (size_t)L);
-    int32_t *cand = (int32_t *)malloc(sizeof(int32_t) * (size_t)(2 * m + 1));
-    double *z = (double *)malloc(sizeof(double) * (size_t)(2 * m + 1));
+    int32_t *cand = (int32_t *)malloc(sizeof(int32_t) * wmax);
+    double *z = (double *)malloc(sizeof(double) * wmax);
     if (!khat || !norm || !cand || !z) { free(khat); free(norm); free(cand); free(z); return -1; }
     normalise_keys(x, L, d, khat, norm);
     const double tau = 1.0 / sqrt((double)d);
@@ -187,7 +195,7 @@ static int attn_round_impl(const double *x, const double *v, long L, int d,
         long s = slots ? (long)slots[q] : q;
         int32_t i = perm[s];
         int self_in;
-        long nc = candidates(perm, L, m, causal, bucket, self_penalty, s, cand, &self_in);
+        long nc = candidates(perm, L, m, before, after, causal, bucket, self_penalty, s, cand, &self_in);
         double zmax = -INFINITY;
         for (long a = 0; a < nc; ++a) {
             double dot = 0.0;
@@ -215,7 +223,7 @@ ORACLE_EXPORT int oracle_attn_round(const double *x, const double *v, long L, in
                                     const int32_t *perm, int m, int causal, const int32_t *bucket,
                                     int self_penalty, double *o, double *lse)
 {
-    return attn_round_impl(x, v, L, d, perm, m, causal, bucket, self_penalty, NULL, L, 1, o, lse);
+    return attn_round_impl(x, v, L, d, perm, m, 1, 0, causal, bucket, self_penalty, NULL, L, 1, o, lse);
 }
 
 /* Same as oracle_attn_round for a list of sorted slots; outputs follow the list. */
@@ -224,7 +232,7 @@ ORACLE_EXPORT int oracle_attn_slots(const double *x, const double *v, long L, in
                                     int self_penalty, const int64_t *slots, long nslots,
                                     double *o, double *lse)
 {
-    return attn_round_impl(x, v, L, d, perm, m, causal, bucket, self_penalty, slots, nslots, 0, o, lse);
+    return attn_round_impl(x, v, L, d, perm, m, 1, 0, causal, bucket, self_penalty, slots, nslots, 0, o, lse);
 }
 
 /* [ROUNDS] y_i = sum_r softmax_r(lse_r,i) o_r,i; also returns LSE_i = logsumexp_r lse_r,i. */
@@ -304,9 +312,9 @@ ORACLE_EXPORT int oracle_fwd_head_perm(const double *x, const double *v, long L,
  * Accumulated in a fixed order (round, slot, candidate).  In the self-penalty
  * reading the query's own entry has a constant score: it adds P G_i to dv_i
  * and nothing to dx.  bucket (nullable, [n_hashes, L]): given -> bucket mask. */
-ORACLE_EXPORT int oracle_bwd_head(const double *x, const double *v, const double *dy, long L, int d,
-                                  const int32_t *perm, int n_hashes, int m, int causal,
-                                  const int32_t *bucket, int self_penalty, double *dx, double *dv)
+static int bwd_impl(const double *x, const double *v, const double *dy, long L, int d, const int32_t *perm,
+                    int n_hashes, int m, int before, int after, int causal, const int32_t *bucket,
+                    int self_penalty, double *dx, double *dv)
 {
     double *y = (double *)malloc(sizeof(double) * (size_t)L * d);
     double *lse = (double *)malloc(sizeof(double) * (size_t)n_hashes * L);
@@ -315,14 +323,14 @@ ORACLE_EXPORT int oracle_bwd_head(const double *x, const double *v, const double
     double *khat = (double *)malloc(sizeof(double) * (size_t)L * d);
     double *norm = (double *)malloc(sizeof(double) * (size_t)L);
     double *dk = (double *)calloc((size_t)L * d, sizeof(double));
-    int32_t *cand = (int32_t *)malloc(sizeof(int32_t) * (size_t)(2 * m + 1));
+    int32_t *cand = (int32_t *)malloc(sizeof(int32_t) * ((size_t)(before + after + 1) * m + 1));
     int rc = -1;
     if (!y || !lse || !o || !big || !khat || !norm || !dk || !cand) goto done;
     rc = 0;
     for (int r = 0; r < n_hashes && rc == 0; ++r)
-        rc |= oracle_attn_round(x, v, L, d, perm + (size_t)r * L, m, causal,
-                                bucket ? bucket + (size_t)r * L : NULL, self_penalty,
-                                o + (size_t)r * L * d, lse + (size_t)r * L);
+        rc |= attn_round_impl(x, v, L, d, perm + (size_t)r * L, m, before, after, causal,
+                              bucket ? bucket + (size_t)r * L : NULL, self_penalty, NULL, L, 1,
+                              o + (size_t)r * L * d, lse + (size_t)r * L);
     if (rc) goto done;
     oracle_combine(o, lse, n_hashes, L, d, y, big);
     normalise_keys(x, L, d, khat, norm);
@@ -337,8 +345,8 @@ ORACLE_EXPORT int oracle_bwd_head(const double *x, const double *v, const double
             double delta = 0.0;
             for (int t = 0; t < d; ++t) delta += gi[t] * y[(size_t)i * d + t];
             int self_in;
-            long nc = candidates(pr, L, m, causal, bucket ? bucket + (size_t)r * L : NULL, self_penalty, s, cand,
-                                 &self_in);
+            long nc = candidates(pr, L, m, before, after, causal, bucket ? bucket + (size_t)r * L : NULL,
+                                 self_penalty, s, cand, &self_in);
             for (long a = 0; a < nc; ++a) {
                 int32_t j = cand[a];
                 const double *kj = khat + (size_t)j * d, *vj = v + (size_t)j * d;
@@ -369,6 +377,39 @@ ORACLE_EXPORT int oracle_bwd_head(const double *x, const double *v, const double
     }
 done:
     free(y); free(lse); free(o); free(big); free(khat); free(norm); free(dk); free(cand);
+    return rc;
+}
+
+ORACLE_EXPORT int oracle_bwd_head(const double *x, const double *v, const double *dy, long L, int d,
+                                  const int32_t *perm, int n_hashes, int m, int causal,
+                                  const int32_t *bucket, int self_penalty, double *dx, double *dv)
+{
+    return bwd_impl(x, v, dy, L, d, perm, n_hashes, m, 1, 0, causal, bucket, self_penalty, dx, dv);
+}
+
+/* Local (non-hashed) chunk attention for one (batch, head): positions in their
+ * own order, chunk c attends to chunks c - before .. c + after, the same keys,
+ * self rule and causal mask as above.  y [L, d], lse [L]. */
+ORACLE_EXPORT int oracle_local_fwd_head(const double *x, const double *v, long L, int d, int m, int before,
+                                        int after, int causal, int self_penalty, double *y, double *lse)
+{
+    int32_t *ident = (int32_t *)malloc(sizeof(int32_t) * (size_t)(L > 0 ? L : 1));
+    if (!ident) return -1;
+    for (long i = 0; i < L; ++i) ident[i] = (int32_t)i;
+    int rc = attn_round_impl(x, v, L, d, ident, m, before, after, causal, NULL, self_penalty, NULL, L, 1, y, lse);
+    free(ident);
+    return rc;
+}
+
+ORACLE_EXPORT int oracle_local_bwd_head(const double *x, const double *v, const double *dy, long L, int d, int m,
+                                        int before, int after, int causal, int self_penalty, double *dx,
+                                        double *dv)
+{
+    int32_t *ident = (int32_t *)malloc(sizeof(int32_t) * (size_t)(L > 0 ? L : 1));
+    if (!ident) return -1;
+    for (long i = 0; i < L; ++i) ident[i] = (int32_t)i;
+    int rc = bwd_impl(x, v, dy, L, d, ident, 1, m, before, after, causal, NULL, self_penalty, dx, dv);
+    free(ident);
     return rc;
 }
 
@@ -419,6 +460,32 @@ ORACLE_EXPORT int oracle_bwd_batch(const double *x, const double *v, const doubl
         rc |= oracle_bwd_head(x + rows * d, v + rows * d, dy + rows * d, L, d, perm + segs, n_hashes,
                               m, causal, bucket ? bucket + segs : NULL, self_penalty, dx + rows * d,
                               dv + rows * d);
+    }
+    return rc;
+}
+
+ORACLE_EXPORT int oracle_local_fwd_batch(const double *x, const double *v, long BH, long L, int d, int m,
+                                         int before, int after, int causal, int self_penalty, double *y,
+                                         double *lse)
+{
+    int rc = 0;
+#pragma omp parallel for schedule(dynamic, 1) reduction(| : rc)
+    for (long h = 0; h < BH; ++h)
+        rc |= oracle_local_fwd_head(x + (size_t)h * L * d, v + (size_t)h * L * d, L, d, m, before, after, causal,
+                                    self_penalty, y + (size_t)h * L * d, lse + (size_t)h * L);
+    return rc;
+}
+
+ORACLE_EXPORT int oracle_local_bwd_batch(const double *x, const double *v, const double *dy, long BH, long L, int d,
+                                         int m, int before, int after, int causal, int self_penalty, double *dx,
+                                         double *dv)
+{
+    int rc = 0;
+#pragma omp parallel for schedule(dynamic, 1) reduction(| : rc)
+    for (long h = 0; h < BH; ++h) {
+        size_t rows = (size_t)h * L * d;
+        rc |= oracle_local_bwd_head(x + rows, v + rows, dy + rows, L, d, m, before, after, causal, self_penalty,
+                                    dx + rows, dv + rows);
     }
     return rc;
 }

@@ -49,6 +49,8 @@ def lib():
         L.oracle_fwd_batch.argtypes = [_D, _D, _L, _L, _C, _D, _C, _C, _C, _C, _C, _C, _D, _D, _I32, _I32, _D]
         L.oracle_fwd_perm_batch.argtypes = [_D, _D, _L, _L, _C, _I32, _C, _C, _C, _I32, _C, _D, _D]
         L.oracle_bwd_batch.argtypes = [_D, _D, _D, _L, _L, _C, _I32, _C, _C, _C, _I32, _C, _D, _D]
+        L.oracle_local_fwd_batch.argtypes = [_D, _D, _L, _L, _C, _C, _C, _C, _C, _C, _D, _D]
+        L.oracle_local_bwd_batch.argtypes = [_D, _D, _D, _L, _L, _C, _C, _C, _C, _C, _C, _D, _D]
         L.oracle_max_threads.argtypes = []
         _lib = L
     return _lib
@@ -171,4 +173,26 @@ def bwd(x, v, dy, perm, chunk, causal, bucket=None, self_penalty=False):
     dx = np.empty_like(x); dv = np.empty_like(x)
     _check(lib().oracle_bwd_batch(_p(x, _D), _p(v, _D), _p(dy, _D), B * H, L, d, _p(perm, _I32), nh,
                                   int(chunk), int(causal), bp, int(bool(self_penalty)), _p(dx, _D), _p(dv, _D)))
+    return dx, dv
+
+
+def local_fwd(x, v, chunk, causal, before=1, after=1, self_penalty=False):
+    """Local (non-hashed) chunk attention on [B, H, L, d]: chunk c of the
+    positions in their own order attends to chunks c - before .. c + after.
+    Returns y [B, H, L, d] and lse [B, H, L]."""
+    x = _d(x); v = _d(v)
+    B, H, L, d = x.shape
+    y = np.empty_like(x); lse = np.empty((B, H, L))
+    _check(lib().oracle_local_fwd_batch(_p(x, _D), _p(v, _D), B * H, L, d, int(chunk), int(before), int(after),
+                                        int(causal), int(bool(self_penalty)), _p(y, _D), _p(lse, _D)))
+    return y, lse
+
+
+def local_bwd(x, v, dy, chunk, causal, before=1, after=1, self_penalty=False):
+    """Gradients (dx, dv) of sum(y * dy) for local chunk attention."""
+    x = _d(x); v = _d(v); dy = _d(dy)
+    B, H, L, d = x.shape
+    dx = np.empty_like(x); dv = np.empty_like(x)
+    _check(lib().oracle_local_bwd_batch(_p(x, _D), _p(v, _D), _p(dy, _D), B * H, L, d, int(chunk), int(before),
+                                        int(after), int(causal), int(bool(self_penalty)), _p(dx, _D), _p(dv, _D)))
     return dx, dv
