@@ -211,6 +211,31 @@ LSH_API lsh_status lsh_attn_bwd(const lsh_attn_desc *desc, const void *qk, const
                         const void *out, const float *lse, const int32_t *perm, const void *dout,
                         void *dqk, void *dv, void *workspace, size_t ws_bytes, void *stream);
 
+/* Local (non-hashed) chunk attention: the local self-attention of the page
+ * "The Reformer - Pushing the limits of language modeling" (section "Approach
+ * / What changed": input cut into chunks that attend with a preceding and a
+ * following overlap).  No hashing or sort: positions keep their own order,
+ * cut into chunks of desc->chunk, and a query in chunk c attends to chunks
+ * c - 1, c and, when chunks_after = 1, c + 1, with the keys, self rule,
+ * causal mask and self penalty of the LSH path (chunks_after = 0 is the LSH
+ * window on unsorted positions; under the causal mask the following chunk
+ * holds no candidate, so both values give the same result).
+ *   desc      n_hashes must be 1; n_buckets is not used; LSH_FLAG_BUCKET_MASK
+ *             is refused (LSH_ERR_ARG); the dtype envelope is that of
+ *             lsh_attn_fwd.
+ *   chunks_after  0 or 1 (other values: LSH_ERR_UNSUPPORTED).
+ *   lse       [B, H, 1, L] float32: the logsumexp over the whole window.
+ *   workspace at least lsh_attn_local_workspace_size() bytes, 256-byte aligned.
+ * The backward takes out and lse from the forward and writes dqk, dv.
+ * Errors and conventions as for lsh_attn_fwd / lsh_attn_bwd. */
+LSH_API size_t lsh_attn_local_workspace_size(const lsh_attn_desc *desc, int32_t chunks_after, int for_backward);
+LSH_API lsh_status lsh_attn_local_fwd(const lsh_attn_desc *desc, int32_t chunks_after, const void *qk,
+                                      const void *v, void *out, float *lse, void *workspace, size_t ws_bytes,
+                                      void *stream);
+LSH_API lsh_status lsh_attn_local_bwd(const lsh_attn_desc *desc, int32_t chunks_after, const void *qk,
+                                      const void *v, const void *out, const float *lse, const void *dout,
+                                      void *dqk, void *dv, void *workspace, size_t ws_bytes, void *stream);
+
 /* Parity bookkeeping: the number of (row, round) pairs of the last hash
  * (lsh_attn_hash, or the hash inside lsh_attn_fwd / lsh_attn_bwd) whose two
  * largest entries of [x R_r ; -x R_r] differ by less than 1e-6 of the

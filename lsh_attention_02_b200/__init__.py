@@ -26,7 +26,8 @@ STATUS = {0: "LSH_OK", -1: "LSH_ERR_ARG", -2: "LSH_ERR_SHAPE", -3: "LSH_ERR_ALIG
 EXPORTED = ("lsh_attn_make_rotations", "lsh_attn_workspace_size", "lsh_attn_hash", "lsh_attn_sort", "lsh_attn_sort_static", "lsh_attn_fwd_sorted", "lsh_attn_fwd",
             "lsh_attn_bwd", "lsh_attn_poll", "lsh_attn_selftest_timeout", "lsh_attn_trace_begin",
             "lsh_attn_trace_end", "lsh_attn_last_near_ties",
-            "lsh_attn_status_str", "lsh_attn_last_error", "lsh_attn_abi_version")
+            "lsh_attn_status_str", "lsh_attn_last_error", "lsh_attn_abi_version",
+            "lsh_attn_local_workspace_size", "lsh_attn_local_fwd", "lsh_attn_local_bwd")
 
 STAGES = ("hash", "sort", "norms", "attn_fwd", "combine", "bwd_prep", "attn_bwd", "bwd_final")
 
@@ -65,6 +66,10 @@ def load_library(path: str = LIB_PATH):
     L.lsh_attn_fwd_sorted.argtypes = [DP, P, P, P, P, P, P, S, P]
     L.lsh_attn_fwd.argtypes = [DP, P, P, P, P, P, P, P, S, P]
     L.lsh_attn_bwd.argtypes = [DP, P, P, P, P, P, P, P, P, P, P, S, P]
+    L.lsh_attn_local_workspace_size.argtypes = [DP, ctypes.c_int32, ctypes.c_int]
+    L.lsh_attn_local_workspace_size.restype = S
+    L.lsh_attn_local_fwd.argtypes = [DP, ctypes.c_int32, P, P, P, P, P, S, P]
+    L.lsh_attn_local_bwd.argtypes = [DP, ctypes.c_int32, P, P, P, P, P, P, P, P, S, P]
     L.lsh_attn_poll.argtypes = [P, P]
     L.lsh_attn_selftest_timeout.argtypes = [P, ctypes.c_int64, P]
     L.lsh_attn_trace_begin.argtypes = [ctypes.c_int32]
@@ -180,6 +185,29 @@ def lsh_attn_bwd(desc: Desc, qk, v, R, out, lse, perm, dout, dqk, dv, ws=None):
     _check(load_library().lsh_attn_bwd(ctypes.byref(desc), _ptr(qk), _ptr(v), _ptr(R), _ptr(out), _ptr(lse),
                                         _ptr(perm), _ptr(dout), _ptr(dqk), _ptr(dv), _ptr(ws), ws.numel(),
                                         _stream(qk)), "lsh_attn_bwd")
+    return dqk, dv
+
+
+def local_workspace(desc: Desc, chunks_after: int, for_backward: bool, device) -> torch.Tensor:
+    n = int(load_library().lsh_attn_local_workspace_size(ctypes.byref(desc), int(chunks_after), int(for_backward)))
+    if n == 0:
+        raise LshAttnError(-1, "lsh_attn_local_workspace_size", "invalid descriptor")
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def lsh_attn_local_fwd(desc: Desc, chunks_after: int, qk, v, out, lse, ws=None):
+    """Local chunk attention (no hashing): out [B,H,L,64], lse [B,H,1,L]."""
+    ws = ws if ws is not None else local_workspace(desc, chunks_after, False, qk.device)
+    _check(load_library().lsh_attn_local_fwd(ctypes.byref(desc), int(chunks_after), _ptr(qk), _ptr(v), _ptr(out),
+                                              _ptr(lse), _ptr(ws), ws.numel(), _stream(qk)), "lsh_attn_local_fwd")
+    return out, lse
+
+
+def lsh_attn_local_bwd(desc: Desc, chunks_after: int, qk, v, out, lse, dout, dqk, dv, ws=None):
+    ws = ws if ws is not None else local_workspace(desc, chunks_after, True, qk.device)
+    _check(load_library().lsh_attn_local_bwd(ctypes.byref(desc), int(chunks_after), _ptr(qk), _ptr(v), _ptr(out),
+                                              _ptr(lse), _ptr(dout), _ptr(dqk), _ptr(dv), _ptr(ws), ws.numel(),
+                                              _stream(qk)), "lsh_attn_local_bwd")
     return dqk, dv
 
 

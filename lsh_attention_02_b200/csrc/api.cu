@@ -77,6 +77,7 @@ Workspace plan_workspace(const Problem &p, bool backward, bool tc_attn, bool tc_
     w.perm = (int32_t *)take(S * L * sizeof(int32_t));
     if (!backward) {
         w.o_r = take(S * L * kDim * (tc_attn ? 2 : 4));
+        w.lse_r = (float *)take(p.prev_mask ? S * L * sizeof(float) : 0);
     } else {
         w.lse_all = (float *)take(T * sizeof(float));
         w.delta = (float *)take(T * sizeof(float));
@@ -167,7 +168,7 @@ static lsh_status run_attn_fwd(const Problem &p, const Choice &c, const void *qk
                            : launch_attn_fwd_simt(p, qk, v, perm, w.invnorm, w.buckets, (float *)w.o_r, lse,
                                                   w.status, st);
             }), "attention forward");
-    LSH_TRY(staged(LSH_STAGE_COMBINE, 1, st, [&] { return launch_combine(p, w.o_r, c.tc_attn, lse, out, st); }),
+    LSH_TRY(staged(LSH_STAGE_COMBINE, 1, st, [&] { return launch_combine(p, w.o_r, c.tc_attn, lse, out, nullptr, st); }),
             "round merge");
     return LSH_OK;
 }
@@ -340,6 +341,104 @@ lsh_status lsh_attn_bwd(const lsh_attn_desc *desc, const void *qk, const void *v
     LSH_TRY(staged(LSH_STAGE_BWD_FINAL, 1, st,
                    [&] { return launch_bwd_finalize(p, w.dx_acc, w.dv_acc, dqk, dv, st); }),
             "backward epilogue");
+    return LSH_OK;
+}
+
+// ------------------------------------------------------------------ local attention
+// Local (non-hashed) chunk attention reuses the attention kernels: round 0 is
+// the positions in their own order with the usual window (previous chunk and
+// own chunk); with a following chunk (non-causal only: under the causal mask
+// it holds no candidate), round 1 runs on the reversed order with the window
+// reduced to the previous chunk, which there is the following chunk.  The two
+// candidate sets are disjoint, so the round merge gives the three-chunk window
+// exactly, and its logsumexp is the window's.
+static lsh_status local_problem(const lsh_attn_desc *desc, int chunks_after, Problem *p)
+{
+    if (!desc) return LSH_ERR_ARG;
+    lsh_attn_desc d = *desc;
+    d.n_buckets = 2;                                     // not used
+    lsh_status s = check_desc(&d, p);
+    if (s != LSH_OK) return s;
+    if (p->R != 1) return LSH_ERR_SHAPE;                 // one set of outputs: lse is [B, H, 1, L]
+    if (p->flags & LSH_FLAG_BUCKET_MASK) return LSH_ERR_ARG;    // no buckets without hashing
+    if (chunks_after != 0 && chunks_after != 1) return LSH_ERR_UNSUPPORTED;
+    const bool following = chunks_after == 1 && !p->causal;
+    p->R = following ? 2 : 1;
+    p->prev_mask = following ? 2 : 0;
+    return LSH_OK;
+}
+
+size_t lsh_attn_local_workspace_size(const lsh_attn_desc *desc, int32_t chunks_after, int for_backward)
+{
+    Problem p;
+    if (local_problem(desc, chunks_after, &p) != LSH_OK) return 0;
+    const Choice c = choose(p);
+    return plan_workspace(p, for_backward != 0, c.tc_attn, c.tc_hash, nullptr).bytes;
+}
+
+lsh_status lsh_attn_local_fwd(const lsh_attn_desc *desc, int32_t chunks_after, const void *qk, const void *v,
+                              void *out, float *lse, void *workspace, size_t ws_bytes, void *stream)
+{
+    Problem p;
+    lsh_status s;
+    if ((s = local_problem(desc, chunks_after, &p)) != LSH_OK) return s;
+    if ((s = check_envelope(p)) != LSH_OK) return s;
+    const Choice c = choose(p);
+    if ((s = check_ptrs({qk, v, out, lse})) != LSH_OK) return s;
+    Workspace w = plan_workspace(p, false, c.tc_attn, c.tc_hash, nullptr);
+    if ((s = check_ws(workspace, ws_bytes, w.bytes)) != LSH_OK) return s;
+    w = plan_workspace(p, false, c.tc_attn, c.tc_hash, (char *)workspace);
+    cudaStream_t st = (cudaStream_t)stream;
+    LSH_TRY(cudaMemsetAsync(w.status, 0, sizeof(uint32_t), st), "status reset");
+    LSH_TRY(launch_local_perm(p, w.perm, st), "local order");
+    float *lse_rounds = p.R == 2 ? w.lse_r : lse;        // one part: its lse is the window's
+    if (!c.tc_attn)
+        LSH_TRY(staged(LSH_STAGE_NORMS, 1, st, [&] { return launch_invnorm(p, qk, w.invnorm, st); }), "key norms");
+    LSH_TRY(staged(LSH_STAGE_ATTN_FWD, 1, st, [&] {
+                return c.tc_attn ? launch_attn_fwd_tc(p, qk, v, w.perm, nullptr, (__nv_bfloat16 *)w.o_r, lse_rounds,
+                                                      w.status, st)
+                                 : launch_attn_fwd_simt(p, qk, v, w.perm, w.invnorm, nullptr, (float *)w.o_r,
+                                                        lse_rounds, w.status, st);
+            }), "local attention forward");
+    LSH_TRY(staged(LSH_STAGE_COMBINE, 1, st, [&] {
+                return launch_combine(p, w.o_r, c.tc_attn, lse_rounds, out, p.R == 2 ? lse : nullptr, st);
+            }), "local merge");
+    return LSH_OK;
+}
+
+lsh_status lsh_attn_local_bwd(const lsh_attn_desc *desc, int32_t chunks_after, const void *qk, const void *v,
+                              const void *out, const float *lse, const void *dout, void *dqk, void *dv,
+                              void *workspace, size_t ws_bytes, void *stream)
+{
+    Problem p;
+    lsh_status s;
+    if ((s = local_problem(desc, chunks_after, &p)) != LSH_OK) return s;
+    if ((s = check_envelope(p)) != LSH_OK) return s;
+    const Choice c = choose(p);
+    if ((s = check_ptrs({qk, v, out, lse, dout, dqk, dv})) != LSH_OK) return s;
+    Workspace w = plan_workspace(p, true, c.tc_attn, c.tc_hash, nullptr);
+    if ((s = check_ws(workspace, ws_bytes, w.bytes)) != LSH_OK) return s;
+    w = plan_workspace(p, true, c.tc_attn, c.tc_hash, (char *)workspace);
+    cudaStream_t st = (cudaStream_t)stream;
+    LSH_TRY(cudaMemsetAsync(w.status, 0, sizeof(uint32_t), st), "status reset");
+    LSH_TRY(launch_local_perm(p, w.perm, st), "local order");
+    if (!c.tc_attn)
+        LSH_TRY(staged(LSH_STAGE_NORMS, 1, st, [&] { return launch_invnorm(p, qk, w.invnorm, st); }), "key norms");
+    // lse holds the whole window's logsumexp already: the prologue's merge is over one set
+    Problem p1 = p;
+    p1.R = 1;
+    LSH_TRY(staged(LSH_STAGE_BWD_PREP, 1, st, [&] {
+                return launch_bwd_prep(p1, lse, out, dout, w.lse_all, w.delta, w.dx_acc, w.dv_acc, st);
+            }), "local backward prologue");
+    LSH_TRY(staged(LSH_STAGE_ATTN_BWD, c.tc_attn ? 1 : 2, st, [&] {
+                return c.tc_attn ? launch_attn_bwd_tc(p, qk, v, dout, w.perm, nullptr, w.lse_all, w.delta, w.dx_acc,
+                                                      w.dv_acc, w.status, st)
+                                 : launch_attn_bwd_simt(p, qk, v, dout, w.perm, w.invnorm, nullptr, w.lse_all,
+                                                        w.delta, w.self_only, w.dx_acc, w.dv_acc, w.status, st);
+            }), "local attention backward");
+    LSH_TRY(staged(LSH_STAGE_BWD_FINAL, 1, st,
+                   [&] { return launch_bwd_finalize(p, w.dx_acc, w.dv_acc, dqk, dv, st); }),
+            "local backward epilogue");
     return LSH_OK;
 }
 

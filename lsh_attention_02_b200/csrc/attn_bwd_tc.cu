@@ -319,7 +319,7 @@ attn_bwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
                    const __nv_bfloat16 *__restrict__ dout, const int32_t *__restrict__ perm,
                    const uint16_t *__restrict__ bkt, const float *__restrict__ lse_all,
                    const float *__restrict__ delta, float *__restrict__ dx_acc, float *__restrict__ dv_acc, int L,
-                   int R, long long n_units, float tau, uint32_t *__restrict__ status)
+                   int R, long long n_units, float tau, uint32_t prev_mask, uint32_t *__restrict__ status)
 {
     extern __shared__ uint8_t smem_raw[];
     BwdSmem &sm = *reinterpret_cast<BwdSmem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -391,7 +391,9 @@ attn_bwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
                 }
             }
             tc::named_bar_sync(1, kProducerThreads);
-            const int tile_k = tile_coord(ti, R, n_k, n_runs).k;
+            const TileCoord pc = tile_coord(ti, R, n_k, n_runs);
+            const int tile_k = pc.k;
+            const bool prev = (prev_mask >> pc.r) & 1u;     // previous chunk alone: no lone queries
             // per-query LSE and delta: loads issued now, used after the copies are issued
             static_assert(kQ == 2 * kProducerThreads, "two queries per producer thread");
             int qp[2];
@@ -445,7 +447,8 @@ attn_bwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
                     // order, so it has a candidate iff the slot before it (or, non-causal, after
                     // it) lies in its window and holds the same bucket.  Non-causal, no mask: never.
                     bool lone = false;
-                    if (FL & kMask) {
+                    if (prev) {
+                    } else if (FL & kMask) {
                         const int e = 64 + q, slot = tile_k * kK + q, b = st.bk[e];
                         const bool prev = slot >= 1 && st.bk[e - 1] == b;
                         const bool next = !CAUSAL && (slot & 63) != 63 && st.bk[e + 1] == b;
@@ -549,8 +552,18 @@ attn_bwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
             float gx;                                // partial g . x of key row kr
             // keys of chunk 2k (quads 0, 1) see queries of chunks 2k, 2k+1 (columns 0..127),
             // keys of chunk 2k+1 those of chunks 2k+1, 2k+2 (64..191); each half takes 64
+            // (a round whose window is the previous chunk alone: keys of chunk 2k+1 see
+            // only the queries of chunk 2k+2, keys of chunk 2k only those of 2k+1, so
+            // the lower column block is zero as well)
             const int c0 = quad < 2 ? half * 64 : 64 + half * 64;
-            gx = key_row_block<CAUSAL, FL>(st, sm.ET, tl, kr, kpos, kb, c0, kinv, tau);
+            const bool prev = (prev_mask >> tcd.r) & 1u;
+            if (prev && half == 0) {
+                gx = 0.f;
+                if (quad < 2) zero_block<0>(sm.ET, tl, kr);
+                else zero_block<64>(sm.ET, tl, kr);
+            } else {
+                gx = key_row_block<CAUSAL, FL>(st, sm.ET, tl, kr, kpos, kb, c0, kinv, tau);
+            }
             if (half == 0) {
                 if (quad < 2) zero_block<128>(sm.ET, tl, kr);
                 else zero_block<0>(sm.ET, tl, kr);
@@ -694,7 +707,7 @@ static cudaError_t launch_bwd(const Problem &p, const void *x, const void *v, co
     const unsigned grid = (unsigned)std::min<long long>(n_units, (long long)sms);
     kern<<<grid, kThreads, smem, st>>>((const __nv_bfloat16 *)x, (const __nv_bfloat16 *)v,
                                        (const __nv_bfloat16 *)dout, perm, bkt, lse_all, delta, dx_acc, dv_acc, p.L,
-                                       p.R, n_units, 1.0f / sqrtf((float)p.d), status);
+                                       p.R, n_units, 1.0f / sqrtf((float)p.d), (uint32_t)p.prev_mask, status);
     return cudaGetLastError();
 }
 

@@ -127,7 +127,7 @@ __device__ __forceinline__ TileCoord tile_coord(long long tile, int R, int n_k)
 // the caller.
 template <bool CAUSAL, int FL>
 __device__ __forceinline__ float softmax_sweep(const Stage &st, uint32_t tl, int qpos, int qb, float shift2, int BASE,
-                                               bool FIRST, uint64_t *half_done)
+                                               bool FIRST, bool PREV, uint64_t *half_done)
 {
     float lsum = 0.f;
     const uint32_t z[8] = {0, 0, 0, 0, 0, 0, 0, 0};
@@ -141,7 +141,7 @@ __device__ __forceinline__ float softmax_sweep(const Stage &st, uint32_t tl, int
     }
 #pragma unroll 1
     for (int h = 0; h < 2; ++h) {
-        if (FIRST && BASE == 0 && h == 0) {                     // missing chunk -1
+        if ((FIRST && BASE == 0 && h == 0) || (PREV && h == 1)) {   // missing chunk -1, or own chunk left out
 #pragma unroll
             for (int c = 0; c < 4; ++c) tc::tmem_st8(tl + (uint32_t)(c * 8), z);
         } else {
@@ -193,11 +193,11 @@ __device__ __forceinline__ float softmax_sweep(const Stage &st, uint32_t tl, int
 // Exact row maximum of the log2-domain scores (only for rows whose bound
 // tau |x_i| is so loose that exp(s - bound) could leave the normal range).
 template <bool CAUSAL, int FL>
-__device__ __forceinline__ float exact_max(const Stage &st, uint32_t tl, int jlo, int qpos, int qb, int BASE)
+__device__ __forceinline__ float exact_max(const Stage &st, uint32_t tl, int jlo, int jhi, int qpos, int qb, int BASE)
 {
     float mx = -INFINITY;
 #pragma unroll 1
-    for (int c = 0; c < 8; ++c) {
+    for (int c = 0; c < jhi / 16; ++c) {
         float v[16];
         tc::tmem_ld16(tl + (uint32_t)(BASE + c * 16), v);
         tc::tmem_ld_wait();
@@ -213,22 +213,25 @@ __device__ __forceinline__ float exact_max(const Stage &st, uint32_t tl, int jlo
 
 // A row has no candidate exactly when its sum l is 0: every admitted term is at
 // least 2^-100 (exp2 of an argument >= -2 bound log2(e) >= -100 when the row is
-// not wide, and the row maximum gives 1 when it is).
+// not wide, and the row maximum gives 1 when it is).  PREV: a round whose window
+// is the previous chunk alone (the following-chunk part of local attention, in
+// reversed order); a row left with no candidate there contributes nothing
+// (lse = -inf, output 0) instead of attending to itself.
 template <bool CAUSAL, int FL>
 __device__ __forceinline__ void softmax_row(const Stage &st, uint32_t tl, int i, int qpos, int qb, float qinv,
-                                            float tau, int BASE, bool FIRST, uint64_t *half_done, float &l,
-                                            float &row_lse)
+                                            float tau, int BASE, bool FIRST, bool PREV, uint64_t *half_done,
+                                            float &l, float &row_lse)
 {
     const float bound = qinv > 0.f ? tau / qinv : 0.f;        // tau |x_i| >= every score of the row
     float shift2 = bound * kLog2e;                              // log2-domain offset
     const bool wide = 2.f * bound * kLog2e > 100.f;             // bound - s <= 2 bound
     if (__any_sync(0xffffffffu, wide)) {
-        const float mx = exact_max<CAUSAL, FL>(st, tl, FIRST && BASE == 0 ? 64 : 0, qpos, qb, BASE);
+        const float mx = exact_max<CAUSAL, FL>(st, tl, FIRST && BASE == 0 ? 64 : 0, PREV ? 64 : 128, qpos, qb, BASE);
         if (wide && mx > -INFINITY) shift2 = mx;
     }
-    l = softmax_sweep<CAUSAL, FL>(st, tl, qpos, qb, shift2, BASE, FIRST, half_done);
+    l = softmax_sweep<CAUSAL, FL>(st, tl, qpos, qb, shift2, BASE, FIRST, PREV, half_done);
     row_lse = kLn2 * (shift2 + log2f(l));
-    const bool self_only = qpos >= 0 && l == 0.f;
+    const bool self_only = qpos >= 0 && l == 0.f && !PREV;
     if (__any_sync(0xffffffffu, self_only)) {
         // A row with no candidate attends to itself: p = 1 on its own key (window
         // row 64 + i), lse = tau x_i . (x_i / |x_i|) = tau |x_i| (with the self
@@ -282,7 +285,8 @@ template <bool CAUSAL, int FL>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_fwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__restrict__ v,
                    const int32_t *__restrict__ perm, const uint16_t *__restrict__ bkt, __nv_bfloat16 *__restrict__ o_r,
-                   float *__restrict__ lse, int L, int R, long long n_tiles, float tau, uint32_t *__restrict__ status)
+                   float *__restrict__ lse, int L, int R, long long n_tiles, float tau, uint32_t prev_mask,
+                   uint32_t *__restrict__ status)
 {
     extern __shared__ uint8_t smem_raw[];
     FwdSmem &sm = *reinterpret_cast<FwdSmem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -500,7 +504,8 @@ attn_fwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
             const bool first = tcd.k == 0;
             float l, row_lse;
             // one run-time-parameterised copy of the row code for every warp (instruction cache)
-            softmax_row<CAUSAL, FL>(st, tl, i, qpos, qb, qinv, tau, q >= 2 ? 64 : 0, first && q < 2, &sm.p_half[g],
+            const bool prev = (prev_mask >> tcd.r) & 1u;    // this round's window: the previous chunk alone
+            softmax_row<CAUSAL, FL>(st, tl, i, qpos, qb, qinv, tau, q >= 2 ? 64 : 0, first && q < 2, prev, &sm.p_half[g],
                                     l, row_lse);
             tc::tmem_st_wait();
             tc::tc_fence_before();
@@ -520,7 +525,7 @@ attn_fwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
                 tc::mbar_arrive(&sm.o_free[g]);
                 tc::mbar_arrive(&sm.empty[s]);
             }
-            const float rl = 1.0f / l;
+            const float rl = l > 0.f ? 1.0f / l : 0.f;        // no candidate (previous-chunk round): output 0
 #pragma unroll
             for (int d = 0; d < kDim; ++d) o[d] *= rl;
             if (qpos >= 0) {                     // an empty query slot has no output
@@ -560,7 +565,7 @@ static cudaError_t launch_fwd(const Problem &p, const void *x, const void *v, co
     const long long n_tiles = p.S() * ((p.L + kQ - 1) / kQ);
     const unsigned grid = (unsigned)std::min<long long>(n_tiles, (long long)sms);
     kern<<<grid, kThreads, smem, st>>>((const __nv_bfloat16 *)x, (const __nv_bfloat16 *)v, perm, bkt, o_r, lse, p.L,
-                                       p.R, n_tiles, 1.0f / sqrtf((float)p.d), status);
+                                       p.R, n_tiles, 1.0f / sqrtf((float)p.d), (uint32_t)p.prev_mask, status);
     return cudaGetLastError();
 }
 

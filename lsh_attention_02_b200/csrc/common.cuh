@@ -15,6 +15,10 @@ constexpr int kDim = 64;              // head dimension supported by every kerne
 // ---------------------------------------------------------------- problem
 struct Problem {
     int B, H, L, d, nb, R, m, causal, dtype, flags;
+    // Rounds whose window is the previous chunk alone (bit r set: round r), with
+    // no self fallback; 0 for LSH attention.  Local attention with a following
+    // chunk runs that part as round 1 on the reversed order.
+    int prev_mask = 0;
     long long BH() const { return (long long)B * H; }
     long long S() const { return BH() * R; }         // (b, h, round) segments
     long long tokens() const { return BH() * L; }
@@ -44,6 +48,7 @@ struct Workspace {
     uint32_t *sort_counts;            // [S, radix, tiles]
     int32_t *perm;                    // [S, L]   internal permutation
     void *o_r;                        // [S, L, 64] per-round outputs
+    float *lse_r;                     // [S, L]   per-round logsumexp (local attention with two parts)
     float *lse_all;                   // [BH, L]  logsumexp over rounds
     float *delta;                     // [BH, L]  dY . Y
     uint8_t *self_only;               // [S, L]   per sorted slot
@@ -144,8 +149,11 @@ cudaError_t launch_attn_fwd_tc(const Problem &p, const void *x, const void *v, c
                                const uint16_t *bkt, __nv_bfloat16 *o_r, float *lse, uint32_t *status,
                                cudaStream_t st);
 bool attn_tc_supported(const Problem &p);
+// lse_out (nullable): receives logsumexp over the rounds, [BH, L]
 cudaError_t launch_combine(const Problem &p, const void *o_r, bool o_r_bf16, const float *lse, void *out,
-                           cudaStream_t st);
+                           float *lse_out, cudaStream_t st);
+// Local attention's slot orders ([S, L]: round 0 identity, round 1 reversed).
+cudaError_t launch_local_perm(const Problem &p, int32_t *perm, cudaStream_t st);
 cudaError_t launch_bwd_prep(const Problem &p, const float *lse, const void *out, const void *dout,
                             float *lse_all, float *delta, float *dx_acc, float *dv_acc, cudaStream_t st);
 cudaError_t launch_attn_bwd_simt(const Problem &p, const void *x, const void *v, const void *dout,

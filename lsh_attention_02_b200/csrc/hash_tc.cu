@@ -8,13 +8,15 @@
 //
 // Persistent CTAs (one per SM) walk blocks of 256 rows (two M=128 tiles);
 // each block runs every round.  Warp roles:
-//   warps 0-7  epilogue: warp w reads TMEM lanes 32*(w%4).. of M-tile w/4,
-//              one row per thread, and keeps the running argmax;
-//   warp 8     producer: the next block's x rows by two TMA tile loads into
+//   warps 0-15 epilogue: warp w reads TMEM lanes 32*(w%4).. of M-tile (w/4)%2,
+//              one row per thread, and one half of every N-tile's columns
+//              (w/8), keeping the running argmax; the halves of a row merge
+//              through shared memory at the end of each round;
+//   warp 16    producer: the next block's x rows by two TMA tile loads into
 //              the idle one of two A buffers, and one bulk copy per (round,
 //              N-tile) of the rotation tile, pre-transposed and pre-swizzled
 //              in global memory, into a 4-stage shared-memory ring;
-//   warp 9     MMA issuer: 4 K-steps per M-tile and N-tile into one of two
+//   warp 17    MMA issuer: 4 K-steps per M-tile and N-tile into one of two
 //              TMEM accumulator buffers (double buffering lets the epilogue
 //              of tile t overlap the MMAs of tile t+1), with a completion
 //              barrier per M-tile so the two epilogue halves start apart and
@@ -35,7 +37,7 @@ namespace {
 constexpr int kRows = 256;          // rows per block
 constexpr int kMaxNT = 128;         // widest N-tile
 constexpr int kStages = 4;          // rotation-tile ring
-constexpr int kEpiWarps = 8;
+constexpr int kEpiWarps = 16;         // 4 lane quadrants x 2 M-tiles x 2 column halves
 constexpr int kThreads = (kEpiWarps + 2) * 32;
 constexpr int kTmemCols = 512;      // 2 buffers x 2 M-tiles x kMaxNT
 
@@ -45,6 +47,8 @@ struct HashSmem {
     uint64_t full[kStages], empty[kStages];
     uint64_t a_full[2], a_empty[2];
     uint64_t acc_full[2][2], acc_empty[2];  // [buffer][M-tile]
+    float mbest[2][kRows];                  // upper column half's running best, by round parity
+    int mbkt[2][kRows];                     // ... and its bucket
     uint64_t drain;                         // timeout path: the MMA issuer's last products
     uint32_t tmem_base;
     int abort;
@@ -191,13 +195,18 @@ hash_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __nv_bfloat16 *__
             if (*reinterpret_cast<volatile int *>(&sm.abort)) tc::mma_drain(&sm.drain, status);
         }
     } else {
-        // ---------------- epilogue: one row per thread
-        const int q = warp & 3, mt = warp >> 2;
-        const uint32_t lane_base = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(mt * kMaxNT);
-        int it = 0;
+        // ---------------- epilogue: warp w reads TMEM lanes 32*(w%4).. of M-tile
+        // (w/4)%2, one row per thread, and columns [NH*hf, NH*hf + NH) of every
+        // N-tile (hf = w/8), so four epilogue warps share each scheduler.  The two
+        // column halves of a row merge through shared memory once per round.
+        constexpr int NH = NT / 2;
+        const int q = warp & 3, mt = (warp >> 2) & 1, hf = warp >> 3;
+        const uint32_t lane_base = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(mt * kMaxNT + hf * NH);
+        const int prow = mt * 128 + q * 32 + lane;               // row within the 256-row block
+        int it = 0, rd = 0;                                      // rd: rounds finished (merge slot parity)
         bool ok = true;
         for (long long blk = blockIdx.x; ok && blk < n_blocks; blk += gridDim.x) {
-            const long long g = blk * kRows + mt * 128 + q * 32 + lane;
+            const long long g = blk * kRows + prow;
             float best = -INFINITY;
             int bucket = 0;
             for (int i = 0; i < items; ++i, ++it) {
@@ -207,9 +216,9 @@ hash_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __nv_bfloat16 *__
                 if (!tc::mbar_wait(&sm.acc_full[ab][mt], aph, &sm.abort, status)) { ok = false; break; }
                 if (threadIdx.x == 0) LSH_PHASE(0, 0, it, 1);
                 tc::tc_fence_after();
-                float v[NT];
+                float v[NH];
 #pragma unroll
-                for (int c = 0; c < NT / 16; ++c)
+                for (int c = 0; c < NH / 16; ++c)
                     tc::tmem_ld16(lane_base + (uint32_t)(ab * 2 * kMaxNT + c * 16), v + c * 16);
                 tc::tmem_ld_wait();
                 tc::tc_fence_before();
@@ -217,8 +226,8 @@ hash_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __nv_bfloat16 *__
                 if (lane == 0) tc::mbar_arrive(&sm.acc_empty[ab]);
                 if (threadIdx.x == 0) LSH_PHASE(0, 0, it, 2);
 
-                // pass 1: extremes of the tile, four independent chains per extreme
-                constexpr int Q = NT / 4;
+                // pass 1: extremes of the half tile, four independent chains per extreme
+                constexpr int Q = NH / 4;
                 float mxq[4], mnq[4];
 #pragma unroll
                 for (int qq = 0; qq < 4; ++qq) {
@@ -238,11 +247,11 @@ hash_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __nv_bfloat16 *__
                 const float target = pos ? mx : mn;
                 if (threadIdx.x == 0) LSH_PHASE(0, 0, it, 3);
                 // pass 2: lowest column holding the extreme.  U = |extreme| bounds every
-                // |v| of the tile; with B = 2^(24 - e(U)), (U - side * v_j) * B is exactly
-                // 0 where v_j is the extreme and at least 1 elsewhere (the closest float
-                // below U is 2^(e(U) - 24) away), so a saturating FMA gives a 0/1 flag
-                // without a compare.  Sixteen flags per chain are summed as the bits of
-                // an integer kept in the mantissa of 2^23 + sum (exact), and the first
+                // |v| of the half tile; with B = 2^(24 - e(U)), (U - side * v_j) * B is
+                // exactly 0 where v_j is the extreme and at least 1 elsewhere (the closest
+                // float below U is 2^(e(U) - 24) away), so a saturating FMA gives a 0/1
+                // flag without a compare.  Sixteen flags per chain are summed as the bits
+                // of an integer kept in the mantissa of 2^23 + sum (exact), and the first
                 // clear bit is the column.  This runs on the FMA pipe while pass 1 uses
                 // the ALU pipe.  Extremes below 2^-103 (B would not be finite) take the
                 // compare-and-select form.
@@ -253,7 +262,7 @@ hash_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __nv_bfloat16 *__
                     int jq[4];
 #pragma unroll
                     for (int qq = 0; qq < 4; ++qq) {
-                        int jj = NT;
+                        int jj = NH;
 #pragma unroll
                         for (int j = qq * Q + Q - 1; j >= qq * Q; --j) jj = (v[j] == target) ? j : jj;
                         jq[qq] = jj;
@@ -263,7 +272,7 @@ hash_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __nv_bfloat16 *__
                     const float B = __int_as_float(min(278 - be, 253) << 23);
                     const float nsB = pos ? -B : B;
                     const float UB = U * B;
-                    constexpr int NC = NT / 16;
+                    constexpr int NC = NH / 16;
                     float acc[NC];
 #pragma unroll
                     for (int c = 0; c < NC; ++c) acc[c] = 8388608.f;
@@ -272,7 +281,7 @@ hash_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __nv_bfloat16 *__
 #pragma unroll
                         for (int c = 0; c < NC; ++c)
                             acc[c] = fmaf(tc::fma_sat(v[c * 16 + k], nsB, UB), (float)(1 << k), acc[c]);
-                    js = NT;
+                    js = NH;
 #pragma unroll
                     for (int c = NC - 1; c >= 0; --c) {
                         const uint32_t eq = ~__float_as_uint(acc[c]) & 0xFFFFu;
@@ -281,15 +290,30 @@ hash_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __nv_bfloat16 *__
                 }
                 const int r = i / n_nt, nt = i % n_nt;
                 const float tbest = pos ? mx : -mn;
-                const int tb = (pos ? 0 : half) + nt * NT + js;
+                const int tb = (pos ? 0 : half) + nt * NT + hf * NH + js;
                 if (tbest > best || (tbest == best && tb < bucket)) { best = tbest; bucket = tb; }
                 if (threadIdx.x == 0) LSH_PHASE(0, 0, it, 4);
                 if (nt == n_nt - 1) {
-                    if (g < rows_total) {
-                        const long long bh = g / L;
-                        const int pos_i = (int)(g % L);
-                        buckets[(bh * rounds + r) * L + pos_i] = (uint16_t)bucket;
+                    // the upper column half hands its (best, bucket) to the lower one, which
+                    // keeps the larger value (the lower bucket on a tie) and writes the id;
+                    // both warps of a pair wait on the same barriers, so both get here
+                    const int slot = rd & 1;
+                    if (hf == 1) {
+                        sm.mbest[slot][prow] = best;
+                        sm.mbkt[slot][prow] = bucket;
                     }
+                    tc::named_bar_sync(1 + (warp & 7), 64);
+                    if (hf == 0) {
+                        const float ob = sm.mbest[slot][prow];
+                        const int obk = sm.mbkt[slot][prow];
+                        if (ob > best || (ob == best && obk < bucket)) { best = ob; bucket = obk; }
+                        if (g < rows_total) {
+                            const long long bh = g / L;
+                            const int pos_i = (int)(g % L);
+                            buckets[(bh * rounds + r) * L + pos_i] = (uint16_t)bucket;
+                        }
+                    }
+                    ++rd;
                     best = -INFINITY;
                     bucket = 0;
                 }

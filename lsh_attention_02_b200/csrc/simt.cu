@@ -145,12 +145,15 @@ long long read_near_ties()
 struct Window {
     int w0, w1;
 };
-__device__ __forceinline__ Window window_of(int s, int m, int L)
+// The window of sorted slot s: chunks c - 1 and c (c = s / m); `prev`: the
+// previous chunk alone (the following-chunk part of local attention, run on
+// the reversed order), empty for c = 0.
+__device__ __forceinline__ Window window_of(int s, int m, int L, bool prev = false)
 {
     int c = s / m;
     Window w;
     w.w0 = c > 0 ? (c - 1) * m : 0;
-    w.w1 = min((c + 1) * m, L);
+    w.w1 = prev ? c * m : min((c + 1) * m, L);
     return w;
 }
 
@@ -196,7 +199,7 @@ __global__ void attn_fwd_simt_kernel(const T *__restrict__ x, const T *__restric
                                      const int32_t *__restrict__ perm, const float *__restrict__ invnorm,
                                      const uint16_t *__restrict__ bkt, float *__restrict__ o_r,
                                      float *__restrict__ lse, int L, int R, int m, int causal, int self_penalty,
-                                     float tau, uint32_t *__restrict__ status)
+                                     float tau, uint32_t prev_mask, uint32_t *__restrict__ status)
 {
     const long long seg = blockIdx.y;
     const int s = blockIdx.x * blockDim.x + threadIdx.x;
@@ -211,7 +214,8 @@ __global__ void attn_fwd_simt_kernel(const T *__restrict__ x, const T *__restric
     const int bi = sv.Bk ? sv.Bk[i] : 0;
     float q[kDim], kv[kDim];
     load_row(X + (long long)i * kDim, q);
-    const Window w = window_of(s, m, L);
+    const bool prev = (prev_mask >> (seg % R)) & 1u;
+    const Window w = window_of(s, m, L, prev);
     float mx = -INFINITY;
     int cnt = 0;
     for (int t = w.w0; t < w.w1; ++t) {
@@ -224,7 +228,11 @@ __global__ void attn_fwd_simt_kernel(const T *__restrict__ x, const T *__restric
     }
     float acc[kDim];
     float lse_i;
-    if (cnt == 0) {                       // self is the only candidate
+    if (cnt == 0 && prev) {               // nothing in the previous chunk: no contribution
+        lse_i = -INFINITY;
+#pragma unroll
+        for (int k = 0; k < kDim; ++k) acc[k] = 0.f;
+    } else if (cnt == 0) {                // self is the only candidate
         lse_i = self_penalty ? kSelfPenalty : tau * (dot64(q, q) * IN[i]);
         load_row(V + (long long)i * kDim, acc);
     } else {
@@ -259,7 +267,7 @@ cudaError_t launch_attn_fwd_simt(const Problem &p, const void *x, const void *v,
     float tau = 1.0f / sqrtf((float)p.d);
     attn_fwd_simt_kernel<float><<<grid, 128, 0, st>>>(
         (const float *)x, (const float *)v, perm, invnorm, (p.flags & LSH_FLAG_BUCKET_MASK) ? bkt : nullptr, o_r,
-        lse, p.L, p.R, p.m, p.causal, (p.flags & LSH_FLAG_SELF_PENALTY) ? 1 : 0, tau, status);
+        lse, p.L, p.R, p.m, p.causal, (p.flags & LSH_FLAG_SELF_PENALTY) ? 1 : 0, tau, (uint32_t)p.prev_mask, status);
     return cudaGetLastError();
 }
 
@@ -268,7 +276,7 @@ cudaError_t launch_attn_fwd_simt(const Problem &p, const void *x, const void *v,
 // 16 threads per token, four features each.
 template <typename T, typename OT>
 __global__ void combine_kernel(const OT *__restrict__ o_r, const float *__restrict__ lse, T *__restrict__ out,
-                               long long tokens, int L, int R)
+                               float *__restrict__ lse_out, long long tokens, int L, int R)
 {
     long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
     long long tok = gid >> 4;
@@ -281,6 +289,7 @@ __global__ void combine_kernel(const OT *__restrict__ o_r, const float *__restri
     float ssum = 0.f;
     for (int r = 0; r < R; ++r) ssum += expf(lse[(bh * R + r) * L + i] - mx);
     float big = mx + logf(ssum);
+    if (lse_out && quad == 0) lse_out[tok] = big;
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
     for (int r = 0; r < R; ++r) {
         float wr = expf(lse[(bh * R + r) * L + i] - big);
@@ -299,7 +308,8 @@ __global__ void combine_kernel(const OT *__restrict__ o_r, const float *__restri
 // their memory latencies overlap; RMAX = 0 handles any R one round at a time.
 template <int RMAX>
 __global__ void combine_bf16_kernel(const __nv_bfloat16 *__restrict__ o_r, const float *__restrict__ lse,
-                                    __nv_bfloat16 *__restrict__ out, long long tokens, int L, int R)
+                                    __nv_bfloat16 *__restrict__ out, float *__restrict__ lse_out, long long tokens,
+                                    int L, int R)
 {
     long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
     long long tok = gid >> 3;
@@ -337,6 +347,7 @@ __global__ void combine_bf16_kernel(const __nv_bfloat16 *__restrict__ o_r, const
             ssum += w[r];
         }
         const float inv = 1.f / ssum;
+        if (lse_out && oct == 0) lse_out[tok] = mx + logf(ssum);
 #pragma unroll
         for (int r = 0; r < RMAX; ++r) accumulate(w[r] * inv, u[r]);
     } else {
@@ -345,6 +356,7 @@ __global__ void combine_bf16_kernel(const __nv_bfloat16 *__restrict__ o_r, const
         float ssum = 0.f;
         for (int r = 0; r < R; ++r) ssum += expf(lp[(long long)r * L] - mx);
         const float big = mx + logf(ssum);
+        if (lse_out && oct == 0) lse_out[tok] = big;
         for (int r = 0; r < R; ++r) accumulate(expf(lp[(long long)r * L] - big), orow[r * rstride]);
     }
     reinterpret_cast<uint4 *>(out + tok * kDim)[oct] =
@@ -353,25 +365,41 @@ __global__ void combine_bf16_kernel(const __nv_bfloat16 *__restrict__ o_r, const
 }
 
 cudaError_t launch_combine(const Problem &p, const void *o_r, bool o_r_bf16, const float *lse, void *out,
-                           cudaStream_t st)
+                           float *lse_out, cudaStream_t st)
 {
-    if (p.dtype == LSH_BF16 && o_r_bf16) {
+    if (p.dtype == LSH_BF16) {
+        if (!o_r_bf16) return cudaErrorInvalidValue;
         long long threads = p.tokens() * 8;
         const unsigned grid = (unsigned)((threads + 255) / 256);
         auto kern = p.R <= 4 ? combine_bf16_kernel<4> : p.R <= 8 ? combine_bf16_kernel<8> : combine_bf16_kernel<0>;
-        kern<<<grid, 256, 0, st>>>((const __nv_bfloat16 *)o_r, lse, (__nv_bfloat16 *)out, p.tokens(), p.L, p.R);
+        kern<<<grid, 256, 0, st>>>((const __nv_bfloat16 *)o_r, lse, (__nv_bfloat16 *)out, lse_out, p.tokens(), p.L,
+                                   p.R);
         return cudaGetLastError();
     }
+    if (o_r_bf16) return cudaErrorInvalidValue;
     long long threads = p.tokens() * 16;
     unsigned grid = (unsigned)((threads + 255) / 256);
-    if (p.dtype == LSH_F32) {
-        if (o_r_bf16) return cudaErrorInvalidValue;
-        combine_kernel<float, float><<<grid, 256, 0, st>>>((const float *)o_r, lse, (float *)out, p.tokens(), p.L,
-                                                           p.R);
-    } else {
-        combine_kernel<__nv_bfloat16, float><<<grid, 256, 0, st>>>((const float *)o_r, lse, (__nv_bfloat16 *)out,
-                                                                   p.tokens(), p.L, p.R);
-    }
+    combine_kernel<float, float><<<grid, 256, 0, st>>>((const float *)o_r, lse, (float *)out, lse_out, p.tokens(),
+                                                       p.L, p.R);
+    return cudaGetLastError();
+}
+
+// Slot orders of local attention: round 0 the positions in their own order,
+// round 1 (its following-chunk part) in reversed order, so that the previous
+// chunk of a slot there holds the following chunk of its position.
+__global__ void local_perm_kernel(int32_t *__restrict__ perm, long long n, int L, int R)
+{
+    const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;   // over BH * R * L
+    if (idx >= n) return;
+    const int s = (int)(idx % L);
+    const int r = (int)((idx / L) % R);
+    perm[idx] = r == 0 ? s : L - 1 - s;
+}
+
+cudaError_t launch_local_perm(const Problem &p, int32_t *perm, cudaStream_t st)
+{
+    const long long n = p.S() * p.L;
+    local_perm_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(perm, n, p.L, p.R);
     return cudaGetLastError();
 }
 
@@ -486,7 +514,7 @@ __global__ void attn_bwd_q_simt_kernel(const T *__restrict__ x, const T *__restr
                                        const uint16_t *__restrict__ bkt, const float *__restrict__ lse_all,
                                        const float *__restrict__ delta, uint8_t *__restrict__ self_only,
                                        float *__restrict__ dx_acc, int L, int R, int m, int causal,
-                                       int self_penalty, float tau, uint32_t *__restrict__ status)
+                                       int self_penalty, float tau, uint32_t prev_mask, uint32_t *__restrict__ status)
 {
     const long long seg = blockIdx.y;
     const int s = blockIdx.x * blockDim.x + threadIdx.x;
@@ -508,7 +536,8 @@ __global__ void attn_bwd_q_simt_kernel(const T *__restrict__ x, const T *__restr
 #pragma unroll
     for (int k = 0; k < kDim; ++k) dq[k] = 0.f;
     const float big = lse_all[bh * L + i], dl = delta[bh * L + i];
-    const Window w = window_of(s, m, L);
+    const bool prev = (prev_mask >> (seg % R)) & 1u;
+    const Window w = window_of(s, m, L, prev);
     int cnt = 0;
     for (int t = w.w0; t < w.w1; ++t) {
         int j;
@@ -523,7 +552,7 @@ __global__ void attn_bwd_q_simt_kernel(const T *__restrict__ x, const T *__restr
 #pragma unroll
         for (int k = 0; k < kDim; ++k) dq[k] = fmaf(dz * c, kv[k], dq[k]);
     }
-    if (cnt == 0 && !self_penalty) {
+    if (cnt == 0 && !self_penalty && !prev) {
         float pij = expf(tau * (dot64(q, q) * IN[i]) - big);
         load_row(V + (long long)i * kDim, kv);
         float dz = pij * (dot64(g, kv) - dl);
@@ -531,7 +560,7 @@ __global__ void attn_bwd_q_simt_kernel(const T *__restrict__ x, const T *__restr
 #pragma unroll
         for (int k = 0; k < kDim; ++k) dq[k] = dz * c * q[k];
     }
-    self_only[seg * L + s] = cnt == 0;
+    self_only[seg * L + s] = cnt == 0 && !prev;
     float *dst = dx_acc + (bh * L + i) * kDim;
 #pragma unroll
     for (int k = 0; k < kDim; ++k) atomicAdd(dst + k, dq[k]);
@@ -550,7 +579,8 @@ __global__ void attn_bwd_k_simt_kernel(const T *__restrict__ x, const T *__restr
                                        const uint16_t *__restrict__ bkt, const float *__restrict__ lse_all,
                                        const float *__restrict__ delta, const uint8_t *__restrict__ self_only,
                                        float *__restrict__ dx_acc, float *__restrict__ dv_acc, int L, int R, int m,
-                                       int causal, int self_penalty, float tau, uint32_t *__restrict__ status)
+                                       int causal, int self_penalty, float tau, uint32_t prev_mask,
+                                       uint32_t *__restrict__ status)
 {
     const long long seg = blockIdx.y;
     const int t = blockIdx.x * blockDim.x + threadIdx.x;
@@ -569,8 +599,11 @@ __global__ void attn_bwd_k_simt_kernel(const T *__restrict__ x, const T *__restr
 #pragma unroll
     for (int k = 0; k < kDim; ++k) { gk[k] = 0.f; dvj[k] = 0.f; }
     const float inj = IN[j];
+    // queries whose window holds slot t: chunks c and c + 1 (c = t / m), or only
+    // c + 1 when the window is the previous chunk alone
     const int c = t / m;
-    const int s0 = c * m, s1 = min((c + 2) * m, L);
+    const bool prev = (prev_mask >> (seg % R)) & 1u;
+    const int s0 = (prev ? c + 1 : c) * m, s1 = min((c + 2) * m, L);
     for (int s = s0; s < s1; ++s) {
         int i = P[s];
         if (!valid_pos(i, L, status)) continue;
@@ -622,10 +655,11 @@ cudaError_t launch_attn_bwd_simt(const Problem &p, const void *x, const void *v,
     const int pen = (p.flags & LSH_FLAG_SELF_PENALTY) ? 1 : 0;
     attn_bwd_q_simt_kernel<float><<<grid, 128, 0, st>>>((const float *)x, (const float *)v, (const float *)dout,
                                                         perm, invnorm, bk, lse_all, delta, self_only, dx_acc, p.L,
-                                                        p.R, p.m, p.causal, pen, tau, status);
+                                                        p.R, p.m, p.causal, pen, tau, (uint32_t)p.prev_mask, status);
     attn_bwd_k_simt_kernel<float><<<grid, 128, 0, st>>>((const float *)x, (const float *)v, (const float *)dout,
                                                         perm, invnorm, bk, lse_all, delta, self_only, dx_acc,
-                                                        dv_acc, p.L, p.R, p.m, p.causal, pen, tau, status);
+                                                        dv_acc, p.L, p.R, p.m, p.causal, pen, tau,
+                                                        (uint32_t)p.prev_mask, status);
     return cudaGetLastError();
 }
 

@@ -156,3 +156,19 @@ def test_flags_accepted_and_their_argument_rules(lib, flags):
         assert lib.lsh_attn_fwd_sorted(ctypes.byref(d), fake, fake, fake, fake, fake, fake, big, None) == -1
         assert lib.lsh_attn_bwd(ctypes.byref(d), fake, fake, None, fake, fake, fake, fake, fake, fake, fake, big,
                                 None) == -1
+
+
+def test_local_attention_argument_rules(lib):
+    """Local attention: one set of outputs (n_hashes 1), no bucket mask, one or
+    no following chunk; n_buckets is not used (fake pointers, never read)."""
+    fake = ctypes.c_void_p(1 << 20)
+    big = 1 << 40
+    ok = _desc(n_hashes=1, n_buckets=0)
+    assert lib.lsh_attn_local_workspace_size(ctypes.byref(ok), 1, 0) > 0
+    assert lib.lsh_attn_local_workspace_size(ctypes.byref(ok), 1, 1) > 0
+    assert lib.lsh_attn_local_fwd(ctypes.byref(_desc(n_hashes=2)), 1, fake, fake, fake, fake, fake, big, None) == -2
+    assert lib.lsh_attn_local_fwd(ctypes.byref(_desc(n_hashes=1, flags=1)), 1, fake, fake, fake, fake, fake, big,
+                                  None) == -1
+    assert lib.lsh_attn_local_fwd(ctypes.byref(ok), 2, fake, fake, fake, fake, fake, big, None) == -4
+    assert lib.lsh_attn_local_bwd(ctypes.byref(ok), 1, fake, fake, None, fake, fake, fake, fake, fake, big,
+                                  None) == -1
