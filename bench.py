@@ -395,7 +395,7 @@ def run_reference(args, w: synth.Workload, world: int = 1) -> dict:
     the measured time of one such sampled step; tokens/s counts sequence tokens
     as the metric does (a (batch, head) slice of Ls tokens is Ls / H of them)."""
     from oracle import oracle
-    cores = cpu_cores()
+    cores = cpu_cores() if args.ref_threads <= 0 else args.ref_threads
     n = max(1, min(cores, w.B * w.H))
     Ls = min(w.L, 4096)
     ws = w.replace(B=1, H=n, L=Ls)
@@ -437,6 +437,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ref-threads", type=int, default=0,
+                    help="--impl reference: OpenMP threads (0 = every host core the process may use)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

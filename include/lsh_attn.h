@@ -236,6 +236,31 @@ LSH_API lsh_status lsh_attn_local_bwd(const lsh_attn_desc *desc, int32_t chunks_
                                       const void *v, const void *out, const float *lse, const void *dout,
                                       void *dqk, void *dv, void *workspace, size_t ws_bytes, void *stream);
 
+/* Reversible residual block with LSH attention as its first function
+ * (paper note "Reformer", section "Reversible Residual Layers"):
+ *   forward   y1 = x1 + F(x2),  y2 = x2 + G(y1)
+ *   backward  from the OUTPUTS: x2 = y2 - G(y1), x1 = y1 - F(x2), so the
+ *             block's inputs need not be kept; gradients
+ *             dx1 = dy1 + J_G(y1)^T dy2,  dx2 = dy2 + J_F(x2)^T dx1.
+ * F(x2) is LSH attention with x2 as both the shared query-key and the value
+ * (hash, sort, chunked attention, round merge: the semantics of lsh_attn_fwd
+ * with this descriptor; R as there).  G is the token-wise layer
+ * G(u) = tanh(u Wg + bg), Wg [64, 64] row-major (input row, output column),
+ * bg [64], float32.  x1, x2, y1, y2, dy1, dy2, dx1, dx2 are float32 [B, H, L,
+ * 64] device buffers: the residual streams stay in fp32 so that the inverse
+ * recovers x2 to fp32 rounding and F hashes it into the same buckets; F runs
+ * in desc->dtype (x2 is rounded to it on the way in).  The backward returns
+ * the recovered inputs in x1, x2 and the input gradients in dx1, dx2 (no
+ * gradient for Wg, bg or R).  Workspace: lsh_rev_workspace_size() bytes,
+ * 256-byte aligned.  Errors as for lsh_attn_fwd / lsh_attn_bwd. */
+LSH_API size_t lsh_rev_workspace_size(const lsh_attn_desc *desc, int for_backward);
+LSH_API lsh_status lsh_rev_fwd(const lsh_attn_desc *desc, const float *x1, const float *x2, const void *R,
+                               const float *Wg, const float *bg, float *y1, float *y2, void *workspace,
+                               size_t ws_bytes, void *stream);
+LSH_API lsh_status lsh_rev_bwd(const lsh_attn_desc *desc, const float *y1, const float *y2, const float *dy1,
+                               const float *dy2, const void *R, const float *Wg, const float *bg, float *x1,
+                               float *x2, float *dx1, float *dx2, void *workspace, size_t ws_bytes, void *stream);
+
 /* Parity bookkeeping: the number of (row, round) pairs of the last hash
  * (lsh_attn_hash, or the hash inside lsh_attn_fwd / lsh_attn_bwd) whose two
  * largest entries of [x R_r ; -x R_r] differ by less than 1e-6 of the

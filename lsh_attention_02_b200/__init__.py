@@ -27,7 +27,8 @@ EXPORTED = ("lsh_attn_make_rotations", "lsh_attn_workspace_size", "lsh_attn_hash
             "lsh_attn_bwd", "lsh_attn_poll", "lsh_attn_selftest_timeout", "lsh_attn_trace_begin",
             "lsh_attn_trace_end", "lsh_attn_last_near_ties",
             "lsh_attn_status_str", "lsh_attn_last_error", "lsh_attn_abi_version",
-            "lsh_attn_local_workspace_size", "lsh_attn_local_fwd", "lsh_attn_local_bwd")
+            "lsh_attn_local_workspace_size", "lsh_attn_local_fwd", "lsh_attn_local_bwd",
+            "lsh_rev_workspace_size", "lsh_rev_fwd", "lsh_rev_bwd")
 
 STAGES = ("hash", "sort", "norms", "attn_fwd", "combine", "bwd_prep", "attn_bwd", "bwd_final")
 
@@ -70,6 +71,10 @@ def load_library(path: str = LIB_PATH):
     L.lsh_attn_local_workspace_size.restype = S
     L.lsh_attn_local_fwd.argtypes = [DP, ctypes.c_int32, P, P, P, P, P, S, P]
     L.lsh_attn_local_bwd.argtypes = [DP, ctypes.c_int32, P, P, P, P, P, P, P, P, S, P]
+    L.lsh_rev_workspace_size.argtypes = [DP, ctypes.c_int]
+    L.lsh_rev_workspace_size.restype = S
+    L.lsh_rev_fwd.argtypes = [DP, P, P, P, P, P, P, P, P, S, P]
+    L.lsh_rev_bwd.argtypes = [DP, P, P, P, P, P, P, P, P, P, P, P, P, S, P]
     L.lsh_attn_poll.argtypes = [P, P]
     L.lsh_attn_selftest_timeout.argtypes = [P, ctypes.c_int64, P]
     L.lsh_attn_trace_begin.argtypes = [ctypes.c_int32]
@@ -209,6 +214,30 @@ def lsh_attn_local_bwd(desc: Desc, chunks_after: int, qk, v, out, lse, dout, dqk
                                               _ptr(lse), _ptr(dout), _ptr(dqk), _ptr(dv), _ptr(ws), ws.numel(),
                                               _stream(qk)), "lsh_attn_local_bwd")
     return dqk, dv
+
+
+def rev_workspace(desc: Desc, for_backward: bool, device) -> torch.Tensor:
+    n = int(load_library().lsh_rev_workspace_size(ctypes.byref(desc), int(for_backward)))
+    if n == 0:
+        raise LshAttnError(-1, "lsh_rev_workspace_size", "invalid descriptor")
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def lsh_rev_fwd(desc: Desc, x1, x2, R, Wg, bg, y1, y2, ws=None):
+    """Reversible block forward: y1 = x1 + LSHAttn(x2, x2), y2 = x2 + tanh(y1 Wg + bg); fp32 streams."""
+    ws = ws if ws is not None else rev_workspace(desc, False, x1.device)
+    _check(load_library().lsh_rev_fwd(ctypes.byref(desc), _ptr(x1), _ptr(x2), _ptr(R), _ptr(Wg), _ptr(bg),
+                                       _ptr(y1), _ptr(y2), _ptr(ws), ws.numel(), _stream(x1)), "lsh_rev_fwd")
+    return y1, y2
+
+
+def lsh_rev_bwd(desc: Desc, y1, y2, dy1, dy2, R, Wg, bg, x1, x2, dx1, dx2, ws=None):
+    """Reversible block backward from the outputs: recovers x1, x2 and writes dx1, dx2."""
+    ws = ws if ws is not None else rev_workspace(desc, True, y1.device)
+    _check(load_library().lsh_rev_bwd(ctypes.byref(desc), _ptr(y1), _ptr(y2), _ptr(dy1), _ptr(dy2), _ptr(R),
+                                       _ptr(Wg), _ptr(bg), _ptr(x1), _ptr(x2), _ptr(dx1), _ptr(dx2), _ptr(ws),
+                                       ws.numel(), _stream(y1)), "lsh_rev_bwd")
+    return x1, x2, dx1, dx2
 
 
 def lsh_attn_poll(ws: torch.Tensor) -> int:

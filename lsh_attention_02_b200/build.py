@@ -10,7 +10,7 @@ CSRC = os.path.join(HERE, "csrc")
 ROOT = os.path.dirname(HERE)
 LIB = os.path.join(HERE, "liblsh_attn.so")
 SOURCES = ["api.cu", "simt.cu", "sort.cu", "hash_tc.cu", "attn_fwd_tc.cu", "attn_bwd_tc.cu", "selftest.cu",
-           "rotations.cu"]
+           "rotations.cu", "revblock.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-shared", "-Xcompiler", "-fPIC,-fvisibility=hidden",
          "--expt-relaxed-constexpr", "-I", os.path.join(ROOT, "include")]

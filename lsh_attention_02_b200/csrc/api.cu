@@ -173,6 +173,30 @@ static lsh_status run_attn_fwd(const Problem &p, const Choice &c, const void *qk
     return LSH_OK;
 }
 
+// prologue, attention backward and epilogue for a given permutation (shared by
+// lsh_attn_bwd and the reversible block)
+static lsh_status run_attn_bwd(const Problem &p, const Choice &c, const void *qk, const void *v, const void *out,
+                               const float *lse, const int32_t *perm, const void *dout, void *dqk, void *dv,
+                               const Workspace &w, cudaStream_t st)
+{
+    // the tensor-core backward computes the key norms from its gathered rows
+    if (!c.tc_attn)
+        LSH_TRY(staged(LSH_STAGE_NORMS, 1, st, [&] { return launch_invnorm(p, qk, w.invnorm, st); }), "key norms");
+    LSH_TRY(staged(LSH_STAGE_BWD_PREP, 1, st, [&] {
+                return launch_bwd_prep(p, lse, out, dout, w.lse_all, w.delta, w.dx_acc, w.dv_acc, st);
+            }), "backward prologue");
+    LSH_TRY(staged(LSH_STAGE_ATTN_BWD, c.tc_attn ? 1 : 2, st, [&] {
+                return c.tc_attn ? launch_attn_bwd_tc(p, qk, v, dout, perm, w.buckets, w.lse_all, w.delta, w.dx_acc,
+                                                      w.dv_acc, w.status, st)
+                                 : launch_attn_bwd_simt(p, qk, v, dout, perm, w.invnorm, w.buckets, w.lse_all,
+                                                        w.delta, w.self_only, w.dx_acc, w.dv_acc, w.status, st);
+            }), "attention backward");
+    LSH_TRY(staged(LSH_STAGE_BWD_FINAL, 1, st,
+                   [&] { return launch_bwd_finalize(p, w.dx_acc, w.dv_acc, dqk, dv, st); }),
+            "backward epilogue");
+    return LSH_OK;
+}
+
 }  // namespace lsh
 
 using namespace lsh;
@@ -326,22 +350,7 @@ lsh_status lsh_attn_bwd(const lsh_attn_desc *desc, const void *qk, const void *v
                                      : launch_hash_simt(p, qk, R, w.buckets, st);
                 }), "hash");
     }
-    // the tensor-core backward computes the key norms from its gathered rows
-    if (!c.tc_attn)
-        LSH_TRY(staged(LSH_STAGE_NORMS, 1, st, [&] { return launch_invnorm(p, qk, w.invnorm, st); }), "key norms");
-    LSH_TRY(staged(LSH_STAGE_BWD_PREP, 1, st, [&] {
-                return launch_bwd_prep(p, lse, out, dout, w.lse_all, w.delta, w.dx_acc, w.dv_acc, st);
-            }), "backward prologue");
-    LSH_TRY(staged(LSH_STAGE_ATTN_BWD, c.tc_attn ? 1 : 2, st, [&] {
-                return c.tc_attn ? launch_attn_bwd_tc(p, qk, v, dout, perm, w.buckets, w.lse_all, w.delta, w.dx_acc,
-                                                      w.dv_acc, w.status, st)
-                                 : launch_attn_bwd_simt(p, qk, v, dout, perm, w.invnorm, w.buckets, w.lse_all,
-                                                        w.delta, w.self_only, w.dx_acc, w.dv_acc, w.status, st);
-            }), "attention backward");
-    LSH_TRY(staged(LSH_STAGE_BWD_FINAL, 1, st,
-                   [&] { return launch_bwd_finalize(p, w.dx_acc, w.dv_acc, dqk, dv, st); }),
-            "backward epilogue");
-    return LSH_OK;
+    return run_attn_bwd(p, c, qk, v, out, lse, perm, dout, dqk, dv, w, st);
 }
 
 // ------------------------------------------------------------------ local attention
@@ -439,6 +448,111 @@ lsh_status lsh_attn_local_bwd(const lsh_attn_desc *desc, int32_t chunks_after, c
     LSH_TRY(staged(LSH_STAGE_BWD_FINAL, 1, st,
                    [&] { return launch_bwd_finalize(p, w.dx_acc, w.dv_acc, dqk, dv, st); }),
             "local backward epilogue");
+    return LSH_OK;
+}
+
+// ------------------------------------------------------------------ reversible block
+// Workspace of the reversible block: its own buffers, then one attention
+// workspace (forward, or the larger of forward and backward) at a 256-byte
+// boundary.
+struct RevPlan {
+    void *xa, *f, *da, *dqk, *dv;     // [T, 64] in the attention dtype
+    float *g;                         // [T, 64] fp32: G(y1)
+    float *lse;                       // [S, L]
+    int32_t *perm;                    // [S, L]
+    char *attn;                       // the attention workspace
+    size_t attn_bytes, bytes;
+};
+static RevPlan plan_rev(const Problem &p, const Choice &c, bool backward, char *base)
+{
+    RevPlan r{};
+    size_t off = 0;
+    auto take = [&](size_t n) -> char * {
+        char *ptr = base ? base + off : nullptr;
+        off = align_up(off + n, 256);
+        return ptr;
+    };
+    const size_t T = (size_t)p.tokens(), e = p.dtype == LSH_BF16 ? 2 : 4, S = (size_t)p.S(), L = (size_t)p.L;
+    r.xa = take(T * kDim * e);
+    r.f = take(T * kDim * e);
+    r.lse = (float *)take(S * L * sizeof(float));
+    r.perm = (int32_t *)take(S * L * sizeof(int32_t));
+    if (backward) {
+        r.g = (float *)take(T * kDim * sizeof(float));
+        r.da = take(T * kDim * e);
+        r.dqk = take(T * kDim * e);
+        r.dv = take(T * kDim * e);
+    }
+    const size_t af = plan_workspace(p, false, c.tc_attn, c.tc_hash, nullptr).bytes;
+    const size_t ab = backward ? plan_workspace(p, true, c.tc_attn, c.tc_hash, nullptr).bytes : 0;
+    r.attn_bytes = af > ab ? af : ab;
+    r.attn = take(r.attn_bytes);
+    r.bytes = off;
+    return r;
+}
+
+size_t lsh_rev_workspace_size(const lsh_attn_desc *desc, int for_backward)
+{
+    Problem p;
+    if (check_desc(desc, &p) != LSH_OK) return 0;
+    return plan_rev(p, choose(p), for_backward != 0, nullptr).bytes;
+}
+
+lsh_status lsh_rev_fwd(const lsh_attn_desc *desc, const float *x1, const float *x2, const void *R, const float *Wg,
+                       const float *bg, float *y1, float *y2, void *workspace, size_t ws_bytes, void *stream)
+{
+    Problem p;
+    lsh_status s;
+    if ((s = check_desc(desc, &p)) != LSH_OK) return s;
+    if ((s = check_envelope(p)) != LSH_OK) return s;
+    const Choice c = choose(p);
+    if ((s = check_ptrs({x1, x2, R, Wg, bg, y1, y2})) != LSH_OK) return s;
+    RevPlan r = plan_rev(p, c, false, nullptr);
+    if ((s = check_ws(workspace, ws_bytes, r.bytes)) != LSH_OK) return s;
+    r = plan_rev(p, c, false, (char *)workspace);
+    const Workspace w = plan_workspace(p, false, c.tc_attn, c.tc_hash, r.attn);
+    cudaStream_t st = (cudaStream_t)stream;
+    LSH_TRY(cudaMemsetAsync(w.status, 0, sizeof(uint32_t), st), "status reset");
+    LSH_TRY(launch_cast(p, x2, r.xa, st), "x2 to the attention dtype");
+    if ((s = run_hash_sort(p, c, r.xa, R, r.perm, w, st)) != LSH_OK) return s;
+    if ((s = run_attn_fwd(p, c, r.xa, r.xa, r.perm, r.f, r.lse, w, st)) != LSH_OK) return s;   // F(x2)
+    LSH_TRY(launch_axpy(p, x1, r.f, 1.f, y1, st), "y1 = x1 + F(x2)");
+    LSH_TRY(launch_g_forward(p, y1, Wg, bg, x2, y2, nullptr, st), "y2 = x2 + G(y1)");
+    return LSH_OK;
+}
+
+lsh_status lsh_rev_bwd(const lsh_attn_desc *desc, const float *y1, const float *y2, const float *dy1,
+                       const float *dy2, const void *R, const float *Wg, const float *bg, float *x1, float *x2,
+                       float *dx1, float *dx2, void *workspace, size_t ws_bytes, void *stream)
+{
+    Problem p;
+    lsh_status s;
+    if ((s = check_desc(desc, &p)) != LSH_OK) return s;
+    if ((s = check_envelope(p)) != LSH_OK) return s;
+    const Choice c = choose(p);
+    if ((s = check_ptrs({y1, y2, dy1, dy2, R, Wg, bg, x1, x2, dx1, dx2})) != LSH_OK) return s;
+    RevPlan r = plan_rev(p, c, true, nullptr);
+    if ((s = check_ws(workspace, ws_bytes, r.bytes)) != LSH_OK) return s;
+    r = plan_rev(p, c, true, (char *)workspace);
+    const Workspace wf = plan_workspace(p, false, c.tc_attn, c.tc_hash, r.attn);
+    const Workspace wb = plan_workspace(p, true, c.tc_attn, c.tc_hash, r.attn);
+    cudaStream_t st = (cudaStream_t)stream;
+    LSH_TRY(cudaMemsetAsync(wf.status, 0, sizeof(uint32_t), st), "status reset");
+    // inverse of the G half: x2 = y2 - G(y1); gradient into y1: dy1 + J_G(y1)^T dy2
+    LSH_TRY(launch_g_forward(p, y1, Wg, bg, nullptr, r.g, nullptr, st), "G(y1)");
+    LSH_TRY(launch_sub(p, y2, r.g, x2, st), "x2 = y2 - G(y1)");
+    LSH_TRY(launch_g_backward(p, r.g, dy2, Wg, dy1, dx1, st), "dx1 = dy1 + J_G^T dy2");
+    // inverse of the F half: F(x2) again (hash, sort, attention), x1 = y1 - F(x2)
+    LSH_TRY(launch_cast(p, x2, r.xa, st), "x2 to the attention dtype");
+    if ((s = run_hash_sort(p, c, r.xa, R, r.perm, wf, st)) != LSH_OK) return s;
+    if ((s = run_attn_fwd(p, c, r.xa, r.xa, r.perm, r.f, r.lse, wf, st)) != LSH_OK) return s;
+    LSH_TRY(launch_axpy(p, y1, r.f, -1.f, x1, st), "x1 = y1 - F(x2)");
+    // gradient through F, whose query-key and value inputs are both x2
+    LSH_TRY(launch_cast(p, dx1, r.da, st), "dF to the attention dtype");
+    // (the bucket ids of the forward above are still in place: the backward's
+    // workspace fields that precede the per-round outputs coincide with the forward's)
+    if ((s = run_attn_bwd(p, c, r.xa, r.xa, r.f, r.lse, r.perm, r.da, r.dqk, r.dv, wb, st)) != LSH_OK) return s;
+    LSH_TRY(launch_sum3(p, dy2, r.dqk, r.dv, dx2, st), "dx2 = dy2 + dF/dx2");
     return LSH_OK;
 }
 

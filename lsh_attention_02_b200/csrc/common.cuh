@@ -169,6 +169,16 @@ cudaError_t launch_bwd_finalize(const Problem &p, const float *dx_acc, const flo
 
 cudaError_t launch_wait_selftest(uint32_t *status, long long budget, cudaStream_t st);
 
+// Reversible block pieces (fp32 streams [tokens, 64]; `b`, `c` in the attention dtype).
+cudaError_t launch_g_forward(const Problem &p, const float *u, const float *W, const float *b, const float *res,
+                             float *out, float *g_out, cudaStream_t st);
+cudaError_t launch_g_backward(const Problem &p, const float *g, const float *dy, const float *W, const float *base,
+                              float *out, cudaStream_t st);
+cudaError_t launch_axpy(const Problem &p, const float *a, const void *b, float s, float *out, cudaStream_t st);
+cudaError_t launch_cast(const Problem &p, const float *a, void *out, cudaStream_t st);
+cudaError_t launch_sum3(const Problem &p, const float *a, const void *b, const void *c, float *out, cudaStream_t st);
+cudaError_t launch_sub(const Problem &p, const float *a, const float *b, float *out, cudaStream_t st);
+
 // Status bits written by kernels into Workspace::status.
 constexpr uint32_t kStatusTimeout = 1u;     // a bounded wait gave up
 constexpr uint32_t kStatusBadPerm = 2u;     // a permutation entry outside [0, L) was read (and ignored)

@@ -196,3 +196,36 @@ def local_bwd(x, v, dy, chunk, causal, before=1, after=1, self_penalty=False):
     _check(lib().oracle_local_bwd_batch(_p(x, _D), _p(v, _D), _p(dy, _D), B * H, L, d, int(chunk), int(before),
                                         int(after), int(causal), int(bool(self_penalty)), _p(dx, _D), _p(dv, _D)))
     return dx, dv
+
+
+def rev_g(u, Wg, bg):
+    """The reversible block's token-wise G(u) = tanh(u Wg + bg), float64."""
+    return np.tanh(_d(u) @ _d(Wg) + _d(bg))
+
+
+def rev_fwd(x1, x2, R, Wg, bg, n_buckets, chunk, causal, round_to=None):
+    """Reversible block ("Reformer" paper note, Reversible Residual Layers):
+    y1 = x1 + F(x2), y2 = x2 + G(y1), F = LSH attention with x2 as query-key and
+    value.  round_to: a function applied to x2 before F (the rounding to the
+    attention dtype), or None.  Returns y1, y2 and F's permutation."""
+    xa = _d(x2) if round_to is None else _d(round_to(x2))
+    f = fwd(xa, xa, R, n_buckets, chunk, causal)
+    y1 = _d(x1) + f["y"]
+    y2 = _d(x2) + rev_g(y1, Wg, bg)
+    return y1, y2, f["perm"]
+
+
+def rev_bwd(y1, y2, dy1, dy2, R, Wg, bg, n_buckets, chunk, causal, round_to=None):
+    """Backward from the outputs: x2 = y2 - G(y1), x1 = y1 - F(x2);
+    dx1 = dy1 + J_G(y1)^T dy2, dx2 = dy2 + J_F(x2)^T dx1 (F's two inputs are both
+    x2, so its query-key and value gradients add).  Returns x1, x2, dx1, dx2."""
+    y1 = _d(y1); y2 = _d(y2); dy1 = _d(dy1); dy2 = _d(dy2)
+    g = rev_g(y1, Wg, bg)
+    x2 = y2 - g
+    dx1 = dy1 + ((dy2 * (1.0 - g * g)) @ _d(Wg).T)
+    xa = x2 if round_to is None else _d(round_to(x2))
+    f = fwd(xa, xa, R, n_buckets, chunk, causal)
+    x1 = y1 - f["y"]
+    # F's output gradient enters F in its dtype, as the rounding of x2 does
+    dq, dv = bwd(xa, xa, dx1 if round_to is None else _d(round_to(dx1)), f["perm"], chunk, causal)
+    return x1, x2, dx1, dy2 + dq + dv

@@ -373,6 +373,46 @@ def test_local_attention_forward_backward(dtype, causal, after, L, chunk, flags)
     assert_close(to_host(dv), odv, dtype, "local dv")
 
 
+# ------------------------------------------------------------------ reversible residual block
+@pytest.mark.parametrize("dtype,causal,L", [("bf16", True, 1024), ("bf16", False, 576), ("f32", True, 512)])
+def test_reversible_block(dtype, causal, L):
+    """Reversible block ("Reformer", Reversible Residual Layers) with LSH
+    attention as F and G = tanh(u Wg + bg): outputs against the oracle; the
+    backward, run from the GPU's outputs, recovers the inputs (fp32 streams) and
+    its input gradients match the oracle's backward from the same outputs."""
+    nb, nh = 64, 2
+    w = small("long_64k", B=1, H=2, L=L, n_buckets=nb, n_hashes=nh, causal=causal, dtype=dtype, backward=True)
+    inp = synth.make_inputs(w)
+    rng = np.random.default_rng(5)
+    x1 = inp["v"].astype(np.float32); x2 = inp["x"].astype(np.float32)
+    Wg = (rng.standard_normal((64, 64)) / 8).astype(np.float32); bg = (0.1 * rng.standard_normal(64)).astype(np.float32)
+    dy1 = inp["dy"].astype(np.float32); dy2 = rng.standard_normal(x1.shape).astype(np.float32)
+
+    def dev(a):
+        return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).cuda()
+
+    R = to_dev(inp["R"], dtype)
+    desc = lsh.make_desc(1, 2, L, 64, nb, nh, 64, causal, torch_dtype(dtype))
+    X1, X2, W, Bg = dev(x1), dev(x2), dev(Wg), dev(bg)
+    Y1 = torch.empty_like(X1); Y2 = torch.empty_like(X1)
+    wsf = lsh.rev_workspace(desc, False, X1.device)
+    lsh.lsh_rev_fwd(desc, X1, X2, R, W, Bg, Y1, Y2, wsf)
+    rnd = synth.round_to_bf16 if dtype == "bf16" else None
+    y1, y2, _ = oracle.rev_fwd(x1, x2, inp["R"], Wg, bg, nb, 64, causal, round_to=rnd)
+    assert_close(to_host(Y1), y1, dtype, "y1")
+    assert_close(to_host(Y2), y2, dtype, "y2")
+    R1, R2, DX1, DX2 = (torch.empty_like(X1) for _ in range(4))
+    wsb = lsh.rev_workspace(desc, True, X1.device)
+    lsh.lsh_rev_bwd(desc, Y1, Y2, dev(dy1), dev(dy2), R, W, Bg, R1, R2, DX1, DX2, wsb)
+    assert lsh.lsh_attn_poll(wsf) == 0 and lsh.lsh_attn_poll(wsb) == 0
+    np.testing.assert_allclose(to_host(R2), x2, rtol=0, atol=2e-6)      # fp32 rounding of the residual adds
+    np.testing.assert_allclose(to_host(R1), x1, rtol=0, atol=2e-6)
+    _, _, odx1, odx2 = oracle.rev_bwd(to_host(Y1), to_host(Y2), dy1, dy2, inp["R"], Wg, bg, nb, 64, causal,
+                                      round_to=rnd)
+    assert_close(to_host(DX1), odx1, dtype, "dx1")
+    assert_close(to_host(DX2), odx2, dtype, "dx2")
+
+
 # ------------------------------------------------------------------ the five workloads
 def test_workload_tiny_f32():
     full_check(synth.WORKLOADS["tiny_f32"])
