@@ -81,6 +81,7 @@ Workspace plan_workspace(const Problem &p, bool backward, bool tc_attn, bool tc_
     } else {
         w.lse_all = (float *)take(T * sizeof(float));
         w.delta = (float *)take(T * sizeof(float));
+        w.own = (float *)take((p.flags & LSH_FLAG_SELF_PENALTY) ? T * sizeof(float) : 0);
         w.self_only = (uint8_t *)take(tc_attn ? 0 : S * L);
         w.dx_acc = (float *)take(T * kDim * sizeof(float));
         w.dv_acc = (float *)take(T * kDim * sizeof(float));
@@ -183,13 +184,14 @@ static lsh_status run_attn_bwd(const Problem &p, const Choice &c, const void *qk
     if (!c.tc_attn)
         LSH_TRY(staged(LSH_STAGE_NORMS, 1, st, [&] { return launch_invnorm(p, qk, w.invnorm, st); }), "key norms");
     LSH_TRY(staged(LSH_STAGE_BWD_PREP, 1, st, [&] {
-                return launch_bwd_prep(p, lse, out, dout, w.lse_all, w.delta, w.dx_acc, w.dv_acc, st);
+                return launch_bwd_prep(p, lse, out, dout, w.lse_all, w.delta,
+                                       (p.flags & LSH_FLAG_SELF_PENALTY) ? w.own : nullptr, w.dx_acc, w.dv_acc, st);
             }), "backward prologue");
     LSH_TRY(staged(LSH_STAGE_ATTN_BWD, c.tc_attn ? 1 : 2, st, [&] {
-                return c.tc_attn ? launch_attn_bwd_tc(p, qk, v, dout, perm, w.buckets, w.lse_all, w.delta, w.dx_acc,
-                                                      w.dv_acc, w.status, st)
+                return c.tc_attn ? launch_attn_bwd_tc(p, qk, v, dout, perm, w.buckets, w.lse_all, w.delta, w.own,
+                                                      w.dx_acc, w.dv_acc, w.status, st)
                                  : launch_attn_bwd_simt(p, qk, v, dout, perm, w.invnorm, w.buckets, w.lse_all,
-                                                        w.delta, w.self_only, w.dx_acc, w.dv_acc, w.status, st);
+                                                        w.delta, w.own, w.self_only, w.dx_acc, w.dv_acc, w.status, st);
             }), "attention backward");
     LSH_TRY(staged(LSH_STAGE_BWD_FINAL, 1, st,
                    [&] { return launch_bwd_finalize(p, w.dx_acc, w.dv_acc, dqk, dv, st); }),
@@ -437,13 +439,14 @@ lsh_status lsh_attn_local_bwd(const lsh_attn_desc *desc, int32_t chunks_after, c
     Problem p1 = p;
     p1.R = 1;
     LSH_TRY(staged(LSH_STAGE_BWD_PREP, 1, st, [&] {
-                return launch_bwd_prep(p1, lse, out, dout, w.lse_all, w.delta, w.dx_acc, w.dv_acc, st);
+                return launch_bwd_prep(p1, lse, out, dout, w.lse_all, w.delta,
+                                       (p.flags & LSH_FLAG_SELF_PENALTY) ? w.own : nullptr, w.dx_acc, w.dv_acc, st);
             }), "local backward prologue");
     LSH_TRY(staged(LSH_STAGE_ATTN_BWD, c.tc_attn ? 1 : 2, st, [&] {
-                return c.tc_attn ? launch_attn_bwd_tc(p, qk, v, dout, w.perm, nullptr, w.lse_all, w.delta, w.dx_acc,
-                                                      w.dv_acc, w.status, st)
+                return c.tc_attn ? launch_attn_bwd_tc(p, qk, v, dout, w.perm, nullptr, w.lse_all, w.delta, w.own,
+                                                      w.dx_acc, w.dv_acc, w.status, st)
                                  : launch_attn_bwd_simt(p, qk, v, dout, w.perm, w.invnorm, nullptr, w.lse_all,
-                                                        w.delta, w.self_only, w.dx_acc, w.dv_acc, w.status, st);
+                                                        w.delta, w.own, w.self_only, w.dx_acc, w.dv_acc, w.status, st);
             }), "local attention backward");
     LSH_TRY(staged(LSH_STAGE_BWD_FINAL, 1, st,
                    [&] { return launch_bwd_finalize(p, w.dx_acc, w.dv_acc, dqk, dv, st); }),

@@ -73,12 +73,12 @@ struct alignas(1024) Stage {
     alignas(16) int32_t qlim[kQ];   // causal: key bound, position + 1 when the query attends to itself alone;
                                     // otherwise: the one key position it does not take (-2: none)
     alignas(16) int32_t bk[256];    // bucket of slots [128k - 64, 128k + 192) (-1 if none); bucket mask only
+    alignas(16) float qown[kQ];     // self penalty: weight of the query's own entry when it is alone
     int32_t cmin[4];                // smallest position of chunks 2k-1 .. 2k+2 (INT_MAX if none)
 };
 
 // Optional readings (template parameter FL, bits of lsh_attn_desc.flags).
 constexpr int kMask = LSH_FLAG_BUCKET_MASK, kPen = LSH_FLAG_SELF_PENALTY;
-constexpr float kSelfPenalty = LSH_SELF_PENALTY_SCORE;
 
 struct BwdSmem {
     Stage st[kStages];
@@ -182,7 +182,8 @@ __device__ __forceinline__ void smem_chunk(const uint8_t *tile, int row, int ch,
 // One step of 16 query columns [C0 + 16 STEP, +16) of key row kr (position
 // kpos, bucket kb) from the S^T and dP^T values s, dp: P^T into TMEM, E^T into
 // shared memory.  With the self penalty, a lone query's own entry has the
-// constant score kSelfPenalty: its P uses that score and its E is 0.
+// constant score (LSH_SELF_PENALTY_SCORE): its P is exp(penalty - LSE), from the
+// prologue, which computes it without forming LSE, and its E is 0.
 template <bool CAUSAL, int FL, int STEP>
 __device__ __forceinline__ void key_row_step(const Stage &st, uint8_t (*ET)[kK * 128], uint32_t tl, int kr, int kpos,
                                              int kb, int C0, float sc, float ec, const float *s, const float *dp,
@@ -198,20 +199,21 @@ __device__ __forceinline__ void key_row_step(const Stage &st, uint8_t (*ET)[kK *
         const float4 qd4 = *reinterpret_cast<const float4 *>(&st.qdelta[q0]);
         const int4 qb4 = (FL & kMask) ? *reinterpret_cast<const int4 *>(&st.bk[64 + q0]) : make_int4(0, 0, 0, 0);
         const int4 qo4 = (FL & kPen) ? *reinterpret_cast<const int4 *>(&st.qpos[q0]) : make_int4(0, 0, 0, 0);
+        const float4 qw4 = (FL & kPen) ? *reinterpret_cast<const float4 *>(&st.qown[q0]) : make_float4(0, 0, 0, 0);
         const int qp[4] = {qp4.x, qp4.y, qp4.z, qp4.w};
         const float ql[4] = {ql4.x, ql4.y, ql4.z, ql4.w};
         const float qd[4] = {qd4.x, qd4.y, qd4.z, qd4.w};
         const int qb[4] = {qb4.x, qb4.y, qb4.z, qb4.w};
         const int qo[4] = {qo4.x, qo4.y, qo4.z, qo4.w};
+        const float qw[4] = {qw4.x, qw4.y, qw4.z, qw4.w};
         float pv[4], ev[4];
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
             bool ok = CAUSAL ? (kpos < qp[u]) : (kpos != qp[u]);
             if (FL & kMask) ok = ok && kb == qb[u];
             const bool own = (FL & kPen) && kpos == qo[u];
-            const float arg = own ? kSelfPenalty * kLog2e - ql[u] : fmaf(s[j4 + u], sc, -ql[u]);
-            const float e2 = tc::fast_exp2(arg);
-            pv[u] = ok ? e2 : 0.f;
+            const float e2 = tc::fast_exp2(fmaf(s[j4 + u], sc, -ql[u]));
+            pv[u] = ok ? (own ? qw[u] : e2) : 0.f;
             ev[u] = own ? 0.f : ec * pv[u] * (dp[j4 + u] - qd[u]);
             gx = fmaf(ev[u], s[j4 + u], gx);
         }
@@ -318,7 +320,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 attn_bwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__restrict__ v,
                    const __nv_bfloat16 *__restrict__ dout, const int32_t *__restrict__ perm,
                    const uint16_t *__restrict__ bkt, const float *__restrict__ lse_all,
-                   const float *__restrict__ delta, float *__restrict__ dx_acc, float *__restrict__ dv_acc, int L,
+                   const float *__restrict__ delta, const float *__restrict__ own, float *__restrict__ dx_acc,
+                   float *__restrict__ dv_acc, int L,
                    int R, long long n_units, float tau, uint32_t prev_mask, uint32_t *__restrict__ status)
 {
     extern __shared__ uint8_t smem_raw[];
@@ -397,7 +400,7 @@ attn_bwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
             // per-query LSE and delta: loads issued now, used after the copies are issued
             static_assert(kQ == 2 * kProducerThreads, "two queries per producer thread");
             int qp[2];
-            float ql[2], qd[2];
+            float ql[2], qd[2], qw[2] = {0.f, 0.f};
 #pragma unroll
             for (int j = 0; j < 2; ++j) {
                 const int q = min(ptid + j * kProducerThreads, kQ - 1);
@@ -405,6 +408,7 @@ attn_bwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
                 const long long rp = rowbase + max(qp[j], 0);
                 ql[j] = lse_all[rp];
                 qd[j] = delta[rp];
+                if (FL & kPen) qw[j] = own[rp];
             }
             // x, dY rows of the 192 query slots and v rows of the 128 key slots: thread t
             // copies chunk t % 8 of rows t / 8 + 12 j (zero fill for a missing slot)
@@ -460,6 +464,7 @@ attn_bwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
                     st.qpos[q] = p;
                     st.qlse2[q] = p >= 0 ? ql[j] * kLog2e : INFINITY;
                     st.qdelta[q] = p >= 0 ? qd[j] : 0.f;
+                    if (FL & kPen) st.qown[q] = p >= 0 ? qw[j] : 0.f;
                     st.qlim[q] = CAUSAL ? (lone ? p + 1 : p) : (lone ? -2 : p);
                 }
             }
@@ -692,8 +697,8 @@ attn_bwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
 
 template <bool CAUSAL, int FL>
 static cudaError_t launch_bwd(const Problem &p, const void *x, const void *v, const void *dout, const int32_t *perm,
-                              const uint16_t *bkt, const float *lse_all, const float *delta, float *dx_acc,
-                              float *dv_acc, uint32_t *status, cudaStream_t st)
+                              const uint16_t *bkt, const float *lse_all, const float *delta, const float *own,
+                              float *dx_acc, float *dv_acc, uint32_t *status, cudaStream_t st)
 {
     static_assert(sizeof(BwdSmem) + 1024 <= 232448, "shared memory per CTA");
     const size_t smem = sizeof(BwdSmem) + 1024;
@@ -706,18 +711,20 @@ static cudaError_t launch_bwd(const Problem &p, const void *x, const void *v, co
     const long long n_units = p.S() * (((p.L + kK - 1) / kK + kRun - 1) / kRun);
     const unsigned grid = (unsigned)std::min<long long>(n_units, (long long)sms);
     kern<<<grid, kThreads, smem, st>>>((const __nv_bfloat16 *)x, (const __nv_bfloat16 *)v,
-                                       (const __nv_bfloat16 *)dout, perm, bkt, lse_all, delta, dx_acc, dv_acc, p.L,
+                                       (const __nv_bfloat16 *)dout, perm, bkt, lse_all, delta, own, dx_acc, dv_acc,
+                                       p.L,
                                        p.R, n_units, 1.0f / sqrtf((float)p.d), (uint32_t)p.prev_mask, status);
     return cudaGetLastError();
 }
 
 cudaError_t launch_attn_bwd_tc(const Problem &p, const void *x, const void *v, const void *dout, const int32_t *perm,
-                               const uint16_t *bkt, const float *lse_all, const float *delta, float *dx_acc,
-                               float *dv_acc, uint32_t *status, cudaStream_t st)
+                               const uint16_t *bkt, const float *lse_all, const float *delta, const float *own,
+                               float *dx_acc, float *dv_acc, uint32_t *status, cudaStream_t st)
 {
     // key norms are computed in the kernel from the gathered rows
     const int fl = p.flags & (kMask | kPen);
-#define LSH_BWD_CASE(C, F) return launch_bwd<C, F>(p, x, v, dout, perm, bkt, lse_all, delta, dx_acc, dv_acc, status, st)
+#define LSH_BWD_CASE(C, F) \
+    return launch_bwd<C, F>(p, x, v, dout, perm, bkt, lse_all, delta, own, dx_acc, dv_acc, status, st)
     if (p.causal) {
         switch (fl) {
         case 0: LSH_BWD_CASE(true, 0);

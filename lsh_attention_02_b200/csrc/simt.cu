@@ -284,15 +284,17 @@ __global__ void combine_kernel(const OT *__restrict__ o_r, const float *__restri
     if (tok >= tokens) return;
     long long bh = tok / L;
     int i = (int)(tok % L);
+    // weights exp(lse_r - mx) / sum: computed relative to the largest lse, so that
+    // lse values far from 0 (the self penalty) lose no precision
     float mx = -INFINITY;
     for (int r = 0; r < R; ++r) mx = fmaxf(mx, lse[(bh * R + r) * L + i]);
     float ssum = 0.f;
     for (int r = 0; r < R; ++r) ssum += expf(lse[(bh * R + r) * L + i] - mx);
-    float big = mx + logf(ssum);
-    if (lse_out && quad == 0) lse_out[tok] = big;
+    if (lse_out && quad == 0) lse_out[tok] = mx + logf(ssum);
+    const float inv = 1.f / ssum;
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
     for (int r = 0; r < R; ++r) {
-        float wr = expf(lse[(bh * R + r) * L + i] - big);
+        float wr = expf(lse[(bh * R + r) * L + i] - mx) * inv;
         const OT *o = o_r + ((bh * R + r) * L + i) * kDim + quad * 4;
 #pragma unroll
         for (int k = 0; k < 4; ++k) acc[k] = fmaf(wr, to_f(o[k]), acc[k]);
@@ -355,9 +357,9 @@ __global__ void combine_bf16_kernel(const __nv_bfloat16 *__restrict__ o_r, const
         for (int r = 0; r < R; ++r) mx = fmaxf(mx, lp[(long long)r * L]);
         float ssum = 0.f;
         for (int r = 0; r < R; ++r) ssum += expf(lp[(long long)r * L] - mx);
-        const float big = mx + logf(ssum);
-        if (lse_out && oct == 0) lse_out[tok] = big;
-        for (int r = 0; r < R; ++r) accumulate(expf(lp[(long long)r * L] - big), orow[r * rstride]);
+        if (lse_out && oct == 0) lse_out[tok] = mx + logf(ssum);
+        const float inv = 1.f / ssum;
+        for (int r = 0; r < R; ++r) accumulate(expf(lp[(long long)r * L] - mx) * inv, orow[r * rstride]);
     }
     reinterpret_cast<uint4 *>(out + tok * kDim)[oct] =
         make_uint4(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]), pack_bf16x2(acc[4], acc[5]),
@@ -409,10 +411,13 @@ cudaError_t launch_local_perm(const Problem &p, int32_t *perm, cudaStream_t st)
 //
 // With P_rij = exp(z_rij - LSE_i) the merged output is y_i = sum_r,j P_rij v_j,
 // so the backward of every round uses P_rij and dz_rij = P_rij (dY_i.v_j - delta_i).
+// own (nullable, self penalty): the weight exp(kSelfPenalty - LSE_i) of a lone
+// query's own entry, as exp(kSelfPenalty - mx) / sum_r exp(lse_r - mx) (mx the
+// largest lse): LSE_i itself near -1e5 carries fp32 steps of 2^-7.
 template <typename T>
 __global__ void bwd_prep_kernel(const float *__restrict__ lse, const T *__restrict__ out, const T *__restrict__ dout,
-                                float *__restrict__ lse_all, float *__restrict__ delta, float *__restrict__ dx_acc,
-                                float *__restrict__ dv_acc, long long tokens, int L, int R)
+                                float *__restrict__ lse_all, float *__restrict__ delta, float *__restrict__ own,
+                                float *__restrict__ dx_acc, float *__restrict__ dv_acc, long long tokens, int L, int R)
 {
     long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
     long long tok = gid >> 4;
@@ -439,12 +444,13 @@ __global__ void bwd_prep_kernel(const float *__restrict__ lse, const T *__restri
         for (int r = 0; r < R; ++r) ssum += expf(lse[(bh * R + r) * L + i] - mx);
         lse_all[tok] = mx + logf(ssum);
         delta[tok] = part;
+        if (own) own[tok] = expf(kSelfPenalty - mx) / ssum;
     }
 }
 
 __global__ void bwd_prep_bf16_kernel(const float *__restrict__ lse, const __nv_bfloat16 *__restrict__ out,
                                      const __nv_bfloat16 *__restrict__ dout, float *__restrict__ lse_all,
-                                     float *__restrict__ delta, float *__restrict__ dx_acc,
+                                     float *__restrict__ delta, float *__restrict__ own, float *__restrict__ dx_acc,
                                      float *__restrict__ dv_acc, long long tokens, int L, int R)
 {
     long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
@@ -478,28 +484,24 @@ __global__ void bwd_prep_bf16_kernel(const float *__restrict__ lse, const __nv_b
         for (int r = 0; r < R; ++r) ssum += expf(lp[(long long)r * L] - mx);
         lse_all[tok] = mx + logf(ssum);
         delta[tok] = part;
+        if (own) own[tok] = expf(kSelfPenalty - mx) / ssum;
     }
 }
 
 cudaError_t launch_bwd_prep(const Problem &p, const float *lse, const void *out, const void *dout,
-                            float *lse_all, float *delta, float *dx_acc, float *dv_acc, cudaStream_t st)
+                            float *lse_all, float *delta, float *own, float *dx_acc, float *dv_acc, cudaStream_t st)
 {
     if (p.dtype == LSH_BF16) {
         long long threads = p.tokens() * 8;
         bwd_prep_bf16_kernel<<<(unsigned)((threads + 255) / 256), 256, 0, st>>>(
-            lse, (const __nv_bfloat16 *)out, (const __nv_bfloat16 *)dout, lse_all, delta, dx_acc, dv_acc,
+            lse, (const __nv_bfloat16 *)out, (const __nv_bfloat16 *)dout, lse_all, delta, own, dx_acc, dv_acc,
             p.tokens(), p.L, p.R);
         return cudaGetLastError();
     }
     long long threads = p.tokens() * 16;
     unsigned grid = (unsigned)((threads + 255) / 256);
-    if (p.dtype == LSH_F32)
-        bwd_prep_kernel<float><<<grid, 256, 0, st>>>(lse, (const float *)out, (const float *)dout, lse_all, delta,
-                                                     dx_acc, dv_acc, p.tokens(), p.L, p.R);
-    else
-        bwd_prep_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(lse, (const __nv_bfloat16 *)out,
-                                                             (const __nv_bfloat16 *)dout, lse_all, delta, dx_acc,
-                                                             dv_acc, p.tokens(), p.L, p.R);
+    bwd_prep_kernel<float><<<grid, 256, 0, st>>>(lse, (const float *)out, (const float *)dout, lse_all, delta, own,
+                                                 dx_acc, dv_acc, p.tokens(), p.L, p.R);
     return cudaGetLastError();
 }
 
@@ -577,7 +579,8 @@ template <typename T>
 __global__ void attn_bwd_k_simt_kernel(const T *__restrict__ x, const T *__restrict__ v, const T *__restrict__ dout,
                                        const int32_t *__restrict__ perm, const float *__restrict__ invnorm,
                                        const uint16_t *__restrict__ bkt, const float *__restrict__ lse_all,
-                                       const float *__restrict__ delta, const uint8_t *__restrict__ self_only,
+                                       const float *__restrict__ delta, const float *__restrict__ own,
+                                       const uint8_t *__restrict__ self_only,
                                        float *__restrict__ dx_acc, float *__restrict__ dv_acc, int L, int R, int m,
                                        int causal, int self_penalty, float tau, uint32_t prev_mask,
                                        uint32_t *__restrict__ status)
@@ -611,7 +614,7 @@ __global__ void attn_bwd_k_simt_kernel(const T *__restrict__ x, const T *__restr
             if (self_only[seg * L + s] == 0) continue;
             if (self_penalty) {
                 load_row(dout + (bh * L + i) * kDim, g);
-                const float pij = expf(kSelfPenalty - lse_all[bh * L + i]);
+                const float pij = own[bh * L + i];                // exp(kSelfPenalty - LSE_i)
 #pragma unroll
                 for (int k = 0; k < kDim; ++k) dvj[k] = fmaf(pij, g[k], dvj[k]);
                 continue;
@@ -645,8 +648,8 @@ __global__ void attn_bwd_k_simt_kernel(const T *__restrict__ x, const T *__restr
 
 cudaError_t launch_attn_bwd_simt(const Problem &p, const void *x, const void *v, const void *dout,
                                  const int32_t *perm, const float *invnorm, const uint16_t *bkt,
-                                 const float *lse_all, const float *delta, uint8_t *self_only, float *dx_acc,
-                                 float *dv_acc, uint32_t *status, cudaStream_t st)
+                                 const float *lse_all, const float *delta, const float *own, uint8_t *self_only,
+                                 float *dx_acc, float *dv_acc, uint32_t *status, cudaStream_t st)
 {
     if (p.dtype != LSH_F32) return cudaErrorInvalidValue;      // bf16 runs on the tensor-core kernels
     dim3 grid((p.L + 127) / 128, (unsigned)p.S());
@@ -657,7 +660,7 @@ cudaError_t launch_attn_bwd_simt(const Problem &p, const void *x, const void *v,
                                                         perm, invnorm, bk, lse_all, delta, self_only, dx_acc, p.L,
                                                         p.R, p.m, p.causal, pen, tau, (uint32_t)p.prev_mask, status);
     attn_bwd_k_simt_kernel<float><<<grid, 128, 0, st>>>((const float *)x, (const float *)v, (const float *)dout,
-                                                        perm, invnorm, bk, lse_all, delta, self_only, dx_acc,
+                                                        perm, invnorm, bk, lse_all, delta, own, self_only, dx_acc,
                                                         dv_acc, p.L, p.R, p.m, p.causal, pen, tau,
                                                         (uint32_t)p.prev_mask, status);
     return cudaGetLastError();

@@ -291,8 +291,9 @@ def test_permutation_entries_out_of_range_are_reported(dtype, L):
 def test_backward_run_to_run_drift_is_one_rounding_step():
     """The backward adds every round's gradient rows into fp32 accumulators with
     atomic vector reductions, so their summation order is not fixed.  Two runs on
-    the same inputs may differ only by the final rounding: elementwise at most
-    one bf16 step (2^-7 of the larger magnitude)."""
+    the same inputs may differ by the fp32 reassociation of those sums (about
+    1e-6 here) and by the final rounding to bf16: elementwise at most one bf16
+    step (2^-7 of the larger magnitude) plus 2^-16 absolute."""
     w = small("long_64k", B=1, H=2, L=8192, backward=True)
     inp = synth.make_inputs(w)
     a = Run(inp, w.n_buckets, w.chunk, w.causal, w.dtype)
@@ -300,9 +301,10 @@ def test_backward_run_to_run_drift_is_one_rounding_step():
     assert torch.equal(a.perm, b.perm) and torch.equal(a.out, b.out)
     for name, u, t in [("dqk", a.dx, b.dx), ("dv", a.dv, b.dv)]:
         u, t = to_host(u), to_host(t)
-        bound = 2.0 ** -7 * np.maximum(np.abs(u), np.abs(t))
+        bound = 2.0 ** -7 * np.maximum(np.abs(u), np.abs(t)) + 2.0 ** -16
         assert (np.abs(u - t) <= bound).all(), name
-        print(f"[drift] {name}: {(u != t).mean():.2e} of elements differ between two runs")
+        print(f"[drift] {name}: {(u != t).mean():.2e} of elements differ between two runs, "
+              f"largest difference {np.abs(u - t).max():.2e}")
 
 
 # ------------------------------------------------------------------ optional readings (flags)
