@@ -82,6 +82,7 @@ Workspace plan_workspace(const Problem &p, bool backward, bool tc_attn, bool tc_
         w.lse_all = (float *)take(T * sizeof(float));
         w.delta = (float *)take(T * sizeof(float));
         w.own = (float *)take((p.flags & LSH_FLAG_SELF_PENALTY) ? T * sizeof(float) : 0);
+        w.counters = (uint32_t *)take(tc_attn ? 2 * (size_t)p.BH() * sizeof(uint32_t) : 0);
         w.self_only = (uint8_t *)take(tc_attn ? 0 : S * L);
         w.dx_acc = (float *)take(T * kDim * sizeof(float));
         w.dv_acc = (float *)take(T * kDim * sizeof(float));
@@ -180,18 +181,28 @@ static lsh_status run_attn_bwd(const Problem &p, const Choice &c, const void *qk
                                const float *lse, const int32_t *perm, const void *dout, void *dqk, void *dv,
                                const Workspace &w, cudaStream_t st)
 {
-    // the tensor-core backward computes the key norms from its gathered rows
-    if (!c.tc_attn)
-        LSH_TRY(staged(LSH_STAGE_NORMS, 1, st, [&] { return launch_invnorm(p, qk, w.invnorm, st); }), "key norms");
+    float *own = (p.flags & LSH_FLAG_SELF_PENALTY) ? w.own : nullptr;
+    if (c.tc_attn) {
+        // the tensor-core backward zeroes its fp32 accumulators head by head and
+        // writes dqk, dv itself; the prologue only resets its per-head counters
+        LSH_TRY(staged(LSH_STAGE_BWD_PREP, 1, st, [&] {
+                    return launch_bwd_prep(p, lse, out, dout, w.lse_all, w.delta, own, nullptr, nullptr, w.counters,
+                                           2 * p.BH(), st);
+                }), "backward prologue");
+        LSH_TRY(staged(LSH_STAGE_ATTN_BWD, 1, st, [&] {
+                    return launch_attn_bwd_tc(p, qk, v, dout, perm, w.buckets, w.lse_all, w.delta, own, w.dx_acc,
+                                              w.dv_acc, dqk, dv, w.counters, w.status, st);
+                }), "attention backward");
+        return LSH_OK;
+    }
+    LSH_TRY(staged(LSH_STAGE_NORMS, 1, st, [&] { return launch_invnorm(p, qk, w.invnorm, st); }), "key norms");
     LSH_TRY(staged(LSH_STAGE_BWD_PREP, 1, st, [&] {
-                return launch_bwd_prep(p, lse, out, dout, w.lse_all, w.delta,
-                                       (p.flags & LSH_FLAG_SELF_PENALTY) ? w.own : nullptr, w.dx_acc, w.dv_acc, st);
+                return launch_bwd_prep(p, lse, out, dout, w.lse_all, w.delta, own, w.dx_acc, w.dv_acc, nullptr, 0,
+                                       st);
             }), "backward prologue");
-    LSH_TRY(staged(LSH_STAGE_ATTN_BWD, c.tc_attn ? 1 : 2, st, [&] {
-                return c.tc_attn ? launch_attn_bwd_tc(p, qk, v, dout, perm, w.buckets, w.lse_all, w.delta, w.own,
-                                                      w.dx_acc, w.dv_acc, w.status, st)
-                                 : launch_attn_bwd_simt(p, qk, v, dout, perm, w.invnorm, w.buckets, w.lse_all,
-                                                        w.delta, w.own, w.self_only, w.dx_acc, w.dv_acc, w.status, st);
+    LSH_TRY(staged(LSH_STAGE_ATTN_BWD, 2, st, [&] {
+                return launch_attn_bwd_simt(p, qk, v, dout, perm, w.invnorm, w.buckets, w.lse_all, w.delta, own,
+                                            w.self_only, w.dx_acc, w.dv_acc, w.status, st);
             }), "attention backward");
     LSH_TRY(staged(LSH_STAGE_BWD_FINAL, 1, st,
                    [&] { return launch_bwd_finalize(p, w.dx_acc, w.dv_acc, dqk, dv, st); }),
@@ -436,28 +447,32 @@ lsh_status lsh_attn_local_bwd(const lsh_attn_desc *desc, int32_t chunks_after, c
     if (!c.tc_attn)
         LSH_TRY(staged(LSH_STAGE_NORMS, 1, st, [&] { return launch_invnorm(p, qk, w.invnorm, st); }), "key norms");
     // lse holds the whole window's logsumexp already: the prologue's merge is over one set
+    float *own = (p.flags & LSH_FLAG_SELF_PENALTY) ? w.own : nullptr;
     Problem p1 = p;
     p1.R = 1;
     LSH_TRY(staged(LSH_STAGE_BWD_PREP, 1, st, [&] {
-                return launch_bwd_prep(p1, lse, out, dout, w.lse_all, w.delta,
-                                       (p.flags & LSH_FLAG_SELF_PENALTY) ? w.own : nullptr, w.dx_acc, w.dv_acc, st);
+                return c.tc_attn ? launch_bwd_prep(p1, lse, out, dout, w.lse_all, w.delta, own, nullptr, nullptr,
+                                                   w.counters, 2 * p.BH(), st)
+                                 : launch_bwd_prep(p1, lse, out, dout, w.lse_all, w.delta, own, w.dx_acc, w.dv_acc,
+                                                   nullptr, 0, st);
             }), "local backward prologue");
     LSH_TRY(staged(LSH_STAGE_ATTN_BWD, c.tc_attn ? 1 : 2, st, [&] {
-                return c.tc_attn ? launch_attn_bwd_tc(p, qk, v, dout, w.perm, nullptr, w.lse_all, w.delta, w.own,
-                                                      w.dx_acc, w.dv_acc, w.status, st)
+                return c.tc_attn ? launch_attn_bwd_tc(p, qk, v, dout, w.perm, nullptr, w.lse_all, w.delta, own,
+                                                      w.dx_acc, w.dv_acc, dqk, dv, w.counters, w.status, st)
                                  : launch_attn_bwd_simt(p, qk, v, dout, w.perm, w.invnorm, nullptr, w.lse_all,
-                                                        w.delta, w.own, w.self_only, w.dx_acc, w.dv_acc, w.status, st);
+                                                        w.delta, own, w.self_only, w.dx_acc, w.dv_acc, w.status, st);
             }), "local attention backward");
-    LSH_TRY(staged(LSH_STAGE_BWD_FINAL, 1, st,
-                   [&] { return launch_bwd_finalize(p, w.dx_acc, w.dv_acc, dqk, dv, st); }),
-            "local backward epilogue");
+    if (!c.tc_attn)
+        LSH_TRY(staged(LSH_STAGE_BWD_FINAL, 1, st,
+                       [&] { return launch_bwd_finalize(p, w.dx_acc, w.dv_acc, dqk, dv, st); }),
+                "local backward epilogue");
     return LSH_OK;
 }
 
 // ------------------------------------------------------------------ reversible block
-// Workspace of the reversible block: its own buffers, then one attention
-// workspace (forward, or the larger of forward and backward) at a 256-byte
-// boundary.
+// Workspace of the reversible block: one attention workspace first (forward,
+// or the larger of forward and backward; its status word at offset 0 is the one
+// lsh_attn_poll reads), then the block's own buffers at 256-byte boundaries.
 struct RevPlan {
     void *xa, *f, *da, *dqk, *dv;     // [T, 64] in the attention dtype
     float *g;                         // [T, 64] fp32: G(y1)
@@ -476,6 +491,10 @@ static RevPlan plan_rev(const Problem &p, const Choice &c, bool backward, char *
         return ptr;
     };
     const size_t T = (size_t)p.tokens(), e = p.dtype == LSH_BF16 ? 2 : 4, S = (size_t)p.S(), L = (size_t)p.L;
+    const size_t af = plan_workspace(p, false, c.tc_attn, c.tc_hash, nullptr).bytes;
+    const size_t ab = backward ? plan_workspace(p, true, c.tc_attn, c.tc_hash, nullptr).bytes : 0;
+    r.attn_bytes = af > ab ? af : ab;
+    r.attn = take(r.attn_bytes);
     r.xa = take(T * kDim * e);
     r.f = take(T * kDim * e);
     r.lse = (float *)take(S * L * sizeof(float));
@@ -486,10 +505,6 @@ static RevPlan plan_rev(const Problem &p, const Choice &c, bool backward, char *
         r.dqk = take(T * kDim * e);
         r.dv = take(T * kDim * e);
     }
-    const size_t af = plan_workspace(p, false, c.tc_attn, c.tc_hash, nullptr).bytes;
-    const size_t ab = backward ? plan_workspace(p, true, c.tc_attn, c.tc_hash, nullptr).bytes : 0;
-    r.attn_bytes = af > ab ? af : ab;
-    r.attn = take(r.attn_bytes);
     r.bytes = off;
     return r;
 }

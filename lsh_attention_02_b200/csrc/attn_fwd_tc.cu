@@ -143,7 +143,7 @@ __device__ __forceinline__ float softmax_sweep(const Stage &st, uint32_t tl, int
     for (int h = 0; h < 2; ++h) {
         if ((FIRST && BASE == 0 && h == 0) || (PREV && h == 1)) {   // missing chunk -1, or own chunk left out
 #pragma unroll
-            for (int c = 0; c < 4; ++c) tc::tmem_st8(tl + (uint32_t)(c * 8), z);
+            for (int c = 0; c < 4; ++c) tc::tmem_st8(tl + (uint32_t)(BASE / 2 + h * 32 + c * 8), z);
         } else {
             float v[64];
     #pragma unroll

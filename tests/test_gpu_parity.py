@@ -319,9 +319,13 @@ def test_flags_forward_backward(dtype, causal, flags, nb, L):
     ("Implementation Reading", same-token question): outputs, lse and both
     gradients against the oracle's readings, with the GPU's permutation and
     bucket ids.  Many queries have no same-bucket key in their window, so the
-    lone-query paths run often."""
+    lone-query paths run often.  With sparse buckets attention concentrates on
+    few keys and |dv| reaches 7, where bf16 output rounding alone costs 0.016 of
+    the 2e-2 absolute bound; dY is scaled by 1/4 (gradients are linear in it, the
+    relative bound is scale-free)."""
     w = small("long_64k", B=1, H=2, L=L, n_buckets=nb, n_hashes=2, causal=causal, dtype=dtype, backward=True)
     inp = synth.make_inputs(w)
+    inp["dy"] = (inp["dy"] / 4.0).astype(np.float32)           # exact: a power of two
     run = Run(inp, w.n_buckets, w.chunk, w.causal, w.dtype, flags)
     gb = run.host_buckets()
     gperm = run.perm.cpu().numpy()
