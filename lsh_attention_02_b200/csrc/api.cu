@@ -153,7 +153,7 @@ static lsh_status run_hash_sort(const Problem &p, const Choice &c, const void *q
                                  : launch_hash_simt(p, qk, R, w.buckets, st);
             }), "hash");
     LSH_TRY(launch_near_ties(p, qk, R, st), "near-tie count");
-    LSH_TRY(staged(LSH_STAGE_SORT, 3 * make_sort_plan(p.nb, p.L).passes, st,
+    LSH_TRY(staged(LSH_STAGE_SORT, sort_kernel_count(p), st,
                    [&] { return launch_sort(p, w.buckets, perm, w, st); }), "sort");
     return LSH_OK;
 }
@@ -261,7 +261,7 @@ lsh_status lsh_attn_sort(const lsh_attn_desc *desc, const uint16_t *buckets, int
     if ((s = check_ws(workspace, ws_bytes, w.bytes)) != LSH_OK) return s;
     w = plan_workspace(p, false, c.tc_attn, c.tc_hash, (char *)workspace);
     cudaStream_t st = (cudaStream_t)stream;
-    LSH_TRY(staged(LSH_STAGE_SORT, 3 * make_sort_plan(p.nb, p.L).passes, st,
+    LSH_TRY(staged(LSH_STAGE_SORT, sort_kernel_count(p), st,
                    [&] { return launch_sort(p, buckets, perm, w, st); }), "sort");
     return LSH_OK;
 }
@@ -290,7 +290,7 @@ lsh_status lsh_attn_sort_static(const lsh_attn_desc *desc, const uint16_t *bucke
     LSH_TRY(static_sort_scratch(&base), "lsh_attn_sort_static: scratch address");
     const Workspace w = plan_sort_scratch(p, (char *)base, nullptr);
     cudaStream_t st = (cudaStream_t)stream;
-    LSH_TRY(staged(LSH_STAGE_SORT, 3 * make_sort_plan(p.nb, p.L).passes, st,
+    LSH_TRY(staged(LSH_STAGE_SORT, sort_kernel_count(p), st,
                    [&] { return launch_sort(p, buckets, perm, w, st); }), "sort_static");
     return LSH_OK;
 }

@@ -38,6 +38,15 @@ struct SortPlan {
     int max_radix;
 };
 SortPlan make_sort_plan(int n_buckets, int L);
+// Segments this short with this few buckets are sorted on chip by one CTA.
+constexpr int kSegMaxL = 16384;
+constexpr int kSegMaxBuckets = 512;
+bool seg_sort_fits(const Problem &p);
+// Kernels one sort launches (for the stage trace).
+inline int sort_kernel_count(const Problem &p)
+{
+    return seg_sort_fits(p) ? 1 : 3 * make_sort_plan(p.nb, p.L).passes;
+}
 
 // ---------------------------------------------------------------- workspace
 struct Workspace {

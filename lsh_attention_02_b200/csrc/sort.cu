@@ -5,7 +5,9 @@
 // order, so the sort is stable.  Each (batch, head, round) segment of L
 // bucket ids is sorted independently.
 //
-// Least-significant-digit radix sort with at most two passes of <= 8 bits
+// Segments of up to kSegMaxL positions with up to kSegMaxBuckets buckets are
+// sorted by one CTA in shared memory (below).  Longer ones: a
+// least-significant-digit radix sort with at most two passes of <= 8 bits
 // (bucket ids have <= 16 bits).  Each pass is three kernels:
 //   count   per 2048-position tile, a shared-memory histogram of the digit;
 //           written digit-major: counts[seg][digit][tile];
@@ -151,9 +153,110 @@ radix_scatter_kernel(const uint16_t *__restrict__ keys_in, const int32_t *__rest
     }
 }
 
+// ------------------------------------------------------------ small segments
+// A segment of at most kSegMaxL positions and kSegMaxBuckets buckets is sorted
+// by one CTA entirely in shared memory: the bucket ids are staged, each warp
+// counts the ids of its own contiguous run of positions, one exclusive scan in
+// (bucket, warp) order gives every warp's first output slot per bucket, and each
+// warp places its run in position order (match_any ranks equal ids inside a
+// 32-position step), so the result is the stable sort.  An id >= n_buckets
+// (invalid input) is counted as n_buckets - 1, which keeps every access in
+// bounds.  The permutation is
+// assembled in shared memory and written out with coalesced stores.
+constexpr int kSegThreads = 1024;
+constexpr int kSegWarps = kSegThreads / 32;
+
+struct SegSortSmem {
+    uint16_t keys[kSegMaxL];
+    int32_t perm[kSegMaxL];
+    uint32_t wh[kSegMaxBuckets * kSegWarps];      // [bucket][warp]
+    uint32_t warp_tot[kSegWarps];
+};
+
+__global__ void __launch_bounds__(kSegThreads)
+seg_sort_kernel(const uint16_t *__restrict__ buckets, int32_t *__restrict__ perm, int L, int nb)
+{
+    extern __shared__ __align__(16) uint8_t seg_smem[];
+    SegSortSmem &sm = *reinterpret_cast<SegSortSmem *>(seg_smem);
+    const long long seg = blockIdx.x;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const uint32_t lt_mask = (1u << lane) - 1u;
+    const uint16_t *k = buckets + seg * L;
+    for (int e = threadIdx.x; e < L; e += kSegThreads) sm.keys[e] = k[e];
+    for (int e = threadIdx.x; e < nb * kSegWarps; e += kSegThreads) sm.wh[e] = 0;
+    __syncthreads();
+    const int run = (L + kSegWarps * 32 - 1) / (kSegWarps * 32) * 32;   // positions per warp, a multiple of 32
+    const int p0 = warp * run;
+    // A: per-warp counts of every bucket id, in position order
+    for (int it = 0; it < run; it += 32) {
+        const int pos = p0 + it + lane;
+        const bool valid = pos < L;
+        const uint32_t b = valid ? min((uint32_t)sm.keys[pos], (uint32_t)(nb - 1)) : 0xFFFFFFFFu;
+        const uint32_t peers = __match_any_sync(0xffffffffu, b);
+        if (valid && (peers & lt_mask) == 0) sm.wh[b * kSegWarps + warp] += __popc(peers);
+        __syncwarp();
+    }
+    __syncthreads();
+    // B: exclusive scan of wh in (bucket, warp) order; thread t scans a contiguous span
+    const int n = nb * kSegWarps, per = (n + kSegThreads - 1) / kSegThreads;
+    const int e0 = min(n, threadIdx.x * per), e1 = min(n, e0 + per);
+    uint32_t tot = 0;
+    for (int e = e0; e < e1; ++e) tot += sm.wh[e];
+    uint32_t incl = tot;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t t = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += t;
+    }
+    if (lane == 31) sm.warp_tot[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+        const uint32_t wv = sm.warp_tot[lane];
+        uint32_t wi = wv;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t t = __shfl_up_sync(0xffffffffu, wi, o);
+            if (lane >= o) wi += t;
+        }
+        sm.warp_tot[lane] = wi - wv;
+    }
+    __syncthreads();
+    uint32_t off = sm.warp_tot[warp] + incl - tot;
+    for (int e = e0; e < e1; ++e) {
+        const uint32_t c = sm.wh[e];
+        sm.wh[e] = off;
+        off += c;
+    }
+    __syncthreads();
+    // C: stable placement into shared memory, then coalesced copy out
+    for (int it = 0; it < run; it += 32) {
+        const int pos = p0 + it + lane;
+        const bool valid = pos < L;
+        const uint32_t b = valid ? min((uint32_t)sm.keys[pos], (uint32_t)(nb - 1)) : 0xFFFFFFFFu;
+        const uint32_t peers = __match_any_sync(0xffffffffu, b);
+        const uint32_t slot = valid ? sm.wh[b * kSegWarps + warp] + __popc(peers & lt_mask) : 0u;
+        __syncwarp();
+        if (valid && (peers & lt_mask) == 0) sm.wh[b * kSegWarps + warp] += __popc(peers);
+        __syncwarp();
+        if (valid) sm.perm[slot] = pos;
+    }
+    __syncthreads();
+    int32_t *out = perm + seg * L;
+    for (int e = threadIdx.x; e < L; e += kSegThreads) out[e] = sm.perm[e];
+}
+
+bool seg_sort_fits(const Problem &p) { return p.L <= kSegMaxL && p.nb <= kSegMaxBuckets; }
+
 cudaError_t launch_sort(const Problem &p, const uint16_t *buckets, int32_t *perm, const Workspace &ws,
                         cudaStream_t st)
 {
+    if (seg_sort_fits(p)) {
+        const size_t smem = sizeof(SegSortSmem);
+        cudaError_t e = cudaFuncSetAttribute(seg_sort_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        seg_sort_kernel<<<(unsigned)p.S(), kSegThreads, smem, st>>>(buckets, perm, p.L, p.nb);
+        return cudaGetLastError();
+    }
     const SortPlan sp = make_sort_plan(p.nb, p.L);
     const dim3 grid(sp.n_tiles, (unsigned)p.S());
     const uint16_t *kin = buckets;
@@ -190,9 +293,10 @@ Workspace plan_sort_scratch(const Problem &p, char *base, size_t *bytes)
     };
     const size_t S = (size_t)p.S(), L = (size_t)p.L;
     const SortPlan sp = make_sort_plan(p.nb, p.L);
-    w.sort_keys = (uint16_t *)take(sp.passes > 1 ? S * L * sizeof(uint16_t) : 0);
-    w.sort_vals = (int32_t *)take(sp.passes > 1 ? S * L * sizeof(int32_t) : 0);
-    w.sort_counts = (uint32_t *)take(S * (size_t)sp.max_radix * sp.n_tiles * sizeof(uint32_t));
+    const bool small = seg_sort_fits(p);                 // sorted on chip: no scratch
+    w.sort_keys = (uint16_t *)take(!small && sp.passes > 1 ? S * L * sizeof(uint16_t) : 0);
+    w.sort_vals = (int32_t *)take(!small && sp.passes > 1 ? S * L * sizeof(int32_t) : 0);
+    w.sort_counts = (uint32_t *)take(small ? 0 : S * (size_t)sp.max_radix * sp.n_tiles * sizeof(uint32_t));
     w.bytes = off;
     if (bytes) *bytes = off;
     return w;
