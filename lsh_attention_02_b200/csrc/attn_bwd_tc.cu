@@ -713,12 +713,14 @@ attn_bwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
                 if (half == 1) tc::mbar_arrive(&sm.gx_ready);
             }
             if (tid == 0) LSH_PHASE(1, 2, it, 3);
-            // the next tile's key norm while this tile's products run
+            // the next tile's key norm while this tile's products run -- only inside a work
+            // unit: the first stage of the next unit may wait on the producer's accumulator
+            // housekeeping, which can depend on this unit being finished
             have_next_kinv = false;
             {
                 TileIter nx = ti;
                 tile_advance(nx, R, n_k, n_runs);
-                if (nx.unit < n_units) {
+                if (nx.unit == ti.unit) {
                     const int s2 = (it + 1) % kStages;
                     if (!tc::mbar_wait(&sm.full[s2], (uint32_t)((it + 1) / kStages) & 1u, &sm.abort, status)) break;
                     next_kinv = key_inv_norm(sm.st[s2].X, kr);
