@@ -261,6 +261,28 @@ LSH_API lsh_status lsh_rev_bwd(const lsh_attn_desc *desc, const float *y1, const
                                const float *dy2, const void *R, const float *Wg, const float *bg, float *x1,
                                float *x2, float *dx1, float *dx2, void *workspace, size_t ws_bytes, void *stream);
 
+/* Forward, and backward when dout_h is given, on HOST buffers (the layouts of
+ * lsh_attn_fwd / lsh_attn_bwd; qk_h, v_h, R_h, dout_h in; out_h, lse_h
+ * (nullable), dqk_h, dv_h out).  The computation is that of lsh_attn_fwd
+ * followed by lsh_attn_bwd with the forward's permutation.  The (batch, head)
+ * slices are independent, so they are processed in chunks of heads_per_chunk
+ * consecutive slices (<= 0: about an eighth of B*H, at least 1) through two
+ * device slots in `scratch`: while one chunk is computed on streams[0], the
+ * next is copied in on streams[1] and the previous copied out on streams[2],
+ * so both copy directions overlap the kernels.  Host buffers should be
+ * page-locked for the copies to be asynchronous.  streams: three cudaStream_t
+ * (distinct for overlap; streams[0] is the one to synchronise: its work ends
+ * after the last copy out).  scratch: a device buffer of at least
+ * lsh_attn_step_host_scratch_size() bytes, 256-byte aligned; lsh_attn_poll
+ * on it reports the device status of the call.  Creates and destroys six CUDA
+ * events per call; allocates no memory. */
+LSH_API size_t lsh_attn_step_host_scratch_size(const lsh_attn_desc *desc, int32_t heads_per_chunk,
+                                               int with_backward);
+LSH_API lsh_status lsh_attn_step_host(const lsh_attn_desc *desc, int32_t heads_per_chunk, const void *qk_h,
+                                      const void *v_h, const void *R_h, const void *dout_h, void *out_h,
+                                      float *lse_h, void *dqk_h, void *dv_h, void *scratch, size_t scratch_bytes,
+                                      void *const *streams);
+
 /* Parity bookkeeping: the number of (row, round) pairs of the last hash
  * (lsh_attn_hash, or the hash inside lsh_attn_fwd / lsh_attn_bwd) whose two
  * largest entries of [x R_r ; -x R_r] differ by less than 1e-6 of the

@@ -28,7 +28,8 @@ EXPORTED = ("lsh_attn_make_rotations", "lsh_attn_workspace_size", "lsh_attn_hash
             "lsh_attn_trace_end", "lsh_attn_last_near_ties",
             "lsh_attn_status_str", "lsh_attn_last_error", "lsh_attn_abi_version",
             "lsh_attn_local_workspace_size", "lsh_attn_local_fwd", "lsh_attn_local_bwd",
-            "lsh_rev_workspace_size", "lsh_rev_fwd", "lsh_rev_bwd")
+            "lsh_rev_workspace_size", "lsh_rev_fwd", "lsh_rev_bwd",
+            "lsh_attn_step_host_scratch_size", "lsh_attn_step_host")
 
 STAGES = ("hash", "sort", "norms", "attn_fwd", "combine", "bwd_prep", "attn_bwd", "bwd_final")
 
@@ -75,6 +76,9 @@ def load_library(path: str = LIB_PATH):
     L.lsh_rev_workspace_size.restype = S
     L.lsh_rev_fwd.argtypes = [DP, P, P, P, P, P, P, P, P, S, P]
     L.lsh_rev_bwd.argtypes = [DP, P, P, P, P, P, P, P, P, P, P, P, P, S, P]
+    L.lsh_attn_step_host_scratch_size.argtypes = [DP, ctypes.c_int32, ctypes.c_int]
+    L.lsh_attn_step_host_scratch_size.restype = S
+    L.lsh_attn_step_host.argtypes = [DP, ctypes.c_int32, P, P, P, P, P, P, P, P, P, S, ctypes.POINTER(P)]
     L.lsh_attn_poll.argtypes = [P, P]
     L.lsh_attn_selftest_timeout.argtypes = [P, ctypes.c_int64, P]
     L.lsh_attn_trace_begin.argtypes = [ctypes.c_int32]
@@ -238,6 +242,26 @@ def lsh_rev_bwd(desc: Desc, y1, y2, dy1, dy2, R, Wg, bg, x1, x2, dx1, dx2, ws=No
                                        _ptr(Wg), _ptr(bg), _ptr(x1), _ptr(x2), _ptr(dx1), _ptr(dx2), _ptr(ws),
                                        ws.numel(), _stream(y1)), "lsh_rev_bwd")
     return x1, x2, dx1, dx2
+
+
+def step_host_scratch(desc: Desc, heads_per_chunk: int, with_backward: bool, device) -> torch.Tensor:
+    n = int(load_library().lsh_attn_step_host_scratch_size(ctypes.byref(desc), int(heads_per_chunk),
+                                                           int(with_backward)))
+    if n == 0:
+        raise LshAttnError(-1, "lsh_attn_step_host_scratch_size", "invalid descriptor")
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def lsh_attn_step_host(desc: Desc, qk_h, v_h, R_h, dout_h, out_h, lse_h, dqk_h, dv_h, scratch, streams,
+                       heads_per_chunk: int = 0):
+    """Forward (+ backward when dout_h is given) on host tensors (pinned for overlap),
+    pipelined per chunk of heads over three torch CUDA streams (compute, copy in,
+    copy out); synchronise on streams[0]."""
+    arr = (ctypes.c_void_p * 3)(*[s.cuda_stream for s in streams])
+    _check(load_library().lsh_attn_step_host(ctypes.byref(desc), int(heads_per_chunk), _ptr(qk_h), _ptr(v_h),
+                                              _ptr(R_h), _ptr(dout_h), _ptr(out_h), _ptr(lse_h), _ptr(dqk_h),
+                                              _ptr(dv_h), _ptr(scratch), scratch.numel(), arr),
+           "lsh_attn_step_host")
 
 
 def lsh_attn_poll(ws: torch.Tensor) -> int:

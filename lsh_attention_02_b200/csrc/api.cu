@@ -574,6 +574,163 @@ lsh_status lsh_rev_bwd(const lsh_attn_desc *desc, const float *y1, const float *
     return LSH_OK;
 }
 
+// ------------------------------------------------------------------ host-buffer pipeline
+// Forward (+ backward) on host buffers.  The (batch, head) slices are
+// independent, so they go in chunks of consecutive slices through two
+// device slots: while chunk i is computed, chunk i+1 is copied in and
+// chunk i-1 copied out, each on its own stream, so both copy directions and
+// the kernels overlap.  The rotations are copied once.
+struct HostPlan {
+    int chunk, n_chunks;
+    size_t R_bytes;
+    char *R;                          // device copy of the rotations
+    struct Slot {
+        char *ws;                     // attention workspace (fwd / bwd share it in turn)
+        void *x, *v, *dy, *out, *dqk, *dv;
+        float *lse;
+        int32_t *perm;
+    } slot[2];
+    size_t ws_bytes, bytes;
+};
+
+static HostPlan plan_host(const Problem &p, const Choice &c, int heads_per_chunk, bool bwd, char *base)
+{
+    HostPlan h{};
+    const long long BH = p.BH();
+    h.chunk = heads_per_chunk > 0 ? (int)std::min<long long>(heads_per_chunk, BH)
+                                  : (int)std::max<long long>(1, (BH + 7) / 8);
+    h.n_chunks = (int)((BH + h.chunk - 1) / h.chunk);
+    Problem pc = p;
+    pc.B = 1;
+    pc.H = h.chunk;
+    const size_t wf = plan_workspace(pc, false, c.tc_attn, c.tc_hash, nullptr).bytes;
+    const size_t wb = bwd ? plan_workspace(pc, true, c.tc_attn, c.tc_hash, nullptr).bytes : 0;
+    h.ws_bytes = std::max(wf, wb);
+    size_t off = 0;
+    auto take = [&](size_t n) -> char * {
+        char *ptr = base ? base + off : nullptr;
+        off = align_up(off + n, 256);
+        return ptr;
+    };
+    const size_t e = p.dtype == LSH_BF16 ? 2 : 4;
+    const size_t rows = (size_t)h.chunk * p.L, seg = (size_t)h.chunk * p.R * p.L;
+    for (int k = 0; k < 2; ++k) {
+        HostPlan::Slot &sl = h.slot[k];
+        sl.ws = take(h.ws_bytes);         // slot 0's status word is at offset 0
+        sl.x = take(rows * kDim * e);
+        sl.v = take(rows * kDim * e);
+        sl.dy = take(bwd ? rows * kDim * e : 0);
+        sl.out = take(rows * kDim * e);
+        sl.dqk = take(bwd ? rows * kDim * e : 0);
+        sl.dv = take(bwd ? rows * kDim * e : 0);
+        sl.lse = (float *)take(seg * sizeof(float));
+        sl.perm = (int32_t *)take(seg * sizeof(int32_t));
+    }
+    h.R_bytes = (size_t)p.R * kDim * (p.nb / 2) * e;
+    h.R = take(h.R_bytes);
+    h.bytes = off;
+    return h;
+}
+
+size_t lsh_attn_step_host_scratch_size(const lsh_attn_desc *desc, int32_t heads_per_chunk, int with_backward)
+{
+    Problem p;
+    if (check_desc(desc, &p) != LSH_OK) return 0;
+    return plan_host(p, choose(p), heads_per_chunk, with_backward != 0, nullptr).bytes;
+}
+
+lsh_status lsh_attn_step_host(const lsh_attn_desc *desc, int32_t heads_per_chunk, const void *qk_h, const void *v_h,
+                              const void *R_h, const void *dout_h, void *out_h, float *lse_h, void *dqk_h,
+                              void *dv_h, void *scratch, size_t scratch_bytes, void *const *streams)
+{
+    Problem p;
+    lsh_status s;
+    if ((s = check_desc(desc, &p)) != LSH_OK) return s;
+    if ((s = check_envelope(p)) != LSH_OK) return s;
+    const Choice c = choose(p);
+    if (!qk_h || !v_h || !R_h || !out_h || !streams) return LSH_ERR_ARG;
+    const bool bwd = dout_h != nullptr;
+    if (bwd && (!dqk_h || !dv_h)) return LSH_ERR_ARG;
+    HostPlan h = plan_host(p, c, heads_per_chunk, bwd, nullptr);
+    if ((s = check_ws(scratch, scratch_bytes, h.bytes)) != LSH_OK) return s;
+    h = plan_host(p, c, heads_per_chunk, bwd, (char *)scratch);
+    cudaStream_t cs = (cudaStream_t)streams[0], in_s = (cudaStream_t)streams[1], out_s = (cudaStream_t)streams[2];
+    const size_t e = p.dtype == LSH_BF16 ? 2 : 4;
+    const size_t slice = (size_t)p.L * kDim * e, seg = (size_t)p.R * p.L;
+    cudaEvent_t ev[2][3];                 // per slot: inputs landed, computed, outputs read
+    for (int k = 0; k < 2; ++k)
+        for (int j = 0; j < 3; ++j) {
+            cudaError_t er = cudaEventCreateWithFlags(&ev[k][j], cudaEventDisableTiming);
+            if (er != cudaSuccess) {
+                for (int kk = 0; kk <= k; ++kk)
+                    for (int jj = 0; jj < (kk < k ? 3 : j); ++jj) cudaEventDestroy(ev[kk][jj]);
+                return cuda_fail(er, "pipeline events");
+            }
+        }
+    lsh_status rc = LSH_OK;
+    auto fail = [&](cudaError_t er, const char *where) {
+        if (er != cudaSuccess && rc == LSH_OK) rc = cuda_fail(er, where);
+        return er != cudaSuccess;
+    };
+    // every slot's kernels report into slot 0's status word
+    uint32_t *status = (uint32_t *)h.slot[0].ws;
+    if (fail(cudaMemsetAsync(status, 0, sizeof(uint32_t), cs), "status reset")) goto done;
+    if (fail(cudaMemcpyAsync(h.R, R_h, h.R_bytes, cudaMemcpyHostToDevice, in_s), "rotations in")) goto done;
+    for (int i = 0; i < h.n_chunks && rc == LSH_OK; ++i) {
+        const int k = i & 1;
+        const HostPlan::Slot &sl = h.slot[k];
+        const long long bh0 = (long long)i * h.chunk;
+        const int nh = (int)std::min<long long>(h.chunk, p.BH() - bh0);
+        const size_t nb = (size_t)nh * slice;
+        // copy in (the slot's inputs are free once chunk i-2 is computed)
+        if (i >= 2 && fail(cudaStreamWaitEvent(in_s, ev[k][1], 0), "wait")) break;
+        if (fail(cudaMemcpyAsync(sl.x, (const char *)qk_h + bh0 * slice, nb, cudaMemcpyHostToDevice, in_s), "qk in") ||
+            fail(cudaMemcpyAsync(sl.v, (const char *)v_h + bh0 * slice, nb, cudaMemcpyHostToDevice, in_s), "v in"))
+            break;
+        if (bwd && fail(cudaMemcpyAsync(sl.dy, (const char *)dout_h + bh0 * slice, nb, cudaMemcpyHostToDevice, in_s),
+                        "dout in"))
+            break;
+        if (fail(cudaEventRecord(ev[k][0], in_s), "record")) break;
+        // compute (after the inputs, and after chunk i-2's outputs were read out)
+        if (fail(cudaStreamWaitEvent(cs, ev[k][0], 0), "wait")) break;
+        if (i >= 2 && fail(cudaStreamWaitEvent(cs, ev[k][2], 0), "wait")) break;
+        Problem pc = p;
+        pc.B = 1;
+        pc.H = nh;
+        Workspace wf = plan_workspace(pc, false, c.tc_attn, c.tc_hash, sl.ws);
+        wf.status = status;
+        if ((rc = run_hash_sort(pc, c, sl.x, h.R, sl.perm, wf, cs)) != LSH_OK) break;
+        if ((rc = run_attn_fwd(pc, c, sl.x, sl.v, sl.perm, sl.out, sl.lse, wf, cs)) != LSH_OK) break;
+        if (bwd) {
+            Workspace wb = plan_workspace(pc, true, c.tc_attn, c.tc_hash, sl.ws);
+            wb.status = status;
+            if ((rc = run_attn_bwd(pc, c, sl.x, sl.v, sl.out, sl.lse, sl.perm, sl.dy, sl.dqk, sl.dv, wb, cs)) !=
+                LSH_OK)
+                break;
+        }
+        if (fail(cudaEventRecord(ev[k][1], cs), "record")) break;
+        // copy out
+        if (fail(cudaStreamWaitEvent(out_s, ev[k][1], 0), "wait")) break;
+        if (fail(cudaMemcpyAsync((char *)out_h + bh0 * slice, sl.out, nb, cudaMemcpyDeviceToHost, out_s), "out"))
+            break;
+        if (lse_h && fail(cudaMemcpyAsync(lse_h + bh0 * seg, sl.lse, (size_t)nh * seg * sizeof(float),
+                                          cudaMemcpyDeviceToHost, out_s), "lse out"))
+            break;
+        if (bwd && (fail(cudaMemcpyAsync((char *)dqk_h + bh0 * slice, sl.dqk, nb, cudaMemcpyDeviceToHost, out_s),
+                         "dqk out") ||
+                    fail(cudaMemcpyAsync((char *)dv_h + bh0 * slice, sl.dv, nb, cudaMemcpyDeviceToHost, out_s),
+                         "dv out")))
+            break;
+        if (fail(cudaEventRecord(ev[k][2], out_s), "record")) break;
+    }
+    // the caller's stream (streams[0]) ends after the last copy out
+    if (rc == LSH_OK && h.n_chunks > 0) fail(cudaStreamWaitEvent(cs, ev[(h.n_chunks - 1) & 1][2], 0), "join");
+done:
+    for (int k = 0; k < 2; ++k)
+        for (int j = 0; j < 3; ++j) cudaEventDestroy(ev[k][j]);
+    return rc;
+}
+
 lsh_status lsh_attn_poll(void *workspace, void *stream)
 {
     if (!workspace) return LSH_ERR_ARG;

@@ -419,6 +419,39 @@ def test_reversible_block(dtype, causal, L):
     assert_close(to_host(DX2), odx2, dtype, "dx2")
 
 
+# ------------------------------------------------------------------ host-buffer pipeline
+@pytest.mark.parametrize("dtype,heads_per_chunk,bwd", [("bf16", 1, True), ("bf16", 3, True), ("bf16", 0, False),
+                                                       ("f32", 2, True)])
+def test_host_pipeline_matches_device_calls(dtype, heads_per_chunk, bwd):
+    """lsh_attn_step_host (host buffers, chunks of heads through two device slots
+    on three streams) gives what lsh_attn_fwd + lsh_attn_bwd give on device
+    buffers: the forward bit for bit (same kernels, same inputs), the gradients
+    within the bf16 bound (their fp32 sums are reassociated), and the oracle's
+    values."""
+    w = small("long_64k", B=2, H=3, L=1024, n_buckets=64, n_hashes=2, dtype=dtype, backward=True)
+    inp = synth.make_inputs(w)
+    run = Run(inp, w.n_buckets, w.chunk, w.causal, w.dtype)
+    tdt = torch_dtype(dtype)
+    host = {k: torch.from_numpy(inp[k]).to(tdt).pin_memory() for k in ("x", "v", "R", "dy")}
+    out_h = torch.empty_like(host["x"]).pin_memory()
+    lse_h = torch.empty(tuple(run.lse.shape), dtype=torch.float32).pin_memory()
+    dqk_h = torch.empty_like(host["x"]).pin_memory(); dv_h = torch.empty_like(host["x"]).pin_memory()
+    streams = [torch.cuda.Stream() for _ in range(3)]
+    scratch = lsh.step_host_scratch(run.desc, heads_per_chunk, bwd, run.x.device)
+    lsh.lsh_attn_step_host(run.desc, host["x"], host["v"], host["R"], host["dy"] if bwd else None, out_h, lse_h,
+                           dqk_h if bwd else None, dv_h if bwd else None, scratch, streams, heads_per_chunk)
+    streams[0].synchronize()
+    assert lsh.lsh_attn_poll(scratch) == 0
+    assert torch.equal(out_h, run.out.cpu()) and torch.equal(lse_h, run.lse.cpu())
+    if bwd:
+        assert_close(to_host(dqk_h), to_host(run.dx), dtype, "dqk host vs device")
+        assert_close(to_host(dv_h), to_host(run.dv), dtype, "dv host vs device")
+        gperm = run.perm.cpu().numpy()
+        dx, dv = oracle.bwd(inp["x"], inp["v"], inp["dy"], gperm, w.chunk, w.causal)
+        assert_close(to_host(dqk_h), dx, dtype, "dqk host vs oracle")
+        assert_close(to_host(dv_h), dv, dtype, "dv host vs oracle")
+
+
 # ------------------------------------------------------------------ the five workloads
 def test_workload_tiny_f32():
     full_check(synth.WORKLOADS["tiny_f32"])
