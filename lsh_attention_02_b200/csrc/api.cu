@@ -82,7 +82,6 @@ Workspace plan_workspace(const Problem &p, bool backward, bool tc_attn, bool tc_
         w.lse_all = (float *)take(T * sizeof(float));
         w.delta = (float *)take(T * sizeof(float));
         w.own = (float *)take((p.flags & LSH_FLAG_SELF_PENALTY) ? T * sizeof(float) : 0);
-        w.counters = (uint32_t *)take(tc_attn ? 2 * (size_t)p.BH() * sizeof(uint32_t) : 0);
         w.self_only = (uint8_t *)take(tc_attn ? 0 : S * L);
         w.dx_acc = (float *)take(T * kDim * sizeof(float));
         w.dv_acc = (float *)take(T * kDim * sizeof(float));
@@ -182,27 +181,17 @@ static lsh_status run_attn_bwd(const Problem &p, const Choice &c, const void *qk
                                const Workspace &w, cudaStream_t st)
 {
     float *own = (p.flags & LSH_FLAG_SELF_PENALTY) ? w.own : nullptr;
-    if (c.tc_attn) {
-        // the tensor-core backward zeroes its fp32 accumulators head by head and
-        // writes dqk, dv itself; the prologue only resets its per-head counters
-        LSH_TRY(staged(LSH_STAGE_BWD_PREP, 1, st, [&] {
-                    return launch_bwd_prep(p, lse, out, dout, w.lse_all, w.delta, own, nullptr, nullptr, w.counters,
-                                           2 * p.BH(), st);
-                }), "backward prologue");
-        LSH_TRY(staged(LSH_STAGE_ATTN_BWD, 1, st, [&] {
-                    return launch_attn_bwd_tc(p, qk, v, dout, perm, w.buckets, w.lse_all, w.delta, own, w.dx_acc,
-                                              w.dv_acc, dqk, dv, w.counters, w.status, st);
-                }), "attention backward");
-        return LSH_OK;
-    }
-    LSH_TRY(staged(LSH_STAGE_NORMS, 1, st, [&] { return launch_invnorm(p, qk, w.invnorm, st); }), "key norms");
+    // the tensor-core backward computes the key norms from its gathered rows
+    if (!c.tc_attn)
+        LSH_TRY(staged(LSH_STAGE_NORMS, 1, st, [&] { return launch_invnorm(p, qk, w.invnorm, st); }), "key norms");
     LSH_TRY(staged(LSH_STAGE_BWD_PREP, 1, st, [&] {
-                return launch_bwd_prep(p, lse, out, dout, w.lse_all, w.delta, own, w.dx_acc, w.dv_acc, nullptr, 0,
-                                       st);
+                return launch_bwd_prep(p, lse, out, dout, w.lse_all, w.delta, own, w.dx_acc, w.dv_acc, st);
             }), "backward prologue");
-    LSH_TRY(staged(LSH_STAGE_ATTN_BWD, 2, st, [&] {
-                return launch_attn_bwd_simt(p, qk, v, dout, perm, w.invnorm, w.buckets, w.lse_all, w.delta, own,
-                                            w.self_only, w.dx_acc, w.dv_acc, w.status, st);
+    LSH_TRY(staged(LSH_STAGE_ATTN_BWD, c.tc_attn ? 1 : 2, st, [&] {
+                return c.tc_attn ? launch_attn_bwd_tc(p, qk, v, dout, perm, w.buckets, w.lse_all, w.delta, own,
+                                                      w.dx_acc, w.dv_acc, w.status, st)
+                                 : launch_attn_bwd_simt(p, qk, v, dout, perm, w.invnorm, w.buckets, w.lse_all,
+                                                        w.delta, own, w.self_only, w.dx_acc, w.dv_acc, w.status, st);
             }), "attention backward");
     LSH_TRY(staged(LSH_STAGE_BWD_FINAL, 1, st,
                    [&] { return launch_bwd_finalize(p, w.dx_acc, w.dv_acc, dqk, dv, st); }),
@@ -451,21 +440,17 @@ lsh_status lsh_attn_local_bwd(const lsh_attn_desc *desc, int32_t chunks_after, c
     Problem p1 = p;
     p1.R = 1;
     LSH_TRY(staged(LSH_STAGE_BWD_PREP, 1, st, [&] {
-                return c.tc_attn ? launch_bwd_prep(p1, lse, out, dout, w.lse_all, w.delta, own, nullptr, nullptr,
-                                                   w.counters, 2 * p.BH(), st)
-                                 : launch_bwd_prep(p1, lse, out, dout, w.lse_all, w.delta, own, w.dx_acc, w.dv_acc,
-                                                   nullptr, 0, st);
+                return launch_bwd_prep(p1, lse, out, dout, w.lse_all, w.delta, own, w.dx_acc, w.dv_acc, st);
             }), "local backward prologue");
     LSH_TRY(staged(LSH_STAGE_ATTN_BWD, c.tc_attn ? 1 : 2, st, [&] {
                 return c.tc_attn ? launch_attn_bwd_tc(p, qk, v, dout, w.perm, nullptr, w.lse_all, w.delta, own,
-                                                      w.dx_acc, w.dv_acc, dqk, dv, w.counters, w.status, st)
+                                                      w.dx_acc, w.dv_acc, w.status, st)
                                  : launch_attn_bwd_simt(p, qk, v, dout, w.perm, w.invnorm, nullptr, w.lse_all,
                                                         w.delta, own, w.self_only, w.dx_acc, w.dv_acc, w.status, st);
             }), "local attention backward");
-    if (!c.tc_attn)
-        LSH_TRY(staged(LSH_STAGE_BWD_FINAL, 1, st,
-                       [&] { return launch_bwd_finalize(p, w.dx_acc, w.dv_acc, dqk, dv, st); }),
-                "local backward epilogue");
+    LSH_TRY(staged(LSH_STAGE_BWD_FINAL, 1, st,
+                   [&] { return launch_bwd_finalize(p, w.dx_acc, w.dv_acc, dqk, dv, st); }),
+            "local backward epilogue");
     return LSH_OK;
 }
 

@@ -315,116 +315,13 @@ __device__ __forceinline__ void tile_advance(TileIter &t, int R, int n_k, int n_
     }
 }
 
-// ------------------------------------------------------------------ accumulator housekeeping
-// The fp32 gradient accumulators of a head are zeroed by the producer warps of
-// every CTA (one chunk of rows each) shortly before the head's first work unit
-// and converted to the bf16 outputs right after its last, so that they live in
-// L2 in between: no separate zero-fill or conversion pass over HBM.  Per-head
-// counters order the steps across CTAs (all waits bounded):
-//   zdone[h]  chunks of head h zeroed            (target: gridDim.x)
-//   cdone[h]  work units of head h finished, counted per compute warp
-//             (target: units per head x compute warps)
-struct Housekeeping {
-    float *dx_acc, *dv_acc;
-    __nv_bfloat16 *dqk, *dv;
-    uint32_t *zdone, *cdone;
-    int L;
-    long long BH, units_per_head;
-};
-
-__device__ __forceinline__ uint32_t ld_acquire(const uint32_t *p)
-{
-    uint32_t v;
-    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-    return v;
-}
-
-// Bounded wait until *ctr >= target (thread 0 of the group spins; the others
-// learn the outcome at the group barrier).  False when it gave up or another
-// role of the CTA already did.
-__device__ __forceinline__ bool wait_count(const uint32_t *ctr, uint32_t target, int ptid, volatile int *abort,
-                                           uint32_t *status)
-{
-    bool fail = false;
-    if (ptid == 0) {
-        const long long t0 = clock64();
-        while (ld_acquire(ctr) < target) {
-            if (*abort) { fail = true; break; }
-            if (clock64() - t0 > tc::kWaitCycles) {
-                *abort = 1;
-                atomicOr(status, kStatusTimeout);
-                fail = true;
-                break;
-            }
-            __nanosleep(256);
-        }
-    }
-    fail = tc::named_bar_or(1, kProducerThreads, fail);
-    __threadfence();                                     // every thread's later accesses after the acquire
-    return !fail;
-}
-
-// This CTA's rows of head h: [h L + r0, h L + r1).
-__device__ __forceinline__ void chunk_rows(const Housekeeping &hk, long long h, long long &r0, long long &r1)
-{
-    const long long per = (hk.L + gridDim.x - 1) / gridDim.x;
-    r0 = h * hk.L + min((long long)hk.L, per * blockIdx.x);
-    r1 = h * hk.L + min((long long)hk.L, per * (blockIdx.x + 1));
-}
-
-__device__ __forceinline__ void zero_chunk(const Housekeeping &hk, long long h, int ptid)
-{
-    long long r0, r1;
-    chunk_rows(hk, h, r0, r1);
-    const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
-    float4 *ax = reinterpret_cast<float4 *>(hk.dx_acc + r0 * kDim);
-    float4 *av = reinterpret_cast<float4 *>(hk.dv_acc + r0 * kDim);
-    const long long n = (r1 - r0) * (kDim / 4);
-    for (long long e = ptid; e < n; e += kProducerThreads) {
-        ax[e] = z;
-        av[e] = z;
-    }
-    __threadfence();
-    tc::named_bar_sync(1, kProducerThreads);
-    if (ptid == 0) atomicAdd(hk.zdone + h, 1u);
-}
-
-// Converts this CTA's rows of head h to bf16 once every unit of the head is done,
-// then drops the fp32 lines from L2 without writing them back (their values are
-// no longer needed).
-__device__ __forceinline__ bool finalize_chunk(const Housekeeping &hk, long long h, int ptid, volatile int *abort,
-                                               uint32_t *status)
-{
-    if (!wait_count(hk.cdone + h, (uint32_t)(hk.units_per_head * kComputeWarps), ptid, abort, status)) return false;
-    long long r0, r1;
-    chunk_rows(hk, h, r0, r1);
-    const float4 *ax = reinterpret_cast<const float4 *>(hk.dx_acc + r0 * kDim);
-    const float4 *av = reinterpret_cast<const float4 *>(hk.dv_acc + r0 * kDim);
-    uint2 *ox = reinterpret_cast<uint2 *>(hk.dqk + r0 * kDim);
-    uint2 *ov = reinterpret_cast<uint2 *>(hk.dv + r0 * kDim);
-    const long long n = (r1 - r0) * (kDim / 4);
-    for (long long e = ptid; e < n; e += kProducerThreads) {
-        const float4 a = __ldcg(ax + e), b = __ldcg(av + e);
-        ox[e] = make_uint2(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w));
-        ov[e] = make_uint2(pack_bf16x2(b.x, b.y), pack_bf16x2(b.z, b.w));
-    }
-    tc::named_bar_sync(1, kProducerThreads);
-    const long long lines = (r1 - r0) * kDim * 4 / 128;
-    for (long long l = ptid; l < lines; l += kProducerThreads) {
-        asm volatile("discard.global.L2 [%0], 128;" ::"l"(hk.dx_acc + r0 * kDim + l * 32) : "memory");
-        asm volatile("discard.global.L2 [%0], 128;" ::"l"(hk.dv_acc + r0 * kDim + l * 32) : "memory");
-    }
-    return true;
-}
-
 template <bool CAUSAL, int FL>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_bwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__restrict__ v,
                    const __nv_bfloat16 *__restrict__ dout, const int32_t *__restrict__ perm,
                    const uint16_t *__restrict__ bkt, const float *__restrict__ lse_all,
                    const float *__restrict__ delta, const float *__restrict__ own, float *__restrict__ dx_acc,
-                   float *__restrict__ dv_acc, __nv_bfloat16 *__restrict__ dqk_out,
-                   __nv_bfloat16 *__restrict__ dv_out, uint32_t *__restrict__ counters, int L, long long BH,
+                   float *__restrict__ dv_acc, int L,
                    int R, long long n_units, float tau, uint32_t prev_mask, uint32_t *__restrict__ status)
 {
     extern __shared__ uint8_t smem_raw[];
@@ -432,7 +329,6 @@ attn_bwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int n_k = (L + kK - 1) / kK;          // the last tile may hold one chunk only
     const int n_runs = (n_k + kRun - 1) / kRun;
-    const Housekeeping hk{dx_acc, dv_acc, dqk_out, dv_out, counters, counters + BH, L, BH, (long long)n_runs * R};
 
     if (tid == 0) {
         for (int s = 0; s < kStages; ++s) {
@@ -480,25 +376,8 @@ attn_bwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
         };
         TileIter ti{blockIdx.x, 0};
         if (ti.unit < n_units) load_pos(ti);
-        long long zeroed = 0, finalized = 0, cur_head = -1;     // heads [0, zeroed) / [0, finalized) done here
         for (int it = 0; ti.unit < n_units; ++it) {
             const int s = it % kStages;
-            {
-                // first tile of a head: zero this CTA's chunk of every head a CTA may start
-                // soon, convert heads two or more behind, and wait until every chunk of this
-                // head is zero before its first stage is published (decisions are uniform
-                // over the producer group: they depend on the tile sequence only)
-                const long long head = tile_coord(ti, R, n_k, n_runs).bh;
-                if (head != cur_head) {
-                    cur_head = head;
-                    const long long zt = min(BH - 1, (ti.unit + (long long)gridDim.x) / hk.units_per_head + 1);
-                    for (; zeroed <= zt; ++zeroed) zero_chunk(hk, zeroed, ptid);
-                    bool good = true;
-                    for (; good && finalized <= head - 2; ++finalized)
-                        good = finalize_chunk(hk, finalized, ptid, &sm.abort, status);
-                    if (!good || !wait_count(hk.zdone + head, gridDim.x, ptid, &sm.abort, status)) break;
-                }
-            }
             if (ptid == 0) LSH_PHASE(1, 0, it, 0);
             bool ok = it < kStages ||
                       tc::mbar_wait(&sm.empty[s], (uint32_t)((it / kStages) - 1) & 1u, &sm.abort, status);
@@ -597,13 +476,6 @@ attn_bwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
             tc::fence_async_smem();
             tc::mbar_arrive(&sm.full[s]);
             if (ptid == 0) LSH_PHASE(1, 0, it, 4);
-        }
-        // the rest of the housekeeping: every chunk must be zeroed (other CTAs wait for
-        // it) before the remaining heads are converted; skipped once a wait gave up
-        if (!tc::named_bar_or(1, kProducerThreads, sm.abort != 0)) {
-            for (; zeroed < BH; ++zeroed) zero_chunk(hk, zeroed, ptid);
-            bool good = true;
-            for (; good && finalized < BH; ++finalized) good = finalize_chunk(hk, finalized, ptid, &sm.abort, status);
         }
     } else if (warp == kMmaWarp) {
         // ================= MMA issuer
@@ -713,14 +585,12 @@ attn_bwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
                 if (half == 1) tc::mbar_arrive(&sm.gx_ready);
             }
             if (tid == 0) LSH_PHASE(1, 2, it, 3);
-            // the next tile's key norm while this tile's products run -- only inside a work
-            // unit: the first stage of the next unit may wait on the producer's accumulator
-            // housekeeping, which can depend on this unit being finished
+            // the next tile's key norm while this tile's products run
             have_next_kinv = false;
             {
                 TileIter nx = ti;
                 tile_advance(nx, R, n_k, n_runs);
-                if (nx.unit == ti.unit) {
+                if (nx.unit < n_units) {
                     const int s2 = (it + 1) % kStages;
                     if (!tc::mbar_wait(&sm.full[s2], (uint32_t)((it + 1) / kStages) & 1u, &sm.abort, status)) break;
                     next_kinv = key_inv_norm(sm.st[s2].X, kr);
@@ -812,12 +682,6 @@ attn_bwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
                 tc::mbar_arrive(&sm.epi_done);
             }
             carry_in = tcd.next_adjacent;
-            if (!tcd.next_adjacent) {
-                // the unit's last tile: all its reductions are issued; count it for the head
-                __threadfence();
-                __syncwarp();
-                if (lane == 0) atomicAdd(hk.cdone + tcd.bh, 1u);
-            }
         }
     }
 
@@ -834,8 +698,7 @@ attn_bwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
 template <bool CAUSAL, int FL>
 static cudaError_t launch_bwd(const Problem &p, const void *x, const void *v, const void *dout, const int32_t *perm,
                               const uint16_t *bkt, const float *lse_all, const float *delta, const float *own,
-                              float *dx_acc, float *dv_acc, void *dqk, void *dv, uint32_t *counters,
-                              uint32_t *status, cudaStream_t st)
+                              float *dx_acc, float *dv_acc, uint32_t *status, cudaStream_t st)
 {
     static_assert(sizeof(BwdSmem) + 1024 <= 232448, "shared memory per CTA");
     const size_t smem = sizeof(BwdSmem) + 1024;
@@ -849,21 +712,19 @@ static cudaError_t launch_bwd(const Problem &p, const void *x, const void *v, co
     const unsigned grid = (unsigned)std::min<long long>(n_units, (long long)sms);
     kern<<<grid, kThreads, smem, st>>>((const __nv_bfloat16 *)x, (const __nv_bfloat16 *)v,
                                        (const __nv_bfloat16 *)dout, perm, bkt, lse_all, delta, own, dx_acc, dv_acc,
-                                       (__nv_bfloat16 *)dqk, (__nv_bfloat16 *)dv, counters, p.L, p.BH(),
+                                       p.L,
                                        p.R, n_units, 1.0f / sqrtf((float)p.d), (uint32_t)p.prev_mask, status);
     return cudaGetLastError();
 }
 
 cudaError_t launch_attn_bwd_tc(const Problem &p, const void *x, const void *v, const void *dout, const int32_t *perm,
                                const uint16_t *bkt, const float *lse_all, const float *delta, const float *own,
-                               float *dx_acc, float *dv_acc, void *dqk, void *dv, uint32_t *counters,
-                               uint32_t *status, cudaStream_t st)
+                               float *dx_acc, float *dv_acc, uint32_t *status, cudaStream_t st)
 {
     // key norms are computed in the kernel from the gathered rows
     const int fl = p.flags & (kMask | kPen);
 #define LSH_BWD_CASE(C, F) \
-    return launch_bwd<C, F>(p, x, v, dout, perm, bkt, lse_all, delta, own, dx_acc, dv_acc, dqk, dv, counters, status, \
-                            st)
+    return launch_bwd<C, F>(p, x, v, dout, perm, bkt, lse_all, delta, own, dx_acc, dv_acc, status, st)
     if (p.causal) {
         switch (fl) {
         case 0: LSH_BWD_CASE(true, 0);

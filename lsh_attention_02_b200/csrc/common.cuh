@@ -64,7 +64,6 @@ struct Workspace {
     float *delta;                     // [BH, L]  dY . Y
     float *own;                       // [BH, L]  penalised own entry's weight (self penalty only)
     uint8_t *self_only;               // [S, L]   per sorted slot
-    uint32_t *counters;               // [2 BH]   per-head progress of the tensor-core backward
     float *dx_acc;                    // [BH, L, 64]
     float *dv_acc;                    // [BH, L, 64]
     size_t bytes;
@@ -167,20 +166,17 @@ cudaError_t launch_combine(const Problem &p, const void *o_r, bool o_r_bf16, con
                            float *lse_out, cudaStream_t st);
 // Local attention's slot orders ([S, L]: round 0 identity, round 1 reversed).
 cudaError_t launch_local_perm(const Problem &p, int32_t *perm, cudaStream_t st);
-// own (nullable): the weight of a lone query's penalised own entry, [BH, L];
-// dx_acc / dv_acc (nullable): zero-filled when given; counters (nullable): the
-// first n_counters words are set to 0.
+// own (nullable): the weight of a lone query's penalised own entry, [BH, L]
 cudaError_t launch_bwd_prep(const Problem &p, const float *lse, const void *out, const void *dout,
-                            float *lse_all, float *delta, float *own, float *dx_acc, float *dv_acc,
-                            uint32_t *counters, long long n_counters, cudaStream_t st);
+                            float *lse_all, float *delta, float *own, float *dx_acc, float *dv_acc, cudaStream_t st);
 cudaError_t launch_attn_bwd_simt(const Problem &p, const void *x, const void *v, const void *dout,
                                  const int32_t *perm, const float *invnorm, const uint16_t *bkt,
                                  const float *lse_all, const float *delta, const float *own, uint8_t *self_only,
                                  float *dx_acc, float *dv_acc, uint32_t *status, cudaStream_t st);
 cudaError_t launch_attn_bwd_tc(const Problem &p, const void *x, const void *v, const void *dout,
                                const int32_t *perm, const uint16_t *bkt, const float *lse_all,
-                               const float *delta, const float *own, float *dx_acc, float *dv_acc, void *dqk,
-                               void *dv, uint32_t *counters, uint32_t *status, cudaStream_t st);
+                               const float *delta, const float *own, float *dx_acc, float *dv_acc, uint32_t *status,
+                               cudaStream_t st);
 cudaError_t launch_bwd_finalize(const Problem &p, const float *dx_acc, const float *dv_acc, void *dqk, void *dv,
                                 cudaStream_t st);
 

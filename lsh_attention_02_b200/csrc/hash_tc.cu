@@ -16,9 +16,9 @@
 //              the idle one of two A buffers, and one bulk copy per (round,
 //              N-tile) of the rotation tile, pre-transposed and pre-swizzled
 //              in global memory, into a 4-stage shared-memory ring;
-//   warp 17    MMA issuer: 4 K-steps per M-tile and N-tile (64 columns) into
-//              one of four TMEM accumulator buffers (the epilogue of tile t
-//              may run up to three tiles behind the MMAs), with a completion
+//   warp 17    MMA issuer: 4 K-steps per M-tile and N-tile into one of two
+//              TMEM accumulator buffers (double buffering lets the epilogue
+//              of tile t overlap the MMAs of tile t+1), with a completion
 //              barrier per M-tile so the two epilogue halves start apart and
 //              their ALU- and FMA-heavy passes overlap.
 //
@@ -35,19 +35,18 @@ namespace lsh {
 namespace {
 
 constexpr int kRows = 256;          // rows per block
-constexpr int kMaxNT = 64;          // widest N-tile
-constexpr int kAccBufs = 4;         // TMEM accumulator buffers (each 2 M-tiles x kMaxNT columns)
+constexpr int kMaxNT = 128;         // widest N-tile
 constexpr int kStages = 4;          // rotation-tile ring
 constexpr int kEpiWarps = 16;         // 4 lane quadrants x 2 M-tiles x 2 column halves
 constexpr int kThreads = (kEpiWarps + 2) * 32;
-constexpr int kTmemCols = 512;      // kAccBufs buffers x 2 M-tiles x kMaxNT
+constexpr int kTmemCols = 512;      // 2 buffers x 2 M-tiles x kMaxNT
 
 struct HashSmem {
     uint8_t A[2][kRows * 128];              // x rows of two row blocks, K-major SW128 (64 KB)
-    uint8_t B[kStages][kMaxNT * 128];       // rotation tiles (32 KB)
+    uint8_t B[kStages][kMaxNT * 128];       // rotation tiles (64 KB)
     uint64_t full[kStages], empty[kStages];
     uint64_t a_full[2], a_empty[2];
-    uint64_t acc_full[kAccBufs][2], acc_empty[kAccBufs];  // [buffer][M-tile]
+    uint64_t acc_full[2][2], acc_empty[2];  // [buffer][M-tile]
     float mbest[2][kRows];                  // upper column half's running best, by round parity
     int mbkt[2][kRows];                     // ... and its bucket
     uint64_t drain;                         // timeout path: the MMA issuer's last products
@@ -96,8 +95,6 @@ hash_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __nv_bfloat16 *__
         for (int b = 0; b < 2; ++b) {
             tc::mbar_init(&sm.a_full[b], 1);
             tc::mbar_init(&sm.a_empty[b], 1);
-        }
-        for (int b = 0; b < kAccBufs; ++b) {
             tc::mbar_init(&sm.acc_full[b][0], 1);
             tc::mbar_init(&sm.acc_full[b][1], 1);
             tc::mbar_init(&sm.acc_empty[b], kEpiWarps);
@@ -172,15 +169,12 @@ hash_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __nv_bfloat16 *__
                 for (int i = 0; i < items; ++i, ++it) {
                     const int s = it % kStages;
                     const uint32_t ph = (uint32_t)(it / kStages) & 1u;
-                    const int ab = it % kAccBufs;
-                    const uint32_t aph = (uint32_t)(it / kAccBufs) & 1u;
+                    const int ab = it & 1;
+                    const uint32_t aph = (uint32_t)(it >> 1) & 1u;
                     LSH_PHASE(0, 2, it, 0);
                     if (!tc::mbar_wait(&sm.full[s], ph, &sm.abort, status)) { ok = false; break; }
                     LSH_PHASE(0, 2, it, 1);
-                    if (it >= kAccBufs && !tc::mbar_wait(&sm.acc_empty[ab], aph ^ 1u, &sm.abort, status)) {
-                        ok = false;
-                        break;
-                    }
+                    if (it >= 2 && !tc::mbar_wait(&sm.acc_empty[ab], aph ^ 1u, &sm.abort, status)) { ok = false; break; }
                     LSH_PHASE(0, 2, it, 2);
                     tc::tc_fence_after();
                     const uint32_t b0 = tc::smem_u32(sm.B[s]);
@@ -216,8 +210,8 @@ hash_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __nv_bfloat16 *__
             float best = -INFINITY;
             int bucket = 0;
             for (int i = 0; i < items; ++i, ++it) {
-                const int ab = it % kAccBufs;
-                const uint32_t aph = (uint32_t)(it / kAccBufs) & 1u;
+                const int ab = it & 1;
+                const uint32_t aph = (uint32_t)(it >> 1) & 1u;
                 if (threadIdx.x == 0) LSH_PHASE(0, 0, it, 0);
                 if (!tc::mbar_wait(&sm.acc_full[ab][mt], aph, &sm.abort, status)) { ok = false; break; }
                 if (threadIdx.x == 0) LSH_PHASE(0, 0, it, 1);
@@ -356,11 +350,14 @@ cudaError_t launch_nt(const Problem &p, const void *x, const __nv_bfloat16 *Rs, 
     return cudaGetLastError();
 }
 
-// N-tile width: 64 when it divides n_buckets/2, else 32 with the last tile
-// padded by zero rotation columns.
+// N-tile width: the widest of 128, 96, 64 that divides n_buckets/2, else 32
+// with the last tile padded by zero rotation columns.
 int pick_nt(int half)
 {
-    return half % 64 == 0 ? 64 : 32;
+    if (half % 128 == 0) return 128;
+    if (half % 96 == 0) return 96;
+    if (half % 64 == 0) return 64;
+    return 32;
 }
 int padded_half(int half)
 {
@@ -391,8 +388,12 @@ cudaError_t launch_hash_tc(const Problem &p, const void *x, const void *R, uint1
                                                                         p.R);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    return pick_nt(half) == 64 ? launch_nt<64>(p, x, Rs, hp, buckets, status, st)
-                               : launch_nt<32>(p, x, Rs, hp, buckets, status, st);
+    switch (pick_nt(half)) {
+    case 128: return launch_nt<128>(p, x, Rs, hp, buckets, status, st);
+    case 96: return launch_nt<96>(p, x, Rs, hp, buckets, status, st);
+    case 64: return launch_nt<64>(p, x, Rs, hp, buckets, status, st);
+    default: return launch_nt<32>(p, x, Rs, hp, buckets, status, st);
+    }
 }
 
 }  // namespace lsh

@@ -417,25 +417,21 @@ cudaError_t launch_local_perm(const Problem &p, int32_t *perm, cudaStream_t st)
 template <typename T>
 __global__ void bwd_prep_kernel(const float *__restrict__ lse, const T *__restrict__ out, const T *__restrict__ dout,
                                 float *__restrict__ lse_all, float *__restrict__ delta, float *__restrict__ own,
-                                float *__restrict__ dx_acc, float *__restrict__ dv_acc, uint32_t *__restrict__ counters,
-                                long long n_counters, long long tokens, int L, int R)
+                                float *__restrict__ dx_acc, float *__restrict__ dv_acc, long long tokens, int L, int R)
 {
     long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
     long long tok = gid >> 4;
     int quad = (int)(gid & 15);
     bool valid = tok < tokens;
     float part = 0.f;
-    if (counters && gid < n_counters) counters[gid] = 0u;
     if (valid) {
         const T *y = out + tok * kDim + quad * 4;
         const T *g = dout + tok * kDim + quad * 4;
 #pragma unroll
         for (int k = 0; k < 4; ++k) part = fmaf(to_f(g[k]), to_f(y[k]), part);
-        if (dx_acc) {
-            float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
-            reinterpret_cast<float4 *>(dx_acc + tok * kDim)[quad] = z;
-            reinterpret_cast<float4 *>(dv_acc + tok * kDim)[quad] = z;
-        }
+        float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+        reinterpret_cast<float4 *>(dx_acc + tok * kDim)[quad] = z;
+        reinterpret_cast<float4 *>(dv_acc + tok * kDim)[quad] = z;
     }
 #pragma unroll
     for (int o = 8; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
@@ -455,15 +451,13 @@ __global__ void bwd_prep_kernel(const float *__restrict__ lse, const T *__restri
 __global__ void bwd_prep_bf16_kernel(const float *__restrict__ lse, const __nv_bfloat16 *__restrict__ out,
                                      const __nv_bfloat16 *__restrict__ dout, float *__restrict__ lse_all,
                                      float *__restrict__ delta, float *__restrict__ own, float *__restrict__ dx_acc,
-                                     float *__restrict__ dv_acc, uint32_t *__restrict__ counters,
-                                     long long n_counters, long long tokens, int L, int R)
+                                     float *__restrict__ dv_acc, long long tokens, int L, int R)
 {
     long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
     long long tok = gid >> 3;
     int oct = (int)(gid & 7);
     bool valid = tok < tokens;
     float part = 0.f;
-    if (counters && gid < n_counters) counters[gid] = 0u;
     if (valid) {
         const uint4 yu = reinterpret_cast<const uint4 *>(out + tok * kDim)[oct];
         const uint4 gu = reinterpret_cast<const uint4 *>(dout + tok * kDim)[oct];
@@ -473,12 +467,10 @@ __global__ void bwd_prep_bf16_kernel(const float *__restrict__ lse, const __nv_b
             part = fmaf(__uint_as_float(gw[e] << 16), __uint_as_float(yw[e] << 16), part);
             part = fmaf(__uint_as_float(gw[e] & 0xFFFF0000u), __uint_as_float(yw[e] & 0xFFFF0000u), part);
         }
-        if (dx_acc) {
-            const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
-            float4 *dxp = reinterpret_cast<float4 *>(dx_acc + tok * kDim) + 2 * oct;
-            float4 *dvp = reinterpret_cast<float4 *>(dv_acc + tok * kDim) + 2 * oct;
-            dxp[0] = z; dxp[1] = z; dvp[0] = z; dvp[1] = z;
-        }
+        const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+        float4 *dxp = reinterpret_cast<float4 *>(dx_acc + tok * kDim) + 2 * oct;
+        float4 *dvp = reinterpret_cast<float4 *>(dv_acc + tok * kDim) + 2 * oct;
+        dxp[0] = z; dxp[1] = z; dvp[0] = z; dvp[1] = z;
     }
 #pragma unroll
     for (int o = 4; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
@@ -497,20 +489,19 @@ __global__ void bwd_prep_bf16_kernel(const float *__restrict__ lse, const __nv_b
 }
 
 cudaError_t launch_bwd_prep(const Problem &p, const float *lse, const void *out, const void *dout,
-                            float *lse_all, float *delta, float *own, float *dx_acc, float *dv_acc,
-                            uint32_t *counters, long long n_counters, cudaStream_t st)
+                            float *lse_all, float *delta, float *own, float *dx_acc, float *dv_acc, cudaStream_t st)
 {
     if (p.dtype == LSH_BF16) {
-        long long threads = std::max(p.tokens() * 8, n_counters);
+        long long threads = p.tokens() * 8;
         bwd_prep_bf16_kernel<<<(unsigned)((threads + 255) / 256), 256, 0, st>>>(
             lse, (const __nv_bfloat16 *)out, (const __nv_bfloat16 *)dout, lse_all, delta, own, dx_acc, dv_acc,
-            counters, n_counters, p.tokens(), p.L, p.R);
+            p.tokens(), p.L, p.R);
         return cudaGetLastError();
     }
-    long long threads = std::max(p.tokens() * 16, n_counters);
+    long long threads = p.tokens() * 16;
     unsigned grid = (unsigned)((threads + 255) / 256);
     bwd_prep_kernel<float><<<grid, 256, 0, st>>>(lse, (const float *)out, (const float *)dout, lse_all, delta, own,
-                                                 dx_acc, dv_acc, counters, n_counters, p.tokens(), p.L, p.R);
+                                                 dx_acc, dv_acc, p.tokens(), p.L, p.R);
     return cudaGetLastError();
 }
 
