@@ -160,17 +160,17 @@ static lsh_status run_hash_sort(const Problem &p, const Choice &c, const void *q
 static lsh_status run_attn_fwd(const Problem &p, const Choice &c, const void *qk, const void *v,
                                const int32_t *perm, void *out, float *lse, const Workspace &w, cudaStream_t st)
 {
-    // the tensor-core forward computes the key norms from its gathered rows
-    if (!c.tc_attn)
-        LSH_TRY(staged(LSH_STAGE_NORMS, 1, st, [&] { return launch_invnorm(p, qk, w.invnorm, st); }), "key norms");
+    LSH_TRY(staged(LSH_STAGE_NORMS, 1, st, [&] { return launch_invnorm(p, qk, w.invnorm, st); }), "key norms");
     LSH_TRY(staged(LSH_STAGE_ATTN_FWD, 1, st, [&] {
                 return c.tc_attn
-                           ? launch_attn_fwd_tc(p, qk, v, perm, w.buckets, (__nv_bfloat16 *)w.o_r, lse, w.status, st)
+                           ? launch_attn_fwd_tc(p, qk, v, perm, w.buckets, w.invnorm, (__nv_bfloat16 *)w.o_r, lse,
+                                                w.status, st)
                            : launch_attn_fwd_simt(p, qk, v, perm, w.invnorm, w.buckets, (float *)w.o_r, lse,
                                                   w.status, st);
             }), "attention forward");
-    LSH_TRY(staged(LSH_STAGE_COMBINE, 1, st, [&] { return launch_combine(p, w.o_r, c.tc_attn, lse, out, nullptr, st); }),
-            "round merge");
+    LSH_TRY(staged(LSH_STAGE_COMBINE, 1, st, [&] {
+                return launch_combine(p, w.o_r, c.tc_attn, lse, out, nullptr, st);
+            }), "round merge");
     return LSH_OK;
 }
 
@@ -403,11 +403,10 @@ lsh_status lsh_attn_local_fwd(const lsh_attn_desc *desc, int32_t chunks_after, c
     LSH_TRY(cudaMemsetAsync(w.status, 0, sizeof(uint32_t), st), "status reset");
     LSH_TRY(launch_local_perm(p, w.perm, st), "local order");
     float *lse_rounds = p.R == 2 ? w.lse_r : lse;        // one part: its lse is the window's
-    if (!c.tc_attn)
-        LSH_TRY(staged(LSH_STAGE_NORMS, 1, st, [&] { return launch_invnorm(p, qk, w.invnorm, st); }), "key norms");
+    LSH_TRY(staged(LSH_STAGE_NORMS, 1, st, [&] { return launch_invnorm(p, qk, w.invnorm, st); }), "key norms");
     LSH_TRY(staged(LSH_STAGE_ATTN_FWD, 1, st, [&] {
-                return c.tc_attn ? launch_attn_fwd_tc(p, qk, v, w.perm, nullptr, (__nv_bfloat16 *)w.o_r, lse_rounds,
-                                                      w.status, st)
+                return c.tc_attn ? launch_attn_fwd_tc(p, qk, v, w.perm, nullptr, w.invnorm, (__nv_bfloat16 *)w.o_r,
+                                                      lse_rounds, w.status, st)
                                  : launch_attn_fwd_simt(p, qk, v, w.perm, w.invnorm, nullptr, (float *)w.o_r,
                                                         lse_rounds, w.status, st);
             }), "local attention forward");

@@ -11,7 +11,8 @@
 // Per tile:
 //   gather   rows x[perm[s]] and v[perm[s]] of the 192 window slots, copied
 //            straight into the 128-byte-swizzled layout the tensor core reads;
-//   norms    1/|x_j| of the window rows, from the gathered tile;
+//   norms    1/|x_j| of the window rows, gathered with the positions from
+//            the per-token norms of a pass before this kernel;
 //   S = Q K^T  tcgen05.mma M=128, N=192, K=64 into tensor memory (raw
 //            dot products x_i . x_j, bf16 in, fp32 accumulate);
 //   softmax  one query row per thread: s_ij = (x_i . x_j) / |x_j| / sqrt(d)
@@ -23,7 +24,8 @@
 //            S columns;
 //   O = P V  tcgen05.mma M=128, N=64, K=192 with A = P read from tensor
 //            memory and V read MN-major from shared memory;
-//   store    o_r and lse_r at the query's original position (the unsort).
+//   store    o_r and lse_r at the query's original position (the unsort),
+//            o_r rows staged in shared memory and written as whole lines.
 //
 // Scores satisfy s_ij <= tau |x_i| (Cauchy-Schwarz with unit keys), so the
 // softmax uses M = tau |x_i| in place of the row maximum: one sweep, no max
@@ -39,8 +41,9 @@
 //   warps 0-3, 4-7  two softmax groups working on alternate tiles, each with
 //                   its own 256 TMEM columns (S/P 192, O 64), so one group's
 //                   softmax overlaps the other's MMAs and stores;
-//   warps 8-10      producer: positions (loaded a tile ahead) and window
-//                   minima; x and v rows by 16-byte cp.async (eight threads
+//   warps 8-10      producer: positions and key norms (and, with the bucket
+//                   mask, buckets) loaded a tile ahead; x and v rows by
+//                   16-byte cp.async (eight threads
 //                   per row, zero fill for a missing slot) into a 4-stage
 //                   shared-memory ring; a stage is published once the next
 //                   stage's copies are in flight;
@@ -257,36 +260,12 @@ __device__ __forceinline__ void softmax_row(const Stage &st, uint32_t tl, int i,
     }
 }
 
-// Key norms of the window rows from the gathered x tile: sinv = tau log2(e) / |x_j|
-// and inv = 1 / |x_j| (0 for a zero or missing row), sum of squares in element
-// order with fused multiply-adds, as the norms kernel does.
-__device__ __forceinline__ void window_norms(Stage &st, int t, float sl2)
-{
-    for (int row = t; row < kW; row += 128) {
-        float ssq = 0.f;
-#pragma unroll
-        for (int ch = 0; ch < 8; ++ch) {
-            const uint4 u = *reinterpret_cast<const uint4 *>(st.X + row * 128 + ((ch ^ (row & 7)) << 4));
-            const uint32_t wd[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const float a = __uint_as_float(wd[e] << 16), b = __uint_as_float(wd[e] & 0xFFFF0000u);
-                ssq = fmaf(a, a, ssq);
-                ssq = fmaf(b, b, ssq);
-            }
-        }
-        const float nv = ssq > 0.f ? 1.0f / sqrtf(ssq) : 0.f;
-        st.inv[row] = nv;
-        st.sinv[row] = nv * sl2;
-    }
-}
-
 template <bool CAUSAL, int FL>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_fwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__restrict__ v,
-                   const int32_t *__restrict__ perm, const uint16_t *__restrict__ bkt, __nv_bfloat16 *__restrict__ o_r,
-                   float *__restrict__ lse, int L, int R, long long n_tiles, float tau, uint32_t prev_mask,
-                   uint32_t *__restrict__ status)
+                   const int32_t *__restrict__ perm, const uint16_t *__restrict__ bkt,
+                   const float *__restrict__ xinv, __nv_bfloat16 *__restrict__ o_r, float *__restrict__ lse,
+                   int L, int R, long long n_tiles, float tau, uint32_t prev_mask, uint32_t *__restrict__ status)
 {
     extern __shared__ uint8_t smem_raw[];
     FwdSmem &sm = *reinterpret_cast<FwdSmem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -322,6 +301,7 @@ attn_fwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
         // positions (and, with the bucket mask, buckets) of the next tile, loaded a
         // tile ahead (two slots per thread)
         int pn[2] = {-1, -1}, bn[2] = {-1, -1};
+        float nn[2] = {0.f, 0.f};                   // 1/|x| of those positions
         // A slot outside [0, L) (chunk -1, or the missing chunk of a last tile
         // when L % 128 == 64) is empty (-1); so is a permutation entry outside
         // [0, L), which is also reported in the status word.
@@ -339,6 +319,7 @@ attn_fwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
                 if (in && !good) atomicOr(status, kStatusBadPerm);
                 pn[j] = in && good ? pl : -1;
                 if (FL & kMask) bn[j] = pn[j] >= 0 ? (int)bkt[c.seg * L + pn[j]] : -1;
+                nn[j] = pn[j] >= 0 ? xinv[c.bh * L + pn[j]] : 0.f;
             }
         };
         if (blockIdx.x < n_tiles) load_pos(blockIdx.x);
@@ -355,6 +336,11 @@ attn_fwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
             const long long rowbase = tile_coord(tile, R, n_k).bh * L;
             st.pos[ptid] = pn[0];
             st.pos[ptid + kProducerThreads] = pn[1];
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                st.inv[ptid + j * kProducerThreads] = nn[j];
+                st.sinv[ptid + j * kProducerThreads] = nn[j] * sl2;
+            }
             if (FL & kMask) {
                 st.kb[ptid] = bn[0];
                 st.kb[ptid + kProducerThreads] = bn[1];
@@ -492,8 +478,6 @@ attn_fwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
             if (!tc::mbar_wait(&sm.full[s], (uint32_t)(it / kStages) & 1u, &sm.abort, status)) break;
             if (mark) LSH_PHASE(0, 2 + g, it, 1);
             Stage &st = sm.st[s];
-            window_norms(st, gt, sl2);
-            tc::named_bar_sync(2 + g, 128);
             if (!tc::mbar_wait(&sm.s_full[g], gph, &sm.abort, status)) break;
             if (mark) LSH_PHASE(0, 2 + g, it, 2);
             tc::tc_fence_after();
@@ -521,17 +505,35 @@ attn_fwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
             tc::tmem_ld_wait();
             tc::tc_fence_before();
             __syncwarp();
-            if (lane == 0) {
-                tc::mbar_arrive(&sm.o_free[g]);
-                tc::mbar_arrive(&sm.empty[s]);
-            }
+            if (lane == 0) tc::mbar_arrive(&sm.o_free[g]);
             const float rl = l > 0.f ? 1.0f / l : 0.f;        // no candidate (previous-chunk round): output 0
+            // o_r at the original positions: each warp stages its 32 rows (bf16, 16-byte
+            // chunks swizzled by row) in this stage's v tile, which no product reads any
+            // more, and stores them four rows per instruction, eight lanes per 128-byte
+            // row, so every store instruction writes four whole lines.
+            {
+                uint8_t *wst = st.V + q * 32 * 128;
 #pragma unroll
-            for (int d = 0; d < kDim; ++d) o[d] *= rl;
-            if (qpos >= 0) {                     // an empty query slot has no output
-                store_row(o_r + (tcd.seg * L + qpos) * kDim, o);
-                lse[tcd.seg * L + qpos] = row_lse;
+                for (int c = 0; c < 8; ++c)
+                    *reinterpret_cast<uint4 *>(wst + lane * 128 + ((c ^ (lane & 7)) << 4)) =
+                        make_uint4(pack_bf16x2(o[8 * c] * rl, o[8 * c + 1] * rl),
+                                   pack_bf16x2(o[8 * c + 2] * rl, o[8 * c + 3] * rl),
+                                   pack_bf16x2(o[8 * c + 4] * rl, o[8 * c + 5] * rl),
+                                   pack_bf16x2(o[8 * c + 6] * rl, o[8 * c + 7] * rl));
+                __syncwarp();
+                const int ch = lane & 7;
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    const int rr = 4 * k + (lane >> 3);
+                    const int p = __shfl_sync(0xffffffffu, qpos, rr);
+                    const uint4 u = *reinterpret_cast<const uint4 *>(wst + rr * 128 + ((ch ^ (rr & 7)) << 4));
+                    if (p >= 0)                  // an empty query slot has no output
+                        *reinterpret_cast<uint4 *>(o_r + (tcd.seg * L + p) * kDim + ch * 8) = u;
+                }
+                __syncwarp();
             }
+            if (qpos >= 0) lse[tcd.seg * L + qpos] = row_lse;
+            if (lane == 0) tc::mbar_arrive(&sm.empty[s]);
             if (mark) LSH_PHASE(0, 2 + g, it, 5);
         }
     }
@@ -553,7 +555,8 @@ bool attn_tc_supported(const Problem &p)
 
 template <bool CAUSAL, int FL>
 static cudaError_t launch_fwd(const Problem &p, const void *x, const void *v, const int32_t *perm,
-                              const uint16_t *bkt, __nv_bfloat16 *o_r, float *lse, uint32_t *status, cudaStream_t st)
+                              const uint16_t *bkt, const float *xinv, __nv_bfloat16 *o_r, float *lse,
+                              uint32_t *status, cudaStream_t st)
 {
     const size_t smem = sizeof(FwdSmem) + 1024;
     auto kern = attn_fwd_tc_kernel<CAUSAL, FL>;
@@ -564,30 +567,29 @@ static cudaError_t launch_fwd(const Problem &p, const void *x, const void *v, co
     if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
     const long long n_tiles = p.S() * ((p.L + kQ - 1) / kQ);
     const unsigned grid = (unsigned)std::min<long long>(n_tiles, (long long)sms);
-    kern<<<grid, kThreads, smem, st>>>((const __nv_bfloat16 *)x, (const __nv_bfloat16 *)v, perm, bkt, o_r, lse, p.L,
-                                       p.R, n_tiles, 1.0f / sqrtf((float)p.d), (uint32_t)p.prev_mask, status);
+    kern<<<grid, kThreads, smem, st>>>((const __nv_bfloat16 *)x, (const __nv_bfloat16 *)v, perm, bkt, xinv, o_r,
+                                       lse, p.L, p.R, n_tiles, 1.0f / sqrtf((float)p.d), (uint32_t)p.prev_mask, status);
     return cudaGetLastError();
 }
 
 cudaError_t launch_attn_fwd_tc(const Problem &p, const void *x, const void *v, const int32_t *perm,
-                               const uint16_t *bkt, __nv_bfloat16 *o_r, float *lse, uint32_t *status,
-                               cudaStream_t st)
+                               const uint16_t *bkt, const float *xinv, __nv_bfloat16 *o_r, float *lse,
+                               uint32_t *status, cudaStream_t st)
 {
-    // key norms are computed in the kernel from the gathered rows
     const int fl = p.flags & (kMask | kPen);
     if (p.causal) {
         switch (fl) {
-        case 0: return launch_fwd<true, 0>(p, x, v, perm, bkt, o_r, lse, status, st);
-        case kMask: return launch_fwd<true, kMask>(p, x, v, perm, bkt, o_r, lse, status, st);
-        case kPen: return launch_fwd<true, kPen>(p, x, v, perm, bkt, o_r, lse, status, st);
-        default: return launch_fwd<true, kMask | kPen>(p, x, v, perm, bkt, o_r, lse, status, st);
+        case 0: return launch_fwd<true, 0>(p, x, v, perm, bkt, xinv, o_r, lse, status, st);
+        case kMask: return launch_fwd<true, kMask>(p, x, v, perm, bkt, xinv, o_r, lse, status, st);
+        case kPen: return launch_fwd<true, kPen>(p, x, v, perm, bkt, xinv, o_r, lse, status, st);
+        default: return launch_fwd<true, kMask | kPen>(p, x, v, perm, bkt, xinv, o_r, lse, status, st);
         }
     }
     switch (fl) {
-    case 0: return launch_fwd<false, 0>(p, x, v, perm, bkt, o_r, lse, status, st);
-    case kMask: return launch_fwd<false, kMask>(p, x, v, perm, bkt, o_r, lse, status, st);
-    case kPen: return launch_fwd<false, kPen>(p, x, v, perm, bkt, o_r, lse, status, st);
-    default: return launch_fwd<false, kMask | kPen>(p, x, v, perm, bkt, o_r, lse, status, st);
+    case 0: return launch_fwd<false, 0>(p, x, v, perm, bkt, xinv, o_r, lse, status, st);
+    case kMask: return launch_fwd<false, kMask>(p, x, v, perm, bkt, xinv, o_r, lse, status, st);
+    case kPen: return launch_fwd<false, kPen>(p, x, v, perm, bkt, xinv, o_r, lse, status, st);
+    default: return launch_fwd<false, kMask | kPen>(p, x, v, perm, bkt, xinv, o_r, lse, status, st);
     }
 }
 

@@ -157,9 +157,10 @@ cudaError_t launch_sort(const Problem &p, const uint16_t *buckets, int32_t *perm
 cudaError_t launch_attn_fwd_simt(const Problem &p, const void *x, const void *v, const int32_t *perm,
                                  const float *invnorm, const uint16_t *bkt, float *o_r, float *lse,
                                  uint32_t *status, cudaStream_t st);
+// xinv: 1/|x| per token [BH, L] (launch_invnorm)
 cudaError_t launch_attn_fwd_tc(const Problem &p, const void *x, const void *v, const int32_t *perm,
-                               const uint16_t *bkt, __nv_bfloat16 *o_r, float *lse, uint32_t *status,
-                               cudaStream_t st);
+                               const uint16_t *bkt, const float *xinv, __nv_bfloat16 *o_r, float *lse,
+                               uint32_t *status, cudaStream_t st);
 bool attn_tc_supported(const Problem &p);
 // lse_out (nullable): receives logsumexp over the rounds, [BH, L]
 cudaError_t launch_combine(const Problem &p, const void *o_r, bool o_r_bf16, const float *lse, void *out,

@@ -27,12 +27,51 @@ __global__ void invnorm_kernel(const T *__restrict__ x, float *__restrict__ invn
     invnorm[r] = s > 0.f ? 1.0f / sqrtf(s) : 0.f;
 }
 
+// bf16 rows: a warp takes 16 consecutive rows, four per load instruction
+// (eight lanes per 128-byte row, 512 contiguous bytes), all four loads in
+// flight before any arithmetic; each row's eight partial sums of squares are
+// added by shuffles.
+constexpr int kNormRowsPerWarp = 16;
+__global__ void invnorm_bf16_kernel(const __nv_bfloat16 *__restrict__ x, float *__restrict__ invnorm, long long rows)
+{
+    const long long w = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    const long long r0 = w * kNormRowsPerWarp + (lane >> 3);
+    uint4 u[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const long long r = r0 + 4 * k;
+        u[k] = r < rows ? __ldg(reinterpret_cast<const uint4 *>(x + r * kDim) + (lane & 7)) : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const uint32_t wd[4] = {u[k].x, u[k].y, u[k].z, u[k].w};
+        float s = 0.f;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const float a = __uint_as_float(wd[e] << 16), b = __uint_as_float(wd[e] & 0xFFFF0000u);
+            s = fmaf(a, a, s);
+            s = fmaf(b, b, s);
+        }
+        s += __shfl_xor_sync(0xffffffffu, s, 1);
+        s += __shfl_xor_sync(0xffffffffu, s, 2);
+        s += __shfl_xor_sync(0xffffffffu, s, 4);
+        const long long r = r0 + 4 * k;
+        if (r < rows && (lane & 7) == 0) invnorm[r] = s > 0.f ? 1.0f / sqrtf(s) : 0.f;
+    }
+}
+
 cudaError_t launch_invnorm(const Problem &p, const void *x, float *invnorm, cudaStream_t st)
 {
-    if (p.dtype != LSH_F32) return cudaErrorInvalidValue;      // the tensor-core kernels compute their own norms
-    long long rows = p.tokens();
-    unsigned grid = (unsigned)((rows + 127) / 128);
-    invnorm_kernel<float><<<grid, 128, 0, st>>>((const float *)x, invnorm, rows);
+    const long long rows = p.tokens();
+    if (p.dtype == LSH_BF16) {
+        const long long warps = (rows + kNormRowsPerWarp - 1) / kNormRowsPerWarp;
+        const unsigned grid = (unsigned)((warps * 32 + 255) / 256);
+        invnorm_bf16_kernel<<<grid, 256, 0, st>>>((const __nv_bfloat16 *)x, invnorm, rows);
+    } else {
+        const unsigned grid = (unsigned)((rows + 127) / 128);
+        invnorm_kernel<float><<<grid, 128, 0, st>>>((const float *)x, invnorm, rows);
+    }
     return cudaGetLastError();
 }
 
