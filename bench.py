@@ -376,15 +376,31 @@ def cpu_cores() -> int:
         return os.cpu_count() or 1
 
 
+CPU_SAMPLE_S = 20.0      # target wall time of the CPU baseline's sample
+
+
 def cpu_baseline(w: synth.Workload) -> dict:
+    """The oracle on the host cores, one (batch, head) slice per OpenMP thread.
+    A short probe (slices of min(L, 2048) tokens) sizes the sample: full-length
+    slices when they finish in about CPU_SAMPLE_S seconds, else slices shortened
+    (multiples of 128 tokens) to fit it -- the oracle's cost is linear in L, so
+    the rate stands for the workload.  Tokens count sequence tokens as the
+    metric does (a slice of Ls tokens of one head is Ls / H of them)."""
     cores = cpu_cores()
-    n = max(1, min(cores, w.B * w.H))
-    secs = oracle_slices(w, n, n)
-    step_s = secs * (w.B * w.H) / n
-    return {"value": w.tokens / step_s, "unit": "tokens/s", "cores": n, "kind": "oracle",
-            "sample": f"{n} of {w.B * w.H} (batch, head) slices of {w.name}, full length, fwd"
-                      f"{'+bwd' if w.backward else ''}, one slice per OpenMP thread; {secs:.1f} s wall, "
-                      f"scaled by slice count"}
+    n0 = max(1, min(cores, w.B * w.H * max(1, w.L // 4096)))
+    Lp = min(w.L, 2048)
+    tp = oracle_slices(w, n0, n0, Lp)
+    est_full = tp * w.L / Lp                  # n0 full-length slices
+    n, Ls = n0, w.L
+    if Lp < w.L and est_full > CPU_SAMPLE_S:
+        Ls = max(Lp, int(CPU_SAMPLE_S / tp * Lp) // 128 * 128)
+    elif est_full * w.B * w.H / n0 <= CPU_SAMPLE_S:
+        n = w.B * w.H                         # the whole workload fits the budget
+    secs = tp if (n, Ls) == (n0, Lp) else oracle_slices(w, n, min(n, cores), Ls)
+    value = n * Ls / w.H / secs
+    return {"value": value, "unit": "tokens/s", "cores": min(n, cores), "kind": "oracle",
+            "sample": f"{n} (batch, head) slices of {Ls} tokens (the workload: {w.B * w.H} x {w.L}) of {w.name}, "
+                      f"fwd{'+bwd' if w.backward else ''}, {min(n, cores)} OpenMP threads; {secs:.1f} s wall"}
 
 
 def run_reference(args, w: synth.Workload, world: int = 1) -> dict:
