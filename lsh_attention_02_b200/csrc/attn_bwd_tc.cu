@@ -20,7 +20,8 @@
 //   elementwise: P^T (bf16, into tensor memory), E^T = tau inv_j dS^T (bf16, shared memory)
 //   dV   = P^T dYq   (A from TMEM, M=128, N=64, K=192)
 //   G    = E^T Xq    (M=128, N=64, K=192)
-//   dQ   = E Xk      (E^T read MN-major; two M=128 halves over the 192 queries, K=128)
+//   dQ   = E Xk      (E^T read MN-major; two M=128 halves over the 192 queries: K=128
+//                     keys for queries 0..127, K=64 (keys of chunk 2k+1) for 128..191)
 // Query slot r < 128 is also key slot r, so G and the first dQ half accumulate
 // into one TMEM block; the key-role correction needs g_j . x_j, which equals
 // sum_i e_ij (x_i . x_j) and is summed from S^T during the elementwise step.
@@ -285,33 +286,53 @@ __device__ __forceinline__ void zero_block(uint8_t (*ET)[kK * 128], uint32_t tl,
 // segment (bh, r), taken in order by one CTA, so the dQ rows of chunk 2k+2
 // that tile k computes can be handed to tile k+1 instead of being reduced
 // twice.  Units in flight at the same time share one head's rows in L2.
+// The iterator keeps the unit's coordinates, so the divisions that locate a
+// unit run once per unit, not once per tile.
 struct TileIter {
     long long unit;                 // >= n_units: done
     int j;                          // tile within the unit
+    int r, k0;                      // round; first key tile of the unit's run
+    long long bh, seg;
 };
 struct TileCoord {
     int r, k;
     long long bh, seg;
     bool next_adjacent;             // the CTA's next tile is (seg, k + 1)
 };
-__device__ __forceinline__ TileCoord tile_coord(const TileIter &t, int R, int n_k, int n_runs)
+__device__ __forceinline__ void tile_locate(TileIter &t, int R, int n_runs)
+{
+    t.r = (int)(t.unit % R);
+    const long long br = t.unit / R;
+    t.k0 = (int)(br % n_runs) * kRun;
+    t.bh = br / n_runs;
+    t.seg = t.bh * R + t.r;
+}
+__device__ __forceinline__ TileIter tile_begin(long long unit, int R, int n_runs)
+{
+    TileIter t;
+    t.unit = unit;
+    t.j = 0;
+    tile_locate(t, R, n_runs);
+    return t;
+}
+__device__ __forceinline__ TileCoord tile_coord(const TileIter &t, int n_k)
 {
     TileCoord c;
-    c.r = (int)(t.unit % R);
-    const long long br = t.unit / R;
-    c.k = (int)(br % n_runs) * kRun + t.j;
-    c.bh = br / n_runs;
-    c.seg = c.bh * R + c.r;
+    c.r = t.r;
+    c.k = t.k0 + t.j;
+    c.bh = t.bh;
+    c.seg = t.seg;
     c.next_adjacent = t.j + 1 < kRun && c.k + 1 < n_k;
     return c;
 }
 __device__ __forceinline__ void tile_advance(TileIter &t, int R, int n_k, int n_runs)
 {
-    if (tile_coord(t, R, n_k, n_runs).next_adjacent) {
+    if (t.j + 1 < kRun && t.k0 + t.j + 1 < n_k) {
         ++t.j;
     } else {
         t.unit += gridDim.x;
         t.j = 0;
+        tile_locate(t, R, n_runs);
     }
 }
 
@@ -358,7 +379,7 @@ attn_bwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
         constexpr int kPosPer = (256 + kProducerThreads - 1) / kProducerThreads;
         int pn[kPosPer], bn[kPosPer];
         auto load_pos = [&](const TileIter &t) {
-            const TileCoord c = tile_coord(t, R, n_k, n_runs);
+            const TileCoord c = tile_coord(t, n_k);
             const int32_t *P = perm + c.seg * L;
             const int slot0 = c.k * kK - 64;
 #pragma unroll
@@ -374,7 +395,7 @@ attn_bwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
                 if (FL & kMask) bn[j] = pn[j] >= 0 ? (int)bkt[c.seg * L + pn[j]] : -1;
             }
         };
-        TileIter ti{blockIdx.x, 0};
+        TileIter ti = tile_begin(blockIdx.x, R, n_runs);
         if (ti.unit < n_units) load_pos(ti);
         for (int it = 0; ti.unit < n_units; ++it) {
             const int s = it % kStages;
@@ -384,7 +405,7 @@ attn_bwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
             if (tc::named_bar_or(1, kProducerThreads, !ok)) break;
             if (ptid == 0) LSH_PHASE(1, 0, it, 1);
             Stage &st = sm.st[s];
-            const long long rowbase = tile_coord(ti, R, n_k, n_runs).bh * L;
+            const long long rowbase = tile_coord(ti, n_k).bh * L;
 #pragma unroll
             for (int j = 0; j < kPosPer; ++j) {
                 const int e = ptid + j * kProducerThreads;
@@ -394,7 +415,7 @@ attn_bwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
                 }
             }
             tc::named_bar_sync(1, kProducerThreads);
-            const TileCoord pc = tile_coord(ti, R, n_k, n_runs);
+            const TileCoord pc = tile_coord(ti, n_k);
             const int tile_k = pc.k;
             const bool prev = (prev_mask >> pc.r) & 1u;     // previous chunk alone: no lone queries
             // per-query LSE and delta: loads issued now, used after the copies are issued
@@ -484,7 +505,7 @@ attn_bwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
             constexpr uint32_t id_kv = tc::idesc_bf16(128, kDim, 0, 1);   // A K-major, B MN-major
             constexpr uint32_t id_q = tc::idesc_bf16(128, kDim, 1, 1);    // A MN-major, B MN-major
             const uint32_t e0 = tc::smem_u32(sm.ET[0]), e1 = tc::smem_u32(sm.ET[1]), e2 = tc::smem_u32(sm.ET[2]);
-            TileIter ti{blockIdx.x, 0};
+            TileIter ti = tile_begin(blockIdx.x, R, n_runs);
             for (int it = 0; ti.unit < n_units; ++it, tile_advance(ti, R, n_k, n_runs)) {
                 const int s = it % kStages;
                 const uint32_t ph = (uint32_t)it & 1u;
@@ -502,6 +523,10 @@ attn_bwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
                     tc::mma_bf16(tmem + cD, tc::sw128_desc(vs + kk * 32), tc::sw128_desc(gs + kk * 32), id_s, kk > 0);
                 }
                 tc::mma_commit(&sm.bar_s);
+#ifdef LSH_PHASE_TRACE
+                // tuning build: when the products complete, as the issuer sees it
+                if (tc::mbar_wait(&sm.bar_s, ph, &sm.abort, status)) LSH_PHASE(1, 1, it, 5);
+#endif
                 if (!tc::mbar_wait(&sm.bar_p, ph, &sm.abort, status)) break;
                 LSH_PHASE(1, 1, it, 3);
                 tc::tc_fence_after();
@@ -511,16 +536,23 @@ attn_bwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
                     tc::mma_bf16_ts(tmem + cDV, tmem + cPT + kk * 8, tc::sw128_desc(gs + kk * 2048), id_kv, kk > 0);
                     tc::mma_bf16(tmem + cDX, tc::sw128_desc(ea), tc::sw128_desc(xs + kk * 2048), id_kv, kk > 0);
                 }
-                // E = (E^T)^T read MN-major: 64-query blocks 16 KB apart (leading byte offset)
+                // E = (E^T)^T read MN-major: 64-query blocks 16 KB apart (leading byte offset).
+                // The second half (queries 64..191) is read only for chunk 2k+2 (rows
+                // 128..191), whose queries see the keys of chunk 2k+1 alone: its K range is
+                // keys 64..127 (rows 64..127 of that product are never read).
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
+                for (int kk = 0; kk < 8; ++kk)
                     tc::mma_bf16(tmem + cDX, tc::sw128_desc(e0 + kk * 2048, kK * 128), tc::sw128_desc(xs + kk * 2048),
                                  id_q, true);
+#pragma unroll
+                for (int kk = 4; kk < 8; ++kk)
                     tc::mma_bf16(tmem + cQb, tc::sw128_desc(e1 + kk * 2048, kK * 128), tc::sw128_desc(xs + kk * 2048),
-                                 id_q, kk > 0);
-                }
+                                 id_q, kk > 4);
                 tc::mma_commit(&sm.bar_o);
                 LSH_PHASE(1, 1, it, 4);
+#ifdef LSH_PHASE_TRACE
+                if (tc::mbar_wait(&sm.bar_o, ph, &sm.abort, status)) LSH_PHASE(1, 1, it, 6);
+#endif
             }
             if (*reinterpret_cast<volatile int *>(&sm.abort)) tc::mma_drain(&sm.drain, status);
         }
@@ -529,7 +561,7 @@ attn_bwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
         const int quad = warp & 3, half = warp >> 2;
         const int kr = quad * 32 + lane;
         const uint32_t tl = tmem + ((uint32_t)(quad * 32) << 16);
-        TileIter ti{blockIdx.x, 0};
+        TileIter ti = tile_begin(blockIdx.x, R, n_runs);
         bool carry_in = false;                       // this tile's chunk-2k rows hold a handed-over dQ part
         bool have_next_kinv = false;
         float next_kinv = 0.f;
@@ -540,7 +572,7 @@ attn_bwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
             if (!tc::mbar_wait(&sm.full[s], (uint32_t)(it / kStages) & 1u, &sm.abort, status)) break;
             if (tid == 0) LSH_PHASE(1, 2, it, 1);
             const Stage &st = sm.st[s];
-            const TileCoord tcd = tile_coord(ti, R, n_k, n_runs);
+            const TileCoord tcd = tile_coord(ti, n_k);
             const long long rowbase = tcd.bh * L;
             const int kpos = st.pos[64 + kr];
             const int kb = (FL & kMask) ? st.bk[64 + kr] : 0;

@@ -70,6 +70,24 @@ constexpr uint32_t kOCol = 192;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 
+struct TileCoord {
+    int r, k;
+    long long bh, seg;
+};
+// Tile order (bh, k, r): tiles in flight at the same time share a head's rows
+// in L2.  Only the producer locates tiles (a tile ahead); the softmax groups
+// read the coordinates from the stage.
+__device__ __forceinline__ TileCoord tile_coord(long long tile, int R, int n_k)
+{
+    TileCoord c;
+    c.r = (int)(tile % R);
+    const long long bk = tile / R;
+    c.k = (int)(bk % n_k);
+    c.bh = bk / n_k;
+    c.seg = c.bh * R + c.r;
+    return c;
+}
+
 struct alignas(1024) Stage {
     uint8_t X[kW * 128];            // gathered x rows, K-major SW128 (24 KB)
     uint8_t V[kW * 128];            // gathered v rows (24 KB)
@@ -77,6 +95,7 @@ struct alignas(1024) Stage {
     alignas(16) float sinv[kW];     // tau * log2(e) / |x_j| (0 for a zero row or no row)
     alignas(16) float inv[kW];      // 1 / |x_j|
     alignas(16) int32_t kb[kW];     // bucket of each window slot (-1: none); bucket mask only
+    TileCoord coord;                // the tile's coordinates
 };
 
 // Optional readings (template parameter FL, bits of lsh_attn_desc.flags).
@@ -101,22 +120,6 @@ struct FwdSmem {
     uint32_t tmem_base;
     int abort;
 };
-
-struct TileCoord {
-    int r, k;
-    long long bh, seg;
-};
-__device__ __forceinline__ TileCoord tile_coord(long long tile, int R, int n_k)
-{
-    // order (bh, k, r): tiles in flight at the same time share a head's rows in L2
-    TileCoord c;
-    c.r = (int)(tile % R);
-    const long long bk = tile / R;
-    c.k = (int)(bk % n_k);
-    c.bh = bk / n_k;
-    c.seg = c.bh * R + c.r;
-    return c;
-}
 
 // Softmax of one query row (thread) over window columns [BASE, BASE + 128)
 // (chunk 2k: BASE = 0, chunk 2k+1: BASE = 64).  FIRST: the segment's first
@@ -305,8 +308,10 @@ attn_fwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
         // A slot outside [0, L) (chunk -1, or the missing chunk of a last tile
         // when L % 128 == 64) is empty (-1); so is a permutation entry outside
         // [0, L), which is also reported in the status word.
+        TileCoord nc{};                             // coordinates of that tile
         auto load_pos = [&](long long tile) {
             const TileCoord c = tile_coord(tile, R, n_k);
+            nc = c;
             const int32_t *P = perm + c.seg * L;
             const int slot0 = c.k * kQ - 64;
 #pragma unroll
@@ -333,7 +338,9 @@ attn_fwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
             if (tc::named_bar_or(1, kProducerThreads, !ok)) { prev_s = -1; break; }
             if (ptid == 0) LSH_PHASE(0, 0, it, 1);
             Stage &st = sm.st[s];
-            const long long rowbase = tile_coord(tile, R, n_k).bh * L;
+            const TileCoord cc = nc;
+            const long long rowbase = cc.bh * L;
+            if (ptid == 0) st.coord = cc;
             st.pos[ptid] = pn[0];
             st.pos[ptid + kProducerThreads] = pn[1];
 #pragma unroll
@@ -481,7 +488,7 @@ attn_fwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
             if (!tc::mbar_wait(&sm.s_full[g], gph, &sm.abort, status)) break;
             if (mark) LSH_PHASE(0, 2 + g, it, 2);
             tc::tc_fence_after();
-            const TileCoord tcd = tile_coord(tile, R, n_k);
+            const TileCoord tcd = st.coord;
             const int qpos = st.pos[64 + i];
             const int qb = (FL & kMask) ? st.kb[64 + i] : 0;
             const float qinv = st.inv[64 + i];
