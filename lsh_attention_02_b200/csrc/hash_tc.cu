@@ -127,14 +127,17 @@ hash_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __nv_bfloat16 *__
             int it = 0, bi = 0, r_issued = 0, a_issued = blockIdx.x < n_blocks ? 1 : 0;
             for (long long blk = blockIdx.x; ok && blk < n_blocks; blk += gridDim.x, ++bi) {
                 const int prefetch_at = min(kStages, items) - 1;
-                for (int i = 0; i < items; ++i, ++it) {
+                for (int i = 0, r = 0, nt = 0; i < items; ++i, ++it) {
                     const int s = it % kStages;
                     const uint32_t ph = (uint32_t)(it / kStages) & 1u;
                     LSH_PHASE(0, 1, it, 0);
                     if (it >= kStages && !tc::mbar_wait(&sm.empty[s], ph ^ 1u, &sm.abort, status)) { ok = false; break; }
                     LSH_PHASE(0, 1, it, 1);
-                    const int r = i / n_nt, nt = i % n_nt;
                     const __nv_bfloat16 *src = Rs + ((long long)r * hp + (long long)nt * NT) * kDim;
+                    if (++nt == n_nt) {
+                        nt = 0;
+                        ++r;
+                    }
                     tc::mbar_arrive_expect_tx(&sm.full[s], NT * 128);
                     tc::bulk_g2s(sm.B[s], src, NT * 128, &sm.full[s]);
                     ++r_issued;
@@ -209,6 +212,7 @@ hash_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __nv_bfloat16 *__
             const long long g = blk * kRows + prow;
             float best = -INFINITY;
             int bucket = 0;
+            int r = 0, nt = 0;                               // item i = (round r, N-tile nt), no division
             for (int i = 0; i < items; ++i, ++it) {
                 const int ab = it & 1;
                 const uint32_t aph = (uint32_t)(it >> 1) & 1u;
@@ -288,7 +292,6 @@ hash_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __nv_bfloat16 *__
                         js = eq ? c * 16 + __ffs((int)eq) - 1 : js;
                     }
                 }
-                const int r = i / n_nt, nt = i % n_nt;
                 const float tbest = pos ? mx : -mn;
                 const int tb = (pos ? 0 : half) + nt * NT + hf * NH + js;
                 if (tbest > best || (tbest == best && tb < bucket)) { best = tbest; bucket = tb; }
@@ -316,6 +319,10 @@ hash_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __nv_bfloat16 *__
                     ++rd;
                     best = -INFINITY;
                     bucket = 0;
+                }
+                if (++nt == n_nt) {
+                    nt = 0;
+                    ++r;
                 }
             }
         }
