@@ -243,28 +243,37 @@ __device__ __forceinline__ void key_row_step(const Stage &st, uint8_t (*ET)[kK *
 // all three column blocks share one copy of the code.
 template <bool CAUSAL, int FL>
 __device__ __forceinline__ float key_row_block(const Stage &st, uint8_t (*ET)[kK * 128], uint32_t tl, int kr, int kpos,
-                                               int kb, int C0, float kinv, float tau)
+                                               int kb, int C0, float kinv, float tau, bool mark = false,
+                                               int it = 0)
 {
     const float sc = tau * kinv * kLog2e;
     const float ec = tau * kinv;
     float gx = 0.f;
     float sa[16], da[16], sb[16], db[16];
+    if (mark) LSH_PHASE(1, 5, it, 0);
     tc::tmem_ld16(tl + cS + C0, sa);
     tc::tmem_ld16(tl + cD + C0, da);
     tc::tmem_ld_wait();
+    if (mark) LSH_PHASE(1, 5, it, 1);
     tc::tmem_ld16(tl + cS + C0 + 16, sb);
     tc::tmem_ld16(tl + cD + C0 + 16, db);
     key_row_step<CAUSAL, FL, 0>(st, ET, tl, kr, kpos, kb, C0, sc, ec, sa, da, gx);
+    if (mark) LSH_PHASE(1, 5, it, 2);
     tc::tmem_ld_wait();
+    if (mark) LSH_PHASE(1, 5, it, 3);
     tc::tmem_ld16(tl + cS + C0 + 32, sa);
     tc::tmem_ld16(tl + cD + C0 + 32, da);
     key_row_step<CAUSAL, FL, 1>(st, ET, tl, kr, kpos, kb, C0, sc, ec, sb, db, gx);
+    if (mark) LSH_PHASE(1, 5, it, 4);
     tc::tmem_ld_wait();
     tc::tmem_ld16(tl + cS + C0 + 48, sb);
     tc::tmem_ld16(tl + cD + C0 + 48, db);
     key_row_step<CAUSAL, FL, 2>(st, ET, tl, kr, kpos, kb, C0, sc, ec, sa, da, gx);
+    if (mark) LSH_PHASE(1, 5, it, 5);
     tc::tmem_ld_wait();
+    if (mark) LSH_PHASE(1, 5, it, 6);
     key_row_step<CAUSAL, FL, 3>(st, ET, tl, kr, kpos, kb, C0, sc, ec, sb, db, gx);
+    if (mark) LSH_PHASE(1, 5, it, 7);
     return gx;
 }
 
@@ -599,7 +608,7 @@ attn_bwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
                 if (quad < 2) zero_block<0>(sm.ET, tl, kr);
                 else zero_block<64>(sm.ET, tl, kr);
             } else {
-                gx = key_row_block<CAUSAL, FL>(st, sm.ET, tl, kr, kpos, kb, c0, kinv, tau);
+                gx = key_row_block<CAUSAL, FL>(st, sm.ET, tl, kr, kpos, kb, c0, kinv, tau, tid == 0, it);
             }
             if (half == 0) {
                 if (quad < 2) zero_block<128>(sm.ET, tl, kr);
@@ -649,7 +658,7 @@ attn_bwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
             };
             if (half == 0) {
                 // slot kr: query-role dQ plus key-role g, less inv^2 (g . x) x
-                const int prole = warp == 0 ? 4 : warp == 2 ? 5 : -1;
+                const int prole = warp == 0 ? 4 : -1;
                 if (prole >= 0 && lane == 0) LSH_PHASE(1, prole, it, 0);
 #pragma unroll
                 for (int c = 0; c < 4; ++c) tc::tmem_ld16(tl + cDX + c * 16, a + c * 16);
