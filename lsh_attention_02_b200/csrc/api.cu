@@ -148,7 +148,7 @@ static lsh_status run_hash_sort(const Problem &p, const Choice &c, const void *q
                                 const Workspace &w, cudaStream_t st)
 {
     LSH_TRY(staged(LSH_STAGE_HASH, c.tc_hash ? 2 : 1, st, [&] {
-                return c.tc_hash ? launch_hash_tc(p, qk, R, w.buckets, w.rot, w.status, st)
+                return c.tc_hash ? launch_hash_tc(p, qk, R, w.buckets, w.rot, w.invnorm, w.status, st)
                                  : launch_hash_simt(p, qk, R, w.buckets, st);
             }), "hash");
     LSH_TRY(launch_near_ties(p, qk, R, st), "near-tie count");
@@ -157,10 +157,13 @@ static lsh_status run_hash_sort(const Problem &p, const Choice &c, const void *q
     return LSH_OK;
 }
 
+// norms_ready: the tensor-core hash of this call already wrote w.invnorm
 static lsh_status run_attn_fwd(const Problem &p, const Choice &c, const void *qk, const void *v,
-                               const int32_t *perm, void *out, float *lse, const Workspace &w, cudaStream_t st)
+                               const int32_t *perm, void *out, float *lse, const Workspace &w, cudaStream_t st,
+                               bool norms_ready = false)
 {
-    LSH_TRY(staged(LSH_STAGE_NORMS, 1, st, [&] { return launch_invnorm(p, qk, w.invnorm, st); }), "key norms");
+    if (!norms_ready)
+        LSH_TRY(staged(LSH_STAGE_NORMS, 1, st, [&] { return launch_invnorm(p, qk, w.invnorm, st); }), "key norms");
     LSH_TRY(staged(LSH_STAGE_ATTN_FWD, 1, st, [&] {
                 return c.tc_attn
                            ? launch_attn_fwd_tc(p, qk, v, perm, w.buckets, w.invnorm, (__nv_bfloat16 *)w.o_r, lse,
@@ -230,7 +233,7 @@ lsh_status lsh_attn_hash(const lsh_attn_desc *desc, const void *qk, const void *
     w = plan_workspace(p, false, c.tc_attn, c.tc_hash, (char *)workspace);
     cudaStream_t st = (cudaStream_t)stream;
     LSH_TRY(staged(LSH_STAGE_HASH, c.tc_hash ? 2 : 1, st, [&] {
-                return c.tc_hash ? launch_hash_tc(p, qk, R, buckets, w.rot, w.status, st)
+                return c.tc_hash ? launch_hash_tc(p, qk, R, buckets, w.rot, nullptr, w.status, st)
                                  : launch_hash_simt(p, qk, R, buckets, st);
             }), "hash");
     LSH_TRY(launch_near_ties(p, qk, R, st), "near-tie count");
@@ -321,7 +324,7 @@ lsh_status lsh_attn_fwd(const lsh_attn_desc *desc, const void *qk, const void *v
     int32_t *perm = perm_out ? perm_out : w.perm;
     LSH_TRY(cudaMemsetAsync(w.status, 0, sizeof(uint32_t), st), "status reset");
     if ((s = run_hash_sort(p, c, qk, R, perm, w, st)) != LSH_OK) return s;
-    return run_attn_fwd(p, c, qk, v, perm, out, lse, w, st);
+    return run_attn_fwd(p, c, qk, v, perm, out, lse, w, st, c.tc_hash);
 }
 
 lsh_status lsh_attn_bwd(const lsh_attn_desc *desc, const void *qk, const void *v, const void *R, const void *out,
@@ -348,7 +351,7 @@ lsh_status lsh_attn_bwd(const lsh_attn_desc *desc, const void *qk, const void *v
     } else if (mask) {
         // the bucket mask needs the bucket ids of this call's rounds
         LSH_TRY(staged(LSH_STAGE_HASH, c.tc_hash ? 2 : 1, st, [&] {
-                    return c.tc_hash ? launch_hash_tc(p, qk, R, w.buckets, w.rot, w.status, st)
+                    return c.tc_hash ? launch_hash_tc(p, qk, R, w.buckets, w.rot, nullptr, w.status, st)
                                      : launch_hash_simt(p, qk, R, w.buckets, st);
                 }), "hash");
     }
@@ -517,7 +520,7 @@ lsh_status lsh_rev_fwd(const lsh_attn_desc *desc, const float *x1, const float *
     LSH_TRY(cudaMemsetAsync(w.status, 0, sizeof(uint32_t), st), "status reset");
     LSH_TRY(launch_cast(p, x2, r.xa, st), "x2 to the attention dtype");
     if ((s = run_hash_sort(p, c, r.xa, R, r.perm, w, st)) != LSH_OK) return s;
-    if ((s = run_attn_fwd(p, c, r.xa, r.xa, r.perm, r.f, r.lse, w, st)) != LSH_OK) return s;   // F(x2)
+    if ((s = run_attn_fwd(p, c, r.xa, r.xa, r.perm, r.f, r.lse, w, st, c.tc_hash)) != LSH_OK) return s;   // F(x2)
     LSH_TRY(launch_axpy(p, x1, r.f, 1.f, y1, st), "y1 = x1 + F(x2)");
     LSH_TRY(launch_g_forward(p, y1, Wg, bg, x2, y2, nullptr, st), "y2 = x2 + G(y1)");
     return LSH_OK;
@@ -547,7 +550,7 @@ lsh_status lsh_rev_bwd(const lsh_attn_desc *desc, const float *y1, const float *
     // inverse of the F half: F(x2) again (hash, sort, attention), x1 = y1 - F(x2)
     LSH_TRY(launch_cast(p, x2, r.xa, st), "x2 to the attention dtype");
     if ((s = run_hash_sort(p, c, r.xa, R, r.perm, wf, st)) != LSH_OK) return s;
-    if ((s = run_attn_fwd(p, c, r.xa, r.xa, r.perm, r.f, r.lse, wf, st)) != LSH_OK) return s;
+    if ((s = run_attn_fwd(p, c, r.xa, r.xa, r.perm, r.f, r.lse, wf, st, c.tc_hash)) != LSH_OK) return s;
     LSH_TRY(launch_axpy(p, y1, r.f, -1.f, x1, st), "x1 = y1 - F(x2)");
     // gradient through F, whose query-key and value inputs are both x2
     LSH_TRY(launch_cast(p, dx1, r.da, st), "dF to the attention dtype");
@@ -684,7 +687,7 @@ lsh_status lsh_attn_step_host(const lsh_attn_desc *desc, int32_t heads_per_chunk
         Workspace wf = plan_workspace(pc, false, c.tc_attn, c.tc_hash, sl.ws);
         wf.status = status;
         if ((rc = run_hash_sort(pc, c, sl.x, h.R, sl.perm, wf, cs)) != LSH_OK) break;
-        if ((rc = run_attn_fwd(pc, c, sl.x, sl.v, sl.perm, sl.out, sl.lse, wf, cs)) != LSH_OK) break;
+        if ((rc = run_attn_fwd(pc, c, sl.x, sl.v, sl.perm, sl.out, sl.lse, wf, cs, c.tc_hash)) != LSH_OK) break;
         if (bwd) {
             Workspace wb = plan_workspace(pc, true, c.tc_attn, c.tc_hash, sl.ws);
             wb.status = status;

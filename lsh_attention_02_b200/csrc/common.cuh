@@ -147,8 +147,9 @@ cudaError_t launch_hash_simt(const Problem &p, const void *x, const void *R, uin
 // (-1 when not compiled in, -2 on a CUDA error).
 cudaError_t launch_near_ties(const Problem &p, const void *x, const void *R, cudaStream_t st);
 long long read_near_ties();
+// invnorm (nullable): receives 1/|x| per token [BH, L] (from the same reads of x)
 cudaError_t launch_hash_tc(const Problem &p, const void *x, const void *R, uint16_t *buckets, void *scratch,
-                           uint32_t *status, cudaStream_t st);
+                           float *invnorm, uint32_t *status, cudaStream_t st);
 bool hash_tc_supported(const Problem &p);
 size_t hash_tc_scratch_bytes(const Problem &p);
 cudaError_t launch_sort(const Problem &p, const uint16_t *buckets, int32_t *perm, const Workspace &ws,

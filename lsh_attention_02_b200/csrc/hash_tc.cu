@@ -20,7 +20,9 @@
 //              TMEM accumulator buffers (double buffering lets the epilogue
 //              of tile t overlap the MMAs of tile t+1), with a completion
 //              barrier per M-tile so the two epilogue halves start apart and
-//              their ALU- and FMA-heavy passes overlap.
+//              their ALU- and FMA-heavy passes overlap;
+//   warp 18    key norms: 1/|x| of the block's rows from the same shared-memory
+//              tile (the attention kernels read them), so x is read once.
 //
 // Epilogue per N-tile of NT columns held in registers: pass 1 takes the
 // max and min with 3-input min/max; the larger of max and -min decides the
@@ -38,7 +40,8 @@ constexpr int kRows = 256;          // rows per block
 constexpr int kMaxNT = 128;         // widest N-tile
 constexpr int kStages = 4;          // rotation-tile ring
 constexpr int kEpiWarps = 16;         // 4 lane quadrants x 2 M-tiles x 2 column halves
-constexpr int kThreads = (kEpiWarps + 2) * 32;
+constexpr int kNormWarp = kEpiWarps + 2;
+constexpr int kThreads = (kNormWarp + 1) * 32;
 constexpr int kTmemCols = 512;      // 2 buffers x 2 M-tiles x kMaxNT
 
 struct HashSmem {
@@ -79,8 +82,8 @@ __global__ void rot_swizzle_kernel(const __nv_bfloat16 *__restrict__ R, __nv_bfl
 template <int NT>
 __global__ void __launch_bounds__(kThreads, 1)
 hash_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __nv_bfloat16 *__restrict__ Rs,
-               uint16_t *__restrict__ buckets, long long rows_total, int L, int rounds, int half, int hp,
-               uint32_t *__restrict__ status)
+               uint16_t *__restrict__ buckets, float *__restrict__ invnorm, long long rows_total, int L, int rounds,
+               int half, int hp, uint32_t *__restrict__ status)
 {
     extern __shared__ uint8_t smem_raw[];
     HashSmem &sm = *reinterpret_cast<HashSmem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -94,7 +97,7 @@ hash_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __nv_bfloat16 *__
         for (int s = 0; s < kStages; ++s) { tc::mbar_init(&sm.full[s], 1); tc::mbar_init(&sm.empty[s], 1); }
         for (int b = 0; b < 2; ++b) {
             tc::mbar_init(&sm.a_full[b], 1);
-            tc::mbar_init(&sm.a_empty[b], 1);
+            tc::mbar_init(&sm.a_empty[b], 2);    // the MMAs and the norm warp
             tc::mbar_init(&sm.acc_full[b][0], 1);
             tc::mbar_init(&sm.acc_full[b][1], 1);
             tc::mbar_init(&sm.acc_empty[b], kEpiWarps);
@@ -196,6 +199,36 @@ hash_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __nv_bfloat16 *__
                 if (ok) tc::mma_commit(&sm.a_empty[xa]);
             }
             if (*reinterpret_cast<volatile int *>(&sm.abort)) tc::mma_drain(&sm.drain, status);
+        }
+    } else if (warp == kNormWarp) {
+        // ---------------- key norms of each block's rows (lane l: rows l, l + 32, ...), sum of
+        // squares in element order as the norm pass does; then the A buffer may be refilled
+        int bi = 0;
+        for (long long blk = blockIdx.x; blk < n_blocks; blk += gridDim.x, ++bi) {
+            const int xa = bi & 1;
+            if (!tc::mbar_wait(&sm.a_full[xa], (uint32_t)(bi >> 1) & 1u, &sm.abort, status)) break;
+            if (invnorm) {
+                const uint8_t *A = sm.A[xa];
+#pragma unroll 1
+                for (int r = lane; r < kRows; r += 32) {
+                    float ssq = 0.f;
+#pragma unroll
+                    for (int ch = 0; ch < 8; ++ch) {
+                        const uint4 u = *reinterpret_cast<const uint4 *>(A + r * 128 + ((ch ^ (r & 7)) << 4));
+                        const uint32_t wd[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const float a = __uint_as_float(wd[e] << 16), b = __uint_as_float(wd[e] & 0xFFFF0000u);
+                            ssq = fmaf(a, a, ssq);
+                            ssq = fmaf(b, b, ssq);
+                        }
+                    }
+                    const long long g = blk * kRows + r;
+                    if (g < rows_total) invnorm[g] = ssq > 0.f ? 1.0f / sqrtf(ssq) : 0.f;
+                }
+            }
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(&sm.a_empty[xa]);
         }
     } else {
         // ---------------- epilogue: warp w reads TMEM lanes 32*(w%4).. of M-tile
@@ -339,7 +372,7 @@ hash_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __nv_bfloat16 *__
 
 template <int NT>
 cudaError_t launch_nt(const Problem &p, const void *x, const __nv_bfloat16 *Rs, int hp, uint16_t *buckets,
-                      uint32_t *status, cudaStream_t st)
+                      float *invnorm, uint32_t *status, cudaStream_t st)
 {
     // one CTA per SM: each holds all 512 TMEM columns
     const size_t smem = sizeof(HashSmem) + 1024;
@@ -353,7 +386,8 @@ cudaError_t launch_nt(const Problem &p, const void *x, const __nv_bfloat16 *Rs, 
     if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
     const long long blocks = (rows + kRows - 1) / kRows;
     const unsigned grid = (unsigned)std::min<long long>(blocks, sms);
-    hash_tc_kernel<NT><<<grid, kThreads, smem, st>>>(xmap, Rs, buckets, rows, p.L, p.R, p.nb / 2, hp, status);
+    hash_tc_kernel<NT><<<grid, kThreads, smem, st>>>(xmap, Rs, buckets, invnorm, rows, p.L, p.R, p.nb / 2, hp,
+                                                     status);
     return cudaGetLastError();
 }
 
@@ -386,7 +420,7 @@ size_t hash_tc_scratch_bytes(const Problem &p)
 }
 
 cudaError_t launch_hash_tc(const Problem &p, const void *x, const void *R, uint16_t *buckets, void *scratch,
-                           uint32_t *status, cudaStream_t st)
+                           float *invnorm, uint32_t *status, cudaStream_t st)
 {
     const int half = p.nb / 2, hp = padded_half(half);
     __nv_bfloat16 *Rs = (__nv_bfloat16 *)scratch;
@@ -396,10 +430,10 @@ cudaError_t launch_hash_tc(const Problem &p, const void *x, const void *R, uint1
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     switch (pick_nt(half)) {
-    case 128: return launch_nt<128>(p, x, Rs, hp, buckets, status, st);
-    case 96: return launch_nt<96>(p, x, Rs, hp, buckets, status, st);
-    case 64: return launch_nt<64>(p, x, Rs, hp, buckets, status, st);
-    default: return launch_nt<32>(p, x, Rs, hp, buckets, status, st);
+    case 128: return launch_nt<128>(p, x, Rs, hp, buckets, invnorm, status, st);
+    case 96: return launch_nt<96>(p, x, Rs, hp, buckets, invnorm, status, st);
+    case 64: return launch_nt<64>(p, x, Rs, hp, buckets, invnorm, status, st);
+    default: return launch_nt<32>(p, x, Rs, hp, buckets, invnorm, status, st);
     }
 }
 
