@@ -325,6 +325,12 @@ typedef enum {
 LSH_API lsh_status lsh_attn_trace_begin(int32_t capacity);
 LSH_API lsh_status lsh_attn_trace_end(float *ms, int32_t *calls, int32_t *kernels, int32_t n);
 
+/* Which stages a trace records: bit s of `mask` for lsh_stage s (default: all).
+ * Process-wide, takes effect for the stages enqueued after the call; a stage
+ * left out is enqueued without events around it, so timing one kernel adds
+ * only its own event pair to the stream.  Always returns LSH_OK. */
+LSH_API lsh_status lsh_attn_trace_stages(uint32_t mask);
+
 /* Self-test of the bounded device-side waits: launches one CTA that waits on a
  * barrier nothing completes, for `budget_cycles` SM cycles (>= 0).  The wait
  * gives up, sets the timeout bit in the status word at the start of

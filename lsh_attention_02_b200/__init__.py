@@ -25,7 +25,7 @@ STATUS = {0: "LSH_OK", -1: "LSH_ERR_ARG", -2: "LSH_ERR_SHAPE", -3: "LSH_ERR_ALIG
 
 EXPORTED = ("lsh_attn_make_rotations", "lsh_attn_workspace_size", "lsh_attn_hash", "lsh_attn_sort", "lsh_attn_sort_static", "lsh_attn_fwd_sorted", "lsh_attn_fwd",
             "lsh_attn_bwd", "lsh_attn_poll", "lsh_attn_selftest_timeout", "lsh_attn_trace_begin",
-            "lsh_attn_trace_end", "lsh_attn_last_near_ties",
+            "lsh_attn_trace_end", "lsh_attn_trace_stages", "lsh_attn_last_near_ties",
             "lsh_attn_status_str", "lsh_attn_last_error", "lsh_attn_abi_version",
             "lsh_attn_local_workspace_size", "lsh_attn_local_fwd", "lsh_attn_local_bwd",
             "lsh_rev_workspace_size", "lsh_rev_fwd", "lsh_rev_bwd",
@@ -82,6 +82,7 @@ def load_library(path: str = LIB_PATH):
     L.lsh_attn_poll.argtypes = [P, P]
     L.lsh_attn_selftest_timeout.argtypes = [P, ctypes.c_int64, P]
     L.lsh_attn_trace_begin.argtypes = [ctypes.c_int32]
+    L.lsh_attn_trace_stages.argtypes = [ctypes.c_uint32]
     L.lsh_attn_trace_end.argtypes = [ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_int32),
                                      ctypes.POINTER(ctypes.c_int32), ctypes.c_int32]
     L.lsh_attn_last_near_ties.argtypes = []
@@ -278,6 +279,12 @@ def lsh_attn_selftest_timeout(ws: torch.Tensor, budget_cycles: int):
 def trace_begin(capacity: int = 4096):
     """Starts recording a CUDA event pair around every stage the library enqueues."""
     _check(load_library().lsh_attn_trace_begin(int(capacity)), "lsh_attn_trace_begin")
+
+
+def trace_stages(names=None):
+    """Restricts what a trace records to the named stages (None: every stage)."""
+    mask = 0xFFFFFFFF if names is None else sum(1 << STAGES.index(n) for n in names)
+    _check(load_library().lsh_attn_trace_stages(mask), "lsh_attn_trace_stages")
 
 
 def trace_end() -> dict:

@@ -33,13 +33,15 @@ struct Trace {
     int *stage = nullptr, *kernels = nullptr;
 };
 static Trace g_trace;
+static uint32_t g_trace_mask = ~0u;  // stages recorded while a trace is on (bit = lsh_stage)
 
 // Records one event pair around a stage; `fn` enqueues the stage's kernels.
 template <typename F>
 static cudaError_t staged(int stage, int n_kernels, cudaStream_t st, F fn)
 {
-    const bool rec = g_trace.on && g_trace.used < g_trace.cap;
-    if (g_trace.on && !rec) g_trace.overflow = true;
+    const bool sel = ((g_trace_mask >> stage) & 1u) != 0;
+    const bool rec = g_trace.on && sel && g_trace.used < g_trace.cap;
+    if (g_trace.on && sel && !rec) g_trace.overflow = true;
     if (rec) {
         cudaError_t e = cudaEventRecord(g_trace.ev[2 * g_trace.used], st);
         if (e != cudaSuccess) return e;
@@ -758,6 +760,12 @@ lsh_status lsh_attn_trace_begin(int32_t capacity)
     }
     t.on = true;
     g_trace = t;
+    return LSH_OK;
+}
+
+lsh_status lsh_attn_trace_stages(uint32_t mask)
+{
+    g_trace_mask = mask;
     return LSH_OK;
 }
 

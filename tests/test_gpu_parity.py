@@ -563,3 +563,30 @@ def test_near_tie_count_in_tuning_build():
             close += int((mg < 1e-4).sum())
     assert 20 <= count <= close, (count, close)
     assert lsh.load_library().lsh_attn_last_near_ties() == -1     # the regular build does not count
+
+
+def test_trace_records_only_selected_stages():
+    """With a stage mask the trace puts events around the selected stages alone
+    (the bench times its dominant kernel this way); the results are unchanged."""
+    w = small("bf16_causal_4k", B=1, H=2, L=1024, n_buckets=64, n_hashes=2)
+    inp = synth.make_inputs(w)
+    x = to_dev(inp["x"], "bf16"); v = to_dev(inp["v"], "bf16"); R = to_dev(inp["R"], "bf16")
+    desc = lsh.desc_for(x, w.n_buckets, w.n_hashes, w.chunk, w.causal)
+    out, lse, perm = lsh.outputs_like(desc, x)
+    ws = lsh.workspace(desc, False, x.device)
+    lsh.lsh_attn_fwd(desc, x, v, R, out, lse, perm, ws)
+    ref = out.clone()
+    try:
+        lsh.trace_stages(["attn_fwd"])
+        lsh.trace_begin(16)
+        lsh.lsh_attn_fwd(desc, x, v, R, out, lse, perm, ws)
+        st = lsh.trace_end()
+    finally:
+        lsh.trace_stages(None)
+    assert st["attn_fwd"][1] == 1 and st["attn_fwd"][0] > 0
+    assert all(st[k][1] == 0 for k in st if k != "attn_fwd")
+    assert torch.equal(out, ref)
+    lsh.trace_begin(16)
+    lsh.lsh_attn_fwd(desc, x, v, R, out, lse, perm, ws)
+    st = lsh.trace_end()
+    assert st["hash"][1] == 1 and st["sort"][1] == 1 and st["combine"][1] == 1
