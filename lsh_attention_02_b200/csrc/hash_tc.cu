@@ -21,7 +21,7 @@
 //              of tile t overlap the MMAs of tile t+1), with a completion
 //              barrier per M-tile so the two epilogue halves start apart and
 //              their ALU- and FMA-heavy passes overlap;
-//   warp 18    key norms: 1/|x| of the block's rows from the same shared-memory
+//   warps 18-19 key norms: 1/|x| of the block's rows from the same shared-memory
 //              tile (the attention kernels read them), so x is read once.
 //
 // Epilogue per N-tile of NT columns held in registers: pass 1 takes the
@@ -40,8 +40,9 @@ constexpr int kRows = 256;          // rows per block
 constexpr int kMaxNT = 128;         // widest N-tile
 constexpr int kStages = 4;          // rotation-tile ring
 constexpr int kEpiWarps = 16;         // 4 lane quadrants x 2 M-tiles x 2 column halves
-constexpr int kNormWarp = kEpiWarps + 2;
-constexpr int kThreads = (kNormWarp + 1) * 32;
+constexpr int kNormWarp = kEpiWarps + 2;   // first of kNormWarps
+constexpr int kNormWarps = 2;
+constexpr int kThreads = (kNormWarp + kNormWarps) * 32;
 constexpr int kTmemCols = 512;      // 2 buffers x 2 M-tiles x kMaxNT
 
 struct HashSmem {
@@ -97,7 +98,7 @@ hash_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __nv_bfloat16 *__
         for (int s = 0; s < kStages; ++s) { tc::mbar_init(&sm.full[s], 1); tc::mbar_init(&sm.empty[s], 1); }
         for (int b = 0; b < 2; ++b) {
             tc::mbar_init(&sm.a_full[b], 1);
-            tc::mbar_init(&sm.a_empty[b], 2);    // the MMAs and the norm warp
+            tc::mbar_init(&sm.a_empty[b], 1 + kNormWarps);   // the MMAs and the norm warps
             tc::mbar_init(&sm.acc_full[b][0], 1);
             tc::mbar_init(&sm.acc_full[b][1], 1);
             tc::mbar_init(&sm.acc_empty[b], kEpiWarps);
@@ -200,9 +201,10 @@ hash_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __nv_bfloat16 *__
             }
             if (*reinterpret_cast<volatile int *>(&sm.abort)) tc::mma_drain(&sm.drain, status);
         }
-    } else if (warp == kNormWarp) {
-        // ---------------- key norms of each block's rows (lane l: rows l, l + 32, ...), sum of
-        // squares in element order as the norm pass does; then the A buffer may be refilled
+    } else if (warp >= kNormWarp) {
+        // ---------------- key norms of each block's rows (norm warp w, lane l: rows 32 w + l,
+        // + 64, ...), sum of squares in element order as the norm pass does; then the A
+        // buffer may be refilled
         int bi = 0;
         for (long long blk = blockIdx.x; blk < n_blocks; blk += gridDim.x, ++bi) {
             const int xa = bi & 1;
@@ -210,7 +212,7 @@ hash_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __nv_bfloat16 *__
             if (invnorm) {
                 const uint8_t *A = sm.A[xa];
 #pragma unroll 1
-                for (int r = lane; r < kRows; r += 32) {
+                for (int r = (warp - kNormWarp) * 32 + lane; r < kRows; r += 32 * kNormWarps) {
                     float ssq = 0.f;
 #pragma unroll
                     for (int ch = 0; ch < 8; ++ch) {
