@@ -14,7 +14,8 @@
 //   scan    per segment, an exclusive scan over (digit, tile) in that order,
 //           which is exactly the output offset of (digit, tile)'s first element;
 //   scatter per tile, a stable rank of each element among equal digits
-//           (warp-private histograms + match_any inside each warp), then the
+//           (warp-private histograms; inside a warp, the lanes holding the
+//           same digit found with one ballot per digit bit), then the
 //           element is written at offset + rank.
 // Pass 0 reads the bucket ids in position order with the position as the
 // value; the last pass writes only the values, i.e. the permutation.
@@ -36,6 +37,26 @@ SortPlan make_sort_plan(int n_buckets, int L)
     sp.n_tiles = (L + kSortTile - 1) / kSortTile;
     sp.max_radix = 1 << sp.bits[0];
     return sp;
+}
+
+// Lanes of the warp whose key equals this lane's, from one ballot per key bit
+// (keys below 2^nbits; a lane with key 2^nbits, an out-of-range marker, matches
+// only lanes with the same marker).
+__device__ __forceinline__ uint32_t peers_of(uint32_t key, int nbits)
+{
+    uint32_t peers = 0xffffffffu;
+    for (int bit = 0; bit <= nbits; ++bit) {
+        const bool set = (key >> bit) & 1u;
+        const uint32_t bal = __ballot_sync(0xffffffffu, set);
+        peers &= set ? bal : ~bal;
+    }
+    return peers;
+}
+__device__ __forceinline__ int bits_for(int n)      // smallest b with 2^b >= n
+{
+    int b = 0;
+    while ((1 << b) < n) ++b;
+    return b;
 }
 
 __global__ void __launch_bounds__(kSortThreads)
@@ -109,6 +130,7 @@ radix_scatter_kernel(const uint16_t *__restrict__ keys_in, const int32_t *__rest
     const int tile = blockIdx.x;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const uint32_t lt_mask = (1u << lane) - 1u;
+    const int rbits = bits_for(radix);
     for (int d = lane; d < radix; d += 32) wh[warp][d] = 0;
     __syncwarp();
     const uint16_t *kin = keys_in + seg * L;
@@ -117,8 +139,8 @@ radix_scatter_kernel(const uint16_t *__restrict__ keys_in, const int32_t *__rest
     for (int it = 0; it < kPerWarp / 32; ++it) {
         int pos = tile * kSortTile + warp * kPerWarp + it * 32 + lane;
         bool valid = pos < L;
-        uint32_t dg = valid ? ((kin[pos] >> shift) & (radix - 1)) : 0xFFFFFFFFu;
-        uint32_t peers = __match_any_sync(0xffffffffu, dg);
+        uint32_t dg = valid ? ((kin[pos] >> shift) & (radix - 1)) : (uint32_t)radix;
+        uint32_t peers = peers_of(dg, rbits);
         if (valid && (peers & lt_mask) == 0) wh[warp][dg] += __popc(peers);
         __syncwarp();
     }
@@ -139,8 +161,8 @@ radix_scatter_kernel(const uint16_t *__restrict__ keys_in, const int32_t *__rest
         int pos = tile * kSortTile + warp * kPerWarp + it * 32 + lane;
         bool valid = pos < L;
         uint16_t key = valid ? kin[pos] : 0;
-        uint32_t dg = valid ? ((key >> shift) & (radix - 1)) : 0xFFFFFFFFu;
-        uint32_t peers = __match_any_sync(0xffffffffu, dg);
+        uint32_t dg = valid ? ((key >> shift) & (radix - 1)) : (uint32_t)radix;
+        uint32_t peers = peers_of(dg, rbits);
         uint32_t rank = valid ? wh[warp][dg] + __popc(peers & lt_mask) : 0u;
         __syncwarp();
         if (valid && (peers & lt_mask) == 0) wh[warp][dg] += __popc(peers);
@@ -158,8 +180,9 @@ radix_scatter_kernel(const uint16_t *__restrict__ keys_in, const int32_t *__rest
 // by one CTA entirely in shared memory: the bucket ids are staged, each warp
 // counts the ids of its own contiguous run of positions, one exclusive scan in
 // (bucket, warp) order gives every warp's first output slot per bucket, and each
-// warp places its run in position order (match_any ranks equal ids inside a
-// 32-position step), so the result is the stable sort.  An id >= n_buckets
+// warp places its run in position order (equal ids inside a 32-position step
+// ranked by lane, the lanes found with one ballot per id bit), so the result
+// is the stable sort.  An id >= n_buckets
 // (invalid input) is counted as n_buckets - 1, which keeps every access in
 // bounds.  The permutation is
 // assembled in shared memory and written out with coalesced stores.
@@ -181,6 +204,7 @@ seg_sort_kernel(const uint16_t *__restrict__ buckets, int32_t *__restrict__ perm
     const long long seg = blockIdx.x;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const uint32_t lt_mask = (1u << lane) - 1u;
+    const int nbits = bits_for(nb);
     const uint16_t *k = buckets + seg * L;
     for (int e = threadIdx.x; e < L; e += kSegThreads) sm.keys[e] = k[e];
     for (int e = threadIdx.x; e < nb * kSegWarps; e += kSegThreads) sm.wh[e] = 0;
@@ -191,8 +215,8 @@ seg_sort_kernel(const uint16_t *__restrict__ buckets, int32_t *__restrict__ perm
     for (int it = 0; it < run; it += 32) {
         const int pos = p0 + it + lane;
         const bool valid = pos < L;
-        const uint32_t b = valid ? min((uint32_t)sm.keys[pos], (uint32_t)(nb - 1)) : 0xFFFFFFFFu;
-        const uint32_t peers = __match_any_sync(0xffffffffu, b);
+        const uint32_t b = valid ? min((uint32_t)sm.keys[pos], (uint32_t)(nb - 1)) : (1u << nbits);
+        const uint32_t peers = peers_of(b, nbits);
         if (valid && (peers & lt_mask) == 0) sm.wh[b * kSegWarps + warp] += __popc(peers);
         __syncwarp();
     }
@@ -232,8 +256,8 @@ seg_sort_kernel(const uint16_t *__restrict__ buckets, int32_t *__restrict__ perm
     for (int it = 0; it < run; it += 32) {
         const int pos = p0 + it + lane;
         const bool valid = pos < L;
-        const uint32_t b = valid ? min((uint32_t)sm.keys[pos], (uint32_t)(nb - 1)) : 0xFFFFFFFFu;
-        const uint32_t peers = __match_any_sync(0xffffffffu, b);
+        const uint32_t b = valid ? min((uint32_t)sm.keys[pos], (uint32_t)(nb - 1)) : (1u << nbits);
+        const uint32_t peers = peers_of(b, nbits);
         const uint32_t slot = valid ? sm.wh[b * kSegWarps + warp] + __popc(peers & lt_mask) : 0u;
         __syncwarp();
         if (valid && (peers & lt_mask) == 0) sm.wh[b * kSegWarps + warp] += __popc(peers);
