@@ -189,18 +189,32 @@ radix_scatter_kernel(const uint16_t *__restrict__ keys_in, const int32_t *__rest
 constexpr int kSegThreads = 1024;
 constexpr int kSegWarps = kSegThreads / 32;
 
+// Shared memory sized to the problem (so that two CTAs share an SM when they
+// fit): perm [L], warp_tot [32], wh [n_buckets][32 warps], keys [L].
 struct SegSortSmem {
-    uint16_t keys[kSegMaxL];
-    int32_t perm[kSegMaxL];
-    uint32_t wh[kSegMaxBuckets * kSegWarps];      // [bucket][warp]
-    uint32_t warp_tot[kSegWarps];
+    int32_t *perm;
+    uint32_t *warp_tot, *wh;
+    uint16_t *keys;
 };
+__host__ __device__ inline size_t seg_sort_smem_bytes(int L, int nb)
+{
+    return (size_t)L * 4 + kSegWarps * 4 + (size_t)nb * kSegWarps * 4 + ((size_t)L * 2 + 15) / 16 * 16;
+}
+__device__ inline SegSortSmem seg_sort_layout(uint8_t *base, int L, int nb)
+{
+    SegSortSmem m;
+    m.perm = reinterpret_cast<int32_t *>(base);
+    m.warp_tot = reinterpret_cast<uint32_t *>(base + (size_t)L * 4);
+    m.wh = m.warp_tot + kSegWarps;
+    m.keys = reinterpret_cast<uint16_t *>(m.wh + (size_t)nb * kSegWarps);
+    return m;
+}
 
 __global__ void __launch_bounds__(kSegThreads)
 seg_sort_kernel(const uint16_t *__restrict__ buckets, int32_t *__restrict__ perm, int L, int nb)
 {
     extern __shared__ __align__(16) uint8_t seg_smem[];
-    SegSortSmem &sm = *reinterpret_cast<SegSortSmem *>(seg_smem);
+    const SegSortSmem sm = seg_sort_layout(seg_smem, L, nb);
     const long long seg = blockIdx.x;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const uint32_t lt_mask = (1u << lane) - 1u;
@@ -275,8 +289,9 @@ cudaError_t launch_sort(const Problem &p, const uint16_t *buckets, int32_t *perm
                         cudaStream_t st)
 {
     if (seg_sort_fits(p)) {
-        const size_t smem = sizeof(SegSortSmem);
-        cudaError_t e = cudaFuncSetAttribute(seg_sort_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        const size_t smem = seg_sort_smem_bytes(p.L, p.nb);
+        cudaError_t e = cudaFuncSetAttribute(seg_sort_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)seg_sort_smem_bytes(kSegMaxL, kSegMaxBuckets));
         if (e != cudaSuccess) return e;
         seg_sort_kernel<<<(unsigned)p.S(), kSegThreads, smem, st>>>(buckets, perm, p.L, p.nb);
         return cudaGetLastError();
