@@ -70,7 +70,12 @@ def algorithmic(w: synth.Workload) -> dict:
         "attn_bwd": tok * (3 * d * e + 12 + R * 4) + tok * 2 * d * 4 * 2,  # x, v, dY, LSE, delta, norms, perm;
                                                                           # fp32 dx, dv accumulators in and out
     }
-    flops = {"hash": hash_flops, "attn_fwd": bh * L * R * 4 * 2 * m * d,
+    # the single-kernel forward of short segments: x and v read, the merged output
+    # written, per round the lse, the permutation and the bucket ids written (the
+    # rounds' outputs pass through L2 to the in-cluster merge)
+    kern["fused_fwd"] = tok * (3 * d * e + R * (4 + 4 + 2))
+    flops = {"hash": hash_flops, "fused_fwd": hash_flops + bh * L * R * 4 * 2 * m * d,
+             "attn_fwd": bh * L * R * 4 * 2 * m * d,
              "attn_bwd": bh * L * R * 10 * 2 * m * d if w.backward else 0, "combine": 0}
     return {"bytes": bh * (fwd + bwd), "attn_flops": attn_flops, "hash_flops": hash_flops, "kernel_bytes": kern,
             "kernel_flops": flops}

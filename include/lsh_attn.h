@@ -69,7 +69,7 @@
 extern "C" {
 #endif
 
-#define LSH_ATTN_ABI_VERSION 2
+#define LSH_ATTN_ABI_VERSION 3
 
 #if defined(__GNUC__)
 #define LSH_API __attribute__((visibility("default")))
@@ -199,7 +199,15 @@ LSH_API lsh_status lsh_attn_fwd_sorted(const lsh_attn_desc *desc, const void *qk
                                void *workspace, size_t ws_bytes, void *stream);
 
 /* Full forward: hash, sort, attention, merge.  perm_out (nullable) receives
- * the permutation so that lsh_attn_bwd need not recompute it. */
+ * the permutation so that lsh_attn_bwd need not recompute it.
+ *
+ * Where a (batch, head, round) segment fits on chip (bf16, L <= 4096,
+ * n_buckets <= 128, n_hashes <= 8; see lsh_attn_fused_forward_fits) the four
+ * steps run as one kernel, one cluster of n_hashes CTAs per head ("Sorting and
+ * Chunking": hash -> sort -> chunked attention with no HBM round trip for the
+ * bucket ids, the permutation or the key norms; the rounds are merged inside
+ * the cluster).  Its results are those of the staged kernels: the same
+ * products, the same argmax tie rule, the same merge arithmetic. */
 LSH_API lsh_status lsh_attn_fwd(const lsh_attn_desc *desc, const void *qk, const void *v, const void *R,
                         void *out, float *lse, int32_t *perm_out,
                         void *workspace, size_t ws_bytes, void *stream);
@@ -319,6 +327,7 @@ typedef enum {
     LSH_STAGE_BWD_PREP,      /* logsumexp over rounds, dY.Y, zero accumulators  */
     LSH_STAGE_ATTN_BWD,      /* chunk attention backward                        */
     LSH_STAGE_BWD_FINAL,     /* fp32 accumulators -> dqk, dv                    */
+    LSH_STAGE_FUSED_FWD,     /* hash + sort + attention + merge in one kernel   */
     LSH_STAGE_COUNT
 } lsh_stage;
 
@@ -330,6 +339,17 @@ LSH_API lsh_status lsh_attn_trace_end(float *ms, int32_t *calls, int32_t *kernel
  * left out is enqueued without events around it, so timing one kernel adds
  * only its own event pair to the stream.  Always returns LSH_OK. */
 LSH_API lsh_status lsh_attn_trace_stages(uint32_t mask);
+
+/* Single-kernel forward of short segments (lsh_attn_fwd, the reversible block
+ * and lsh_attn_step_host): enable = 1 (the default) uses it wherever it
+ * applies, 0 always runs the staged kernels (hash, sort, attention, merge),
+ * for comparisons.  Process-wide; takes effect for calls made after it.
+ * Returns LSH_ERR_ARG for any other value. */
+LSH_API lsh_status lsh_attn_fused_forward(int32_t enable);
+
+/* 1 if a forward with this descriptor runs as the single kernel under the
+ * current setting, 0 otherwise (also for an invalid descriptor). */
+LSH_API int32_t lsh_attn_fused_forward_fits(const lsh_attn_desc *desc);
 
 /* Self-test of the bounded device-side waits: launches one CTA that waits on a
  * barrier nothing completes, for `budget_cycles` SM cycles (>= 0).  The wait

@@ -25,13 +25,14 @@ STATUS = {0: "LSH_OK", -1: "LSH_ERR_ARG", -2: "LSH_ERR_SHAPE", -3: "LSH_ERR_ALIG
 
 EXPORTED = ("lsh_attn_make_rotations", "lsh_attn_workspace_size", "lsh_attn_hash", "lsh_attn_sort", "lsh_attn_sort_static", "lsh_attn_fwd_sorted", "lsh_attn_fwd",
             "lsh_attn_bwd", "lsh_attn_poll", "lsh_attn_selftest_timeout", "lsh_attn_trace_begin",
-            "lsh_attn_trace_end", "lsh_attn_trace_stages", "lsh_attn_last_near_ties",
+            "lsh_attn_trace_end", "lsh_attn_trace_stages", "lsh_attn_fused_forward",
+            "lsh_attn_fused_forward_fits", "lsh_attn_last_near_ties",
             "lsh_attn_status_str", "lsh_attn_last_error", "lsh_attn_abi_version",
             "lsh_attn_local_workspace_size", "lsh_attn_local_fwd", "lsh_attn_local_bwd",
             "lsh_rev_workspace_size", "lsh_rev_fwd", "lsh_rev_bwd",
             "lsh_attn_step_host_scratch_size", "lsh_attn_step_host")
 
-STAGES = ("hash", "sort", "norms", "attn_fwd", "combine", "bwd_prep", "attn_bwd", "bwd_final")
+STAGES = ("hash", "sort", "norms", "attn_fwd", "combine", "bwd_prep", "attn_bwd", "bwd_final", "fused_fwd")
 
 
 class LshAttnError(RuntimeError):
@@ -83,6 +84,9 @@ def load_library(path: str = LIB_PATH):
     L.lsh_attn_selftest_timeout.argtypes = [P, ctypes.c_int64, P]
     L.lsh_attn_trace_begin.argtypes = [ctypes.c_int32]
     L.lsh_attn_trace_stages.argtypes = [ctypes.c_uint32]
+    L.lsh_attn_fused_forward.argtypes = [ctypes.c_int32]
+    L.lsh_attn_fused_forward_fits.argtypes = [DP]
+    L.lsh_attn_fused_forward_fits.restype = ctypes.c_int32
     L.lsh_attn_trace_end.argtypes = [ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_int32),
                                      ctypes.POINTER(ctypes.c_int32), ctypes.c_int32]
     L.lsh_attn_last_near_ties.argtypes = []
@@ -285,6 +289,16 @@ def trace_stages(names=None):
     """Restricts what a trace records to the named stages (None: every stage)."""
     mask = 0xFFFFFFFF if names is None else sum(1 << STAGES.index(n) for n in names)
     _check(load_library().lsh_attn_trace_stages(mask), "lsh_attn_trace_stages")
+
+
+def fused_forward(enable: bool = True):
+    """Single-kernel forward of short segments on (default) or off (staged kernels), process-wide."""
+    _check(load_library().lsh_attn_fused_forward(1 if enable else 0), "lsh_attn_fused_forward")
+
+
+def fused_forward_fits(desc) -> bool:
+    """Whether a forward with this descriptor runs as the single kernel under the current setting."""
+    return bool(load_library().lsh_attn_fused_forward_fits(ctypes.byref(desc)))
 
 
 def trace_end() -> dict:

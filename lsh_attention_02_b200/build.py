@@ -9,8 +9,8 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 ROOT = os.path.dirname(HERE)
 LIB = os.path.join(HERE, "liblsh_attn.so")
-SOURCES = ["api.cu", "simt.cu", "sort.cu", "hash_tc.cu", "attn_fwd_tc.cu", "attn_bwd_tc.cu", "selftest.cu",
-           "rotations.cu", "revblock.cu"]
+SOURCES = ["api.cu", "simt.cu", "sort.cu", "hash_tc.cu", "attn_fwd_tc.cu", "fused_fwd_tc.cu", "attn_bwd_tc.cu",
+           "selftest.cu", "rotations.cu", "revblock.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-shared", "-Xcompiler", "-fPIC,-fvisibility=hidden",
          "--expt-relaxed-constexpr", "-I", os.path.join(ROOT, "include")]

@@ -179,6 +179,25 @@ static lsh_status run_attn_fwd(const Problem &p, const Choice &c, const void *qk
     return LSH_OK;
 }
 
+// The whole forward from the rotations: one kernel per head's rounds where a
+// segment fits on chip (and the single-kernel forward is enabled), otherwise
+// hash, sort, attention and merge as separate stages.
+static int g_fused_forward = 1;
+static bool use_fused(const Problem &p, const Choice &c) { return g_fused_forward && c.tc_attn && fused_fwd_fits(p); }
+static lsh_status run_forward(const Problem &p, const Choice &c, const void *qk, const void *v, const void *R,
+                              int32_t *perm, void *out, float *lse, const Workspace &w, cudaStream_t st)
+{
+    if (use_fused(p, c)) {
+        LSH_TRY(staged(LSH_STAGE_FUSED_FWD, 1, st, [&] {
+                    return launch_fused_fwd_tc(p, qk, v, R, perm, w.buckets, w.invnorm, w.o_r, lse, out, w.status, st);
+                }), "single-kernel forward");
+        return LSH_OK;
+    }
+    lsh_status s;
+    if ((s = run_hash_sort(p, c, qk, R, perm, w, st)) != LSH_OK) return s;
+    return run_attn_fwd(p, c, qk, v, perm, out, lse, w, st, c.tc_hash);
+}
+
 // prologue, attention backward and epilogue for a given permutation (shared by
 // lsh_attn_bwd and the reversible block)
 static lsh_status run_attn_bwd(const Problem &p, const Choice &c, const void *qk, const void *v, const void *out,
@@ -325,8 +344,7 @@ lsh_status lsh_attn_fwd(const lsh_attn_desc *desc, const void *qk, const void *v
     cudaStream_t st = (cudaStream_t)stream;
     int32_t *perm = perm_out ? perm_out : w.perm;
     LSH_TRY(cudaMemsetAsync(w.status, 0, sizeof(uint32_t), st), "status reset");
-    if ((s = run_hash_sort(p, c, qk, R, perm, w, st)) != LSH_OK) return s;
-    return run_attn_fwd(p, c, qk, v, perm, out, lse, w, st, c.tc_hash);
+    return run_forward(p, c, qk, v, R, perm, out, lse, w, st);
 }
 
 lsh_status lsh_attn_bwd(const lsh_attn_desc *desc, const void *qk, const void *v, const void *R, const void *out,
@@ -521,8 +539,7 @@ lsh_status lsh_rev_fwd(const lsh_attn_desc *desc, const float *x1, const float *
     cudaStream_t st = (cudaStream_t)stream;
     LSH_TRY(cudaMemsetAsync(w.status, 0, sizeof(uint32_t), st), "status reset");
     LSH_TRY(launch_cast(p, x2, r.xa, st), "x2 to the attention dtype");
-    if ((s = run_hash_sort(p, c, r.xa, R, r.perm, w, st)) != LSH_OK) return s;
-    if ((s = run_attn_fwd(p, c, r.xa, r.xa, r.perm, r.f, r.lse, w, st, c.tc_hash)) != LSH_OK) return s;   // F(x2)
+    if ((s = run_forward(p, c, r.xa, r.xa, R, r.perm, r.f, r.lse, w, st)) != LSH_OK) return s;   // F(x2)
     LSH_TRY(launch_axpy(p, x1, r.f, 1.f, y1, st), "y1 = x1 + F(x2)");
     LSH_TRY(launch_g_forward(p, y1, Wg, bg, x2, y2, nullptr, st), "y2 = x2 + G(y1)");
     return LSH_OK;
@@ -551,8 +568,7 @@ lsh_status lsh_rev_bwd(const lsh_attn_desc *desc, const float *y1, const float *
     LSH_TRY(launch_g_backward(p, r.g, dy2, Wg, dy1, dx1, st), "dx1 = dy1 + J_G^T dy2");
     // inverse of the F half: F(x2) again (hash, sort, attention), x1 = y1 - F(x2)
     LSH_TRY(launch_cast(p, x2, r.xa, st), "x2 to the attention dtype");
-    if ((s = run_hash_sort(p, c, r.xa, R, r.perm, wf, st)) != LSH_OK) return s;
-    if ((s = run_attn_fwd(p, c, r.xa, r.xa, r.perm, r.f, r.lse, wf, st, c.tc_hash)) != LSH_OK) return s;
+    if ((s = run_forward(p, c, r.xa, r.xa, R, r.perm, r.f, r.lse, wf, st)) != LSH_OK) return s;
     LSH_TRY(launch_axpy(p, y1, r.f, -1.f, x1, st), "x1 = y1 - F(x2)");
     // gradient through F, whose query-key and value inputs are both x2
     LSH_TRY(launch_cast(p, dx1, r.da, st), "dF to the attention dtype");
@@ -688,8 +704,7 @@ lsh_status lsh_attn_step_host(const lsh_attn_desc *desc, int32_t heads_per_chunk
         pc.H = nh;
         Workspace wf = plan_workspace(pc, false, c.tc_attn, c.tc_hash, sl.ws);
         wf.status = status;
-        if ((rc = run_hash_sort(pc, c, sl.x, h.R, sl.perm, wf, cs)) != LSH_OK) break;
-        if ((rc = run_attn_fwd(pc, c, sl.x, sl.v, sl.perm, sl.out, sl.lse, wf, cs, c.tc_hash)) != LSH_OK) break;
+        if ((rc = run_forward(pc, c, sl.x, sl.v, h.R, sl.perm, sl.out, sl.lse, wf, cs)) != LSH_OK) break;
         if (bwd) {
             Workspace wb = plan_workspace(pc, true, c.tc_attn, c.tc_hash, sl.ws);
             wb.status = status;
@@ -767,6 +782,20 @@ lsh_status lsh_attn_trace_stages(uint32_t mask)
 {
     g_trace_mask = mask;
     return LSH_OK;
+}
+
+lsh_status lsh_attn_fused_forward(int32_t enable)
+{
+    if (enable != 0 && enable != 1) return LSH_ERR_ARG;
+    g_fused_forward = enable;
+    return LSH_OK;
+}
+
+int32_t lsh_attn_fused_forward_fits(const lsh_attn_desc *desc)
+{
+    Problem p;
+    if (check_desc(desc, &p) != LSH_OK || check_envelope(p) != LSH_OK) return 0;
+    return use_fused(p, choose(p)) ? 1 : 0;
 }
 
 lsh_status lsh_attn_trace_end(float *ms, int32_t *calls, int32_t *kernels, int32_t n)

@@ -163,6 +163,14 @@ cudaError_t launch_attn_fwd_tc(const Problem &p, const void *x, const void *v, c
                                const uint16_t *bkt, const float *xinv, __nv_bfloat16 *o_r, float *lse,
                                uint32_t *status, cudaStream_t st);
 bool attn_tc_supported(const Problem &p);
+// Single-kernel forward of short segments (hash, sort, attention and merge in one
+// cluster of R CTAs per head): perm [S, L], bkt [S, L] (bucket ids by position),
+// xinv [BH, L] (1/|x|) and lse [S, L] are outputs, o_r [S, L, 64] bf16 is
+// scratch, out [BH, L, 64] bf16 the merged output.
+bool fused_fwd_fits(const Problem &p);
+cudaError_t launch_fused_fwd_tc(const Problem &p, const void *x, const void *v, const void *R, int32_t *perm,
+                                uint16_t *bkt, float *xinv, void *o_r, float *lse, void *out, uint32_t *status,
+                                cudaStream_t st);
 // lse_out (nullable): receives logsumexp over the rounds, [BH, L]
 cudaError_t launch_combine(const Problem &p, const void *o_r, bool o_r_bf16, const float *lse, void *out,
                            float *lse_out, cudaStream_t st);

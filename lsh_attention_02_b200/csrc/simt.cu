@@ -10,7 +10,7 @@
 // equation); a (b, h, r) segment holds one round's permutation.
 #include <math.h>
 
-#include "common.cuh"
+#include "combine.cuh"
 
 namespace lsh {
 
@@ -343,10 +343,8 @@ __global__ void combine_kernel(const OT *__restrict__ o_r, const float *__restri
     for (int k = 0; k < 4; ++k) y[k] = from_f<T>(acc[k]);
 }
 
-// bf16 round outputs: 8 threads per token, eight features each (16-byte loads
-// and stores); the token's logsumexps are read by every thread of its group.
-// RMAX > 0: the R <= RMAX round rows are all loaded before any arithmetic, so
-// their memory latencies overlap; RMAX = 0 handles any R one round at a time.
+// bf16 round outputs: 8 threads per token, eight features each
+// (combine_token_bf16).
 template <int RMAX>
 __global__ void combine_bf16_kernel(const __nv_bfloat16 *__restrict__ o_r, const float *__restrict__ lse,
                                     __nv_bfloat16 *__restrict__ out, float *__restrict__ lse_out, long long tokens,
@@ -361,48 +359,8 @@ __global__ void combine_bf16_kernel(const __nv_bfloat16 *__restrict__ o_r, const
     const float *lp = lse + bh * R * (long long)L + i;
     const uint4 *orow = reinterpret_cast<const uint4 *>(o_r + (bh * R * (long long)L + i) * kDim) + oct;
     const long long rstride = (long long)L * kDim / 8;          // one round, in 16-byte units
-    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    auto accumulate = [&](float wr, const uint4 &u) {
-        const uint32_t wd[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            acc[2 * e] = fmaf(wr, __uint_as_float(wd[e] << 16), acc[2 * e]);
-            acc[2 * e + 1] = fmaf(wr, __uint_as_float(wd[e] & 0xFFFF0000u), acc[2 * e + 1]);
-        }
-    };
-    if (RMAX > 0) {
-        uint4 u[RMAX > 0 ? RMAX : 1];
-        float lr[RMAX > 0 ? RMAX : 1];
-#pragma unroll
-        for (int r = 0; r < RMAX; ++r) {
-            u[r] = r < R ? __ldg(orow + r * rstride) : make_uint4(0, 0, 0, 0);
-            lr[r] = r < R ? __ldg(lp + (long long)r * L) : -INFINITY;
-        }
-        float mx = -INFINITY;
-#pragma unroll
-        for (int r = 0; r < RMAX; ++r) mx = fmaxf(mx, lr[r]);
-        float w[RMAX > 0 ? RMAX : 1], ssum = 0.f;
-#pragma unroll
-        for (int r = 0; r < RMAX; ++r) {
-            w[r] = r < R ? expf(lr[r] - mx) : 0.f;
-            ssum += w[r];
-        }
-        const float inv = 1.f / ssum;
-        if (lse_out && oct == 0) lse_out[tok] = mx + logf(ssum);
-#pragma unroll
-        for (int r = 0; r < RMAX; ++r) accumulate(w[r] * inv, u[r]);
-    } else {
-        float mx = -INFINITY;
-        for (int r = 0; r < R; ++r) mx = fmaxf(mx, lp[(long long)r * L]);
-        float ssum = 0.f;
-        for (int r = 0; r < R; ++r) ssum += expf(lp[(long long)r * L] - mx);
-        if (lse_out && oct == 0) lse_out[tok] = mx + logf(ssum);
-        const float inv = 1.f / ssum;
-        for (int r = 0; r < R; ++r) accumulate(expf(lp[(long long)r * L] - mx) * inv, orow[r * rstride]);
-    }
-    reinterpret_cast<uint4 *>(out + tok * kDim)[oct] =
-        make_uint4(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]), pack_bf16x2(acc[4], acc[5]),
-                   pack_bf16x2(acc[6], acc[7]));
+    combine_token_bf16<RMAX, false>(orow, rstride, lp, L, R, reinterpret_cast<uint4 *>(out + tok * kDim) + oct,
+                                    lse_out ? lse_out + tok : nullptr, oct);
 }
 
 cudaError_t launch_combine(const Problem &p, const void *o_r, bool o_r_bf16, const float *lse, void *out,

@@ -20,7 +20,7 @@
 // Pass 0 reads the bucket ids in position order with the position as the
 // value; the last pass writes only the values, i.e. the permutation.
 
-#include "common.cuh"
+#include "seg_sort.cuh"
 
 namespace lsh {
 
@@ -39,25 +39,6 @@ SortPlan make_sort_plan(int n_buckets, int L)
     return sp;
 }
 
-// Lanes of the warp whose key equals this lane's, from one ballot per key bit
-// (keys below 2^nbits; a lane with key 2^nbits, an out-of-range marker, matches
-// only lanes with the same marker).
-__device__ __forceinline__ uint32_t peers_of(uint32_t key, int nbits)
-{
-    uint32_t peers = 0xffffffffu;
-    for (int bit = 0; bit <= nbits; ++bit) {
-        const bool set = (key >> bit) & 1u;
-        const uint32_t bal = __ballot_sync(0xffffffffu, set);
-        peers &= set ? bal : ~bal;
-    }
-    return peers;
-}
-__device__ __forceinline__ int bits_for(int n)      // smallest b with 2^b >= n
-{
-    int b = 0;
-    while ((1 << b) < n) ++b;
-    return b;
-}
 
 __global__ void __launch_bounds__(kSortThreads)
 radix_count_kernel(const uint16_t *__restrict__ keys, uint32_t *__restrict__ counts, int L, int n_tiles,
@@ -177,14 +158,8 @@ radix_scatter_kernel(const uint16_t *__restrict__ keys_in, const int32_t *__rest
 
 // ------------------------------------------------------------ small segments
 // A segment of at most kSegMaxL positions and kSegMaxBuckets buckets is sorted
-// by one CTA entirely in shared memory: the bucket ids are staged, each warp
-// counts the ids of its own contiguous run of positions, one exclusive scan in
-// (bucket, warp) order gives every warp's first output slot per bucket, and each
-// warp places its run in position order (equal ids inside a 32-position step
-// ranked by lane, the lanes found with one ballot per id bit), so the result
-// is the stable sort.  An id >= n_buckets
-// (invalid input) is counted as n_buckets - 1, which keeps every access in
-// bounds.  The permutation is
+// by one CTA entirely in shared memory (seg_sort_block: per-warp counts, one
+// scan in (bucket, warp) order, stable placement); the permutation is
 // assembled in shared memory and written out with coalesced stores.
 constexpr int kSegThreads = 1024;
 constexpr int kSegWarps = kSegThreads / 32;
@@ -216,69 +191,10 @@ seg_sort_kernel(const uint16_t *__restrict__ buckets, int32_t *__restrict__ perm
     extern __shared__ __align__(16) uint8_t seg_smem[];
     const SegSortSmem sm = seg_sort_layout(seg_smem, L, nb);
     const long long seg = blockIdx.x;
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const uint32_t lt_mask = (1u << lane) - 1u;
-    const int nbits = bits_for(nb);
     const uint16_t *k = buckets + seg * L;
     for (int e = threadIdx.x; e < L; e += kSegThreads) sm.keys[e] = k[e];
-    for (int e = threadIdx.x; e < nb * kSegWarps; e += kSegThreads) sm.wh[e] = 0;
     __syncthreads();
-    const int run = (L + kSegWarps * 32 - 1) / (kSegWarps * 32) * 32;   // positions per warp, a multiple of 32
-    const int p0 = warp * run;
-    // A: per-warp counts of every bucket id, in position order
-    for (int it = 0; it < run; it += 32) {
-        const int pos = p0 + it + lane;
-        const bool valid = pos < L;
-        const uint32_t b = valid ? min((uint32_t)sm.keys[pos], (uint32_t)(nb - 1)) : (1u << nbits);
-        const uint32_t peers = peers_of(b, nbits);
-        if (valid && (peers & lt_mask) == 0) sm.wh[b * kSegWarps + warp] += __popc(peers);
-        __syncwarp();
-    }
-    __syncthreads();
-    // B: exclusive scan of wh in (bucket, warp) order; thread t scans a contiguous span
-    const int n = nb * kSegWarps, per = (n + kSegThreads - 1) / kSegThreads;
-    const int e0 = min(n, threadIdx.x * per), e1 = min(n, e0 + per);
-    uint32_t tot = 0;
-    for (int e = e0; e < e1; ++e) tot += sm.wh[e];
-    uint32_t incl = tot;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const uint32_t t = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += t;
-    }
-    if (lane == 31) sm.warp_tot[warp] = incl;
-    __syncthreads();
-    if (warp == 0) {
-        const uint32_t wv = sm.warp_tot[lane];
-        uint32_t wi = wv;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const uint32_t t = __shfl_up_sync(0xffffffffu, wi, o);
-            if (lane >= o) wi += t;
-        }
-        sm.warp_tot[lane] = wi - wv;
-    }
-    __syncthreads();
-    uint32_t off = sm.warp_tot[warp] + incl - tot;
-    for (int e = e0; e < e1; ++e) {
-        const uint32_t c = sm.wh[e];
-        sm.wh[e] = off;
-        off += c;
-    }
-    __syncthreads();
-    // C: stable placement into shared memory, then coalesced copy out
-    for (int it = 0; it < run; it += 32) {
-        const int pos = p0 + it + lane;
-        const bool valid = pos < L;
-        const uint32_t b = valid ? min((uint32_t)sm.keys[pos], (uint32_t)(nb - 1)) : (1u << nbits);
-        const uint32_t peers = peers_of(b, nbits);
-        const uint32_t slot = valid ? sm.wh[b * kSegWarps + warp] + __popc(peers & lt_mask) : 0u;
-        __syncwarp();
-        if (valid && (peers & lt_mask) == 0) sm.wh[b * kSegWarps + warp] += __popc(peers);
-        __syncwarp();
-        if (valid) sm.perm[slot] = pos;
-    }
-    __syncthreads();
+    seg_sort_block<kSegWarps>(sm.keys, L, nb, sm.wh, sm.warp_tot, sm.perm);
     int32_t *out = perm + seg * L;
     for (int e = threadIdx.x; e < L; e += kSegThreads) out[e] = sm.perm[e];
 }

@@ -172,3 +172,24 @@ def test_local_attention_argument_rules(lib):
     assert lib.lsh_attn_local_fwd(ctypes.byref(ok), 2, fake, fake, fake, fake, fake, big, None) == -4
     assert lib.lsh_attn_local_bwd(ctypes.byref(ok), 1, fake, fake, None, fake, fake, fake, fake, fake, big,
                                   None) == -1
+
+
+def test_fused_forward_applies_to_short_bf16_segments_only(lib):
+    """The single-kernel forward is chosen on the host from the descriptor alone:
+    bf16, chunk 64, L a multiple of 64 up to 4096, n_buckets <= 128,
+    n_hashes <= 8; the switch turns it off for every shape."""
+    fits = lambda **kw: lib.lsh_attn_fused_forward_fits(ctypes.byref(_desc(**kw)))
+    assert fits(L=4096, n_buckets=64, n_hashes=2, B=8, H=8, causal=1) == 1
+    assert fits(L=64) == 1 and fits(L=960, n_buckets=2) == 1 and fits(n_buckets=128, n_hashes=8) == 1
+    assert fits(L=4160) == 0                       # longer than a segment held on chip
+    assert fits(n_buckets=130) == 0                # more rotation columns than the kernel holds
+    assert fits(n_hashes=9) == 0                   # more rounds than a portable cluster has CTAs
+    assert fits(dtype=lsh.LSH_F32) == 0            # fp32 runs on the CUDA-core kernels
+    assert fits(chunk=32) == 0 and fits(B=1, H=1, L=64) == 0
+    assert lib.lsh_attn_fused_forward(2) == -1     # LSH_ERR_ARG
+    assert lib.lsh_attn_fused_forward(0) == 0
+    try:
+        assert fits(L=4096, n_buckets=64) == 0
+    finally:
+        assert lib.lsh_attn_fused_forward(1) == 0
+    assert fits(L=4096, n_buckets=64) == 1

@@ -574,19 +574,29 @@ def test_trace_records_only_selected_stages():
     desc = lsh.desc_for(x, w.n_buckets, w.n_hashes, w.chunk, w.causal)
     out, lse, perm = lsh.outputs_like(desc, x)
     ws = lsh.workspace(desc, False, x.device)
-    lsh.lsh_attn_fwd(desc, x, v, R, out, lse, perm, ws)
-    ref = out.clone()
+    lsh.fused_forward(False)                     # the staged kernels, one stage each
     try:
-        lsh.trace_stages(["attn_fwd"])
+        lsh.lsh_attn_fwd(desc, x, v, R, out, lse, perm, ws)
+        ref = out.clone()
+        try:
+            lsh.trace_stages(["attn_fwd"])
+            lsh.trace_begin(16)
+            lsh.lsh_attn_fwd(desc, x, v, R, out, lse, perm, ws)
+            st = lsh.trace_end()
+        finally:
+            lsh.trace_stages(None)
+        assert st["attn_fwd"][1] == 1 and st["attn_fwd"][0] > 0
+        assert all(st[k][1] == 0 for k in st if k != "attn_fwd")
+        assert torch.equal(out, ref)
         lsh.trace_begin(16)
         lsh.lsh_attn_fwd(desc, x, v, R, out, lse, perm, ws)
         st = lsh.trace_end()
+        assert st["hash"][1] == 1 and st["sort"][1] == 1 and st["combine"][1] == 1
     finally:
-        lsh.trace_stages(None)
-    assert st["attn_fwd"][1] == 1 and st["attn_fwd"][0] > 0
-    assert all(st[k][1] == 0 for k in st if k != "attn_fwd")
-    assert torch.equal(out, ref)
+        lsh.fused_forward(True)
+    # the single kernel: one stage of its own, same output
     lsh.trace_begin(16)
     lsh.lsh_attn_fwd(desc, x, v, R, out, lse, perm, ws)
     st = lsh.trace_end()
-    assert st["hash"][1] == 1 and st["sort"][1] == 1 and st["combine"][1] == 1
+    assert st["fused_fwd"][1] == 1 and all(st[k][1] == 0 for k in st if k != "fused_fwd")
+    assert torch.equal(out, ref)
