@@ -5,15 +5,17 @@
 // rounds' outputs, which the merge reads back from L2.
 //
 // Per CTA (segment (bh, r), L <= kMaxL positions, n_buckets <= 2 kMaxHalf):
-//   hash       the segment's x rows by TMA tile loads (128 rows, 128-byte
-//              swizzle) into a ring of kHashTiles tiles laid over the attention
-//              stages' memory; x R_r on the tensor cores (M = 128, N = n_buckets/2
-//              rounded up to 16, K = 64) into kAccBufs TMEM buffers; two groups
-//              of four warps take alternate tiles: the first maximum of
+//   hash       split over the cluster: CTA r loads x tiles r, r + R, ... of the
+//              head (TMA tile loads, 128 rows, 128-byte swizzle) into a ring laid
+//              over the attention stages' memory and multiplies each by the
+//              rotations of every round at once on the tensor cores (M = 128, N up
+//              to 128 columns per MMA, into TMEM); two groups of four warps take
+//              alternate products: per round the first maximum of
 //              [x R_r ; -x R_r] ("LSH Attention", hash equation; the oracle's tie
-//              rule) and 1/|x| of each row, kept in shared memory; each warp's 32
-//              consecutive positions also get their rank among equal bucket ids
-//              and the group's count per bucket (one ballot per id bit);
+//              rule), and for each warp's 32 consecutive positions their rank
+//              among equal ids and the group's count per id (one ballot per id
+//              bit), all written into that round's CTA (distributed shared
+//              memory); 1/|x| of each row to global memory;
 //   sort       a stable counting sort from those counts: one exclusive scan in
 //              (bucket, group) order gives every group's first slot per bucket,
 //              and each position goes to that slot plus its rank; the
@@ -29,9 +31,34 @@
 // Every wait on an mbarrier is bounded (the status word gets the timeout bit
 // and every role unwinds); the cluster barrier is reached by every thread of
 // every CTA on every path.
+#include <cooperative_groups.h>
+
 #include "attn_fwd_roles.cuh"
 #include "combine.cuh"
 #include "seg_sort.cuh"
+
+namespace cg = cooperative_groups;
+
+// Tuning build: the global timer (ns) of every CTA at its phase boundaries.
+#ifdef LSH_PHASE_TRACE
+static __device__ unsigned long long lsh_cta_trace[1024][6];
+#define LSH_CTA_MARK(ev)                                                          \
+    do {                                                                          \
+        if (threadIdx.x == 0 && blockIdx.x < 1024) {                              \
+            unsigned long long t_;                                                \
+            asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t_));                \
+            lsh_cta_trace[blockIdx.x][ev] = t_;                                   \
+        }                                                                         \
+    } while (0)
+extern "C" LSH_API int lsh_attn_cta_trace_fused(unsigned long long *out)
+{
+    return (int)cudaMemcpyFromSymbol(out, lsh_cta_trace, sizeof(lsh_cta_trace));
+}
+#else
+#define LSH_CTA_MARK(ev) \
+    do {                 \
+    } while (0)
+#endif
 
 namespace lsh {
 
@@ -43,8 +70,9 @@ constexpr int kMaxL = 4096;             // positions per segment
 constexpr int kMaxHalf = 64;            // n_buckets / 2
 constexpr int kMaxRounds = 8;           // CTAs per cluster (portable cluster size)
 constexpr int kRingStages = 4;
-constexpr int kHashTiles = 8;           // x tiles of 128 rows (16 KB) in flight during the hash
-constexpr int kAccBufs = 8;             // TMEM accumulators of 64 columns
+constexpr int kHashTiles = 8;           // at most this many x tiles of 128 rows (16 KB) in flight
+constexpr int kAccBufs = 4;             // TMEM accumulators of 128 columns
+constexpr int kAccCols = 128;
 constexpr int kWarps = kThreads / 32;
 constexpr int kHashProducerWarp = kSoftmaxWarps;   // TMA loads of the hash phase
 constexpr uint32_t kTileBytes = 128 * 128;
@@ -57,22 +85,23 @@ struct FusedSmem {
     uint64_t a_full[kHashTiles], a_empty[kHashTiles];
     uint64_t acc_full[kAccBufs], acc_empty[kAccBufs];
 };
-static_assert(kHashTiles * kTileBytes <= sizeof(Stage) * kRingStages, "hash tiles fit in the stage memory");
+static_assert(kAccBufs * kAccCols <= kTmemCols, "hash accumulators fit in tensor memory");
 
-// Hash and sort scratch in the stage memory.  During the hash, beyond the x
-// tiles: the count of each bucket in each group of 32 consecutive positions
-// (u8, [bucket][group]), each position's rank among the equal buckets of its
-// group (u8), and R_r^T (rows n of 64 k, K-major SW128).  After the hash, over
-// the x tiles: the first sorted slot of each (bucket, group) (u16, same order).
+// Hash and sort scratch in the stage memory, during the hash: n_buf x tiles
+// (16 KB each), then this CTA's round's count of each bucket in each group of
+// 32 consecutive positions (u8, [bucket][group]) and each position's rank among
+// the equal buckets of its group (u8), then the rotations of every round
+// (R_r^T stacked: rows r * hp + n of 64 k, K-major SW128).  After the hash,
+// over the x tiles: the first sorted slot of each (bucket, group) (u16, same
+// order).
 constexpr int kGroups = kMaxL / 32;
-constexpr size_t kCntOff = (size_t)kHashTiles * kTileBytes;
-constexpr size_t kRankOff = kCntOff + (size_t)2 * kMaxHalf * kGroups;
-constexpr size_t kRotOff = kRankOff + kMaxL;
-constexpr size_t kSlotOff = 0;
-static_assert(kRotOff % 1024 == 0, "the rotation tile is 1024-byte aligned");
-static_assert(kRotOff + (size_t)kMaxHalf * 128 <= sizeof(Stage) * kRingStages, "hash scratch fits in the stages");
-static_assert(kSlotOff + (size_t)2 * kMaxHalf * kGroups * 2 <= kCntOff, "first slots fit over the hash tiles");
-static_assert(kAccBufs * 64 <= kTmemCols, "hash accumulators fit in tensor memory");
+constexpr size_t kStageBytes = sizeof(Stage) * kRingStages;
+constexpr size_t kCntBytes = (size_t)2 * kMaxHalf * kGroups;
+constexpr size_t kTablesBytes = kCntBytes + kMaxL;
+constexpr size_t kRotMaxBytes = (size_t)kMaxRounds * kMaxHalf * 128;
+static_assert(kTablesBytes % 1024 == 0, "the rotation tile stays 1024-byte aligned");
+static_assert(7 * kTileBytes + kTablesBytes + kRotMaxBytes <= kStageBytes, "at least 7 x tiles beside the tables");
+static_assert(kCntBytes * 2 <= 7 * kTileBytes, "first slots fit over the x tiles");
 
 __device__ __forceinline__ uint8_t *hash_tile(FusedSmem &sm, int b)
 {
@@ -181,12 +210,28 @@ fused_fwd_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __nv_bfloat1
     const int half = nb / 2, hp = half <= 32 ? 32 : 64;        // rotation columns, zero beyond half
     const int n_mt = (L + 127) / 128;               // hash tiles
     const int n_k = (L + kQ - 1) / kQ;              // attention tiles
+    // The hash is split over the cluster: CTA r loads x tiles t = r, r + R, ...
+    // and hashes them for every round at once (all rounds' rotations side by side,
+    // rg rounds per MMA of N = rg * hp <= 128 columns, n_rg MMAs per tile); each
+    // round's bucket ids, ranks and counts go to that round's CTA.
+    const int rg = kAccCols / hp, n_rg = (R + rg - 1) / rg;
+    const int n_local = r < n_mt ? (n_mt - r + R - 1) / R : 0;
+    const int n_items = n_local * n_rg;
+    const size_t rot_bytes = (size_t)R * hp * 128;
+    const int n_buf = (int)min((size_t)kHashTiles, (kStageBytes - kTablesBytes - rot_bytes) / kTileBytes);
+    uint8_t *const stage_mem = reinterpret_cast<uint8_t *>(ring.st);
+    uint8_t *const cnt = stage_mem + (size_t)n_buf * kTileBytes;
+    uint8_t *const rank = cnt + kCntBytes;
+    uint8_t *const rot_t = rank + kMaxL;
+    uint16_t *const first = reinterpret_cast<uint16_t *>(stage_mem);
+    const int n_groups = (L + 31) / 32, nbits = bits_for(nb);
+    cg::cluster_group cluster = cg::this_cluster();
 
     if (threadIdx.x == 0) {
         ring_init(ring);
         for (int b = 0; b < kHashTiles; ++b) {
             tc::mbar_init(&sm.a_full[b], 1);
-            tc::mbar_init(&sm.a_empty[b], 4);
+            tc::mbar_init(&sm.a_empty[b], 4 * n_rg);    // every item of the tile has read it
         }
         for (int a = 0; a < kAccBufs; ++a) {
             tc::mbar_init(&sm.acc_full[a], 1);
@@ -195,127 +240,139 @@ fused_fwd_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __nv_bfloat1
         tc::fence_mbar_init();
     }
     if (warp == 0) tc::tmem_alloc(&ring.tmem_base, kTmemCols);
-    uint8_t *const stage_mem = reinterpret_cast<uint8_t *>(ring.st);
-    uint8_t *const cnt = stage_mem + kCntOff;
-    uint8_t *const rank = stage_mem + kRankOff;
-    uint16_t *const first = reinterpret_cast<uint16_t *>(stage_mem + kSlotOff);
-    uint8_t *const rot_t = stage_mem + kRotOff;
-    const int n_groups = (L + 31) / 32, nbits = bits_for(nb);
     for (int e = threadIdx.x; e < (nb * n_groups + 15) / 16; e += kThreads)   // within the 16 KB table
         reinterpret_cast<uint4 *>(cnt)[e] = make_uint4(0, 0, 0, 0);
-    // R_r^T into the K-major swizzled B layout; columns n >= half are zero (never
-    // a first maximum: see the argmax below, which reads only n < half)
-    for (int e = threadIdx.x; e < hp * kDim; e += kThreads) {
-        const int n = e % hp, k = e / hp;
-        const __nv_bfloat16 val = n < half ? rot[((long long)r * kDim + k) * half + n] : __float2bfloat16_rn(0.f);
-        *reinterpret_cast<__nv_bfloat16 *>(rot_t + tc::sw128_offset((uint32_t)n, (uint32_t)k)) = val;
+    // R_r^T of every round into the K-major swizzled B layout; columns n >= half
+    // of a round are zero (never a first maximum: see first_max_bucket)
+    for (int e = threadIdx.x; e < R * hp * kDim; e += kThreads) {
+        const int nn = e % (R * hp), k = e / (R * hp), rr = nn / hp, n = nn % hp;
+        const __nv_bfloat16 val =
+            n < half ? rot[((long long)rr * kDim + k) * half + n] : __float2bfloat16_rn(0.f);
+        *reinterpret_cast<__nv_bfloat16 *>(rot_t + tc::sw128_offset((uint32_t)nn, (uint32_t)k)) = val;
     }
     tc::fence_async_smem();
     tc::tc_fence_before();
-    __syncthreads();
+    cluster_sync_all();                 // every CTA's tables are zero before any peer writes into them
     tc::tc_fence_after();
     const uint32_t tmem = ring.tmem_base;
     if (threadIdx.x == 0) LSH_PHASE(0, 7, 0, 0);
+    LSH_CTA_MARK(0);
 
     // ================= hash
     if (warp == kHashProducerWarp) {
         if (lane == 0) {
             tc::prefetch_tmap(&xmap);
-            for (int t = 0; t < n_mt; ++t) {
-                const int b = t % kHashTiles;
-                if (t >= kHashTiles &&
-                    !tc::mbar_wait(&sm.a_empty[b], (uint32_t)((t / kHashTiles) - 1) & 1u, &ring.abort, status))
+            for (int u = 0; u < n_local; ++u) {
+                const int b = u % n_buf, t = r + u * R;
+                if (u >= n_buf &&
+                    !tc::mbar_wait(&sm.a_empty[b], (uint32_t)((u / n_buf) - 1) & 1u, &ring.abort, status))
                     break;
-                LSH_PHASE(0, 4, t, 0);
+                LSH_PHASE(0, 4, u, 0);
                 tc::mbar_arrive_expect_tx(&sm.a_full[b], kTileBytes);
                 tc::tma_load_2d(hash_tile(sm, b), &xmap, 0, (int)(bh * L + (long long)t * 128), &sm.a_full[b]);
             }
         }
     } else if (warp == kMmaWarp) {
         if (lane == 0) {
-            const uint32_t id = tc::idesc_bf16(128, hp, 0, 0);
             const uint32_t rs = tc::smem_u32(rot_t);
-            for (int t = 0; t < n_mt; ++t) {
-                const int b = t % kHashTiles, a = t % kAccBufs;
-                if (!tc::mbar_wait(&sm.a_full[b], (uint32_t)(t / kHashTiles) & 1u, &ring.abort, status)) break;
-                LSH_PHASE(0, 5, t, 0);
-                if (t >= kAccBufs &&
-                    !tc::mbar_wait(&sm.acc_empty[a], (uint32_t)((t / kAccBufs) - 1) & 1u, &ring.abort, status))
-                    break;
-                tc::tc_fence_after();
+            bool go = true;
+            for (int u = 0; go && u < n_local; ++u) {
+                const int b = u % n_buf;
+                if (!tc::mbar_wait(&sm.a_full[b], (uint32_t)(u / n_buf) & 1u, &ring.abort, status)) break;
+                LSH_PHASE(0, 5, u, 0);
                 const uint32_t xs = tc::smem_u32(hash_tile(sm, b));
+                for (int g = 0; g < n_rg; ++g) {
+                    const int it = u * n_rg + g, a = it % kAccBufs;
+                    if (it >= kAccBufs &&
+                        !tc::mbar_wait(&sm.acc_empty[a], (uint32_t)((it / kAccBufs) - 1) & 1u, &ring.abort, status)) {
+                        go = false;
+                        break;
+                    }
+                    tc::tc_fence_after();
+                    const int nr = min(rg, R - g * rg);
+                    const uint32_t id = tc::idesc_bf16(128, nr * hp, 0, 0);
+                    const uint32_t bs = rs + (uint32_t)(g * rg * hp * 128);
 #pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                    tc::mma_bf16(tmem + (uint32_t)(a * 64), tc::sw128_desc(xs + kk * 32), tc::sw128_desc(rs + kk * 32),
-                                 id, kk > 0);
-                tc::mma_commit(&sm.acc_full[a]);
-                LSH_PHASE(0, 5, t, 1);
+                    for (int kk = 0; kk < 4; ++kk)
+                        tc::mma_bf16(tmem + (uint32_t)(a * kAccCols), tc::sw128_desc(xs + kk * 32),
+                                     tc::sw128_desc(bs + kk * 32), id, kk > 0);
+                    tc::mma_commit(&sm.acc_full[a]);
+                }
+                LSH_PHASE(0, 5, u, 1);
             }
             if (*reinterpret_cast<volatile int *>(&ring.abort)) tc::mma_drain(&ring.drain, status);
         }
     } else if (warp < kSoftmaxWarps) {
-        // group g takes tiles t = g, g + 2, ...; warp q of it reads TMEM lanes 32 q..
-        const int g = warp >> 2, q = warp & 3;
+        // group eg takes items it = eg, eg + 2, ...; warp q of it reads TMEM lanes 32 q..
+        const int eg = warp >> 2, q = warp & 3;
         const int row = q * 32 + lane;
-        for (int t = g; t < n_mt; t += 2) {
-            const int a = t % kAccBufs, b = t % kHashTiles;
-            if (!tc::mbar_wait(&sm.acc_full[a], (uint32_t)(t / kAccBufs) & 1u, &ring.abort, status)) break;
-            if (q == 0 && lane == 0) LSH_PHASE(0, 6, t, 0);
+        for (int it = eg; it < n_items; it += 2) {
+            const int u = it / n_rg, g = it % n_rg, a = it % kAccBufs, b = u % n_buf;
+            const int t = r + u * R, pos = t * 128 + row;
+            const bool valid = pos < L;
+            if (!tc::mbar_wait(&sm.acc_full[a], (uint32_t)(it / kAccBufs) & 1u, &ring.abort, status)) break;
+            if (q == 0 && lane == 0) LSH_PHASE(0, 6, it, 0);
             tc::tc_fence_after();
-            const uint32_t tacc = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(a * 64);
-            int bi;
-            if (hp == 32) {
-                float pv[32];
-                tc::tmem_ld16(tacc, pv);
-                tc::tmem_ld16(tacc + 16, pv + 16);
-                tc::tmem_ld_wait();
-                release_acc(sm.acc_empty[a], lane);
-                bi = first_max_bucket<32>(pv, half);
-            } else {
-                float pv[64];
+            const uint32_t tacc = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(a * kAccCols);
+            const int nr = min(rg, R - g * rg);
+            for (int j = 0; j < nr; ++j) {
+                const int rr = g * rg + j;
+                int bi;
+                if (hp == 32) {
+                    float pv[32];
+                    tc::tmem_ld16(tacc + (uint32_t)(j * 32), pv);
+                    tc::tmem_ld16(tacc + (uint32_t)(j * 32 + 16), pv + 16);
+                    tc::tmem_ld_wait();
+                    bi = first_max_bucket<32>(pv, half);
+                } else {
+                    float pv[64];
 #pragma unroll
-                for (int c = 0; c < 4; ++c) tc::tmem_ld16(tacc + (uint32_t)(c * 16), pv + c * 16);
-                tc::tmem_ld_wait();
-                release_acc(sm.acc_empty[a], lane);
-                bi = first_max_bucket<64>(pv, half);
-            }
-            // 1/|x| of the row, sum of squares in element order (as the norm pass)
-            const uint8_t *A = hash_tile(sm, b);
-            float ssq = 0.f;
-#pragma unroll
-            for (int ch = 0; ch < 8; ++ch) {
-                const uint4 u = *reinterpret_cast<const uint4 *>(A + row * 128 + ((ch ^ (row & 7)) << 4));
-                const uint32_t wd[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float lo = __uint_as_float(wd[e] << 16), hi = __uint_as_float(wd[e] & 0xFFFF0000u);
-                    ssq = fmaf(lo, lo, ssq);
-                    ssq = fmaf(hi, hi, ssq);
+                    for (int c = 0; c < 4; ++c) tc::tmem_ld16(tacc + (uint32_t)(j * 64 + c * 16), pv + c * 16);
+                    tc::tmem_ld_wait();
+                    bi = first_max_bucket<64>(pv, half);
                 }
+                // the warp's 32 consecutive positions form one sort group of round rr:
+                // each position's rank among the equal ids before it, and the group's
+                // count per id, written into round rr's CTA
+                const uint32_t peers = peers_of(valid ? (uint32_t)bi : (1u << nbits), nbits);
+                const uint32_t before = peers & ((1u << lane) - 1u);
+                if (valid) {
+                    *cluster.map_shared_rank(&sm.bkt[pos], rr) = (uint8_t)bi;
+                    *cluster.map_shared_rank(rank + pos, rr) = (uint8_t)__popc(before);
+                    if (before == 0) *cluster.map_shared_rank(cnt + bi * n_groups + (pos >> 5), rr) = (uint8_t)__popc(peers);
+                }
+            }
+            release_acc(sm.acc_empty[a], lane);
+            if (g == 0) {
+                // 1/|x| of the row, sum of squares in element order (as the norm pass)
+                const uint8_t *A = hash_tile(sm, b);
+                float ssq = 0.f;
+#pragma unroll
+                for (int ch = 0; ch < 8; ++ch) {
+                    const uint4 w4 = *reinterpret_cast<const uint4 *>(A + row * 128 + ((ch ^ (row & 7)) << 4));
+                    const uint32_t wd[4] = {w4.x, w4.y, w4.z, w4.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float lo = __uint_as_float(wd[e] << 16), hi = __uint_as_float(wd[e] & 0xFFFF0000u);
+                        ssq = fmaf(lo, lo, ssq);
+                        ssq = fmaf(hi, hi, ssq);
+                    }
+                }
+                if (valid) xinv[bh * L + pos] = ssq > 0.f ? 1.0f / sqrtf(ssq) : 0.f;
             }
             __syncwarp();
             if (lane == 0) tc::mbar_arrive(&sm.a_empty[b]);
-            const int pos = t * 128 + row;
-            // the warp's 32 consecutive positions form one sort group: each position's
-            // rank among the equal buckets before it, and the group's count per bucket
-            const bool valid = pos < L;
-            const uint32_t peers = peers_of(valid ? (uint32_t)bi : (1u << nbits), nbits);
-            const uint32_t before = peers & ((1u << lane) - 1u);
-            if (valid) {
-                sm.bkt[pos] = (uint8_t)bi;
-                xinv[bh * L + pos] = ssq > 0.f ? 1.0f / sqrtf(ssq) : 0.f;   // both rounds write the same bits
-                rank[pos] = (uint8_t)__popc(before);
-                if (before == 0) cnt[bi * n_groups + (pos >> 5)] = (uint8_t)__popc(peers);
-            }
-            if (q == 0 && lane == 0) LSH_PHASE(0, 6, t, 1);
+            if (q == 0 && lane == 0) LSH_PHASE(0, 6, it, 1);
         }
     }
     tc::fence_async_smem();
     tc::tc_fence_before();
-    __syncthreads();
+    cluster_sync_all();                 // every round's ids, ranks and counts and every norm are written
     tc::tc_fence_after();
-    const bool ok = *reinterpret_cast<volatile int *>(&ring.abort) == 0;   // the same for every thread
+    bool ok = true;                     // the same for every thread of the cluster
+    for (int c = 0; c < R; ++c) ok = ok && *cluster.map_shared_rank(&ring.abort, c) == 0;
     if (threadIdx.x == 0) LSH_PHASE(0, 7, 0, 1);
+    LSH_CTA_MARK(1);
 
     // ================= sort
     if (ok) {
@@ -358,6 +415,7 @@ fused_fwd_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __nv_bfloat1
             __syncthreads();
         }
         if (threadIdx.x == 0) LSH_PHASE(0, 7, 0, 2);
+        LSH_CTA_MARK(2);
         int32_t *pg = perm_out + seg * L;
         uint16_t *bg = bkt_out + seg * L;
         for (int e = threadIdx.x; e < L; e += kThreads) {
@@ -378,10 +436,12 @@ fused_fwd_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __nv_bfloat1
     tc::tc_fence_before();
     __syncthreads();
     if (threadIdx.x == 0) LSH_PHASE(0, 7, 0, 3);
+    LSH_CTA_MARK(3);
 
     // ================= merge: every round's o_r and lse_r of this head are written
     cluster_sync_all();
     if (threadIdx.x == 0) LSH_PHASE(0, 7, 0, 4);
+    LSH_CTA_MARK(4);
     if (ok && *reinterpret_cast<volatile int *>(&ring.abort) == 0) {
         const int rows = (L + R - 1) / R, i0 = r * rows, i1 = min(L, i0 + rows);
         if (R <= 4)
@@ -390,6 +450,7 @@ fused_fwd_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __nv_bfloat1
             merge_rows<8, 2>(o_r, lse, out, bh, L, R, i0, i1);
     }
     if (threadIdx.x == 0) LSH_PHASE(0, 7, 0, 5);
+    LSH_CTA_MARK(5);
     if (warp == 0) {
         tc::tc_fence_after();
         tc::tmem_dealloc(tmem, kTmemCols);
