@@ -112,7 +112,7 @@ __device__ __forceinline__ uint8_t *hash_tile(FusedSmem &sm, int b)
 // padding): the first maximum of [v ; -v].  Pass 1 takes the largest and
 // smallest value (3-input max/min, four independent chains); the larger of max
 // and -min picks the side (+ wins an exact tie: its indices come first); pass 2
-// finds the lowest column holding that extreme.  A padding column (exactly 0)
+// finds the lowest column holding that extreme.  Called by whole warps.  A padding column (exactly 0)
 // never decides: max(v_j, -v_j) >= 0 for every real column, and real columns
 // come first.  This is the hash kernel's rule, so both give the same ids.
 template <int NH>
@@ -136,15 +136,44 @@ __device__ __forceinline__ int first_max_bucket(const float *v, int half)
     const float mn = fminf(fminf(mnq[0], mnq[1]), fminf(mnq[2], mnq[3]));
     const bool pos = mx >= -mn;
     const float target = pos ? mx : mn;
-    int jq[4];
+    // pass 2 on the FMA pipe (pass 1 runs on the ALU pipe): U = |extreme| bounds
+    // every |v_j|; with B = 2^(24 - e(U)), (U - side v_j) B is exactly 0 where v_j
+    // is the extreme and at least 1 elsewhere, so a saturating FMA gives an exact
+    // 0/1 flag; sixteen flags are summed as the bits of an integer held in the
+    // mantissa of 2^23 + sum, and the first clear bit is the column.  Extremes
+    // whose B would not be finite take the compare-and-select form.
+    const float U = pos ? mx : -mn;
+    const int be = (__float_as_int(U) >> 23) & 0xFF;
+    int js;
+    if (__any_sync(0xffffffffu, U != 0.f && be < 24)) {
+        int jq[4];
 #pragma unroll
-    for (int qq = 0; qq < 4; ++qq) {
-        int jj = NH;
+        for (int qq = 0; qq < 4; ++qq) {
+            int jj = NH;
 #pragma unroll
-        for (int j = qq * Q + Q - 1; j >= qq * Q; --j) jj = (v[j] == target) ? j : jj;
-        jq[qq] = jj;
+            for (int j = qq * Q + Q - 1; j >= qq * Q; --j) jj = (v[j] == target) ? j : jj;
+            jq[qq] = jj;
+        }
+        js = min(min(jq[0], jq[1]), min(jq[2], jq[3]));
+    } else {
+        const float B = __int_as_float(min(278 - be, 253) << 23);
+        const float nsB = pos ? -B : B;
+        const float UB = U * B;
+        constexpr int NC = NH / 16;
+        float acc[NC];
+#pragma unroll
+        for (int c = 0; c < NC; ++c) acc[c] = 8388608.f;
+#pragma unroll
+        for (int k = 0; k < 16; ++k)
+#pragma unroll
+            for (int c = 0; c < NC; ++c) acc[c] = fmaf(tc::fma_sat(v[c * 16 + k], nsB, UB), (float)(1 << k), acc[c]);
+        js = NH;
+#pragma unroll
+        for (int c = NC - 1; c >= 0; --c) {
+            const uint32_t eq = ~__float_as_uint(acc[c]) & 0xFFFFu;
+            js = eq ? c * 16 + __ffs((int)eq) - 1 : js;
+        }
     }
-    const int js = min(min(jq[0], jq[1]), min(jq[2], jq[3]));
     return (pos ? 0 : half) + js;
 }
 
@@ -164,7 +193,7 @@ __device__ __forceinline__ void cluster_sync_all()
 
 // Rows [i0, i1) of head bh merged over its R <= RMAX rounds, eight threads per
 // row; every thread loads K rows' round data before merging any, so that K
-// L2 round trips overlap.
+// memory round trips overlap.
 template <int RMAX, int K>
 __device__ __forceinline__ void merge_rows(const __nv_bfloat16 *__restrict__ o_r, const float *__restrict__ lse,
                                            __nv_bfloat16 *__restrict__ out, long long bh, int L, int R, int i0, int i1)
@@ -444,7 +473,9 @@ fused_fwd_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __nv_bfloat1
     LSH_CTA_MARK(4);
     if (ok && *reinterpret_cast<volatile int *>(&ring.abort) == 0) {
         const int rows = (L + R - 1) / R, i0 = r * rows, i1 = min(L, i0 + rows);
-        if (R <= 4)
+        if (R <= 2)
+            merge_rows<2, 8>(o_r, lse, out, bh, L, R, i0, i1);
+        else if (R <= 4)
             merge_rows<4, 4>(o_r, lse, out, bh, L, R, i0, i1);
         else
             merge_rows<8, 2>(o_r, lse, out, bh, L, R, i0, i1);
