@@ -94,6 +94,8 @@ NCU_TRAFFIC = {
                         "sha256": "b54830b6cfe4d2feaf659e8a40f03fccbf6d7ef640792c7e33f322330c258560"},
     ("long_64k", "combine"): {"bytes": 324_419_328, "files": ('simt.cu', 'common.cuh'),
                            "sha256": "cb3ac11b02abc61346fa8ff9109a7092f182a3472b5146ae262b68789f870c09"},
+    ("bf16_causal_4k", "fused_fwd"): {"bytes": 170_126_848, "files": ('fused_fwd_tc.cu', 'attn_fwd_roles.cuh', 'combine.cuh', 'seg_sort.cuh', 'tc_common.cuh', 'common.cuh'),
+                                   "sha256": "dccc8dc89fa3f671b74b1c90de306c3b919b36a962da8d032c633a771dcdbb43"},
     ("half_million", "hash"): {"bytes": 141_445_376, "files": ('hash_tc.cu', 'tc_common.cuh', 'common.cuh'),
                             "sha256": "b54830b6cfe4d2feaf659e8a40f03fccbf6d7ef640792c7e33f322330c258560"},
 }
