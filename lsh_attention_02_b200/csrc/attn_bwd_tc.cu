@@ -513,7 +513,11 @@ attn_bwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
             constexpr uint32_t id_s = tc::idesc_bf16(128, kQ, 0, 0);
             constexpr uint32_t id_kv = tc::idesc_bf16(128, kDim, 0, 1);   // A K-major, B MN-major
             constexpr uint32_t id_q = tc::idesc_bf16(128, kDim, 1, 1);    // A MN-major, B MN-major
-            const uint32_t e0 = tc::smem_u32(sm.ET[0]), e1 = tc::smem_u32(sm.ET[1]), e2 = tc::smem_u32(sm.ET[2]);
+            const uint64_t de0 = tc::sw128_desc(tc::smem_u32(sm.ET[0])), de1 = tc::sw128_desc(tc::smem_u32(sm.ET[1])),
+                           de2 = tc::sw128_desc(tc::smem_u32(sm.ET[2]));
+            // E = (E^T)^T read MN-major: 64-query blocks 16 KB apart (leading byte offset)
+            const uint64_t de0l = tc::sw128_desc(tc::smem_u32(sm.ET[0]), kK * 128),
+                           de1l = tc::sw128_desc(tc::smem_u32(sm.ET[1]), kK * 128);
             TileIter ti = tile_begin(blockIdx.x, R, n_runs);
             for (int it = 0; ti.unit < n_units; ++it, tile_advance(ti, R, n_k, n_runs)) {
                 const int s = it % kStages;
@@ -525,11 +529,12 @@ attn_bwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
                 LSH_PHASE(1, 1, it, 2);
                 tc::tc_fence_after();
                 const Stage &st = sm.st[s];
-                const uint32_t xs = tc::smem_u32(st.X), vs = tc::smem_u32(st.V), gs = tc::smem_u32(st.G);
+                const uint64_t dxs = tc::sw128_desc(tc::smem_u32(st.X)), dvs = tc::sw128_desc(tc::smem_u32(st.V)),
+                               dgs = tc::sw128_desc(tc::smem_u32(st.G));
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk) {
-                    tc::mma_bf16(tmem + cS, tc::sw128_desc(xs + kk * 32), tc::sw128_desc(xs + kk * 32), id_s, kk > 0);
-                    tc::mma_bf16(tmem + cD, tc::sw128_desc(vs + kk * 32), tc::sw128_desc(gs + kk * 32), id_s, kk > 0);
+                    tc::mma_bf16(tmem + cS, tc::desc_add(dxs, kk * 32), tc::desc_add(dxs, kk * 32), id_s, kk > 0);
+                    tc::mma_bf16(tmem + cD, tc::desc_add(dvs, kk * 32), tc::desc_add(dgs, kk * 32), id_s, kk > 0);
                 }
                 tc::mma_commit(&sm.bar_s);
 #ifdef LSH_PHASE_TRACE
@@ -541,9 +546,9 @@ attn_bwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
                 tc::tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < 12; ++kk) {
-                    const uint32_t ea = (kk < 4 ? e0 : kk < 8 ? e1 : e2) + (kk & 3) * 32;
-                    tc::mma_bf16_ts(tmem + cDV, tmem + cPT + kk * 8, tc::sw128_desc(gs + kk * 2048), id_kv, kk > 0);
-                    tc::mma_bf16(tmem + cDX, tc::sw128_desc(ea), tc::sw128_desc(xs + kk * 2048), id_kv, kk > 0);
+                    const uint64_t dea = tc::desc_add(kk < 4 ? de0 : kk < 8 ? de1 : de2, (kk & 3) * 32);
+                    tc::mma_bf16_ts(tmem + cDV, tmem + cPT + kk * 8, tc::desc_add(dgs, kk * 2048), id_kv, kk > 0);
+                    tc::mma_bf16(tmem + cDX, dea, tc::desc_add(dxs, kk * 2048), id_kv, kk > 0);
                 }
                 // E = (E^T)^T read MN-major: 64-query blocks 16 KB apart (leading byte offset).
                 // The second half (queries 64..191) is read only for chunk 2k+2 (rows
@@ -551,11 +556,11 @@ attn_bwd_tc_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
                 // keys 64..127 (rows 64..127 of that product are never read).
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
-                    tc::mma_bf16(tmem + cDX, tc::sw128_desc(e0 + kk * 2048, kK * 128), tc::sw128_desc(xs + kk * 2048),
+                    tc::mma_bf16(tmem + cDX, tc::desc_add(de0l, kk * 2048), tc::desc_add(dxs, kk * 2048),
                                  id_q, true);
 #pragma unroll
                 for (int kk = 4; kk < 8; ++kk)
-                    tc::mma_bf16(tmem + cQb, tc::sw128_desc(e1 + kk * 2048, kK * 128), tc::sw128_desc(xs + kk * 2048),
+                    tc::mma_bf16(tmem + cQb, tc::desc_add(de1l, kk * 2048), tc::desc_add(dxs, kk * 2048),
                                  id_q, kk > 4);
                 tc::mma_commit(&sm.bar_o);
                 LSH_PHASE(1, 1, it, 4);

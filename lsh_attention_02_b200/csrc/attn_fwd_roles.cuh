@@ -202,8 +202,7 @@ __device__ __forceinline__ float softmax_sweep(const Stage &st, uint32_t tl, int
             for (int c = 0; c < 4; ++c) tc::tmem_st8(tl + (uint32_t)(BASE / 2 + h * 32 + c * 8), z);
         } else {
             float v[64];
-    #pragma unroll
-            for (int c = 0; c < 4; ++c) tc::tmem_ld16(tl + (uint32_t)(BASE + h * 64 + c * 16), v + c * 16);
+            tc::tmem_ld64(tl + (uint32_t)(BASE + h * 64), v);
             tc::tmem_ld_wait();
     #pragma unroll
             for (int c = 0; c < 4; ++c) {
@@ -436,11 +435,11 @@ __device__ __forceinline__ void mma_role(Ring<NST> &sm, int n_mine, uint32_t tme
                     (it < 2 || tc::mbar_test_wait(&sm.o_free[g], (uint32_t)((it >> 1) - 1) & 1u))) {
                     LSH_PHASE(0, 1, it, 1);
                     tc::tc_fence_after();
-                    const uint32_t xs = tc::smem_u32(sm.st[s].X);
+                    const uint64_t dx = tc::sw128_desc(tc::smem_u32(sm.st[s].X));
                     const uint32_t d = tmem + (uint32_t)g * kGroupCols;
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
-                        tc::mma_bf16(d, tc::sw128_desc(xs + 64 * 128 + kk * 32), tc::sw128_desc(xs + kk * 32),
+                        tc::mma_bf16(d, tc::desc_add(dx, 64 * 128 + kk * 32), tc::desc_add(dx, kk * 32),
                                      id_s, kk > 0);
                     tc::mma_commit(&sm.s_full[g]);
                     LSH_PHASE(0, 1, it, 2);
@@ -453,11 +452,11 @@ __device__ __forceinline__ void mma_role(Ring<NST> &sm, int n_mine, uint32_t tme
                 const int it = next_oh, s = it % NST, g = it & 1;
                 if (tc::mbar_test_wait(&sm.p_half[g], (uint32_t)(it >> 1) & 1u)) {
                     tc::tc_fence_after();
-                    const uint32_t vs = tc::smem_u32(sm.st[s].V);
+                    const uint64_t dv = tc::sw128_desc(tc::smem_u32(sm.st[s].V));
                     const uint32_t base = tmem + (uint32_t)g * kGroupCols;
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
-                        tc::mma_bf16_ts(base + kOCol, base + kk * 8, tc::sw128_desc(vs + kk * 16 * 128), id_o,
+                        tc::mma_bf16_ts(base + kOCol, base + kk * 8, tc::desc_add(dv, kk * 16 * 128), id_o,
                                         kk > 0);
                     ++next_oh;
                     progressed = true;
@@ -468,11 +467,11 @@ __device__ __forceinline__ void mma_role(Ring<NST> &sm, int n_mine, uint32_t tme
                 if (tc::mbar_test_wait(&sm.p_full[g], (uint32_t)(it >> 1) & 1u)) {
                     LSH_PHASE(0, 1, it, 3);
                     tc::tc_fence_after();
-                    const uint32_t vs = tc::smem_u32(sm.st[s].V);
+                    const uint64_t dv = tc::sw128_desc(tc::smem_u32(sm.st[s].V));
                     const uint32_t base = tmem + (uint32_t)g * kGroupCols;
 #pragma unroll
                     for (int kk = 4; kk < 12; ++kk)
-                        tc::mma_bf16_ts(base + kOCol, base + kk * 8, tc::sw128_desc(vs + kk * 16 * 128), id_o,
+                        tc::mma_bf16_ts(base + kOCol, base + kk * 8, tc::desc_add(dv, kk * 16 * 128), id_o,
                                         true);
                     tc::mma_commit(&sm.o_full[g]);
                     LSH_PHASE(0, 1, it, 4);

@@ -309,7 +309,7 @@ fused_fwd_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __nv_bfloat1
                 const int b = u % n_buf;
                 if (!tc::mbar_wait(&sm.a_full[b], (uint32_t)(u / n_buf) & 1u, &ring.abort, status)) break;
                 LSH_PHASE(0, 5, u, 0);
-                const uint32_t xs = tc::smem_u32(hash_tile(sm, b));
+                const uint64_t da = tc::sw128_desc(tc::smem_u32(hash_tile(sm, b)));
                 for (int g = 0; g < n_rg; ++g) {
                     const int it = u * n_rg + g, a = it % kAccBufs;
                     if (it >= kAccBufs &&
@@ -320,11 +320,11 @@ fused_fwd_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __nv_bfloat1
                     tc::tc_fence_after();
                     const int nr = min(rg, R - g * rg);
                     const uint32_t id = tc::idesc_bf16(128, nr * hp, 0, 0);
-                    const uint32_t bs = rs + (uint32_t)(g * rg * hp * 128);
+                    const uint64_t db = tc::sw128_desc(rs + (uint32_t)(g * rg * hp * 128));
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
-                        tc::mma_bf16(tmem + (uint32_t)(a * kAccCols), tc::sw128_desc(xs + kk * 32),
-                                     tc::sw128_desc(bs + kk * 32), id, kk > 0);
+                        tc::mma_bf16(tmem + (uint32_t)(a * kAccCols), tc::desc_add(da, kk * 32),
+                                     tc::desc_add(db, kk * 32), id, kk > 0);
                     tc::mma_commit(&sm.acc_full[a]);
                 }
                 LSH_PHASE(0, 5, u, 1);
@@ -349,14 +349,12 @@ fused_fwd_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __nv_bfloat1
                 int bi;
                 if (hp == 32) {
                     float pv[32];
-                    tc::tmem_ld16(tacc + (uint32_t)(j * 32), pv);
-                    tc::tmem_ld16(tacc + (uint32_t)(j * 32 + 16), pv + 16);
+                    tc::tmem_ld32(tacc + (uint32_t)(j * 32), pv);
                     tc::tmem_ld_wait();
                     bi = first_max_bucket<32>(pv, half);
                 } else {
                     float pv[64];
-#pragma unroll
-                    for (int c = 0; c < 4; ++c) tc::tmem_ld16(tacc + (uint32_t)(j * 64 + c * 16), pv + c * 16);
+                    tc::tmem_ld64(tacc + (uint32_t)(j * 64), pv);
                     tc::tmem_ld_wait();
                     bi = first_max_bucket<64>(pv, half);
                 }

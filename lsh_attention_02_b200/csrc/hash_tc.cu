@@ -172,7 +172,7 @@ hash_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __nv_bfloat16 *__
             for (long long blk = blockIdx.x; ok && blk < n_blocks; blk += gridDim.x, ++bi) {
                 const int xa = bi & 1;
                 if (!tc::mbar_wait(&sm.a_full[xa], (uint32_t)(bi >> 1) & 1u, &sm.abort, status)) break;
-                const uint32_t a0 = tc::smem_u32(sm.A[xa]);
+                const uint64_t da = tc::sw128_desc(tc::smem_u32(sm.A[xa]));
                 for (int i = 0; i < items; ++i, ++it) {
                     const int s = it % kStages;
                     const uint32_t ph = (uint32_t)(it / kStages) & 1u;
@@ -184,13 +184,13 @@ hash_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __nv_bfloat16 *__
                     if (it >= 2 && !tc::mbar_wait(&sm.acc_empty[ab], aph ^ 1u, &sm.abort, status)) { ok = false; break; }
                     LSH_PHASE(0, 2, it, 2);
                     tc::tc_fence_after();
-                    const uint32_t b0 = tc::smem_u32(sm.B[s]);
+                    const uint64_t db = tc::sw128_desc(tc::smem_u32(sm.B[s]));
 #pragma unroll
                     for (int mt = 0; mt < 2; ++mt) {
                         const uint32_t d = tmem + (uint32_t)(ab * 2 * kMaxNT + mt * kMaxNT);
 #pragma unroll
                         for (int k = 0; k < 4; ++k)
-                            tc::mma_bf16(d, tc::sw128_desc(a0 + mt * 128 * 128 + k * 32), tc::sw128_desc(b0 + k * 32),
+                            tc::mma_bf16(d, tc::desc_add(da, mt * 128 * 128 + k * 32), tc::desc_add(db, k * 32),
                                          idesc, k > 0);
                         tc::mma_commit(&sm.acc_full[ab][mt]);
                     }
@@ -256,9 +256,15 @@ hash_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __nv_bfloat16 *__
                 if (threadIdx.x == 0) LSH_PHASE(0, 0, it, 1);
                 tc::tc_fence_after();
                 float v[NH];
+                if constexpr (NH == 64) {
+                    tc::tmem_ld64(lane_base + (uint32_t)(ab * 2 * kMaxNT), v);
+                } else if constexpr (NH == 32) {
+                    tc::tmem_ld32(lane_base + (uint32_t)(ab * 2 * kMaxNT), v);
+                } else {
 #pragma unroll
-                for (int c = 0; c < NH / 16; ++c)
-                    tc::tmem_ld16(lane_base + (uint32_t)(ab * 2 * kMaxNT + c * 16), v + c * 16);
+                    for (int c = 0; c < NH / 16; ++c)
+                        tc::tmem_ld16(lane_base + (uint32_t)(ab * 2 * kMaxNT + c * 16), v + c * 16);
+                }
                 tc::tmem_ld_wait();
                 tc::tc_fence_before();
                 __syncwarp();
