@@ -86,18 +86,16 @@ def algorithmic(w: synth.Workload) -> dict:
 # profiles/).  A record counts only while the kernel's sources hash to the
 # value taken with it; after any change the traffic is reported as null.
 NCU_TRAFFIC = {
-    ("long_64k", "attn_bwd"): {"bytes": 753_787_904, "files": ('attn_bwd_tc.cu', 'tc_common.cuh', 'common.cuh'),
-                            "sha256": "8c1115c0961760452ef90c95d78b632cf51f891a7212c09e088fca417544cbc5"},
-    ("long_64k", "attn_fwd"): {"bytes": 368_326_912, "files": ('attn_fwd_tc.cu', 'tc_common.cuh', 'common.cuh'),
-                            "sha256": "e2f365cb31fb2a739c6346617af9f62f5f9310a341613c27166f9f5e072756e0"},
-    ("long_64k", "hash"): {"bytes": 67_636_480, "files": ('hash_tc.cu', 'tc_common.cuh', 'common.cuh'),
-                        "sha256": "b54830b6cfe4d2feaf659e8a40f03fccbf6d7ef640792c7e33f322330c258560"},
-    ("long_64k", "combine"): {"bytes": 324_419_328, "files": ('simt.cu', 'common.cuh'),
-                           "sha256": "cb3ac11b02abc61346fa8ff9109a7092f182a3472b5146ae262b68789f870c09"},
-    ("bf16_causal_4k", "fused_fwd"): {"bytes": 170_126_848, "files": ('fused_fwd_tc.cu', 'attn_fwd_roles.cuh', 'combine.cuh', 'seg_sort.cuh', 'tc_common.cuh', 'common.cuh'),
-                                   "sha256": "dccc8dc89fa3f671b74b1c90de306c3b919b36a962da8d032c633a771dcdbb43"},
-    ("half_million", "hash"): {"bytes": 141_445_376, "files": ('hash_tc.cu', 'tc_common.cuh', 'common.cuh'),
-                            "sha256": "b54830b6cfe4d2feaf659e8a40f03fccbf6d7ef640792c7e33f322330c258560"},
+    ("long_64k", "attn_bwd"): {"bytes": 763_595_776, "files": ('attn_bwd_tc.cu', 'tc_common.cuh', 'common.cuh'),
+                               "sha256": "bd2fe6864fa283d2da546f9f29634c18911c48ef364b9d4d20bca9ddd5952aff"},
+    ("long_64k", "attn_fwd"): {"bytes": 368_641_024, "files": ('attn_fwd_tc.cu', 'attn_fwd_roles.cuh', 'tc_common.cuh', 'common.cuh'),
+                               "sha256": "3574c081cae3bf556dea136f53c4727fdeff0fedd2183e3b459c46e680033229"},
+    ("long_64k", "hash"): {"bytes": 67_439_872, "files": ('hash_tc.cu', 'tc_common.cuh', 'common.cuh'),
+                           "sha256": "2e61e9680746c0fc3fee9fc9a7445655758a98a901f4f98dee20d76ece2e532f"},
+    ("long_64k", "combine"): {"bytes": 323_120_896, "files": ('simt.cu', 'combine.cuh', 'common.cuh'),
+                              "sha256": "97ef77b8f0ae6ca8adf9980ab97b87be2355dc3af93242b3c9d737142db2030f"},
+    ("half_million", "hash"): {"bytes": 141_867_008, "files": ('hash_tc.cu', 'tc_common.cuh', 'common.cuh'),
+                               "sha256": "2e61e9680746c0fc3fee9fc9a7445655758a98a901f4f98dee20d76ece2e532f"},
 }
 
 
