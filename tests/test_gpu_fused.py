@@ -99,3 +99,25 @@ def test_fused_forward_full_workload_equals_staged():
     assert torch.equal(fused.perm, staged.perm)
     assert torch.equal(fused.lse, staged.lse)
     assert torch.equal(fused.out, staged.out)
+
+
+def test_fused_forward_without_permutation_output_then_recomputing_backward():
+    """The single kernel writes the permutation into the workspace when the
+    caller passes none; the outputs equal those of the call that asks for it,
+    and a backward that recomputes the permutation from R gives the gradients
+    of the backward that is handed it (same buckets, so the same bits up to
+    the fp32 reductions' order)."""
+    w = small(B=2, H=2, L=2048, n_buckets=64, n_hashes=2, causal=True, backward=True)
+    inp = synth.make_inputs(w)
+    lsh.fused_forward(True)
+    run = Run(inp, w.n_buckets, w.chunk, w.causal, w.dtype)
+    assert lsh.fused_forward_fits(run.desc)
+    out2, lse2 = torch.empty_like(run.out), torch.empty_like(run.lse)
+    lsh.lsh_attn_fwd(run.desc, run.x, run.v, run.R, out2, lse2, None)
+    torch.cuda.synchronize()
+    assert torch.equal(out2, run.out) and torch.equal(lse2, run.lse)
+    dx2, dv2 = torch.empty_like(run.x), torch.empty_like(run.v)
+    lsh.lsh_attn_bwd(run.desc, run.x, run.v, run.R, run.out, run.lse, None, run.dy, dx2, dv2)
+    torch.cuda.synchronize()
+    assert_close(to_host(dx2), to_host(run.dx), "bf16", "dqk, permutation recomputed")
+    assert_close(to_host(dv2), to_host(run.dv), "bf16", "dv, permutation recomputed")
