@@ -92,8 +92,6 @@ NCU_TRAFFIC = {
                                "sha256": "3574c081cae3bf556dea136f53c4727fdeff0fedd2183e3b459c46e680033229"},
     ("long_64k", "hash"): {"bytes": 67_439_872, "files": ('hash_tc.cu', 'tc_common.cuh', 'common.cuh'),
                            "sha256": "2e61e9680746c0fc3fee9fc9a7445655758a98a901f4f98dee20d76ece2e532f"},
-    ("long_64k", "combine"): {"bytes": 323_120_896, "files": ('simt.cu', 'combine.cuh', 'common.cuh'),
-                              "sha256": "97ef77b8f0ae6ca8adf9980ab97b87be2355dc3af93242b3c9d737142db2030f"},
     ("half_million", "hash"): {"bytes": 141_867_008, "files": ('hash_tc.cu', 'tc_common.cuh', 'common.cuh'),
                                "sha256": "2e61e9680746c0fc3fee9fc9a7445655758a98a901f4f98dee20d76ece2e532f"},
 }

@@ -664,30 +664,39 @@ cudaError_t launch_attn_bwd_simt(const Problem &p, const void *x, const void *v,
 }
 
 // ------------------------------------------------------------------ backward epilogue
+// Eight elements of each accumulator per thread: two 16-byte loads per array
+// and one 16-byte store of eight bf16 (or two of fp32) per output.
 template <typename T>
 __global__ void bwd_finalize_kernel(const float *__restrict__ dx_acc, const float *__restrict__ dv_acc,
-                                    T *__restrict__ dqk, T *__restrict__ dv, long long n4)
+                                    T *__restrict__ dqk, T *__restrict__ dv, long long n8)
 {
     long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-    if (i >= n4) return;
-    float4 a = reinterpret_cast<const float4 *>(dx_acc)[i];
-    float4 b = reinterpret_cast<const float4 *>(dv_acc)[i];
-    T *o1 = dqk + 4 * i;
-    T *o2 = dv + 4 * i;
-    o1[0] = from_f<T>(a.x); o1[1] = from_f<T>(a.y); o1[2] = from_f<T>(a.z); o1[3] = from_f<T>(a.w);
-    o2[0] = from_f<T>(b.x); o2[1] = from_f<T>(b.y); o2[2] = from_f<T>(b.z); o2[3] = from_f<T>(b.w);
+    if (i >= n8) return;
+    const float4 a0 = reinterpret_cast<const float4 *>(dx_acc)[2 * i], a1 = reinterpret_cast<const float4 *>(dx_acc)[2 * i + 1];
+    const float4 b0 = reinterpret_cast<const float4 *>(dv_acc)[2 * i], b1 = reinterpret_cast<const float4 *>(dv_acc)[2 * i + 1];
+    if constexpr (sizeof(T) == 2) {
+        reinterpret_cast<uint4 *>(dqk)[i] = make_uint4(pack_bf16x2(a0.x, a0.y), pack_bf16x2(a0.z, a0.w),
+                                                       pack_bf16x2(a1.x, a1.y), pack_bf16x2(a1.z, a1.w));
+        reinterpret_cast<uint4 *>(dv)[i] = make_uint4(pack_bf16x2(b0.x, b0.y), pack_bf16x2(b0.z, b0.w),
+                                                      pack_bf16x2(b1.x, b1.y), pack_bf16x2(b1.z, b1.w));
+    } else {
+        reinterpret_cast<float4 *>(dqk)[2 * i] = a0;
+        reinterpret_cast<float4 *>(dqk)[2 * i + 1] = a1;
+        reinterpret_cast<float4 *>(dv)[2 * i] = b0;
+        reinterpret_cast<float4 *>(dv)[2 * i + 1] = b1;
+    }
 }
 
 cudaError_t launch_bwd_finalize(const Problem &p, const float *dx_acc, const float *dv_acc, void *dqk, void *dv,
                                 cudaStream_t st)
 {
-    long long n4 = p.tokens() * kDim / 4;
-    unsigned grid = (unsigned)((n4 + 255) / 256);
+    long long n8 = p.tokens() * kDim / 8;
+    unsigned grid = (unsigned)((n8 + 255) / 256);
     if (p.dtype == LSH_F32)
-        bwd_finalize_kernel<float><<<grid, 256, 0, st>>>(dx_acc, dv_acc, (float *)dqk, (float *)dv, n4);
+        bwd_finalize_kernel<float><<<grid, 256, 0, st>>>(dx_acc, dv_acc, (float *)dqk, (float *)dv, n8);
     else
         bwd_finalize_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(dx_acc, dv_acc, (__nv_bfloat16 *)dqk,
-                                                                 (__nv_bfloat16 *)dv, n4);
+                                                                 (__nv_bfloat16 *)dv, n8);
     return cudaGetLastError();
 }
 
