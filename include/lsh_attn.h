@@ -341,14 +341,19 @@ LSH_API lsh_status lsh_attn_trace_end(float *ms, int32_t *calls, int32_t *kernel
 LSH_API lsh_status lsh_attn_trace_stages(uint32_t mask);
 
 /* Single-kernel forward of short segments (lsh_attn_fwd, the reversible block
- * and lsh_attn_step_host): enable = 1 (the default) uses it wherever it
- * applies, 0 always runs the staged kernels (hash, sort, attention, merge),
- * for comparisons.  Process-wide; takes effect for calls made after it.
- * Returns LSH_ERR_ARG for any other value. */
-LSH_API lsh_status lsh_attn_fused_forward(int32_t enable);
+ * and lsh_attn_step_host).  mode = 1 (the default): used where a segment fits
+ * and the B*H*n_hashes segments fill the GPU's waves (one CTA per segment: a
+ * wave of at least three quarters as many segments as SMs); otherwise the
+ * staged kernels, which spread every tile over all SMs, are faster.  mode = 2:
+ * used wherever a segment fits.  mode = 0: never (the staged kernels: hash,
+ * sort, attention, merge).  Both forms give the same bits.  Process-wide;
+ * takes effect for calls made after it.  Returns LSH_ERR_ARG for any other
+ * value. */
+LSH_API lsh_status lsh_attn_fused_forward(int32_t mode);
 
 /* 1 if a forward with this descriptor runs as the single kernel under the
- * current setting, 0 otherwise (also for an invalid descriptor). */
+ * current setting (on the current device), 0 otherwise (also for an invalid
+ * descriptor). */
 LSH_API int32_t lsh_attn_fused_forward_fits(const lsh_attn_desc *desc);
 
 /* Self-test of the bounded device-side waits: launches one CTA that waits on a

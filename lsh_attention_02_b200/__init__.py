@@ -291,9 +291,12 @@ def trace_stages(names=None):
     _check(load_library().lsh_attn_trace_stages(mask), "lsh_attn_trace_stages")
 
 
-def fused_forward(enable: bool = True):
-    """Single-kernel forward of short segments on (default) or off (staged kernels), process-wide."""
-    _check(load_library().lsh_attn_fused_forward(1 if enable else 0), "lsh_attn_fused_forward")
+def fused_forward(mode=1):
+    """Single-kernel forward of short segments, process-wide: 1 (or True; the
+    default) where it fits and its segments fill the GPU's waves, 2 wherever it
+    fits, 0 (or False) never."""
+    mode = int(mode)
+    _check(load_library().lsh_attn_fused_forward(mode), "lsh_attn_fused_forward")
 
 
 def fused_forward_fits(desc) -> bool:

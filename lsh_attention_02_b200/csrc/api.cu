@@ -180,10 +180,33 @@ static lsh_status run_attn_fwd(const Problem &p, const Choice &c, const void *qk
 }
 
 // The whole forward from the rotations: one kernel per head's rounds where a
-// segment fits on chip (and the single-kernel forward is enabled), otherwise
-// hash, sort, attention and merge as separate stages.
+// segment fits on chip and the setting allows it, otherwise hash, sort,
+// attention and merge as separate stages.  Setting 1 (the default) takes the
+// single kernel only where its segments fill the GPU's waves: it runs one CTA
+// per segment, so with few segments most SMs would idle while the staged
+// kernels spread every tile over all of them.  From the measured costs (4K
+// workload: 0.124 ms in one wave of 128 CTAs against 0.137 ms staged, the
+// staged time growing with the segment count) the single kernel is ahead when
+// a wave holds at least about three quarters as many segments as there are SMs.
+// Setting 2 takes it wherever it fits (tests), 0 never.
 static int g_fused_forward = 1;
-static bool use_fused(const Problem &p, const Choice &c) { return g_fused_forward && c.tc_attn && fused_fwd_fits(p); }
+static int sm_count()
+{
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) !=
+                                                   cudaSuccess || sms <= 0) {
+        cudaGetLastError();
+        sms = 148;                          // no device: the B200's count
+    }
+    return sms;
+}
+static bool use_fused(const Problem &p, const Choice &c)
+{
+    if (g_fused_forward == 0 || !c.tc_attn || !fused_fwd_fits(p)) return false;
+    if (g_fused_forward == 2) return true;
+    const long long sms = sm_count(), S = p.S(), waves = (S + sms - 1) / sms;
+    return 4 * S >= 3 * waves * sms;
+}
 static lsh_status run_forward(const Problem &p, const Choice &c, const void *qk, const void *v, const void *R,
                               int32_t *perm, void *out, float *lse, const Workspace &w, cudaStream_t st)
 {
@@ -784,10 +807,10 @@ lsh_status lsh_attn_trace_stages(uint32_t mask)
     return LSH_OK;
 }
 
-lsh_status lsh_attn_fused_forward(int32_t enable)
+lsh_status lsh_attn_fused_forward(int32_t mode)
 {
-    if (enable != 0 && enable != 1) return LSH_ERR_ARG;
-    g_fused_forward = enable;
+    if (mode < 0 || mode > 2) return LSH_ERR_ARG;
+    g_fused_forward = mode;
     return LSH_OK;
 }
 

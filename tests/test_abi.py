@@ -175,21 +175,36 @@ def test_local_attention_argument_rules(lib):
 
 
 def test_fused_forward_applies_to_short_bf16_segments_only(lib):
-    """The single-kernel forward is chosen on the host from the descriptor alone:
-    bf16, chunk 64, L a multiple of 64 up to 4096, n_buckets <= 128,
-    n_hashes <= 8; the switch turns it off for every shape."""
+    """The single-kernel forward is chosen on the host from the descriptor alone.
+    Setting 2: wherever it fits (bf16, chunk 64, L a multiple of 64 up to 4096,
+    n_buckets <= 128, n_hashes <= 8, B*H*L >= 128).  Setting 1 (the default):
+    also only where the B*H*n_hashes segments fill the GPU's waves (at least
+    three quarters of the SMs per wave; without a device the B200's 148).
+    Setting 0: never."""
     fits = lambda **kw: lib.lsh_attn_fused_forward_fits(ctypes.byref(_desc(**kw)))
-    assert fits(L=4096, n_buckets=64, n_hashes=2, B=8, H=8, causal=1) == 1
-    assert fits(L=64) == 1 and fits(L=960, n_buckets=2) == 1 and fits(n_buckets=128, n_hashes=8) == 1
-    assert fits(L=4160) == 0                       # longer than a segment held on chip
-    assert fits(n_buckets=130) == 0                # more rotation columns than the kernel holds
-    assert fits(n_hashes=9) == 0                   # more rounds than a portable cluster has CTAs
-    assert fits(dtype=lsh.LSH_F32) == 0            # fp32 runs on the CUDA-core kernels
-    assert fits(chunk=32) == 0 and fits(B=1, H=1, L=64) == 0
-    assert lib.lsh_attn_fused_forward(2) == -1     # LSH_ERR_ARG
-    assert lib.lsh_attn_fused_forward(0) == 0
+    assert lib.lsh_attn_fused_forward(3) == -1     # LSH_ERR_ARG
     try:
-        assert fits(L=4096, n_buckets=64) == 0
+        assert lib.lsh_attn_fused_forward(2) == 0
+        assert fits(L=4096, n_buckets=64, n_hashes=2, B=8, H=8, causal=1) == 1
+        assert fits(L=64) == 1 and fits(L=960, n_buckets=2) == 1 and fits(n_buckets=128, n_hashes=8) == 1
+        assert fits(L=4160) == 0                       # longer than a segment held on chip
+        assert fits(n_buckets=130) == 0                # more rotation columns than the kernel holds
+        assert fits(n_hashes=9) == 0                   # more rounds than a portable cluster has CTAs
+        assert fits(dtype=lsh.LSH_F32) == 0            # fp32 runs on the CUDA-core kernels
+        assert fits(chunk=32) == 0 and fits(B=1, H=1, L=64) == 0
+        assert lib.lsh_attn_fused_forward(1) == 0
+        sms = 148 if not torch_cuda_available() else None
+        if sms is not None:
+            assert fits(L=4096, n_buckets=64, n_hashes=2, B=8, H=8) == 1    # 128 segments, one wave
+            assert fits(L=4096, n_buckets=64, n_hashes=2, B=1, H=2) == 0    # 4 segments: staged
+            assert fits(L=1024, n_buckets=64, n_hashes=2, B=8, H=10) == 0   # 160 segments, two thin waves
+            assert fits(L=1024, n_buckets=64, n_hashes=2, B=8, H=16) == 1   # 256 segments, two full waves
+        assert lib.lsh_attn_fused_forward(0) == 0
+        assert fits(L=4096, n_buckets=64, B=8, H=8) == 0
     finally:
         assert lib.lsh_attn_fused_forward(1) == 0
-    assert fits(L=4096, n_buckets=64) == 1
+
+
+def torch_cuda_available():
+    import torch
+    return torch.cuda.is_available()

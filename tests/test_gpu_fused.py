@@ -22,17 +22,18 @@ def small(**kw):
     return synth.WORKLOADS["bf16_causal_4k"].replace(**kw)
 
 
-def run_both(w, inp, flags=0):
-    """The forward with the single kernel, then with the staged kernels."""
-    lsh.fused_forward(True)
-    fused = Run(inp, w.n_buckets, w.chunk, w.causal, w.dtype, flags)
-    assert lsh.fused_forward_fits(fused.desc)
-    lsh.fused_forward(False)
+def run_both(w, inp, flags=0, mode=2):
+    """The forward with the single kernel (setting `mode`; 2: wherever it fits,
+    so that small shapes reach it), then with the staged kernels."""
     try:
+        lsh.fused_forward(mode)
+        fused = Run(inp, w.n_buckets, w.chunk, w.causal, w.dtype, flags)
+        assert lsh.fused_forward_fits(fused.desc)
+        lsh.fused_forward(0)
         staged = Run(inp, w.n_buckets, w.chunk, w.causal, w.dtype, flags)
         assert not lsh.fused_forward_fits(staged.desc)
     finally:
-        lsh.fused_forward(True)
+        lsh.fused_forward(1)
     return fused, staged
 
 
@@ -68,9 +69,12 @@ def test_fused_forward_then_backward_against_oracle(L, nb, nh, causal, flags):
     w = small(B=1, H=3, L=L, n_buckets=nb, n_hashes=nh, causal=causal, backward=True)
     inp = synth.make_inputs(w)
     inp["dy"] = (inp["dy"] / 4.0).astype(np.float32)           # exact: a power of two
-    lsh.fused_forward(True)
-    run = Run(inp, w.n_buckets, w.chunk, w.causal, w.dtype, flags)
-    assert lsh.fused_forward_fits(run.desc)
+    try:
+        lsh.fused_forward(2)
+        run = Run(inp, w.n_buckets, w.chunk, w.causal, w.dtype, flags)
+        assert lsh.fused_forward_fits(run.desc)
+    finally:
+        lsh.fused_forward(1)
     gb = run.host_buckets()
     gperm = run.perm.cpu().numpy()
     check_perm_is_stable_sort(gperm, gb, "fused perm")
@@ -95,7 +99,7 @@ def test_fused_forward_full_workload_equals_staged():
     launch configuration the benchmark times: both paths bit for bit."""
     w = synth.WORKLOADS["bf16_causal_4k"]
     inp = synth.make_inputs(w)
-    fused, staged = run_both(w, inp)
+    fused, staged = run_both(w, inp, mode=1)             # the default setting takes it (128 segments)
     assert torch.equal(fused.perm, staged.perm)
     assert torch.equal(fused.lse, staged.lse)
     assert torch.equal(fused.out, staged.out)
@@ -109,12 +113,15 @@ def test_fused_forward_without_permutation_output_then_recomputing_backward():
     the fp32 reductions' order)."""
     w = small(B=2, H=2, L=2048, n_buckets=64, n_hashes=2, causal=True, backward=True)
     inp = synth.make_inputs(w)
-    lsh.fused_forward(True)
-    run = Run(inp, w.n_buckets, w.chunk, w.causal, w.dtype)
-    assert lsh.fused_forward_fits(run.desc)
-    out2, lse2 = torch.empty_like(run.out), torch.empty_like(run.lse)
-    lsh.lsh_attn_fwd(run.desc, run.x, run.v, run.R, out2, lse2, None)
-    torch.cuda.synchronize()
+    try:
+        lsh.fused_forward(2)
+        run = Run(inp, w.n_buckets, w.chunk, w.causal, w.dtype)
+        assert lsh.fused_forward_fits(run.desc)
+        out2, lse2 = torch.empty_like(run.out), torch.empty_like(run.lse)
+        lsh.lsh_attn_fwd(run.desc, run.x, run.v, run.R, out2, lse2, None)
+        torch.cuda.synchronize()
+    finally:
+        lsh.fused_forward(1)
     assert torch.equal(out2, run.out) and torch.equal(lse2, run.lse)
     dx2, dv2 = torch.empty_like(run.x), torch.empty_like(run.v)
     lsh.lsh_attn_bwd(run.desc, run.x, run.v, run.R, run.out, run.lse, None, run.dy, dx2, dv2)

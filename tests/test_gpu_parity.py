@@ -574,7 +574,7 @@ def test_trace_records_only_selected_stages():
     desc = lsh.desc_for(x, w.n_buckets, w.n_hashes, w.chunk, w.causal)
     out, lse, perm = lsh.outputs_like(desc, x)
     ws = lsh.workspace(desc, False, x.device)
-    lsh.fused_forward(False)                     # the staged kernels, one stage each
+    lsh.fused_forward(0)                         # the staged kernels, one stage each
     try:
         lsh.lsh_attn_fwd(desc, x, v, R, out, lse, perm, ws)
         ref = out.clone()
@@ -593,10 +593,14 @@ def test_trace_records_only_selected_stages():
         st = lsh.trace_end()
         assert st["hash"][1] == 1 and st["sort"][1] == 1 and st["combine"][1] == 1
     finally:
-        lsh.fused_forward(True)
-    # the single kernel: one stage of its own, same output
-    lsh.trace_begin(16)
-    lsh.lsh_attn_fwd(desc, x, v, R, out, lse, perm, ws)
-    st = lsh.trace_end()
+        lsh.fused_forward(1)
+    # the single kernel (wherever it fits: this shape has 4 segments): one stage of its own, same output
+    try:
+        lsh.fused_forward(2)
+        lsh.trace_begin(16)
+        lsh.lsh_attn_fwd(desc, x, v, R, out, lse, perm, ws)
+        st = lsh.trace_end()
+    finally:
+        lsh.fused_forward(1)
     assert st["fused_fwd"][1] == 1 and all(st[k][1] == 0 for k in st if k != "fused_fwd")
     assert torch.equal(out, ref)
