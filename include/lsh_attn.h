@@ -342,9 +342,9 @@ LSH_API lsh_status lsh_attn_trace_stages(uint32_t mask);
 
 /* Single-kernel forward of short segments (lsh_attn_fwd, the reversible block
  * and lsh_attn_step_host).  mode = 1 (the default): used where a segment fits
- * and the B*H*n_hashes segments fill the GPU's waves (one CTA per segment: a
- * wave of at least three quarters as many segments as SMs); otherwise the
- * staged kernels, which spread every tile over all SMs, are faster.  mode = 2:
+ * and the B*H*n_hashes segments make one well-filled wave (one CTA per
+ * segment: from three quarters of the SM count up to the SM count); otherwise
+ * the staged kernels, which spread every tile over all SMs, are faster.  mode = 2:
  * used wherever a segment fits.  mode = 0: never (the staged kernels: hash,
  * sort, attention, merge).  Both forms give the same bits.  Process-wide;
  * takes effect for calls made after it.  Returns LSH_ERR_ARG for any other

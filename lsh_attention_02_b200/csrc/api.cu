@@ -182,13 +182,14 @@ static lsh_status run_attn_fwd(const Problem &p, const Choice &c, const void *qk
 // The whole forward from the rotations: one kernel per head's rounds where a
 // segment fits on chip and the setting allows it, otherwise hash, sort,
 // attention and merge as separate stages.  Setting 1 (the default) takes the
-// single kernel only where its segments fill the GPU's waves: it runs one CTA
-// per segment, so with few segments most SMs would idle while the staged
-// kernels spread every tile over all of them.  From the measured costs (4K
-// workload: 0.124 ms in one wave of 128 CTAs against 0.137 ms staged, the
-// staged time growing with the segment count) the single kernel is ahead when
-// a wave holds at least about three quarters as many segments as there are SMs.
-// Setting 2 takes it wherever it fits (tests), 0 never.
+// single kernel only where its segments make one well-filled wave: it runs one
+// CTA per segment, so with few segments most SMs idle while the staged kernels
+// spread every tile over all of them, and a second wave doubles its time while
+// the staged time grows less than linearly.  Measured at L = 4096 (64 buckets,
+// 2 rounds; single kernel against staged, us): 4 segments 117 / 43, 64 116 /
+// 85, 128 124 / 131, 160 227 / 164, 256 236 / 228.  So: at least three
+// quarters as many segments as SMs, and no more than the SMs.  Setting 2 takes
+// it wherever it fits (tests), 0 never.
 static int g_fused_forward = 1;
 static int sm_count()
 {
@@ -204,8 +205,8 @@ static bool use_fused(const Problem &p, const Choice &c)
 {
     if (g_fused_forward == 0 || !c.tc_attn || !fused_fwd_fits(p)) return false;
     if (g_fused_forward == 2) return true;
-    const long long sms = sm_count(), S = p.S(), waves = (S + sms - 1) / sms;
-    return 4 * S >= 3 * waves * sms;
+    const long long sms = sm_count(), S = p.S();
+    return 4 * S >= 3 * sms && S <= sms;
 }
 static lsh_status run_forward(const Problem &p, const Choice &c, const void *qk, const void *v, const void *R,
                               int32_t *perm, void *out, float *lse, const Workspace &w, cudaStream_t st)

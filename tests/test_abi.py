@@ -178,8 +178,8 @@ def test_fused_forward_applies_to_short_bf16_segments_only(lib):
     """The single-kernel forward is chosen on the host from the descriptor alone.
     Setting 2: wherever it fits (bf16, chunk 64, L a multiple of 64 up to 4096,
     n_buckets <= 128, n_hashes <= 8, B*H*L >= 128).  Setting 1 (the default):
-    also only where the B*H*n_hashes segments fill the GPU's waves (at least
-    three quarters of the SMs per wave; without a device the B200's 148).
+    also only where the B*H*n_hashes segments make one well-filled wave (from
+    three quarters of the SM count up to it; without a device the B200's 148).
     Setting 0: never."""
     fits = lambda **kw: lib.lsh_attn_fused_forward_fits(ctypes.byref(_desc(**kw)))
     assert lib.lsh_attn_fused_forward(3) == -1     # LSH_ERR_ARG
@@ -197,8 +197,9 @@ def test_fused_forward_applies_to_short_bf16_segments_only(lib):
         if sms is not None:
             assert fits(L=4096, n_buckets=64, n_hashes=2, B=8, H=8) == 1    # 128 segments, one wave
             assert fits(L=4096, n_buckets=64, n_hashes=2, B=1, H=2) == 0    # 4 segments: staged
-            assert fits(L=1024, n_buckets=64, n_hashes=2, B=8, H=10) == 0   # 160 segments, two thin waves
-            assert fits(L=1024, n_buckets=64, n_hashes=2, B=8, H=16) == 1   # 256 segments, two full waves
+            assert fits(L=1024, n_buckets=64, n_hashes=2, B=8, H=9) == 1    # 144 segments, one wave
+            assert fits(L=1024, n_buckets=64, n_hashes=2, B=8, H=10) == 0   # 160 segments: a second wave
+            assert fits(L=1024, n_buckets=64, n_hashes=2, B=8, H=16) == 0   # 256 segments: staged
         assert lib.lsh_attn_fused_forward(0) == 0
         assert fits(L=4096, n_buckets=64, B=8, H=8) == 0
     finally:
