@@ -1,8 +1,10 @@
 // Single-kernel forward of short segments: lsh_hash, bucket_sort, gather +
 // chunk_attn and unsort_combine of one (batch, head) in one cluster of R CTAs,
 // CTA r taking round r ("Sorting and Chunking", "Multiple Hash Rounds", paper
-// note "Reformer").  Nothing between the steps goes through HBM except the
-// rounds' outputs, which the merge reads back from L2.
+// note "Reformer").  The bucket ids, ranks, counts and the permutation stay in
+// shared memory between the steps; the key norms pass through L2, and the
+// rounds' outputs are read back by the merge (from L2 where they are still
+// resident, otherwise from HBM).
 //
 // Per CTA (segment (bh, r), L <= kMaxL positions, n_buckets <= 2 kMaxHalf):
 //   hash       split over the cluster: CTA r loads x tiles r, r + R, ... of the
@@ -112,9 +114,10 @@ __device__ __forceinline__ uint8_t *hash_tile(FusedSmem &sm, int b)
 // padding): the first maximum of [v ; -v].  Pass 1 takes the largest and
 // smallest value (3-input max/min, four independent chains); the larger of max
 // and -min picks the side (+ wins an exact tie: its indices come first); pass 2
-// finds the lowest column holding that extreme.  Called by whole warps.  A padding column (exactly 0)
+// finds the lowest column holding that extreme.  A padding column (exactly 0)
 // never decides: max(v_j, -v_j) >= 0 for every real column, and real columns
 // come first.  This is the hash kernel's rule, so both give the same ids.
+// Called by whole warps.
 template <int NH>
 __device__ __forceinline__ int first_max_bucket(const float *v, int half)
 {
