@@ -37,23 +37,29 @@ def build(force: bool = False) -> str:
 def lib():
     global _lib
     if _lib is None:
-        build()
-        L = ctypes.CDLL(_LIB)
-        L.oracle_hash.argtypes = [_D, _L, _C, _D, _C, _I32, _D]
-        L.oracle_sort.argtypes = [_I32, _L, _I32]
-        L.oracle_attn_round.argtypes = [_D, _D, _L, _C, _I32, _C, _C, _I32, _C, _D, _D]
-        L.oracle_attn_slots.argtypes = [_D, _D, _L, _C, _I32, _C, _C, _I32, _C, _I64, _L, _D, _D]
-        L.oracle_combine.argtypes = [_D, _D, _C, _L, _C, _D, _D]
-        L.oracle_fwd_head.argtypes = [_D, _D, _L, _C, _D, _C, _C, _C, _C, _C, _C, _D, _D, _I32, _I32, _D]
-        L.oracle_bwd_head.argtypes = [_D, _D, _D, _L, _C, _I32, _C, _C, _C, _I32, _C, _D, _D]
-        L.oracle_fwd_batch.argtypes = [_D, _D, _L, _L, _C, _D, _C, _C, _C, _C, _C, _C, _D, _D, _I32, _I32, _D]
-        L.oracle_fwd_perm_batch.argtypes = [_D, _D, _L, _L, _C, _I32, _C, _C, _C, _I32, _C, _D, _D]
-        L.oracle_bwd_batch.argtypes = [_D, _D, _D, _L, _L, _C, _I32, _C, _C, _C, _I32, _C, _D, _D]
-        L.oracle_local_fwd_batch.argtypes = [_D, _D, _L, _L, _C, _C, _C, _C, _C, _C, _D, _D]
-        L.oracle_local_bwd_batch.argtypes = [_D, _D, _D, _L, _L, _C, _C, _C, _C, _C, _C, _D, _D]
-        L.oracle_max_threads.argtypes = []
-        _lib = L
+        _lib = open_library(build())
     return _lib
+
+
+def open_library(path: str):
+    """Loads an oracle library and declares its entry points.  lib() opens the
+    one built from lsh_oracle.c; the oracle tests' planted-mistake check opens
+    altered copies of that source through this function."""
+    L = ctypes.CDLL(path)
+    L.oracle_hash.argtypes = [_D, _L, _C, _D, _C, _I32, _D]
+    L.oracle_sort.argtypes = [_I32, _L, _I32]
+    L.oracle_attn_round.argtypes = [_D, _D, _L, _C, _I32, _C, _C, _I32, _C, _D, _D]
+    L.oracle_attn_slots.argtypes = [_D, _D, _L, _C, _I32, _C, _C, _I32, _C, _I64, _L, _D, _D]
+    L.oracle_combine.argtypes = [_D, _D, _C, _L, _C, _D, _D]
+    L.oracle_fwd_head.argtypes = [_D, _D, _L, _C, _D, _C, _C, _C, _C, _C, _C, _D, _D, _I32, _I32, _D]
+    L.oracle_bwd_head.argtypes = [_D, _D, _D, _L, _C, _I32, _C, _C, _C, _I32, _C, _D, _D]
+    L.oracle_fwd_batch.argtypes = [_D, _D, _L, _L, _C, _D, _C, _C, _C, _C, _C, _C, _D, _D, _I32, _I32, _D]
+    L.oracle_fwd_perm_batch.argtypes = [_D, _D, _L, _L, _C, _I32, _C, _C, _C, _I32, _C, _D, _D]
+    L.oracle_bwd_batch.argtypes = [_D, _D, _D, _L, _L, _C, _I32, _C, _C, _C, _I32, _C, _D, _D]
+    L.oracle_local_fwd_batch.argtypes = [_D, _D, _L, _L, _C, _C, _C, _C, _C, _C, _D, _D]
+    L.oracle_local_bwd_batch.argtypes = [_D, _D, _D, _L, _L, _C, _C, _C, _C, _C, _C, _D, _D]
+    L.oracle_max_threads.argtypes = []
+    return L
 
 
 def _d(a):
