@@ -58,13 +58,14 @@ def test_hash_scale_and_negation(dtype, nb, nh):
 
 
 @pytest.mark.parametrize("mode", [0, 2])
-@pytest.mark.parametrize("causal", [True, False])
-def test_output_doubles_with_values(mode, causal):
-    """mode 0: the staged kernels; mode 2: the single kernel of short segments."""
+@pytest.mark.parametrize("causal,flags", [(True, 0), (False, 0), (True, lsh.FLAG_BUCKET_MASK | lsh.FLAG_SELF_PENALTY)])
+def test_output_doubles_with_values(mode, causal, flags):
+    """mode 0: the staged kernels; mode 2: the single kernel of short segments;
+    flags: the bucket mask and the self penalty."""
     w = synth.WORKLOADS["bf16_causal_4k"].replace(B=1, H=2, L=2048, causal=causal)
     inp = synth.make_inputs(w)
     x = to_dev(inp["x"], "bf16"); v = to_dev(inp["v"], "bf16"); R = to_dev(inp["R"], "bf16")
-    desc = lsh.desc_for(x, w.n_buckets, w.n_hashes, w.chunk, causal)
+    desc = lsh.desc_for(x, w.n_buckets, w.n_hashes, w.chunk, causal, flags)
     try:
         lsh.fused_forward(mode)
         assert lsh.fused_forward_fits(desc) == (mode == 2)
@@ -80,3 +81,52 @@ def test_output_doubles_with_values(mode, causal):
     assert torch.equal(o2, o1 * 2)
     assert torch.equal(l2, l1)
     assert torch.equal(p2, p1)
+
+
+@pytest.mark.parametrize("after", [0, 1])
+def test_local_output_doubles_with_values(after):
+    """Local chunk attention (no hashing), with and without the following chunk."""
+    L = 1024
+    w = synth.WORKLOADS["long_64k"].replace(B=1, H=2, L=L, n_hashes=1, causal=after == 0)
+    inp = synth.make_inputs(w)
+    x = to_dev(inp["x"], "bf16"); v = to_dev(inp["v"], "bf16")
+    desc = lsh.make_desc(1, 2, L, 64, 2, 1, 64, after == 0, dtype=torch.bfloat16)
+    res = []
+    for vv in (v, v * 2):
+        out = torch.empty_like(x)
+        lse = torch.empty((1, 2, 1, L), dtype=torch.float32, device="cuda")
+        lsh.lsh_attn_local_fwd(desc, after, x, vv, out, lse)
+        res.append((out, lse))
+    torch.cuda.synchronize()
+    (o1, l1), (o2, l2) = res
+    assert torch.equal(o2, o1 * 2)
+    assert torch.equal(l2, l1)
+
+
+@pytest.mark.parametrize("mode", [0, 2])
+def test_heads_are_independent(mode):
+    """Each (batch, head) slice is its own problem: the forward of a 2 x 2
+    problem equals the forward of every slice alone, bit for bit (merged
+    output, per-round lse and permutation), through the staged kernels (mode
+    0) and the single kernel (mode 2)."""
+    w = synth.WORKLOADS["bf16_causal_4k"].replace(B=2, H=2, L=1024)
+    inp = synth.make_inputs(w)
+    x = to_dev(inp["x"], "bf16"); v = to_dev(inp["v"], "bf16"); R = to_dev(inp["R"], "bf16")
+    desc = lsh.desc_for(x, w.n_buckets, w.n_hashes, w.chunk, w.causal)
+    try:
+        lsh.fused_forward(mode)
+        out, lse, perm = lsh.outputs_like(desc, x)
+        lsh.lsh_attn_fwd(desc, x, v, R, out, lse, perm)
+        for b in range(2):
+            for h in range(2):
+                xs = x[b:b + 1, h:h + 1].contiguous(); vs = v[b:b + 1, h:h + 1].contiguous()
+                ds = lsh.desc_for(xs, w.n_buckets, w.n_hashes, w.chunk, w.causal)
+                assert lsh.fused_forward_fits(ds) == (mode == 2)
+                o1, l1, p1 = lsh.outputs_like(ds, xs)
+                lsh.lsh_attn_fwd(ds, xs, vs, R, o1, l1, p1)
+                torch.cuda.synchronize()
+                assert torch.equal(o1[0, 0], out[b, h]), (b, h)
+                assert torch.equal(l1[0, 0], lse[b, h]), (b, h)
+                assert torch.equal(p1[0, 0], perm[b, h]), (b, h)
+    finally:
+        lsh.fused_forward(1)
