@@ -209,3 +209,16 @@ def test_fused_forward_applies_to_short_bf16_segments_only(lib):
 def torch_cuda_available():
     import torch
     return torch.cuda.is_available()
+
+
+def test_missing_library_fails_loudly(tmp_path, monkeypatch):
+    """Without the CUDA library every entry point raises: there is no other
+    implementation to fall back on."""
+    absent = str(tmp_path / "liblsh_attn.so")
+    monkeypatch.setattr(lsh, "_lib", None)
+    monkeypatch.setattr(lsh.load_library, "__defaults__", (absent,))
+    with pytest.raises(ImportError, match="missing"):
+        lsh.load_library()
+    desc = lsh.make_desc(1, 1, 256, 64, 16, 1, 64, True, lsh.LSH_BF16)
+    with pytest.raises(ImportError, match="missing"):
+        lsh.workspace_size(desc, False)
